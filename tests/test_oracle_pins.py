@@ -1,0 +1,335 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Every check here is independent of the oracle's own formulas: closed forms,
+library routines on special cases, invariants, and brute force on tiny inputs.
+A plausible slip anywhere in the oracle (a dropped term, a wrong sign, a
+transposed operand, gate/up swapped, a lost shared expert, a wrong tie rule)
+fails at least one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import cases
+
+# --------------------------------------------------------------------- decoding
+
+
+def test_f16_decode_matches_numpy_on_all_finite_patterns():
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    finite = np.isfinite(ref)
+    got = np.array([oracle.f16(int(b)) for b in bits[finite][::7]])
+    np.testing.assert_array_equal(got, ref[finite][::7])
+    # the few landmarks exactly
+    assert oracle.f16(0x3C00) == 1.0
+    assert oracle.f16(0xC000) == -2.0
+    assert oracle.f16(0x7BFF) == 65504.0
+    assert oracle.f16(0x0001) == 2.0 ** -24
+    assert oracle.f16(0x0400) == 2.0 ** -14
+    assert math.isinf(oracle.f16(0x7C00))
+
+
+def test_bf16_decode():
+    assert oracle.bf16(0x3F80) == 1.0
+    assert oracle.bf16(0xC040) == -3.0
+    assert oracle.bf16(0x0001) == 2.0 ** -133
+    v = np.float32(-1.2345678e-3)
+    b = int(np.array([v]).view(np.uint32)[0] >> 16)
+    assert oracle.bf16(b) == float(np.array([b << 16], np.uint32).view(np.float32)[0])
+
+
+def test_nibble_decode_handcrafted():
+    # 0x8F: low nibble 0xF -> -1 (element 0), high nibble 0x8 -> -8 (element 1)
+    # 0x70: low 0 (element 2), high 7 (element 3)
+    row = np.array([0x8F, 0x70, 0x21, 0xE9], np.uint8)
+    assert [oracle.code(row, c) for c in range(8)] == [-1, -8, 0, 7, 1, 2, -7, -2]
+
+
+def test_dequant_handcrafted_group_scales():
+    codes = np.array([[(c % 16) - 8 for c in range(128)]], np.int64)
+    q = cases.pack_codes(codes)
+    s = cases.f16_bits([[0.5, -0.25]])
+    w = oracle.dequant(q, s, 1, 128)
+    expect = np.concatenate([codes[0, :64] * 0.5, codes[0, 64:] * -0.25])
+    np.testing.assert_array_equal(w[0], expect)
+
+
+@pytest.mark.parametrize("matrix,rows,cols", [(synth.GATE, 256, 512), (synth.UP, 256, 512), (synth.DOWN, 512, 256)])
+def test_int4_gs64_round_trip_within_half_step(matrix, rows, cols):
+    """Encoding then decoding moves every weight by at most half a step s/2
+    (int4 gs64 container); codes stay in [-8, 7]; the scale is absmax/7 in fp16."""
+    H, I = 512, 256
+    q, s = synth.expert(3, 0, 5, H, I)
+    nq, ns = H * I // 2, H * I // 64
+    qm = q[matrix * nq:(matrix + 1) * nq]
+    sm = s[matrix * ns:(matrix + 1) * ns]
+    w = synth.matrix_f32(3, 0, 5, matrix, rows, cols).astype(np.float64)
+    wd = oracle.dequant(qm, sm, rows, cols)
+    sc = np.repeat(sm.view(np.float16).astype(np.float64).reshape(rows, cols // 64), 64, axis=1)
+    assert np.all(np.abs(w - wd) <= sc / 2 + 0.0)
+    # the scale rule, through numpy's own fp16 rounding
+    amax = np.abs(w.reshape(rows, cols // 64, 64)).max(axis=2).astype(np.float32)
+    np.testing.assert_array_equal(sm.reshape(rows, cols // 64), (amax / np.float32(7)).astype(np.float16).view(np.uint16))
+    codes = np.rint(wd / np.where(sc == 0, 1, sc))
+    assert codes.min() >= -8 and codes.max() <= 7
+
+
+# ----------------------------------------------------------------------- router
+
+
+def test_router_logits_are_a_matmul_plus_bias():
+    rng = np.random.default_rng(1)
+    wr = rng.standard_normal((16, 128)).astype(np.float32)
+    x = rng.standard_normal((5, 128)).astype(np.float32)
+    b = rng.standard_normal(16).astype(np.float32)
+    got = oracle.router_logits(wr, b, x)
+    ref = x.astype(np.float64) @ wr.astype(np.float64).T + b.astype(np.float64)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # bf16 activations are widened exactly
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+    xw = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    np.testing.assert_allclose(oracle.router_logits(wr, None, xb), xw @ wr.astype(np.float64).T, rtol=0, atol=1e-12)
+
+
+def test_topk_brute_force_and_exactly_k_distinct():
+    rng = np.random.default_rng(2)
+    T, E, K = 64, 256, 8
+    logits = rng.standard_normal((T, E))
+    ids, w = oracle.topk(logits, K)
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-logits[t, e], e))
+        assert list(ids[t]) == order[:K]
+        assert len(set(ids[t])) == K
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+
+
+def test_topk_ties_go_to_lower_id_and_k_equals_e():
+    logits = np.zeros((2, 6))
+    logits[1] = [1.0, 3.0, 3.0, 0.5, 3.0, -1.0]
+    ids, w = oracle.topk(logits, 3)
+    assert list(ids[0]) == [0, 1, 2]
+    assert list(ids[1]) == [1, 2, 4]
+    np.testing.assert_allclose(w, 1.0 / 3.0, rtol=0, atol=1e-16)
+    ids, _ = oracle.topk(logits, 6)
+    assert sorted(ids[0]) == list(range(6)) and list(ids[1]) == [1, 2, 4, 0, 3, 5]
+
+
+def test_topk_weights_closed_form_and_full_softmax_form():
+    # logits ln 1, ln 2, ln 3, ln 4 -> top-2 picks ids 3, 2 with weights 4/7, 3/7
+    logits = np.log(np.array([[1.0, 2.0, 3.0, 4.0]]))
+    ids, w = oracle.topk(logits, 2)
+    assert list(ids[0]) == [3, 2]
+    np.testing.assert_allclose(w[0], [4 / 7, 3 / 7], rtol=0, atol=1e-15)
+    rng = np.random.default_rng(3)
+    lg = rng.standard_normal((32, 256)) * 3
+    ids, w = oracle.topk(lg, 8)
+    np.testing.assert_allclose(oracle.weights_full_softmax(lg, ids), w, rtol=0, atol=1e-15)
+
+
+def test_topk_rejects_nan():
+    with pytest.raises(ValueError):
+        oracle.topk(np.array([[0.0, np.nan, 1.0]]), 2)
+
+
+# ------------------------------------------------------------------------ union
+
+
+def test_union_invariants_against_python_sets():
+    rng = np.random.default_rng(4)
+    T, K, E = 40, 8, 256
+    ids = np.stack([rng.choice(E, K, replace=False, p=None) for _ in range(T)]).astype(np.int32)
+    # skew: half the tokens share experts 0..7
+    ids[::2] = np.arange(8)
+    u = oracle.union(ids, E)
+    assert int(u["cnt"].sum()) == T * K
+    assert list(u["unique"]) == sorted(set(ids.ravel().tolist()))
+    assert len(set(u["unique"].tolist())) == len(u["unique"])
+    for e in range(E):
+        toks = [t for t in range(T) for k in range(K) if ids[t, k] == e]
+        assert u["cnt"][e] == len(toks)
+        assert list(u["tok"][u["off"][e]:u["off"][e + 1]]) == toks  # ascending tokens
+    for t in range(T):
+        for k in range(K):
+            p = u["pos"][t, k]
+            assert u["tok"][p] == t and u["off"][ids[t, k]] <= p < u["off"][ids[t, k] + 1]
+    assert sorted(u["pos"].ravel().tolist()) == list(range(T * K))  # a permutation
+
+
+def test_union_touches_each_unique_expert_once_and_the_per_layer_fraction():
+    """Batch 1, full-size shapes: 8 of 256 chosen; streamed parameters are the
+    8 routed + 1 shared experts plus the router, 3.52% of the layer."""
+    H, I, E, K = 6144, 2048, 256, 8
+    rng = np.random.default_rng(5)
+    logits = rng.standard_normal((1, E))
+    ids, _ = oracle.topk(logits, K)
+    u = oracle.union(ids, E)
+    assert len(u["unique"]) == 8
+    per_expert = 3 * H * I
+    touched = (len(u["unique"]) + 1) * per_expert + E * H
+    total = (E + 1) * per_expert + E * H
+    assert touched == 9 * 37_748_736 + 1_572_864
+    assert abs(touched / total - 0.0352) < 5e-4
+    # the pages' whole-model figure (40B of 744B, ~5.4%) from their own counts:
+    # 75 layers x 8 routed experts + 17B dense part, over 19,456 experts + 17B
+    whole = (75 * 8 * per_expert + 17e9) / (19456 * per_expert + 17e9)
+    assert abs(whole - 0.054) < 0.002
+
+
+# ----------------------------------------------------------------------- expert
+
+
+def _basis_expert(H, I, j, gate_q, up_q, sg, su):
+    """Gate/up have one nonzero column j; down is the identity on the first I rows."""
+    G = np.zeros((I, H), np.int64)
+    U = np.zeros((I, H), np.int64)
+    G[:, j] = gate_q
+    U[:, j] = up_q
+    D = np.zeros((H, I), np.int64)
+    D[np.arange(I), np.arange(I)] = 1
+    return cases.expert_from_codes(G, U, D, np.full((I, H // 64), sg), np.full((I, H // 64), su),
+                                   np.full((H, I // 64), 1.0))
+
+
+def test_expert_ffn_closed_form_on_a_basis_vector():
+    """x = a e_j: g_r = a G[r][j], u_r = a U[r][j], h_r = silu(g_r) u_r, and with
+    D = [I; 0] the output is h followed by zeros. H != I catches transposes;
+    distinct gate/up codes catch a gate/up swap."""
+    H, I, j, a = 128, 64, 37, 1.5
+    gate_q = np.array([(r % 15) - 7 for r in range(I)])
+    up_q = np.array([7 - (r % 13) for r in range(I)])
+    q, s = _basis_expert(H, I, j, gate_q, up_q, 0.5, 0.25)
+    x = np.zeros(H)
+    x[j] = a
+    out, h = oracle.expert_ffn(q, s, H, I, x, want_h=True)
+    for r in range(I):
+        g = a * gate_q[r] * 0.5
+        u = a * up_q[r] * 0.25
+        hr = g / (1 + math.exp(-g)) * u
+        assert h[r] == pytest.approx(hr, rel=1e-15, abs=1e-300)
+        assert out[r] == pytest.approx(hr, rel=1e-15, abs=1e-300)
+    assert np.all(out[I:] == 0.0)
+
+
+def test_expert_ffn_silu_zero_and_dense_library_form():
+    H, I = 128, 64
+    q, s = synth.expert(7, 0, 0, H, I)
+    assert np.all(oracle.expert_ffn(q, s, H, I, np.zeros(H)) == 0.0)
+    # same expert through numpy's matmul on the decoded matrices
+    nq, ns = H * I // 2, H * I // 64
+    G = oracle.dequant(q[:nq], s[:ns], I, H)
+    U = oracle.dequant(q[nq:2 * nq], s[ns:2 * ns], I, H)
+    D = oracle.dequant(q[2 * nq:], s[2 * ns:], H, I)
+    x = np.random.default_rng(6).standard_normal(H)
+    g, u = G @ x, U @ x
+    ref = D @ (g / (1 + np.exp(-g)) * u)
+    np.testing.assert_allclose(oracle.expert_ffn(q, s, H, I, x), ref, rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------------------------------ layer
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    c = cases.TINY
+    L = cases.host_layer(c, seed=c["seed"])
+    x = synth.x_f32(c["seed"], 0, c["T"], c["H"])
+    return c, L, x
+
+
+def test_sparse_equals_dense_with_unselected_gates_zeroed(tiny):
+    """Sparse selection is checked by forcing full selection against the dense
+    computation (as the colibri pages validate their sparse attention)."""
+    c, L, x = tiny
+    cfg = cases.oracle_cfg(c)
+    y, ids, w = oracle.moe_forward(cfg, L["wr"], L["bias"], L["experts"], x)
+    yd = oracle.moe_forward(cfg, L["wr"], L["bias"], L["experts"], x, dense=True)
+    np.testing.assert_allclose(y, yd, rtol=0, atol=1e-12 * np.abs(yd).max())
+    assert ids.shape == (c["T"], c["K"]) and all(len(set(r)) == c["K"] for r in ids)
+
+
+def test_layer_decomposes_into_shared_plus_weighted_routed(tiny):
+    """y = shared(x) + sum_k w_k E_k(x): rebuilt from single-expert calls."""
+    c, L, x = tiny
+    cfg = cases.oracle_cfg(c)
+    y, ids, w = oracle.moe_forward(cfg, L["wr"], L["bias"], L["experts"], x)
+    logits = oracle.router_logits(L["wr"], None, x)
+    ids2, w2 = oracle.topk(logits, c["K"])
+    np.testing.assert_array_equal(ids, ids2)
+    for t in range(c["T"]):
+        xt = x[t].astype(np.float64)
+        ref = oracle.expert_ffn(*L["experts"][c["E"]], c["H"], c["I"], xt)
+        for k in range(c["K"]):
+            ref = ref + w2[t, k] * oracle.expert_ffn(*L["experts"][ids[t, k]], c["H"], c["I"], xt)
+        np.testing.assert_allclose(y[t], ref, rtol=0, atol=1e-13 * np.abs(ref).max())
+
+
+def test_shared_only_when_routed_experts_are_zero(tiny):
+    c, L, x = tiny
+    cfg = cases.oracle_cfg(c)
+    zero = (np.zeros_like(L["experts"][0][0]), np.zeros_like(L["experts"][0][1]))
+    experts = [zero] * c["E"] + L["experts"][c["E"]:]
+    y, _, _ = oracle.moe_forward(cfg, L["wr"], None, experts, x)
+    for t in range(c["T"]):
+        ref = oracle.expert_ffn(*L["experts"][c["E"]], c["H"], c["I"], x[t].astype(np.float64))
+        np.testing.assert_array_equal(y[t], ref)
+
+
+def test_bias_changes_selection_and_no_shared_expert():
+    """A large bias on experts 3 and 9 forces them to be chosen (top-2); with no
+    shared expert the output is exactly the two weighted routed experts."""
+    c = dict(cases.TINY, S=0)
+    L = cases.host_layer(c, seed=1)
+    bias = np.zeros(c["E"], np.float32)
+    bias[3], bias[9] = 50.0, 49.0
+    x = synth.x_f32(1, 0, 2, c["H"])
+    cfg = cases.oracle_cfg(c)
+    y, ids, w = oracle.moe_forward(cfg, L["wr"], bias, L["experts"], x)
+    assert ids.tolist() == [[3, 9], [3, 9]]
+    for t in range(2):
+        xt = x[t].astype(np.float64)
+        ref = w[t, 0] * oracle.expert_ffn(*L["experts"][3], c["H"], c["I"], xt) + \
+            w[t, 1] * oracle.expert_ffn(*L["experts"][9], c["H"], c["I"], xt)
+        np.testing.assert_allclose(y[t], ref, rtol=0, atol=1e-13 * np.abs(ref).max())
+
+
+def test_empty_batch():
+    c = cases.TINY
+    L = cases.host_layer(c, seed=0, which=[])
+    y, ids, w = oracle.moe_forward(cases.oracle_cfg(c), L["wr"], None, L["experts"], np.zeros((0, c["H"]), np.float32))
+    assert y.shape == (0, c["H"])
+
+
+def test_missing_selected_expert_is_an_error():
+    c = cases.TINY
+    L = cases.host_layer(c, seed=0, which=[c["E"]])
+    with pytest.raises(ValueError):
+        oracle.moe_forward(cases.oracle_cfg(c), L["wr"], None, L["experts"], synth.x_f32(0, 0, 1, c["H"]))
+
+
+# ------------------------------------------------------------------------ stack
+
+
+def test_rmsnorm_closed_forms():
+    x = np.full((1, 64), -3.0)
+    np.testing.assert_allclose(oracle.rmsnorm(x, eps=0.0), -1.0, rtol=1e-15)
+    x = np.random.default_rng(7).standard_normal((3, 256)) * 5
+    n = oracle.rmsnorm(x, eps=0.0)
+    np.testing.assert_allclose((n ** 2).mean(axis=1), 1.0, rtol=1e-14)
+    r = n / x
+    np.testing.assert_allclose(r, np.broadcast_to(r[:, :1], r.shape), rtol=1e-14)  # one scale per token
+
+
+def test_stack_step_is_residual_of_normalised_layer(tiny):
+    c, L, x = tiny
+    cfg = cases.oracle_cfg(c)
+    x0 = (x * 7.0).astype(np.float32)
+    xs = x0.copy()
+    ids = oracle.stack_step(cfg, L["wr"], None, L["experts"], xs)
+    nf = oracle.rmsnorm(x0.astype(np.float64)).astype(np.float32)
+    y, ids2, _ = oracle.moe_forward(cfg, L["wr"], None, L["experts"], nf)
+    np.testing.assert_array_equal(ids, ids2)
+    np.testing.assert_array_equal(xs, (x0.astype(np.float64) + y).astype(np.float32))
