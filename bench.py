@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""Benchmark of the int4 expert-FFN MoE layer on B200.
+
+Default workload: one full-size MoE layer (hidden 6144, expert intermediate
+2048, 256 routed experts top-8 with softmax-renormalised weights, one shared
+expert; int4 gs64 weights with fp16 scales, N(0, 0.02) before encoding; router
+fp32, bias 0), decode batch 1, a fresh seeded N(0,1) fp32 token every step.
+
+One step = one forward of the layer (router, top-k, batch-union plan, fused
+int4 gate/up + SwiGLU, down, weighted combine with the shared expert) for one
+batch. Inputs are resident in HBM before the timed region; L2 is flushed
+between steps by a 256 MiB memset recorded outside the per-step events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_b1|decode_b32|prefill_2048]
+
+Prints one JSON line (rank 0). N > 1 runs N independent replicas (one per
+rank, launched by torch.distributed.run), weak scaling, max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE int4 layer tokens/s; streamed-expert HBM GB/s vs ~8 TB/s (batch 1–2048)"
+H, I, E, K, S = 6144, 2048, 256, 8, 1
+EXPERT_BYTES = 20_054_016          # int4 nibbles + fp16 scales of one expert
+GU_BYTES = 13_369_344              # gate + up of one expert
+DOWN_BYTES = 6_684_672             # down of one expert
+ROUTER_BYTES = E * H * 4           # fp32 router matrix
+
+WORKLOADS = {
+    "decode_b1": dict(T=1, zipf=False, bf16=False,
+                      desc="one full-size layer, decode batch 1, bias 0, fresh fp32 token per step"),
+    "decode_b32": dict(T=32, zipf=True, bf16=False,
+                       desc="one full-size layer, decode batch 32, Zipf(1.1) router bias, fp32"),
+    "prefill_2048": dict(T=2048, zipf=True, bf16=True,
+                         desc="one full-size layer, prefill 2048 tokens, Zipf(1.1) router bias, bf16"),
+}
+X_SEED0 = 1000  # step s draws its activations with seed X_SEED0 + s
+
+
+DEFAULT_STEPS = {"decode_b1": 10000, "decode_b32": 2000, "prefill_2048": 100}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None, help="default: 10000 (decode_b1), 2000 (decode_b32), 100 (prefill)")
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b1")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.steps is None:
+        a.steps = DEFAULT_STEPS[a.workload]
+    return a
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# --------------------------------------------------------------- CPU oracle leg
+class OracleLeg:
+    """The fp64 oracle on the host cores, one bounded sample per step (input
+    generation, including the selected experts, is untimed and cached)."""
+
+    def __init__(self, wl):
+        import oracle
+        import synth
+        self.oracle, self.synth, self.wl = oracle, synth, wl
+        self.bias = synth.zipf_bias(0, 0, E)[0] if wl["zipf"] else None
+        self.wr = synth.router(0, 0, E, H)
+        self.cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S)
+        self.cache = {}
+        self.Ts = wl["T"] if wl["T"] <= 2 else 2   # tokens of a step the sample covers
+
+    def step(self, i):
+        """Returns (tokens, oracle seconds) of the sample of step i."""
+        import numpy as np
+        wl, syn = self.wl, self.synth
+        x = syn.x_bf16(X_SEED0 + i, 0, wl["T"], H) if wl["bf16"] else syn.x_f32(X_SEED0 + i, 0, wl["T"], H)
+        x = np.ascontiguousarray(x[:self.Ts])
+        ids, _ = self.oracle.topk(self.oracle.router_logits(self.wr, self.bias, x), K)
+        experts = [None] * (E + S)
+        for e in set(ids.ravel().tolist()) | set(range(E, E + S)):
+            if e not in self.cache:
+                self.cache[e] = syn.expert(0, 0, e, H, I)
+            experts[e] = self.cache[e]
+        t0 = time.perf_counter()
+        self.oracle.moe_forward(self.cfg, self.wr, self.bias, experts, x)
+        return self.Ts, time.perf_counter() - t0
+
+    def cores(self):
+        return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def oracle_sample(wl, budget_s):
+    leg = OracleLeg(wl)
+    tokens, spent, steps = 0, 0.0, 0
+    wall = time.time()
+    while spent < budget_s and time.time() - wall < 4 * budget_s:
+        n, dt = leg.step(steps)
+        tokens += n
+        spent += dt
+        steps += 1
+    return dict(value=round(tokens / spent, 4), unit="tokens/s", cores=leg.cores(), kind="oracle",
+                sample=f"{steps} steps x {leg.Ts} token(s) of the workload through the fp64 oracle, "
+                       f"{spent:.1f} s of oracle time (input and expert generation untimed)")
+
+
+# -------------------------------------------------------------------- GPU side
+class Clocks:
+    """nvidia-smi sampler for the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def build_layer(torch, coli, synth, wl, device, max_tokens):
+    nq, ns = synth.expert_sizes(H, I)
+    dev = torch.device("cuda", device)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    wr = torch.empty(E * H, dtype=torch.float32, device=dev)
+    synth.router_dev(0, 0, E, H, wr.data_ptr(), stream)
+    q = torch.empty((E + S) * nq, dtype=torch.uint8, device=dev)
+    s = torch.empty((E + S) * ns, dtype=torch.int16, device=dev)
+    synth.expert_dev(0, 0, 0, E + S, H, I, q.data_ptr(), s.data_ptr(), stream)
+    bias = None
+    if wl["zipf"]:
+        bias = torch.from_numpy(synth.zipf_bias(0, 0, E)[0]).to(dev)
+    torch.cuda.synchronize(dev)
+    cfg = coli.make_config(H, I, E, K, S, max_tokens)
+    layer = coli.Layer(cfg, wr, bias, q[:E * nq], s[:E * ns], q[E * nq:], s[E * ns:], device=device)
+    del q, s, wr
+    torch.cuda.empty_cache()
+    return layer
+
+
+def run_ours(args, wl, ws, rank, local):
+    import torch
+    import synth
+    import int4_expert_ffn_router_b200 as coli
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    T = wl["T"]
+    layer = build_layer(torch, coli, synth, wl, local, max_tokens=T)
+    nsteps = args.warmup + args.steps
+    xdt = torch.bfloat16 if wl["bf16"] else torch.float32
+    xs = torch.empty((nsteps, T, H), dtype=xdt, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for i in range(nsteps):  # rank r draws its own token stream
+        synth.x_dev(X_SEED0 + i + 100000 * rank, 0, T, H, 1 if wl["bf16"] else 0, xs[i].data_ptr(), stream.cuda_stream)
+    y = torch.empty((T, H), dtype=xdt, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    # routing statistics of every step (untimed pre-pass): unique experts -> bytes
+    uniq = []
+    for i in range(nsteps):
+        layer.forward(xs[i], y, stream=stream)
+        uniq.append(layer.stats()[0])
+    torch.cuda.synchronize(dev)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
+    # warm-up
+    for i in range(args.warmup):
+        layer.forward(xs[i], y, stream=stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    layer.set_profiling(True)
+    clocks = Clocks(local)
+    for i in range(args.warmup, nsteps):
+        ev[i][0].record(stream)
+        layer.forward(xs[i], y, stream=stream)
+        ev[i][1].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, nsteps)]
+    stages, nprof = layer.profile()
+    layer.set_profiling(False)
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the C ABI with host buffers: pinned H2D of the step's
+    # x, forward, D2H of y, every step inside the events.
+    xh = xs[args.warmup:].cpu().pin_memory()
+    yh = torch.empty((T, H), dtype=xdt).pin_memory()
+    xin = torch.empty((T, H), dtype=xdt, device=dev)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for j in range(args.steps):
+        ev2[j][0].record(stream)
+        xin.copy_(xh[j], non_blocking=True)
+        layer.forward(xin, y, stream=stream)
+        yh.copy_(y, non_blocking=True)
+        ev2[j][1].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(ev2[j][0].elapsed_time(ev2[j][1]) for j in range(args.steps))
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+
+    if rank != 0:
+        layer.close()
+        if dist:
+            dist.destroy_process_group()
+        return None
+
+    tokens = ws * args.steps * T
+    u = uniq[args.warmup:]
+    mean_unique = sum(u) / len(u)
+    bytes_step = [(n + S) * EXPERT_BYTES + ROUTER_BYTES for n in u]
+    gbs = sum(bytes_step) / (sum(step_ms) * 1e-3) / 1e9
+    # dominant kernel by device time
+    launches = {k: nprof for k in stages}
+    dom = max(stages, key=lambda k: stages[k])
+    dom_avg_s = stages[dom] / max(nprof, 1) * 1e-3
+    gu_bytes = sum((n + S) * GU_BYTES for n in u) / len(u) + T * H * xs.element_size() + (T * K + T * S) * I * 4
+    down_bytes = sum((n + S) * DOWN_BYTES for n in u) / len(u) + (T * K + T * S) * (I + H) * 4
+    alg = {"gateup": gu_bytes, "down": down_bytes, "router": ROUTER_BYTES + T * H * xs.element_size()}
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except OSError:
+        pass
+    peak_gbs = peaks.get("hbm_gbs", 6650.0)
+    roof = None
+    if dom in alg:
+        ach = alg[dom] / dom_avg_s / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak_gbs, "unit": "GB/s",
+                "frac": round(ach / peak_gbs, 4), "traffic": None,
+                "peak_source": "measured" if "hbm_gbs" in peaks else "fallback",
+                "bytes_per_launch": int(alg[dom]), "avg_launch_us": round(dom_avg_s * 1e6, 2)}
+    out = {
+        "metric": METRIC, "value": round(tokens / (total_ms * 1e-3), 2), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl["bf16"] else "f32",
+        "data": "synthetic (seeded generator; random-init int4 weights of the full-size layer shape)",
+        "config": {"workload": args.workload, "desc": wl["desc"], "hidden": H, "inter": I, "experts": E,
+                   "top_k": K, "shared": S, "tokens_per_step": T, "weights": "int4 gs64 + fp16 scales",
+                   "l2": "flushed between steps (256 MiB memset outside the step events)",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / 8000.0, 4),
+        "hbm_frac_of_measured": round(gbs / peak_gbs, 4),
+        "unique_experts_per_step": round(mean_unique, 2),
+        "bytes_per_step": int(sum(bytes_step) / len(bytes_step)),
+        "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items()},
+        "roofline": roof,
+        "gpu_launches": 6 * args.steps,
+        "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * xs.element_size(), "d2h_bytes_per_step": T * H * xs.element_size()},
+        "clocks": clk,
+    }
+    layer.close()
+    if dist:
+        dist.destroy_process_group()
+    return out
+
+
+def main():
+    args = parse()
+    wl = WORKLOADS[args.workload]
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        leg = OracleLeg(wl)
+        for i in range(args.warmup):
+            leg.step(i)
+        tok, total = 0, 0.0
+        for i in range(args.warmup, args.warmup + args.steps):
+            n, dt = leg.step(i)
+            tok += n
+            total += dt
+        val = tok / total
+        cb = {"value": round(val, 4), "unit": "tokens/s", "cores": leg.cores(), "kind": "oracle",
+              "sample": f"{args.steps} steps, each the fp64 oracle on {leg.Ts} token(s) of the step's batch "
+                        f"(input and expert generation untimed)"}
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "tokens/s",
+                          "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                          "data": "synthetic", "config": {"workload": args.workload, "desc": wl["desc"]},
+                          "cpu_baseline": cb,
+                          "e2e": {"value": round(val, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return 0
+
+    # the CPU oracle sample runs first (before any CUDA call in this process)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(wl, args.cpu_seconds)
+    out = run_ours(args, wl, ws, rank, local)
+    if out is not None:
+        out["cpu_baseline"] = cpu
+        print(json.dumps(out))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,177 @@
+/*
+ * coli_moe.h -- C ABI of the int4 expert-FFN MoE layer for one NVIDIA B200.
+ *
+ * The layer is the sparse MoE block of the Colibri engine pages:
+ *   "Colibri: 2400 lines of pure C ..." (kechuai.cn/articles/colibri),
+ *     section 一: every layer routes each token to 8 of its 256 experts; the
+ *     shared expert belongs to the always-on dense part; an int4 expert is
+ *     about 19 MB; section 二: an expert's three matrices are stored
+ *     adjacently and a batch reads each unique expert once (batch-union);
+ *   "colibri" project page (gh.puless.com/p/colibri.html), section on
+ *     correctness: the int4 container uses groups of 64 (gs64).
+ * Readings where the pages are silent: router scores are the logits
+ * Wr x + b; the top-k is taken in descending logit order, equal logits going
+ * to the lower expert id; routing weights are the softmax over the k selected
+ * logits; each expert is a SwiGLU FFN  D (silu(G x) * (U x)); shared experts
+ * have weight 1; y = sum(shared) + sum_k w_k E_k(x).
+ *
+ * Conventions
+ *  - Every call returns a coli_status. Argument errors return COLI_EINVAL
+ *    before any work is enqueued and change nothing. CUDA failures return
+ *    COLI_ECUDA; coli_last_error() gives the message (thread-local).
+ *    The library never prints, exits or aborts.
+ *  - A `coli_stream` is a cudaStream_t passed as void* (NULL: legacy default
+ *    stream). Route and forward are asynchronous and stream-ordered; their
+ *    tensor arguments are DEVICE pointers on the layer's device.
+ *  - A layer owns its weights and a workspace sized for cfg.max_tokens. The
+ *    workspace is single-stream: calls on one layer must not overlap.
+ *  - Dimensions: hidden % 128 == 0, inter % 64 == 0, group_size == 64,
+ *    1 <= top_k <= n_experts <= 1024, n_shared >= 0, max_tokens >= 1.
+ */
+#ifndef COLI_MOE_H
+#define COLI_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    COLI_OK = 0,
+    COLI_EINVAL = 1,       /* bad argument (null, size, alignment, dtype)      */
+    COLI_ENOMEM = 2,       /* device or host allocation failed                  */
+    COLI_ECUDA = 3,        /* a CUDA call or kernel launch failed               */
+    COLI_EUNSUPPORTED = 4  /* valid request this build does not implement       */
+} coli_status;
+
+typedef enum { COLI_F32 = 0, COLI_BF16 = 1 } coli_dtype;
+
+typedef void* coli_stream; /* cudaStream_t */
+
+typedef struct {
+    int hidden;      /* H: model width (input of gate/up, output of down)           */
+    int inter;       /* I: expert intermediate width                               */
+    int n_experts;   /* E: routed experts (256 in the pages' model)                */
+    int top_k;       /* K: experts per token (8 in the pages' model)               */
+    int n_shared;    /* always-on shared experts, weight 1 each                    */
+    int group_size;  /* must be 64: one fp16 scale per 64 inputs of a row          */
+    int max_tokens;  /* largest n_tokens a route/forward call may pass             */
+} coli_moe_config;
+
+typedef struct coli_moe_layer coli_moe_layer; /* opaque */
+
+/*
+ * Create a layer on `device` from canonical weights.
+ *
+ * router_w    [E][H] fp32, row-major.
+ * router_bias [E] fp32, or NULL for zero bias. The bias enters the logits, so
+ *             it moves both the selection and the weights.
+ * expert_q    canonical int4 weights of the E routed experts, expert after
+ *             expert; one expert is  gate [I][H/2] | up [I][H/2] | down [H][I/2]
+ *             bytes (3*H*I/2 per expert). Byte j of a row holds elements 2j
+ *             (low nibble) and 2j+1 (high nibble) as two's complement codes.
+ * expert_scales  fp16 bit patterns, expert after expert:
+ *             gate [I][H/64] | up [I][H/64] | down [H][I/64] (3*H*I/64 per
+ *             expert); element c of row r is code(r, c) * scale(r, c/64).
+ * shared_q / shared_scales  the n_shared shared experts, same layout (NULL
+ *             when n_shared == 0).
+ * Every input pointer may be host or device memory (detected per pointer) and
+ * is only read during the call; the caller keeps ownership. expert_q and
+ * shared_q may be NULL (with their scales NULL) to create a layer whose
+ * experts are loaded afterwards with coli_moe_layer_set_experts.
+ * The call is synchronous. On failure *out is NULL and nothing leaks.
+ */
+coli_status coli_moe_layer_create(const coli_moe_config* cfg, const float* router_w, const float* router_bias,
+                                  const uint8_t* expert_q, const uint16_t* expert_scales,
+                                  const uint8_t* shared_q, const uint16_t* shared_scales,
+                                  int device, coli_moe_layer** out);
+
+/*
+ * (Re)load `count` experts starting at expert id `first` (routed ids
+ * 0..E-1, shared ids E..E+n_shared-1) from canonical buffers holding `count`
+ * consecutive experts (layout as in coli_moe_layer_create; host or device).
+ * Synchronous.
+ */
+coli_status coli_moe_layer_set_experts(coli_moe_layer* layer, int first, int count,
+                                       const uint8_t* q, const uint16_t* scales);
+
+void coli_moe_layer_destroy(coli_moe_layer* layer);
+
+/* Copy of the layer's configuration. */
+coli_status coli_moe_layer_config(const coli_moe_layer* layer, coli_moe_config* cfg);
+
+/*
+ * Router only: ids[t][k] (int32) and weights[t][k] (fp32, summing to 1 per
+ * token) for x [n_tokens][H] (fp32 or bf16 bits). Logits are accumulated in
+ * fp64 from the exact products of fp32 inputs. 0 <= n_tokens <= max_tokens.
+ */
+coli_status coli_moe_route(coli_moe_layer* layer, const void* x, coli_dtype dtype, int n_tokens,
+                           int32_t* ids, float* weights, coli_stream stream);
+
+/*
+ * The layer: y [n_tokens][H] = MoE(x), y of the same dtype as x. x and y must
+ * not overlap. fp32 runs the CUDA-core path; bf16 the tensor-core path where
+ * an expert has enough tokens for a dense contraction.
+ */
+coli_status coli_moe_forward(coli_moe_layer* layer, const void* x, void* y, coli_dtype dtype, int n_tokens,
+                             coli_stream stream);
+
+/*
+ * Residual stack over fp32 activations, in place:
+ *   x <- x + MoE_l(RMSNorm(x)) for l = 0..n_layers-1,
+ * RMSNorm with unit gain: x / sqrt(mean(x^2) + eps). All layers must share
+ * H and live on one device; n_tokens <= every layer's max_tokens.
+ */
+coli_status coli_moe_stack_forward(coli_moe_layer* const* layers, int n_layers, float* x, int n_tokens,
+                                   float eps, coli_stream stream);
+
+/*
+ * Statistics of the last forward on this layer (synchronises its stream):
+ * number of distinct routed experts, bytes of expert and router weights the
+ * plan streams ((unique + n_shared) * expert bytes + router bytes), and, if
+ * per_expert_counts != NULL, the routed-slot count of each of the E experts.
+ */
+coli_status coli_moe_get_stats(coli_moe_layer* layer, int* n_unique, int64_t* bytes_streamed,
+                               int32_t* per_expert_counts);
+
+/*
+ * The batch-union plan of the last forward (synchronises; host outputs, any
+ * of them NULL to skip):
+ *   ids [T][K], weights [T][K]      routing
+ *   counts [E], offsets [E+1]       slots per expert and their exclusive scan
+ *   unique [E], *n_unique           distinct experts, ascending
+ *   pos [T][K]                      position of slot (t,k) in the permuted list
+ *   tok [T*K]                       token of each permuted position
+ * T is the n_tokens of that forward.
+ */
+coli_status coli_moe_get_plan(coli_moe_layer* layer, int32_t* ids, float* weights, int32_t* counts,
+                              int32_t* offsets, int32_t* unique, int32_t* n_unique, int32_t* pos, int32_t* tok);
+
+/*
+ * Per-stage device timing of forward calls, for profiling. While enabled,
+ * every forward records CUDA events between its kernels on its own stream
+ * (no host synchronisation; a ring of event sets is recycled, folding each
+ * finished forward into running totals). coli_moe_get_profile waits for the
+ * profiled forwards to finish and writes, per stage, the total device ms over
+ * all forwards since profiling was enabled, and their number. Enabling again
+ * resets the totals.
+ */
+enum { COLI_STAGE_ROUTER = 0, COLI_STAGE_TOPK, COLI_STAGE_PLAN, COLI_STAGE_GATEUP, COLI_STAGE_DOWN,
+       COLI_STAGE_COMBINE, COLI_N_STAGES };
+coli_status coli_moe_set_profiling(coli_moe_layer* layer, int enable);
+coli_status coli_moe_get_profile(coli_moe_layer* layer, double* stage_ms_total, int64_t* n_forwards);
+const char* coli_moe_stage_name(int stage);
+
+/* Bytes of one expert in the int4 gs64 container (nibbles + fp16 scales). */
+int64_t coli_moe_expert_bytes(int hidden, int inter);
+
+const char* coli_status_string(coli_status status);
+/* Detail of the last failure on the calling thread ("" if none). */
+const char* coli_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* COLI_MOE_H */

@@ -1,0 +1,204 @@
+"""Python binding of the int4 expert-FFN MoE layer (``libcoli_moe.so``).
+
+Argument marshalling only: every step of the layer runs in the CUDA library
+behind the C ABI declared in ``include/coli_moe.h``. Tensors are passed as raw
+pointers (``torch.Tensor.data_ptr()`` or numpy arrays for host inputs of
+``Layer``); streams as ``torch.cuda.Stream.cuda_stream`` handles. If the
+library is missing this module raises at import: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libcoli_moe.so")
+
+COLI_OK, COLI_EINVAL, COLI_ENOMEM, COLI_ECUDA, COLI_EUNSUPPORTED = range(5)
+F32, BF16 = 0, 1
+
+# Every symbol the header declares.
+EXPORTS = (
+    "coli_moe_layer_create", "coli_moe_layer_set_experts", "coli_moe_layer_destroy", "coli_moe_layer_config",
+    "coli_moe_route", "coli_moe_forward", "coli_moe_stack_forward", "coli_moe_get_stats", "coli_moe_get_plan",
+    "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
+    "coli_moe_get_profile", "coli_moe_stage_name",
+)
+N_STAGES = 6
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("n_experts", ctypes.c_int),
+                ("top_k", ctypes.c_int), ("n_shared", ctypes.c_int), ("group_size", ctypes.c_int),
+                ("max_tokens", ctypes.c_int)]
+
+
+class ColiError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: status {status} ({detail})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                          "(the CUDA library is required; there is no CPU path)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    pcfg = ctypes.POINTER(Config)
+    L.coli_moe_layer_create.argtypes = [pcfg, vp, vp, vp, vp, vp, vp, i32, ctypes.POINTER(vp)]
+    L.coli_moe_layer_set_experts.argtypes = [vp, i32, i32, vp, vp]
+    L.coli_moe_layer_destroy.argtypes = [vp]
+    L.coli_moe_layer_destroy.restype = None
+    L.coli_moe_layer_config.argtypes = [vp, pcfg]
+    L.coli_moe_route.argtypes = [vp, vp, i32, i32, vp, vp, vp]
+    L.coli_moe_forward.argtypes = [vp, vp, vp, i32, i32, vp]
+    L.coli_moe_stack_forward.argtypes = [vp, i32, vp, i32, f32, vp]
+    L.coli_moe_get_stats.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_int64), vp]
+    L.coli_moe_get_plan.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(i32), vp, vp]
+    L.coli_moe_expert_bytes.argtypes = [i32, i32]
+    L.coli_moe_expert_bytes.restype = ctypes.c_int64
+    L.coli_moe_set_profiling.argtypes = [vp, i32]
+    L.coli_moe_get_profile.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int64)]
+    L.coli_moe_stage_name.argtypes = [i32]
+    L.coli_moe_stage_name.restype = ctypes.c_char_p
+    L.coli_status_string.argtypes = [i32]
+    L.coli_status_string.restype = ctypes.c_char_p
+    L.coli_last_error.argtypes = []
+    L.coli_last_error.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != COLI_OK:
+        raise ColiError(status, where, (lib.coli_last_error() or b"").decode())
+
+
+def _ptr(a) -> int | None:
+    """Address of a torch tensor or numpy array (None stays None)."""
+    if a is None:
+        return None
+    if hasattr(a, "data_ptr"):
+        return a.data_ptr() if a.numel() else None
+    if hasattr(a, "ctypes"):
+        if not a.flags["C_CONTIGUOUS"]:
+            raise ValueError("array must be C-contiguous")
+        return a.ctypes.data
+    return int(a)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        try:
+            import torch
+            return torch.cuda.current_stream().cuda_stream
+        except Exception:
+            return None
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _dtype_of(t) -> int:
+    name = str(getattr(t, "dtype", ""))
+    if name.endswith("float32"):
+        return F32
+    if name.endswith("bfloat16") or name.endswith("uint16") or name.endswith("int16"):
+        return BF16
+    raise TypeError(f"unsupported activation dtype {name}")
+
+
+def expert_bytes(hidden: int, inter: int) -> int:
+    return lib.coli_moe_expert_bytes(hidden, inter)
+
+
+class Layer:
+    """One MoE layer resident on a CUDA device."""
+
+    def __init__(self, cfg: Config, router_w, router_bias=None, expert_q=None, expert_scales=None,
+                 shared_q=None, shared_scales=None, device: int = 0):
+        h = ctypes.c_void_p()
+        _check(lib.coli_moe_layer_create(ctypes.byref(cfg), _ptr(router_w), _ptr(router_bias), _ptr(expert_q),
+                                         _ptr(expert_scales), _ptr(shared_q), _ptr(shared_scales), device,
+                                         ctypes.byref(h)), "coli_moe_layer_create")
+        self._h = h
+        self.cfg = cfg
+        self.device = device
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise ValueError("layer is destroyed")
+        return self._h
+
+    def set_experts(self, first: int, count: int, q, scales) -> None:
+        _check(lib.coli_moe_layer_set_experts(self.handle, first, count, _ptr(q), _ptr(scales)),
+               "coli_moe_layer_set_experts")
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None:
+            lib.coli_moe_layer_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def route(self, x, ids, weights, n_tokens: int | None = None, stream=None) -> None:
+        T = x.shape[0] if n_tokens is None else n_tokens
+        _check(lib.coli_moe_route(self.handle, _ptr(x), _dtype_of(x), T, _ptr(ids), _ptr(weights), _stream(stream)),
+               "coli_moe_route")
+
+    def forward(self, x, y, n_tokens: int | None = None, stream=None) -> None:
+        T = x.shape[0] if n_tokens is None else n_tokens
+        _check(lib.coli_moe_forward(self.handle, _ptr(x), _ptr(y), _dtype_of(x), T, _stream(stream)),
+               "coli_moe_forward")
+
+    def stats(self, counts=None):
+        nu = ctypes.c_int()
+        b = ctypes.c_int64()
+        _check(lib.coli_moe_get_stats(self.handle, ctypes.byref(nu), ctypes.byref(b), _ptr(counts)),
+               "coli_moe_get_stats")
+        return nu.value, b.value
+
+    def set_profiling(self, on: bool) -> None:
+        _check(lib.coli_moe_set_profiling(self.handle, 1 if on else 0), "coli_moe_set_profiling")
+
+    def profile(self):
+        """(stage name -> total device ms, number of forwards) since profiling was enabled."""
+        buf = (ctypes.c_double * N_STAGES)()
+        n = ctypes.c_int64()
+        _check(lib.coli_moe_get_profile(self.handle, ctypes.cast(buf, ctypes.c_void_p), ctypes.byref(n)),
+               "coli_moe_get_profile")
+        return {lib.coli_moe_stage_name(i).decode(): float(buf[i]) for i in range(N_STAGES)}, n.value
+
+    def plan(self, T: int):
+        """Host copies of the last forward's routing and batch-union plan."""
+        import numpy as np
+        E, K = self.cfg.n_experts, self.cfg.top_k
+        out = dict(ids=np.zeros((T, K), np.int32), weights=np.zeros((T, K), np.float32),
+                   cnt=np.zeros(E, np.int32), off=np.zeros(E + 1, np.int32), unique=np.zeros(E, np.int32),
+                   pos=np.zeros((T, K), np.int32), tok=np.zeros(max(T * K, 1), np.int32))
+        nu = ctypes.c_int()
+        _check(lib.coli_moe_get_plan(self.handle, _ptr(out["ids"]), _ptr(out["weights"]), _ptr(out["cnt"]),
+                                     _ptr(out["off"]), _ptr(out["unique"]), ctypes.byref(nu), _ptr(out["pos"]),
+                                     _ptr(out["tok"])), "coli_moe_get_plan")
+        out["unique"] = out["unique"][:nu.value]
+        out["tok"] = out["tok"][:T * K]
+        return out
+
+
+def stack_forward(layers, x, n_tokens: int | None = None, eps: float = 1e-6, stream=None) -> None:
+    """x <- x + MoE_l(RMSNorm(x)) over the layers, in place on fp32 x."""
+    T = x.shape[0] if n_tokens is None else n_tokens
+    arr = (ctypes.c_void_p * len(layers))(*[l.handle.value for l in layers])
+    _check(lib.coli_moe_stack_forward(ctypes.cast(arr, ctypes.c_void_p), len(layers), _ptr(x), T, eps,
+                                      _stream(stream)), "coli_moe_stack_forward")
+
+
+def make_config(hidden, inter, n_experts, top_k, n_shared, max_tokens) -> Config:
+    return Config(hidden=hidden, inter=inter, n_experts=n_experts, top_k=top_k, n_shared=n_shared,
+                  group_size=64, max_tokens=max_tokens)

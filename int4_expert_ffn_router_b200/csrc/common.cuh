@@ -1,0 +1,98 @@
+// common.cuh -- shared definitions of the CUDA path: device weight layout,
+// workspace, launch helpers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/coli_moe.h"
+
+namespace coli {
+
+// ---------------------------------------------------------------------------
+// Device-native weight layout (written once by the repack at create).
+//
+// A matrix of R rows (R % 128 == 0) and C inputs (C % 64 == 0) is stored as
+// blocks of 128 rows x one 64-input group:
+//     block(rt, g) at ((rt * C/64) + g) * kBlockBytes
+// so the 128-row tile `rt` is one contiguous run over its groups. A block is
+//     nibbles [8 sub-tiles of 16 rows][32 lanes][16 bytes]  (4096 B)
+//     scales  [8 sub-tiles][8] x {fp16 of row i, fp16 of row i+8} (256 B)
+// Lane l = 4*gi + ti of a sub-tile owns rows gi and gi+8 and, for each
+// 16-input step s = 0..3 of the group, the inputs 16s + {2ti, 2ti+1, 2ti+8,
+// 2ti+9}: 32 nibbles in four 32-bit words, word s holding
+//     bits 0-3  (row gi,   col 2ti)    bits 16-19 (row gi,   col 2ti+1)
+//     bits 4-7  (row gi+8, col 2ti)    bits 20-23 (row gi+8, col 2ti+1)
+//     bits 8-11 (row gi,   col 2ti+8)  bits 24-27 (row gi,   col 2ti+9)
+//     bits 12-15(row gi+8, col 2ti+8)  bits 28-31 (row gi+8, col 2ti+9)
+// as offset-binary codes v = q + 8 in [0, 15]. This is the A-fragment order
+// of a 16x16 tensor-core tile, and it lets a CUDA-core lane turn each nibble
+// into a float with one logic op (the nibble lands in an fp32 mantissa).
+//
+// Gate and up are stored as one matrix of 2I rows interleaved by 8: rows
+// 16b..16b+7 are gate rows 8b..8b+7 and rows 16b+8..16b+15 are up rows
+// 8b..8b+7, so the lane that owns row gi also owns the matching up row gi+8
+// and SwiGLU is formed in registers.
+// ---------------------------------------------------------------------------
+constexpr int kGroup = 64;
+constexpr int kTileRows = 128;
+constexpr int kSubRows = 16;
+constexpr int kNibbleBytes = 4096;
+constexpr int kScaleBytes = 256;
+constexpr int kBlockBytes = kNibbleBytes + kScaleBytes;  // 4352
+
+inline int64_t matrix_bytes(int rows, int cols) {
+    return (int64_t)(rows / kTileRows) * (cols / kGroup) * kBlockBytes;
+}
+
+struct Dims {
+    int H, I, E, K, S, max_tokens;
+    int64_t gu_bytes;      // gate/up matrix [2I][H]
+    int64_t d_bytes;       // down matrix [H][I]
+    int64_t expert_stride; // gu_bytes + d_bytes (multiple of 256)
+};
+
+// Per-call workspace views (device pointers into the layer's workspace).
+struct Plan {
+    int32_t* ids;        // [T][K]
+    float* w;            // [T][K]
+    int32_t* cnt;        // [E]
+    int32_t* off;        // [E+1]
+    int32_t* unique;     // [E]
+    int32_t* n_unique;   // [1]
+    int32_t* pos;        // [T][K] -> permuted position
+    int32_t* tok;        // [T*K + S*T] permuted token list (shared experts appended)
+    int32_t* act_expert; // [E+S] expert id of active slot a (unique experts, then shared)
+    int32_t* act_off;    // [E+S] first permuted position of active expert a
+    int32_t* act_cnt;    // [E+S] tokens of active expert a
+    int32_t* n_active;   // [1] n_unique + S
+};
+
+// ---------------------------------------------------------------------------
+// Small device helpers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t ldg_stream32(const void* p) {
+    uint32_t r;
+    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t orv) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(orv));  // (a & b) | c
+    return d;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+}  // namespace coli

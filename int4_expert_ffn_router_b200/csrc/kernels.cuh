@@ -1,0 +1,37 @@
+// kernels.cuh -- launchers of the CUDA path (defined in router.cu, ffn_core.cu,
+// repack.cu, combine.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace coli {
+
+// router.cu
+cudaError_t launch_router_logits(const float* wr, const float* bias, const void* x, coli_dtype dt, int T, int H, int E,
+                                 double* logits, cudaStream_t st);
+cudaError_t launch_topk(const double* logits, int T, int E, int K, int32_t* ids, float* w, cudaStream_t st);
+size_t plan_smem_bytes(int E);
+cudaError_t launch_plan(const int32_t* ids, int T, int K, int E, int S, const Plan& p, cudaStream_t st);
+
+// repack.cu: canonical matrix [R][C] (nibbles + fp16 scales, device memory)
+// into the device layout. `interleave_gu`: src0 = gate [I][H], src1 = up
+// [I][H], written as one [2I][H] matrix interleaved by 8 rows.
+cudaError_t launch_repack(const uint8_t* q0, const uint16_t* s0, const uint8_t* q1, const uint16_t* s1, int R, int C,
+                          bool interleave_gu, uint8_t* dst, cudaStream_t st);
+
+// ffn_core.cu: CUDA-core int4 expert matrices over the active experts.
+// Gate/up + SwiGLU: h[pos][I] (fp32) for every active (expert, token).
+cudaError_t launch_gateup_core(const uint8_t* weights, const Dims& d, const void* x, coli_dtype dt, int T,
+                               const Plan& p, float* h, int max_active, int n_sm, cudaStream_t st);
+// Down: o[pos][H] (fp32) for every active (expert, token).
+cudaError_t launch_down_core(const uint8_t* weights, const Dims& d, const float* h, int T, const Plan& p, float* o,
+                             int max_active, int n_sm, cudaStream_t st);
+
+// combine.cu
+// y[t] = residual[t] (optional) + sum_j o[TK + j*T + t] + sum_k w[t][k] o[pos[t][k]]
+cudaError_t launch_combine(const float* o, const Plan& p, int T, int H, int K, int S, const float* residual, void* y,
+                           coli_dtype ydt, cudaStream_t st);
+// out[t] = x[t] / sqrt(mean(x[t]^2) + eps), fp64 statistics, fp32 output
+cudaError_t launch_rmsnorm(const float* x, int T, int H, float eps, float* out, cudaStream_t st);
+
+}  // namespace coli

@@ -1,0 +1,443 @@
+// layer.cu -- the C ABI (include/coli_moe.h): layer object, weight upload and
+// repack, workspace, and the forward sequence on one stream.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+#define COLI_API extern "C" __attribute__((visibility("default")))
+
+using namespace coli;
+
+namespace {
+thread_local std::string g_last_error;
+
+coli_status fail(coli_status s, const char* what) {
+    g_last_error = what;
+    return s;
+}
+
+coli_status cuda_fail(cudaError_t e, const char* where) {
+    g_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+    return COLI_ECUDA;
+}
+
+#define CUDA_TRY(call, where)                         \
+    do {                                              \
+        cudaError_t _e = (call);                      \
+        if (_e != cudaSuccess) return cuda_fail(_e, where); \
+    } while (0)
+
+size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// Switches to `dev` for the lifetime of the guard.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+        if (prev != dev) ok = cudaSetDevice(dev) == cudaSuccess;
+    }
+    ~DeviceGuard() {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+bool is_device_ptr(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+}  // namespace
+
+struct coli_moe_layer {
+    coli_moe_config cfg;
+    Dims d;
+    int device = 0;
+    int n_sm = 148;
+    int max_active = 0;
+    uint8_t* weights = nullptr;
+    float* router_w = nullptr;
+    float* router_b = nullptr;
+    uint8_t* ws = nullptr;
+    size_t ws_bytes = 0;
+    double* logits = nullptr;
+    Plan plan{};
+    float* h = nullptr;
+    float* o = nullptr;
+    float* xn = nullptr;
+    uint8_t* staging = nullptr;  // one canonical expert, for host sources
+    int last_T = -1;
+    cudaStream_t last_stream = nullptr;
+    // profiling: a ring of event sets, folded into totals when recycled
+    static constexpr int kRing = 64;
+    bool profiling = false;
+    int prof_next = 0;                 // ring slot of the next forward
+    int64_t prof_issued = 0;           // forwards recorded since enable
+    int64_t prof_folded = 0;           // forwards folded into the totals
+    double prof_total[COLI_N_STAGES] = {};
+    cudaEvent_t ev[kRing][COLI_N_STAGES + 1] = {};
+};
+
+// Adds the durations of ring slot `r` to the totals (waits for its last event).
+static cudaError_t prof_fold(coli_moe_layer* L, int r) {
+    cudaError_t e = cudaEventSynchronize(L->ev[r][COLI_N_STAGES]);
+    if (e != cudaSuccess) return e;
+    for (int i = 0; i < COLI_N_STAGES; ++i) {
+        float ms = 0.0f;
+        e = cudaEventElapsedTime(&ms, L->ev[r][i], L->ev[r][i + 1]);
+        if (e != cudaSuccess) return e;
+        L->prof_total[i] += ms;
+    }
+    L->prof_folded += 1;
+    return cudaSuccess;
+}
+
+// Records the boundary before stage `i` of the current forward
+// (i == COLI_N_STAGES: after the last stage).
+static void prof_mark(coli_moe_layer* L, int i, cudaStream_t s) {
+    if (L->profiling) cudaEventRecord(L->ev[L->prof_next][i], s);
+}
+
+static coli_status check_cfg(const coli_moe_config* c) {
+    if (!c) return fail(COLI_EINVAL, "config is NULL");
+    if (c->hidden <= 0 || c->hidden % 128) return fail(COLI_EINVAL, "hidden must be a positive multiple of 128");
+    if (c->inter <= 0 || c->inter % 64) return fail(COLI_EINVAL, "inter must be a positive multiple of 64");
+    if (c->group_size != 64) return fail(COLI_EINVAL, "group_size must be 64");
+    if (c->n_experts < 1 || c->n_experts > 1024) return fail(COLI_EINVAL, "n_experts must be in [1, 1024]");
+    if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > 32) return fail(COLI_EINVAL, "top_k must be in [1, min(n_experts, 32)]");
+    if (c->n_shared < 0 || c->n_shared > 64) return fail(COLI_EINVAL, "n_shared must be in [0, 64]");
+    if (c->max_tokens < 1 || c->max_tokens > (1 << 20)) return fail(COLI_EINVAL, "max_tokens must be in [1, 2^20]");
+    if ((int64_t)c->max_tokens * c->top_k > (1 << 24)) return fail(COLI_EINVAL, "max_tokens * top_k too large");
+    return COLI_OK;
+}
+
+static void free_layer(coli_moe_layer* L) {
+    if (!L) return;
+    if (L->weights) cudaFree(L->weights);
+    if (L->router_w) cudaFree(L->router_w);
+    if (L->router_b) cudaFree(L->router_b);
+    if (L->ws) cudaFree(L->ws);
+    if (L->staging) cudaFree(L->staging);
+    for (auto& set : L->ev)
+        for (auto& e : set)
+            if (e) cudaEventDestroy(e);
+    delete L;
+}
+
+COLI_API int64_t coli_moe_expert_bytes(int hidden, int inter) {
+    return 3LL * hidden * inter / 2 + 3LL * hidden * inter / 64 * 2;
+}
+
+COLI_API coli_status coli_moe_layer_set_experts(coli_moe_layer* L, int first, int count, const uint8_t* q,
+                                                const uint16_t* scales) {
+    if (!L || !q || !scales) return fail(COLI_EINVAL, "NULL layer or weights");
+    const int total = L->cfg.n_experts + L->cfg.n_shared;
+    if (first < 0 || count < 0 || first + count > total) return fail(COLI_EINVAL, "expert range out of bounds");
+    if (((uintptr_t)scales) & 1u) return fail(COLI_EINVAL, "scales must be 2-byte aligned");
+    DeviceGuard guard(L->device);
+    if (!guard.ok) return fail(COLI_ECUDA, "cudaSetDevice failed");
+    const int H = L->d.H, I = L->d.I;
+    const size_t nq = 3ull * H * I / 2, ns = 3ull * H * I / 64;
+    const size_t mq = (size_t)I * H / 2, ms = (size_t)I * H / 64;
+    const bool dev_q = is_device_ptr(q), dev_s = is_device_ptr(scales);
+    for (int i = 0; i < count; ++i) {
+        const uint8_t* eq = q + (size_t)i * nq;
+        const uint16_t* es = scales + (size_t)i * ns;
+        if (!dev_q || !dev_s) {
+            if (!L->staging) CUDA_TRY(cudaMalloc(&L->staging, align256(nq) + ns * 2), "cudaMalloc(staging)");
+            CUDA_TRY(cudaMemcpy(L->staging, eq, nq, cudaMemcpyDefault), "copy expert nibbles");
+            CUDA_TRY(cudaMemcpy(L->staging + align256(nq), es, ns * 2, cudaMemcpyDefault), "copy expert scales");
+            eq = L->staging;
+            es = reinterpret_cast<const uint16_t*>(L->staging + align256(nq));
+        }
+        uint8_t* dst = L->weights + (size_t)(first + i) * L->d.expert_stride;
+        CUDA_TRY(launch_repack(eq, es, eq + mq, es + ms, 2 * I, H, true, dst, 0), "repack gate/up");
+        CUDA_TRY(launch_repack(eq + 2 * mq, es + 2 * ms, nullptr, nullptr, H, I, false, dst + L->d.gu_bytes, 0),
+                 "repack down");
+        if (!dev_q || !dev_s) CUDA_TRY(cudaDeviceSynchronize(), "repack");  // staging is reused
+    }
+    CUDA_TRY(cudaDeviceSynchronize(), "repack");
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const float* router_w, const float* router_bias,
+                                           const uint8_t* expert_q, const uint16_t* expert_scales,
+                                           const uint8_t* shared_q, const uint16_t* shared_scales, int device,
+                                           coli_moe_layer** out) {
+    if (!out) return fail(COLI_EINVAL, "out is NULL");
+    *out = nullptr;
+    coli_status st = check_cfg(cfg);
+    if (st != COLI_OK) return st;
+    if (!router_w) return fail(COLI_EINVAL, "router_w is NULL");
+    if ((expert_q == nullptr) != (expert_scales == nullptr)) return fail(COLI_EINVAL, "expert_q/expert_scales: both or neither");
+    if ((shared_q == nullptr) != (shared_scales == nullptr)) return fail(COLI_EINVAL, "shared_q/shared_scales: both or neither");
+    if (cfg->n_shared == 0 && shared_q) return fail(COLI_EINVAL, "shared weights given with n_shared == 0");
+    int ndev = 0;
+    if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+        cudaGetLastError();
+        return fail(COLI_EINVAL, "no such CUDA device");
+    }
+    DeviceGuard guard(device);
+    if (!guard.ok) return fail(COLI_ECUDA, "cudaSetDevice failed");
+
+    coli_moe_layer* L = new (std::nothrow) coli_moe_layer();
+    if (!L) return fail(COLI_ENOMEM, "host allocation failed");
+    L->cfg = *cfg;
+    L->device = device;
+    Dims& d = L->d;
+    d.H = cfg->hidden; d.I = cfg->inter; d.E = cfg->n_experts; d.K = cfg->top_k; d.S = cfg->n_shared;
+    d.max_tokens = cfg->max_tokens;
+    d.gu_bytes = matrix_bytes(2 * d.I, d.H);
+    d.d_bytes = matrix_bytes(d.H, d.I);
+    d.expert_stride = (int64_t)align256((size_t)(d.gu_bytes + d.d_bytes));
+    cudaDeviceGetAttribute(&L->n_sm, cudaDevAttrMultiProcessorCount, device);
+    const int Tm = d.max_tokens;
+    L->max_active = (int)std::min<int64_t>((int64_t)Tm * d.K, d.E) + d.S;
+
+    auto bail = [&](cudaError_t e, const char* where) {
+        coli_status s = (e == cudaErrorMemoryAllocation) ? fail(COLI_ENOMEM, where) : cuda_fail(e, where);
+        cudaGetLastError();
+        free_layer(L);
+        return s;
+    };
+    cudaError_t e;
+    if ((e = cudaMalloc(&L->weights, (size_t)(d.E + d.S) * d.expert_stride)) != cudaSuccess) return bail(e, "cudaMalloc(weights)");
+    if ((e = cudaMalloc(&L->router_w, (size_t)d.E * d.H * 4)) != cudaSuccess) return bail(e, "cudaMalloc(router)");
+    if ((e = cudaMalloc(&L->router_b, (size_t)d.E * 4)) != cudaSuccess) return bail(e, "cudaMalloc(bias)");
+
+    // workspace
+    const size_t TK = (size_t)Tm * d.K, slots = TK + (size_t)d.S * Tm, EA = (size_t)d.E + d.S;
+    size_t sz[] = {Tm * (size_t)d.E * 8, TK * 4, TK * 4, (size_t)d.E * 4, (size_t)(d.E + 1) * 4, (size_t)d.E * 4, 4,
+                   TK * 4, slots * 4, EA * 4, EA * 4, EA * 4, 4, slots * d.I * 4, slots * d.H * 4, (size_t)Tm * d.H * 4};
+    size_t total = 0;
+    for (size_t s : sz) total += align256(s);
+    if ((e = cudaMalloc(&L->ws, total)) != cudaSuccess) return bail(e, "cudaMalloc(workspace)");
+    L->ws_bytes = total;
+    uint8_t* cur = L->ws;
+    void* ptrs[16];
+    for (int i = 0; i < 16; ++i) { ptrs[i] = cur; cur += align256(sz[i]); }
+    L->logits = (double*)ptrs[0];
+    Plan& p = L->plan;
+    p.ids = (int32_t*)ptrs[1]; p.w = (float*)ptrs[2]; p.cnt = (int32_t*)ptrs[3]; p.off = (int32_t*)ptrs[4];
+    p.unique = (int32_t*)ptrs[5]; p.n_unique = (int32_t*)ptrs[6]; p.pos = (int32_t*)ptrs[7]; p.tok = (int32_t*)ptrs[8];
+    p.act_expert = (int32_t*)ptrs[9]; p.act_off = (int32_t*)ptrs[10]; p.act_cnt = (int32_t*)ptrs[11];
+    p.n_active = (int32_t*)ptrs[12];
+    L->h = (float*)ptrs[13]; L->o = (float*)ptrs[14]; L->xn = (float*)ptrs[15];
+    if ((e = cudaMemset(L->ws, 0, total)) != cudaSuccess) return bail(e, "cudaMemset(workspace)");
+    if ((e = cudaMemset(L->weights, 0, (size_t)(d.E + d.S) * d.expert_stride)) != cudaSuccess) return bail(e, "cudaMemset(weights)");
+
+    if ((e = cudaMemcpy(L->router_w, router_w, (size_t)d.E * d.H * 4, cudaMemcpyDefault)) != cudaSuccess) return bail(e, "copy router");
+    if (router_bias) {
+        if ((e = cudaMemcpy(L->router_b, router_bias, (size_t)d.E * 4, cudaMemcpyDefault)) != cudaSuccess) return bail(e, "copy bias");
+    } else if ((e = cudaMemset(L->router_b, 0, (size_t)d.E * 4)) != cudaSuccess) {
+        return bail(e, "clear bias");
+    }
+    if (expert_q) {
+        st = coli_moe_layer_set_experts(L, 0, d.E, expert_q, expert_scales);
+        if (st != COLI_OK) { free_layer(L); return st; }
+    }
+    if (shared_q) {
+        st = coli_moe_layer_set_experts(L, d.E, d.S, shared_q, shared_scales);
+        if (st != COLI_OK) { free_layer(L); return st; }
+    }
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(e, "create");
+    *out = L;
+    return COLI_OK;
+}
+
+COLI_API void coli_moe_layer_destroy(coli_moe_layer* L) {
+    if (!L) return;
+    DeviceGuard guard(L->device);
+    cudaDeviceSynchronize();
+    free_layer(L);
+}
+
+COLI_API coli_status coli_moe_layer_config(const coli_moe_layer* L, coli_moe_config* cfg) {
+    if (!L || !cfg) return fail(COLI_EINVAL, "NULL argument");
+    *cfg = L->cfg;
+    return COLI_OK;
+}
+
+static coli_status check_call(const coli_moe_layer* L, const void* x, coli_dtype dt, int T) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (dt != COLI_F32 && dt != COLI_BF16) return fail(COLI_EINVAL, "dtype must be COLI_F32 or COLI_BF16");
+    if (T < 0 || T > L->cfg.max_tokens) return fail(COLI_EINVAL, "n_tokens out of [0, max_tokens]");
+    if (T > 0 && !x) return fail(COLI_EINVAL, "x is NULL");
+    if (((uintptr_t)x) & 15u) return fail(COLI_EINVAL, "x must be 16-byte aligned");
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_route(coli_moe_layer* L, const void* x, coli_dtype dt, int T, int32_t* ids,
+                                    float* weights, coli_stream stream) {
+    coli_status st = check_call(L, x, dt, T);
+    if (st != COLI_OK) return st;
+    if (T > 0 && (!ids || !weights)) return fail(COLI_EINVAL, "ids/weights is NULL");
+    if (T == 0) return COLI_OK;
+    DeviceGuard guard(L->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    const Dims& d = L->d;
+    CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s), "router");
+    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, ids, weights, s), "topk");
+    return COLI_OK;
+}
+
+// x: layer input; residual: added to the output (stack) or NULL; y: output.
+static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_dtype dt, int T, const float* residual,
+                                cudaStream_t s) {
+    const Dims& d = L->d;
+    const Plan& p = L->plan;
+    if (L->profiling && L->prof_issued - L->prof_folded >= coli_moe_layer::kRing)
+        CUDA_TRY(prof_fold(L, L->prof_next), "profile");  // recycle the oldest slot
+    prof_mark(L, COLI_STAGE_ROUTER, s);
+    CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s), "router");
+    prof_mark(L, COLI_STAGE_TOPK, s);
+    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+    prof_mark(L, COLI_STAGE_PLAN, s);
+    CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
+    prof_mark(L, COLI_STAGE_GATEUP, s);
+    CUDA_TRY(launch_gateup_core(L->weights, d, x, dt, T, p, L->h, L->max_active, L->n_sm, s), "gate/up");
+    prof_mark(L, COLI_STAGE_DOWN, s);
+    CUDA_TRY(launch_down_core(L->weights, d, L->h, T, p, L->o, L->max_active, L->n_sm, s), "down");
+    prof_mark(L, COLI_STAGE_COMBINE, s);
+    CUDA_TRY(launch_combine(L->o, p, T, d.H, d.K, d.S, residual, y, dt, s), "combine");
+    prof_mark(L, COLI_N_STAGES, s);
+    if (L->profiling) {
+        L->prof_issued += 1;
+        L->prof_next = (L->prof_next + 1) % coli_moe_layer::kRing;
+    }
+    L->last_T = T;
+    L->last_stream = s;
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_forward(coli_moe_layer* L, const void* x, void* y, coli_dtype dt, int T,
+                                      coli_stream stream) {
+    coli_status st = check_call(L, x, dt, T);
+    if (st != COLI_OK) return st;
+    if (T > 0 && !y) return fail(COLI_EINVAL, "y is NULL");
+    if (((uintptr_t)y) & 15u) return fail(COLI_EINVAL, "y must be 16-byte aligned");
+    if (T > 0) {
+        const size_t bytes = (size_t)T * L->d.H * (dt == COLI_F32 ? 4 : 2);
+        const uint8_t *xb = (const uint8_t*)x, *yb = (const uint8_t*)y;
+        if (xb < yb + bytes && yb < xb + bytes) return fail(COLI_EINVAL, "x and y overlap");
+    }
+    if (T == 0) return COLI_OK;
+    DeviceGuard guard(L->device);
+    return forward_impl(L, x, y, dt, T, nullptr, (cudaStream_t)stream);
+}
+
+COLI_API coli_status coli_moe_stack_forward(coli_moe_layer* const* layers, int n_layers, float* x, int T, float eps,
+                                            coli_stream stream) {
+    if (!layers || n_layers < 0) return fail(COLI_EINVAL, "bad layer list");
+    if (n_layers == 0 || T == 0) return COLI_OK;
+    if (!(eps >= 0.0f)) return fail(COLI_EINVAL, "eps must be >= 0");
+    const coli_moe_layer* L0 = layers[0];
+    for (int l = 0; l < n_layers; ++l) {
+        coli_status st = check_call(layers[l], x, COLI_F32, T);
+        if (st != COLI_OK) return st;
+        if (layers[l]->d.H != L0->d.H || layers[l]->device != L0->device)
+            return fail(COLI_EINVAL, "layers must share hidden size and device");
+    }
+    DeviceGuard guard(L0->device);
+    cudaStream_t s = (cudaStream_t)stream;
+    for (int l = 0; l < n_layers; ++l) {
+        coli_moe_layer* L = layers[l];
+        CUDA_TRY(launch_rmsnorm(x, T, L->d.H, eps, L->xn, s), "rmsnorm");
+        coli_status st = forward_impl(L, L->xn, x, COLI_F32, T, x, s);
+        if (st != COLI_OK) return st;
+    }
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_get_stats(coli_moe_layer* L, int* n_unique, int64_t* bytes_streamed,
+                                        int32_t* per_expert_counts) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (L->last_T < 0) return fail(COLI_EINVAL, "no forward has run on this layer");
+    DeviceGuard guard(L->device);
+    CUDA_TRY(cudaStreamSynchronize(L->last_stream), "sync");
+    int nu = 0;
+    CUDA_TRY(cudaMemcpy(&nu, L->plan.n_unique, 4, cudaMemcpyDeviceToHost), "read n_unique");
+    if (n_unique) *n_unique = nu;
+    if (bytes_streamed)
+        *bytes_streamed = (int64_t)(nu + L->d.S) * coli_moe_expert_bytes(L->d.H, L->d.I) + (int64_t)L->d.E * L->d.H * 4;
+    if (per_expert_counts)
+        CUDA_TRY(cudaMemcpy(per_expert_counts, L->plan.cnt, (size_t)L->d.E * 4, cudaMemcpyDeviceToHost), "read counts");
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_get_plan(coli_moe_layer* L, int32_t* ids, float* weights, int32_t* counts, int32_t* offsets,
+                                       int32_t* unique, int32_t* n_unique, int32_t* pos, int32_t* tok) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (L->last_T < 0) return fail(COLI_EINVAL, "no forward has run on this layer");
+    DeviceGuard guard(L->device);
+    CUDA_TRY(cudaStreamSynchronize(L->last_stream), "sync");
+    const size_t TK = (size_t)L->last_T * L->d.K;
+    const Plan& p = L->plan;
+    int nu = 0;
+    CUDA_TRY(cudaMemcpy(&nu, p.n_unique, 4, cudaMemcpyDeviceToHost), "read n_unique");
+    if (n_unique) *n_unique = nu;
+    if (ids && TK) CUDA_TRY(cudaMemcpy(ids, p.ids, TK * 4, cudaMemcpyDeviceToHost), "read ids");
+    if (weights && TK) CUDA_TRY(cudaMemcpy(weights, p.w, TK * 4, cudaMemcpyDeviceToHost), "read weights");
+    if (counts) CUDA_TRY(cudaMemcpy(counts, p.cnt, (size_t)L->d.E * 4, cudaMemcpyDeviceToHost), "read counts");
+    if (offsets) CUDA_TRY(cudaMemcpy(offsets, p.off, (size_t)(L->d.E + 1) * 4, cudaMemcpyDeviceToHost), "read offsets");
+    if (unique && nu) CUDA_TRY(cudaMemcpy(unique, p.unique, (size_t)nu * 4, cudaMemcpyDeviceToHost), "read unique");
+    if (pos && TK) CUDA_TRY(cudaMemcpy(pos, p.pos, TK * 4, cudaMemcpyDeviceToHost), "read pos");
+    if (tok && TK) CUDA_TRY(cudaMemcpy(tok, p.tok, TK * 4, cudaMemcpyDeviceToHost), "read tok");
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_set_profiling(coli_moe_layer* L, int enable) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    DeviceGuard guard(L->device);
+    if (enable && !L->ev[0][0]) {
+        for (auto& set : L->ev)
+            for (auto& e : set) CUDA_TRY(cudaEventCreate(&e), "cudaEventCreate");
+    }
+    if (L->ev[0][0]) CUDA_TRY(cudaDeviceSynchronize(), "sync");
+    L->profiling = enable != 0;
+    L->prof_next = 0;
+    L->prof_issued = L->prof_folded = 0;
+    for (double& t : L->prof_total) t = 0.0;
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_get_profile(coli_moe_layer* L, double* stage_ms_total, int64_t* n_forwards) {
+    if (!L || !stage_ms_total) return fail(COLI_EINVAL, "NULL argument");
+    DeviceGuard guard(L->device);
+    const int K = coli_moe_layer::kRing;
+    while (L->prof_folded < L->prof_issued) {
+        const int64_t pending = L->prof_issued - L->prof_folded;   // <= K
+        const int r = (int)(((L->prof_next - pending) % K + K) % K);  // oldest pending slot
+        CUDA_TRY(prof_fold(L, r), "profile");
+    }
+    for (int i = 0; i < COLI_N_STAGES; ++i) stage_ms_total[i] = L->prof_total[i];
+    if (n_forwards) *n_forwards = L->prof_folded;
+    return COLI_OK;
+}
+
+COLI_API const char* coli_moe_stage_name(int stage) {
+    static const char* names[COLI_N_STAGES] = {"router", "topk", "plan", "gateup", "down", "combine"};
+    return (stage >= 0 && stage < COLI_N_STAGES) ? names[stage] : "";
+}
+
+COLI_API const char* coli_status_string(coli_status s) {
+    switch (s) {
+        case COLI_OK: return "ok";
+        case COLI_EINVAL: return "invalid argument";
+        case COLI_ENOMEM: return "out of memory";
+        case COLI_ECUDA: return "CUDA error";
+        case COLI_EUNSUPPORTED: return "unsupported";
+    }
+    return "unknown status";
+}
+
+COLI_API const char* coli_last_error(void) { return g_last_error.c_str(); }

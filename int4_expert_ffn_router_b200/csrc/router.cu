@@ -1,0 +1,289 @@
+// router.cu -- router GEMV (fp64 accumulation), top-k selection with
+// softmax renormalisation, and the batch-union planner.
+//
+// Router: "Colibri: 2400 lines of pure C ..." (kechuai.cn), section 一: each
+// layer routes a token to 8 of its 256 experts. Batch-union: same page,
+// section 二: the positions of a batch read each unique expert once.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace coli {
+
+// ---------------------------------------------------------------------------
+// Router logits: l[t][e] = sum_h Wr[e][h] x[t][h] + b[e], accumulated in fp64.
+// Products of two fp32 (or bf16 x fp32) values are exact in fp64, so the
+// logits agree with an fp64 reference up to summation order (~1e-16
+// relative): the top-k ids are then reproducible bit for bit.
+//
+// Grid (ceil(E/2), ceil(T/kRouterTok)); 256 threads: warp w handles expert
+// 2*blockIdx.x + w/4 and quarter (w%4) of H for up to kRouterTok tokens; the
+// four quarters are summed in a fixed order through shared memory.
+// ---------------------------------------------------------------------------
+constexpr int kRouterTok = 4;
+
+template <typename XT>
+__device__ __forceinline__ void load4(const XT* p, double v[4]);
+
+template <>
+__device__ __forceinline__ void load4<float>(const float* p, double v[4]) {
+    float4 f = *reinterpret_cast<const float4*>(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+}
+
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, double v[4]) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    v[0] = __uint_as_float(u.x << 16);
+    v[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(u.y << 16);
+    v[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(256) router_logits_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
+                                                            const XT* __restrict__ x, int T, int H, int E,
+                                                            double* __restrict__ logits) {
+    __shared__ double part[8][kRouterTok];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 2 + (warp >> 2);
+    const int quarter = warp & 3;
+    const int t0 = blockIdx.y * kRouterTok;
+    const int nt = min(kRouterTok, T - t0);
+    const int seg = H / 4;
+    double acc[kRouterTok];
+#pragma unroll
+    for (int j = 0; j < kRouterTok; ++j) acc[j] = 0.0;
+    if (e < E) {
+        const float* wrow = wr + (size_t)e * H + quarter * seg;
+        for (int i = lane * 4; i < seg; i += 128) {
+            float4 w4 = *reinterpret_cast<const float4*>(wrow + i);
+            double wd[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int j = 0; j < kRouterTok; ++j) {
+                if (j < nt) {
+                    double xv[4];
+                    load4<XT>(x + (size_t)(t0 + j) * H + quarter * seg + i, xv);
+                    acc[j] = fma(wd[0], xv[0], acc[j]);
+                    acc[j] = fma(wd[1], xv[1], acc[j]);
+                    acc[j] = fma(wd[2], xv[2], acc[j]);
+                    acc[j] = fma(wd[3], xv[3], acc[j]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kRouterTok; ++j) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < kRouterTok; ++j) part[warp][j] = acc[j];
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * kRouterTok) {
+        int ew = threadIdx.x / kRouterTok, j = threadIdx.x % kRouterTok;
+        int ee = blockIdx.x * 2 + ew;
+        if (ee < E && j < nt) {
+            double s = ((part[ew * 4 + 0][j] + part[ew * 4 + 1][j]) + part[ew * 4 + 2][j]) + part[ew * 4 + 3][j];
+            logits[(size_t)(t0 + j) * E + ee] = s + (bias ? (double)bias[ee] : 0.0);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Top-k: one warp per token. Lane l holds the logits of experts l, l+32, ...
+// K rounds each take the best remaining (largest logit, ties to the lower
+// id). Weights: softmax over the K selected logits, in fp64, summed in a
+// fixed order.
+// ---------------------------------------------------------------------------
+constexpr int kMaxPerLane = 32;  // E <= 1024
+
+__device__ __forceinline__ bool better(double a, int ia, double b, int ib) {
+    return a > b || (a == b && ia < ib);
+}
+
+__global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ logits, int T, int E, int K,
+                                                   int32_t* __restrict__ ids, float* __restrict__ w) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= T) return;
+    const double* l = logits + (size_t)t * E;
+    const int per = (E + 31) / 32;
+    double v[kMaxPerLane];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+        int e = lane + 32 * i;
+        v[i] = (i < per && e < E) ? l[e] : -INFINITY;
+    }
+    double my_sel = 0.0;
+    int my_id = -1;
+    double top = 0.0;
+    for (int k = 0; k < K; ++k) {
+        double bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < kMaxPerLane; ++i) {
+            int e = lane + 32 * i;
+            if (i < per && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) { bv = v[i]; bi = e; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        if (k == 0) top = bv;
+        if (lane == k) { my_sel = bv; my_id = bi; }
+    }
+    // softmax over the selected logits; lane k < K owns slot k
+    double ex = (lane < K) ? exp(my_sel - top) : 0.0;
+    double z = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane < K) {
+        ids[(size_t)t * K + lane] = my_id;
+        w[(size_t)t * K + lane] = (float)(ex / z);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Batch-union planner, one CTA of 1024 threads. For the T*K routed slots:
+//   cnt[e], off = exclusive scan, unique = {e : cnt[e] > 0} ascending,
+//   pos[t][k] = off[e] + (rank of t among e's tokens, ascending t),
+//   tok[pos] = t,
+// then the active-expert list (unique experts, then the S shared experts,
+// each shared expert taking all T tokens at positions T*K + j*T + t).
+// Deterministic: positions come from per-warp counts over token chunks and a
+// sequential walk inside each chunk, never from atomics.
+// ---------------------------------------------------------------------------
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanWarps = kPlanThreads / 32;
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ ids, int T, int K, int E, int S,
+                                                            Plan p) {
+    extern __shared__ int32_t sm[];
+    int32_t* wcnt = sm;                          // [kPlanWarps][E]  -> per-warp cursor
+    int32_t* off = wcnt + kPlanWarps * E;        // [E+1]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunk = (T + kPlanWarps - 1) / kPlanWarps;
+    const int tb = warp * chunk, te = min(T, tb + chunk);
+
+    for (int i = threadIdx.x; i < kPlanWarps * E; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    // per-warp counts over its token chunk (distinct ids within a token: lane k owns slot k)
+    for (int t = tb; t < te; ++t) {
+        if (lane < K) {
+            int e = ids[(size_t)t * K + lane];
+            wcnt[warp * E + e] += 1;
+        }
+        __syncwarp();
+    }
+    __syncthreads();
+    // per expert: exclusive scan over warps -> warp cursor base, total count
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int w = 0; w < kPlanWarps; ++w) {
+            int c = wcnt[w * E + e];
+            wcnt[w * E + e] = run;
+            run += c;
+        }
+        off[e + 1] = run;  // count for now
+    }
+    __syncthreads();
+    // exclusive scan of counts over experts (E <= 1024: one thread each, Hillis-Steele)
+    if (threadIdx.x == 0) off[0] = 0;
+    int cnt_e = 0;
+    if (threadIdx.x < E) cnt_e = off[threadIdx.x + 1];
+    __syncthreads();
+    // inclusive scan in place over off[1..E]
+    for (int d = 1; d < E; d <<= 1) {
+        int add = 0;
+        if (threadIdx.x < E && threadIdx.x >= d) add = off[threadIdx.x + 1 - d];
+        __syncthreads();
+        if (threadIdx.x < E) off[threadIdx.x + 1] += add;
+        __syncthreads();
+    }
+    if (threadIdx.x < E) {
+        p.cnt[threadIdx.x] = cnt_e;
+        p.off[threadIdx.x] = off[threadIdx.x];
+    }
+    if (threadIdx.x == 0) p.off[E] = off[E];
+    // unique list: rank among experts with cnt > 0
+    __shared__ int32_t flag_scan[1024];
+    if (threadIdx.x < 1024) flag_scan[threadIdx.x] = (threadIdx.x < E && cnt_e > 0) ? 1 : 0;
+    __syncthreads();
+    for (int d = 1; d < 1024; d <<= 1) {
+        int add = (threadIdx.x >= d) ? flag_scan[threadIdx.x - d] : 0;
+        __syncthreads();
+        flag_scan[threadIdx.x] += add;
+        __syncthreads();
+    }
+    const int n_unique = flag_scan[1023];
+    if (threadIdx.x < E && cnt_e > 0) {
+        int r = flag_scan[threadIdx.x] - 1;
+        p.unique[r] = threadIdx.x;
+        p.act_expert[r] = threadIdx.x;
+        p.act_off[r] = off[threadIdx.x];
+        p.act_cnt[r] = cnt_e;
+    }
+    if (threadIdx.x < S) {
+        int r = n_unique + threadIdx.x;
+        p.act_expert[r] = E + threadIdx.x;
+        p.act_off[r] = T * K + threadIdx.x * T;
+        p.act_cnt[r] = T;
+    }
+    if (threadIdx.x == 0) {
+        *p.n_unique = n_unique;
+        *p.n_active = n_unique + S;
+    }
+    // positions: each warp walks its chunk in token order
+    for (int t = tb; t < te; ++t) {
+        if (lane < K) {
+            int e = ids[(size_t)t * K + lane];
+            int q = off[e] + wcnt[warp * E + e];
+            wcnt[warp * E + e] += 1;
+            p.pos[(size_t)t * K + lane] = q;
+            p.tok[q] = t;
+        }
+        __syncwarp();
+    }
+    // shared experts: all tokens in order
+    for (int i = threadIdx.x; i < S * T; i += blockDim.x) p.tok[T * K + i] = i % T;
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers.
+// ---------------------------------------------------------------------------
+cudaError_t launch_router_logits(const float* wr, const float* bias, const void* x, coli_dtype dt, int T, int H, int E,
+                                 double* logits, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    dim3 grid((E + 1) / 2, (T + kRouterTok - 1) / kRouterTok);
+    if (dt == COLI_F32)
+        router_logits_kernel<float><<<grid, 256, 0, st>>>(wr, bias, (const float*)x, T, H, E, logits);
+    else
+        router_logits_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(wr, bias, (const __nv_bfloat16*)x, T, H, E, logits);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const double* logits, int T, int E, int K, int32_t* ids, float* w, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, K, ids, w);
+    return cudaGetLastError();
+}
+
+size_t plan_smem_bytes(int E) { return sizeof(int32_t) * ((size_t)kPlanWarps * E + E + 1); }
+
+cudaError_t launch_plan(const int32_t* ids, int T, int K, int E, int S, const Plan& p, cudaStream_t st) {
+    const size_t smem = plan_smem_bytes(E);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    plan_kernel<<<1, kPlanThreads, smem, st>>>(ids, T, K, E, S, p);
+    return cudaGetLastError();
+}
+
+}  // namespace coli

@@ -153,3 +153,25 @@ def zipf_bias(seed: int, layer: int, E: int, kappa: float | None = None, s_exp: 
     r = np.empty(E, np.int32)
     host_lib().synth_zipf_bias(seed, layer, E, ZIPF_KAPPA if kappa is None else kappa, s_exp, _ptr(b), _ptr(r))
     return b, r
+
+
+# ----------------------------------------------------------------- device twin
+def expert_dev(seed: int, layer: int, e0: int, n: int, H: int, I: int, q_ptr: int, s_ptr: int, stream=None,
+               wscale: float = WSCALE) -> None:
+    """Write experts e0..e0+n-1 (canonical) into device buffers."""
+    rc = dev_lib().synth_expert_dev(seed, layer, e0, n, H, I, wscale, q_ptr, s_ptr, stream)
+    if rc:
+        raise RuntimeError(f"synth_expert_dev failed: cudaError {rc}")
+
+
+def router_dev(seed: int, layer: int, E: int, H: int, ptr: int, stream=None, wscale: float = WSCALE) -> None:
+    rc = dev_lib().synth_router_dev(seed, layer, E, H, wscale, ptr, stream)
+    if rc:
+        raise RuntimeError(f"synth_router_dev failed: cudaError {rc}")
+
+
+def x_dev(seed: int, step: int, T: int, H: int, dtype: int, ptr: int, stream=None) -> None:
+    """dtype 0: fp32, 1: bf16 bits."""
+    rc = dev_lib().synth_x_dev(seed, step, T, H, dtype, ptr, stream)
+    if rc:
+        raise RuntimeError(f"synth_x_dev failed: cudaError {rc}")
