@@ -159,10 +159,24 @@ coli_status coli_moe_get_plan(coli_moe_layer* layer, int32_t* ids, float* weight
  * resets the totals.
  */
 enum { COLI_STAGE_ROUTER = 0, COLI_STAGE_TOPK, COLI_STAGE_PLAN, COLI_STAGE_GATEUP, COLI_STAGE_DOWN,
-       COLI_STAGE_COMBINE, COLI_N_STAGES };
+       COLI_STAGE_COMBINE, COLI_STAGE_FUSED, COLI_N_STAGES };
 coli_status coli_moe_set_profiling(coli_moe_layer* layer, int enable);
 coli_status coli_moe_get_profile(coli_moe_layer* layer, double* stage_ms_total, int64_t* n_forwards);
 const char* coli_moe_stage_name(int stage);
+
+/*
+ * Waits for the layer's last forward. Returns COLI_ECUDA if the persistent
+ * decode kernel gave up on a bounded wait (its inputs are then invalid); the
+ * layer is reset and stays usable. get_stats and get_plan do the same check.
+ */
+coli_status coli_moe_sync(coli_moe_layer* layer);
+
+/*
+ * Selects the path for n_tokens <= 4: 1 (default) runs the whole layer in one
+ * persistent kernel (router, top-k, plan, experts, combine), 0 runs the
+ * separate kernels. Results agree within rounding; routing is identical.
+ */
+coli_status coli_moe_set_fused(coli_moe_layer* layer, int enable);
 
 /* Bytes of one expert in the int4 gs64 container (nibbles + fp16 scales). */
 int64_t coli_moe_expert_bytes(int hidden, int inter);

@@ -22,9 +22,9 @@ EXPORTS = (
     "coli_moe_layer_create", "coli_moe_layer_set_experts", "coli_moe_layer_destroy", "coli_moe_layer_config",
     "coli_moe_route", "coli_moe_forward", "coli_moe_stack_forward", "coli_moe_get_stats", "coli_moe_get_plan",
     "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
-    "coli_moe_get_profile", "coli_moe_stage_name",
+    "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused",
 )
-N_STAGES = 6
+N_STAGES = 7
 
 
 class Config(ctypes.Structure):
@@ -62,6 +62,8 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_get_profile.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_int64)]
     L.coli_moe_stage_name.argtypes = [i32]
     L.coli_moe_stage_name.restype = ctypes.c_char_p
+    L.coli_moe_sync.argtypes = [vp]
+    L.coli_moe_set_fused.argtypes = [vp, i32]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
     L.coli_last_error.argtypes = []
@@ -163,6 +165,13 @@ class Layer:
         _check(lib.coli_moe_get_stats(self.handle, ctypes.byref(nu), ctypes.byref(b), _ptr(counts)),
                "coli_moe_get_stats")
         return nu.value, b.value
+
+    def sync(self) -> None:
+        """Wait for the last forward; raises if the device reported a timeout."""
+        _check(lib.coli_moe_sync(self.handle), "coli_moe_sync")
+
+    def set_fused(self, on: bool) -> None:
+        _check(lib.coli_moe_set_fused(self.handle, 1 if on else 0), "coli_moe_set_fused")
 
     def set_profiling(self, on: bool) -> None:
         _check(lib.coli_moe_set_profiling(self.handle, 1 if on else 0), "coli_moe_set_profiling")

@@ -43,6 +43,17 @@ constexpr int kNibbleBytes = 4096;
 constexpr int kScaleBytes = 256;
 constexpr int kBlockBytes = kNibbleBytes + kScaleBytes;  // 4352
 
+// Persistent decode kernel: tokens per launch, ring stages, control block.
+constexpr int kFusedMaxTok = 4;
+constexpr int kMaxStages = 24;
+// Control block (ints in the workspace, zero between launches):
+//   [kCtlTicket] work ticket, [kCtlRouter] finished router rows,
+//   [kCtlPlan] plan published, [kCtlExit] CTAs done, [kCtlError] timeout code,
+//   [kCtlGuDone + e] finished gate/up tiles of expert e (E + S entries),
+//   then [kCtlGuDone + E + S + rt] finished down tiles of output block rt.
+enum { kCtlTicket = 0, kCtlRouter = 1, kCtlPlan = 2, kCtlExit = 3, kCtlError = 4, kCtlGuDone = 8 };
+inline int ctl_ints(int E, int S, int H) { return kCtlGuDone + E + S + H / 128; }
+
 inline int64_t matrix_bytes(int rows, int cols) {
     return (int64_t)(rows / kTileRows) * (cols / kGroup) * kBlockBytes;
 }
@@ -94,5 +105,73 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+}  // namespace coli
+
+namespace coli {
+
+// ---------------------------------------------------------------------------
+// mbarrier / bulk-copy / ordering helpers (sm_90+ PTX, used on sm_100a).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bulk copy global -> this CTA's shared memory, completing on `bar`.
+// dst, src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(int* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void named_bar(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 }  // namespace coli

@@ -1,0 +1,549 @@
+// decode_fused.cu -- the whole MoE layer for a few tokens in one persistent
+// kernel: router, top-k, batch-union plan, fused int4 gate/up + SwiGLU,
+// down, and the weighted combine with the shared expert.
+//
+// Decode streams each active expert's ~20 MB once ("Colibri: 2400 lines of
+// pure C ...", kechuai.cn, section 二: one read per unique expert per batch,
+// the three matrices adjacent), so the kernel is HBM-bound: it must keep
+// enough bytes in flight and never leave the memory system idle between the
+// dependent steps. Design:
+//  * one CTA per SM; a producer warp streams weight tiles into a shared-memory
+//    ring with bulk asynchronous copies (the TMA engine) completing on
+//    mbarriers; 16 consumer warps dequantise and multiply out of the ring;
+//  * work items are handed out by a global ticket counter in dependency
+//    order: router rows, the plan, shared-expert gate/up, shared-expert down,
+//    routed gate/up, routed down. An item only waits for items with smaller
+//    tickets, which running CTAs already hold, so the schedule cannot
+//    deadlock; every wait is bounded in time and reports a timeout through
+//    the control block instead of hanging;
+//  * the producer prefetches an item's weights before its inputs are ready
+//    (routed experts only need the plan, down tiles only the gate/up of the
+//    same expert), so weight streaming overlaps the top-k, the plan and the
+//    gate/up -> down dependency;
+//  * the last down tile of each 128-row output block to finish combines
+//    that block of y in a fixed order (shared experts, then the routed ones
+//    in routing order), so no extra pass and no atomics on y.
+#include "common.cuh"
+#include "int4_math.cuh"
+#include "kernels.cuh"
+#include "topk.cuh"
+
+namespace coli {
+
+constexpr int kCW = 16;                      // consumer warps
+constexpr int kCT = kCW * 32;                // consumer threads
+constexpr int kFT = kCT + 32;                // + the producer warp
+constexpr int kSB = 2;                       // 4352-byte blocks per ring stage
+constexpr int kStage = kSB * kBlockBytes;    // 8704 bytes
+constexpr int kQ = 2;                        // item queue slots (lookahead of one item)
+constexpr uint64_t kWaitNs = 1000000000ull;  // every wait gives up after 1 s
+
+enum { IT_END = 0, IT_ROUTER = 1, IT_PLAN = 2, IT_GU = 3, IT_DOWN = 4 };
+
+struct Item {
+    int kind, ex, rt, off, cnt, shared;
+};
+
+struct FusedArgs {
+    const uint8_t* weights;
+    Dims d;
+    const float* wr;
+    const float* bias;
+    const void* x;
+    void* y;
+    const float* residual;
+    int T;
+    Plan p;
+    double* logits;
+    float* h;
+    float* o;
+    int* ctl;
+    int umax;     // min(T*K, E): upper bound of distinct routed experts
+    int nstages;  // ring stages
+};
+
+// Shared-memory layout (dynamic).
+struct FusedSmem {
+    uint64_t full[kMaxStages], empty[kMaxStages], qfull[kQ], qempty[kQ];
+    Item items[kQ];
+    int abort_flag;
+    Item cur[2];
+    int staged_n, staged_rows[kFusedMaxTok];
+    int srow[kFusedMaxTok];
+    int sflag;
+    double rpart[kCW][kFusedMaxTok];
+    int sids[kFusedMaxTok * 32];
+    float red[8 * 8 * 2 * kFusedMaxTok];
+};
+
+__device__ __forceinline__ void set_error(FusedArgs& a, volatile int* abort_flag, int code) {
+    *abort_flag = 1;
+    atomicCAS(&a.ctl[kCtlError], 0, code);
+}
+
+// Bounded wait on an mbarrier phase; gives up when the CTA aborts or after kWaitNs.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, FusedArgs& a,
+                                         int code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitNs) {
+            set_error(a, abort_flag, code);
+            return false;
+        }
+    }
+}
+
+// Bounded wait until *p >= target (acquire).
+__device__ __forceinline__ bool wait_geq(const int* p, int target, volatile int* abort_flag, FusedArgs& a, int code) {
+    if (ld_acquire(p) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (ld_acquire(p) >= target) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitNs) {
+            set_error(a, abort_flag, code);
+            return false;
+        }
+        __nanosleep(64);
+    }
+}
+
+// ------------------------------------------------------------------ producer
+__device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
+    const Dims& d = a.d;
+    const int T = a.T;
+    const int RTgu = 2 * d.I / kTileRows, RTd = d.H / kTileRows;
+    const int Ggu = d.H / kGroup, Gd = d.I / kGroup;
+    const int t_plan = d.E, t_sg = t_plan + 1, t_sd = t_sg + d.S * RTgu, t_ug = t_sd + d.S * RTd;
+    const int t_ud = t_ug + a.umax * RTgu, t_end = t_ud + a.umax * RTd;
+    volatile int* abort_flag = &S.abort_flag;
+    int n_unique = -1;
+    uint32_t q = 0, gs = 0;
+    while (true) {
+        Item it{IT_END, 0, 0, 0, 0, 0};
+        if (!*abort_flag) {
+            const int t = atomicAdd(&a.ctl[kCtlTicket], 1);
+            if (t < t_plan) {
+                it = Item{IT_ROUTER, t, 0, 0, 0, 0};
+            } else if (t == t_plan) {
+                it = Item{IT_PLAN, 0, 0, 0, 0, 0};
+            } else if (t < t_sd) {
+                const int j = (t - t_sg) / RTgu, rt = (t - t_sg) % RTgu;
+                it = Item{IT_GU, d.E + j, rt, T * d.K + j * T, T, 1};
+            } else if (t < t_ug) {
+                const int j = (t - t_sd) / RTd, rt = (t - t_sd) % RTd;
+                it = Item{IT_DOWN, d.E + j, rt, T * d.K + j * T, T, 1};
+            } else if (t < t_end) {
+                if (n_unique < 0) {
+                    if (!wait_geq(&a.ctl[kCtlPlan], 1, abort_flag, a, 2)) continue;
+                    n_unique = __ldcg(a.p.n_unique);
+                }
+                const bool gu = t < t_ud;
+                const int r = gu ? t - t_ug : t - t_ud;
+                const int RT = gu ? RTgu : RTd;
+                const int u = r / RT, rt = r % RT;
+                if (u >= n_unique) continue;  // fewer distinct experts than the bound
+                const int ex = __ldcg(a.p.unique + u);
+                it = Item{gu ? IT_GU : IT_DOWN, ex, rt, __ldcg(a.p.off + ex), __ldcg(a.p.cnt + ex), 0};
+            }
+        }
+        const uint32_t slot = q % kQ;
+        if (q >= kQ && !wait_bar(&S.qempty[slot], ((q / kQ) - 1) & 1, abort_flag, a, 3)) it.kind = IT_END;
+        S.items[slot] = it;
+        mbar_arrive(&S.qfull[slot]);
+        ++q;
+        if (it.kind == IT_END) break;
+        if (it.kind == IT_GU || it.kind == IT_DOWN) {
+            const bool gu = it.kind == IT_GU;
+            const int G = gu ? Ggu : Gd;
+            const uint8_t* tile = a.weights + (size_t)it.ex * d.expert_stride + (gu ? 0 : d.gu_bytes) +
+                                  (size_t)it.rt * G * kBlockBytes;
+            for (int b0 = 0; b0 < G; b0 += kSB) {
+                const int nb = min(kSB, G - b0);
+                const uint32_t s = gs % a.nstages;
+                if (gs >= (uint32_t)a.nstages &&
+                    !wait_bar(&S.empty[s], ((gs / a.nstages) - 1) & 1, abort_flag, a, 4)) {
+                    break;
+                }
+                mbar_arrive_expect_tx(&S.full[s], nb * kBlockBytes);
+                bulk_g2s(ring + (size_t)s * kStage, tile + (size_t)b0 * kBlockBytes, nb * kBlockBytes, &S.full[s]);
+                ++gs;
+            }
+        }
+    }
+    // let the copies in flight land before the CTA exits (bounded)
+    const uint32_t ns = a.nstages;
+    for (uint32_t k = (gs > ns ? gs - ns : 0); k < gs; ++k) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&S.full[k % ns], (k / ns) & 1) && globaltimer_ns() - t0 < kWaitNs) {
+        }
+    }
+}
+
+// ------------------------------------------------------------------ consumers
+template <typename XT, int NT>
+__device__ void router_item(FusedArgs& a, FusedSmem& S, int e, int ctid) {
+    const Dims& d = a.d;
+    const int cw = ctid >> 5, lane = ctid & 31;
+    const int chunk = d.H / kCW;
+    const float* wrow = a.wr + (size_t)e * d.H + cw * chunk;
+    const XT* x = reinterpret_cast<const XT*>(a.x);
+    double acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.0;
+    for (int i = lane * 4; i < chunk; i += 128) {
+        const float4 w4 = __ldg(reinterpret_cast<const float4*>(wrow + i));
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            if (t < a.T) {
+                const XT* xp = x + (size_t)t * d.H + cw * chunk + i;
+                double x0, x1, x2, x3;
+                if constexpr (sizeof(XT) == 4) {
+                    const float4 v = __ldg(reinterpret_cast<const float4*>(xp));
+                    x0 = v.x; x1 = v.y; x2 = v.z; x3 = v.w;
+                } else {
+                    const uint2 u = __ldg(reinterpret_cast<const uint2*>(xp));
+                    x0 = __uint_as_float(u.x << 16); x1 = __uint_as_float(u.x & 0xFFFF0000u);
+                    x2 = __uint_as_float(u.y << 16); x3 = __uint_as_float(u.y & 0xFFFF0000u);
+                }
+                acc[t] = fma((double)w4.x, x0, acc[t]);
+                acc[t] = fma((double)w4.y, x1, acc[t]);
+                acc[t] = fma((double)w4.z, x2, acc[t]);
+                acc[t] = fma((double)w4.w, x3, acc[t]);
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+        if (lane == 0) S.rpart[cw][t] = acc[t];
+    }
+    named_bar(1, kCT);
+    if (ctid < a.T) {
+        double s = 0.0;
+        for (int w = 0; w < kCW; ++w) s += S.rpart[w][ctid];
+        a.logits[(size_t)ctid * d.E + e] = s + (double)a.bias[e];
+    }
+    named_bar(1, kCT);
+    if (ctid == 0) {
+        __threadfence();
+        atomicAdd(&a.ctl[kCtlRouter], 1);
+    }
+}
+
+// Top-k of every token (warp t) and the batch-union plan (warp 0).
+__device__ void plan_item(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* soff) {
+    const Dims& d = a.d;
+    const int T = a.T, E = d.E, K = d.K;
+    const int cw = ctid >> 5, lane = ctid & 31;
+    volatile int* abort_flag = &S.abort_flag;
+    // Control flow below never depends on the abort flag around a barrier:
+    // on abort the work is skipped but every thread meets every barrier.
+    if (ctid == 0) wait_geq(&a.ctl[kCtlRouter], E, abort_flag, a, 5);
+    named_bar(1, kCT);
+    if (cw < T && !*abort_flag) {
+        int id;
+        float wt;
+        warp_topk<true>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
+        if (lane < K) {
+            a.p.ids[cw * K + lane] = id;
+            a.p.w[cw * K + lane] = wt;
+            S.sids[cw * K + lane] = id;
+        }
+    }
+    named_bar(1, kCT);
+    if (cw == 0 && !*abort_flag) {
+        for (int e = lane; e < E; e += 32) scnt[e] = 0;
+        __syncwarp();
+        for (int t = 0; t < T; ++t) {
+            if (lane < K) scnt[S.sids[t * K + lane]] += 1;  // ids of one token are distinct
+            __syncwarp();
+        }
+        const int per = (E + 31) / 32, b = lane * per, be = min(E, b + per);
+        int sum = 0, fl = 0;
+        for (int e = b; e < be; ++e) { sum += scnt[e]; fl += scnt[e] > 0; }
+        int incl = sum, fincl = fl;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n1 = __shfl_up_sync(0xffffffffu, incl, o), n2 = __shfl_up_sync(0xffffffffu, fincl, o);
+            if (lane >= o) { incl += n1; fincl += n2; }
+        }
+        const int n_unique = __shfl_sync(0xffffffffu, fincl, 31);
+        int run = incl - sum, ur = fincl - fl;
+        for (int e = b; e < be; ++e) {
+            const int c = scnt[e];
+            soff[e] = run;
+            a.p.off[e] = run;
+            a.p.cnt[e] = c;
+            if (c > 0) {
+                a.p.unique[ur] = e;
+                a.p.act_expert[ur] = e;
+                a.p.act_off[ur] = run;
+                a.p.act_cnt[ur] = c;
+                ++ur;
+            }
+            run += c;
+        }
+        if (lane == 31) a.p.off[E] = run;
+        if (lane == 0) {
+            *a.p.n_unique = n_unique;
+            *a.p.n_active = n_unique + d.S;
+        }
+        for (int j = lane; j < d.S; j += 32) {
+            a.p.act_expert[n_unique + j] = E + j;
+            a.p.act_off[n_unique + j] = T * K + j * T;
+            a.p.act_cnt[n_unique + j] = T;
+        }
+        __syncwarp();
+        for (int e = lane; e < E; e += 32) scnt[e] = 0;
+        __syncwarp();
+        for (int t = 0; t < T; ++t) {
+            if (lane < K) {
+                const int e = S.sids[t * K + lane];
+                const int q = soff[e] + scnt[e];
+                scnt[e] += 1;
+                a.p.pos[t * K + lane] = q;
+                a.p.tok[q] = t;
+            }
+            __syncwarp();
+        }
+        for (int i = lane; i < d.S * T; i += 32) a.p.tok[T * K + i] = i % T;
+    }
+    named_bar(1, kCT);
+    if (ctid == 0) {
+        __threadfence();
+        st_release(&a.ctl[kCtlPlan], 1);
+    }
+}
+
+template <typename XT, int NT>
+__device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t* ring, float4* xs, uint32_t& gs,
+                            int ctid) {
+    const Dims& d = a.d;
+    const int T = a.T;
+    const int cw = ctid >> 5, lane = ctid & 31, gi = lane >> 2, ti = lane & 3;
+    const bool gu = it.kind == IT_GU;
+    const int C = gu ? d.H : d.I;
+    const int G = C / kGroup;
+    const int nt = it.cnt;
+    volatile int* abort_flag = &S.abort_flag;
+
+    // inputs: x rows of the item's tokens (gate/up) or its h rows (down)
+    if (ctid == 0) {
+        if (!gu) wait_geq(&a.ctl[kCtlGuDone + it.ex], 2 * d.I / kTileRows, abort_flag, a, 6);
+        for (int i = 0; i < nt; ++i)
+            S.srow[i] = gu ? (it.shared ? i : __ldcg(a.p.tok + it.off + i)) : it.off + i;
+    }
+    named_bar(1, kCT);
+    bool same = gu && S.staged_n == nt;
+    for (int i = 0; same && i < nt; ++i) same = S.staged_rows[i] == S.srow[i];
+    if (!same && !*abort_flag) {
+        if (gu) stage_rows<XT, false>(xs, reinterpret_cast<const XT*>(a.x), S.srow, nt, C, ctid, kCT);
+        else stage_rows<float, true>(xs, a.h, S.srow, nt, C, ctid, kCT);
+    }
+    named_bar(1, kCT);
+    if (ctid == 0) {
+        S.staged_n = gu ? nt : -1;
+        for (int i = 0; i < nt; ++i) S.staged_rows[i] = S.srow[i];
+    }
+
+    float acc0[NT], acc1[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) { acc0[t] = 0.f; acc1[t] = 0.f; }
+    const int half = cw >> 3, sub = cw & 7;
+    const int nst = (G + kSB - 1) / kSB;
+    for (int i = 0; i < nst; ++i) {
+        const uint32_t s = gs % a.nstages;
+        const uint32_t par = (gs / a.nstages) & 1;
+        ++gs;
+        const bool ok = wait_bar(&S.full[s], par, abort_flag, a, 7);
+        const int g = i * kSB + half;
+        if (ok && g < G) {
+            const uint8_t* bp = ring + (size_t)s * kStage + half * kBlockBytes;
+            const uint4 w = *reinterpret_cast<const uint4*>(bp + sub * 512 + lane * 16);
+            const uint32_t sv = *reinterpret_cast<const uint32_t*>(bp + kNibbleBytes + sub * 32 + gi * 4);
+            group_dot<NT>(w, sv, xs + g * 16, G * 16, ti, nt, acc0, acc1);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[s]);
+    }
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+        acc0[t] += __shfl_xor_sync(0xffffffffu, acc0[t], 1);
+        acc0[t] += __shfl_xor_sync(0xffffffffu, acc0[t], 2);
+        acc1[t] += __shfl_xor_sync(0xffffffffu, acc1[t], 1);
+        acc1[t] += __shfl_xor_sync(0xffffffffu, acc1[t], 2);
+    }
+    if (half == 1 && ti == 0) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            S.red[((sub * 8 + gi) * NT + t) * 2 + 0] = acc0[t];
+            S.red[((sub * 8 + gi) * NT + t) * 2 + 1] = acc1[t];
+        }
+    }
+    named_bar(1, kCT);
+    if (half == 0 && ti == 0 && !*abort_flag) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            if (t < nt) {
+                const float v0 = acc0[t] + S.red[((sub * 8 + gi) * NT + t) * 2 + 0];
+                const float v1 = acc1[t] + S.red[((sub * 8 + gi) * NT + t) * 2 + 1];
+                if (gu) {
+                    const int j = (it.rt * 8 + sub) * 8 + gi;
+                    a.h[(size_t)(it.off + t) * d.I + j] = silu_f(v0) * v1;
+                } else {
+                    const int r0 = it.rt * kTileRows + sub * kSubRows + gi;
+                    a.o[(size_t)(it.off + t) * d.H + r0] = v0;
+                    a.o[(size_t)(it.off + t) * d.H + r0 + 8] = v1;
+                }
+            }
+        }
+    }
+    named_bar(1, kCT);
+    if (gu) {
+        if (ctid == 0) {
+            __threadfence();
+            atomicAdd(&a.ctl[kCtlGuDone + it.ex], 1);
+        }
+        return;
+    }
+    // down: the last of the active experts to finish this 128-row block combines it
+    if (ctid == 0) {
+        __threadfence();
+        int last = 0;
+        if (wait_geq(&a.ctl[kCtlPlan], 1, abort_flag, a, 8)) {
+            const int n_active = __ldcg(a.p.n_active);
+            const int prev = atomicAdd(&a.ctl[kCtlGuDone + d.E + d.S + it.rt], 1);
+            last = prev + 1 == n_active;
+            __threadfence();
+        }
+        S.sflag = last;
+    }
+    named_bar(1, kCT);
+    if (!S.sflag || *abort_flag) return;
+    const int K = d.K, TK = T * d.K;
+    for (int idx = ctid; idx < T * kTileRows; idx += kCT) {
+        const int t = idx / kTileRows, r = it.rt * kTileRows + (idx % kTileRows);
+        float acc = a.residual ? a.residual[(size_t)t * d.H + r] : 0.0f;
+        for (int j = 0; j < d.S; ++j) acc += __ldcg(a.o + (size_t)(TK + j * T + t) * d.H + r);
+        for (int k = 0; k < K; ++k) {
+            const float wk = __ldcg(a.p.w + t * K + k);
+            const int q = __ldcg(a.p.pos + t * K + k);
+            acc = fmaf(wk, __ldcg(a.o + (size_t)q * d.H + r), acc);
+        }
+        if constexpr (sizeof(XT) == 4) reinterpret_cast<float*>(a.y)[(size_t)t * d.H + r] = acc;
+        else reinterpret_cast<__nv_bfloat16*>(a.y)[(size_t)t * d.H + r] = __float2bfloat16_rn(acc);
+    }
+}
+
+template <typename XT, int NT>
+__global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    FusedSmem& S = *reinterpret_cast<FusedSmem*>(smem);
+    uint8_t* ring = smem + ((sizeof(FusedSmem) + 127) & ~(size_t)127);
+    float4* xs = reinterpret_cast<float4*>(ring + (size_t)a.nstages * kStage);
+    int* scnt = reinterpret_cast<int*>(xs + (size_t)NT * (a.d.H > a.d.I ? a.d.H : a.d.I) / 4);
+    int* soff = scnt + a.d.E + 1;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int i = 0; i < a.nstages; ++i) { mbar_init(&S.full[i], 1); mbar_init(&S.empty[i], kCW); }
+        for (int i = 0; i < kQ; ++i) { mbar_init(&S.qfull[i], 1); mbar_init(&S.qempty[i], 1); }
+        S.abort_flag = 0;
+        S.staged_n = -1;
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (warp == kCW) {
+        if (lane == 0) fused_producer(a, S, ring);
+        __syncwarp();
+    } else {
+        const int ctid = tid;
+        uint32_t q = 0, gs = 0;
+        while (true) {
+            // thread 0 takes the next item and publishes it, so every consumer
+            // thread takes the same branch below
+            const uint32_t slot = q % kQ;
+            if (ctid == 0) {
+                const bool ok = wait_bar(&S.qfull[slot], (q / kQ) & 1, &S.abort_flag, a, 9);
+                S.cur[q & 1] = S.items[slot];
+                if (!ok || S.abort_flag) S.cur[q & 1].kind = IT_END;
+            }
+            named_bar(1, kCT);
+            const Item it = S.cur[q & 1];
+            if (it.kind == IT_ROUTER) router_item<XT, NT>(a, S, it.ex, ctid);
+            else if (it.kind == IT_PLAN) plan_item(a, S, ctid, scnt, soff);
+            else if (it.kind == IT_GU || it.kind == IT_DOWN) weight_item<XT, NT>(a, S, it, ring, xs, gs, ctid);
+            named_bar(1, kCT);
+            if (ctid == 0 && it.kind != IT_END) mbar_arrive(&S.qempty[slot]);
+            ++q;
+            if (it.kind == IT_END) break;
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(&a.ctl[kCtlExit], 1) == (int)gridDim.x - 1) {
+            // last CTA out: clear the counters for the next launch (keep the error)
+            const int n = kCtlGuDone + a.d.E + a.d.S + a.d.H / kTileRows;
+            for (int i = 0; i < n; ++i)
+                if (i != kCtlError) a.ctl[i] = 0;
+            __threadfence();
+        }
+    }
+}
+
+size_t fused_smem_bytes(const Dims& d, int NT, int nstages) {
+    const size_t head = (sizeof(FusedSmem) + 127) & ~(size_t)127;
+    const int C = d.H > d.I ? d.H : d.I;
+    return head + (size_t)nstages * kStage + (size_t)NT * C * 4 + (size_t)(2 * d.E + 2) * 4;
+}
+
+template <typename XT, int NT>
+static cudaError_t launch_fused_t(const FusedArgs& a, int n_sm, size_t smem_limit, cudaStream_t st) {
+    static int configured_device = -1;  // the opt-in limit is set once per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_device != dev) {
+        cudaError_t e = cudaFuncSetAttribute(moe_decode_fused_kernel<XT, NT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_limit);
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+    }
+    const size_t smem = fused_smem_bytes(a.d, NT, a.nstages);
+    moe_decode_fused_kernel<XT, NT><<<n_sm, kFT, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+int fused_stages_for(const Dims& d, int NT, size_t smem_limit) {
+    int ns = kMaxStages;
+    while (ns > 2 && fused_smem_bytes(d, NT, ns) > smem_limit) --ns;
+    return fused_smem_bytes(d, NT, ns) <= smem_limit ? ns : 0;
+}
+
+cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const float* wr, const float* bias,
+                                const void* x, coli_dtype dt, int T, void* y, const float* residual, const Plan& p,
+                                double* logits, float* h, float* o, int* ctl, int n_sm, size_t smem_limit,
+                                cudaStream_t st) {
+    if (T < 1 || T > kFusedMaxTok) return cudaErrorInvalidValue;
+    const int NT = T == 1 ? 1 : (T == 2 ? 2 : 4);
+    FusedArgs a;
+    a.weights = weights; a.d = d; a.wr = wr; a.bias = bias; a.x = x; a.y = y; a.residual = residual;
+    a.T = T; a.p = p; a.logits = logits; a.h = h; a.o = o; a.ctl = ctl;
+    a.umax = T * d.K < d.E ? T * d.K : d.E;
+    a.nstages = fused_stages_for(d, NT, smem_limit);
+    if (a.nstages < 2) return cudaErrorInvalidConfiguration;
+    if (dt == COLI_F32) {
+        if (NT == 1) return launch_fused_t<float, 1>(a, n_sm, smem_limit, st);
+        if (NT == 2) return launch_fused_t<float, 2>(a, n_sm, smem_limit, st);
+        return launch_fused_t<float, 4>(a, n_sm, smem_limit, st);
+    }
+    if (NT == 1) return launch_fused_t<__nv_bfloat16, 1>(a, n_sm, smem_limit, st);
+    if (NT == 2) return launch_fused_t<__nv_bfloat16, 2>(a, n_sm, smem_limit, st);
+    return launch_fused_t<__nv_bfloat16, 4>(a, n_sm, smem_limit, st);
+}
+
+}  // namespace coli

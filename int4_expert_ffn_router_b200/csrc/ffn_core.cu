@@ -15,58 +15,13 @@
 // packed FFMA2 with per-group accumulators scaled by the group's fp16 scale.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "int4_math.cuh"
 
 namespace coli {
 
 constexpr int kThreads = 256;  // 8 warps = 8 sub-tiles of one 128-row tile
 constexpr int kTB = 4;         // tokens per pass over the weights
 constexpr int kNP = 8;         // groups in flight per warp
-
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
-
-__device__ __forceinline__ float2 as_f2(uint32_t lo_bits, uint32_t hi_bits) {
-    return make_float2(__uint_as_float(lo_bits), __uint_as_float(hi_bits));
-}
-
-// Codes of one 32-bit word (layout in common.cuh) as four float pairs:
-// p04 = (row gi: col a, col a+1), p26 = (row gi: col a+8, a+9),
-// p15 = (row gi+8: col a, a+1),   p37 = (row gi+8: col a+8, a+9).
-__device__ __forceinline__ void decode_word(uint32_t w, float2& p04, float2& p26, float2& p15, float2& p37) {
-    constexpr uint32_t M = 0x4B000000u;  // 2^23
-    const uint32_t wh = w >> 12;
-    float2 f04 = as_f2(lop3_and_or(w, 0x0000000Fu, M), lop3_and_or(w, 0x000F0000u, M));
-    float2 f15 = as_f2(lop3_and_or(w, 0x000000F0u, M), lop3_and_or(wh, 0x00000F00u, M));
-    float2 f26 = as_f2(lop3_and_or(w, 0x00000F00u, M), lop3_and_or(wh, 0x0000F000u, M));
-    float2 f37 = as_f2(lop3_and_or(w, 0x0000F000u, M), lop3_and_or(wh, 0x000F0000u, M));
-    // f = 2^23 + v * 2^k  ->  q = f * 2^-k - (2^(23-k) + 8): exact
-    p04 = ffma2(f04, make_float2(1.0f, 0x1p-16f), make_float2(-8388616.0f, -136.0f));
-    p15 = ffma2(f15, make_float2(0x1p-4f, 0x1p-8f), make_float2(-524296.0f, -32776.0f));
-    p26 = ffma2(f26, make_float2(0x1p-8f, 0x1p-12f), make_float2(-32776.0f, -2056.0f));
-    p37 = ffma2(f37, make_float2(0x1p-12f, 0x1p-16f), make_float2(-2056.0f, -136.0f));
-}
-
-template <typename XT>
-__device__ __forceinline__ float to_f32(XT v);
-template <>
-__device__ __forceinline__ float to_f32<float>(float v) { return v; }
-template <>
-__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
-
-// Stage rows of the input (C inputs each) into shared memory in lane order:
-// xs[tb][g][ti][s] = float4(x[c], x[c+1], x[c+8], x[c+9]), c = 64g + 16s + 2ti.
-template <typename XT>
-__device__ __forceinline__ void stage_rows(float4* xs, const XT* __restrict__ in, const int32_t* rows, int nt, int C) {
-    const int G = C / kGroup;
-    for (int idx = threadIdx.x; idx < nt * G * 16; idx += blockDim.x) {
-        int tb = idx / (G * 16);
-        int r = idx - tb * G * 16;
-        int g = r >> 4, ti = (r >> 2) & 3, s = r & 3;
-        int c = g * 64 + s * 16 + ti * 2;
-        const XT* src = in + (size_t)rows[tb] * C + c;
-        xs[((tb * G + g) * 4 + ti) * 4 + s] =
-            make_float4(to_f32<XT>(src[0]), to_f32<XT>(src[1]), to_f32<XT>(src[8]), to_f32<XT>(src[9]));
-    }
-}
 
 // One 128-row tile of an int4 matrix times up to kTB staged input rows.
 // Returns, per token, the fp32 results of rows gi (acc0) and gi+8 (acc1) of
@@ -100,34 +55,7 @@ __device__ __forceinline__ void tile_dot(const uint8_t* __restrict__ tile, int G
                     wb[i] = ldg_stream(wp + (size_t)(g + kNP) * kBlockBytes);
                     sb[i] = ldg_stream32(sp + (size_t)(g + kNP) * kBlockBytes);
                 }
-                const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sv));
-                float2 a0[kTB], a1[kTB];
-#pragma unroll
-                for (int tb = 0; tb < kTB; ++tb) { a0[tb] = make_float2(0.f, 0.f); a1[tb] = make_float2(0.f, 0.f); }
-                const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    float2 p04, p26, p15, p37;
-                    decode_word(words[s], p04, p26, p15, p37);
-#pragma unroll
-                    for (int tb = 0; tb < kTB; ++tb) {
-                        if (tb < nt) {
-                            const float4 xv = xs[((tb * G + g) * 4 + ti) * 4 + s];
-                            const float2 x01 = make_float2(xv.x, xv.y), x89 = make_float2(xv.z, xv.w);
-                            a0[tb] = ffma2(p04, x01, a0[tb]);
-                            a0[tb] = ffma2(p26, x89, a0[tb]);
-                            a1[tb] = ffma2(p15, x01, a1[tb]);
-                            a1[tb] = ffma2(p37, x89, a1[tb]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int tb = 0; tb < kTB; ++tb) {
-                    if (tb < nt) {
-                        acc0[tb] = fmaf(sc.x, a0[tb].x + a0[tb].y, acc0[tb]);
-                        acc1[tb] = fmaf(sc.y, a1[tb].x + a1[tb].y, acc1[tb]);
-                    }
-                }
+                group_dot<kTB>(wv, sv, xs + g * 16, G * 16, ti, nt, acc0, acc1);
             }
         }
     }
@@ -162,7 +90,7 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_core_kernel(const uint8_t*
             __syncthreads();
             if (threadIdx.x < nt) rows[threadIdx.x] = p.tok[off + t0 + threadIdx.x];
             __syncthreads();
-            stage_rows<XT>(xs, x, rows, nt, d.H);
+            stage_rows<XT>(xs, x, rows, nt, d.H, threadIdx.x, blockDim.x);
             __syncthreads();
             float g_acc[kTB], u_acc[kTB];
             tile_dot(tile, G, xs, nt, g_acc, u_acc);
@@ -195,7 +123,7 @@ __global__ void __launch_bounds__(kThreads, 2) down_core_kernel(const uint8_t* _
             __syncthreads();
             if (threadIdx.x < nt) rows[threadIdx.x] = off + t0 + threadIdx.x;  // h is indexed by position
             __syncthreads();
-            stage_rows<float>(xs, h, rows, nt, d.I);
+            stage_rows<float>(xs, h, rows, nt, d.I, threadIdx.x, blockDim.x);
             __syncthreads();
             float a0[kTB], a1[kTB];
             tile_dot(tile, G, xs, nt, a0, a1);

@@ -27,6 +27,15 @@ cudaError_t launch_gateup_core(const uint8_t* weights, const Dims& d, const void
 cudaError_t launch_down_core(const uint8_t* weights, const Dims& d, const float* h, int T, const Plan& p, float* o,
                              int max_active, int n_sm, cudaStream_t st);
 
+// decode_fused.cu: the whole layer for 1..kFusedMaxTok tokens in one
+// persistent launch (n_sm CTAs). ctl: control block of ctl_ints() ints,
+// zero at launch (the kernel leaves it zero, except a timeout code).
+cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const float* wr, const float* bias,
+                                const void* x, coli_dtype dt, int T, void* y, const float* residual, const Plan& p,
+                                double* logits, float* h, float* o, int* ctl, int n_sm, size_t smem_limit,
+                                cudaStream_t st);
+int fused_stages_for(const Dims& d, int NT, size_t smem_limit);
+
 // combine.cu
 // y[t] = residual[t] (optional) + sum_j o[TK + j*T + t] + sum_k w[t][k] o[pos[t][k]]
 cudaError_t launch_combine(const float* o, const Plan& p, int T, int H, int K, int S, const float* residual, void* y,

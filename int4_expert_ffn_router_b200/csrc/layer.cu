@@ -74,6 +74,9 @@ struct coli_moe_layer {
     float* h = nullptr;
     float* o = nullptr;
     float* xn = nullptr;
+    int* ctl = nullptr;             // control block of the persistent decode kernel
+    size_t smem_optin = 0;
+    bool fused = true;              // use the persistent kernel for n_tokens <= kFusedMaxTok
     uint8_t* staging = nullptr;  // one canonical expert, for host sources
     int last_T = -1;
     cudaStream_t last_stream = nullptr;
@@ -217,14 +220,23 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     // workspace
     const size_t TK = (size_t)Tm * d.K, slots = TK + (size_t)d.S * Tm, EA = (size_t)d.E + d.S;
     size_t sz[] = {Tm * (size_t)d.E * 8, TK * 4, TK * 4, (size_t)d.E * 4, (size_t)(d.E + 1) * 4, (size_t)d.E * 4, 4,
-                   TK * 4, slots * 4, EA * 4, EA * 4, EA * 4, 4, slots * d.I * 4, slots * d.H * 4, (size_t)Tm * d.H * 4};
+                   TK * 4, slots * 4, EA * 4, EA * 4, EA * 4, 4, slots * d.I * 4, slots * d.H * 4, (size_t)Tm * d.H * 4,
+                   (size_t)ctl_ints(d.E, d.S, d.H) * 4};
+    constexpr int kRegions = sizeof(sz) / sizeof(sz[0]);
     size_t total = 0;
     for (size_t s : sz) total += align256(s);
     if ((e = cudaMalloc(&L->ws, total)) != cudaSuccess) return bail(e, "cudaMalloc(workspace)");
     L->ws_bytes = total;
     uint8_t* cur = L->ws;
-    void* ptrs[16];
-    for (int i = 0; i < 16; ++i) { ptrs[i] = cur; cur += align256(sz[i]); }
+    void* ptrs[kRegions];
+    for (int i = 0; i < kRegions; ++i) { ptrs[i] = cur; cur += align256(sz[i]); }
+    L->ctl = (int*)ptrs[16];
+    {
+        int optin = 0;
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+        L->smem_optin = (size_t)optin;
+        L->fused = fused_stages_for(d, kFusedMaxTok, L->smem_optin) >= 4;
+    }
     L->logits = (double*)ptrs[0];
     Plan& p = L->plan;
     p.ids = (int32_t*)ptrs[1]; p.w = (float*)ptrs[2]; p.cnt = (int32_t*)ptrs[3]; p.off = (int32_t*)ptrs[4];
@@ -297,18 +309,26 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
     const Plan& p = L->plan;
     if (L->profiling && L->prof_issued - L->prof_folded >= coli_moe_layer::kRing)
         CUDA_TRY(prof_fold(L, L->prof_next), "profile");  // recycle the oldest slot
-    prof_mark(L, COLI_STAGE_ROUTER, s);
-    CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s), "router");
-    prof_mark(L, COLI_STAGE_TOPK, s);
-    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
-    prof_mark(L, COLI_STAGE_PLAN, s);
-    CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
-    prof_mark(L, COLI_STAGE_GATEUP, s);
-    CUDA_TRY(launch_gateup_core(L->weights, d, x, dt, T, p, L->h, L->max_active, L->n_sm, s), "gate/up");
-    prof_mark(L, COLI_STAGE_DOWN, s);
-    CUDA_TRY(launch_down_core(L->weights, d, L->h, T, p, L->o, L->max_active, L->n_sm, s), "down");
-    prof_mark(L, COLI_STAGE_COMBINE, s);
-    CUDA_TRY(launch_combine(L->o, p, T, d.H, d.K, d.S, residual, y, dt, s), "combine");
+    if (L->fused && T <= kFusedMaxTok) {
+        for (int i = 0; i <= COLI_STAGE_FUSED; ++i) prof_mark(L, i, s);
+        CUDA_TRY(launch_decode_fused(L->weights, d, L->router_w, L->router_b, x, dt, T, y, residual, p, L->logits, L->h,
+                                     L->o, L->ctl, L->n_sm, L->smem_optin, s),
+                 "persistent decode kernel");
+    } else {
+        prof_mark(L, COLI_STAGE_ROUTER, s);
+        CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s), "router");
+        prof_mark(L, COLI_STAGE_TOPK, s);
+        CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+        prof_mark(L, COLI_STAGE_PLAN, s);
+        CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
+        prof_mark(L, COLI_STAGE_GATEUP, s);
+        CUDA_TRY(launch_gateup_core(L->weights, d, x, dt, T, p, L->h, L->max_active, L->n_sm, s), "gate/up");
+        prof_mark(L, COLI_STAGE_DOWN, s);
+        CUDA_TRY(launch_down_core(L->weights, d, L->h, T, p, L->o, L->max_active, L->n_sm, s), "down");
+        prof_mark(L, COLI_STAGE_COMBINE, s);
+        CUDA_TRY(launch_combine(L->o, p, T, d.H, d.K, d.S, residual, y, dt, s), "combine");
+        prof_mark(L, COLI_STAGE_FUSED, s);
+    }
     prof_mark(L, COLI_N_STAGES, s);
     if (L->profiling) {
         L->prof_issued += 1;
@@ -358,12 +378,46 @@ COLI_API coli_status coli_moe_stack_forward(coli_moe_layer* const* layers, int n
     return COLI_OK;
 }
 
+// Waits for the layer's last forward and reports a device-side timeout of the
+// persistent kernel (then clears the control block so the layer stays usable).
+static coli_status sync_and_check(coli_moe_layer* L) {
+    CUDA_TRY(cudaStreamSynchronize(L->last_stream), "sync");
+    int err = 0;
+    CUDA_TRY(cudaMemcpy(&err, L->ctl + kCtlError, 4, cudaMemcpyDeviceToHost), "read status");
+    if (err != 0) {
+        CUDA_TRY(cudaMemset(L->ctl, 0, (size_t)ctl_ints(L->d.E, L->d.S, L->d.H) * 4), "reset control block");
+        char msg[96];
+        snprintf(msg, sizeof msg, "persistent decode kernel: a bounded wait timed out (site %d)", err);
+        g_last_error = msg;
+        return COLI_ECUDA;
+    }
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_sync(coli_moe_layer* L) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (L->last_T < 0) return COLI_OK;
+    DeviceGuard guard(L->device);
+    return sync_and_check(L);
+}
+
+COLI_API coli_status coli_moe_set_fused(coli_moe_layer* L, int enable) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (enable && fused_stages_for(L->d, kFusedMaxTok, L->smem_optin) < 4)
+        return fail(COLI_EUNSUPPORTED, "shapes too large for the persistent kernel's shared memory");
+    L->fused = enable != 0;
+    return COLI_OK;
+}
+
 COLI_API coli_status coli_moe_get_stats(coli_moe_layer* L, int* n_unique, int64_t* bytes_streamed,
                                         int32_t* per_expert_counts) {
     if (!L) return fail(COLI_EINVAL, "layer is NULL");
     if (L->last_T < 0) return fail(COLI_EINVAL, "no forward has run on this layer");
     DeviceGuard guard(L->device);
-    CUDA_TRY(cudaStreamSynchronize(L->last_stream), "sync");
+    {
+        coli_status st = sync_and_check(L);
+        if (st != COLI_OK) return st;
+    }
     int nu = 0;
     CUDA_TRY(cudaMemcpy(&nu, L->plan.n_unique, 4, cudaMemcpyDeviceToHost), "read n_unique");
     if (n_unique) *n_unique = nu;
@@ -379,7 +433,10 @@ COLI_API coli_status coli_moe_get_plan(coli_moe_layer* L, int32_t* ids, float* w
     if (!L) return fail(COLI_EINVAL, "layer is NULL");
     if (L->last_T < 0) return fail(COLI_EINVAL, "no forward has run on this layer");
     DeviceGuard guard(L->device);
-    CUDA_TRY(cudaStreamSynchronize(L->last_stream), "sync");
+    {
+        coli_status st = sync_and_check(L);
+        if (st != COLI_OK) return st;
+    }
     const size_t TK = (size_t)L->last_T * L->d.K;
     const Plan& p = L->plan;
     int nu = 0;
@@ -425,7 +482,7 @@ COLI_API coli_status coli_moe_get_profile(coli_moe_layer* L, double* stage_ms_to
 }
 
 COLI_API const char* coli_moe_stage_name(int stage) {
-    static const char* names[COLI_N_STAGES] = {"router", "topk", "plan", "gateup", "down", "combine"};
+    static const char* names[COLI_N_STAGES] = {"router", "topk", "plan", "gateup", "down", "combine", "fused"};
     return (stage >= 0 && stage < COLI_N_STAGES) ? names[stage] : "";
 }
 

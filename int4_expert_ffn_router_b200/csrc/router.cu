@@ -6,6 +6,7 @@
 // section 二: the positions of a batch read each unique expert once.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "topk.cuh"
 
 namespace coli {
 
@@ -92,60 +93,24 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const float* __restr
 }
 
 // ---------------------------------------------------------------------------
-// Top-k: one warp per token. Lane l holds the logits of experts l, l+32, ...
-// K rounds each take the best remaining (largest logit, ties to the lower
-// id). Weights: softmax over the K selected logits, in fp64, summed in a
-// fixed order.
+// Top-k. Lane l of a warp holds the logits of experts l, l+32, ...; K rounds
+// each take the best remaining (largest logit, ties to the lower id); weights
+// are the softmax over the K selected logits, in fp64, fixed summation order.
 // ---------------------------------------------------------------------------
-constexpr int kMaxPerLane = 32;  // E <= 1024
-
-__device__ __forceinline__ bool better(double a, int ia, double b, int ib) {
-    return a > b || (a == b && ia < ib);
-}
-
+// ---------------------------------------------------------------------------
+// Top-k: one warp per token (warp_topk in topk.cuh).
+// ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ logits, int T, int E, int K,
                                                    int32_t* __restrict__ ids, float* __restrict__ w) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + warp;
     if (t >= T) return;
-    const double* l = logits + (size_t)t * E;
-    const int per = (E + 31) / 32;
-    double v[kMaxPerLane];
-    uint32_t taken = 0;
-#pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
-        int e = lane + 32 * i;
-        v[i] = (i < per && e < E) ? l[e] : -INFINITY;
-    }
-    double my_sel = 0.0;
-    int my_id = -1;
-    double top = 0.0;
-    for (int k = 0; k < K; ++k) {
-        double bv = -INFINITY;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < kMaxPerLane; ++i) {
-            int e = lane + 32 * i;
-            if (i < per && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) { bv = v[i]; bi = e; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-        }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (k == 0) top = bv;
-        if (lane == k) { my_sel = bv; my_id = bi; }
-    }
-    // softmax over the selected logits; lane k < K owns slot k
-    double ex = (lane < K) ? exp(my_sel - top) : 0.0;
-    double z = ex;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    int id;
+    float wt;
+    warp_topk<false>(logits + (size_t)t * E, E, K, lane, &id, &wt);
     if (lane < K) {
-        ids[(size_t)t * K + lane] = my_id;
-        w[(size_t)t * K + lane] = (float)(ex / z);
+        ids[(size_t)t * K + lane] = id;
+        w[(size_t)t * K + lane] = wt;
     }
 }
 

@@ -124,6 +124,29 @@ def test_tiny_fp32_parity(gpu, tiny, T):
     assert _max_rel(yd.cpu().numpy().astype(np.float64), y_ref) <= FP32_TOL
 
 
+@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
+def test_tiny_small_batch_both_paths(gpu, tiny, T, fused):
+    """n_tokens <= 4 runs the persistent kernel by default; both paths must
+    route identically and match the oracle."""
+    c, L, layer = tiny
+    layer.set_fused(fused)
+    try:
+        x = synth.x_f32(c["seed"], 50 + T, T, c["H"])
+        xd = torch.from_numpy(x).to(gpu)
+        yd = torch.full_like(xd, float("nan"))
+        for _ in range(3):  # repeated launches reuse the control block
+            layer.forward(xd, yd)
+        layer.sync()
+        y_ref, ids_ref, w_ref = oracle.moe_forward(cases.oracle_cfg(c), L["wr"], None, L["experts"], x)
+        plan = layer.plan(T)
+        _check_plan(plan, ids_ref, c["E"])
+        np.testing.assert_allclose(plan["weights"], w_ref, rtol=0, atol=1e-6)
+        assert _max_rel(yd.cpu().numpy().astype(np.float64), y_ref) <= FP32_TOL
+    finally:
+        layer.set_fused(True)
+
+
 def test_tiny_bf16_parity(gpu, tiny):
     c, L, layer = tiny
     T = 6
@@ -232,19 +255,36 @@ def _oracle_for_tokens(c, wr, bias, x, seed=0, layer=0):
     return oracle.moe_forward(cases.oracle_cfg(c), wr, bias, experts, x)
 
 
-@pytest.mark.parametrize("step", [0, 1])
-def test_full_decode_batch1(gpu, full, step):
+@pytest.mark.parametrize("step,fused", [(0, True), (1, True), (0, False)])
+def test_full_decode_batch1(gpu, full, step, fused):
     """One full-size layer (H 6144, I 2048, 256 experts top-8 + shared), one token."""
     c, layer, wr = full
+    layer.set_fused(fused)
     x = synth.x_f32(1000 + step, 0, 1, c["H"])
     xd = torch.from_numpy(x).to(gpu)
     yd = torch.empty_like(xd)
     layer.forward(xd, yd)
-    torch.cuda.synchronize()
+    layer.sync()
+    layer.set_fused(True)
     y_ref, ids_ref, _ = _oracle_for_tokens(c, wr, None, x)
     _check_plan(layer.plan(1), ids_ref, c["E"])
     nu, nbytes = layer.stats()
     assert nu == 8 and nbytes == 9 * 20_054_016 + 6_291_456
+    assert _max_rel(yd.cpu().numpy().astype(np.float64), y_ref) <= FP32_TOL
+
+
+def test_full_decode_batch4_zipf_fused_matches_oracle(gpu, full):
+    """Four tokens through the persistent kernel, Zipf-skewed bias absent:
+    routing/union bit-exact, all four outputs against the oracle."""
+    c, layer, wr = full
+    T = 4
+    x = synth.x_f32(4000, 0, T, c["H"])
+    xd = torch.from_numpy(x).to(gpu)
+    yd = torch.empty_like(xd)
+    layer.forward(xd, yd)
+    layer.sync()
+    y_ref, ids_ref, _ = _oracle_for_tokens(c, wr, None, x)
+    _check_plan(layer.plan(T), ids_ref, c["E"])
     assert _max_rel(yd.cpu().numpy().astype(np.float64), y_ref) <= FP32_TOL
 
 
