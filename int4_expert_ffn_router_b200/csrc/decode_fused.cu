@@ -9,7 +9,9 @@
 // dependent steps. Design:
 //  * one CTA per SM; a producer warp streams weight tiles into a shared-memory
 //    ring with bulk asynchronous copies (the TMA engine) completing on
-//    mbarriers; 16 consumer warps dequantise and multiply out of the ring;
+//    mbarriers; 16 consumer warps dequantise and multiply out of the ring on
+//    the tensor cores from registers (int4_mma.cuh): the CUDA-core budget per
+//    streamed weight, not the tensor pipe, is what limits a decode GEMV;
 //  * work items are handed out by a global ticket counter in dependency
 //    order: router rows, the plan, shared-expert gate/up, shared-expert down,
 //    routed gate/up, routed down. An item only waits for items with smaller
@@ -24,7 +26,7 @@
 //    that block of y in a fixed order (shared experts, then the routed ones
 //    in routing order), so no extra pass and no atomics on y.
 #include "common.cuh"
-#include "int4_math.cuh"
+#include "int4_mma.cuh"
 #include "kernels.cuh"
 #include "topk.cuh"
 
@@ -37,6 +39,7 @@ constexpr int kSB = 2;                       // 4352-byte blocks per ring stage
 constexpr int kStage = kSB * kBlockBytes;    // 8704 bytes
 constexpr int kQ = 2;                        // item queue slots (lookahead of one item)
 constexpr uint64_t kWaitNs = 1000000000ull;  // every wait gives up after 1 s
+constexpr int kRouterExperts = 2;            // experts per router item (8 warps each)
 
 enum { IT_END = 0, IT_ROUTER = 1, IT_PLAN = 2, IT_GU = 3, IT_DOWN = 4 };
 
@@ -60,6 +63,8 @@ struct FusedArgs {
     int* ctl;
     int umax;     // min(T*K, E): upper bound of distinct routed experts
     int nstages;  // ring stages
+    long long* trace;  // item timeline (NULL: off); [0] = records written
+    int trace_cap;     // records of 4 x int64 after the header
 };
 
 // Shared-memory layout (dynamic).
@@ -71,9 +76,12 @@ struct FusedSmem {
     int staged_n, staged_rows[kFusedMaxTok];
     int srow[kFusedMaxTok];
     int sflag;
+    unsigned long long first_wait_ns;
+    float xscale[kFusedMaxTok];
+    float mred[(kCW + 1) * kFusedMaxTok];
     double rpart[kCW][kFusedMaxTok];
     int sids[kFusedMaxTok * 32];
-    float red[8 * 8 * 2 * kFusedMaxTok];
+    float red[8 * 32 * 4];
 };
 
 __device__ __forceinline__ void set_error(FusedArgs& a, volatile int* abort_flag, int code) {
@@ -117,17 +125,18 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
     const int T = a.T;
     const int RTgu = 2 * d.I / kTileRows, RTd = d.H / kTileRows;
     const int Ggu = d.H / kGroup, Gd = d.I / kGroup;
-    const int t_plan = d.E, t_sg = t_plan + 1, t_sd = t_sg + d.S * RTgu, t_ug = t_sd + d.S * RTd;
+    const int n_router = (d.E + kRouterExperts - 1) / kRouterExperts;
+    const int t_plan = n_router, t_sg = t_plan + 1, t_sd = t_sg + d.S * RTgu, t_ug = t_sd + d.S * RTd;
     const int t_ud = t_ug + a.umax * RTgu, t_end = t_ud + a.umax * RTd;
     volatile int* abort_flag = &S.abort_flag;
     int n_unique = -1;
-    uint32_t q = 0, gs = 0;
+    uint32_t q = 0, gs = 0, slot_s = 0, phase_s = 0;
     while (true) {
         Item it{IT_END, 0, 0, 0, 0, 0};
         if (!*abort_flag) {
             const int t = atomicAdd(&a.ctl[kCtlTicket], 1);
             if (t < t_plan) {
-                it = Item{IT_ROUTER, t, 0, 0, 0, 0};
+                it = Item{IT_ROUTER, t * kRouterExperts, 0, 0, 0, 0};
             } else if (t == t_plan) {
                 it = Item{IT_PLAN, 0, 0, 0, 0, 0};
             } else if (t < t_sd) {
@@ -161,16 +170,19 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
             const int G = gu ? Ggu : Gd;
             const uint8_t* tile = a.weights + (size_t)it.ex * d.expert_stride + (gu ? 0 : d.gu_bytes) +
                                   (size_t)it.rt * G * kBlockBytes;
-            for (int b0 = 0; b0 < G; b0 += kSB) {
+            bool stop = false;
+            for (int b0 = 0; b0 < G && !stop; b0 += kSB) {
                 const int nb = min(kSB, G - b0);
-                const uint32_t s = gs % a.nstages;
-                if (gs >= (uint32_t)a.nstages &&
-                    !wait_bar(&S.empty[s], ((gs / a.nstages) - 1) & 1, abort_flag, a, 4)) {
+                // slot_s = gs % nstages, phase_s = (gs / nstages) & 1
+                if (gs >= (uint32_t)a.nstages && !wait_bar(&S.empty[slot_s], phase_s ^ 1, abort_flag, a, 4)) {
+                    stop = true;
                     break;
                 }
-                mbar_arrive_expect_tx(&S.full[s], nb * kBlockBytes);
-                bulk_g2s(ring + (size_t)s * kStage, tile + (size_t)b0 * kBlockBytes, nb * kBlockBytes, &S.full[s]);
+                mbar_arrive_expect_tx(&S.full[slot_s], nb * kBlockBytes);
+                bulk_g2s(ring + (size_t)slot_s * kStage, tile + (size_t)b0 * kBlockBytes, nb * kBlockBytes,
+                         &S.full[slot_s]);
                 ++gs;
+                if (++slot_s == (uint32_t)a.nstages) { slot_s = 0; phase_s ^= 1; }
             }
         }
     }
@@ -184,35 +196,52 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
 }
 
 // ------------------------------------------------------------------ consumers
+// Router rows e0, e0+1: warps 8r..8r+7 take expert e0 + r, each an eighth of
+// H, loads issued before the fp64 products; fixed-order reduction.
 template <typename XT, int NT>
-__device__ void router_item(FusedArgs& a, FusedSmem& S, int e, int ctid) {
+__device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
     const Dims& d = a.d;
     const int cw = ctid >> 5, lane = ctid & 31;
-    const int chunk = d.H / kCW;
-    const float* wrow = a.wr + (size_t)e * d.H + cw * chunk;
+    const int r = cw >> 3, part = cw & 7;
+    const int e = e0 + r;
+    const int chunk = d.H / 8;
     const XT* x = reinterpret_cast<const XT*>(a.x);
     double acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.0;
-    for (int i = lane * 4; i < chunk; i += 128) {
-        const float4 w4 = __ldg(reinterpret_cast<const float4*>(wrow + i));
+    if (e < d.E) {
+        const float* wrow = a.wr + (size_t)e * d.H + part * chunk;
+        for (int base = 0; base < chunk; base += 1024) {
+            float4 wv[8];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            if (t < a.T) {
-                const XT* xp = x + (size_t)t * d.H + cw * chunk + i;
-                double x0, x1, x2, x3;
-                if constexpr (sizeof(XT) == 4) {
-                    const float4 v = __ldg(reinterpret_cast<const float4*>(xp));
-                    x0 = v.x; x1 = v.y; x2 = v.z; x3 = v.w;
-                } else {
-                    const uint2 u = __ldg(reinterpret_cast<const uint2*>(xp));
-                    x0 = __uint_as_float(u.x << 16); x1 = __uint_as_float(u.x & 0xFFFF0000u);
-                    x2 = __uint_as_float(u.y << 16); x3 = __uint_as_float(u.y & 0xFFFF0000u);
+            for (int j = 0; j < 8; ++j) {
+                const int i = base + lane * 4 + j * 128;
+                wv[j] = i < chunk ? __ldg(reinterpret_cast<const float4*>(wrow + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                if (t < a.T) {
+                    const XT* xr = x + (size_t)t * d.H + part * chunk;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int i = base + lane * 4 + j * 128;
+                        if (i < chunk) {
+                            double x0, x1, x2, x3;
+                            if constexpr (sizeof(XT) == 4) {
+                                const float4 v = __ldg(reinterpret_cast<const float4*>(xr + i));
+                                x0 = v.x; x1 = v.y; x2 = v.z; x3 = v.w;
+                            } else {
+                                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr + i));
+                                x0 = __uint_as_float(u.x << 16); x1 = __uint_as_float(u.x & 0xFFFF0000u);
+                                x2 = __uint_as_float(u.y << 16); x3 = __uint_as_float(u.y & 0xFFFF0000u);
+                            }
+                            acc[t] = fma((double)wv[j].x, x0, acc[t]);
+                            acc[t] = fma((double)wv[j].y, x1, acc[t]);
+                            acc[t] = fma((double)wv[j].z, x2, acc[t]);
+                            acc[t] = fma((double)wv[j].w, x3, acc[t]);
+                        }
+                    }
                 }
-                acc[t] = fma((double)w4.x, x0, acc[t]);
-                acc[t] = fma((double)w4.y, x1, acc[t]);
-                acc[t] = fma((double)w4.z, x2, acc[t]);
-                acc[t] = fma((double)w4.w, x3, acc[t]);
             }
         }
     }
@@ -223,10 +252,13 @@ __device__ void router_item(FusedArgs& a, FusedSmem& S, int e, int ctid) {
         if (lane == 0) S.rpart[cw][t] = acc[t];
     }
     named_bar(1, kCT);
-    if (ctid < a.T) {
-        double s = 0.0;
-        for (int w = 0; w < kCW; ++w) s += S.rpart[w][ctid];
-        a.logits[(size_t)ctid * d.E + e] = s + (double)a.bias[e];
+    if (ctid < kRouterExperts * a.T) {
+        const int rr = ctid / a.T, t = ctid % a.T, ee = e0 + rr;
+        if (ee < d.E) {
+            double sum = 0.0;
+            for (int w = 0; w < 8; ++w) sum += S.rpart[rr * 8 + w][t];
+            a.logits[(size_t)t * d.E + ee] = sum + (double)a.bias[ee];
+        }
     }
     named_bar(1, kCT);
     if (ctid == 0) {
@@ -243,12 +275,17 @@ __device__ void plan_item(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* 
     volatile int* abort_flag = &S.abort_flag;
     // Control flow below never depends on the abort flag around a barrier:
     // on abort the work is skipped but every thread meets every barrier.
-    if (ctid == 0) wait_geq(&a.ctl[kCtlRouter], E, abort_flag, a, 5);
+    if (ctid == 0) {
+        const uint64_t t0 = a.trace ? globaltimer_ns() : 0;
+        wait_geq(&a.ctl[kCtlRouter], (E + kRouterExperts - 1) / kRouterExperts, abort_flag, a, 5);
+        if (a.trace) S.first_wait_ns = globaltimer_ns() - t0;
+    }
     named_bar(1, kCT);
     if (cw < T && !*abort_flag) {
         int id;
         float wt;
-        warp_topk<true>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
+        if (E <= 256) warp_topk<true, 8>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
+        else warp_topk<true>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
         if (lane < K) {
             a.p.ids[cw * K + lane] = id;
             a.p.w[cw * K + lane] = wt;
@@ -321,11 +358,11 @@ __device__ void plan_item(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* 
 }
 
 template <typename XT, int NT>
-__device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t* ring, float4* xs, uint32_t& gs,
-                            int ctid) {
+__device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t* ring, uint4* xa, uint32_t& slot_s,
+                            uint32_t& phase_s, int ctid) {
     const Dims& d = a.d;
     const int T = a.T;
-    const int cw = ctid >> 5, lane = ctid & 31, gi = lane >> 2, ti = lane & 3;
+    const int cw = ctid >> 5, lane = ctid & 31, tok = lane >> 2, t4 = lane & 3;
     const bool gu = it.kind == IT_GU;
     const int C = gu ? d.H : d.I;
     const int G = C / kGroup;
@@ -341,9 +378,9 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
     named_bar(1, kCT);
     bool same = gu && S.staged_n == nt;
     for (int i = 0; same && i < nt; ++i) same = S.staged_rows[i] == S.srow[i];
-    if (!same && !*abort_flag) {
-        if (gu) stage_rows<XT, false>(xs, reinterpret_cast<const XT*>(a.x), S.srow, nt, C, ctid, kCT);
-        else stage_rows<float, true>(xs, a.h, S.srow, nt, C, ctid, kCT);
+    if (!same) {  // uniform: every consumer reads the same shared values
+        if (gu) stage_afrag<XT, NT>(xa, S.xscale, reinterpret_cast<const XT*>(a.x), S.srow, nt, C, false, ctid, kCT, 1, S.mred);
+        else stage_afrag<float, NT>(xa, S.xscale, a.h, S.srow, nt, C, true, ctid, kCT, 1, S.mred);
     }
     named_bar(1, kCT);
     if (ctid == 0) {
@@ -351,56 +388,46 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
         for (int i = 0; i < nt; ++i) S.staged_rows[i] = S.srow[i];
     }
 
-    float acc0[NT], acc1[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) { acc0[t] = 0.f; acc1[t] = 0.f; }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
     const int half = cw >> 3, sub = cw & 7;
     const int nst = (G + kSB - 1) / kSB;
     for (int i = 0; i < nst; ++i) {
-        const uint32_t s = gs % a.nstages;
-        const uint32_t par = (gs / a.nstages) & 1;
-        ++gs;
-        const bool ok = wait_bar(&S.full[s], par, abort_flag, a, 7);
+        uint64_t tw = 0;
+        if (a.trace && ctid == 0 && i == 0) tw = globaltimer_ns();
+        const bool ok = wait_bar(&S.full[slot_s], phase_s, abort_flag, a, 7);
+        if (a.trace && ctid == 0 && i == 0) S.first_wait_ns = globaltimer_ns() - tw;
         const int g = i * kSB + half;
         if (ok && g < G) {
-            const uint8_t* bp = ring + (size_t)s * kStage + half * kBlockBytes;
+            const uint8_t* bp = ring + (size_t)slot_s * kStage + half * kBlockBytes;
             const uint4 w = *reinterpret_cast<const uint4*>(bp + sub * 512 + lane * 16);
-            const uint32_t sv = *reinterpret_cast<const uint32_t*>(bp + kNibbleBytes + sub * 32 + gi * 4);
-            group_dot<NT>(w, sv, xs + g * 16, G * 16, ti, nt, acc0, acc1);
+            const uint2 sc = *reinterpret_cast<const uint2*>(bp + kNibbleBytes + sub * 32 + t4 * 8);
+            group_mma<NT>(w, sc, xa + (size_t)g * 4 * NT * 4, tok, t4, nt, acc);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[s]);
+        if (lane == 0) mbar_arrive(&S.empty[slot_s]);
+        if (++slot_s == (uint32_t)a.nstages) { slot_s = 0; phase_s ^= 1; }
     }
+    // odd-group warps hand their partial sums to the even-group warps
+    if (half == 1) {
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-        acc0[t] += __shfl_xor_sync(0xffffffffu, acc0[t], 1);
-        acc0[t] += __shfl_xor_sync(0xffffffffu, acc0[t], 2);
-        acc1[t] += __shfl_xor_sync(0xffffffffu, acc1[t], 1);
-        acc1[t] += __shfl_xor_sync(0xffffffffu, acc1[t], 2);
-    }
-    if (half == 1 && ti == 0) {
-#pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            S.red[((sub * 8 + gi) * NT + t) * 2 + 0] = acc0[t];
-            S.red[((sub * 8 + gi) * NT + t) * 2 + 1] = acc1[t];
-        }
+        for (int j = 0; j < 4; ++j) S.red[(sub * 32 + lane) * 4 + j] = acc[j];
     }
     named_bar(1, kCT);
-    if (half == 0 && ti == 0 && !*abort_flag) {
+    if (half == 0 && tok < nt && !*abort_flag) {
+        const float xs = S.xscale[tok];
+        float v[4];
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-            if (t < nt) {
-                const float v0 = acc0[t] + S.red[((sub * 8 + gi) * NT + t) * 2 + 0];
-                const float v1 = acc1[t] + S.red[((sub * 8 + gi) * NT + t) * 2 + 1];
-                if (gu) {
-                    const int j = (it.rt * 8 + sub) * 8 + gi;
-                    a.h[(size_t)(it.off + t) * d.I + j] = silu_f(v0) * v1;
-                } else {
-                    const int r0 = it.rt * kTileRows + sub * kSubRows + gi;
-                    a.o[(size_t)(it.off + t) * d.H + r0] = v0;
-                    a.o[(size_t)(it.off + t) * d.H + r0 + 8] = v1;
-                }
-            }
+        for (int j = 0; j < 4; ++j) v[j] = (acc[j] + S.red[(sub * 32 + lane) * 4 + j]) * xs;
+        if (gu) {
+            // rows 2t, 2t+1 of the sub-tile are gate rows j, j+1; rows 8+2t, 9+2t the matching up rows
+            const int j = (it.rt * 8 + sub) * 8 + 2 * t4;
+            float2 hv = make_float2(silu_f(v[0]) * v[2], silu_f(v[1]) * v[3]);
+            *reinterpret_cast<float2*>(a.h + (size_t)(it.off + tok) * d.I + j) = hv;
+        } else {
+            const int r0 = it.rt * kTileRows + sub * kSubRows + 2 * t4;
+            float* orow = a.o + (size_t)(it.off + tok) * d.H;
+            *reinterpret_cast<float2*>(orow + r0) = make_float2(v[0], v[1]);
+            *reinterpret_cast<float2*>(orow + r0 + 8) = make_float2(v[2], v[3]);
         }
     }
     named_bar(1, kCT);
@@ -445,8 +472,8 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     FusedSmem& S = *reinterpret_cast<FusedSmem*>(smem);
     uint8_t* ring = smem + ((sizeof(FusedSmem) + 127) & ~(size_t)127);
-    float4* xs = reinterpret_cast<float4*>(ring + (size_t)a.nstages * kStage);
-    int* scnt = reinterpret_cast<int*>(xs + (size_t)NT * (a.d.H > a.d.I ? a.d.H : a.d.I) / 4);
+    uint4* xa = reinterpret_cast<uint4*>(ring + (size_t)a.nstages * kStage);
+    int* scnt = reinterpret_cast<int*>(xa + (size_t)NT * (a.d.H > a.d.I ? a.d.H : a.d.I) / 4);
     int* soff = scnt + a.d.E + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -462,7 +489,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
         __syncwarp();
     } else {
         const int ctid = tid;
-        uint32_t q = 0, gs = 0;
+        uint32_t q = 0, slot_s = 0, phase_s = 0;
         while (true) {
             // thread 0 takes the next item and publishes it, so every consumer
             // thread takes the same branch below
@@ -474,10 +501,24 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
             }
             named_bar(1, kCT);
             const Item it = S.cur[q & 1];
+            const uint64_t t_begin = (a.trace && ctid == 0) ? globaltimer_ns() : 0;
+            if (ctid == 0) S.first_wait_ns = 0;
             if (it.kind == IT_ROUTER) router_item<XT, NT>(a, S, it.ex, ctid);
             else if (it.kind == IT_PLAN) plan_item(a, S, ctid, scnt, soff);
-            else if (it.kind == IT_GU || it.kind == IT_DOWN) weight_item<XT, NT>(a, S, it, ring, xs, gs, ctid);
+            else if (it.kind == IT_GU || it.kind == IT_DOWN)
+                weight_item<XT, NT>(a, S, it, ring, xa, slot_s, phase_s, ctid);
             named_bar(1, kCT);
+            if (a.trace && ctid == 0 && it.kind != IT_END) {
+                // record: (cta << 40 | kind << 32 | ex << 16 | rt), begin, end, first-data wait
+                const unsigned long long r = atomicAdd(reinterpret_cast<unsigned long long*>(a.trace), 1ull);
+                if (r < (unsigned long long)a.trace_cap) {
+                    long long* rec = a.trace + 4 + 4 * r;
+                    rec[0] = ((long long)blockIdx.x << 40) | ((long long)it.kind << 32) | ((long long)it.ex << 16) | it.rt;
+                    rec[1] = (long long)t_begin;
+                    rec[2] = (long long)globaltimer_ns();
+                    rec[3] = (long long)S.first_wait_ns;
+                }
+            }
             if (ctid == 0 && it.kind != IT_END) mbar_arrive(&S.qempty[slot]);
             ++q;
             if (it.kind == IT_END) break;
@@ -527,12 +568,13 @@ int fused_stages_for(const Dims& d, int NT, size_t smem_limit) {
 cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const float* wr, const float* bias,
                                 const void* x, coli_dtype dt, int T, void* y, const float* residual, const Plan& p,
                                 double* logits, float* h, float* o, int* ctl, int n_sm, size_t smem_limit,
-                                cudaStream_t st) {
+                                long long* trace, int trace_cap, cudaStream_t st) {
     if (T < 1 || T > kFusedMaxTok) return cudaErrorInvalidValue;
     const int NT = T == 1 ? 1 : (T == 2 ? 2 : 4);
     FusedArgs a;
     a.weights = weights; a.d = d; a.wr = wr; a.bias = bias; a.x = x; a.y = y; a.residual = residual;
     a.T = T; a.p = p; a.logits = logits; a.h = h; a.o = o; a.ctl = ctl;
+    a.trace = trace; a.trace_cap = trace_cap;
     a.umax = T * d.K < d.E ? T * d.K : d.E;
     a.nstages = fused_stages_for(d, NT, smem_limit);
     if (a.nstages < 2) return cudaErrorInvalidConfiguration;

@@ -1,0 +1,158 @@
+// int4_mma.cuh -- int4 x (few tokens) products on the tensor cores from
+// register operands, for the decode kernel.
+//
+// A decode step multiplies each streamed weight by one to four tokens: the
+// contraction is far too thin for shared-memory tensor-core tiles, but the
+// CUDA-core instruction budget per streamed weight is the limit at HBM speed.
+// Here the weights are the B operand of mma.m16n8k16 (8 weight rows x 16
+// inputs per instruction) and the tokens the A operand: row m < 8 of A is the
+// high fp16 part of token m, row 8 + m its low part (x = hi + lo to ~22 bits
+// after a per-token power-of-two scale), so one instruction serves up to 8
+// tokens at full precision and the dequantisation costs 9 instructions per 8
+// weights: the nibbles are OR-ed into the mantissa of fp16 1024 (one LOP3 per
+// two weights) and one HFMA2 removes the bias, the bit position and the +8
+// offset exactly.
+#pragma once
+
+#include "common.cuh"
+
+namespace coli {
+
+__device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// d += A (16x16 fp16, row) * B (16x8 fp16, col), fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float d[4], const uint4& a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
+}
+
+// One 32-bit weight word (layout in common.cuh) -> the B fragments of the two
+// 8-row halves of the sub-tile for one 16-input step:
+//   b00/b01: rows gi   (k = 2ti,2ti+1 | 2ti+8,2ti+9)
+//   b10/b11: rows gi+8 (same k)
+__device__ __forceinline__ void dequant_word_f16(uint32_t w, uint32_t& b00, uint32_t& b01, uint32_t& b10,
+                                                 uint32_t& b11) {
+    constexpr uint32_t MAGIC = 0x64006400u;    // fp16 1024, 1024
+    constexpr uint32_t ONE = 0x3C003C00u;      // 1.0, 1.0
+    constexpr uint32_t M1032 = 0xE408E408u;    // -1032, -1032
+    constexpr uint32_t SIXTEENTH = 0x2C002C00u;  // 1/16
+    constexpr uint32_t M72 = 0xD480D480u;      // -72, -72
+    const uint32_t ws = w >> 8;
+    const uint32_t lo0 = lop3_and_or(w, 0x000F000Fu, MAGIC);   // 1024 + v   (row gi,   k lo)
+    const uint32_t hi0 = lop3_and_or(w, 0x00F000F0u, MAGIC);   // 1024 + 16v (row gi+8, k lo)
+    const uint32_t lo1 = lop3_and_or(ws, 0x000F000Fu, MAGIC);  // row gi,   k hi
+    const uint32_t hi1 = lop3_and_or(ws, 0x00F000F0u, MAGIC);  // row gi+8, k hi
+    b00 = hfma2_u(lo0, ONE, M1032);        // v - 8
+    b01 = hfma2_u(lo1, ONE, M1032);
+    b10 = hfma2_u(hi0, SIXTEENTH, M72);    // (1024 + 16v)/16 - 72 = v - 8
+    b11 = hfma2_u(hi1, SIXTEENTH, M72);
+}
+
+// One 64-input group of a 16-row sub-tile for up to 8 tokens.
+// w: this lane's 16 bytes of the group; sc: the lane's two fp16 scale pairs
+// {(row 2t, row 2t+8), (row 2t+1, row 2t+9)}; xa: the group's A fragments
+// (4 steps x ntok x 4 lanes-of-row x 16 B); tok = lane / 4.
+// acc[0..3]: token `tok`, sub-tile rows 2t, 2t+1, 8+2t, 9+2t.
+template <int NT>
+__device__ __forceinline__ void group_mma(uint4 w, uint2 sc, const uint4* __restrict__ xa, int tok, int t, int nt,
+                                          float acc[4]) {
+    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        uint4 a = make_uint4(0u, 0u, 0u, 0u);
+        if (tok < nt) a = xa[(s * NT + tok) * 4 + t];
+        uint32_t b00, b01, b10, b11;
+        dequant_word_f16(words[s], b00, b01, b10, b11);
+        mma_16816(d0, a, b00, b01);
+        mma_16816(d1, a, b10, b11);
+    }
+    const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));  // rows 2t, 2t+8
+    const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));  // rows 2t+1, 2t+9
+    acc[0] = fmaf(s01.x, d0[0] + d0[2], acc[0]);
+    acc[1] = fmaf(s23.x, d0[1] + d0[3], acc[1]);
+    acc[2] = fmaf(s01.y, d1[0] + d1[2], acc[2]);
+    acc[3] = fmaf(s23.y, d1[1] + d1[3], acc[3]);
+}
+
+// 2^k as a float for k in [-126, 127].
+__device__ __forceinline__ float exp2i(int k) { return __uint_as_float((uint32_t)(127 + k) << 23); }
+
+template <typename XT>
+__device__ __forceinline__ float load_in(const XT* p, bool coherent);
+template <>
+__device__ __forceinline__ float load_in<float>(const float* p, bool coherent) { return coherent ? __ldcg(p) : __ldg(p); }
+template <>
+__device__ __forceinline__ float load_in<__nv_bfloat16>(const __nv_bfloat16* p, bool coherent) {
+    return __bfloat162float(*p);
+}
+
+__device__ __forceinline__ uint32_t split_pair(float a, float b, uint32_t& lo) {
+    const __half ha = __float2half_rn(a), hb = __float2half_rn(b);
+    const __half la = __float2half_rn(a - __half2float(ha)), lb = __float2half_rn(b - __half2float(hb));
+    lo = (uint32_t)__half_as_ushort(la) | ((uint32_t)__half_as_ushort(lb) << 16);
+    return (uint32_t)__half_as_ushort(ha) | ((uint32_t)__half_as_ushort(hb) << 16);
+}
+
+// Stage nt (<= NT) input rows of C values as A fragments, scaled per row by a
+// power of two so that the row's largest magnitude lies in [2^14, 2^15), and
+// split into fp16 hi + lo. xa[((g*4 + s)*NT + tok)*4 + t] = {hi(k,k+1),
+// lo(k,k+1), hi(k+8,k+9), lo(k+8,k+9)}, k = 64g + 16s + 2t. scale_out[tok] =
+// the factor that undoes the row scaling. Uses consumer threads tid < nthr
+// and named barrier `bar` (two barriers); red: nthr/32 * NT floats.
+template <typename XT, int NT>
+__device__ __forceinline__ void stage_afrag(uint4* __restrict__ xa, float* scale_out, const XT* __restrict__ in,
+                                            const int* rows, int nt, int C, bool coherent, int tid, int nthr,
+                                            int bar, float* red) {
+    const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
+    float m[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        m[j] = 0.0f;
+        if (j < nt) {
+            const XT* r = in + (size_t)rows[j] * C;
+            for (int c = tid; c < C; c += nthr) m[j] = fmaxf(m[j], fabsf(load_in<XT>(r + c, coherent)));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], o));
+        if (lane == 0) red[warp * NT + j] = m[j];
+    }
+    named_bar(bar, nthr);
+    if (tid < NT) {
+        float mx = 0.0f;
+        for (int w = 0; w < nw; ++w) mx = fmaxf(mx, red[w * NT + tid]);
+        int k = 0;  // zero, subnormal or non-finite maxima: no scaling
+        const uint32_t eb = (__float_as_uint(mx) >> 23) & 0xFF;
+        if (eb != 0 && eb != 0xFF) {
+            k = 14 - ((int)eb - 127);
+            k = k < -126 ? -126 : (k > 126 ? 126 : k);
+        }
+        red[nw * NT + tid] = exp2i(k);       // multiply inputs by this
+        scale_out[tid] = exp2i(-k);          // multiply results by this
+    }
+    named_bar(bar, nthr);
+    const int G = C / kGroup;
+    for (int idx = tid; idx < nt * G * 16; idx += nthr) {
+        const int tok = idx / (G * 16);
+        const int r = idx - tok * G * 16;
+        const int g = r >> 4, s = (r >> 2) & 3, t = r & 3;
+        const int k = g * 64 + s * 16 + t * 2;
+        const XT* src = in + (size_t)rows[tok] * C + k;
+        const float f = red[nw * NT + tok];
+        const float v0 = load_in<XT>(src, coherent) * f, v1 = load_in<XT>(src + 1, coherent) * f;
+        const float v8 = load_in<XT>(src + 8, coherent) * f, v9 = load_in<XT>(src + 9, coherent) * f;
+        uint4 o;
+        o.x = split_pair(v0, v1, o.y);
+        o.z = split_pair(v8, v9, o.w);
+        xa[((g * 4 + s) * NT + tok) * 4 + t] = o;
+    }
+}
+
+}  // namespace coli

@@ -33,7 +33,7 @@ cudaError_t launch_down_core(const uint8_t* weights, const Dims& d, const float*
 cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const float* wr, const float* bias,
                                 const void* x, coli_dtype dt, int T, void* y, const float* residual, const Plan& p,
                                 double* logits, float* h, float* o, int* ctl, int n_sm, size_t smem_limit,
-                                cudaStream_t st);
+                                long long* trace, int trace_cap, cudaStream_t st);
 int fused_stages_for(const Dims& d, int NT, size_t smem_limit);
 
 // combine.cu

@@ -77,6 +77,8 @@ struct coli_moe_layer {
     int* ctl = nullptr;             // control block of the persistent decode kernel
     size_t smem_optin = 0;
     bool fused = true;              // use the persistent kernel for n_tokens <= kFusedMaxTok
+    long long* trace = nullptr;     // caller-owned device buffer for the item timeline
+    int trace_cap = 0;
     uint8_t* staging = nullptr;  // one canonical expert, for host sources
     int last_T = -1;
     cudaStream_t last_stream = nullptr;
@@ -312,7 +314,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
     if (L->fused && T <= kFusedMaxTok) {
         for (int i = 0; i <= COLI_STAGE_FUSED; ++i) prof_mark(L, i, s);
         CUDA_TRY(launch_decode_fused(L->weights, d, L->router_w, L->router_b, x, dt, T, y, residual, p, L->logits, L->h,
-                                     L->o, L->ctl, L->n_sm, L->smem_optin, s),
+                                     L->o, L->ctl, L->n_sm, L->smem_optin, L->trace, L->trace_cap, s),
                  "persistent decode kernel");
     } else {
         prof_mark(L, COLI_STAGE_ROUTER, s);
@@ -406,6 +408,14 @@ COLI_API coli_status coli_moe_set_fused(coli_moe_layer* L, int enable) {
     if (enable && fused_stages_for(L->d, kFusedMaxTok, L->smem_optin) < 4)
         return fail(COLI_EUNSUPPORTED, "shapes too large for the persistent kernel's shared memory");
     L->fused = enable != 0;
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_set_trace(coli_moe_layer* L, void* buffer, int capacity) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (buffer && (capacity < 1 || ((uintptr_t)buffer & 7u))) return fail(COLI_EINVAL, "bad trace buffer");
+    L->trace = (long long*)buffer;
+    L->trace_cap = buffer ? capacity : 0;
     return COLI_OK;
 }
 

@@ -15,13 +15,13 @@ __device__ __forceinline__ bool better(double a, int ia, double b, int ib) {
 // the lower id) and their softmax weights over the selection (fp64, fixed
 // summation order). Lane k < K returns slot k in (*id, *wt). `coherent`:
 // read the logits through L2 only (they were written by another CTA).
-template <bool coherent>
+template <bool coherent, int PER = kMaxPerLane>
 __device__ __forceinline__ void warp_topk(const double* __restrict__ l, int E, int K, int lane, int* id, float* wt) {
-    const int per = (E + 31) / 32;
-    double v[kMaxPerLane];
+    const int per = (E + 31) / 32;  // <= PER
+    double v[PER];
     uint32_t taken = 0;
 #pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
+    for (int i = 0; i < PER; ++i) {
         int e = lane + 32 * i;
         double val = -INFINITY;
         if (i < per && e < E) val = coherent ? __ldcg(l + e) : l[e];
@@ -33,7 +33,7 @@ __device__ __forceinline__ void warp_topk(const double* __restrict__ l, int E, i
         double bv = -INFINITY;
         int bi = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < kMaxPerLane; ++i) {
+        for (int i = 0; i < PER; ++i) {
             int e = lane + 32 * i;
             if (i < per && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) { bv = v[i]; bi = e; }
         }
