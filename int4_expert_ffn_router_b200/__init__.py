@@ -177,7 +177,7 @@ class Layer:
 
     def set_trace(self, buffer, capacity: int) -> None:
         """Record the persistent kernel's item timeline into a zeroed device
-        int64 buffer of 4 + 4 * capacity entries (None disables)."""
+        int64 buffer of 8 + 8 * capacity entries (None disables)."""
         _check(lib.coli_moe_set_trace(self.handle, _ptr(buffer), capacity), "coli_moe_set_trace")
 
     def set_profiling(self, on: bool) -> None:

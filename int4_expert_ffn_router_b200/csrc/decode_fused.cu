@@ -35,8 +35,7 @@ namespace coli {
 constexpr int kCW = 16;                      // consumer warps
 constexpr int kCT = kCW * 32;                // consumer threads
 constexpr int kFT = kCT + 32;                // + the producer warp
-constexpr int kSB = 2;                       // 4352-byte blocks per ring stage
-constexpr int kStage = kSB * kBlockBytes;    // 8704 bytes
+constexpr int kMaxSB = 8;                    // 4352-byte blocks per ring stage (at most)
 constexpr int kQ = 2;                        // item queue slots (lookahead of one item)
 constexpr uint64_t kWaitNs = 1000000000ull;  // every wait gives up after 1 s
 constexpr int kRouterExperts = 2;            // experts per router item (8 warps each)
@@ -45,6 +44,7 @@ enum { IT_END = 0, IT_ROUTER = 1, IT_PLAN = 2, IT_GU = 3, IT_DOWN = 4 };
 
 struct Item {
     int kind, ex, rt, off, cnt, shared;
+    long long pushed_ns;  // trace only: when the producer published the item
 };
 
 struct FusedArgs {
@@ -63,6 +63,7 @@ struct FusedArgs {
     int* ctl;
     int umax;     // min(T*K, E): upper bound of distinct routed experts
     int nstages;  // ring stages
+    int sb;       // 4352-byte blocks per stage (even); the bulk copies are sb * 4352 bytes
     long long* trace;  // item timeline (NULL: off); [0] = records written
     int trace_cap;     // records of 4 x int64 after the header
 };
@@ -76,12 +77,12 @@ struct FusedSmem {
     int staged_n, staged_rows[kFusedMaxTok];
     int srow[kFusedMaxTok];
     int sflag;
-    unsigned long long first_wait_ns;
+    unsigned long long first_wait_ns, total_wait_ns;
     float xscale[kFusedMaxTok];
     float mred[(kCW + 1) * kFusedMaxTok];
     double rpart[kCW][kFusedMaxTok];
     int sids[kFusedMaxTok * 32];
-    float red[8 * 32 * 4];
+    float red[8 * 32 * 2];
 };
 
 __device__ __forceinline__ void set_error(FusedArgs& a, volatile int* abort_flag, int code) {
@@ -132,19 +133,19 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
     int n_unique = -1;
     uint32_t q = 0, gs = 0, slot_s = 0, phase_s = 0;
     while (true) {
-        Item it{IT_END, 0, 0, 0, 0, 0};
+        Item it{IT_END, 0, 0, 0, 0, 0, 0};
         if (!*abort_flag) {
             const int t = atomicAdd(&a.ctl[kCtlTicket], 1);
             if (t < t_plan) {
-                it = Item{IT_ROUTER, t * kRouterExperts, 0, 0, 0, 0};
+                it = Item{IT_ROUTER, t * kRouterExperts, 0, 0, 0, 0, 0};
             } else if (t == t_plan) {
-                it = Item{IT_PLAN, 0, 0, 0, 0, 0};
+                it = Item{IT_PLAN, 0, 0, 0, 0, 0, 0};
             } else if (t < t_sd) {
                 const int j = (t - t_sg) / RTgu, rt = (t - t_sg) % RTgu;
-                it = Item{IT_GU, d.E + j, rt, T * d.K + j * T, T, 1};
+                it = Item{IT_GU, d.E + j, rt, T * d.K + j * T, T, 1, 0};
             } else if (t < t_ug) {
                 const int j = (t - t_sd) / RTd, rt = (t - t_sd) % RTd;
-                it = Item{IT_DOWN, d.E + j, rt, T * d.K + j * T, T, 1};
+                it = Item{IT_DOWN, d.E + j, rt, T * d.K + j * T, T, 1, 0};
             } else if (t < t_end) {
                 if (n_unique < 0) {
                     if (!wait_geq(&a.ctl[kCtlPlan], 1, abort_flag, a, 2)) continue;
@@ -156,11 +157,12 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
                 const int u = r / RT, rt = r % RT;
                 if (u >= n_unique) continue;  // fewer distinct experts than the bound
                 const int ex = __ldcg(a.p.unique + u);
-                it = Item{gu ? IT_GU : IT_DOWN, ex, rt, __ldcg(a.p.off + ex), __ldcg(a.p.cnt + ex), 0};
+                it = Item{gu ? IT_GU : IT_DOWN, ex, rt, __ldcg(a.p.off + ex), __ldcg(a.p.cnt + ex), 0, 0};
             }
         }
         const uint32_t slot = q % kQ;
         if (q >= kQ && !wait_bar(&S.qempty[slot], ((q / kQ) - 1) & 1, abort_flag, a, 3)) it.kind = IT_END;
+        if (a.trace) it.pushed_ns = (long long)globaltimer_ns();
         S.items[slot] = it;
         mbar_arrive(&S.qfull[slot]);
         ++q;
@@ -170,16 +172,17 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
             const int G = gu ? Ggu : Gd;
             const uint8_t* tile = a.weights + (size_t)it.ex * d.expert_stride + (gu ? 0 : d.gu_bytes) +
                                   (size_t)it.rt * G * kBlockBytes;
+            const uint32_t stage_bytes = (uint32_t)a.sb * kBlockBytes;
             bool stop = false;
-            for (int b0 = 0; b0 < G && !stop; b0 += kSB) {
-                const int nb = min(kSB, G - b0);
+            for (int b0 = 0; b0 < G && !stop; b0 += a.sb) {
+                const int nb = min(a.sb, G - b0);
                 // slot_s = gs % nstages, phase_s = (gs / nstages) & 1
                 if (gs >= (uint32_t)a.nstages && !wait_bar(&S.empty[slot_s], phase_s ^ 1, abort_flag, a, 4)) {
                     stop = true;
                     break;
                 }
                 mbar_arrive_expect_tx(&S.full[slot_s], nb * kBlockBytes);
-                bulk_g2s(ring + (size_t)slot_s * kStage, tile + (size_t)b0 * kBlockBytes, nb * kBlockBytes,
+                bulk_g2s(ring + (size_t)slot_s * stage_bytes, tile + (size_t)b0 * kBlockBytes, nb * kBlockBytes,
                          &S.full[slot_s]);
                 ++gs;
                 if (++slot_s == (uint32_t)a.nstages) { slot_s = 0; phase_s ^= 1; }
@@ -275,10 +278,11 @@ __device__ void plan_item(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* 
     volatile int* abort_flag = &S.abort_flag;
     // Control flow below never depends on the abort flag around a barrier:
     // on abort the work is skipped but every thread meets every barrier.
+    uint64_t tp0 = 0;
     if (ctid == 0) {
-        const uint64_t t0 = a.trace ? globaltimer_ns() : 0;
+        tp0 = a.trace ? globaltimer_ns() : 0;
         wait_geq(&a.ctl[kCtlRouter], (E + kRouterExperts - 1) / kRouterExperts, abort_flag, a, 5);
-        if (a.trace) S.first_wait_ns = globaltimer_ns() - t0;
+        if (a.trace) S.first_wait_ns = globaltimer_ns() - tp0;
     }
     named_bar(1, kCT);
     if (cw < T && !*abort_flag) {
@@ -293,6 +297,7 @@ __device__ void plan_item(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* 
         }
     }
     named_bar(1, kCT);
+    if (a.trace && ctid == 0) a.trace[1] = (long long)(globaltimer_ns() - tp0);  // top-k done
     if (cw == 0 && !*abort_flag) {
         for (int e = lane; e < E; e += 32) scnt[e] = 0;
         __syncwarp();
@@ -352,21 +357,23 @@ __device__ void plan_item(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* 
     }
     named_bar(1, kCT);
     if (ctid == 0) {
+        if (a.trace) a.trace[2] = (long long)(globaltimer_ns() - tp0);  // plan written
         __threadfence();
         st_release(&a.ctl[kCtlPlan], 1);
+        if (a.trace) a.trace[3] = (long long)(globaltimer_ns() - tp0);  // published
     }
 }
 
 template <typename XT, int NT>
-__device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t* ring, uint4* xa, uint32_t& slot_s,
+__device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t* ring, uint4* xb, uint32_t& slot_s,
                             uint32_t& phase_s, int ctid) {
     const Dims& d = a.d;
-    const int T = a.T;
-    const int cw = ctid >> 5, lane = ctid & 31, tok = lane >> 2, t4 = lane & 3;
+    const int cw = ctid >> 5, lane = ctid & 31, gi = lane >> 2, t4 = lane & 3;
     const bool gu = it.kind == IT_GU;
     const int C = gu ? d.H : d.I;
     const int G = C / kGroup;
     const int nt = it.cnt;
+    constexpr int L = 8 * NT;  // lanes holding B-fragment columns of NT tokens
     volatile int* abort_flag = &S.abort_flag;
 
     // inputs: x rows of the item's tokens (gate/up) or its h rows (down)
@@ -379,8 +386,8 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
     bool same = gu && S.staged_n == nt;
     for (int i = 0; same && i < nt; ++i) same = S.staged_rows[i] == S.srow[i];
     if (!same) {  // uniform: every consumer reads the same shared values
-        if (gu) stage_afrag<XT, NT>(xa, S.xscale, reinterpret_cast<const XT*>(a.x), S.srow, nt, C, false, ctid, kCT, 1, S.mred);
-        else stage_afrag<float, NT>(xa, S.xscale, a.h, S.srow, nt, C, true, ctid, kCT, 1, S.mred);
+        if (gu) stage_bfrag<XT, NT>(xb, S.xscale, reinterpret_cast<const XT*>(a.x), S.srow, nt, C, false, ctid, kCT, 1, S.mred);
+        else stage_bfrag<float, NT>(xb, S.xscale, a.h, S.srow, nt, C, true, ctid, kCT, 1, S.mred);
     }
     named_bar(1, kCT);
     if (ctid == 0) {
@@ -388,46 +395,60 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
         for (int i = 0; i < nt; ++i) S.staged_rows[i] = S.srow[i];
     }
 
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc0 = 0.f, acc1 = 0.f;
     const int half = cw >> 3, sub = cw & 7;
-    const int nst = (G + kSB - 1) / kSB;
+    const uint32_t stage_bytes = (uint32_t)a.sb * kBlockBytes;
+    const bool has_b = lane < L;
+    const int nst = (G + a.sb - 1) / a.sb;
     for (int i = 0; i < nst; ++i) {
         uint64_t tw = 0;
-        if (a.trace && ctid == 0 && i == 0) tw = globaltimer_ns();
+        if (a.trace && ctid == 0) tw = globaltimer_ns();
         const bool ok = wait_bar(&S.full[slot_s], phase_s, abort_flag, a, 7);
-        if (a.trace && ctid == 0 && i == 0) S.first_wait_ns = globaltimer_ns() - tw;
-        const int g = i * kSB + half;
-        if (ok && g < G) {
-            const uint8_t* bp = ring + (size_t)slot_s * kStage + half * kBlockBytes;
-            const uint4 w = *reinterpret_cast<const uint4*>(bp + sub * 512 + lane * 16);
-            const uint2 sc = *reinterpret_cast<const uint2*>(bp + kNibbleBytes + sub * 32 + t4 * 8);
-            group_mma<NT>(w, sc, xa + (size_t)g * 4 * NT * 4, tok, t4, nt, acc);
+        if (a.trace && ctid == 0) {
+            const uint64_t dw = globaltimer_ns() - tw;
+            if (i == 0) S.first_wait_ns = dw;
+            S.total_wait_ns += dw;
+        }
+        if (ok) {
+            const uint8_t* stage = ring + (size_t)slot_s * stage_bytes;
+            const int g0 = i * a.sb;
+            const int nb = min(a.sb, G - g0);
+#pragma unroll 2
+            for (int bb = half; bb < nb; bb += 2) {
+                const int g = g0 + bb;
+                const uint8_t* bp = stage + bb * kBlockBytes;
+                const uint4 w = *reinterpret_cast<const uint4*>(bp + sub * 512 + lane * 16);
+                const uint32_t sv = *reinterpret_cast<const uint32_t*>(bp + kNibbleBytes + sub * 32 + gi * 4);
+                uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
+                if (has_b) {
+                    x0 = xb[(size_t)(g * 2 + 0) * L + lane];
+                    x1 = xb[(size_t)(g * 2 + 1) * L + lane];
+                }
+                group_mma_aw(w, sv, x0, x1, acc0, acc1);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[slot_s]);
         if (++slot_s == (uint32_t)a.nstages) { slot_s = 0; phase_s ^= 1; }
     }
-    // odd-group warps hand their partial sums to the even-group warps
+    // odd-block warps hand their partial sums to the even-block warps
     if (half == 1) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) S.red[(sub * 32 + lane) * 4 + j] = acc[j];
+        S.red[(sub * 32 + lane) * 2 + 0] = acc0;
+        S.red[(sub * 32 + lane) * 2 + 1] = acc1;
     }
     named_bar(1, kCT);
-    if (half == 0 && tok < nt && !*abort_flag) {
-        const float xs = S.xscale[tok];
-        float v[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = (acc[j] + S.red[(sub * 32 + lane) * 4 + j]) * xs;
+    if (half == 0 && t4 < nt && !*abort_flag) {
+        const float xs = S.xscale[t4];
+        const float v0 = (acc0 + S.red[(sub * 32 + lane) * 2 + 0]) * xs;  // row gi of the sub-tile
+        const float v1 = (acc1 + S.red[(sub * 32 + lane) * 2 + 1]) * xs;  // row gi+8
         if (gu) {
-            // rows 2t, 2t+1 of the sub-tile are gate rows j, j+1; rows 8+2t, 9+2t the matching up rows
-            const int j = (it.rt * 8 + sub) * 8 + 2 * t4;
-            float2 hv = make_float2(silu_f(v[0]) * v[2], silu_f(v[1]) * v[3]);
-            *reinterpret_cast<float2*>(a.h + (size_t)(it.off + tok) * d.I + j) = hv;
+            // row gi is gate row j, row gi+8 the up row j of the same j
+            const int j = (it.rt * 8 + sub) * 8 + gi;
+            a.h[(size_t)(it.off + t4) * d.I + j] = silu_f(v0) * v1;
         } else {
-            const int r0 = it.rt * kTileRows + sub * kSubRows + 2 * t4;
-            float* orow = a.o + (size_t)(it.off + tok) * d.H;
-            *reinterpret_cast<float2*>(orow + r0) = make_float2(v[0], v[1]);
-            *reinterpret_cast<float2*>(orow + r0 + 8) = make_float2(v[2], v[3]);
+            const int r0 = it.rt * kTileRows + sub * kSubRows + gi;
+            a.o[(size_t)(it.off + t4) * d.H + r0] = v0;
+            a.o[(size_t)(it.off + t4) * d.H + r0 + 8] = v1;
         }
     }
     named_bar(1, kCT);
@@ -452,7 +473,7 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
     }
     named_bar(1, kCT);
     if (!S.sflag || *abort_flag) return;
-    const int K = d.K, TK = T * d.K;
+    const int T = a.T, K = d.K, TK = T * d.K;
     for (int idx = ctid; idx < T * kTileRows; idx += kCT) {
         const int t = idx / kTileRows, r = it.rt * kTileRows + (idx % kTileRows);
         float acc = a.residual ? a.residual[(size_t)t * d.H + r] : 0.0f;
@@ -472,8 +493,8 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     FusedSmem& S = *reinterpret_cast<FusedSmem*>(smem);
     uint8_t* ring = smem + ((sizeof(FusedSmem) + 127) & ~(size_t)127);
-    uint4* xa = reinterpret_cast<uint4*>(ring + (size_t)a.nstages * kStage);
-    int* scnt = reinterpret_cast<int*>(xa + (size_t)NT * (a.d.H > a.d.I ? a.d.H : a.d.I) / 4);
+    uint4* xb = reinterpret_cast<uint4*>(ring + (size_t)a.nstages * a.sb * kBlockBytes);
+    int* scnt = reinterpret_cast<int*>(xb + (size_t)NT * (a.d.H > a.d.I ? a.d.H : a.d.I) / 4);
     int* soff = scnt + a.d.E + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -502,21 +523,25 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
             named_bar(1, kCT);
             const Item it = S.cur[q & 1];
             const uint64_t t_begin = (a.trace && ctid == 0) ? globaltimer_ns() : 0;
-            if (ctid == 0) S.first_wait_ns = 0;
+            if (ctid == 0) S.first_wait_ns = S.total_wait_ns = 0;
             if (it.kind == IT_ROUTER) router_item<XT, NT>(a, S, it.ex, ctid);
             else if (it.kind == IT_PLAN) plan_item(a, S, ctid, scnt, soff);
             else if (it.kind == IT_GU || it.kind == IT_DOWN)
-                weight_item<XT, NT>(a, S, it, ring, xa, slot_s, phase_s, ctid);
+                weight_item<XT, NT>(a, S, it, ring, xb, slot_s, phase_s, ctid);
             named_bar(1, kCT);
             if (a.trace && ctid == 0 && it.kind != IT_END) {
-                // record: (cta << 40 | kind << 32 | ex << 16 | rt), begin, end, first-data wait
+                // record: (cta << 40 | kind << 32 | ex << 16 | rt), begin, end, first-data wait,
+                // pushed by the producer, total weight-stage wait of warp 0
                 const unsigned long long r = atomicAdd(reinterpret_cast<unsigned long long*>(a.trace), 1ull);
                 if (r < (unsigned long long)a.trace_cap) {
-                    long long* rec = a.trace + 4 + 4 * r;
+                    long long* rec = a.trace + 8 + 8 * r;
                     rec[0] = ((long long)blockIdx.x << 40) | ((long long)it.kind << 32) | ((long long)it.ex << 16) | it.rt;
                     rec[1] = (long long)t_begin;
                     rec[2] = (long long)globaltimer_ns();
                     rec[3] = (long long)S.first_wait_ns;
+                    rec[4] = it.pushed_ns;
+                    rec[5] = (long long)S.total_wait_ns;
+                    rec[6] = rec[7] = 0;
                 }
             }
             if (ctid == 0 && it.kind != IT_END) mbar_arrive(&S.qempty[slot]);
@@ -537,10 +562,26 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
     }
 }
 
-size_t fused_smem_bytes(const Dims& d, int NT, int nstages) {
+size_t fused_smem_bytes(const Dims& d, int NT, int nstages, int sb) {
     const size_t head = (sizeof(FusedSmem) + 127) & ~(size_t)127;
     const int C = d.H > d.I ? d.H : d.I;
-    return head + (size_t)nstages * kStage + (size_t)NT * C * 4 + (size_t)(2 * d.E + 2) * 4;
+    return head + (size_t)nstages * sb * kBlockBytes + (size_t)NT * C * 4 + (size_t)(2 * d.E + 2) * 4;
+}
+
+// Ring geometry for NT tokens: the largest copies (up to 8 blocks = 34,816 B;
+// bulk copies of that size stream best) with at least 4 stages in flight.
+static bool fused_geometry(const Dims& d, int NT, size_t smem_limit, int* nstages, int* sb) {
+    for (int b = kMaxSB; b >= 2; b -= 2) {
+        int ns = kMaxStages;
+        while (ns > 0 && fused_smem_bytes(d, NT, ns, b) > smem_limit) --ns;
+        if (ns >= 4) { *nstages = ns; *sb = b; return true; }
+    }
+    return false;
+}
+
+int fused_stages_for(const Dims& d, int NT, size_t smem_limit) {
+    int ns = 0, sb = 0;
+    return fused_geometry(d, NT, smem_limit, &ns, &sb) ? ns : 0;
 }
 
 template <typename XT, int NT>
@@ -554,15 +595,9 @@ static cudaError_t launch_fused_t(const FusedArgs& a, int n_sm, size_t smem_limi
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    const size_t smem = fused_smem_bytes(a.d, NT, a.nstages);
+    const size_t smem = fused_smem_bytes(a.d, NT, a.nstages, a.sb);
     moe_decode_fused_kernel<XT, NT><<<n_sm, kFT, smem, st>>>(a);
     return cudaGetLastError();
-}
-
-int fused_stages_for(const Dims& d, int NT, size_t smem_limit) {
-    int ns = kMaxStages;
-    while (ns > 2 && fused_smem_bytes(d, NT, ns) > smem_limit) --ns;
-    return fused_smem_bytes(d, NT, ns) <= smem_limit ? ns : 0;
 }
 
 cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const float* wr, const float* bias,
@@ -576,8 +611,7 @@ cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const flo
     a.T = T; a.p = p; a.logits = logits; a.h = h; a.o = o; a.ctl = ctl;
     a.trace = trace; a.trace_cap = trace_cap;
     a.umax = T * d.K < d.E ? T * d.K : d.E;
-    a.nstages = fused_stages_for(d, NT, smem_limit);
-    if (a.nstages < 2) return cudaErrorInvalidConfiguration;
+    if (!fused_geometry(d, NT, smem_limit, &a.nstages, &a.sb)) return cudaErrorInvalidConfiguration;
     if (dt == COLI_F32) {
         if (NT == 1) return launch_fused_t<float, 1>(a, n_sm, smem_limit, st);
         if (NT == 2) return launch_fused_t<float, 2>(a, n_sm, smem_limit, st);

@@ -82,6 +82,33 @@ __device__ __forceinline__ void group_mma(uint4 w, uint2 sc, const uint4* __rest
     acc[3] = fmaf(s23.y, d1[1] + d1[3], acc[3]);
 }
 
+// Weights as the A operand (16 rows x 16 inputs per mma), tokens as B: column
+// n = 2j + p of B is part p (0 hi, 1 lo) of token j, so one instruction covers
+// 256 weights for up to 4 tokens. The word's four dequantised pairs are
+// exactly A fragments a0 (row gi, k lo), a1 (row gi+8, k lo), a2 (row gi,
+// k hi), a3 (row gi+8, k hi).
+// w: this lane's 16 bytes of the group; sv: fp16 scales (row gi, row gi+8);
+// xb0/xb1: the lane's B fragments for steps 0,1 and 2,3 of the group.
+// acc0/acc1: token t = lane % 4, rows gi and gi+8 (valid for t < tokens).
+__device__ __forceinline__ void group_mma_aw(uint4 w, uint32_t sv, uint4 xb0, uint4 xb1, float& acc0, float& acc1) {
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t bx[8] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w};
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        uint32_t r0, r1, r8, r9;  // (row gi, k lo), (row gi, k hi), (row gi+8, k lo), (row gi+8, k hi)
+        dequant_word_f16(words[s], r0, r1, r8, r9);
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(r0), "r"(r8), "r"(r1), "r"(r9), "r"(bx[2 * s]), "r"(bx[2 * s + 1]));
+    }
+    const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sv));
+    acc0 = fmaf(sc.x, d[0] + d[1], acc0);  // row gi: hi + lo columns of token t
+    acc1 = fmaf(sc.y, d[2] + d[3], acc1);  // row gi+8
+}
+
 // 2^k as a float for k in [-126, 127].
 __device__ __forceinline__ float exp2i(int k) { return __uint_as_float((uint32_t)(127 + k) << 23); }
 
@@ -152,6 +179,67 @@ __device__ __forceinline__ void stage_afrag(uint4* __restrict__ xa, float* scale
         o.x = split_pair(v0, v1, o.y);
         o.z = split_pair(v8, v9, o.w);
         xa[((g * 4 + s) * NT + tok) * 4 + t] = o;
+    }
+}
+
+// Stage nt (<= NT) rows as B fragments for group_mma_aw, per-row power-of-two
+// scaling and fp16 hi + lo split as in stage_afrag. Entry
+//   xb[(g*2 + h)*8*NT + lane], lane < 8*NT: column n = lane/4 (token n/2, part
+//   n%2), t = lane%4, steps s = 2h, 2h+1: {b0(s), b1(s), b0(s+1), b1(s+1)},
+//   b0(s) = pair (k, k+1), b1(s) = pair (k+8, k+9), k = 64g + 16s + 2t.
+// Columns of tokens >= nt hold zeros.
+template <typename XT, int NT>
+__device__ __forceinline__ void stage_bfrag(uint4* __restrict__ xb, float* scale_out, const XT* __restrict__ in,
+                                            const int* rows, int nt, int C, bool coherent, int tid, int nthr,
+                                            int bar, float* red) {
+    const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
+    float m[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        m[j] = 0.0f;
+        if (j < nt) {
+            const XT* r = in + (size_t)rows[j] * C;
+            for (int c = tid; c < C; c += nthr) m[j] = fmaxf(m[j], fabsf(load_in<XT>(r + c, coherent)));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], o));
+        if (lane == 0) red[warp * NT + j] = m[j];
+    }
+    named_bar(bar, nthr);
+    if (tid < NT) {
+        float mx = 0.0f;
+        for (int w = 0; w < nw; ++w) mx = fmaxf(mx, red[w * NT + tid]);
+        int k = 0;
+        const uint32_t eb = (__float_as_uint(mx) >> 23) & 0xFF;
+        if (eb != 0 && eb != 0xFF) {
+            k = 14 - ((int)eb - 127);
+            k = k < -126 ? -126 : (k > 126 ? 126 : k);
+        }
+        red[nw * NT + tid] = exp2i(k);
+        scale_out[tid] = exp2i(-k);
+    }
+    named_bar(bar, nthr);
+    const int G = C / kGroup, L = 8 * NT;
+    for (int idx = tid; idx < G * 2 * L; idx += nthr) {
+        const int l = idx % L, gh = idx / L;
+        const int g = gh >> 1, h = gh & 1;
+        const int n = l >> 2, t = l & 3, j = n >> 1, part = n & 1;
+        uint4 o = make_uint4(0u, 0u, 0u, 0u);
+        if (j < nt) {
+            const XT* src = in + (size_t)rows[j] * C;
+            const float f = red[nw * NT + j];
+            uint32_t outw[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {  // q: (s = 2h + q/2, which = q%2 -> k offset 0 or 8)
+                const int s = 2 * h + (q >> 1);
+                const int k = g * 64 + s * 16 + 2 * t + ((q & 1) ? 8 : 0);
+                uint32_t lo;
+                const uint32_t hi = split_pair(load_in<XT>(src + k, coherent) * f, load_in<XT>(src + k + 1, coherent) * f, lo);
+                outw[q] = part ? lo : hi;
+            }
+            o = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+        }
+        xb[(size_t)gh * L + l] = o;
     }
 }
 
