@@ -32,13 +32,13 @@
 
 namespace coli {
 
-constexpr int kCW = 16;                      // consumer warps
+constexpr int kCW = 8;                       // consumer warps (one 16-row sub-tile each)
 constexpr int kCT = kCW * 32;                // consumer threads
 constexpr int kFT = kCT + 32;                // + the producer warp
 constexpr int kMaxSB = 8;                    // 4352-byte blocks per ring stage (at most)
 constexpr int kQ = 2;                        // item queue slots (lookahead of one item)
 constexpr uint64_t kWaitNs = 1000000000ull;  // every wait gives up after 1 s
-constexpr int kRouterExperts = 2;            // experts per router item (8 warps each)
+constexpr int kRouterExperts = 2;            // experts per router item (4 warps each)
 
 enum { IT_END = 0, IT_ROUTER = 1, IT_PLAN = 2, IT_GU = 3, IT_DOWN = 4 };
 
@@ -82,7 +82,6 @@ struct FusedSmem {
     float mred[(kCW + 1) * kFusedMaxTok];
     double rpart[kCW][kFusedMaxTok];
     int sids[kFusedMaxTok * 32];
-    float red[8 * 32 * 2];
 };
 
 __device__ __forceinline__ void set_error(FusedArgs& a, volatile int* abort_flag, int code) {
@@ -199,52 +198,61 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
 }
 
 // ------------------------------------------------------------------ consumers
-// Router rows e0, e0+1: warps 8r..8r+7 take expert e0 + r, each an eighth of
-// H, loads issued before the fp64 products; fixed-order reduction.
+// Router rows e0, e0+1: warps 4r..4r+3 take expert e0 + r, each a quarter of
+// H, with the weight loads issued before the fp64 products; the four partial
+// sums are added in a fixed order.
 template <typename XT, int NT>
 __device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
     const Dims& d = a.d;
     const int cw = ctid >> 5, lane = ctid & 31;
-    const int r = cw >> 3, part = cw & 7;
+    constexpr int kParts = kCW / kRouterExperts;
+    const int r = cw / kParts, part = cw % kParts;
     const int e = e0 + r;
-    const int chunk = d.H / 8;
+    const int chunk = d.H / kParts;
     const XT* x = reinterpret_cast<const XT*>(a.x);
     double acc[NT];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t] = 0.0;
     if (e < d.E) {
         const float* wrow = a.wr + (size_t)e * d.H + part * chunk;
-        for (int base = 0; base < chunk; base += 1024) {
-            float4 wv[8];
+        constexpr int kV = 6;  // float4 per lane per pass (weights then each token's x)
+        for (int base = 0; base < chunk; base += kV * 128) {
+            float4 wv[kV];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < kV; ++j) {
                 const int i = base + lane * 4 + j * 128;
                 wv[j] = i < chunk ? __ldg(reinterpret_cast<const float4*>(wrow + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
+#pragma unroll 1
+            for (int t = 0; t < a.T; ++t) {
+                const XT* xr = x + (size_t)t * d.H + part * chunk;
+                double xv[kV][4];
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                if (t < a.T) {
-                    const XT* xr = x + (size_t)t * d.H + part * chunk;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int i = base + lane * 4 + j * 128;
-                        if (i < chunk) {
-                            double x0, x1, x2, x3;
-                            if constexpr (sizeof(XT) == 4) {
-                                const float4 v = __ldg(reinterpret_cast<const float4*>(xr + i));
-                                x0 = v.x; x1 = v.y; x2 = v.z; x3 = v.w;
-                            } else {
-                                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr + i));
-                                x0 = __uint_as_float(u.x << 16); x1 = __uint_as_float(u.x & 0xFFFF0000u);
-                                x2 = __uint_as_float(u.y << 16); x3 = __uint_as_float(u.y & 0xFFFF0000u);
-                            }
-                            acc[t] = fma((double)wv[j].x, x0, acc[t]);
-                            acc[t] = fma((double)wv[j].y, x1, acc[t]);
-                            acc[t] = fma((double)wv[j].z, x2, acc[t]);
-                            acc[t] = fma((double)wv[j].w, x3, acc[t]);
+                for (int j = 0; j < kV; ++j) {
+                    const int i = base + lane * 4 + j * 128;
+                    xv[j][0] = xv[j][1] = xv[j][2] = xv[j][3] = 0.0;
+                    if (i < chunk) {
+                        if constexpr (sizeof(XT) == 4) {
+                            const float4 v = __ldg(reinterpret_cast<const float4*>(xr + i));
+                            xv[j][0] = v.x; xv[j][1] = v.y; xv[j][2] = v.z; xv[j][3] = v.w;
+                        } else {
+                            const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr + i));
+                            xv[j][0] = __uint_as_float(u.x << 16); xv[j][1] = __uint_as_float(u.x & 0xFFFF0000u);
+                            xv[j][2] = __uint_as_float(u.y << 16); xv[j][3] = __uint_as_float(u.y & 0xFFFF0000u);
                         }
                     }
                 }
+                double sacc = 0.0;
+#pragma unroll
+                for (int j = 0; j < kV; ++j) {
+                    sacc = fma((double)wv[j].x, xv[j][0], sacc);
+                    sacc = fma((double)wv[j].y, xv[j][1], sacc);
+                    sacc = fma((double)wv[j].z, xv[j][2], sacc);
+                    sacc = fma((double)wv[j].w, xv[j][3], sacc);
+                }
+#pragma unroll
+                for (int tt = 0; tt < NT; ++tt)
+                    if (tt == t) acc[tt] += sacc;
             }
         }
     }
@@ -259,7 +267,7 @@ __device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
         const int rr = ctid / a.T, t = ctid % a.T, ee = e0 + rr;
         if (ee < d.E) {
             double sum = 0.0;
-            for (int w = 0; w < 8; ++w) sum += S.rpart[rr * 8 + w][t];
+            for (int w = 0; w < kParts; ++w) sum += S.rpart[rr * kParts + w][t];
             a.logits[(size_t)t * d.E + ee] = sum + (double)a.bias[ee];
         }
     }
@@ -396,7 +404,7 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
     }
 
     float acc0 = 0.f, acc1 = 0.f;
-    const int half = cw >> 3, sub = cw & 7;
+    const int sub = cw;
     const uint32_t stage_bytes = (uint32_t)a.sb * kBlockBytes;
     const bool has_b = lane < L;
     const int nst = (G + a.sb - 1) / a.sb;
@@ -414,7 +422,7 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
             const int g0 = i * a.sb;
             const int nb = min(a.sb, G - g0);
 #pragma unroll 2
-            for (int bb = half; bb < nb; bb += 2) {
+            for (int bb = 0; bb < nb; ++bb) {
                 const int g = g0 + bb;
                 const uint8_t* bp = stage + bb * kBlockBytes;
                 const uint4 w = *reinterpret_cast<const uint4*>(bp + sub * 512 + lane * 16);
@@ -431,16 +439,10 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
         if (lane == 0) mbar_arrive(&S.empty[slot_s]);
         if (++slot_s == (uint32_t)a.nstages) { slot_s = 0; phase_s ^= 1; }
     }
-    // odd-block warps hand their partial sums to the even-block warps
-    if (half == 1) {
-        S.red[(sub * 32 + lane) * 2 + 0] = acc0;
-        S.red[(sub * 32 + lane) * 2 + 1] = acc1;
-    }
-    named_bar(1, kCT);
-    if (half == 0 && t4 < nt && !*abort_flag) {
+    if (t4 < nt && !*abort_flag) {
         const float xs = S.xscale[t4];
-        const float v0 = (acc0 + S.red[(sub * 32 + lane) * 2 + 0]) * xs;  // row gi of the sub-tile
-        const float v1 = (acc1 + S.red[(sub * 32 + lane) * 2 + 1]) * xs;  // row gi+8
+        const float v0 = acc0 * xs;  // row gi of the sub-tile
+        const float v1 = acc1 * xs;  // row gi+8
         if (gu) {
             // row gi is gate row j, row gi+8 the up row j of the same j
             const int j = (it.rt * 8 + sub) * 8 + gi;
