@@ -47,12 +47,14 @@ constexpr int kBlockBytes = kNibbleBytes + kScaleBytes;  // 4352
 constexpr int kFusedMaxTok = 4;
 constexpr int kMaxStages = 24;
 // Control block (ints in the workspace, zero between launches):
-//   [kCtlTicket] work ticket, [kCtlRouter] finished router rows,
-//   [kCtlPlan] plan published, [kCtlExit] CTAs done, [kCtlError] timeout code,
+//   [kCtlTicket] work ticket, [kCtlRouter] finished router items,
+//   [kCtlPlan] 0, or 1 + number of distinct routed experts once the plan is
+//   published, [kCtlExit] CTAs done, [kCtlError] timeout code,
 //   [kCtlGuDone + e] finished gate/up tiles of expert e (E + S entries),
-//   then [kCtlGuDone + E + S + rt] finished down tiles of output block rt.
+//   [kCtlGuDone + E + S + rt] finished down tiles of output block rt (H/128),
+//   then kFusedMaxTok * (K + S) float bit patterns: max |h| of each position.
 enum { kCtlTicket = 0, kCtlRouter = 1, kCtlPlan = 2, kCtlExit = 3, kCtlError = 4, kCtlGuDone = 8 };
-inline int ctl_ints(int E, int S, int H) { return kCtlGuDone + E + S + H / 128; }
+__host__ __device__ inline int ctl_ints(int E, int S, int H, int K) { return kCtlGuDone + E + S + H / 128 + kFusedMaxTok * (K + S); }
 
 inline int64_t matrix_bytes(int rows, int cols) {
     return (int64_t)(rows / kTileRows) * (cols / kGroup) * kBlockBytes;
@@ -79,6 +81,8 @@ struct Plan {
     int32_t* act_off;    // [E+S] first permuted position of active expert a
     int32_t* act_cnt;    // [E+S] tokens of active expert a
     int32_t* n_active;   // [1] n_unique + S
+    int4* table;         // [E] per distinct expert u (ascending): {expert, first position, tokens,
+                         //     tokens packed 8 bits each when <= 4} (persistent decode kernel)
 };
 
 // ---------------------------------------------------------------------------

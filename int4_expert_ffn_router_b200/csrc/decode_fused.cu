@@ -5,26 +5,25 @@
 // Decode streams each active expert's ~20 MB once ("Colibri: 2400 lines of
 // pure C ...", kechuai.cn, section 二: one read per unique expert per batch,
 // the three matrices adjacent), so the kernel is HBM-bound: it must keep
-// enough bytes in flight and never leave the memory system idle between the
-// dependent steps. Design:
-//  * one CTA per SM; a producer warp streams weight tiles into a shared-memory
-//    ring with bulk asynchronous copies (the TMA engine) completing on
-//    mbarriers; 16 consumer warps dequantise and multiply out of the ring on
-//    the tensor cores from registers (int4_mma.cuh): the CUDA-core budget per
-//    streamed weight, not the tensor pipe, is what limits a decode GEMV;
-//  * work items are handed out by a global ticket counter in dependency
-//    order: router rows, the plan, shared-expert gate/up, shared-expert down,
-//    routed gate/up, routed down. An item only waits for items with smaller
-//    tickets, which running CTAs already hold, so the schedule cannot
-//    deadlock; every wait is bounded in time and reports a timeout through
-//    the control block instead of hanging;
-//  * the producer prefetches an item's weights before its inputs are ready
-//    (routed experts only need the plan, down tiles only the gate/up of the
-//    same expert), so weight streaming overlaps the top-k, the plan and the
-//    gate/up -> down dependency;
-//  * the last down tile of each 128-row output block to finish combines
-//    that block of y in a fixed order (shared experts, then the routed ones
-//    in routing order), so no extra pass and no atomics on y.
+// enough bytes in flight and keep global-memory round trips (about 1-2 us
+// each while HBM is saturated) off the path of the warps that do the math.
+// One CTA per SM, three warp roles:
+//  * a producer warp takes work tickets and streams each item's weight tile
+//    into a shared-memory ring with bulk asynchronous copies (the TMA engine)
+//    of up to 34,816 bytes, completing on mbarriers;
+//  * eight consumer warps (one 16-row sub-tile each) dequantise int4 to
+//    exact fp16 and multiply on the tensor cores from registers
+//    (int4_mma.cuh): for a decode GEMV the CUDA-core instruction budget per
+//    streamed weight, not the tensor pipe, is the limit;
+//  * a signaler warp publishes completions (release atomics), builds the
+//    top-k and the batch-union plan when the last router item lands, and
+//    combines each 128-row block of y when its last down tile lands, so the
+//    consumers never wait on a global round trip to hand work off.
+// Tickets are handed out in dependency order: router rows, shared-expert
+// gate/up, shared-expert down, routed gate/up, routed down. An item only
+// waits for items with smaller tickets, which running CTAs already hold, so
+// the schedule cannot deadlock; every wait is bounded in time and reports a
+// timeout through the control block instead of hanging.
 #include "common.cuh"
 #include "int4_mma.cuh"
 #include "kernels.cuh"
@@ -34,17 +33,23 @@ namespace coli {
 
 constexpr int kCW = 8;                       // consumer warps (one 16-row sub-tile each)
 constexpr int kCT = kCW * 32;                // consumer threads
-constexpr int kFT = kCT + 32;                // + the producer warp
+constexpr int kProducerWarp = kCW;
+constexpr int kSignalWarp = kCW + 1;
+constexpr int kFT = (kCW + 2) * 32;          // all threads
 constexpr int kMaxSB = 8;                    // 4352-byte blocks per ring stage (at most)
 constexpr int kQ = 2;                        // item queue slots (lookahead of one item)
+constexpr int kSQ = 4;                       // completion records in flight to the signaler
 constexpr uint64_t kWaitNs = 1000000000ull;  // every wait gives up after 1 s
 constexpr int kRouterExperts = 2;            // experts per router item (4 warps each)
 
-enum { IT_END = 0, IT_ROUTER = 1, IT_PLAN = 2, IT_GU = 3, IT_DOWN = 4 };
+enum { IT_END = 0, IT_ROUTER = 1, IT_GU = 2, IT_DOWN = 3 };
 
 struct Item {
-    int kind, ex, rt, off, cnt, shared;
-    long long pushed_ns;  // trace only: when the producer published the item
+    int kind, ex, rt, off, cnt;
+    int tokens;  // gate/up: token ids, 8 bits each, ascending
+    int ready;   // down: gate/up of `ex` already complete when published
+    int pad;
+    long long pushed_ns;  // trace only
 };
 
 struct FusedArgs {
@@ -63,26 +68,39 @@ struct FusedArgs {
     int* ctl;
     int umax;     // min(T*K, E): upper bound of distinct routed experts
     int nstages;  // ring stages
-    int sb;       // 4352-byte blocks per stage (even); the bulk copies are sb * 4352 bytes
-    long long* trace;  // item timeline (NULL: off); [0] = records written
-    int trace_cap;     // records of 4 x int64 after the header
+    int sb;       // 4352-byte blocks per stage; the bulk copies are sb * 4352 bytes
+    long long* trace;  // item timeline (NULL: off)
+    int trace_cap;
 };
 
-// Shared-memory layout (dynamic).
 struct FusedSmem {
-    uint64_t full[kMaxStages], empty[kMaxStages], qfull[kQ], qempty[kQ];
+    uint64_t full[kMaxStages], empty[kMaxStages], qfull[kQ], qempty[kQ], dfull[kSQ], dempty[kSQ];
     Item items[kQ];
-    int abort_flag;
     Item cur[2];
+    Item done[kSQ];
+    int abort_flag;
     int staged_n, staged_rows[kFusedMaxTok];
-    int srow[kFusedMaxTok];
-    int sflag;
-    unsigned long long first_wait_ns, total_wait_ns;
     float xscale[kFusedMaxTok];
     float mred[(kCW + 1) * kFusedMaxTok];
     double rpart[kCW][kFusedMaxTok];
     int sids[kFusedMaxTok * 32];
+    unsigned long long first_wait_ns, total_wait_ns;
 };
+
+// ------------------------------------------------------------- small helpers
+__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void red_add_release(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_max_u32(unsigned* p, unsigned v) {
+    asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 __device__ __forceinline__ void set_error(FusedArgs& a, volatile int* abort_flag, int code) {
     *abort_flag = 1;
@@ -119,6 +137,12 @@ __device__ __forceinline__ bool wait_geq(const int* p, int target, volatile int*
     }
 }
 
+// Running max |h| of each position (float bits; non-negative floats order as
+// unsigned integers), after the tile counters in the control block.
+__device__ __forceinline__ unsigned* hmax_of(FusedArgs& a) {
+    return reinterpret_cast<unsigned*>(a.ctl + kCtlGuDone + a.d.E + a.d.S + a.d.H / kTileRows);
+}
+
 // ------------------------------------------------------------------ producer
 __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
     const Dims& d = a.d;
@@ -126,38 +150,40 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
     const int RTgu = 2 * d.I / kTileRows, RTd = d.H / kTileRows;
     const int Ggu = d.H / kGroup, Gd = d.I / kGroup;
     const int n_router = (d.E + kRouterExperts - 1) / kRouterExperts;
-    const int t_plan = n_router, t_sg = t_plan + 1, t_sd = t_sg + d.S * RTgu, t_ug = t_sd + d.S * RTd;
+    const int t_sg = n_router, t_sd = t_sg + d.S * RTgu, t_ug = t_sd + d.S * RTd;
     const int t_ud = t_ug + a.umax * RTgu, t_end = t_ud + a.umax * RTd;
+    int all_tokens = 0;
+    for (int t = 0; t < T; ++t) all_tokens |= t << (8 * t);
     volatile int* abort_flag = &S.abort_flag;
     int n_unique = -1;
     uint32_t q = 0, gs = 0, slot_s = 0, phase_s = 0;
     while (true) {
-        Item it{IT_END, 0, 0, 0, 0, 0, 0};
+        Item it{IT_END, 0, 0, 0, 0, 0, 0, 0, 0};
         if (!*abort_flag) {
             const int t = atomicAdd(&a.ctl[kCtlTicket], 1);
-            if (t < t_plan) {
-                it = Item{IT_ROUTER, t * kRouterExperts, 0, 0, 0, 0, 0};
-            } else if (t == t_plan) {
-                it = Item{IT_PLAN, 0, 0, 0, 0, 0, 0};
+            if (t < t_sg) {
+                it.kind = IT_ROUTER;
+                it.ex = t * kRouterExperts;
             } else if (t < t_sd) {
-                const int j = (t - t_sg) / RTgu, rt = (t - t_sg) % RTgu;
-                it = Item{IT_GU, d.E + j, rt, T * d.K + j * T, T, 1, 0};
+                const int j = (t - t_sg) / RTgu;
+                it = Item{IT_GU, d.E + j, (t - t_sg) % RTgu, T * d.K + j * T, T, all_tokens, 0, 0, 0};
             } else if (t < t_ug) {
-                const int j = (t - t_sd) / RTd, rt = (t - t_sd) % RTd;
-                it = Item{IT_DOWN, d.E + j, rt, T * d.K + j * T, T, 1, 0};
+                const int j = (t - t_sd) / RTd;
+                it = Item{IT_DOWN, d.E + j, (t - t_sd) % RTd, T * d.K + j * T, T, 0, 0, 0, 0};
             } else if (t < t_end) {
                 if (n_unique < 0) {
                     if (!wait_geq(&a.ctl[kCtlPlan], 1, abort_flag, a, 2)) continue;
-                    n_unique = __ldcg(a.p.n_unique);
+                    n_unique = ld_acquire(&a.ctl[kCtlPlan]) - 1;
                 }
                 const bool gu = t < t_ud;
                 const int r = gu ? t - t_ug : t - t_ud;
                 const int RT = gu ? RTgu : RTd;
-                const int u = r / RT, rt = r % RT;
+                const int u = r / RT;
                 if (u >= n_unique) continue;  // fewer distinct experts than the bound
-                const int ex = __ldcg(a.p.unique + u);
-                it = Item{gu ? IT_GU : IT_DOWN, ex, rt, __ldcg(a.p.off + ex), __ldcg(a.p.cnt + ex), 0, 0};
+                const int4 ent = __ldcg(a.p.table + u);
+                it = Item{gu ? IT_GU : IT_DOWN, ent.x, r % RT, ent.y, ent.z, ent.w, 0, 0, 0};
             }
+            if (it.kind == IT_DOWN) it.ready = ld_acquire(&a.ctl[kCtlGuDone + it.ex]) >= RTgu;
         }
         const uint32_t slot = q % kQ;
         if (q >= kQ && !wait_bar(&S.qempty[slot], ((q / kQ) - 1) & 1, abort_flag, a, 3)) it.kind = IT_END;
@@ -172,14 +198,10 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
             const uint8_t* tile = a.weights + (size_t)it.ex * d.expert_stride + (gu ? 0 : d.gu_bytes) +
                                   (size_t)it.rt * G * kBlockBytes;
             const uint32_t stage_bytes = (uint32_t)a.sb * kBlockBytes;
-            bool stop = false;
-            for (int b0 = 0; b0 < G && !stop; b0 += a.sb) {
+            for (int b0 = 0; b0 < G; b0 += a.sb) {
                 const int nb = min(a.sb, G - b0);
                 // slot_s = gs % nstages, phase_s = (gs / nstages) & 1
-                if (gs >= (uint32_t)a.nstages && !wait_bar(&S.empty[slot_s], phase_s ^ 1, abort_flag, a, 4)) {
-                    stop = true;
-                    break;
-                }
+                if (gs >= (uint32_t)a.nstages && !wait_bar(&S.empty[slot_s], phase_s ^ 1, abort_flag, a, 4)) break;
                 mbar_arrive_expect_tx(&S.full[slot_s], nb * kBlockBytes);
                 bulk_g2s(ring + (size_t)slot_s * stage_bytes, tile + (size_t)b0 * kBlockBytes, nb * kBlockBytes,
                          &S.full[slot_s]);
@@ -194,6 +216,145 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&S.full[k % ns], (k / ns) & 1) && globaltimer_ns() - t0 < kWaitNs) {
         }
+    }
+}
+
+// ------------------------------------------------------------------ signaler
+// Top-k of the T tokens and the batch-union plan, by the signaler warp of the
+// CTA that finished the last router item.
+__device__ void signal_plan(FusedArgs& a, FusedSmem& S, int lane, int* scnt, int* soff, int* stok) {
+    const Dims& d = a.d;
+    const int T = a.T, E = d.E, K = d.K;
+    for (int t = 0; t < T; ++t) {
+        int id;
+        float wt;
+        if (E <= 256) warp_topk<true, 8>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
+        else warp_topk<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
+        if (lane < K) {
+            a.p.ids[t * K + lane] = id;
+            a.p.w[t * K + lane] = wt;
+            S.sids[t * K + lane] = id;
+        }
+    }
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) { scnt[e] = 0; stok[e] = 0; }
+    __syncwarp();
+    for (int t = 0; t < T; ++t) {  // ids of one token are distinct: lane k owns slot k
+        if (lane < K) {
+            const int e = S.sids[t * K + lane];
+            stok[e] |= t << (8 * scnt[e]);
+            scnt[e] += 1;
+        }
+        __syncwarp();
+    }
+    // counts, offsets (exclusive scan) and the distinct experts, 32 at a time
+    int carry = 0, ucarry = 0;
+    for (int c0 = 0; c0 < E; c0 += 32) {
+        const int e = c0 + lane;
+        const int c = e < E ? scnt[e] : 0;
+        const int f = c > 0;
+        int incl = c, fincl = f;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n1 = __shfl_up_sync(0xffffffffu, incl, o), n2 = __shfl_up_sync(0xffffffffu, fincl, o);
+            if (lane >= o) { incl += n1; fincl += n2; }
+        }
+        const int off = carry + incl - c, rank = ucarry + fincl - f;
+        if (e < E) {
+            soff[e] = off;
+            a.p.off[e] = off;
+            a.p.cnt[e] = c;
+            if (f) {
+                a.p.unique[rank] = e;
+                a.p.act_expert[rank] = e;
+                a.p.act_off[rank] = off;
+                a.p.act_cnt[rank] = c;
+                a.p.table[rank] = make_int4(e, off, c, stok[e]);
+            }
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+        ucarry += __shfl_sync(0xffffffffu, fincl, 31);
+    }
+    const int n_unique = ucarry;
+    if (lane == 0) {
+        a.p.off[E] = carry;
+        *a.p.n_unique = n_unique;
+        *a.p.n_active = n_unique + d.S;
+    }
+    for (int j = lane; j < d.S; j += 32) {
+        a.p.act_expert[n_unique + j] = E + j;
+        a.p.act_off[n_unique + j] = T * K + j * T;
+        a.p.act_cnt[n_unique + j] = T;
+    }
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) scnt[e] = 0;
+    __syncwarp();
+    for (int t = 0; t < T; ++t) {
+        if (lane < K) {
+            const int e = S.sids[t * K + lane];
+            const int q = soff[e] + scnt[e];
+            scnt[e] += 1;
+            a.p.pos[t * K + lane] = q;
+            a.p.tok[q] = t;
+        }
+        __syncwarp();
+    }
+    for (int i = lane; i < d.S * T; i += 32) a.p.tok[T * K + i] = i % T;
+    __syncwarp();
+    if (lane == 0) st_release(&a.ctl[kCtlPlan], n_unique + 1);
+}
+
+// y rows of output block rt: residual + shared experts + routed experts in
+// routing order (fixed order, same as the separate combine kernel).
+template <typename XT>
+__device__ void signal_combine(FusedArgs& a, int rt, int lane) {
+    const Dims& d = a.d;
+    const int T = a.T, K = d.K, TK = T * d.K;
+    for (int idx = lane; idx < T * kTileRows; idx += 32) {
+        const int t = idx / kTileRows, r = rt * kTileRows + (idx % kTileRows);
+        float acc = a.residual ? a.residual[(size_t)t * d.H + r] : 0.0f;
+        for (int j = 0; j < d.S; ++j) acc += __ldcg(a.o + (size_t)(TK + j * T + t) * d.H + r);
+        for (int k = 0; k < K; ++k) {
+            const float wk = __ldcg(a.p.w + t * K + k);
+            const int q = __ldcg(a.p.pos + t * K + k);
+            acc = fmaf(wk, __ldcg(a.o + (size_t)q * d.H + r), acc);
+        }
+        if constexpr (sizeof(XT) == 4) reinterpret_cast<float*>(a.y)[(size_t)t * d.H + r] = acc;
+        else reinterpret_cast<__nv_bfloat16*>(a.y)[(size_t)t * d.H + r] = __float2bfloat16_rn(acc);
+    }
+}
+
+template <typename XT>
+__device__ void fused_signaler(FusedArgs& a, FusedSmem& S, int lane, int* scnt, int* soff, int* stok) {
+    const Dims& d = a.d;
+    const int n_router = (d.E + kRouterExperts - 1) / kRouterExperts;
+    volatile int* abort_flag = &S.abort_flag;
+    for (uint32_t k = 0;; ++k) {
+        const uint32_t slot = k % kSQ;
+        const bool ok = wait_bar(&S.dfull[slot], (k / kSQ) & 1, abort_flag, a, 10);
+        const Item r = S.done[slot];
+        if (!ok || r.kind == IT_END) break;
+        int last = 0;
+        if (lane == 0) {
+            if (r.kind == IT_ROUTER) {
+                last = atom_add_acq_rel(&a.ctl[kCtlRouter], 1) == n_router - 1;
+            } else if (r.kind == IT_GU) {
+                red_add_release(&a.ctl[kCtlGuDone + r.ex], 1);
+            } else {
+                const int prev = atom_add_acq_rel(&a.ctl[kCtlGuDone + d.E + d.S + r.rt], 1);
+                // no output block can be complete before the plan is published,
+                // so an unpublished plan means this was not the last tile
+                const int plan = ld_acquire(&a.ctl[kCtlPlan]);
+                last = plan > 0 && prev + 1 == plan - 1 + d.S;
+            }
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last && !*abort_flag) {
+            if (r.kind == IT_ROUTER) signal_plan(a, S, lane, scnt, soff, stok);
+            else signal_combine<XT>(a, r.rt, lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.dempty[slot]);
     }
 }
 
@@ -215,7 +376,7 @@ __device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
     for (int t = 0; t < NT; ++t) acc[t] = 0.0;
     if (e < d.E) {
         const float* wrow = a.wr + (size_t)e * d.H + part * chunk;
-        constexpr int kV = 6;  // float4 per lane per pass (weights then each token's x)
+        constexpr int kV = 6;  // float4 per lane per pass (weights, then each token's x)
         for (int base = 0; base < chunk; base += kV * 128) {
             float4 wv[kV];
 #pragma unroll
@@ -271,104 +432,46 @@ __device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
             a.logits[(size_t)t * d.E + ee] = sum + (double)a.bias[ee];
         }
     }
-    named_bar(1, kCT);
-    if (ctid == 0) {
-        __threadfence();
-        atomicAdd(&a.ctl[kCtlRouter], 1);
-    }
 }
 
-// Top-k of every token (warp t) and the batch-union plan (warp 0).
-__device__ void plan_item(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* soff) {
-    const Dims& d = a.d;
-    const int T = a.T, E = d.E, K = d.K;
-    const int cw = ctid >> 5, lane = ctid & 31;
-    volatile int* abort_flag = &S.abort_flag;
-    // Control flow below never depends on the abort flag around a barrier:
-    // on abort the work is skipped but every thread meets every barrier.
-    uint64_t tp0 = 0;
-    if (ctid == 0) {
-        tp0 = a.trace ? globaltimer_ns() : 0;
-        wait_geq(&a.ctl[kCtlRouter], (E + kRouterExperts - 1) / kRouterExperts, abort_flag, a, 5);
-        if (a.trace) S.first_wait_ns = globaltimer_ns() - tp0;
+// Stage the h rows of a down item in B-fragment order, scaled by the powers
+// of two that the gate/up items' running maxima select (one pass over h).
+__device__ void stage_h(FusedArgs& a, FusedSmem& S, uint4* xb, const Item& it, int ctid, int NT) {
+    const int C = a.d.I, G = C / kGroup, L = 8 * NT, nt = it.cnt;
+    const unsigned* hm = hmax_of(a);
+    if (ctid < nt) {
+        const float mx = __uint_as_float(__ldcg(hm + it.off + ctid));
+        int k = 0;
+        const uint32_t eb = (__float_as_uint(mx) >> 23) & 0xFF;
+        if (eb != 0 && eb != 0xFF) {
+            k = 14 - ((int)eb - 127);
+            k = k < -126 ? -126 : (k > 126 ? 126 : k);
+        }
+        S.mred[ctid] = exp2i(k);
+        S.xscale[ctid] = exp2i(-k);
     }
     named_bar(1, kCT);
-    if (cw < T && !*abort_flag) {
-        int id;
-        float wt;
-        if (E <= 256) warp_topk<true, 8>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
-        else warp_topk<true>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
-        if (lane < K) {
-            a.p.ids[cw * K + lane] = id;
-            a.p.w[cw * K + lane] = wt;
-            S.sids[cw * K + lane] = id;
-        }
-    }
-    named_bar(1, kCT);
-    if (a.trace && ctid == 0) a.trace[1] = (long long)(globaltimer_ns() - tp0);  // top-k done
-    if (cw == 0 && !*abort_flag) {
-        for (int e = lane; e < E; e += 32) scnt[e] = 0;
-        __syncwarp();
-        for (int t = 0; t < T; ++t) {
-            if (lane < K) scnt[S.sids[t * K + lane]] += 1;  // ids of one token are distinct
-            __syncwarp();
-        }
-        const int per = (E + 31) / 32, b = lane * per, be = min(E, b + per);
-        int sum = 0, fl = 0;
-        for (int e = b; e < be; ++e) { sum += scnt[e]; fl += scnt[e] > 0; }
-        int incl = sum, fincl = fl;
+    for (int idx = ctid; idx < G * 2 * L; idx += kCT) {
+        const int l = idx % L, gh = idx / L;
+        const int g = gh >> 1, hh = gh & 1;
+        const int n = l >> 2, t = l & 3, j = n >> 1, part = n & 1;
+        uint4 o = make_uint4(0u, 0u, 0u, 0u);
+        if (j < nt) {
+            const float* src = a.h + (size_t)(it.off + j) * C;
+            const float f = S.mred[j];
+            uint32_t outw[4];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n1 = __shfl_up_sync(0xffffffffu, incl, o), n2 = __shfl_up_sync(0xffffffffu, fincl, o);
-            if (lane >= o) { incl += n1; fincl += n2; }
-        }
-        const int n_unique = __shfl_sync(0xffffffffu, fincl, 31);
-        int run = incl - sum, ur = fincl - fl;
-        for (int e = b; e < be; ++e) {
-            const int c = scnt[e];
-            soff[e] = run;
-            a.p.off[e] = run;
-            a.p.cnt[e] = c;
-            if (c > 0) {
-                a.p.unique[ur] = e;
-                a.p.act_expert[ur] = e;
-                a.p.act_off[ur] = run;
-                a.p.act_cnt[ur] = c;
-                ++ur;
+            for (int q = 0; q < 4; ++q) {
+                const int s = 2 * hh + (q >> 1);
+                const int kk = g * 64 + s * 16 + 2 * t + ((q & 1) ? 8 : 0);
+                const float2 v = __ldcg(reinterpret_cast<const float2*>(src + kk));
+                uint32_t lo;
+                const uint32_t hi = split_pair(v.x * f, v.y * f, lo);
+                outw[q] = part ? lo : hi;
             }
-            run += c;
+            o = make_uint4(outw[0], outw[1], outw[2], outw[3]);
         }
-        if (lane == 31) a.p.off[E] = run;
-        if (lane == 0) {
-            *a.p.n_unique = n_unique;
-            *a.p.n_active = n_unique + d.S;
-        }
-        for (int j = lane; j < d.S; j += 32) {
-            a.p.act_expert[n_unique + j] = E + j;
-            a.p.act_off[n_unique + j] = T * K + j * T;
-            a.p.act_cnt[n_unique + j] = T;
-        }
-        __syncwarp();
-        for (int e = lane; e < E; e += 32) scnt[e] = 0;
-        __syncwarp();
-        for (int t = 0; t < T; ++t) {
-            if (lane < K) {
-                const int e = S.sids[t * K + lane];
-                const int q = soff[e] + scnt[e];
-                scnt[e] += 1;
-                a.p.pos[t * K + lane] = q;
-                a.p.tok[q] = t;
-            }
-            __syncwarp();
-        }
-        for (int i = lane; i < d.S * T; i += 32) a.p.tok[T * K + i] = i % T;
-    }
-    named_bar(1, kCT);
-    if (ctid == 0) {
-        if (a.trace) a.trace[2] = (long long)(globaltimer_ns() - tp0);  // plan written
-        __threadfence();
-        st_release(&a.ctl[kCtlPlan], 1);
-        if (a.trace) a.trace[3] = (long long)(globaltimer_ns() - tp0);  // published
+        xb[(size_t)gh * L + l] = o;
     }
 }
 
@@ -384,23 +487,28 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
     constexpr int L = 8 * NT;  // lanes holding B-fragment columns of NT tokens
     volatile int* abort_flag = &S.abort_flag;
 
-    // inputs: x rows of the item's tokens (gate/up) or its h rows (down)
-    if (ctid == 0) {
-        if (!gu) wait_geq(&a.ctl[kCtlGuDone + it.ex], 2 * d.I / kTileRows, abort_flag, a, 6);
-        for (int i = 0; i < nt; ++i)
-            S.srow[i] = gu ? (it.shared ? i : __ldcg(a.p.tok + it.off + i)) : it.off + i;
-    }
-    named_bar(1, kCT);
-    bool same = gu && S.staged_n == nt;
-    for (int i = 0; same && i < nt; ++i) same = S.staged_rows[i] == S.srow[i];
-    if (!same) {  // uniform: every consumer reads the same shared values
-        if (gu) stage_bfrag<XT, NT>(xb, S.xscale, reinterpret_cast<const XT*>(a.x), S.srow, nt, C, false, ctid, kCT, 1, S.mred);
-        else stage_bfrag<float, NT>(xb, S.xscale, a.h, S.srow, nt, C, true, ctid, kCT, 1, S.mred);
-    }
-    named_bar(1, kCT);
-    if (ctid == 0) {
-        S.staged_n = gu ? nt : -1;
-        for (int i = 0; i < nt; ++i) S.staged_rows[i] = S.srow[i];
+    if (gu) {
+        bool same = S.staged_n == nt;
+        for (int i = 0; same && i < nt; ++i) same = S.staged_rows[i] == ((it.tokens >> (8 * i)) & 0xFF);
+        if (!same) {  // uniform: every consumer reads the same shared values
+            int rows[NT];
+#pragma unroll
+            for (int i = 0; i < NT; ++i) rows[i] = i < nt ? (it.tokens >> (8 * i)) & 0xFF : 0;
+            named_bar(1, kCT);  // nobody still reads the previous staging
+            stage_bfrag<XT, NT>(xb, S.xscale, reinterpret_cast<const XT*>(a.x), rows, nt, C, false, ctid, kCT, 1,
+                                S.mred);
+            named_bar(1, kCT);
+            if (ctid == 0) {
+                S.staged_n = nt;
+                for (int i = 0; i < nt; ++i) S.staged_rows[i] = rows[i];
+            }
+        }
+    } else {
+        if (ctid == 0 && !it.ready) wait_geq(&a.ctl[kCtlGuDone + it.ex], 2 * d.I / kTileRows, abort_flag, a, 6);
+        named_bar(1, kCT);
+        stage_h(a, S, xb, it, ctid, NT);
+        named_bar(1, kCT);
+        if (ctid == 0) S.staged_n = -1;
     }
 
     float acc0 = 0.f, acc1 = 0.f;
@@ -439,54 +547,29 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
         if (lane == 0) mbar_arrive(&S.empty[slot_s]);
         if (++slot_s == (uint32_t)a.nstages) { slot_s = 0; phase_s ^= 1; }
     }
-    if (t4 < nt && !*abort_flag) {
+    const bool live = t4 < nt && !*abort_flag;
+    float hv = 0.0f;
+    if (live) {
         const float xs = S.xscale[t4];
         const float v0 = acc0 * xs;  // row gi of the sub-tile
         const float v1 = acc1 * xs;  // row gi+8
         if (gu) {
             // row gi is gate row j, row gi+8 the up row j of the same j
             const int j = (it.rt * 8 + sub) * 8 + gi;
-            a.h[(size_t)(it.off + t4) * d.I + j] = silu_f(v0) * v1;
+            hv = silu_f(v0) * v1;
+            a.h[(size_t)(it.off + t4) * d.I + j] = hv;
         } else {
             const int r0 = it.rt * kTileRows + sub * kSubRows + gi;
             a.o[(size_t)(it.off + t4) * d.H + r0] = v0;
             a.o[(size_t)(it.off + t4) * d.H + r0 + 8] = v1;
         }
     }
-    named_bar(1, kCT);
-    if (gu) {
-        if (ctid == 0) {
-            __threadfence();
-            atomicAdd(&a.ctl[kCtlGuDone + it.ex], 1);
-        }
-        return;
-    }
-    // down: the last of the active experts to finish this 128-row block combines it
-    if (ctid == 0) {
-        __threadfence();
-        int last = 0;
-        if (wait_geq(&a.ctl[kCtlPlan], 1, abort_flag, a, 8)) {
-            const int n_active = __ldcg(a.p.n_active);
-            const int prev = atomicAdd(&a.ctl[kCtlGuDone + d.E + d.S + it.rt], 1);
-            last = prev + 1 == n_active;
-            __threadfence();
-        }
-        S.sflag = last;
-    }
-    named_bar(1, kCT);
-    if (!S.sflag || *abort_flag) return;
-    const int T = a.T, K = d.K, TK = T * d.K;
-    for (int idx = ctid; idx < T * kTileRows; idx += kCT) {
-        const int t = idx / kTileRows, r = it.rt * kTileRows + (idx % kTileRows);
-        float acc = a.residual ? a.residual[(size_t)t * d.H + r] : 0.0f;
-        for (int j = 0; j < d.S; ++j) acc += __ldcg(a.o + (size_t)(TK + j * T + t) * d.H + r);
-        for (int k = 0; k < K; ++k) {
-            const float wk = __ldcg(a.p.w + t * K + k);
-            const int q = __ldcg(a.p.pos + t * K + k);
-            acc = fmaf(wk, __ldcg(a.o + (size_t)q * d.H + r), acc);
-        }
-        if constexpr (sizeof(XT) == 4) reinterpret_cast<float*>(a.y)[(size_t)t * d.H + r] = acc;
-        else reinterpret_cast<__nv_bfloat16*>(a.y)[(size_t)t * d.H + r] = __float2bfloat16_rn(acc);
+    if (gu) {  // running max |h| of each position, for the down items' scaling
+        float m = fabsf(hv);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        if (live && gi == 0) red_max_u32(hmax_of(a) + it.off + t4, __float_as_uint(m));
     }
 }
 
@@ -498,22 +581,26 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
     uint4* xb = reinterpret_cast<uint4*>(ring + (size_t)a.nstages * a.sb * kBlockBytes);
     int* scnt = reinterpret_cast<int*>(xb + (size_t)NT * (a.d.H > a.d.I ? a.d.H : a.d.I) / 4);
     int* soff = scnt + a.d.E + 1;
+    int* stok = soff + a.d.E + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int i = 0; i < a.nstages; ++i) { mbar_init(&S.full[i], 1); mbar_init(&S.empty[i], kCW); }
         for (int i = 0; i < kQ; ++i) { mbar_init(&S.qfull[i], 1); mbar_init(&S.qempty[i], 1); }
+        for (int i = 0; i < kSQ; ++i) { mbar_init(&S.dfull[i], kCT); mbar_init(&S.dempty[i], 1); }
         S.abort_flag = 0;
         S.staged_n = -1;
         mbar_fence_init();
     }
     __syncthreads();
-    if (warp == kCW) {
+    if (warp == kProducerWarp) {
         if (lane == 0) fused_producer(a, S, ring);
         __syncwarp();
+    } else if (warp == kSignalWarp) {
+        fused_signaler<XT>(a, S, lane, scnt, soff, stok);
     } else {
         const int ctid = tid;
         uint32_t q = 0, slot_s = 0, phase_s = 0;
-        while (true) {
+        for (uint32_t k = 0;; ++k) {
             // thread 0 takes the next item and publishes it, so every consumer
             // thread takes the same branch below
             const uint32_t slot = q % kQ;
@@ -527,13 +614,18 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
             const uint64_t t_begin = (a.trace && ctid == 0) ? globaltimer_ns() : 0;
             if (ctid == 0) S.first_wait_ns = S.total_wait_ns = 0;
             if (it.kind == IT_ROUTER) router_item<XT, NT>(a, S, it.ex, ctid);
-            else if (it.kind == IT_PLAN) plan_item(a, S, ctid, scnt, soff);
             else if (it.kind == IT_GU || it.kind == IT_DOWN)
                 weight_item<XT, NT>(a, S, it, ring, xb, slot_s, phase_s, ctid);
+            // hand the completion to the signaler: the record first, then every
+            // consumer thread arrives after its own global writes
+            const uint32_t ds = k % kSQ;
+            if (ctid == 0) {
+                if (k >= kSQ) wait_bar(&S.dempty[ds], ((k / kSQ) - 1) & 1, &S.abort_flag, a, 11);
+                S.done[ds] = it;
+            }
             named_bar(1, kCT);
+            mbar_arrive(&S.dfull[ds]);
             if (a.trace && ctid == 0 && it.kind != IT_END) {
-                // record: (cta << 40 | kind << 32 | ex << 16 | rt), begin, end, first-data wait,
-                // pushed by the producer, total weight-stage wait of warp 0
                 const unsigned long long r = atomicAdd(reinterpret_cast<unsigned long long*>(a.trace), 1ull);
                 if (r < (unsigned long long)a.trace_cap) {
                     long long* rec = a.trace + 8 + 8 * r;
@@ -555,8 +647,8 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
     if (tid == 0) {
         __threadfence();
         if (atomicAdd(&a.ctl[kCtlExit], 1) == (int)gridDim.x - 1) {
-            // last CTA out: clear the counters for the next launch (keep the error)
-            const int n = kCtlGuDone + a.d.E + a.d.S + a.d.H / kTileRows;
+            // last CTA out: clear the control block for the next launch (keep the error)
+            const int n = ctl_ints(a.d.E, a.d.S, a.d.H, a.d.K);
             for (int i = 0; i < n; ++i)
                 if (i != kCtlError) a.ctl[i] = 0;
             __threadfence();
@@ -567,7 +659,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
 size_t fused_smem_bytes(const Dims& d, int NT, int nstages, int sb) {
     const size_t head = (sizeof(FusedSmem) + 127) & ~(size_t)127;
     const int C = d.H > d.I ? d.H : d.I;
-    return head + (size_t)nstages * sb * kBlockBytes + (size_t)NT * C * 4 + (size_t)(2 * d.E + 2) * 4;
+    return head + (size_t)nstages * sb * kBlockBytes + (size_t)NT * C * 4 + (size_t)(3 * d.E + 3) * 4;
 }
 
 // Ring geometry for NT tokens: the largest copies (up to 8 blocks = 34,816 B;

@@ -223,7 +223,7 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     const size_t TK = (size_t)Tm * d.K, slots = TK + (size_t)d.S * Tm, EA = (size_t)d.E + d.S;
     size_t sz[] = {Tm * (size_t)d.E * 8, TK * 4, TK * 4, (size_t)d.E * 4, (size_t)(d.E + 1) * 4, (size_t)d.E * 4, 4,
                    TK * 4, slots * 4, EA * 4, EA * 4, EA * 4, 4, slots * d.I * 4, slots * d.H * 4, (size_t)Tm * d.H * 4,
-                   (size_t)ctl_ints(d.E, d.S, d.H) * 4};
+                   (size_t)ctl_ints(d.E, d.S, d.H, d.K) * 4, (size_t)d.E * 16};
     constexpr int kRegions = sizeof(sz) / sizeof(sz[0]);
     size_t total = 0;
     for (size_t s : sz) total += align256(s);
@@ -233,6 +233,7 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     void* ptrs[kRegions];
     for (int i = 0; i < kRegions; ++i) { ptrs[i] = cur; cur += align256(sz[i]); }
     L->ctl = (int*)ptrs[16];
+    L->plan.table = (int4*)ptrs[17];
     {
         int optin = 0;
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
@@ -387,7 +388,7 @@ static coli_status sync_and_check(coli_moe_layer* L) {
     int err = 0;
     CUDA_TRY(cudaMemcpy(&err, L->ctl + kCtlError, 4, cudaMemcpyDeviceToHost), "read status");
     if (err != 0) {
-        CUDA_TRY(cudaMemset(L->ctl, 0, (size_t)ctl_ints(L->d.E, L->d.S, L->d.H) * 4), "reset control block");
+        CUDA_TRY(cudaMemset(L->ctl, 0, (size_t)ctl_ints(L->d.E, L->d.S, L->d.H, L->d.K) * 4), "reset control block");
         char msg[96];
         snprintf(msg, sizeof msg, "persistent decode kernel: a bounded wait timed out (site %d)", err);
         g_last_error = msg;
