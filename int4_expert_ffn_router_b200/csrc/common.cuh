@@ -52,9 +52,17 @@ constexpr int kMaxStages = 24;
 //   published, [kCtlExit] CTAs done, [kCtlError] timeout code,
 //   [kCtlGuDone + e] finished gate/up tiles of expert e (E + S entries),
 //   [kCtlGuDone + E + S + rt] finished down tiles of output block rt (H/128),
-//   then kFusedMaxTok * (K + S) float bit patterns: max |h| of each position.
+//   then kFusedMaxTok * (K + S) float bit patterns: max |h| of each position,
+//   then 2 * kFusedMaxTok * K ints: one 64-bit plan entry per distinct routed
+//   expert u (bit 63 valid; expert, first position, tokens, token ids).
 enum { kCtlTicket = 0, kCtlRouter = 1, kCtlPlan = 2, kCtlExit = 3, kCtlError = 4, kCtlGuDone = 8 };
-__host__ __device__ inline int ctl_ints(int E, int S, int H, int K) { return kCtlGuDone + E + S + H / 128 + kFusedMaxTok * (K + S); }
+__host__ __device__ inline int ctl_hmax_at(int E, int S, int H) { return kCtlGuDone + E + S + H / 128; }
+__host__ __device__ inline int ctl_entries_at(int E, int S, int H, int K) {
+    return (ctl_hmax_at(E, S, H) + kFusedMaxTok * (K + S) + 1) & ~1;  // 8-byte aligned
+}
+__host__ __device__ inline int ctl_ints(int E, int S, int H, int K) {
+    return ctl_entries_at(E, S, H, K) + 2 * kFusedMaxTok * K;
+}
 
 inline int64_t matrix_bytes(int rows, int cols) {
     return (int64_t)(rows / kTileRows) * (cols / kGroup) * kBlockBytes;

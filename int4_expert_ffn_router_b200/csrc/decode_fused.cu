@@ -20,7 +20,7 @@
 //    combines each 128-row block of y when its last down tile lands, so the
 //    consumers never wait on a global round trip to hand work off.
 // Tickets are handed out in dependency order: router rows, shared-expert
-// gate/up, shared-expert down, routed gate/up, routed down. An item only
+// gate/up, routed gate/up, shared-expert down, routed down. An item only
 // waits for items with smaller tickets, which running CTAs already hold, so
 // the schedule cannot deadlock; every wait is bounded in time and reports a
 // timeout through the control block instead of hanging.
@@ -140,7 +140,23 @@ __device__ __forceinline__ bool wait_geq(const int* p, int target, volatile int*
 // Running max |h| of each position (float bits; non-negative floats order as
 // unsigned integers), after the tile counters in the control block.
 __device__ __forceinline__ unsigned* hmax_of(FusedArgs& a) {
-    return reinterpret_cast<unsigned*>(a.ctl + kCtlGuDone + a.d.E + a.d.S + a.d.H / kTileRows);
+    return reinterpret_cast<unsigned*>(a.ctl + ctl_hmax_at(a.d.E, a.d.S, a.d.H));
+}
+
+// Packed plan entries: bit 63 valid, [0,16) expert, [16,32) first position,
+// [32,40) tokens, [40,48) token ids (2 bits each, ascending).
+__device__ __forceinline__ unsigned long long* entries_of(FusedArgs& a) {
+    return reinterpret_cast<unsigned long long*>(a.ctl + ctl_entries_at(a.d.E, a.d.S, a.d.H, a.d.K));
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 // ------------------------------------------------------------------ producer
@@ -150,38 +166,51 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
     const int RTgu = 2 * d.I / kTileRows, RTd = d.H / kTileRows;
     const int Ggu = d.H / kGroup, Gd = d.I / kGroup;
     const int n_router = (d.E + kRouterExperts - 1) / kRouterExperts;
-    const int t_sg = n_router, t_sd = t_sg + d.S * RTgu, t_ug = t_sd + d.S * RTd;
-    const int t_ud = t_ug + a.umax * RTgu, t_end = t_ud + a.umax * RTd;
+    // ticket ranges: router | shared gate/up | routed gate/up | shared down | routed down
+    const int t_sg = n_router, t_ug = t_sg + d.S * RTgu, t_sd = t_ug + a.umax * RTgu;
+    const int t_ud = t_sd + d.S * RTd, t_end = t_ud + a.umax * RTd;
     int all_tokens = 0;
     for (int t = 0; t < T; ++t) all_tokens |= t << (8 * t);
     volatile int* abort_flag = &S.abort_flag;
-    int n_unique = -1;
+    const unsigned long long* entries = entries_of(a);
     uint32_t q = 0, gs = 0, slot_s = 0, phase_s = 0;
     while (true) {
         Item it{IT_END, 0, 0, 0, 0, 0, 0, 0, 0};
         if (!*abort_flag) {
             const int t = atomicAdd(&a.ctl[kCtlTicket], 1);
+            const bool routed = (t >= t_ug && t < t_sd) || (t >= t_ud && t < t_end);
             if (t < t_sg) {
                 it.kind = IT_ROUTER;
                 it.ex = t * kRouterExperts;
-            } else if (t < t_sd) {
+            } else if (t < t_ug) {
                 const int j = (t - t_sg) / RTgu;
                 it = Item{IT_GU, d.E + j, (t - t_sg) % RTgu, T * d.K + j * T, T, all_tokens, 0, 0, 0};
-            } else if (t < t_ug) {
+            } else if (t >= t_sd && t < t_ud) {
                 const int j = (t - t_sd) / RTd;
                 it = Item{IT_DOWN, d.E + j, (t - t_sd) % RTd, T * d.K + j * T, T, 0, 0, 0, 0};
-            } else if (t < t_end) {
-                if (n_unique < 0) {
-                    if (!wait_geq(&a.ctl[kCtlPlan], 1, abort_flag, a, 2)) continue;
-                    n_unique = ld_acquire(&a.ctl[kCtlPlan]) - 1;
-                }
-                const bool gu = t < t_ud;
+            } else if (routed) {
+                const bool gu = t < t_sd;
                 const int r = gu ? t - t_ug : t - t_ud;
                 const int RT = gu ? RTgu : RTd;
                 const int u = r / RT;
-                if (u >= n_unique) continue;  // fewer distinct experts than the bound
-                const int4 ent = __ldcg(a.p.table + u);
-                it = Item{gu ? IT_GU : IT_DOWN, ent.x, r % RT, ent.y, ent.z, ent.w, 0, 0, 0};
+                // wait for this expert's plan entry, or for a plan with fewer experts
+                unsigned long long v = ld_acquire_u64(entries + u);
+                bool skip = false;
+                const uint64_t t0 = globaltimer_ns();
+                while (!(v >> 63)) {
+                    const int f = ld_acquire(&a.ctl[kCtlPlan]);
+                    if (f > 0 && u >= f - 1) { skip = true; break; }
+                    if (*abort_flag) break;
+                    if (globaltimer_ns() - t0 > kWaitNs) { set_error(a, abort_flag, 2); break; }
+                    __nanosleep(32);
+                    v = ld_acquire_u64(entries + u);
+                }
+                if (skip) continue;  // fewer distinct experts than the bound
+                if (!(v >> 63)) continue;  // aborted
+                int toks = 0;
+                const int cnt = (int)((v >> 32) & 0xFF);
+                for (int i = 0; i < cnt; ++i) toks |= (int)((v >> (40 + 2 * i)) & 3) << (8 * i);
+                it = Item{gu ? IT_GU : IT_DOWN, (int)(v & 0xFFFF), r % RT, (int)((v >> 16) & 0xFFFF), cnt, toks, 0, 0, 0};
             }
             if (it.kind == IT_DOWN) it.ready = ld_acquire(&a.ctl[kCtlGuDone + it.ex]) >= RTgu;
         }
@@ -270,6 +299,11 @@ __device__ void signal_plan(FusedArgs& a, FusedSmem& S, int lane, int* scnt, int
                 a.p.act_off[rank] = off;
                 a.p.act_cnt[rank] = c;
                 a.p.table[rank] = make_int4(e, off, c, stok[e]);
+                unsigned long long v = (1ull << 63) | (unsigned long long)e | ((unsigned long long)off << 16) |
+                                       ((unsigned long long)c << 32);
+                for (int i = 0; i < c && i < 4; ++i)
+                    v |= (unsigned long long)((stok[e] >> (8 * i)) & 3) << (40 + 2 * i);
+                st_release_u64(entries_of(a) + rank, v);
             }
         }
         carry += __shfl_sync(0xffffffffu, incl, 31);
@@ -376,7 +410,7 @@ __device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
     for (int t = 0; t < NT; ++t) acc[t] = 0.0;
     if (e < d.E) {
         const float* wrow = a.wr + (size_t)e * d.H + part * chunk;
-        constexpr int kV = 6;  // float4 per lane per pass (weights, then each token's x)
+        constexpr int kV = 12;  // float4 per lane per pass: one pass for H = 6144
         for (int base = 0; base < chunk; base += kV * 128) {
             float4 wv[kV];
 #pragma unroll
@@ -387,29 +421,32 @@ __device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
 #pragma unroll 1
             for (int t = 0; t < a.T; ++t) {
                 const XT* xr = x + (size_t)t * d.H + part * chunk;
-                double xv[kV][4];
-#pragma unroll
-                for (int j = 0; j < kV; ++j) {
-                    const int i = base + lane * 4 + j * 128;
-                    xv[j][0] = xv[j][1] = xv[j][2] = xv[j][3] = 0.0;
-                    if (i < chunk) {
-                        if constexpr (sizeof(XT) == 4) {
-                            const float4 v = __ldg(reinterpret_cast<const float4*>(xr + i));
-                            xv[j][0] = v.x; xv[j][1] = v.y; xv[j][2] = v.z; xv[j][3] = v.w;
-                        } else {
-                            const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr + i));
-                            xv[j][0] = __uint_as_float(u.x << 16); xv[j][1] = __uint_as_float(u.x & 0xFFFF0000u);
-                            xv[j][2] = __uint_as_float(u.y << 16); xv[j][3] = __uint_as_float(u.y & 0xFFFF0000u);
-                        }
-                    }
-                }
                 double sacc = 0.0;
 #pragma unroll
-                for (int j = 0; j < kV; ++j) {
-                    sacc = fma((double)wv[j].x, xv[j][0], sacc);
-                    sacc = fma((double)wv[j].y, xv[j][1], sacc);
-                    sacc = fma((double)wv[j].z, xv[j][2], sacc);
-                    sacc = fma((double)wv[j].w, xv[j][3], sacc);
+                for (int h2 = 0; h2 < kV; h2 += kV / 2) {  // x in two halves keeps registers bounded
+                    float4 xv[kV / 2];
+#pragma unroll
+                    for (int jj = 0; jj < kV / 2; ++jj) {
+                        const int i = base + lane * 4 + (h2 + jj) * 128;
+                        xv[jj] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (i < chunk) {
+                            if constexpr (sizeof(XT) == 4) {
+                                xv[jj] = __ldg(reinterpret_cast<const float4*>(xr + i));
+                            } else {
+                                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr + i));
+                                xv[jj] = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                                                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < kV / 2; ++jj) {
+                        const float4 wj = wv[h2 + jj];
+                        sacc = fma((double)wj.x, (double)xv[jj].x, sacc);
+                        sacc = fma((double)wj.y, (double)xv[jj].y, sacc);
+                        sacc = fma((double)wj.z, (double)xv[jj].z, sacc);
+                        sacc = fma((double)wj.w, (double)xv[jj].w, sacc);
+                    }
                 }
 #pragma unroll
                 for (int tt = 0; tt < NT; ++tt)
