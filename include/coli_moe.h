@@ -182,12 +182,13 @@ coli_status coli_moe_set_fused(coli_moe_layer* layer, int enable);
  * Item timeline of the persistent decode kernel, for profiling. `buffer` is a
  * caller-owned DEVICE buffer of 8 * (8 + 8 * capacity) bytes, zeroed by the
  * caller; int64 [0] counts records (it may exceed capacity: later records are
- * dropped), [1..3] are the plan item's top-k / plan-written / published times
- * (ns after it began). Record r at int64 8 + 8r: {cta << 40 | kind << 32 |
+ * dropped); [1..5] global-timer stamps of the plan path: the last router
+ * completion seen, its atomic done, plan published, top-k started, top-k
+ * done. Record r at int64 8 + 8r: {cta << 40 | kind << 32 |
  * expert << 16 | tile, begin ns, end ns, ns waited for the item's first weight
  * stage, ns the item was published by the CTA's producer, total ns warp 0
- * waited for weight stages, 0, 0}; kind 1 router rows, 2 plan, 3 gate/up
- * tile, 4 down tile; times from the GPU global timer. NULL disables tracing.
+ * waited for weight stages, 0, 0}; kind 1 router rows, 2 gate/up tile,
+ * 3 down tile; times from the GPU global timer. NULL disables tracing.
  */
 coli_status coli_moe_set_trace(coli_moe_layer* layer, void* buffer, int capacity);
 

@@ -254,6 +254,7 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
 __device__ void signal_plan(FusedArgs& a, FusedSmem& S, int lane, int* scnt, int* soff, int* stok) {
     const Dims& d = a.d;
     const int T = a.T, E = d.E, K = d.K;
+    if (lane == 0 && a.trace) a.trace[4] = (long long)globaltimer_ns();
     for (int t = 0; t < T; ++t) {
         int id;
         float wt;
@@ -266,6 +267,7 @@ __device__ void signal_plan(FusedArgs& a, FusedSmem& S, int lane, int* scnt, int
         }
     }
     __syncwarp();
+    if (lane == 0 && a.trace) a.trace[5] = (long long)globaltimer_ns();
     for (int e = lane; e < E; e += 32) { scnt[e] = 0; stok[e] = 0; }
     __syncwarp();
     for (int t = 0; t < T; ++t) {  // ids of one token are distinct: lane k owns slot k
@@ -336,6 +338,7 @@ __device__ void signal_plan(FusedArgs& a, FusedSmem& S, int lane, int* scnt, int
     for (int i = lane; i < d.S * T; i += 32) a.p.tok[T * K + i] = i % T;
     __syncwarp();
     if (lane == 0) st_release(&a.ctl[kCtlPlan], n_unique + 1);
+    if (lane == 0 && a.trace) a.trace[3] = (long long)globaltimer_ns();
 }
 
 // y rows of output block rt: residual + shared experts + routed experts in
@@ -371,7 +374,9 @@ __device__ void fused_signaler(FusedArgs& a, FusedSmem& S, int lane, int* scnt, 
         int last = 0;
         if (lane == 0) {
             if (r.kind == IT_ROUTER) {
+                const uint64_t t0 = a.trace ? globaltimer_ns() : 0;
                 last = atom_add_acq_rel(&a.ctl[kCtlRouter], 1) == n_router - 1;
+                if (last && a.trace) { a.trace[1] = (long long)t0; a.trace[2] = (long long)globaltimer_ns(); }
             } else if (r.kind == IT_GU) {
                 red_add_release(&a.ctl[kCtlGuDone + r.ex], 1);
             } else {
@@ -411,34 +416,46 @@ __device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
     if (e < d.E) {
         const float* wrow = a.wr + (size_t)e * d.H + part * chunk;
         constexpr int kV = 12;  // float4 per lane per pass: one pass for H = 6144
+        auto load_x = [&](const XT* xr, int i) -> float4 {
+            if (i >= chunk) return make_float4(0.f, 0.f, 0.f, 0.f);
+            if constexpr (sizeof(XT) == 4) {
+                return __ldg(reinterpret_cast<const float4*>(xr + i));
+            } else {
+                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr + i));
+                return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                                   __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+            }
+        };
         for (int base = 0; base < chunk; base += kV * 128) {
-            float4 wv[kV];
+            // weights and the first token's x in one batch of loads (one round trip)
+            float4 wv[kV], xv0[kV];
+            const XT* x0 = x + part * chunk;
 #pragma unroll
             for (int j = 0; j < kV; ++j) {
                 const int i = base + lane * 4 + j * 128;
                 wv[j] = i < chunk ? __ldg(reinterpret_cast<const float4*>(wrow + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                xv0[j] = load_x(x0, i);
+            }
+            {
+                double sacc = 0.0;
+#pragma unroll
+                for (int j = 0; j < kV; ++j) {
+                    sacc = fma((double)wv[j].x, (double)xv0[j].x, sacc);
+                    sacc = fma((double)wv[j].y, (double)xv0[j].y, sacc);
+                    sacc = fma((double)wv[j].z, (double)xv0[j].z, sacc);
+                    sacc = fma((double)wv[j].w, (double)xv0[j].w, sacc);
+                }
+                acc[0] += sacc;
             }
 #pragma unroll 1
-            for (int t = 0; t < a.T; ++t) {
+            for (int t = 1; t < a.T; ++t) {
                 const XT* xr = x + (size_t)t * d.H + part * chunk;
                 double sacc = 0.0;
 #pragma unroll
                 for (int h2 = 0; h2 < kV; h2 += kV / 2) {  // x in two halves keeps registers bounded
                     float4 xv[kV / 2];
 #pragma unroll
-                    for (int jj = 0; jj < kV / 2; ++jj) {
-                        const int i = base + lane * 4 + (h2 + jj) * 128;
-                        xv[jj] = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (i < chunk) {
-                            if constexpr (sizeof(XT) == 4) {
-                                xv[jj] = __ldg(reinterpret_cast<const float4*>(xr + i));
-                            } else {
-                                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr + i));
-                                xv[jj] = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
-                                                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
-                            }
-                        }
-                    }
+                    for (int jj = 0; jj < kV / 2; ++jj) xv[jj] = load_x(xr, base + lane * 4 + (h2 + jj) * 128);
 #pragma unroll
                     for (int jj = 0; jj < kV / 2; ++jj) {
                         const float4 wj = wv[h2 + jj];
@@ -449,7 +466,7 @@ __device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
                     }
                 }
 #pragma unroll
-                for (int tt = 0; tt < NT; ++tt)
+                for (int tt = 1; tt < NT; ++tt)
                     if (tt == t) acc[tt] += sacc;
             }
         }
