@@ -79,6 +79,7 @@ struct FusedSmem {
     Item cur[2];
     Item done[kSQ];
     int abort_flag;
+    int last;
     int staged_n, staged_rows[kFusedMaxTok];
     float xscale[kFusedMaxTok];
     float mred[(kCW + 1) * kFusedMaxTok];
@@ -248,99 +249,114 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
     }
 }
 
-// ------------------------------------------------------------------ signaler
-// Top-k of the T tokens and the batch-union plan, by the signaler warp of the
-// CTA that finished the last router item.
-__device__ void signal_plan(FusedArgs& a, FusedSmem& S, int lane, int* scnt, int* soff, int* stok) {
-    const Dims& d = a.d;
-    const int T = a.T, E = d.E, K = d.K;
-    if (lane == 0 && a.trace) a.trace[4] = (long long)globaltimer_ns();
-    for (int t = 0; t < T; ++t) {
-        int id;
-        float wt;
-        if (E <= 256) warp_topk<true, 8>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
-        else warp_topk<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
-        if (lane < K) {
-            a.p.ids[t * K + lane] = id;
-            a.p.w[t * K + lane] = wt;
-            S.sids[t * K + lane] = id;
-        }
-    }
-    __syncwarp();
-    if (lane == 0 && a.trace) a.trace[5] = (long long)globaltimer_ns();
-    for (int e = lane; e < E; e += 32) { scnt[e] = 0; stok[e] = 0; }
-    __syncwarp();
-    for (int t = 0; t < T; ++t) {  // ids of one token are distinct: lane k owns slot k
-        if (lane < K) {
-            const int e = S.sids[t * K + lane];
-            stok[e] |= t << (8 * scnt[e]);
-            scnt[e] += 1;
-        }
-        __syncwarp();
-    }
-    // counts, offsets (exclusive scan) and the distinct experts, 32 at a time
-    int carry = 0, ucarry = 0;
-    for (int c0 = 0; c0 < E; c0 += 32) {
-        const int e = c0 + lane;
-        const int c = e < E ? scnt[e] : 0;
-        const int f = c > 0;
-        int incl = c, fincl = f;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n1 = __shfl_up_sync(0xffffffffu, incl, o), n2 = __shfl_up_sync(0xffffffffu, fincl, o);
-            if (lane >= o) { incl += n1; fincl += n2; }
-        }
-        const int off = carry + incl - c, rank = ucarry + fincl - f;
-        if (e < E) {
-            soff[e] = off;
-            a.p.off[e] = off;
-            a.p.cnt[e] = c;
-            if (f) {
-                a.p.unique[rank] = e;
-                a.p.act_expert[rank] = e;
-                a.p.act_off[rank] = off;
-                a.p.act_cnt[rank] = c;
-                a.p.table[rank] = make_int4(e, off, c, stok[e]);
-                unsigned long long v = (1ull << 63) | (unsigned long long)e | ((unsigned long long)off << 16) |
-                                       ((unsigned long long)c << 32);
-                for (int i = 0; i < c && i < 4; ++i)
-                    v |= (unsigned long long)((stok[e] >> (8 * i)) & 3) << (40 + 2 * i);
-                st_release_u64(entries_of(a) + rank, v);
-            }
-        }
-        carry += __shfl_sync(0xffffffffu, incl, 31);
-        ucarry += __shfl_sync(0xffffffffu, fincl, 31);
-    }
-    const int n_unique = ucarry;
-    if (lane == 0) {
-        a.p.off[E] = carry;
-        *a.p.n_unique = n_unique;
-        *a.p.n_active = n_unique + d.S;
-    }
-    for (int j = lane; j < d.S; j += 32) {
-        a.p.act_expert[n_unique + j] = E + j;
-        a.p.act_off[n_unique + j] = T * K + j * T;
-        a.p.act_cnt[n_unique + j] = T;
-    }
-    __syncwarp();
-    for (int e = lane; e < E; e += 32) scnt[e] = 0;
-    __syncwarp();
-    for (int t = 0; t < T; ++t) {
-        if (lane < K) {
-            const int e = S.sids[t * K + lane];
-            const int q = soff[e] + scnt[e];
-            scnt[e] += 1;
-            a.p.pos[t * K + lane] = q;
-            a.p.tok[q] = t;
-        }
-        __syncwarp();
-    }
-    for (int i = lane; i < d.S * T; i += 32) a.p.tok[T * K + i] = i % T;
-    __syncwarp();
-    if (lane == 0) st_release(&a.ctl[kCtlPlan], n_unique + 1);
-    if (lane == 0 && a.trace) a.trace[3] = (long long)globaltimer_ns();
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// Top-k of the T tokens (warp t) and the batch-union plan (warp 0), by the
+// consumers of the CTA that finished the last router item. Each distinct
+// expert's packed entry is stored as soon as it is known (a single 64-bit
+// store, so a producer polling it sees all of it or nothing); the remaining
+// plan arrays are ordered before the one release of the plan flag.
+__device__ __noinline__ void consumer_plan(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* soff, int* stok) {
+    const Dims& d = a.d;
+    const int T = a.T, E = d.E, K = d.K;
+    const int cw = ctid >> 5, lane = ctid & 31;
+    if (a.trace && ctid == 0) a.trace[4] = (long long)globaltimer_ns();
+    if (cw < T) {
+        int id;
+        float wt;
+        if (E <= 256) warp_topk<true, 8>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
+        else warp_topk<true>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
+        if (lane < K) {
+            a.p.ids[cw * K + lane] = id;
+            a.p.w[cw * K + lane] = wt;
+            S.sids[cw * K + lane] = id;
+        }
+    }
+    named_bar(1, kCT);
+    if (a.trace && ctid == 0) a.trace[5] = (long long)globaltimer_ns();
+    if (cw == 0) {
+        for (int e = lane; e < E; e += 32) { scnt[e] = 0; stok[e] = 0; }
+        __syncwarp();
+        for (int t = 0; t < T; ++t) {  // ids of one token are distinct: lane k owns slot k
+            if (lane < K) {
+                const int e = S.sids[t * K + lane];
+                stok[e] |= t << (8 * scnt[e]);
+                scnt[e] += 1;
+            }
+            __syncwarp();
+        }
+        // counts, offsets (exclusive scan) and the distinct experts, 32 at a time
+        int carry = 0, ucarry = 0;
+        unsigned long long* entries = entries_of(a);
+        for (int c0 = 0; c0 < E; c0 += 32) {
+            const int e = c0 + lane;
+            const int c = e < E ? scnt[e] : 0;
+            const int f = c > 0;
+            int incl = c, fincl = f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n1 = __shfl_up_sync(0xffffffffu, incl, o), n2 = __shfl_up_sync(0xffffffffu, fincl, o);
+                if (lane >= o) { incl += n1; fincl += n2; }
+            }
+            const int off = carry + incl - c, rank = ucarry + fincl - f;
+            if (e < E) {
+                soff[e] = off;
+                if (f) {
+                    unsigned long long v = (1ull << 63) | (unsigned long long)e | ((unsigned long long)off << 16) |
+                                           ((unsigned long long)c << 32);
+                    for (int i = 0; i < c && i < 4; ++i)
+                        v |= (unsigned long long)((stok[e] >> (8 * i)) & 3) << (40 + 2 * i);
+                    st_relaxed_u64(entries + rank, v);
+                }
+                a.p.off[e] = off;
+                a.p.cnt[e] = c;
+                if (f) {
+                    a.p.unique[rank] = e;
+                    a.p.act_expert[rank] = e;
+                    a.p.act_off[rank] = off;
+                    a.p.act_cnt[rank] = c;
+                    a.p.table[rank] = make_int4(e, off, c, stok[e]);
+                }
+            }
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+            ucarry += __shfl_sync(0xffffffffu, fincl, 31);
+        }
+        const int n_unique = ucarry;
+        if (lane == 0) {
+            a.p.off[E] = carry;
+            *a.p.n_unique = n_unique;
+            *a.p.n_active = n_unique + d.S;
+        }
+        for (int j = lane; j < d.S; j += 32) {
+            a.p.act_expert[n_unique + j] = E + j;
+            a.p.act_off[n_unique + j] = T * K + j * T;
+            a.p.act_cnt[n_unique + j] = T;
+        }
+        __syncwarp();
+        for (int e = lane; e < E; e += 32) scnt[e] = 0;
+        __syncwarp();
+        for (int t = 0; t < T; ++t) {
+            if (lane < K) {
+                const int e = S.sids[t * K + lane];
+                const int q = soff[e] + scnt[e];
+                scnt[e] += 1;
+                a.p.pos[t * K + lane] = q;
+                a.p.tok[q] = t;
+            }
+            __syncwarp();
+        }
+        for (int i = lane; i < d.S * T; i += 32) a.p.tok[T * K + i] = i % T;
+        __syncwarp();
+        if (lane == 0) {
+            st_release(&a.ctl[kCtlPlan], n_unique + 1);
+            if (a.trace) a.trace[3] = (long long)globaltimer_ns();
+        }
+    }
+}
+
+// ------------------------------------------------------------------ signaler
 // y rows of output block rt: residual + shared experts + routed experts in
 // routing order (fixed order, same as the separate combine kernel).
 template <typename XT>
@@ -362,9 +378,8 @@ __device__ void signal_combine(FusedArgs& a, int rt, int lane) {
 }
 
 template <typename XT>
-__device__ void fused_signaler(FusedArgs& a, FusedSmem& S, int lane, int* scnt, int* soff, int* stok) {
+__device__ void fused_signaler(FusedArgs& a, FusedSmem& S, int lane) {
     const Dims& d = a.d;
-    const int n_router = (d.E + kRouterExperts - 1) / kRouterExperts;
     volatile int* abort_flag = &S.abort_flag;
     for (uint32_t k = 0;; ++k) {
         const uint32_t slot = k % kSQ;
@@ -373,13 +388,9 @@ __device__ void fused_signaler(FusedArgs& a, FusedSmem& S, int lane, int* scnt, 
         if (!ok || r.kind == IT_END) break;
         int last = 0;
         if (lane == 0) {
-            if (r.kind == IT_ROUTER) {
-                const uint64_t t0 = a.trace ? globaltimer_ns() : 0;
-                last = atom_add_acq_rel(&a.ctl[kCtlRouter], 1) == n_router - 1;
-                if (last && a.trace) { a.trace[1] = (long long)t0; a.trace[2] = (long long)globaltimer_ns(); }
-            } else if (r.kind == IT_GU) {
+            if (r.kind == IT_GU) {
                 red_add_release(&a.ctl[kCtlGuDone + r.ex], 1);
-            } else {
+            } else if (r.kind == IT_DOWN) {
                 const int prev = atom_add_acq_rel(&a.ctl[kCtlGuDone + d.E + d.S + r.rt], 1);
                 // no output block can be complete before the plan is published,
                 // so an unpublished plan means this was not the last tile
@@ -388,10 +399,7 @@ __device__ void fused_signaler(FusedArgs& a, FusedSmem& S, int lane, int* scnt, 
             }
         }
         last = __shfl_sync(0xffffffffu, last, 0);
-        if (last && !*abort_flag) {
-            if (r.kind == IT_ROUTER) signal_plan(a, S, lane, scnt, soff, stok);
-            else signal_combine<XT>(a, r.rt, lane);
-        }
+        if (last && !*abort_flag) signal_combine<XT>(a, r.rt, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.dempty[slot]);
     }
@@ -402,7 +410,7 @@ __device__ void fused_signaler(FusedArgs& a, FusedSmem& S, int lane, int* scnt, 
 // H, with the weight loads issued before the fp64 products; the four partial
 // sums are added in a fixed order.
 template <typename XT, int NT>
-__device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
+__device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid, int* scnt, int* soff, int* stok) {
     const Dims& d = a.d;
     const int cw = ctid >> 5, lane = ctid & 31;
     constexpr int kParts = kCW / kRouterExperts;
@@ -486,6 +494,16 @@ __device__ void router_item(FusedArgs& a, FusedSmem& S, int e0, int ctid) {
             a.logits[(size_t)t * d.E + ee] = sum + (double)a.bias[ee];
         }
     }
+    // the CTA that finishes the last router item builds the plan
+    named_bar(1, kCT);
+    if (ctid == 0) {
+        const int n_router = (d.E + kRouterExperts - 1) / kRouterExperts;
+        const uint64_t t0 = a.trace ? globaltimer_ns() : 0;
+        S.last = atom_add_acq_rel(&a.ctl[kCtlRouter], 1) == n_router - 1;
+        if (S.last && a.trace) { a.trace[1] = (long long)t0; a.trace[2] = (long long)globaltimer_ns(); }
+    }
+    named_bar(1, kCT);
+    if (S.last) consumer_plan(a, S, ctid, scnt, soff, stok);  // uniform: S.last is read after the barrier
 }
 
 // Stage the h rows of a down item in B-fragment order, scaled by the powers
@@ -650,7 +668,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
         if (lane == 0) fused_producer(a, S, ring);
         __syncwarp();
     } else if (warp == kSignalWarp) {
-        fused_signaler<XT>(a, S, lane, scnt, soff, stok);
+        fused_signaler<XT>(a, S, lane);
     } else {
         const int ctid = tid;
         uint32_t q = 0, slot_s = 0, phase_s = 0;
@@ -667,7 +685,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
             const Item it = S.cur[q & 1];
             const uint64_t t_begin = (a.trace && ctid == 0) ? globaltimer_ns() : 0;
             if (ctid == 0) S.first_wait_ns = S.total_wait_ns = 0;
-            if (it.kind == IT_ROUTER) router_item<XT, NT>(a, S, it.ex, ctid);
+            if (it.kind == IT_ROUTER) router_item<XT, NT>(a, S, it.ex, ctid, scnt, soff, stok);
             else if (it.kind == IT_GU || it.kind == IT_DOWN)
                 weight_item<XT, NT>(a, S, it, ring, xb, slot_s, phase_s, ctid);
             // hand the completion to the signaler: the record first, then every
