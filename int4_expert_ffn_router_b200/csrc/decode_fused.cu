@@ -85,6 +85,8 @@ struct FusedSmem {
     float mred[(kCW + 1) * kFusedMaxTok];
     double rpart[kCW][kFusedMaxTok];
     int sids[kFusedMaxTok * 32];
+    float sw[kFusedMaxTok * 32];
+    int wsum[kCW], wflag[kCW];
     unsigned long long first_wait_ns, total_wait_ns;
 };
 
@@ -253,14 +255,14 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
     asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// Top-k of the T tokens (warp t) and the batch-union plan (warp 0), by the
-// consumers of the CTA that finished the last router item. Each distinct
-// expert's packed entry is stored as soon as it is known (a single 64-bit
-// store, so a producer polling it sees all of it or nothing); the remaining
+// Top-k of the T tokens (warp t) and the batch-union plan (all eight warps),
+// by the consumers of the CTA that finished the last router item. Each
+// distinct expert's packed entry is stored as soon as it is known (a single
+// 64-bit store: a producer polling it sees all of it or nothing); the other
 // plan arrays are ordered before the one release of the plan flag.
 __device__ __noinline__ void consumer_plan(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* soff, int* stok) {
     const Dims& d = a.d;
-    const int T = a.T, E = d.E, K = d.K;
+    const int T = a.T, E = d.E, K = d.K, TK = T * K;
     const int cw = ctid >> 5, lane = ctid & 31;
     if (a.trace && ctid == 0) a.trace[4] = (long long)globaltimer_ns();
     if (cw < T) {
@@ -269,90 +271,85 @@ __device__ __noinline__ void consumer_plan(FusedArgs& a, FusedSmem& S, int ctid,
         if (E <= 256) warp_topk<true, 8>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
         else warp_topk<true>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
         if (lane < K) {
-            a.p.ids[cw * K + lane] = id;
-            a.p.w[cw * K + lane] = wt;
             S.sids[cw * K + lane] = id;
+            S.sw[cw * K + lane] = wt;
         }
     }
     named_bar(1, kCT);
     if (a.trace && ctid == 0) a.trace[5] = (long long)globaltimer_ns();
-    if (cw == 0) {
-        for (int e = lane; e < E; e += 32) { scnt[e] = 0; stok[e] = 0; }
-        __syncwarp();
-        for (int t = 0; t < T; ++t) {  // ids of one token are distinct: lane k owns slot k
-            if (lane < K) {
-                const int e = S.sids[t * K + lane];
-                stok[e] |= t << (8 * scnt[e]);
-                scnt[e] += 1;
+    // experts in chunks of 256, 32 per warp: count the slots routed to each,
+    // pack their tokens (ascending), scan counts and distinct flags
+    unsigned long long* entries = entries_of(a);
+    int carry = 0, ucarry = 0;
+    for (int c0 = 0; c0 < E; c0 += kCT) {
+        const int e = c0 + ctid;
+        int c = 0, tk = 0;
+        if (e < E) {
+            for (int sl = 0; sl < TK; ++sl) {
+                if (S.sids[sl] == e) {
+                    if (c < 4) tk |= (sl / K) << (8 * c);
+                    ++c;
+                }
             }
-            __syncwarp();
         }
-        // counts, offsets (exclusive scan) and the distinct experts, 32 at a time
-        int carry = 0, ucarry = 0;
-        unsigned long long* entries = entries_of(a);
-        for (int c0 = 0; c0 < E; c0 += 32) {
-            const int e = c0 + lane;
-            const int c = e < E ? scnt[e] : 0;
-            const int f = c > 0;
-            int incl = c, fincl = f;
+        const int f = c > 0;
+        int incl = c, fincl = f;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n1 = __shfl_up_sync(0xffffffffu, incl, o), n2 = __shfl_up_sync(0xffffffffu, fincl, o);
-                if (lane >= o) { incl += n1; fincl += n2; }
+        for (int o = 1; o < 32; o <<= 1) {
+            const int n1 = __shfl_up_sync(0xffffffffu, incl, o), n2 = __shfl_up_sync(0xffffffffu, fincl, o);
+            if (lane >= o) { incl += n1; fincl += n2; }
+        }
+        if (lane == 31) { S.wsum[cw] = incl; S.wflag[cw] = fincl; }
+        named_bar(1, kCT);
+        int base = carry, ubase = ucarry;
+        for (int w = 0; w < cw; ++w) { base += S.wsum[w]; ubase += S.wflag[w]; }
+        const int off = base + incl - c, rank = ubase + fincl - f;
+        if (e < E) {
+            if (f) {
+                unsigned long long v = (1ull << 63) | (unsigned long long)e | ((unsigned long long)off << 16) |
+                                       ((unsigned long long)c << 32);
+                for (int i = 0; i < c && i < 4; ++i) v |= (unsigned long long)((tk >> (8 * i)) & 3) << (40 + 2 * i);
+                st_relaxed_u64(entries + rank, v);
+                a.p.unique[rank] = e;
+                a.p.act_expert[rank] = e;
+                a.p.act_off[rank] = off;
+                a.p.act_cnt[rank] = c;
+                a.p.table[rank] = make_int4(e, off, c, tk);
             }
-            const int off = carry + incl - c, rank = ucarry + fincl - f;
-            if (e < E) {
-                soff[e] = off;
-                if (f) {
-                    unsigned long long v = (1ull << 63) | (unsigned long long)e | ((unsigned long long)off << 16) |
-                                           ((unsigned long long)c << 32);
-                    for (int i = 0; i < c && i < 4; ++i)
-                        v |= (unsigned long long)((stok[e] >> (8 * i)) & 3) << (40 + 2 * i);
-                    st_relaxed_u64(entries + rank, v);
-                }
-                a.p.off[e] = off;
-                a.p.cnt[e] = c;
-                if (f) {
-                    a.p.unique[rank] = e;
-                    a.p.act_expert[rank] = e;
-                    a.p.act_off[rank] = off;
-                    a.p.act_cnt[rank] = c;
-                    a.p.table[rank] = make_int4(e, off, c, stok[e]);
-                }
-            }
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-            ucarry += __shfl_sync(0xffffffffu, fincl, 31);
+            a.p.off[e] = off;
+            a.p.cnt[e] = c;
+            soff[e] = off;
         }
-        const int n_unique = ucarry;
-        if (lane == 0) {
-            a.p.off[E] = carry;
-            *a.p.n_unique = n_unique;
-            *a.p.n_active = n_unique + d.S;
-        }
-        for (int j = lane; j < d.S; j += 32) {
-            a.p.act_expert[n_unique + j] = E + j;
-            a.p.act_off[n_unique + j] = T * K + j * T;
-            a.p.act_cnt[n_unique + j] = T;
-        }
-        __syncwarp();
-        for (int e = lane; e < E; e += 32) scnt[e] = 0;
-        __syncwarp();
-        for (int t = 0; t < T; ++t) {
-            if (lane < K) {
-                const int e = S.sids[t * K + lane];
-                const int q = soff[e] + scnt[e];
-                scnt[e] += 1;
-                a.p.pos[t * K + lane] = q;
-                a.p.tok[q] = t;
-            }
-            __syncwarp();
-        }
-        for (int i = lane; i < d.S * T; i += 32) a.p.tok[T * K + i] = i % T;
-        __syncwarp();
-        if (lane == 0) {
-            st_release(&a.ctl[kCtlPlan], n_unique + 1);
-            if (a.trace) a.trace[3] = (long long)globaltimer_ns();
-        }
+        for (int w = 0; w < kCW; ++w) { carry += S.wsum[w]; ucarry += S.wflag[w]; }
+        named_bar(1, kCT);
+    }
+    const int n_unique = ucarry;
+    // slot (t, k): position = first position of its expert + earlier tokens of that expert
+    if (ctid < TK) {
+        const int e = S.sids[ctid], t = ctid / K;
+        int rank = 0;
+        for (int sl = 0; sl < t * K; ++sl) rank += S.sids[sl] == e;
+        const int q = soff[e] + rank;
+        a.p.pos[ctid] = q;
+        a.p.tok[q] = t;
+        a.p.ids[ctid] = e;
+        a.p.w[ctid] = S.sw[ctid];
+    }
+    for (int i = ctid; i < d.S * T; i += kCT) a.p.tok[TK + i] = i % T;
+    for (int j = ctid; j < d.S; j += kCT) {
+        a.p.act_expert[n_unique + j] = E + j;
+        a.p.act_off[n_unique + j] = TK + j * T;
+        a.p.act_cnt[n_unique + j] = T;
+    }
+    if (ctid == 0) {
+        a.p.off[E] = carry;
+        *a.p.n_unique = n_unique;
+        *a.p.n_active = n_unique + d.S;
+    }
+    named_bar(1, kCT);
+    if (ctid == 0) {
+        st_release(&a.ctl[kCtlPlan], n_unique + 1);
+        if (a.trace) a.trace[3] = (long long)globaltimer_ns();
     }
 }
 
