@@ -180,17 +180,26 @@ coli_status coli_moe_set_fused(coli_moe_layer* layer, int enable);
 
 /*
  * Item timeline of the persistent decode kernel, for profiling. `buffer` is a
- * caller-owned DEVICE buffer of 8 * (8 + 8 * capacity) bytes, zeroed by the
+ * caller-owned DEVICE buffer of 8 * (16 + 8 * capacity) bytes, zeroed by the
  * caller; int64 [0] counts records (it may exceed capacity: later records are
  * dropped); [1..5] global-timer stamps of the plan path: the last router
  * completion seen, its atomic done, plan published, top-k started, top-k
- * done. Record r at int64 8 + 8r: {cta << 40 | kind << 32 |
+ * done, [6..8] plan steps (scan, entries stored, before the flag release).
+ * Record r at int64 16 + 8r: {cta << 40 | kind << 32 |
  * expert << 16 | tile, begin ns, end ns, ns waited for the item's first weight
  * stage, ns the item was published by the CTA's producer, total ns warp 0
  * waited for weight stages, 0, 0}; kind 1 router rows, 2 gate/up tile,
  * 3 down tile; times from the GPU global timer. NULL disables tracing.
  */
 coli_status coli_moe_set_trace(coli_moe_layer* layer, void* buffer, int capacity);
+
+/*
+ * Weight-streaming geometry of the persistent decode kernel: each SM keeps up
+ * to `stages` bulk copies of `blocks_per_stage` x 4352 bytes in flight
+ * (defaults 3 and 8; fewer if shared memory is short). stages in [2, 24],
+ * blocks_per_stage even in [2, 8]. A tuning knob: results do not change.
+ */
+coli_status coli_moe_set_ring(coli_moe_layer* layer, int stages, int blocks_per_stage);
 
 /* Bytes of one expert in the int4 gs64 container (nibbles + fp16 scales). */
 int64_t coli_moe_expert_bytes(int hidden, int inter);

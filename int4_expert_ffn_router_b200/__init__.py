@@ -23,7 +23,7 @@ EXPORTS = (
     "coli_moe_route", "coli_moe_forward", "coli_moe_stack_forward", "coli_moe_get_stats", "coli_moe_get_plan",
     "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
     "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused",
-    "coli_moe_set_trace",
+    "coli_moe_set_trace", "coli_moe_set_ring",
 )
 N_STAGES = 7
 
@@ -65,6 +65,7 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_stage_name.restype = ctypes.c_char_p
     L.coli_moe_sync.argtypes = [vp]
     L.coli_moe_set_trace.argtypes = [vp, vp, i32]
+    L.coli_moe_set_ring.argtypes = [vp, i32, i32]
     L.coli_moe_set_fused.argtypes = [vp, i32]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
@@ -177,8 +178,11 @@ class Layer:
 
     def set_trace(self, buffer, capacity: int) -> None:
         """Record the persistent kernel's item timeline into a zeroed device
-        int64 buffer of 8 + 8 * capacity entries (None disables)."""
+        int64 buffer of 16 + 8 * capacity entries (None disables)."""
         _check(lib.coli_moe_set_trace(self.handle, _ptr(buffer), capacity), "coli_moe_set_trace")
+
+    def set_ring(self, stages: int, blocks_per_stage: int = 8) -> None:
+        _check(lib.coli_moe_set_ring(self.handle, stages, blocks_per_stage), "coli_moe_set_ring")
 
     def set_profiling(self, on: bool) -> None:
         _check(lib.coli_moe_set_profiling(self.handle, 1 if on else 0), "coli_moe_set_profiling")

@@ -260,7 +260,13 @@ __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned l
 // distinct expert's packed entry is stored as soon as it is known (a single
 // 64-bit store: a producer polling it sees all of it or nothing); the other
 // plan arrays are ordered before the one release of the plan flag.
-__device__ __noinline__ void consumer_plan(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* soff, int* stok) {
+// One token's top-k.
+__device__ __forceinline__ void topk_token(const double* l, int E, int K, int lane, int* id, float* wt) {
+    if (E <= 256) warp_topk<true, 8>(l, E, K, lane, id, wt);
+    else warp_topk<true>(l, E, K, lane, id, wt);
+}
+
+__device__ __forceinline__ void consumer_plan(FusedArgs& a, FusedSmem& S, int ctid, int* scnt, int* soff, int* stok) {
     const Dims& d = a.d;
     const int T = a.T, E = d.E, K = d.K, TK = T * K;
     const int cw = ctid >> 5, lane = ctid & 31;
@@ -268,8 +274,7 @@ __device__ __noinline__ void consumer_plan(FusedArgs& a, FusedSmem& S, int ctid,
     if (cw < T) {
         int id;
         float wt;
-        if (E <= 256) warp_topk<true, 8>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
-        else warp_topk<true>(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
+        topk_token(a.logits + (size_t)cw * E, E, K, lane, &id, &wt);
         if (lane < K) {
             S.sids[cw * K + lane] = id;
             S.sw[cw * K + lane] = wt;
@@ -301,6 +306,7 @@ __device__ __noinline__ void consumer_plan(FusedArgs& a, FusedSmem& S, int ctid,
         }
         if (lane == 31) { S.wsum[cw] = incl; S.wflag[cw] = fincl; }
         named_bar(1, kCT);
+        if (a.trace && ctid == 0) a.trace[6] = (long long)globaltimer_ns();
         int base = carry, ubase = ucarry;
         for (int w = 0; w < cw; ++w) { base += S.wsum[w]; ubase += S.wflag[w]; }
         const int off = base + incl - c, rank = ubase + fincl - f;
@@ -322,6 +328,7 @@ __device__ __noinline__ void consumer_plan(FusedArgs& a, FusedSmem& S, int ctid,
         }
         for (int w = 0; w < kCW; ++w) { carry += S.wsum[w]; ucarry += S.wflag[w]; }
         named_bar(1, kCT);
+        if (a.trace && ctid == 0) a.trace[7] = (long long)globaltimer_ns();
     }
     const int n_unique = ucarry;
     // slot (t, k): position = first position of its expert + earlier tokens of that expert
@@ -348,6 +355,7 @@ __device__ __noinline__ void consumer_plan(FusedArgs& a, FusedSmem& S, int ctid,
     }
     named_bar(1, kCT);
     if (ctid == 0) {
+        if (a.trace) a.trace[8] = (long long)globaltimer_ns();
         st_release(&a.ctl[kCtlPlan], n_unique + 1);
         if (a.trace) a.trace[3] = (long long)globaltimer_ns();
     }
@@ -697,7 +705,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
             if (a.trace && ctid == 0 && it.kind != IT_END) {
                 const unsigned long long r = atomicAdd(reinterpret_cast<unsigned long long*>(a.trace), 1ull);
                 if (r < (unsigned long long)a.trace_cap) {
-                    long long* rec = a.trace + 8 + 8 * r;
+                    long long* rec = a.trace + 16 + 8 * r;
                     rec[0] = ((long long)blockIdx.x << 40) | ((long long)it.kind << 32) | ((long long)it.ex << 16) | it.rt;
                     rec[1] = (long long)t_begin;
                     rec[2] = (long long)globaltimer_ns();
@@ -731,20 +739,23 @@ size_t fused_smem_bytes(const Dims& d, int NT, int nstages, int sb) {
     return head + (size_t)nstages * sb * kBlockBytes + (size_t)NT * C * 4 + (size_t)(3 * d.E + 3) * 4;
 }
 
-// Ring geometry for NT tokens: the largest copies (up to 8 blocks = 34,816 B;
-// bulk copies of that size stream best) with at least 4 stages in flight.
-static bool fused_geometry(const Dims& d, int NT, size_t smem_limit, int* nstages, int* sb) {
-    for (int b = kMaxSB; b >= 2; b -= 2) {
-        int ns = kMaxStages;
+// Ring geometry for NT tokens: copies of sb blocks (34,816 B at sb = 8: bulk
+// copies that large stream best) and up to max_stages of them in flight per
+// SM. More bytes in flight than bandwidth x latency only lengthen the queues
+// every dependent load waits in.
+static bool fused_geometry(const Dims& d, int NT, size_t smem_limit, int max_stages, int max_sb, int* nstages,
+                           int* sb) {
+    for (int b = max_sb; b >= 2; b -= 2) {
+        int ns = max_stages < kMaxStages ? max_stages : kMaxStages;
         while (ns > 0 && fused_smem_bytes(d, NT, ns, b) > smem_limit) --ns;
-        if (ns >= 4) { *nstages = ns; *sb = b; return true; }
+        if (ns >= 2) { *nstages = ns; *sb = b; return true; }
     }
     return false;
 }
 
 int fused_stages_for(const Dims& d, int NT, size_t smem_limit) {
     int ns = 0, sb = 0;
-    return fused_geometry(d, NT, smem_limit, &ns, &sb) ? ns : 0;
+    return fused_geometry(d, NT, smem_limit, kMaxStages, kMaxSB, &ns, &sb) ? ns : 0;
 }
 
 template <typename XT, int NT>
@@ -766,7 +777,7 @@ static cudaError_t launch_fused_t(const FusedArgs& a, int n_sm, size_t smem_limi
 cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const float* wr, const float* bias,
                                 const void* x, coli_dtype dt, int T, void* y, const float* residual, const Plan& p,
                                 double* logits, float* h, float* o, int* ctl, int n_sm, size_t smem_limit,
-                                long long* trace, int trace_cap, cudaStream_t st) {
+                                long long* trace, int trace_cap, int max_stages, int max_sb, cudaStream_t st) {
     if (T < 1 || T > kFusedMaxTok) return cudaErrorInvalidValue;
     const int NT = T == 1 ? 1 : (T == 2 ? 2 : 4);
     FusedArgs a;
@@ -774,7 +785,8 @@ cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const flo
     a.T = T; a.p = p; a.logits = logits; a.h = h; a.o = o; a.ctl = ctl;
     a.trace = trace; a.trace_cap = trace_cap;
     a.umax = T * d.K < d.E ? T * d.K : d.E;
-    if (!fused_geometry(d, NT, smem_limit, &a.nstages, &a.sb)) return cudaErrorInvalidConfiguration;
+    if (!fused_geometry(d, NT, smem_limit, max_stages, max_sb, &a.nstages, &a.sb))
+        return cudaErrorInvalidConfiguration;
     if (dt == COLI_F32) {
         if (NT == 1) return launch_fused_t<float, 1>(a, n_sm, smem_limit, st);
         if (NT == 2) return launch_fused_t<float, 2>(a, n_sm, smem_limit, st);

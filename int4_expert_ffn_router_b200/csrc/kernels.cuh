@@ -33,8 +33,10 @@ cudaError_t launch_down_core(const uint8_t* weights, const Dims& d, const float*
 cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const float* wr, const float* bias,
                                 const void* x, coli_dtype dt, int T, void* y, const float* residual, const Plan& p,
                                 double* logits, float* h, float* o, int* ctl, int n_sm, size_t smem_limit,
-                                long long* trace, int trace_cap, cudaStream_t st);
+                                long long* trace, int trace_cap, int max_stages, int max_sb, cudaStream_t st);
 int fused_stages_for(const Dims& d, int NT, size_t smem_limit);
+constexpr int kDefaultStages = 3;  // ring stages in flight per SM (see fused_geometry)
+constexpr int kDefaultStageBlocks = 8;
 
 // combine.cu
 // y[t] = residual[t] (optional) + sum_j o[TK + j*T + t] + sum_k w[t][k] o[pos[t][k]]

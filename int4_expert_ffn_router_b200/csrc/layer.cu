@@ -79,6 +79,8 @@ struct coli_moe_layer {
     bool fused = true;              // use the persistent kernel for n_tokens <= kFusedMaxTok
     long long* trace = nullptr;     // caller-owned device buffer for the item timeline
     int trace_cap = 0;
+    int ring_stages = kDefaultStages;        // persistent kernel: bulk copies in flight per SM
+    int ring_blocks = kDefaultStageBlocks;   // 4352-byte blocks per copy
     uint8_t* staging = nullptr;  // one canonical expert, for host sources
     int last_T = -1;
     cudaStream_t last_stream = nullptr;
@@ -238,7 +240,7 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
         int optin = 0;
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
         L->smem_optin = (size_t)optin;
-        L->fused = fused_stages_for(d, kFusedMaxTok, L->smem_optin) >= 4;
+        L->fused = fused_stages_for(d, kFusedMaxTok, L->smem_optin) >= 2;
     }
     L->logits = (double*)ptrs[0];
     Plan& p = L->plan;
@@ -315,7 +317,8 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
     if (L->fused && T <= kFusedMaxTok) {
         for (int i = 0; i <= COLI_STAGE_FUSED; ++i) prof_mark(L, i, s);
         CUDA_TRY(launch_decode_fused(L->weights, d, L->router_w, L->router_b, x, dt, T, y, residual, p, L->logits, L->h,
-                                     L->o, L->ctl, L->n_sm, L->smem_optin, L->trace, L->trace_cap, s),
+                                     L->o, L->ctl, L->n_sm, L->smem_optin, L->trace, L->trace_cap, L->ring_stages,
+                                     L->ring_blocks, s),
                  "persistent decode kernel");
     } else {
         prof_mark(L, COLI_STAGE_ROUTER, s);
@@ -406,9 +409,18 @@ COLI_API coli_status coli_moe_sync(coli_moe_layer* L) {
 
 COLI_API coli_status coli_moe_set_fused(coli_moe_layer* L, int enable) {
     if (!L) return fail(COLI_EINVAL, "layer is NULL");
-    if (enable && fused_stages_for(L->d, kFusedMaxTok, L->smem_optin) < 4)
+    if (enable && fused_stages_for(L->d, kFusedMaxTok, L->smem_optin) < 2)
         return fail(COLI_EUNSUPPORTED, "shapes too large for the persistent kernel's shared memory");
     L->fused = enable != 0;
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_set_ring(coli_moe_layer* L, int stages, int blocks_per_stage) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (stages < 2 || stages > 24 || blocks_per_stage < 2 || blocks_per_stage > 8 || (blocks_per_stage & 1))
+        return fail(COLI_EINVAL, "stages in [2, 24], blocks_per_stage even in [2, 8]");
+    L->ring_stages = stages;
+    L->ring_blocks = blocks_per_stage;
     return COLI_OK;
 }
 

@@ -29,33 +29,30 @@ __device__ __forceinline__ bool key_better(unsigned long long ka, int ia, unsign
 // the best of its own values; a round takes the warp's best and only the lane
 // that supplied it refreshes its own best. `coherent`: read the logits
 // through L2 only (they were written by another CTA).
+// Inverse of order_key.
+__device__ __forceinline__ double key_value(unsigned long long k) {
+    const unsigned long long u = (k >> 63) ? (k & 0x7FFFFFFFFFFFFFFFull) : ~k;
+    return __longlong_as_double((long long)u);
+}
+
 template <bool coherent, int PER = kMaxPerLane>
 __device__ __forceinline__ void warp_topk(const double* __restrict__ l, int E, int K, int lane, int* id, float* wt) {
     const int per = (E + 31) / 32;  // <= PER
-    double v[PER];
-    unsigned long long key[PER];
+    unsigned long long key[PER];     // 0: absent or taken (below every logit's key)
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-        int e = lane + 32 * i;
-        double val = -INFINITY;
-        if (i < per && e < E) val = coherent ? __ldcg(l + e) : l[e];
-        v[i] = val;
-        key[i] = (i < per && e < E) ? order_key(val) : 0ull;  // key 0: below every logit
+        const int e = lane + 32 * i;
+        key[i] = 0ull;
+        if (i < per && e < E) key[i] = order_key(coherent ? __ldcg(l + e) : l[e]);
     }
     // this lane's best: largest key, then lowest id (lower i = lower id)
-    auto local_best = [&](unsigned long long& bk, int& bi) {
-        bk = 0ull;
-        bi = 0x7fffffff;
+    unsigned long long mk = 0ull;
+    int mi = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            const int e = lane + 32 * i;
-            if (i < per && e < E && key_better(key[i], e, bk, bi)) { bk = key[i]; bi = e; }
-        }
-    };
-    unsigned long long mk;
-    int mi;
-    local_best(mk, mi);
-    double my_sel = 0.0, top = 0.0;
+    for (int i = 0; i < PER; ++i) {
+        if (key[i] > mk) { mk = key[i]; mi = lane + 32 * i; }
+    }
+    unsigned long long my_key = 0ull, top_key = 0ull;
     int my_id = -1;
     for (int k = 0; k < K; ++k) {
         unsigned long long bk = mk;
@@ -66,19 +63,19 @@ __device__ __forceinline__ void warp_topk(const double* __restrict__ l, int E, i
             const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
             if (key_better(ok, oi, bk, bi)) { bk = ok; bi = oi; }
         }
-        const bool mine = (bi & 31) == lane && bi != 0x7fffffff;
-        double bv = 0.0;
-        if (mine) {
+        if ((bi & 31) == lane && bi != 0x7fffffff) {  // the supplier drops it and refreshes its best
+            mk = 0ull;
+            mi = 0x7fffffff;
 #pragma unroll
-            for (int i = 0; i < PER; ++i)
-                if (lane + 32 * i == bi) { bv = v[i]; key[i] = 0ull; }  // taken
-            local_best(mk, mi);
+            for (int i = 0; i < PER; ++i) {
+                if (lane + 32 * i == bi) key[i] = 0ull;
+                if (key[i] > mk) { mk = key[i]; mi = lane + 32 * i; }
+            }
         }
-        bv = __shfl_sync(0xffffffffu, bv, bi & 31);
-        if (k == 0) top = bv;
-        if (lane == k) { my_sel = bv; my_id = bi; }
+        if (k == 0) top_key = bk;
+        if (lane == k) { my_key = bk; my_id = bi; }
     }
-    double ex = (lane < K) ? exp(my_sel - top) : 0.0;
+    const double ex = (lane < K) ? exp(key_value(my_key) - key_value(top_key)) : 0.0;
     double z = ex;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
