@@ -224,6 +224,10 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
         mbar_arrive(&S.qfull[slot]);
         ++q;
         if (it.kind == IT_END) break;
+        // A router item's loads (and the plan, when this CTA finishes the last
+        // one) would queue behind this SM's in-flight weight copies: start the
+        // next item only once the router item is done.
+        if (it.kind == IT_ROUTER && !wait_bar(&S.qempty[slot], ((q - 1) / kQ) & 1, abort_flag, a, 12)) continue;
         if (it.kind == IT_GU || it.kind == IT_DOWN) {
             const bool gu = it.kind == IT_GU;
             const int G = gu ? Ggu : Gd;
