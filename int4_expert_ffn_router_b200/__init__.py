@@ -23,8 +23,9 @@ EXPORTS = (
     "coli_moe_route", "coli_moe_forward", "coli_moe_stack_forward", "coli_moe_get_stats", "coli_moe_get_plan",
     "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
     "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused",
-    "coli_moe_set_trace", "coli_moe_set_ring",
+    "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc",
 )
+NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 64, 1024
 N_STAGES = 7
 
 
@@ -66,6 +67,7 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_sync.argtypes = [vp]
     L.coli_moe_set_trace.argtypes = [vp, vp, i32]
     L.coli_moe_set_ring.argtypes = [vp, i32, i32]
+    L.coli_moe_route_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, i32, i32, vp, vp, vp]
     L.coli_moe_set_fused.argtypes = [vp, i32]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
@@ -209,6 +211,16 @@ class Layer:
         out["unique"] = out["unique"][:nu.value]
         out["tok"] = out["tok"][:T * K]
         return out
+
+
+def route_noalloc(router_w, router_bias, n_experts: int, hidden: int, top_k: int, x, ids, weights,
+                  n_tokens: int | None = None, stream=None) -> None:
+    """Routing without a layer and without any device allocation (fixed
+    512 KiB scratch in the library; at most 64 tokens and 1024 experts)."""
+    T = x.shape[0] if n_tokens is None else n_tokens
+    _check(lib.coli_moe_route_noalloc(_ptr(router_w), _ptr(router_bias), n_experts, hidden, top_k, _ptr(x),
+                                      _dtype_of(x), T, _ptr(ids), _ptr(weights), _stream(stream)),
+           "coli_moe_route_noalloc")
 
 
 def stack_forward(layers, x, n_tokens: int | None = None, eps: float = 1e-6, stream=None) -> None:

@@ -2,6 +2,8 @@
 // repack.cu, combine.cu).
 #pragma once
 
+#include <string>
+
 #include "common.cuh"
 
 namespace coli {
@@ -37,6 +39,9 @@ cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const flo
 int fused_stages_for(const Dims& d, int NT, size_t smem_limit);
 constexpr int kDefaultStages = 3;  // ring stages in flight per SM (see fused_geometry)
 constexpr int kDefaultStageBlocks = 8;
+
+// layer.cu: record the message coli_last_error() returns on this thread.
+void set_last_error(const std::string& what);
 
 // combine.cu
 // y[t] = residual[t] (optional) + sum_j o[TK + j*T + t] + sum_k w[t][k] o[pos[t][k]]

@@ -521,3 +521,7 @@ COLI_API const char* coli_status_string(coli_status s) {
 }
 
 COLI_API const char* coli_last_error(void) { return g_last_error.c_str(); }
+
+namespace coli {
+void set_last_error(const std::string& what) { g_last_error = what; }
+}  // namespace coli
