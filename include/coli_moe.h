@@ -112,8 +112,17 @@ coli_status coli_moe_route(coli_moe_layer* layer, const void* x, coli_dtype dtyp
 
 /*
  * The layer: y [n_tokens][H] = MoE(x), y of the same dtype as x. x and y must
- * not overlap. fp32 runs the CUDA-core path; bf16 the tensor-core path where
- * an expert has enough tokens for a dense contraction.
+ * not overlap. Paths: n_tokens <= 4 runs the persistent decode kernel (see
+ * coli_moe_set_fused); above that fp32 runs the CUDA-core kernels (fp32
+ * arithmetic) and bf16 the tcgen05 tensor-core grouped GEMMs (fp16 operands:
+ * tokens scaled by powers of two so the conversion is exact, weights rounded
+ * once to fp16, fp32 accumulation; the combine adds with fp32 atomics, so the
+ * summation order, and the last bits of y, may vary between runs). The
+ * tensor-core path needs an sm_100 device, hidden % 256 == 0, inter % 128 == 0
+ * and weight scales of magnitude <= 4096; otherwise bf16 also runs the CUDA-core
+ * kernels. Sparse-expert forward as the Colibrì pages describe it (top-8 of
+ * 256 routed experts plus the always-on shared expert, each distinct expert's
+ * int4 weights read once per batch).
  */
 coli_status coli_moe_forward(coli_moe_layer* layer, const void* x, void* y, coli_dtype dtype, int n_tokens,
                              coli_stream stream);
@@ -177,6 +186,14 @@ coli_status coli_moe_sync(coli_moe_layer* layer);
  * separate kernels. Results agree within rounding; routing is identical.
  */
 coli_status coli_moe_set_fused(coli_moe_layer* layer, int enable);
+
+/*
+ * Selects the path for bf16 batches of more than 4 tokens: 1 (default) the
+ * tcgen05 tensor-core kernels, 0 the CUDA-core kernels. Enabling returns
+ * COLI_EUNSUPPORTED when the device, the shapes or the weight scales rule the
+ * tensor-core path out (see coli_moe_forward).
+ */
+coli_status coli_moe_set_tensor_cores(coli_moe_layer* layer, int enable);
 
 /*
  * Item timeline of the persistent decode kernel, for profiling. `buffer` is a

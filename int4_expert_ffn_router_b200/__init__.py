@@ -22,7 +22,7 @@ EXPORTS = (
     "coli_moe_layer_create", "coli_moe_layer_set_experts", "coli_moe_layer_destroy", "coli_moe_layer_config",
     "coli_moe_route", "coli_moe_forward", "coli_moe_stack_forward", "coli_moe_get_stats", "coli_moe_get_plan",
     "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
-    "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused",
+    "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused", "coli_moe_set_tensor_cores",
     "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc",
 )
 NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 64, 1024
@@ -69,6 +69,7 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_set_ring.argtypes = [vp, i32, i32]
     L.coli_moe_route_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, i32, i32, vp, vp, vp]
     L.coli_moe_set_fused.argtypes = [vp, i32]
+    L.coli_moe_set_tensor_cores.argtypes = [vp, i32]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
     L.coli_last_error.argtypes = []
@@ -177,6 +178,9 @@ class Layer:
 
     def set_fused(self, on: bool) -> None:
         _check(lib.coli_moe_set_fused(self.handle, 1 if on else 0), "coli_moe_set_fused")
+
+    def set_tensor_cores(self, on: bool) -> None:
+        _check(lib.coli_moe_set_tensor_cores(self.handle, 1 if on else 0), "coli_moe_set_tensor_cores")
 
     def set_trace(self, buffer, capacity: int) -> None:
         """Record the persistent kernel's item timeline into a zeroed device

@@ -45,6 +45,8 @@ constexpr int kBlockBytes = kNibbleBytes + kScaleBytes;  // 4352
 
 // Persistent decode kernel: tokens per launch, ring stages, control block.
 constexpr int kFusedMaxTok = 4;
+// Tensor-core path: tokens of one expert per GEMM tile (the MMA N).
+constexpr int kTcMaxTok = 128;
 constexpr int kMaxStages = 24;
 // Control block (ints in the workspace, zero between launches):
 //   [kCtlTicket] work ticket, [kCtlRouter] finished router items,

@@ -40,6 +40,26 @@ int fused_stages_for(const Dims& d, int NT, size_t smem_limit);
 constexpr int kDefaultStages = 3;  // ring stages in flight per SM (see fused_geometry)
 constexpr int kDefaultStageBlocks = 8;
 
+// prefill_tc.cu: the expert FFNs of a bf16 token batch on the tensor cores.
+// meta: [0] max over gate/up row pairs of L1(gate row) * L1(up row) (float
+// bits), [1] max |scale| (float bits); folded in per expert by launch_l1_bound
+// from the canonical container (device memory).
+cudaError_t launch_l1_bound(const uint8_t* q, const uint16_t* s, int H, int I, unsigned* meta, cudaStream_t st);
+// x16[t] = fp16(x[t] * 2^e_t), tscale[t] = {2^-e_t, 2^f_t, 2^-f_t, 0}.
+cudaError_t launch_prefill_prep(const void* x, int T, int H, const float* meta, __half* x16, float4* tscale,
+                                cudaStream_t st);
+// Per-position epilogue factors and the tile list.
+cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, const float4* tscale, float4* slot, int4* tiles,
+                                int* n_tiles, cudaStream_t st);
+// phase 0: h16 = fp16(2^f silu(G x) (U x)); phase 1: y32 += (w / 2^f) D h16.
+cudaError_t launch_prefill_gemm(int phase, const uint8_t* weights, const Dims& d, const __half* src, const Plan& p,
+                                const float4* slot, const int4* tiles, const int* n_tiles, __half* h16, float* y32,
+                                int* err, int n_sm, cudaStream_t st);
+// y = bf16(y32 (+ residual)).
+cudaError_t launch_prefill_out(const float* y32, const float* residual, int T, int H, void* y, cudaStream_t st);
+size_t prefill_tc_smem_bytes();
+int prefill_tc_max_tiles(const Dims& d, int T);
+
 // layer.cu: record the message coli_last_error() returns on this thread.
 void set_last_error(const std::string& what);
 

@@ -75,6 +75,16 @@ struct coli_moe_layer {
     float* o = nullptr;
     float* xn = nullptr;
     int* ctl = nullptr;             // control block of the persistent decode kernel
+    // tensor-core path (bf16 batches of more than kFusedMaxTok tokens)
+    __half* x16 = nullptr;          // [max_tokens][H] scaled fp16 copy of x
+    float4* tscale = nullptr;       // [max_tokens] per-token power-of-two scales
+    float4* slot = nullptr;         // [slots] per-position epilogue factors
+    int4* tiles = nullptr;          // tile list
+    int* n_tiles = nullptr;
+    unsigned* meta = nullptr;       // [0] max L1(gate row) * L1(up row), [1] max |scale| (float bits)
+    bool tc_shape_ok = false;       // shapes and shared memory allow the tensor-core kernels
+    bool tc_scale_ok = true;        // every weight scale keeps q * scale finite in fp16
+    bool use_tc = true;             // caller switch (coli_moe_set_tensor_cores)
     size_t smem_optin = 0;
     bool fused = true;              // use the persistent kernel for n_tokens <= kFusedMaxTok
     long long* trace = nullptr;     // caller-owned device buffer for the item timeline
@@ -155,7 +165,8 @@ COLI_API coli_status coli_moe_layer_set_experts(coli_moe_layer* L, int first, in
     const int H = L->d.H, I = L->d.I;
     const size_t nq = 3ull * H * I / 2, ns = 3ull * H * I / 64;
     const size_t mq = (size_t)I * H / 2, ms = (size_t)I * H / 64;
-    const bool dev_q = is_device_ptr(q), dev_s = is_device_ptr(scales);
+    // device sources are read in place when 16-byte aligned; anything else goes through the staging buffer
+    const bool dev_q = is_device_ptr(q) && ((uintptr_t)q & 15u) == 0, dev_s = is_device_ptr(scales);
     for (int i = 0; i < count; ++i) {
         const uint8_t* eq = q + (size_t)i * nq;
         const uint16_t* es = scales + (size_t)i * ns;
@@ -170,9 +181,16 @@ COLI_API coli_status coli_moe_layer_set_experts(coli_moe_layer* L, int first, in
         CUDA_TRY(launch_repack(eq, es, eq + mq, es + ms, 2 * I, H, true, dst, 0), "repack gate/up");
         CUDA_TRY(launch_repack(eq + 2 * mq, es + 2 * ms, nullptr, nullptr, H, I, false, dst + L->d.gu_bytes, 0),
                  "repack down");
+        CUDA_TRY(launch_l1_bound(eq, es, H, I, L->meta, 0), "weight bounds");
         if (!dev_q || !dev_s) CUDA_TRY(cudaDeviceSynchronize(), "repack");  // staging is reused
     }
     CUDA_TRY(cudaDeviceSynchronize(), "repack");
+    unsigned meta[2] = {0, 0};
+    CUDA_TRY(cudaMemcpy(meta, L->meta, sizeof meta, cudaMemcpyDeviceToHost), "read weight bounds");
+    float max_scale;
+    memcpy(&max_scale, &meta[1], 4);
+    // fp16 products q * scale (|q| <= 8) stay finite for |scale| <= 4096
+    L->tc_scale_ok = max_scale <= 4096.0f;
     return COLI_OK;
 }
 
@@ -225,7 +243,8 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     const size_t TK = (size_t)Tm * d.K, slots = TK + (size_t)d.S * Tm, EA = (size_t)d.E + d.S;
     size_t sz[] = {Tm * (size_t)d.E * 8, TK * 4, TK * 4, (size_t)d.E * 4, (size_t)(d.E + 1) * 4, (size_t)d.E * 4, 4,
                    TK * 4, slots * 4, EA * 4, EA * 4, EA * 4, 4, slots * d.I * 4, slots * d.H * 4, (size_t)Tm * d.H * 4,
-                   (size_t)ctl_ints(d.E, d.S, d.H, d.K) * 4, (size_t)d.E * 16};
+                   (size_t)ctl_ints(d.E, d.S, d.H, d.K) * 4, (size_t)d.E * 16, (size_t)Tm * d.H * 2, (size_t)Tm * 16,
+                   slots * 16, (size_t)prefill_tc_max_tiles(d, Tm) * 16, 4, 16};
     constexpr int kRegions = sizeof(sz) / sizeof(sz[0]);
     size_t total = 0;
     for (size_t s : sz) total += align256(s);
@@ -236,11 +255,20 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     for (int i = 0; i < kRegions; ++i) { ptrs[i] = cur; cur += align256(sz[i]); }
     L->ctl = (int*)ptrs[16];
     L->plan.table = (int4*)ptrs[17];
+    L->x16 = (__half*)ptrs[18];
+    L->tscale = (float4*)ptrs[19];
+    L->slot = (float4*)ptrs[20];
+    L->tiles = (int4*)ptrs[21];
+    L->n_tiles = (int*)ptrs[22];
+    L->meta = (unsigned*)ptrs[23];
     {
         int optin = 0;
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
         L->smem_optin = (size_t)optin;
         L->fused = fused_stages_for(d, kFusedMaxTok, L->smem_optin) >= 2;
+        int cc_major = 0;
+        cudaDeviceGetAttribute(&cc_major, cudaDevAttrComputeCapabilityMajor, device);
+        L->tc_shape_ok = cc_major == 10 && d.H % 256 == 0 && d.I % 128 == 0 && L->smem_optin >= prefill_tc_smem_bytes();
     }
     L->logits = (double*)ptrs[0];
     Plan& p = L->plan;
@@ -320,6 +348,28 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
                                      L->o, L->ctl, L->n_sm, L->smem_optin, L->trace, L->trace_cap, L->ring_stages,
                                      L->ring_blocks, s),
                  "persistent decode kernel");
+    } else if (dt == COLI_BF16 && L->use_tc && L->tc_shape_ok && L->tc_scale_ok) {
+        prof_mark(L, COLI_STAGE_ROUTER, s);
+        CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s), "router");
+        prof_mark(L, COLI_STAGE_TOPK, s);
+        CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+        prof_mark(L, COLI_STAGE_PLAN, s);
+        CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
+        prof_mark(L, COLI_STAGE_GATEUP, s);
+        __half* h16 = reinterpret_cast<__half*>(L->h);
+        CUDA_TRY(launch_prefill_prep(x, T, d.H, reinterpret_cast<const float*>(L->meta), L->x16, L->tscale, s), "prep");
+        CUDA_TRY(launch_prefill_plan(p, T, d.K, d.S, L->tscale, L->slot, L->tiles, L->n_tiles, s), "tile plan");
+        CUDA_TRY(launch_prefill_gemm(0, L->weights, d, L->x16, p, L->slot, L->tiles, L->n_tiles, h16, nullptr,
+                                     L->ctl + kCtlError, L->n_sm, s),
+                 "gate/up (tensor cores)");
+        prof_mark(L, COLI_STAGE_DOWN, s);
+        CUDA_TRY(cudaMemsetAsync(L->o, 0, (size_t)T * d.H * 4, s), "clear output");
+        CUDA_TRY(launch_prefill_gemm(1, L->weights, d, h16, p, L->slot, L->tiles, L->n_tiles, nullptr, L->o,
+                                     L->ctl + kCtlError, L->n_sm, s),
+                 "down (tensor cores)");
+        prof_mark(L, COLI_STAGE_COMBINE, s);
+        CUDA_TRY(launch_prefill_out(L->o, residual, T, d.H, y, s), "output");
+        prof_mark(L, COLI_STAGE_FUSED, s);
     } else {
         prof_mark(L, COLI_STAGE_ROUTER, s);
         CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s), "router");
@@ -393,7 +443,7 @@ static coli_status sync_and_check(coli_moe_layer* L) {
     if (err != 0) {
         CUDA_TRY(cudaMemset(L->ctl, 0, (size_t)ctl_ints(L->d.E, L->d.S, L->d.H, L->d.K) * 4), "reset control block");
         char msg[96];
-        snprintf(msg, sizeof msg, "persistent decode kernel: a bounded wait timed out (site %d)", err);
+        snprintf(msg, sizeof msg, "a bounded wait in a persistent kernel timed out (site %d)", err);
         g_last_error = msg;
         return COLI_ECUDA;
     }
@@ -412,6 +462,15 @@ COLI_API coli_status coli_moe_set_fused(coli_moe_layer* L, int enable) {
     if (enable && fused_stages_for(L->d, kFusedMaxTok, L->smem_optin) < 2)
         return fail(COLI_EUNSUPPORTED, "shapes too large for the persistent kernel's shared memory");
     L->fused = enable != 0;
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_set_tensor_cores(coli_moe_layer* L, int enable) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (enable && !L->tc_shape_ok)
+        return fail(COLI_EUNSUPPORTED, "tensor-core path needs sm_100, hidden % 256 == 0 and inter % 128 == 0");
+    if (enable && !L->tc_scale_ok) return fail(COLI_EUNSUPPORTED, "a weight scale exceeds 4096 in magnitude");
+    L->use_tc = enable != 0;
     return COLI_OK;
 }
 

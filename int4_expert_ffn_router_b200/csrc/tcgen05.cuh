@@ -1,0 +1,117 @@
+// tcgen05.cuh -- thin wrappers over the sm_100a fifth-generation tensor-core
+// instructions (PTX ISA 8.7: tcgen05.alloc/dealloc, tcgen05.mma, tcgen05.ld/st,
+// tcgen05.commit, tcgen05 fences) and the descriptors they take.
+//
+// Encodings (PTX ISA, "Instruction descriptor" and "Shared memory descriptor"
+// tables of the tcgen05 section):
+//   instruction descriptor, kind::f16, dense:
+//     bits 4-5 D format (1 = f32), bits 7-9 A format, bits 10-12 B format
+//     (0 = f16, 1 = bf16), bit 15/16 A/B major (0 = K-major), bits 17-22 N/8,
+//     bits 24-28 M/16.
+//   shared memory matrix descriptor:
+//     bits 0-13 start address / 16, bits 16-29 leading byte offset / 16,
+//     bits 32-45 stride byte offset / 16, bits 46-47 version (1),
+//     bits 49-51 base offset, bit 52 LBO mode, bits 61-63 swizzle
+//     (2 = 128-byte swizzle).
+// A K-major operand with 128-byte swizzling is stored as rows of 128 bytes
+// (64 16-bit elements), eight rows forming a 1024-byte atom in which the
+// 16-byte chunk c of row r sits at chunk position c ^ (r & 7); atoms follow
+// each other at the stride byte offset (1024). One MMA consumes 16 elements
+// (32 bytes) of K, so the k-th step advances the start address by 32 bytes.
+#pragma once
+
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace coli {
+
+__device__ __forceinline__ uint32_t tc_idesc_f16(int n, bool bf16) {
+    const uint32_t ab = bf16 ? 1u : 0u;
+    return (1u << 4) | (ab << 7) | (ab << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// K-major, 128-byte swizzled operand at shared address `saddr` (1024-aligned
+// atom base), atoms 1024 bytes apart.
+__device__ __forceinline__ uint64_t tc_sdesc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Allocation (one full warp; the column count is a power of two >= 32).
+__device__ __forceinline__ void tc_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tc_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Arrives once on `bar` when every tcgen05.mma this thread issued so far has completed.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// D[tmem d] (+)= A[tmem a] * B[smem desc]^T, M = 128, kind::f16.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Thread i of the warp writes lane (taddr.lane + i), columns taddr.col .. +15.
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Thread i reads lane (taddr.lane + i), columns taddr.col .. +15; waits for
+// the load inside the same statement so the registers are valid on return.
+__device__ __forceinline__ void tc_ld16_wait(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+// 16-byte global -> shared copy; completion tracked by the issuing thread's
+// cp.async groups or by cp_async_mbar_arrive.
+__device__ __forceinline__ void cp_async16(uint32_t dst_saddr, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_saddr), "l"(src) : "memory");
+}
+// Arrive on `bar` once this thread's earlier cp.async copies have landed
+// (the arrival is one of the barrier's expected arrivals).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t hmul2_rn(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+}  // namespace coli
