@@ -51,11 +51,15 @@ WORKLOADS = {
     # experts per token, 0.34 GB resident instead of 5.16 GB)
     "decode_b1_e16": dict(T=1, zipf=False, bf16=False, E=16,
                           desc="full-size experts, 16 routed experts top-8 + shared, decode batch 1 (profiling case)"),
+    # profiling case for the tensor-core kernels: 64 routed experts, 512 bf16
+    # tokens (about 64 tokens per expert, as in the full prefill; 1.3 GB resident)
+    "prefill_e64": dict(T=512, zipf=True, bf16=True, E=64,
+                        desc="full-size experts, 64 routed experts top-8 + shared, 512 bf16 tokens, Zipf(1.1) (profiling case)"),
 }
 X_SEED0 = 1000  # step s draws its activations with seed X_SEED0 + s
 
 
-DEFAULT_STEPS = {"decode_b1": 10000, "decode_b32": 2000, "prefill_2048": 100, "decode_b1_e16": 1000}
+DEFAULT_STEPS = {"decode_b1": 10000, "decode_b32": 2000, "prefill_2048": 100, "decode_b1_e16": 1000, "prefill_e64": 100}
 
 
 def parse():

@@ -207,6 +207,13 @@ coli_status coli_moe_set_tensor_cores(coli_moe_layer* layer, int enable);
  * stage, ns the item was published by the CTA's producer, total ns warp 0
  * waited for weight stages, 0, 0}; kind 1 router rows, 2 gate/up tile,
  * 3 down tile; times from the GPU global timer. NULL disables tracing.
+ * The tensor-core path writes, with c = (capacity - 256) / 16 when positive,
+ * the timeline of CTA 0 of its gate/up launch at int64 0 and of its down
+ * launch at int64 8c + 128: per 64-input block b < c, 8 SM clock stamps at
+ * 8b (transform warp has the block, its A stage is free, its stores issued,
+ * MMA thread has the block, has the A stage, issued; producer has the stage,
+ * issued the copies), then per work item i < 64 two stamps at 8c + 2i
+ * (epilogue start, end).
  */
 coli_status coli_moe_set_trace(coli_moe_layer* layer, void* buffer, int capacity);
 

@@ -18,9 +18,12 @@ namespace coli {
 // blocks of 128 rows x one 64-input group:
 //     block(rt, g) at ((rt * C/64) + g) * kBlockBytes
 // so the 128-row tile `rt` is one contiguous run over its groups. A block is
-//     nibbles [8 sub-tiles of 16 rows][32 lanes][16 bytes]  (4096 B)
+//     nibbles [8 sub-tiles of 16 rows][4 ti][8 gi][16 bytes]  (4096 B)
 //     scales  [8 sub-tiles][8] x {fp16 of row i, fp16 of row i+8} (256 B)
-// Lane l = 4*gi + ti of a sub-tile owns rows gi and gi+8 and, for each
+// Lane l = 4*gi + ti of a sub-tile (its 16 bytes at lane_slot(l) * 16 within
+// the sub-tile: ti-major, so the four lanes of one row lie 128 bytes apart
+// and the eight rows of one ti are 128 contiguous bytes) owns rows gi and
+// gi+8 and, for each
 // 16-input step s = 0..3 of the group, the inputs 16s + {2ti, 2ti+1, 2ti+8,
 // 2ti+9}: 32 nibbles in four 32-bit words, word s holding
 //     bits 0-3  (row gi,   col 2ti)    bits 16-19 (row gi,   col 2ti+1)
@@ -38,6 +41,8 @@ namespace coli {
 // ---------------------------------------------------------------------------
 constexpr int kGroup = 64;
 constexpr int kTileRows = 128;
+// 16-byte slot of lane l = 4*gi + ti within a 512-byte sub-tile.
+__host__ __device__ constexpr int lane_slot(int l) { return (l & 3) * 8 + (l >> 2); }
 constexpr int kSubRows = 16;
 constexpr int kNibbleBytes = 4096;
 constexpr int kScaleBytes = 256;
@@ -119,6 +124,8 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+// silu with the approximate division (relative error a few ulp)
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 }  // namespace coli
 

@@ -614,7 +614,7 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
             for (int bb = 0; bb < nb; ++bb) {
                 const int g = g0 + bb;
                 const uint8_t* bp = stage + bb * kBlockBytes;
-                const uint4 w = *reinterpret_cast<const uint4*>(bp + sub * 512 + lane * 16);
+                const uint4 w = *reinterpret_cast<const uint4*>(bp + sub * 512 + lane_slot(lane) * 16);
                 const uint32_t sv = *reinterpret_cast<const uint32_t*>(bp + kNibbleBytes + sub * 32 + gi * 4);
                 uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
                 if (has_b) {

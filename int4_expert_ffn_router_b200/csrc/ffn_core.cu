@@ -30,7 +30,7 @@ __device__ __forceinline__ void tile_dot(const uint8_t* __restrict__ tile, int G
                                          float acc0[kTB], float acc1[kTB]) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gi = lane >> 2, ti = lane & 3;
-    const uint8_t* wp = tile + warp * 512 + lane * 16;
+    const uint8_t* wp = tile + warp * 512 + lane_slot(lane) * 16;
     const uint8_t* sp = tile + kNibbleBytes + warp * 32 + gi * 4;
 #pragma unroll
     for (int tb = 0; tb < kTB; ++tb) { acc0[tb] = 0.0f; acc1[tb] = 0.0f; }

@@ -9,8 +9,10 @@
 namespace coli {
 
 // router.cu
+// part: optional scratch of part_cap doubles for split-input partial sums
+// (batches of kRouterGemmMinTok tokens and more use the blocked GEMM form).
 cudaError_t launch_router_logits(const float* wr, const float* bias, const void* x, coli_dtype dt, int T, int H, int E,
-                                 double* logits, cudaStream_t st);
+                                 double* logits, cudaStream_t st, double* part = nullptr, size_t part_cap = 0);
 cudaError_t launch_topk(const double* logits, int T, int E, int K, int32_t* ids, float* w, cudaStream_t st);
 size_t plan_smem_bytes(int E);
 cudaError_t launch_plan(const int32_t* ids, int T, int K, int E, int S, const Plan& p, cudaStream_t st);
@@ -45,16 +47,23 @@ constexpr int kDefaultStageBlocks = 8;
 // bits), [1] max |scale| (float bits); folded in per expert by launch_l1_bound
 // from the canonical container (device memory).
 cudaError_t launch_l1_bound(const uint8_t* q, const uint16_t* s, int H, int I, unsigned* meta, cudaStream_t st);
-// x16[t] = fp16(x[t] * 2^e_t), tscale[t] = {2^-e_t, 2^f_t, 2^-f_t, 0}.
-cudaError_t launch_prefill_prep(const void* x, int T, int H, const float* meta, __half* x16, float4* tscale,
-                                cudaStream_t st);
+// xs[p] = fp16(x[t] * 2^e_t) for every position p of token t (its K routed
+// positions and one per shared expert), tscale[t] = {2^-e_t, 2^f_t, 2^-f_t, 0}.
+cudaError_t launch_prefill_prep(const void* x, int T, int H, int K, int S, const int32_t* pos, const float* meta,
+                                __half* xs, float4* tscale, cudaStream_t st);
 // Per-position epilogue factors and the tile list.
 cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, const float4* tscale, float4* slot, int4* tiles,
                                 int* n_tiles, cudaStream_t st);
 // phase 0: h16 = fp16(2^f silu(G x) (U x)); phase 1: y32 += (w / 2^f) D h16.
-cudaError_t launch_prefill_gemm(int phase, const uint8_t* weights, const Dims& d, const __half* src, const Plan& p,
-                                const float4* slot, const int4* tiles, const int* n_tiles, __half* h16, float* y32,
-                                int* err, int n_sm, cudaStream_t st);
+// token_maps: host copies of two 2D tensor maps (make_token_map; boxes of
+// kTcMaxTok and 32 rows) over xs (phase 0) or h16 (phase 1).
+cudaError_t launch_prefill_gemm(int phase, const uint8_t* weights, const Dims& d, const void* token_maps,
+                                const Plan& p, const float4* slot, const int4* tiles, const int* n_tiles, __half* h16,
+                                float* y32, int* err, int n_sm, long long* trace, int trace_cap, cudaStream_t st);
+// Encodes a 2D fp16 tensor map (128 bytes, written to `map`) over
+// [rows][cols] at `base`: box 64 x box_rows, 128-byte swizzle.
+cudaError_t make_token_map(void* map, const void* base, int rows, int cols, int box_rows);
+constexpr int kTensorMapBytes = 128;
 // y = bf16(y32 (+ residual)).
 cudaError_t launch_prefill_out(const float* y32, const float* residual, int T, int H, void* y, cudaStream_t st);
 size_t prefill_tc_smem_bytes();

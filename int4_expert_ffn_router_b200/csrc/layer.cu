@@ -76,15 +76,19 @@ struct coli_moe_layer {
     float* xn = nullptr;
     int* ctl = nullptr;             // control block of the persistent decode kernel
     // tensor-core path (bf16 batches of more than kFusedMaxTok tokens)
-    __half* x16 = nullptr;          // [max_tokens][H] scaled fp16 copy of x
+    __half* xs = nullptr;           // [slots][H] scaled fp16 rows of x in position order
     float4* tscale = nullptr;       // [max_tokens] per-token power-of-two scales
     float4* slot = nullptr;         // [slots] per-position epilogue factors
     int4* tiles = nullptr;          // tile list
     int* n_tiles = nullptr;
     unsigned* meta = nullptr;       // [0] max L1(gate row) * L1(up row), [1] max |scale| (float bits)
+    double* rpart = nullptr;        // router partial sums (split input dimension)
+    size_t rpart_cap = 0;           // doubles
     bool tc_shape_ok = false;       // shapes and shared memory allow the tensor-core kernels
     bool tc_scale_ok = true;        // every weight scale keeps q * scale finite in fp16
     bool use_tc = true;             // caller switch (coli_moe_set_tensor_cores)
+    alignas(64) unsigned char xs_maps[2 * kTensorMapBytes] = {};  // TMA maps of the token operands
+    alignas(64) unsigned char h16_maps[2 * kTensorMapBytes] = {};  // (boxes of kTcMaxTok and 32 rows)
     size_t smem_optin = 0;
     bool fused = true;              // use the persistent kernel for n_tokens <= kFusedMaxTok
     long long* trace = nullptr;     // caller-owned device buffer for the item timeline
@@ -240,11 +244,13 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     if ((e = cudaMalloc(&L->router_b, (size_t)d.E * 4)) != cudaSuccess) return bail(e, "cudaMalloc(bias)");
 
     // workspace
+    const size_t TE = (size_t)Tm * d.E;
+    const size_t rpart_cap = std::min<size_t>(8 * TE, std::max<size_t>(TE, (size_t)1 << 23));
     const size_t TK = (size_t)Tm * d.K, slots = TK + (size_t)d.S * Tm, EA = (size_t)d.E + d.S;
     size_t sz[] = {Tm * (size_t)d.E * 8, TK * 4, TK * 4, (size_t)d.E * 4, (size_t)(d.E + 1) * 4, (size_t)d.E * 4, 4,
                    TK * 4, slots * 4, EA * 4, EA * 4, EA * 4, 4, slots * d.I * 4, slots * d.H * 4, (size_t)Tm * d.H * 4,
-                   (size_t)ctl_ints(d.E, d.S, d.H, d.K) * 4, (size_t)d.E * 16, (size_t)Tm * d.H * 2, (size_t)Tm * 16,
-                   slots * 16, (size_t)prefill_tc_max_tiles(d, Tm) * 16, 4, 16};
+                   (size_t)ctl_ints(d.E, d.S, d.H, d.K) * 4, (size_t)d.E * 16, slots * d.H * 2, (size_t)Tm * 16,
+                   slots * 16, (size_t)prefill_tc_max_tiles(d, Tm) * 16, 4, 16, rpart_cap * 8};
     constexpr int kRegions = sizeof(sz) / sizeof(sz[0]);
     size_t total = 0;
     for (size_t s : sz) total += align256(s);
@@ -255,12 +261,14 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     for (int i = 0; i < kRegions; ++i) { ptrs[i] = cur; cur += align256(sz[i]); }
     L->ctl = (int*)ptrs[16];
     L->plan.table = (int4*)ptrs[17];
-    L->x16 = (__half*)ptrs[18];
+    L->xs = (__half*)ptrs[18];
     L->tscale = (float4*)ptrs[19];
     L->slot = (float4*)ptrs[20];
     L->tiles = (int4*)ptrs[21];
     L->n_tiles = (int*)ptrs[22];
     L->meta = (unsigned*)ptrs[23];
+    L->rpart = (double*)ptrs[24];
+    L->rpart_cap = rpart_cap;
     {
         int optin = 0;
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
@@ -269,6 +277,16 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
         int cc_major = 0;
         cudaDeviceGetAttribute(&cc_major, cudaDevAttrComputeCapabilityMajor, device);
         L->tc_shape_ok = cc_major == 10 && d.H % 256 == 0 && d.I % 128 == 0 && L->smem_optin >= prefill_tc_smem_bytes();
+    }
+    if (L->tc_shape_ok) {
+        // xs [slots][H] and h16 [slots][I] (in the h region) as token operands
+        if (make_token_map(L->xs_maps, ptrs[18], (int)slots, d.H, kTcMaxTok) != cudaSuccess ||
+            make_token_map(L->xs_maps + kTensorMapBytes, ptrs[18], (int)slots, d.H, 32) != cudaSuccess ||
+            make_token_map(L->h16_maps, ptrs[13], (int)slots, d.I, kTcMaxTok) != cudaSuccess ||
+            make_token_map(L->h16_maps + kTensorMapBytes, ptrs[13], (int)slots, d.I, 32) != cudaSuccess) {
+            cudaGetLastError();
+            L->tc_shape_ok = false;
+        }
     }
     L->logits = (double*)ptrs[0];
     Plan& p = L->plan;
@@ -330,7 +348,7 @@ COLI_API coli_status coli_moe_route(coli_moe_layer* L, const void* x, coli_dtype
     DeviceGuard guard(L->device);
     cudaStream_t s = (cudaStream_t)stream;
     const Dims& d = L->d;
-    CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s), "router");
+    CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
     CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, ids, weights, s), "topk");
     return COLI_OK;
 }
@@ -350,29 +368,34 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
                  "persistent decode kernel");
     } else if (dt == COLI_BF16 && L->use_tc && L->tc_shape_ok && L->tc_scale_ok) {
         prof_mark(L, COLI_STAGE_ROUTER, s);
-        CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s), "router");
+        CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
         prof_mark(L, COLI_STAGE_TOPK, s);
         CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
         prof_mark(L, COLI_STAGE_GATEUP, s);
         __half* h16 = reinterpret_cast<__half*>(L->h);
-        CUDA_TRY(launch_prefill_prep(x, T, d.H, reinterpret_cast<const float*>(L->meta), L->x16, L->tscale, s), "prep");
+        CUDA_TRY(launch_prefill_prep(x, T, d.H, d.K, d.S, p.pos, reinterpret_cast<const float*>(L->meta), L->xs,
+                                     L->tscale, s),
+                 "prep");
         CUDA_TRY(launch_prefill_plan(p, T, d.K, d.S, L->tscale, L->slot, L->tiles, L->n_tiles, s), "tile plan");
-        CUDA_TRY(launch_prefill_gemm(0, L->weights, d, L->x16, p, L->slot, L->tiles, L->n_tiles, h16, nullptr,
-                                     L->ctl + kCtlError, L->n_sm, s),
+        // with a trace buffer: block timeline of the gate/up launch, then of the down launch
+        const int tcap = L->trace ? (L->trace_cap - 256) / 16 : 0;
+        CUDA_TRY(launch_prefill_gemm(0, L->weights, d, L->xs_maps, p, L->slot, L->tiles, L->n_tiles, h16, nullptr,
+                                     L->ctl + kCtlError, L->n_sm, tcap > 0 ? L->trace : nullptr, tcap, s),
                  "gate/up (tensor cores)");
         prof_mark(L, COLI_STAGE_DOWN, s);
         CUDA_TRY(cudaMemsetAsync(L->o, 0, (size_t)T * d.H * 4, s), "clear output");
-        CUDA_TRY(launch_prefill_gemm(1, L->weights, d, h16, p, L->slot, L->tiles, L->n_tiles, nullptr, L->o,
-                                     L->ctl + kCtlError, L->n_sm, s),
+        CUDA_TRY(launch_prefill_gemm(1, L->weights, d, L->h16_maps, p, L->slot, L->tiles, L->n_tiles, nullptr, L->o,
+                                     L->ctl + kCtlError, L->n_sm, tcap > 0 ? L->trace + (size_t)tcap * 8 + 128 : nullptr,
+                                     tcap, s),
                  "down (tensor cores)");
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_prefill_out(L->o, residual, T, d.H, y, s), "output");
         prof_mark(L, COLI_STAGE_FUSED, s);
     } else {
         prof_mark(L, COLI_STAGE_ROUTER, s);
-        CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s), "router");
+        CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
         prof_mark(L, COLI_STAGE_TOPK, s);
         CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
         prof_mark(L, COLI_STAGE_PLAN, s);

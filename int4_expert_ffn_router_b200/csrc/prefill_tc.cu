@@ -4,14 +4,16 @@
 // The layer (Colibrì pages: experts are three int4 matrices in 64-input
 // groups; every token goes to its top-8 experts plus the shared expert; the
 // batch reads each distinct expert once) becomes, per active expert e with
-// tokens X_e (gathered by index, never copied out):
+// tokens X_e (rows of the fp16 operand written in position order, so the
+// rows of one expert are consecutive):
 //     H_e = silu(X_e G_e^T) * (X_e U_e^T)      gate/up GEMM + SwiGLU epilogue
 //     y  += w_e * (H_e D_e^T)                   down GEMM + weighted scatter-add
 // Each GEMM runs as one persistent kernel: a work item is (token tile of up to
 // 128 tokens of one expert) x (two 128-row weight tiles). Per 64-input block:
-//   producer warps   bulk-copy the two int4 weight blocks (2 x 4352 B) and
-//                    gather the 64-element slices of the tile's token rows into
-//                    a 128-byte-swizzled K-major operand in shared memory;
+//   producer thread  bulk-copies the two int4 weight blocks (2 x 4352 B) and
+//                    loads the 64-element slices of the tile's token rows (one
+//                    TMA tile load from the position-ordered operand) into a
+//                    128-byte-swizzled K-major operand in shared memory;
 //   transform warps  dequantise one weight row per thread (exact int4 ->
 //                    fp16 via the 0x6400 magic, times the fp16 group scale,
 //                    one rounding) and store it to tensor memory;
@@ -29,6 +31,10 @@
 // product of row L1 norms, measured when the weights are loaded), so h cannot
 // overflow fp16; the down epilogue multiplies by w / 2^f. Every weight is
 // rounded once to fp16 (relative error <= 2^-11); all sums are fp32.
+#include <cuda.h>
+
+#include <cstring>
+
 #include "common.cuh"
 #include "int4_mma.cuh"
 #include "kernels.cuh"
@@ -37,14 +43,22 @@
 namespace coli {
 namespace {
 
-constexpr int kSStages = 6;                        // shared-memory stages (weights + token slices)
+constexpr int kSStages = 8;                        // shared-memory stages (weights + token slices)
 constexpr int kAStages = 4;                        // tensor-memory stages of dequantised weights
 constexpr int kBTileBytes = kTcMaxTok * 128;       // token slice: 128 rows x 64 fp16
 constexpr int kWStageBytes = 2 * kBlockBytes;      // two 128-row tiles
-constexpr int kTransformWarps = 8;
-constexpr int kProducerThreads = 64;
-constexpr int kMmaWarp = kTransformWarps + kProducerThreads / 32;  // 10
-constexpr int kThreadsTc = (kMmaWarp + 1) * 32;                     // 352
+// Transform warp w = 8 par + 4 rt2 + q dequantises rows 32q..32q+31 (its
+// TMEM lane quarter) of row tile rt2 for the blocks kb with kb % 2 == par
+// (every warp has two block periods for one block), and in the epilogue
+// handles the accumulator columns of chunks 16j..16j+15 with j % 2 == par.
+constexpr int kTransformWarps = 16;
+constexpr int kProducerWarps = 1;
+// Two MMA warps (lane 0 issues): warp kMmaWarp + t2 drives the accumulator of
+// row tile t2. One issuing thread sustains about one tcgen05.mma per 54 SM
+// clocks; two keep the tensor pipe busy down to N = 64.
+constexpr int kProducerWarp = kTransformWarps;                     // 16
+constexpr int kMmaWarp = kTransformWarps + kProducerWarps;          // 17
+constexpr int kThreadsTc = (kMmaWarp + 2) * 32;                     // 608
 constexpr uint32_t kTmemCols = 512;
 // Tensor memory columns: dequantised weights of A stage s at 64 s (+32 for
 // the second row tile; 16 fp16 of K per MMA = 8 columns), the two fp32
@@ -58,22 +72,24 @@ constexpr uint64_t kTcWaitNs = 1000000000ull;      // every wait gives up after 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int kOffB = 0;
 constexpr int kOffW = kOffB + kSStages * kBTileBytes;
-constexpr int kOffBar = kOffW + kSStages * kWStageBytes;
-constexpr int kNumBars = 2 * kSStages + 2 * kAStages + 3;
+constexpr int kOffSlot = kOffW + kSStages * kWStageBytes;          // per transform warp: its columns' factors
+constexpr int kSlotPerWarp = kTcMaxTok / 2;
+constexpr int kOffBar = kOffSlot + kTransformWarps * kSlotPerWarp * 16;
+constexpr int kNumBars = 2 * kSStages + 4 * kAStages + 6;
+static_assert((kSStages & (kSStages - 1)) == 0 && (kAStages & (kAStages - 1)) == 0, "stage counts are powers of two");
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemTc = kOffMisc + 16 + 1024;                      // + alignment slack
 static_assert(kOffBar % 8 == 0, "alignment");
-static_assert(kTcMaxTok % (kProducerThreads / 8) == 0, "producer row split");
+constexpr int kSmallBox = 32;                      // token rows per TMA load for tiles of up to 32 tokens
 
-struct TcArgs {
+struct __align__(64) TcArgs {
+    CUtensorMap tmap_big;   // 2D map over the token operand (xs or h16), box 64 x kTcMaxTok rows
+    CUtensorMap tmap_small; // the same with box 64 x kSmallBox rows (tiles of up to kSmallBox tokens)
     const uint8_t* weights;
     int64_t expert_stride;
     int64_t mat_offset;     // 0 (gate/up) or the down matrix offset within an expert
     int KB;                 // 64-input blocks per row (H/64 or I/64)
     int RT2;                // pairs of 128-row tiles
-    const __half* src;      // gate/up: x16 [T][H]; down: h16 [slots][I]
-    int src_pitch;          // elements per source row
-    const int32_t* tok;     // gate/up: token of each position
     const float4* slot;     // per position {x scale, h scale, w / h scale, token}
     const int4* tiles;      // {weight index, first position, tokens, 0}
     const int* n_tiles;
@@ -81,12 +97,27 @@ struct TcArgs {
     float* y32;             // down output [T][H] (accumulated)
     int I, H;
     int* err;               // timeout site (control block)
+    long long* trace;       // CTA 0 timeline (clock64 stamps) or NULL
+    int trace_cap;          // 64-input blocks recorded
 };
+
+// Timeline of CTA 0 (when a.trace is set): per 64-input block `it`,
+// trace[it * 8 + j] for j = 0 transform warp 0 has the block, 1 its A
+// stage is free, 2 its stores are issued, 3 MMA has the block, 4 MMA has the
+// A stage, 5 MMAs issued, 6 producer has the stage, 7 copies issued; then per
+// item i, trace[cap * 8 + 2 i] epilogue start, [.. + 1] epilogue end.
+__device__ __forceinline__ void tc_stamp(const TcArgs& a, uint32_t it, int j) {
+    if (a.trace && blockIdx.x == 0 && it < (uint32_t)a.trace_cap) a.trace[(size_t)it * 8 + j] = clock64();
+}
+__device__ __forceinline__ void tc_stamp_item(const TcArgs& a, uint32_t i, int j) {
+    if (a.trace && blockIdx.x == 0 && i < 64u) a.trace[(size_t)a.trace_cap * 8 + 2 * i + j] = clock64();
+}
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site);
 
-// All lanes of a warp wait; the warp goes on only if every lane saw the phase
-// complete, so warp-collective tcgen05 instructions stay converged.
+// Every lane polls (a one-lane poll plus broadcast costs more); the warp goes
+// on only if all lanes saw the phase complete, so warp-collective tcgen05
+// instructions stay converged.
 __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
                                              int site) {
     const bool ok = tc_wait(bar, parity, abort_flag, err, site);
@@ -108,33 +139,35 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 }
 
 template <int kPhase>
-__global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(TcArgs a) {
+__global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
-    uint64_t* full = bars;                        // [kSStages] producer -> transform/MMA
-    uint64_t* sempty = full + kSStages;           // [kSStages] MMA -> producer
-    uint64_t* aready = sempty + kSStages;         // [kAStages] transform -> MMA
-    uint64_t* aempty = aready + kAStages;         // [kAStages] MMA -> transform
-    uint64_t* accfull = aempty + kAStages;        // MMA -> epilogue
-    uint64_t* accempty = accfull + 1;             // epilogue -> MMA
-    uint64_t* drained = accempty + 1;             // MMA: all issued MMAs complete
+    uint64_t* full = bars;                        // [kSStages] producer -> transform (1 arrival + bytes)
+    uint64_t* sempty = full + kSStages;           // [kSStages] both MMA issuers -> producer
+    uint64_t* aready = sempty + kSStages;         // [kAStages][2] transform warps of tile t2 -> issuer t2
+    uint64_t* aempty = aready + 2 * kAStages;     // [kAStages][2] issuer t2 -> transform warps of tile t2
+    uint64_t* accfull = aempty + 2 * kAStages;    // [2] issuer t2 -> epilogue of tile t2
+    uint64_t* accempty = accfull + 2;             // [2] epilogue of tile t2 -> issuer t2
+    uint64_t* drained = accempty + 2;             // [2] issuer t2: all its MMAs complete
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kSStages; ++s) {
-            mbar_init(&full[s], kProducerThreads + 1);
-            mbar_init(&sempty[s], 1);
+            mbar_init(&full[s], 1);
+            mbar_init(&sempty[s], 2);
         }
-        for (int s = 0; s < kAStages; ++s) {
-            mbar_init(&aready[s], kTransformWarps);
+        for (int s = 0; s < 2 * kAStages; ++s) {
+            mbar_init(&aready[s], kTransformWarps / 4);
             mbar_init(&aempty[s], 1);
         }
-        mbar_init(accfull, 1);
-        mbar_init(accempty, kTransformWarps);
-        mbar_init(drained, 1);
+        for (int t2 = 0; t2 < 2; ++t2) {
+            mbar_init(&accfull[t2], 1);
+            mbar_init(&accempty[t2], kTransformWarps / 2);
+            mbar_init(&drained[t2], 1);
+        }
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -151,29 +184,40 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(TcArgs a)
 
     if (warp < kTransformWarps) {
         // ------------------------------------------------ transform + epilogue
-        const int q = warp & 3, rt2 = warp >> 2;
+        const int q = warp & 3, rt2 = (warp >> 2) & 1, par = warp >> 3, kh = par;
         const int m = 32 * q + lane;                 // row within the 128-row tile
         const int sub = m >> 4, gi = m & 7, isb = (m >> 3) & 1;
         const uint32_t mask = isb ? 0x00F000F0u : 0x000F000Fu;
         const uint32_t mul = isb ? 0x2C002C00u : 0x3C003C00u;   // 1/16 : 1
         const uint32_t add = isb ? 0xD480D480u : 0xE408E408u;   // -72 : -1032
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint32_t it = 0, icount = 0;
+        // factors of this warp's columns: local index (j / 2) * 16 + (c & 15) for column c of chunk j
+        float4* sinfo = reinterpret_cast<float4*>(sm + kOffSlot) + warp * kSlotPerWarp;
+        uint32_t it0 = 0, icount = 0;  // block counter at the item's first block (KB is even)
         bool ok = true;
-        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+        for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, it0 += KB) {
             const int4 tile = a.tiles[item / a.RT2];
             const int pair = item % a.RT2;
             const int n = tile.z, start = tile.y, nm = (n + 15) & ~15;
-            for (int kb = 0; kb < KB; ++kb, ++it) {
-                const int s = it % kSStages, sa = it % kAStages;
+#pragma unroll
+            for (int h = 0; h < kSlotPerWarp / 32; ++h) {
+                const int lc = lane + 32 * h;
+                const int c = 16 * (2 * (lc >> 4) + kh) + (lc & 15);
+                if (c < n) sinfo[lc] = a.slot[start + c];
+            }
+            for (int kb = par; kb < KB; kb += 2) {
+                const uint32_t it = it0 + kb;
+                const uint32_t s = it & (kSStages - 1), sa = it & (kAStages - 1);
                 if (!tc_wait_warp(&full[s], (it / kSStages) & 1, abort_flag, a.err, 21)) { ok = false; break; }
-                if (!tc_wait_warp(&aempty[sa], ((it / kAStages) & 1) ^ 1, abort_flag, a.err, 22)) { ok = false; break; }
+                if (warp == 0 && lane == 0) tc_stamp(a, it, 0);
+                if (!tc_wait_warp(&aempty[2 * sa + rt2], ((it / kAStages) & 1) ^ 1, abort_flag, a.err, 22)) { ok = false; break; }
+                if (warp == 0 && lane == 0) tc_stamp(a, it, 1);
                 tc_fence_after();
                 const uint8_t* blk = sm + kOffW + s * kWStageBytes + rt2 * kBlockBytes;
-                const uint8_t* rowp = blk + sub * 512 + gi * 64;  // lanes 4gi..4gi+3 of the sub-tile
+                const uint8_t* rowp = blk + sub * 512 + gi * 16;  // lane 4gi+ti at slot 8ti+gi
                 uint4 wv[4];
 #pragma unroll
-                for (int ti = 0; ti < 4; ++ti) wv[ti] = *reinterpret_cast<const uint4*>(rowp + 16 * ti);
+                for (int ti = 0; ti < 4; ++ti) wv[ti] = *reinterpret_cast<const uint4*>(rowp + 128 * ti);
                 const uint32_t sp = *reinterpret_cast<const uint32_t*>(blk + kNibbleBytes + sub * 32 + gi * 4);
                 const uint32_t s2 = __byte_perm(sp, 0, isb ? 0x3232 : 0x1010);
                 uint32_t r[32];
@@ -195,21 +239,24 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(TcArgs a)
                 tc_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&aready[sa]);
+                mbar_arrive_elect(&aready[2 * sa + rt2]);
+                if (warp == 0 && lane == 0) tc_stamp(a, it, 2);
             }
             if (!ok) break;
             // ---------------------------------------------------- epilogue
-            if (!tc_wait_warp(accfull, icount & 1, abort_flag, a.err, 23)) { ok = false; break; }
+            if (!tc_wait_warp(&accfull[rt2], icount & 1, abort_flag, a.err, 23)) { ok = false; break; }
+            if (warp == 0 && lane == 0) tc_stamp_item(a, icount, 0);
             tc_fence_after();
             const uint32_t tacc = tmem + lane_base + kAccBase + rt2 * kAccCols;
             const int row = (2 * pair + rt2) * 128 + m;  // row of the weight matrix
-            for (int c16 = 0; c16 < nm; c16 += 16) {
+            for (int j = kh; 16 * j < nm; j += 2) {
+                const int c16 = 16 * j, lc0 = (j >> 1) * 16;
                 uint32_t v[16];
                 tc_ld16_wait(tacc + c16, v);
                 if (kPhase == 0) {
                     // gate row (isb = 0) and up row (isb = 1) of the same h index sit 8 lanes apart:
                     // the gate lane forms h for even tokens, the up lane for odd ones.
-                    const int j = (row >> 4) * 8 + (row & 7);
+                    const int jh = (row >> 4) * 8 + (row & 7);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const float send = __uint_as_float(isb ? v[2 * i] : v[2 * i + 1]);
@@ -218,9 +265,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(TcArgs a)
                         const float u = isb ? __uint_as_float(v[2 * i + 1]) : recv;
                         const int nn = c16 + 2 * i + isb;
                         if (nn < n) {
-                            const float4 si = a.slot[start + nn];
-                            const float hv = silu_f(g * si.x) * (u * si.x);
-                            a.h16[(size_t)(start + nn) * a.I + j] = __float2half_rn(hv * si.y);
+                            const float4 si = sinfo[lc0 + 2 * i + isb];
+                            const float hv = silu_fast(g * si.x) * (u * si.x);
+                            a.h16[(size_t)(start + nn) * a.I + jh] = __float2half_rn(hv * si.y);
                         }
                     }
                 } else {
@@ -228,7 +275,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(TcArgs a)
                     for (int i = 0; i < 16; ++i) {
                         const int nn = c16 + i;
                         if (nn < n) {
-                            const float4 si = a.slot[start + nn];
+                            const float4 si = sinfo[lc0 + i];
                             const int t = __float_as_int(si.w);
                             atomicAdd(a.y32 + (size_t)t * a.H + row, __uint_as_float(v[i]) * si.z);
                         }
@@ -237,102 +284,94 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(TcArgs a)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(accempty);
+            mbar_arrive_elect(&accempty[rt2]);
+            if (warp == 0 && lane == 0) tc_stamp_item(a, icount, 1);
             ++icount;
         }
-    } else if (warp < kMmaWarp) {
+    } else if (warp == kProducerWarp) {
+      if (lane == 0) {
         // ------------------------------------------------------- producer
-        // Thread tid copies 16-byte chunk (tid & 7) of rows tid/8, tid/8 + 8, ...
-        constexpr int kRowsPer = kTcMaxTok / (kProducerThreads / 8);  // 16
-        const int tid = threadIdx.x - kTransformWarps * 32;
-        const int chunk = tid & 7, r0 = tid >> 3;
+        // Per block: the two weight blocks (bulk copies) and the tile's token
+        // rows start..start+n-1 of the position-ordered operand (one TMA
+        // tile load; rows past the tile belong to other experts or lie past
+        // the tensor, where TMA fills zeros; their columns are never read).
         uint32_t it = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const int4 tile = a.tiles[item / a.RT2];
             const int pair = item % a.RT2;
             const int n = tile.z, start = tile.y;
-            int64_t off[kRowsPer];
-#pragma unroll
-            for (int i = 0; i < kRowsPer; ++i) {
-                const int r = r0 + 8 * i;
-                off[i] = r < n ? (kPhase == 0 ? (int64_t)a.tok[start + r] : (int64_t)(start + r)) * a.src_pitch : 0;
-            }
+            const bool small = n <= kSmallBox;
+            const void* map = small ? (const void*)&a.tmap_small : (const void*)&a.tmap_big;
+            const uint32_t tx_bytes = 2 * kBlockBytes + (small ? kSmallBox : kTcMaxTok) * 128;
             const uint8_t* w0 = a.weights + (size_t)tile.x * a.expert_stride + a.mat_offset +
                                 (size_t)(2 * pair) * KB * kBlockBytes;
             const uint8_t* w1 = w0 + (size_t)KB * kBlockBytes;
             for (int kb = 0; kb < KB; ++kb, ++it) {
-                const int s = it % kSStages;
+                const uint32_t s = it & (kSStages - 1);
                 if (!tc_wait(&sempty[s], ((it / kSStages) & 1) ^ 1, abort_flag, a.err, 24)) { ok = false; break; }
+                tc_stamp(a, it, 6);
                 uint8_t* wdst = sm + kOffW + s * kWStageBytes;
-                if (tid == 0) {
-                    mbar_arrive_expect_tx(&full[s], 2 * kBlockBytes);
-                    bulk_g2s(wdst, w0 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s]);
-                    bulk_g2s(wdst + kBlockBytes, w1 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s]);
-                }
-                const uint32_t bdst = smem_addr(sm + kOffB + s * kBTileBytes) + ((r0 & 7) << 7) + ((chunk ^ (r0 & 7)) << 4);
-                const __half* src = a.src + (size_t)kb * 64 + chunk * 8;
-#pragma unroll
-                for (int i = 0; i < kRowsPer; ++i) {
-                    const int r = r0 + 8 * i;  // r & 7 == r0 & 7: same swizzle for every row of this thread
-                    if (r < n) cp_async16(bdst + (r >> 3) * 1024, src + off[i]);
-                }
-                cp_async_mbar_arrive(&full[s]);
+                mbar_arrive_expect_tx(&full[s], tx_bytes);
+                bulk_g2s(wdst, w0 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s]);
+                bulk_g2s(wdst + kBlockBytes, w1 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s]);
+                tma_load_2d(smem_addr(sm + kOffB + s * kBTileBytes), map, kb * 64, start, &full[s]);
+                tc_stamp(a, it, 7);
             }
         }
-        cp_async_wait_all();
-        if (tid == 0) {
-            // bulk copies still in flight (after an abort) must land before the CTA exits
-            const uint32_t first = it > (uint32_t)kSStages ? it - kSStages : 0;
-            const uint64_t t0 = globaltimer_ns();
-            for (uint32_t k = first; k < it; ++k) {
-                while (!mbar_try_wait(&full[k % kSStages], (k / kSStages) & 1) && globaltimer_ns() - t0 < kTcWaitNs) {
-                }
+        // copies still in flight (after an abort) must land before the CTA exits
+        const uint32_t first = it > (uint32_t)kSStages ? it - kSStages : 0;
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t k = first; k < it; ++k) {
+            while (!mbar_try_wait(&full[k % kSStages], (k / kSStages) & 1) && globaltimer_ns() - t0 < kTcWaitNs) {
             }
         }
-        __syncwarp();
+      }
+      __syncwarp();
     } else {
-      if (lane == 0) {
         // ------------------------------------------------------------ MMA
+        // issuer warp t2 (converged; one elected lane issues): accumulator of
+        // row tile t2, A from its half of each A stage
+        const int t2 = warp - kMmaWarp;
+        const uint32_t dacc = tmem + kAccBase + t2 * kAccCols;
+        const uint32_t abase = tmem + kABase + 32 * t2;
+        const uint64_t bdesc0 = tc_sdesc_sw128(smem_addr(sm + kOffB));
         uint32_t it = 0, icount = 0;
         bool ok = true, issued = false;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const int4 tile = a.tiles[item / a.RT2];
             const int nm = (tile.z + 15) & ~15;
             const uint32_t idesc = tc_idesc_f16(nm, false);
-            if (!tc_wait(accempty, (icount & 1) ^ 1, abort_flag, a.err, 25)) { ok = false; break; }
+            if (!tc_wait_warp(&accempty[t2], (icount & 1) ^ 1, abort_flag, a.err, 25)) { ok = false; break; }
             tc_fence_after();
             for (int kb = 0; kb < KB; ++kb, ++it) {
-                const int s = it % kSStages, sa = it % kAStages;
-                if (!tc_wait(&full[s], (it / kSStages) & 1, abort_flag, a.err, 26)) { ok = false; break; }
-                if (!tc_wait(&aready[sa], (it / kAStages) & 1, abort_flag, a.err, 27)) { ok = false; break; }
-                fence_proxy_async_smem();
+                const uint32_t s = it & (kSStages - 1), sa = it & (kAStages - 1);
+                // aready implies full: the transform warps waited for the stage before arriving
+                if (!tc_wait_warp(&aready[2 * sa + t2], (it / kAStages) & 1, abort_flag, a.err, 27)) { ok = false; break; }
                 tc_fence_after();
-                const uint64_t bdesc = tc_sdesc_sw128(smem_addr(sm + kOffB + s * kBTileBytes));
-#pragma unroll
-                for (int t2 = 0; t2 < 2; ++t2) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tc_mma_ts(tmem + kAccBase + t2 * kAccCols, tmem + kABase + 64 * sa + 32 * t2 + 8 * j, bdesc + 2 * j, idesc,
-                                  (kb | j) != 0);
-                }
+                const uint64_t bdesc = bdesc0 + s * (kBTileBytes >> 4);
+                const uint32_t acol = abase + 64 * sa;
+                tc_mma_ts_elect(dacc, acol, bdesc, idesc, kb != 0);
+                tc_mma_ts_elect(dacc, acol + 8, bdesc + 2, idesc, 1);
+                tc_mma_ts_elect(dacc, acol + 16, bdesc + 4, idesc, 1);
+                tc_mma_ts_elect(dacc, acol + 24, bdesc + 6, idesc, 1);
                 issued = true;
-                tc_commit(&sempty[s]);
-                tc_commit(&aempty[sa]);
+                tc_commit_elect(&sempty[s]);
+                tc_commit_elect(&aempty[2 * sa + t2]);
+                if (t2 == 0 && lane == 0) tc_stamp(a, it, 5);
             }
             if (!ok) break;
-            tc_commit(accfull);
+            tc_commit_elect(&accfull[t2]);
             ++icount;
         }
         if (issued) {
             // every MMA must complete before the tensor memory is released
-            tc_commit(drained);
+            tc_commit_elect(&drained[t2]);
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(drained, 0) && globaltimer_ns() - t0 < kTcWaitNs) {
+            while (!mbar_try_wait(&drained[t2], 0) && globaltimer_ns() - t0 < kTcWaitNs) {
             }
         }
-      }
-      __syncwarp();
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
@@ -340,9 +379,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(TcArgs a)
     if (warp == kMmaWarp) tc_dealloc(tmem, kTmemCols);
 }
 
-// One warp per token: max |x_t|, the power-of-two scales, x16 = fp16(x * 2^e).
-__global__ void prefill_prep_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, const float* __restrict__ meta,
-                                    __half* __restrict__ x16, float4* __restrict__ tscale) {
+// One warp per token: max |x_t|, the power-of-two scales, and the row
+// fp16(x_t * 2^e_t) written to every position of the token (its K routed
+// positions pos[t][k], then T*K + j*T + t for each shared expert j), so each
+// expert's tokens are consecutive rows of xs.
+__global__ void prefill_prep_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int K, int S,
+                                    const int32_t* __restrict__ pos, const float* __restrict__ meta,
+                                    __half* __restrict__ xs, float4* __restrict__ tscale) {
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (blockDim.x >> 5);
     const double bound = (double)meta[0] * (1.0 + 1e-3);  // max_j L1(gate_j) L1(up_j), with rounding margin
@@ -366,7 +409,10 @@ __global__ void prefill_prep_kernel(const __nv_bfloat16* __restrict__ x, int T, 
             const double hb = bound * (double)mx * (double)mx;
             if (hb > 0.0) f = min(120, max(-120, ilogb(16384.0 / hb)));
         }
-        uint4* out = reinterpret_cast<uint4*>(x16 + (size_t)t * H);
+        int dst[32 + 64];  // positions of this token (K <= 32 routed + S <= 64 shared)
+        const int np = K + S;
+        for (int k = 0; k < K; ++k) dst[k] = pos[(size_t)t * K + k];
+        for (int j = 0; j < S; ++j) dst[K + j] = T * K + j * T + t;
         for (int i = lane; i < H / 8; i += 32) {
             const uint4 v = row[i];
             const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -377,7 +423,8 @@ __global__ void prefill_prep_kernel(const __nv_bfloat16* __restrict__ x, int T, 
                 const __half hi = __float2half_rn(ldexpf(__uint_as_float(w[k] & 0xFFFF0000u), e));
                 o4[k] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
             }
-            out[i] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            const uint4 ov = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+            for (int q = 0; q < np; ++q) reinterpret_cast<uint4*>(xs + (size_t)dst[q] * H)[i] = ov;
         }
         if (lane == 0) tscale[t] = make_float4(ldexpf(1.0f, -e), ldexpf(1.0f, f), ldexpf(1.0f, -f), 0.0f);
     }
@@ -508,6 +555,34 @@ __global__ void scale_max_kernel(const uint16_t* __restrict__ s, size_t n, unsig
 
 size_t prefill_tc_smem_bytes() { return kSmemTc; }
 
+// 2D fp16 tensor map over rows x cols (row pitch cols * 2 bytes) for the
+// token operand: box 64 elements x box_rows rows, 128-byte swizzle.
+cudaError_t make_token_map(void* map, const void* base, int rows, int cols, int box_rows) {
+    using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeFn encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+        encode = reinterpret_cast<EncodeFn>(fn);
+    }
+    if (((uintptr_t)base & 15u) || (cols * 2) % 16 || rows < 1 || box_rows < 1 || box_rows > 256)
+        return cudaErrorInvalidValue;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(reinterpret_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 int prefill_tc_max_tiles(const Dims& d, int T) {
     return d.E + d.S + (T * d.K + d.S * T) / kTcMaxTok + 1;
 }
@@ -521,11 +596,11 @@ cudaError_t launch_l1_bound(const uint8_t* q, const uint16_t* s, int H, int I, u
     return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_prep(const void* x, int T, int H, const float* meta, __half* x16, float4* tscale,
-                                cudaStream_t st) {
+cudaError_t launch_prefill_prep(const void* x, int T, int H, int K, int S, const int32_t* pos, const float* meta,
+                                __half* xs, float4* tscale, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int grid = (T + 7) / 8 < 1184 ? (T + 7) / 8 : 1184;
-    prefill_prep_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, H, meta, x16, tscale);
+    prefill_prep_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, H, K, S, pos, meta, xs, tscale);
     return cudaGetLastError();
 }
 
@@ -535,18 +610,19 @@ cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, const float4
     return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_gemm(int phase, const uint8_t* weights, const Dims& d, const __half* src, const Plan& p,
-                                const float4* slot, const int4* tiles, const int* n_tiles, __half* h16, float* y32,
-                                int* err, int n_sm, cudaStream_t st) {
+cudaError_t launch_prefill_gemm(int phase, const uint8_t* weights, const Dims& d, const void* token_maps,
+                                const Plan& p, const float4* slot, const int4* tiles, const int* n_tiles, __half* h16,
+                                float* y32, int* err, int n_sm, long long* trace, int trace_cap, cudaStream_t st) {
     TcArgs a;
+    memcpy(&a.tmap_big, token_maps, sizeof(CUtensorMap));
+    memcpy(&a.tmap_small, static_cast<const uint8_t*>(token_maps) + sizeof(CUtensorMap), sizeof(CUtensorMap));
+    a.trace = trace;
+    a.trace_cap = trace_cap;
     a.weights = weights;
     a.expert_stride = d.expert_stride;
     a.mat_offset = phase == 0 ? 0 : d.gu_bytes;
     a.KB = phase == 0 ? d.H / kGroup : d.I / kGroup;
     a.RT2 = phase == 0 ? (2 * d.I / kTileRows) / 2 : (d.H / kTileRows) / 2;
-    a.src = src;
-    a.src_pitch = phase == 0 ? d.H : d.I;
-    a.tok = p.tok;
     a.slot = slot;
     a.tiles = tiles;
     a.n_tiles = n_tiles;

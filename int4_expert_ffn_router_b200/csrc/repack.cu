@@ -43,7 +43,7 @@ __global__ void repack_kernel(const uint8_t* __restrict__ q0, const uint16_t* __
                      ((b00 >> 4) << 16) | ((b10 >> 4) << 20) | ((b01 >> 4) << 24) | ((b11 >> 4) << 28);
         w ^= 0x88888888u;  // two's complement code q -> offset binary q + 8
         uint8_t* block = dst + (size_t)blk * kBlockBytes;
-        reinterpret_cast<uint32_t*>(block + sub * 512 + lane * 16)[s] = w;
+        reinterpret_cast<uint32_t*>(block + sub * 512 + lane_slot(lane) * 16)[s] = w;
         if (ti == 0 && s == 0) {
             const uint32_t pair = (uint32_t)sca[g] | ((uint32_t)scb[g] << 16);
             reinterpret_cast<uint32_t*>(block + kNibbleBytes + sub * 32)[gi] = pair;

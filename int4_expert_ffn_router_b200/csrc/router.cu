@@ -21,6 +21,7 @@ namespace coli {
 // four quarters are summed in a fixed order through shared memory.
 // ---------------------------------------------------------------------------
 constexpr int kRouterTok = 4;
+constexpr int kRouterGemmMinTok = 64;  // from this batch size on, the blocked GEMM form
 
 template <typename XT>
 __device__ __forceinline__ void load4(const XT* p, double v[4]);
@@ -89,6 +90,128 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const float* __restr
             double s = ((part[ew * 4 + 0][j] + part[ew * 4 + 1][j]) + part[ew * 4 + 2][j]) + part[ew * 4 + 3][j];
             logits[(size_t)(t0 + j) * E + ee] = s + (bias ? (double)bias[ee] : 0.0);
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Router logits for token batches: the same fp64 sums as a blocked GEMM.
+// CTA tile 64 tokens x 128 experts, 128 threads; thread (ty, tx) owns tokens
+// 8ty..8ty+7 and experts tx + 16j (j < 8): 64 fp64 accumulators. 16-input
+// chunks of x and Wr are widened to fp64 in shared memory (double-buffered;
+// the next chunk is fetched into registers while the current one is
+// multiplied). The input dimension may be split into `nsplit` ranges
+// (blockIdx.z) whose partial sums land in part[z] and are added in a fixed
+// order by router_reduce_kernel, so the result does not depend on timing.
+// ---------------------------------------------------------------------------
+constexpr int kRgT = 64, kRgE = 128, kRgK = 16;
+
+template <typename XT>
+__device__ __forceinline__ void rg_load8(const XT* p, float v[8]);
+template <>
+__device__ __forceinline__ void rg_load8<float>(const float* p, float v[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void rg_load8<__nv_bfloat16>(const __nv_bfloat16* p, float v[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(128) router_gemm_kernel(const float* __restrict__ wr, const float* __restrict__ bias,
+                                                          const XT* __restrict__ x, int T, int H, int E, int nsplit,
+                                                          double* __restrict__ out) {
+    __shared__ __align__(16) double xs[2][kRgK][kRgT];   // 16 KB
+    __shared__ __align__(16) double ws[2][kRgK][kRgE];   // 32 KB
+    const int tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+    const int t0 = blockIdx.x * kRgT, e0 = blockIdx.y * kRgE;
+    const int hspan = H / nsplit, h0 = blockIdx.z * hspan;
+    // loaders: x row tid/2, inputs 8 (tid & 1) .. +7; Wr row tid, inputs 0..15
+    const int xr = tid >> 1, xk = (tid & 1) * 8;
+    const bool xok = t0 + xr < T, wok = e0 + tid < E;
+    const XT* xp = x + (size_t)(xok ? t0 + xr : 0) * H + h0 + xk;
+    const float* wp = wr + (size_t)(wok ? e0 + tid : 0) * H + h0;
+    float xv[8], wv[16];
+    auto fetch = [&](int k0) {
+        if (xok) {
+            rg_load8<XT>(xp + k0, xv);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) xv[i] = 0.0f;
+        }
+        if (wok) {
+            rg_load8<float>(wp + k0, wv);
+            rg_load8<float>(wp + k0 + 8, wv + 8);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) wv[i] = 0.0f;
+        }
+    };
+    auto stash = [&](int b) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xs[b][xk + i][xr] = (double)xv[i];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ws[b][i][tid] = (double)wv[i];
+    };
+    double acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    fetch(0);
+    stash(0);
+    __syncthreads();
+    const int nk = hspan / kRgK;
+    for (int c = 0; c < nk; ++c) {
+        const int b = c & 1;
+        if (c + 1 < nk) fetch((c + 1) * kRgK);
+#pragma unroll 4
+        for (int k = 0; k < kRgK; ++k) {
+            double xr8[8], wc[8];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+                const double2 v = *reinterpret_cast<const double2*>(&xs[b][k][ty * 8 + i]);
+                xr8[i] = v.x;
+                xr8[i + 1] = v.y;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) wc[j] = ws[b][k][tx + 16 * j];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fma(xr8[i], wc[j], acc[i][j]);
+        }
+        if (c + 1 < nk) stash(b ^ 1);
+        __syncthreads();
+    }
+    double* dst = out + (size_t)blockIdx.z * T * E;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int t = t0 + ty * 8 + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = e0 + tx + 16 * j;
+            if (e < E) dst[(size_t)t * E + e] = acc[i][j] + ((nsplit == 1 && bias) ? (double)bias[e] : 0.0);
+        }
+    }
+}
+
+// logits = sum over splits s = 0, 1, ... of part[s] (in that order) + bias.
+__global__ void router_reduce_kernel(const double* __restrict__ part, const float* __restrict__ bias, int T, int E,
+                                     int nsplit, double* __restrict__ logits) {
+    const size_t n = (size_t)T * E;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        double v = part[i];
+        for (int s = 1; s < nsplit; ++s) v += part[(size_t)s * n + i];
+        logits[i] = v + (bias ? (double)bias[i % E] : 0.0);
     }
 }
 
@@ -223,8 +346,28 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
 // Host launchers.
 // ---------------------------------------------------------------------------
 cudaError_t launch_router_logits(const float* wr, const float* bias, const void* x, coli_dtype dt, int T, int H, int E,
-                                 double* logits, cudaStream_t st) {
+                                 double* logits, cudaStream_t st, double* part, size_t part_cap) {
     if (T == 0) return cudaSuccess;
+    if (T >= kRouterGemmMinTok && part && part_cap >= (size_t)T * E) {
+        // split the input dimension until about two CTAs per SM are busy
+        const int tiles = ((T + kRgT - 1) / kRgT) * ((E + kRgE - 1) / kRgE);
+        const int nk = H / kRgK;
+        int nsplit = 1;
+        for (int sp = 2; sp <= 16; ++sp)
+            if (nk % sp == 0 && (size_t)sp * T * E <= part_cap && tiles * sp <= 2 * 148) nsplit = sp;
+        dim3 g((T + kRgT - 1) / kRgT, (E + kRgE - 1) / kRgE, nsplit);
+        double* dst = nsplit == 1 ? logits : part;
+        if (dt == COLI_F32)
+            router_gemm_kernel<float><<<g, 128, 0, st>>>(wr, bias, (const float*)x, T, H, E, nsplit, dst);
+        else
+            router_gemm_kernel<__nv_bfloat16><<<g, 128, 0, st>>>(wr, bias, (const __nv_bfloat16*)x, T, H, E, nsplit, dst);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess || nsplit == 1) return e;
+        const size_t n = (size_t)T * E;
+        router_reduce_kernel<<<(int)((n + 255) / 256 < 2048 ? (n + 255) / 256 : 2048), 256, 0, st>>>(part, bias, T, E,
+                                                                                                    nsplit, logits);
+        return cudaGetLastError();
+    }
     dim3 grid((E + 1) / 2, (T + kRouterTok - 1) / kRouterTok);
     if (dt == COLI_F32)
         router_logits_kernel<float><<<grid, 256, 0, st>>>(wr, bias, (const float*)x, T, H, E, logits);

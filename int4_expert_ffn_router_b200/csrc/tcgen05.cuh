@@ -69,6 +69,30 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a, uint64_t bdesc
         : "memory");
 }
 
+// Warp-converged forms: the whole warp executes them, one elected lane
+// performs the operation (keeps the operands on the uniform datapath, which
+// is several times cheaper to issue from than a one-lane branch).
+__device__ __forceinline__ void tc_mma_ts_elect(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_elect(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_addr(bar))
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_elect(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b64 st;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_addr(bar))
+        : "memory");
+}
+
 // Thread i of the warp writes lane (taddr.lane + i), columns taddr.col .. +15.
 __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t* r) {
     asm volatile(
@@ -106,6 +130,31 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// TMA gather: rows r0..r3 of a 2D tensor map (box: one row of 128 bytes,
+// 128-byte swizzle) into 4 consecutive 128-byte rows of shared memory at
+// `dst`, completing 512 bytes of transaction on `bar`. x: innermost
+// coordinate (elements; x * element size must be a multiple of 16 bytes).
+// `tmap` must be a global, constant or __grid_constant__ parameter address.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int x, int r0, int r1, int r2, int r3,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// TMA tile load: box at (x, y) of a 2D tensor map into shared memory at
+// `dst` (1024-byte aligned for 128-byte swizzling), completing the box's
+// bytes on `bar` (out-of-bounds elements are filled with zeros and counted).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
 }
 
 __device__ __forceinline__ uint32_t hmul2_rn(uint32_t a, uint32_t b) {
