@@ -44,27 +44,28 @@ namespace coli {
 namespace {
 
 constexpr int kSStages = 8;                        // shared-memory stages (weights + token slices)
-constexpr int kAStages = 4;                        // tensor-memory stages of dequantised weights
+constexpr int kAStages = 2;                        // tensor-memory stages, each two 64-input blocks
 constexpr int kBTileBytes = kTcMaxTok * 128;       // token slice: 128 rows x 64 fp16
 constexpr int kWStageBytes = 2 * kBlockBytes;      // two 128-row tiles
-// Transform warp w = 8 par + 4 rt2 + q dequantises rows 32q..32q+31 (its
-// TMEM lane quarter) of row tile rt2 for the blocks kb with kb % 2 == par
-// (every warp has two block periods for one block), and in the epilogue
-// handles the accumulator columns of chunks 16j..16j+15 with j % 2 == par.
+// Transform warp w = 8 hb + 4 rt2 + q dequantises rows 32q..32q+31 (its
+// TMEM lane quarter) of row tile rt2 for block hb of every pair of 64-input
+// blocks (so both halves of an A stage are produced in parallel), and in the
+// epilogue handles the accumulator columns of chunks 16j..16j+15 with
+// j % 2 == hb.
 constexpr int kTransformWarps = 16;
 constexpr int kProducerWarps = 1;
-// Two MMA warps (lane 0 issues): warp kMmaWarp + t2 drives the accumulator of
-// row tile t2. One issuing thread sustains about one tcgen05.mma per 54 SM
-// clocks; two keep the tensor pipe busy down to N = 64.
+// Two MMA warps (converged, one elected lane issues): warp kMmaWarp + t2
+// drives the accumulator of row tile t2, 8 MMAs (one A stage) per wait.
 constexpr int kProducerWarp = kTransformWarps;                     // 16
 constexpr int kMmaWarp = kTransformWarps + kProducerWarps;          // 17
 constexpr int kThreadsTc = (kMmaWarp + 2) * 32;                     // 608
 constexpr uint32_t kTmemCols = 512;
-// Tensor memory columns: dequantised weights of A stage s at 64 s (+32 for
-// the second row tile; 16 fp16 of K per MMA = 8 columns), the two fp32
-// accumulators from column 256 (kTcMaxTok columns each).
+// Tensor memory columns: A stage s (two 64-input blocks of both row tiles)
+// at 128 s, + 64 t2 for row tile t2, + 32 hb for block hb of the pair (16
+// fp16 of K per MMA = 8 columns); the two fp32 accumulators from column 256
+// (kTcMaxTok columns each).
 constexpr int kABase = 0;
-constexpr int kAccBase = kAStages * 64;            // 256
+constexpr int kAccBase = kAStages * 128;           // 256
 constexpr int kAccCols = kTcMaxTok;                // accumulator of one row tile
 static_assert(kAccBase + 2 * kAccCols <= (int)kTmemCols, "tensor memory budget");
 constexpr uint64_t kTcWaitNs = 1000000000ull;      // every wait gives up after 1 s
@@ -125,10 +126,11 @@ __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, vol
 }
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site) {
-    if (mbar_try_wait(bar, parity)) return true;
+    // sleep in the barrier for up to 0.2 ms at a time; the bound stays 1 s
+    if (mbar_try_wait_sleep(bar, parity, 200000)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 200000)) return true;
         if (*abort_flag) return false;
         if (globaltimer_ns() - t0 > kTcWaitNs) {
             *abort_flag = 1;
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
             mbar_init(&sempty[s], 2);
         }
         for (int s = 0; s < 2 * kAStages; ++s) {
-            mbar_init(&aready[s], kTransformWarps / 4);
+            mbar_init(&aready[s], kTransformWarps / 2);  // 4 quarters x 2 blocks of the pair
             mbar_init(&aempty[s], 1);
         }
         for (int t2 = 0; t2 < 2; ++t2) {
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
 
     if (warp < kTransformWarps) {
         // ------------------------------------------------ transform + epilogue
-        const int q = warp & 3, rt2 = (warp >> 2) & 1, par = warp >> 3, kh = par;
+        const int q = warp & 3, rt2 = (warp >> 2) & 1, hb = warp >> 3, kh = hb;
         const int m = 32 * q + lane;                 // row within the 128-row tile
         const int sub = m >> 4, gi = m & 7, isb = (m >> 3) & 1;
         const uint32_t mask = isb ? 0x00F000F0u : 0x000F000Fu;
@@ -205,12 +207,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                 const int c = 16 * (2 * (lc >> 4) + kh) + (lc & 15);
                 if (c < n) sinfo[lc] = a.slot[start + c];
             }
-            for (int kb = par; kb < KB; kb += 2) {
+            for (int kb = hb; kb < KB; kb += 2) {
                 const uint32_t it = it0 + kb;
-                const uint32_t s = it & (kSStages - 1), sa = it & (kAStages - 1);
+                const uint32_t p2 = it >> 1;           // A stage use counter
+                const uint32_t s = it & (kSStages - 1), sa = p2 & (kAStages - 1);
                 if (!tc_wait_warp(&full[s], (it / kSStages) & 1, abort_flag, a.err, 21)) { ok = false; break; }
                 if (warp == 0 && lane == 0) tc_stamp(a, it, 0);
-                if (!tc_wait_warp(&aempty[2 * sa + rt2], ((it / kAStages) & 1) ^ 1, abort_flag, a.err, 22)) { ok = false; break; }
+                if (!tc_wait_warp(&aempty[2 * sa + rt2], ((p2 / kAStages) & 1) ^ 1, abort_flag, a.err, 22)) { ok = false; break; }
                 if (warp == 0 && lane == 0) tc_stamp(a, it, 1);
                 tc_fence_after();
                 const uint8_t* blk = sm + kOffW + s * kWStageBytes + rt2 * kBlockBytes;
@@ -233,7 +236,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                         r[8 * ws + 4 + ti] = hmul2_rn(hi, s2);  // inputs 16ws + 2ti + 8, +9
                     }
                 }
-                const uint32_t ta = tmem + lane_base + kABase + 64 * sa + 32 * rt2;
+                const uint32_t ta = tmem + lane_base + kABase + 128 * sa + 64 * rt2 + 32 * hb;
                 tc_st16(ta, r);
                 tc_st16(ta + 16, r + 16);
                 tc_wait_st();
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
         // row tile t2, A from its half of each A stage
         const int t2 = warp - kMmaWarp;
         const uint32_t dacc = tmem + kAccBase + t2 * kAccCols;
-        const uint32_t abase = tmem + kABase + 32 * t2;
+        const uint32_t abase = tmem + kABase + 64 * t2;
         const uint64_t bdesc0 = tc_sdesc_sw128(smem_addr(sm + kOffB));
         uint32_t it = 0, icount = 0;
         bool ok = true, issued = false;
@@ -344,21 +347,31 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
             const uint32_t idesc = tc_idesc_f16(nm, false);
             if (!tc_wait_warp(&accempty[t2], (icount & 1) ^ 1, abort_flag, a.err, 25)) { ok = false; break; }
             tc_fence_after();
-            for (int kb = 0; kb < KB; ++kb, ++it) {
-                const uint32_t s = it & (kSStages - 1), sa = it & (kAStages - 1);
-                // aready implies full: the transform warps waited for the stage before arriving
-                if (!tc_wait_warp(&aready[2 * sa + t2], (it / kAStages) & 1, abort_flag, a.err, 27)) { ok = false; break; }
+            for (int kb = 0; kb < KB; kb += 2, it += 2) {
+                const uint32_t p2 = it >> 1;
+                const uint32_t s0 = it & (kSStages - 1), sa = p2 & (kAStages - 1);
+                // aready implies full: the transform warps waited for both blocks' stages before arriving
+                if (!tc_wait_warp(&aready[2 * sa + t2], (p2 / kAStages) & 1, abort_flag, a.err, 27)) { ok = false; break; }
                 tc_fence_after();
-                const uint64_t bdesc = bdesc0 + s * (kBTileBytes >> 4);
-                const uint32_t acol = abase + 64 * sa;
-                tc_mma_ts_elect(dacc, acol, bdesc, idesc, kb != 0);
-                tc_mma_ts_elect(dacc, acol + 8, bdesc + 2, idesc, 1);
-                tc_mma_ts_elect(dacc, acol + 16, bdesc + 4, idesc, 1);
-                tc_mma_ts_elect(dacc, acol + 24, bdesc + 6, idesc, 1);
+                const uint64_t bd0 = bdesc0 + s0 * (kBTileBytes >> 4);
+                const uint64_t bd1 = bdesc0 + ((s0 + 1) & (kSStages - 1)) * (kBTileBytes >> 4);
+                const uint32_t acol = abase + 128 * sa;
+                tc_mma_ts_elect(dacc, acol, bd0, idesc, kb != 0);
+                tc_mma_ts_elect(dacc, acol + 8, bd0 + 2, idesc, 1);
+                tc_mma_ts_elect(dacc, acol + 16, bd0 + 4, idesc, 1);
+                tc_mma_ts_elect(dacc, acol + 24, bd0 + 6, idesc, 1);
+                tc_mma_ts_elect(dacc, acol + 32, bd1, idesc, 1);
+                tc_mma_ts_elect(dacc, acol + 40, bd1 + 2, idesc, 1);
+                tc_mma_ts_elect(dacc, acol + 48, bd1 + 4, idesc, 1);
+                tc_mma_ts_elect(dacc, acol + 56, bd1 + 6, idesc, 1);
                 issued = true;
-                tc_commit_elect(&sempty[s]);
+                tc_commit_elect(&sempty[s0]);
+                tc_commit_elect(&sempty[(s0 + 1) & (kSStages - 1)]);
                 tc_commit_elect(&aempty[2 * sa + t2]);
-                if (t2 == 0 && lane == 0) tc_stamp(a, it, 5);
+                if (t2 == 0 && lane == 0) {
+                    tc_stamp(a, it, 5);
+                    tc_stamp(a, it + 1, 5);
+                }
             }
             if (!ok) break;
             tc_commit_elect(&accfull[t2]);
