@@ -12,7 +12,7 @@ batch. Inputs are resident in HBM before the timed region; L2 is flushed
 between steps by a 256 MiB memset recorded outside the per-step events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_b1|decode_b32|prefill_2048]
+                    [--workload decode_b1|decode_b32|prefill_2048|stack30_b1|stack30_b8|stack30_b64]
 
 Prints one JSON line (rank 0). N > 1 runs N independent replicas (one per
 rank, launched by torch.distributed.run), weak scaling, max time over ranks.
@@ -55,11 +55,20 @@ WORKLOADS = {
     # tokens (about 64 tokens per expert, as in the full prefill; 1.3 GB resident)
     "prefill_e64": dict(T=512, zipf=True, bf16=True, E=64,
                         desc="full-size experts, 64 routed experts top-8 + shared, 512 bf16 tokens, Zipf(1.1) (profiling case)"),
+    # 30 full-size layers (154.8 GB of int4 experts resident), x <- x + MoE_l(RMSNorm(x)),
+    # independent seeded routers and Zipf(1.1) biases per layer, fp32 residual stream
+    "stack30_b1": dict(T=1, zipf=True, bf16=False, layers=30,
+                       desc="30-layer stack of the full-size layer, decode batch 1, Zipf(1.1) per layer"),
+    "stack30_b8": dict(T=8, zipf=True, bf16=False, layers=30,
+                       desc="30-layer stack of the full-size layer, decode batch 8, Zipf(1.1) per layer"),
+    "stack30_b64": dict(T=64, zipf=True, bf16=False, layers=30,
+                        desc="30-layer stack of the full-size layer, decode batch 64, Zipf(1.1) per layer"),
 }
 X_SEED0 = 1000  # step s draws its activations with seed X_SEED0 + s
 
 
-DEFAULT_STEPS = {"decode_b1": 10000, "decode_b32": 2000, "prefill_2048": 100, "decode_b1_e16": 1000, "prefill_e64": 100}
+DEFAULT_STEPS = {"decode_b1": 10000, "decode_b32": 2000, "prefill_2048": 100, "decode_b1_e16": 1000, "prefill_e64": 100,
+                 "stack30_b1": 300, "stack30_b8": 200, "stack30_b64": 100}
 
 
 def parse():
@@ -99,11 +108,19 @@ class OracleLeg:
         self.cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S)
         self.cache = {}
         self.Ts = wl["T"] if wl["T"] <= 2 else 2   # tokens of a step the sample covers
+        self.layers = wl.get("layers", 0)
+        if self.layers:
+            # stack: one token through the first Ls layers, time scaled to all layers
+            self.Ts, self.Ls = 1, 2
+            self.wrs = [synth.router(0, l, E, H) for l in range(self.Ls)]
+            self.biases = [synth.zipf_bias(0, l, E)[0] for l in range(self.Ls)]
 
     def step(self, i):
         """Returns (tokens, oracle seconds) of the sample of step i."""
         import numpy as np
         wl, syn = self.wl, self.synth
+        if self.layers:
+            return self._stack_step(i)
         x = syn.x_bf16(X_SEED0 + i, 0, wl["T"], H) if wl["bf16"] else syn.x_f32(X_SEED0 + i, 0, wl["T"], H)
         x = np.ascontiguousarray(x[:self.Ts])
         ids, _ = self.oracle.topk(self.oracle.router_logits(self.wr, self.bias, x), K)
@@ -116,6 +133,24 @@ class OracleLeg:
         t0 = time.perf_counter()
         self.oracle.moe_forward(self.cfg, self.wr, self.bias, experts, x)
         return self.Ts, time.perf_counter() - t0
+
+    def _stack_step(self, i):
+        import numpy as np
+        syn, orc, E = self.synth, self.oracle, self.E
+        x = np.ascontiguousarray(syn.x_f32(X_SEED0 + i, 0, self.wl["T"], H)[:1])
+        spent = 0.0
+        for l in range(self.Ls):
+            xn = orc.rmsnorm(x).astype(np.float32)  # the layer input the oracle step forms
+            ids, _ = orc.topk(orc.router_logits(self.wrs[l], self.biases[l], xn), K)
+            experts = [None] * (E + S)
+            for e in set(ids.ravel().tolist()) | set(range(E, E + S)):
+                if (l, e) not in self.cache:
+                    self.cache[(l, e)] = syn.expert(0, l, e, H, I)
+                experts[e] = self.cache[(l, e)]
+            t0 = time.perf_counter()
+            orc.stack_step(self.cfg, self.wrs[l], self.biases[l], experts, x)
+            spent += time.perf_counter() - t0
+        return 1, spent * self.layers / self.Ls
 
     def cores(self):
         return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
@@ -130,9 +165,11 @@ def oracle_sample(wl, budget_s):
         tokens += n
         spent += dt
         steps += 1
+    what = (f"{steps} steps x 1 token through the first {leg.Ls} of {leg.layers} layers (time scaled to "
+            f"{leg.layers} layers)") if leg.layers else f"{steps} steps x {leg.Ts} token(s) of the workload"
     return dict(value=round(tokens / spent, 4), unit="tokens/s", cores=leg.cores(), kind="oracle",
-                sample=f"{steps} steps x {leg.Ts} token(s) of the workload through the fp64 oracle, "
-                       f"{spent:.1f} s of oracle time (input and expert generation untimed)")
+                sample=f"{what} through the fp64 oracle, {spent:.1f} s of oracle time (input and expert "
+                       f"generation untimed)")
 
 
 # -------------------------------------------------------------------- GPU side
@@ -181,19 +218,21 @@ class Clocks:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def build_layer(torch, coli, synth, wl, device, max_tokens):
+def build_layer(torch, coli, synth, wl, device, max_tokens, layer_idx=0):
+    """Layer `layer_idx` of the workload: router, Zipf bias and experts drawn
+    with the generator's layer index."""
     E = wl.get("E", E_FULL)
     nq, ns = synth.expert_sizes(H, I)
     dev = torch.device("cuda", device)
     stream = torch.cuda.current_stream(dev).cuda_stream
     wr = torch.empty(E * H, dtype=torch.float32, device=dev)
-    synth.router_dev(0, 0, E, H, wr.data_ptr(), stream)
+    synth.router_dev(0, layer_idx, E, H, wr.data_ptr(), stream)
     q = torch.empty((E + S) * nq, dtype=torch.uint8, device=dev)
     s = torch.empty((E + S) * ns, dtype=torch.int16, device=dev)
-    synth.expert_dev(0, 0, 0, E + S, H, I, q.data_ptr(), s.data_ptr(), stream)
+    synth.expert_dev(0, layer_idx, 0, E + S, H, I, q.data_ptr(), s.data_ptr(), stream)
     bias = None
     if wl["zipf"]:
-        bias = torch.from_numpy(synth.zipf_bias(0, 0, E)[0]).to(dev)
+        bias = torch.from_numpy(synth.zipf_bias(0, layer_idx, E)[0]).to(dev)
     torch.cuda.synchronize(dev)
     cfg = coli.make_config(H, I, E, K, S, max_tokens)
     layer = coli.Layer(cfg, wr, bias, q[:E * nq], s[:E * ns], q[E * nq:], s[E * ns:], device=device)
@@ -242,7 +281,6 @@ def run_ours(args, wl, ws, rank, local):
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    layer.set_profiling(True)
     clocks = Clocks(local)
     for i in range(args.warmup, nsteps):
         ev[i][0].record(stream)
@@ -255,6 +293,12 @@ def run_ours(args, wl, ws, rank, local):
         dist.barrier()
     torch.cuda.synchronize(dev)
     step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, nsteps)]
+    # per-stage device times from a separate pass (the stage events are not in the timed region)
+    layer.set_profiling(True)
+    for i in range(args.warmup, min(nsteps, args.warmup + 200)):
+        layer.forward(xs[i], y, stream=stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
     stages, nprof = layer.profile()
     layer.set_profiling(False)
     total_ms = sum(step_ms)
@@ -331,6 +375,7 @@ def run_ours(args, wl, ws, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl["bf16"] else "f32",
+        "stage_note": "stage_us from a separate profiled pass (stage events add host gaps)",
         "data": "synthetic (seeded generator; random-init int4 weights of the full-size layer shape)",
         "config": {"workload": args.workload, "desc": wl["desc"], "hidden": H, "inter": I, "experts": wl.get("E", E_FULL),
                    "top_k": K, "shared": S, "tokens_per_step": T, "weights": "int4 gs64 + fp16 scales",
@@ -353,6 +398,146 @@ def run_ours(args, wl, ws, rank, local):
     return out
 
 
+def run_stack(args, wl, ws, rank, local):
+    """The 30-layer stack workloads: x <- x + MoE_l(RMSNorm(x)) for l = 0..L-1
+    (coli_moe_stack_forward), one step = one batch through all layers."""
+    import torch
+    import synth
+    import int4_expert_ffn_router_b200 as coli
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+    T, NL = wl["T"], wl["layers"]
+    layers = [build_layer(torch, coli, synth, wl, local, max_tokens=T, layer_idx=l) for l in range(NL)]
+    nsteps = args.warmup + args.steps
+    xs = torch.empty((nsteps, T, H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for i in range(nsteps):
+        synth.x_dev(X_SEED0 + i + 100000 * rank, 0, T, H, 0, xs[i].data_ptr(), stream.cuda_stream)
+    xw = torch.empty((T, H), dtype=torch.float32, device=dev)
+
+    # routing statistics from a few untimed steps: distinct experts per layer -> bytes
+    per_step, uniq = [], []
+    for i in range(min(4, nsteps)):
+        xw.copy_(xs[i])
+        coli.stack_forward(layers, xw, stream=stream)
+        u = [L.stats()[0] for L in layers]
+        uniq.append(sum(u) / NL)
+        per_step.append(sum((n + S) * EXPERT_BYTES + E_FULL * H * 4 for n in u))
+    mean_unique = sum(uniq) / len(uniq)
+    bytes_step = sum(per_step) / len(per_step)
+    torch.cuda.synchronize(dev)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
+    for i in range(args.warmup):
+        xw.copy_(xs[i])
+        coli.stack_forward(layers, xw, stream=stream)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = Clocks(local)
+    for i in range(args.warmup, nsteps):
+        xw.copy_(xs[i])
+        ev[i][0].record(stream)
+        coli.stack_forward(layers, xw, stream=stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    total_ms = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, nsteps))
+    # per-stage device times from a separate pass (not in the timed region)
+    for L in layers:
+        L.set_profiling(True)
+    for i in range(args.warmup, min(nsteps, args.warmup + 20)):
+        xw.copy_(xs[i])
+        coli.stack_forward(layers, xw, stream=stream)
+    torch.cuda.synchronize(dev)
+    stages = {}
+    nprof = 0
+    for L in layers:
+        st, n = L.profile()
+        nprof = n
+        for k, v in st.items():
+            stages[k] = stages.get(k, 0.0) + v
+        L.set_profiling(False)
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the C ABI with host buffers (pinned x in, result out)
+    xh = xs[args.warmup:].cpu().pin_memory()
+    yh = torch.empty((T, H), dtype=torch.float32).pin_memory()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for j in range(args.steps):
+        ev2[j][0].record(stream)
+        xw.copy_(xh[j], non_blocking=True)
+        coli.stack_forward(layers, xw, stream=stream)
+        yh.copy_(xw, non_blocking=True)
+        ev2[j][1].record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(ev2[j][0].elapsed_time(ev2[j][1]) for j in range(args.steps))
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+    for L in layers:
+        L.close()
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return None
+
+    tokens = ws * args.steps * T
+    gbs = bytes_step / (total_ms / args.steps * 1e-3) / 1e9
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except OSError:
+        pass
+    peak_gbs = peaks.get("hbm_gbs", 6650.0)
+    fused = stages.get("fused", 0.0) > 0.5 * sum(stages.values())
+    per_layer_launches = 2 if fused else (8 if T >= 64 else 7)
+    out = {
+        "metric": METRIC, "value": round(tokens / (total_ms * 1e-3), 2), "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded generator; random-init int4 weights of the full-size layer shape, per layer)",
+        "config": {"workload": args.workload, "desc": wl["desc"], "layers": NL, "hidden": H, "inter": I,
+                   "experts": E_FULL, "top_k": K, "shared": S, "tokens_per_step": T,
+                   "weights": "int4 gs64 + fp16 scales, 154.8 GB resident",
+                   "l2": f"not flushed: each step streams {bytes_step / 1e9:.2f} GB of weights (L2 is 126 MB)",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / 8000.0, 4),
+        "hbm_frac_of_measured": round(gbs / peak_gbs, 4),
+        "bytes_per_step": int(bytes_step), "unique_experts_per_layer": round(mean_unique, 2),
+        "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items()},
+        "roofline": {"bound": "hbm", "kernel": "whole stack step", "achieved": round(gbs, 1), "peak": peak_gbs,
+                     "unit": "GB/s", "frac": round(gbs / peak_gbs, 4), "traffic": None,
+                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in peaks else "fallback"},
+        "gpu_launches": per_layer_launches * NL * args.steps,
+        "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4},
+        "clocks": clk,
+    }
+    if dist:
+        dist.destroy_process_group()
+    return out
+
+
 def main():
     args = parse()
     wl = WORKLOADS[args.workload]
@@ -370,8 +555,10 @@ def main():
             total += dt
         val = tok / total
         cb = {"value": round(val, 4), "unit": "tokens/s", "cores": leg.cores(), "kind": "oracle",
-              "sample": f"{args.steps} steps, each the fp64 oracle on {leg.Ts} token(s) of the step's batch "
-                        f"(input and expert generation untimed)"}
+              "sample": (f"{args.steps} steps, each the fp64 oracle on 1 token through the first {leg.Ls} of "
+                         f"{leg.layers} layers, time scaled to {leg.layers} layers" if leg.layers else
+                         f"{args.steps} steps, each the fp64 oracle on {leg.Ts} token(s) of the step's batch") +
+                        " (input and expert generation untimed)"}
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "tokens/s",
                           "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
                           "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
@@ -386,7 +573,7 @@ def main():
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(wl, args.cpu_seconds)
-    out = run_ours(args, wl, ws, rank, local)
+    out = run_stack(args, wl, ws, rank, local) if wl.get("layers") else run_ours(args, wl, ws, rank, local)
     if out is not None:
         out["cpu_baseline"] = cpu
         print(json.dumps(out))

@@ -113,16 +113,16 @@ coli_status coli_moe_route(coli_moe_layer* layer, const void* x, coli_dtype dtyp
 /*
  * The layer: y [n_tokens][H] = MoE(x), y of the same dtype as x. x and y must
  * not overlap. Paths: n_tokens <= 4 runs the persistent decode kernel (see
- * coli_moe_set_fused); above that fp32 runs the CUDA-core kernels (fp32
- * arithmetic) and bf16 the tcgen05 tensor-core grouped GEMMs (fp16 operands:
- * tokens scaled by powers of two so the conversion is exact, weights rounded
- * once to fp16, fp32 accumulation; the combine adds with fp32 atomics, so the
- * summation order, and the last bits of y, may vary between runs). The
- * tensor-core path needs an sm_100 device, hidden % 256 == 0, inter % 128 == 0
- * and weight scales of magnitude <= 4096; otherwise bf16 also runs the CUDA-core
- * kernels. Sparse-expert forward as the Colibrì pages describe it (top-8 of
- * 256 routed experts plus the always-on shared expert, each distinct expert's
- * int4 weights read once per batch).
+ * coli_moe_set_fused). Above that, bf16 runs the tcgen05 tensor-core grouped
+ * GEMMs (fp16 operands: tokens scaled by powers of two and converted
+ * exactly, weights rounded once to fp16, fp32 accumulation; the combine adds
+ * with fp32 atomics, so the summation order, and the last bits of y, may vary
+ * between runs) and fp32 the CUDA-core kernels (fp32 arithmetic); see
+ * coli_moe_set_tensor_cores. The tensor-core path needs an sm_100 device,
+ * hidden % 256 == 0, inter % 128 == 0 and weight scales of magnitude <= 4096;
+ * otherwise bf16 also runs the CUDA-core kernels. Sparse-expert forward as the
+ * Colibrì pages describe it (top-8 of 256 routed experts plus the always-on
+ * shared expert, each distinct expert's int4 weights read once per batch).
  */
 coli_status coli_moe_forward(coli_moe_layer* layer, const void* x, void* y, coli_dtype dtype, int n_tokens,
                              coli_stream stream);
@@ -188,12 +188,15 @@ coli_status coli_moe_sync(coli_moe_layer* layer);
 coli_status coli_moe_set_fused(coli_moe_layer* layer, int enable);
 
 /*
- * Selects the path for bf16 batches of more than 4 tokens: 1 (default) the
- * tcgen05 tensor-core kernels, 0 the CUDA-core kernels. Enabling returns
- * COLI_EUNSUPPORTED when the device, the shapes or the weight scales rule the
- * tensor-core path out (see coli_moe_forward).
+ * Path for batches of more than 4 tokens: mode 0 the CUDA-core kernels for
+ * both dtypes; 1 (default) the tcgen05 tensor-core kernels for bf16; 2 the
+ * tensor cores for fp32 as well, each fp32 token entering as an fp16 hi + lo
+ * pair (about 22 bits; weights and the SwiGLU output h are fp16, so a layer's
+ * relative error is a few 1e-4 against the fp32 kernels' 1e-6). Returns
+ * COLI_EUNSUPPORTED for modes 1 and 2 when the device, the shapes or the
+ * weight scales rule the tensor-core path out.
  */
-coli_status coli_moe_set_tensor_cores(coli_moe_layer* layer, int enable);
+coli_status coli_moe_set_tensor_cores(coli_moe_layer* layer, int mode);
 
 /*
  * Item timeline of the persistent decode kernel, for profiling. `buffer` is a

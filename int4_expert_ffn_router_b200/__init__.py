@@ -179,8 +179,10 @@ class Layer:
     def set_fused(self, on: bool) -> None:
         _check(lib.coli_moe_set_fused(self.handle, 1 if on else 0), "coli_moe_set_fused")
 
-    def set_tensor_cores(self, on: bool) -> None:
-        _check(lib.coli_moe_set_tensor_cores(self.handle, 1 if on else 0), "coli_moe_set_tensor_cores")
+    def set_tensor_cores(self, mode) -> None:
+        """0 / False: CUDA-core kernels; 1 / True: tensor cores for bf16 (default);
+        2: tensor cores for fp32 too (fp16 hi + lo tokens)."""
+        _check(lib.coli_moe_set_tensor_cores(self.handle, int(mode)), "coli_moe_set_tensor_cores")
 
     def set_trace(self, buffer, capacity: int) -> None:
         """Record the persistent kernel's item timeline into a zeroed device

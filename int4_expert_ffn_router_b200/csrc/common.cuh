@@ -50,6 +50,8 @@ constexpr int kBlockBytes = kNibbleBytes + kScaleBytes;  // 4352
 
 // Persistent decode kernel: tokens per launch, ring stages, control block.
 constexpr int kFusedMaxTok = 4;
+// CUDA-core expert kernels: tokens per pass over a weight tile (one work item).
+constexpr int kCoreTok = 4;
 // Tensor-core path: tokens of one expert per GEMM tile (the MMA N).
 constexpr int kTcMaxTok = 128;
 constexpr int kMaxStages = 24;
@@ -96,6 +98,7 @@ struct Plan {
     int32_t* act_off;    // [E+S] first permuted position of active expert a
     int32_t* act_cnt;    // [E+S] tokens of active expert a
     int32_t* n_active;   // [1] n_unique + S
+    int32_t* act_chunk;  // [E+S+1] prefix of ceil(act_cnt / kCoreTok) over the active experts
     int4* table;         // [E] per distinct expert u (ascending): {expert, first position, tokens,
                          //     tokens packed 8 bits each when <= 4} (persistent decode kernel)
 };

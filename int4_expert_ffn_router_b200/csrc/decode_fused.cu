@@ -557,8 +557,8 @@ __device__ void stage_h(FusedArgs& a, FusedSmem& S, uint4* xb, const Item& it, i
 }
 
 template <typename XT, int NT>
-__device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t* ring, uint4* xb, uint32_t& slot_s,
-                            uint32_t& phase_s, int ctid) {
+__device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t* ring, uint4* xb, float4* corr,
+                            uint32_t& slot_s, uint32_t& phase_s, int ctid) {
     const Dims& d = a.d;
     const int cw = ctid >> 5, lane = ctid & 31, gi = lane >> 2, t4 = lane & 3;
     const bool gu = it.kind == IT_GU;
@@ -579,6 +579,8 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
             stage_bfrag<XT, NT>(xb, S.xscale, reinterpret_cast<const XT*>(a.x), rows, nt, C, false, ctid, kCT, 1,
                                 S.mred);
             named_bar(1, kCT);
+            stage_offset_corr(xb, corr, G, NT, nt, ctid, kCT);
+            named_bar(1, kCT);
             if (ctid == 0) {
                 S.staged_n = nt;
                 for (int i = 0; i < nt; ++i) S.staged_rows[i] = rows[i];
@@ -588,6 +590,8 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
         if (ctid == 0 && !it.ready) wait_geq(&a.ctl[kCtlGuDone + it.ex], 2 * d.I / kTileRows, abort_flag, a, 6);
         named_bar(1, kCT);
         stage_h(a, S, xb, it, ctid, NT);
+        named_bar(1, kCT);
+        stage_offset_corr(xb, corr, G, NT, nt, ctid, kCT);
         named_bar(1, kCT);
         if (ctid == 0) S.staged_n = -1;
     }
@@ -621,7 +625,7 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
                     x0 = xb[(size_t)(g * 2 + 0) * L + lane];
                     x1 = xb[(size_t)(g * 2 + 1) * L + lane];
                 }
-                group_mma_aw(w, sv, x0, x1, acc0, acc1);
+                group_mma_aw_off(w, sv, x0, x1, corr[g * 4 + t4], acc0, acc1);
             }
         }
         __syncwarp();
@@ -660,7 +664,9 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
     FusedSmem& S = *reinterpret_cast<FusedSmem*>(smem);
     uint8_t* ring = smem + ((sizeof(FusedSmem) + 127) & ~(size_t)127);
     uint4* xb = reinterpret_cast<uint4*>(ring + (size_t)a.nstages * a.sb * kBlockBytes);
-    int* scnt = reinterpret_cast<int*>(xb + (size_t)NT * (a.d.H > a.d.I ? a.d.H : a.d.I) / 4);
+    const int Cmax = a.d.H > a.d.I ? a.d.H : a.d.I;
+    float4* corr = reinterpret_cast<float4*>(xb + (size_t)NT * Cmax / 4);  // [Cmax / 64][4] offset corrections
+    int* scnt = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(corr) + Cmax);
     int* soff = scnt + a.d.E + 1;
     int* stok = soff + a.d.E + 1;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -696,7 +702,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
             if (ctid == 0) S.first_wait_ns = S.total_wait_ns = 0;
             if (it.kind == IT_ROUTER) router_item<XT, NT>(a, S, it.ex, ctid, scnt, soff, stok);
             else if (it.kind == IT_GU || it.kind == IT_DOWN)
-                weight_item<XT, NT>(a, S, it, ring, xb, slot_s, phase_s, ctid);
+                weight_item<XT, NT>(a, S, it, ring, xb, corr, slot_s, phase_s, ctid);
             // hand the completion to the signaler: the record first, then every
             // consumer thread arrives after its own global writes
             const uint32_t ds = k % kSQ;
@@ -740,7 +746,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
 size_t fused_smem_bytes(const Dims& d, int NT, int nstages, int sb) {
     const size_t head = (sizeof(FusedSmem) + 127) & ~(size_t)127;
     const int C = d.H > d.I ? d.H : d.I;
-    return head + (size_t)nstages * sb * kBlockBytes + (size_t)NT * C * 4 + (size_t)(3 * d.E + 3) * 4;
+    return head + (size_t)nstages * sb * kBlockBytes + (size_t)NT * C * 4 + (size_t)C + (size_t)(3 * d.E + 3) * 4;
 }
 
 // Ring geometry for NT tokens: copies of sb blocks (34,816 B at sb = 8: bulk

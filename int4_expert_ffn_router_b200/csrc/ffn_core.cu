@@ -6,7 +6,9 @@
 // once per batch; the batch-1 matvec in fp32 beat the int4 SIMD kernel on the
 // CPU, colibri daily, jsqmd.com, section 四 highlight 4).
 //
-// Work item = (active expert, 128-row tile). A CTA of 8 warps owns one tile;
+// Work item = (chunk of up to kTB tokens of an active expert, 128-row tile),
+// so an expert with many tokens (the shared one) spreads over many CTAs. A
+// CTA of 8 warps owns one tile;
 // warp w owns 16-row sub-tile w and streams its 512 + 32 bytes per 64-input
 // group with 128-bit non-allocating loads, NP groups in flight. Each lane
 // turns a nibble into an exact float with one LOP3 (the nibble is OR-ed into
@@ -20,7 +22,7 @@
 namespace coli {
 
 constexpr int kThreads = 256;  // 8 warps = 8 sub-tiles of one 128-row tile
-constexpr int kTB = 4;         // tokens per pass over the weights
+constexpr int kTB = kCoreTok;  // tokens per pass over the weights (one work item)
 constexpr int kNP = 8;         // groups in flight per warp
 
 // One 128-row tile of an int4 matrix times up to kTB staged input rows.
@@ -68,7 +70,18 @@ __device__ __forceinline__ void tile_dot(const uint8_t* __restrict__ tile, int G
     }
 }
 
-// Gate/up + SwiGLU. Item = (active expert a, 128-row tile rt of the [2I][H]
+// Active expert owning global chunk c: the last a with act_chunk[a] <= c.
+__device__ __forceinline__ int chunk_owner(const int32_t* __restrict__ act_chunk, int n_active, int c) {
+    int lo = 0, hi = n_active - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(act_chunk + mid) <= c) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Gate/up + SwiGLU. Item = (chunk of an active expert a, 128-row tile rt of the [2I][H]
 // interleaved gate/up matrix). h[pos][j] = silu(g_j) * u_j.
 template <typename XT>
 __global__ void __launch_bounds__(kThreads, 2) gateup_core_kernel(const uint8_t* __restrict__ weights, Dims d,
@@ -77,15 +90,18 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_core_kernel(const uint8_t*
     __shared__ int32_t rows[kTB];
     const int G = d.H / kGroup;
     const int RT = 2 * d.I / kTileRows;
-    const int n_items = *p.n_active * RT;
+    const int n_active = *p.n_active;
+    const int n_items = p.act_chunk[n_active] * RT;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gi = lane >> 2, ti = lane & 3;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int a = item / RT, rt = item - a * RT;
+        const int c = item / RT, rt = item - c * RT;
+        const int a = chunk_owner(p.act_chunk, n_active, c);
         const int ex = p.act_expert[a], off = p.act_off[a], cnt = p.act_cnt[a];
         const uint8_t* tile = weights + (size_t)ex * d.expert_stride + (size_t)rt * G * kBlockBytes;
         const int j = (rt * 8 + warp) * 8 + gi;  // gate row of this lane's row gi
-        for (int t0 = 0; t0 < cnt; t0 += kTB) {
+        const int t0 = (c - p.act_chunk[a]) * kTB;
+        {
             const int nt = min(kTB, cnt - t0);
             __syncthreads();
             if (threadIdx.x < nt) rows[threadIdx.x] = p.tok[off + t0 + threadIdx.x];
@@ -110,15 +126,18 @@ __global__ void __launch_bounds__(kThreads, 2) down_core_kernel(const uint8_t* _
     __shared__ int32_t rows[kTB];
     const int G = d.I / kGroup;
     const int RT = d.H / kTileRows;
-    const int n_items = *p.n_active * RT;
+    const int n_active = *p.n_active;
+    const int n_items = p.act_chunk[n_active] * RT;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gi = lane >> 2, ti = lane & 3;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int a = item / RT, rt = item - a * RT;
+        const int c = item / RT, rt = item - c * RT;
+        const int a = chunk_owner(p.act_chunk, n_active, c);
         const int ex = p.act_expert[a], off = p.act_off[a], cnt = p.act_cnt[a];
         const uint8_t* tile = weights + (size_t)ex * d.expert_stride + d.gu_bytes + (size_t)rt * G * kBlockBytes;
         const int r0 = rt * kTileRows + warp * kSubRows + gi;
-        for (int t0 = 0; t0 < cnt; t0 += kTB) {
+        const int t0 = (c - p.act_chunk[a]) * kTB;
+        {
             const int nt = min(kTB, cnt - t0);
             __syncthreads();
             if (threadIdx.x < nt) rows[threadIdx.x] = off + t0 + threadIdx.x;  // h is indexed by position

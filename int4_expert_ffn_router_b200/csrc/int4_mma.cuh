@@ -109,6 +109,64 @@ __device__ __forceinline__ void group_mma_aw(uint4 w, uint32_t sv, uint4 xb0, ui
     acc1 = fmaf(sc.y, d[2] + d[3], acc1);  // row gi+8
 }
 
+// As group_mma_aw, without removing the nibble offset per weight: the A
+// fragments are the raw fp16 values 1024 + v (row gi) and 1024 + 16 v (row
+// gi+8) of the offset-binary codes v = q + 8 (one logic op per pair), and the
+// accumulators start at the group's offset correction
+//     row gi:   -1032 * X,   row gi+8:  -1152 * X     (X = the column's sum of
+// the group's 64 B values), so the MMAs return sum(q x) and 16 sum(q x).
+// c = {row gi hi, row gi lo, row gi+8 hi, row gi+8 lo} corrections of token t.
+__device__ __forceinline__ void group_mma_aw_off(uint4 w, uint32_t sv, uint4 xb0, uint4 xb1, float4 c, float& acc0,
+                                                 float& acc1) {
+    float d[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    const uint32_t bx[8] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w};
+    constexpr uint32_t MAGIC = 0x64006400u;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+        const uint32_t wv = words[s], ws = wv >> 8;
+        const uint32_t r0 = lop3_and_or(wv, 0x000F000Fu, MAGIC);  // row gi,   k lo: 1024 + v
+        const uint32_t r8 = lop3_and_or(wv, 0x00F000F0u, MAGIC);  // row gi+8, k lo: 1024 + 16 v
+        const uint32_t r1 = lop3_and_or(ws, 0x000F000Fu, MAGIC);  // row gi,   k hi
+        const uint32_t r9 = lop3_and_or(ws, 0x00F000F0u, MAGIC);  // row gi+8, k hi
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(r0), "r"(r8), "r"(r1), "r"(r9), "r"(bx[2 * s]), "r"(bx[2 * s + 1]));
+    }
+    const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sv));
+    acc0 = fmaf(sc.x, d[0] + d[1], acc0);            // row gi: hi + lo columns of token t
+    acc1 = fmaf(sc.y * 0.0625f, d[2] + d[3], acc1);  // row gi+8 (values carry a factor 16)
+}
+
+// Offset corrections for group_mma_aw_off from B fragments staged as in
+// stage_bfrag: c[g * 4 + t] for token slot t < nt (zero otherwise), the
+// column sums taken in a fixed order. xb: L = 8 * NT lanes per (g, half).
+__device__ __forceinline__ void stage_offset_corr(const uint4* __restrict__ xb, float4* __restrict__ c, int G, int NT,
+                                                  int nt, int tid, int nthr) {
+    const int L = 8 * NT;
+    for (int idx = tid; idx < G * 4; idx += nthr) {
+        const int g = idx >> 2, t = idx & 3;
+        float sum[2] = {0.0f, 0.0f};
+        if (t < nt) {
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+                for (int h = 0; h < 2; ++h)
+                    for (int tt = 0; tt < 4; ++tt) {
+                        const uint4 e = xb[(size_t)(2 * g + h) * L + 4 * (2 * t + part) + tt];
+                        const uint32_t ev[4] = {e.x, e.y, e.z, e.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ev[q]));
+                            sum[part] += f.x + f.y;
+                        }
+                    }
+        }
+        c[idx] = make_float4(-1032.0f * sum[0], -1032.0f * sum[1], -1152.0f * sum[0], -1152.0f * sum[1]);
+    }
+}
+
 // 2^k as a float for k in [-126, 127].
 __device__ __forceinline__ float exp2i(int k) { return __uint_as_float((uint32_t)(127 + k) << 23); }
 

@@ -49,23 +49,26 @@ constexpr int kDefaultStageBlocks = 8;
 cudaError_t launch_l1_bound(const uint8_t* q, const uint16_t* s, int H, int I, unsigned* meta, cudaStream_t st);
 // xs[p] = fp16(x[t] * 2^e_t) for every position p of token t (its K routed
 // positions and one per shared expert), tscale[t] = {2^-e_t, 2^f_t, 2^-f_t, 0}.
-cudaError_t launch_prefill_prep(const void* x, int T, int H, int K, int S, const int32_t* pos, const float* meta,
-                                __half* xs, float4* tscale, cudaStream_t st);
+// fp32 x: two rows per position (2p hi, 2p + 1 lo).
+cudaError_t launch_prefill_prep(const void* x, coli_dtype dt, int T, int H, int K, int S, const int32_t* pos,
+                                const float* meta, __half* xs, float4* tscale, cudaStream_t st);
 // Per-position epilogue factors and the tile list.
-cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, const float4* tscale, float4* slot, int4* tiles,
-                                int* n_tiles, cudaStream_t st);
+cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, int max_tok, const float4* tscale, float4* slot,
+                                int4* tiles, int* n_tiles, cudaStream_t st);
 // phase 0: h16 = fp16(2^f silu(G x) (U x)); phase 1: y32 += (w / 2^f) D h16.
 // token_maps: host copies of two 2D tensor maps (make_token_map; boxes of
 // kTcMaxTok and 32 rows) over xs (phase 0) or h16 (phase 1).
-cudaError_t launch_prefill_gemm(int phase, const uint8_t* weights, const Dims& d, const void* token_maps,
+// pairs (phase 0): the operand holds hi and lo rows per position (fp32 input).
+cudaError_t launch_prefill_gemm(int phase, bool pairs, const uint8_t* weights, const Dims& d, const void* token_maps,
                                 const Plan& p, const float4* slot, const int4* tiles, const int* n_tiles, __half* h16,
                                 float* y32, int* err, int n_sm, long long* trace, int trace_cap, cudaStream_t st);
 // Encodes a 2D fp16 tensor map (128 bytes, written to `map`) over
 // [rows][cols] at `base`: box 64 x box_rows, 128-byte swizzle.
 cudaError_t make_token_map(void* map, const void* base, int rows, int cols, int box_rows);
 constexpr int kTensorMapBytes = 128;
-// y = bf16(y32 (+ residual)).
-cudaError_t launch_prefill_out(const float* y32, const float* residual, int T, int H, void* y, cudaStream_t st);
+// y = y32 (+ residual), stored as fp32 or bf16.
+cudaError_t launch_prefill_out(const float* y32, const float* residual, int T, int H, void* y, coli_dtype dt,
+                               cudaStream_t st);
 size_t prefill_tc_smem_bytes();
 int prefill_tc_max_tiles(const Dims& d, int T);
 

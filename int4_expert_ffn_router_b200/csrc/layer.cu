@@ -76,7 +76,7 @@ struct coli_moe_layer {
     float* xn = nullptr;
     int* ctl = nullptr;             // control block of the persistent decode kernel
     // tensor-core path (bf16 batches of more than kFusedMaxTok tokens)
-    __half* xs = nullptr;           // [slots][H] scaled fp16 rows of x in position order
+    __half* xs = nullptr;           // [2 slots][H] scaled fp16 rows of x in position order (hi, lo for fp32 x)
     float4* tscale = nullptr;       // [max_tokens] per-token power-of-two scales
     float4* slot = nullptr;         // [slots] per-position epilogue factors
     int4* tiles = nullptr;          // tile list
@@ -86,7 +86,7 @@ struct coli_moe_layer {
     size_t rpart_cap = 0;           // doubles
     bool tc_shape_ok = false;       // shapes and shared memory allow the tensor-core kernels
     bool tc_scale_ok = true;        // every weight scale keeps q * scale finite in fp16
-    bool use_tc = true;             // caller switch (coli_moe_set_tensor_cores)
+    int tc_mode = 1;                // coli_moe_set_tensor_cores: 0 CUDA cores, 1 bf16 on tensor cores, 2 bf16 and fp32
     alignas(64) unsigned char xs_maps[2 * kTensorMapBytes] = {};  // TMA maps of the token operands
     alignas(64) unsigned char h16_maps[2 * kTensorMapBytes] = {};  // (boxes of kTcMaxTok and 32 rows)
     size_t smem_optin = 0;
@@ -245,12 +245,12 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
 
     // workspace
     const size_t TE = (size_t)Tm * d.E;
-    const size_t rpart_cap = std::min<size_t>(8 * TE, std::max<size_t>(TE, (size_t)1 << 23));
+    const size_t rpart_cap = std::max<size_t>(TE, std::min<size_t>(64 * TE, (size_t)1 << 23));  // <= 64 MB unless TE is larger
     const size_t TK = (size_t)Tm * d.K, slots = TK + (size_t)d.S * Tm, EA = (size_t)d.E + d.S;
     size_t sz[] = {Tm * (size_t)d.E * 8, TK * 4, TK * 4, (size_t)d.E * 4, (size_t)(d.E + 1) * 4, (size_t)d.E * 4, 4,
                    TK * 4, slots * 4, EA * 4, EA * 4, EA * 4, 4, slots * d.I * 4, slots * d.H * 4, (size_t)Tm * d.H * 4,
-                   (size_t)ctl_ints(d.E, d.S, d.H, d.K) * 4, (size_t)d.E * 16, slots * d.H * 2, (size_t)Tm * 16,
-                   slots * 16, (size_t)prefill_tc_max_tiles(d, Tm) * 16, 4, 16, rpart_cap * 8};
+                   (size_t)ctl_ints(d.E, d.S, d.H, d.K) * 4, (size_t)d.E * 16, 2 * slots * d.H * 2, (size_t)Tm * 16,
+                   slots * 16, (size_t)prefill_tc_max_tiles(d, Tm) * 16, 4, 16, rpart_cap * 8, (EA + 1) * 4};
     constexpr int kRegions = sizeof(sz) / sizeof(sz[0]);
     size_t total = 0;
     for (size_t s : sz) total += align256(s);
@@ -268,6 +268,7 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     L->n_tiles = (int*)ptrs[22];
     L->meta = (unsigned*)ptrs[23];
     L->rpart = (double*)ptrs[24];
+    L->plan.act_chunk = (int32_t*)ptrs[25];
     L->rpart_cap = rpart_cap;
     {
         int optin = 0;
@@ -280,8 +281,8 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     }
     if (L->tc_shape_ok) {
         // xs [slots][H] and h16 [slots][I] (in the h region) as token operands
-        if (make_token_map(L->xs_maps, ptrs[18], (int)slots, d.H, kTcMaxTok) != cudaSuccess ||
-            make_token_map(L->xs_maps + kTensorMapBytes, ptrs[18], (int)slots, d.H, 32) != cudaSuccess ||
+        if (make_token_map(L->xs_maps, ptrs[18], 2 * (int)slots, d.H, kTcMaxTok) != cudaSuccess ||
+            make_token_map(L->xs_maps + kTensorMapBytes, ptrs[18], 2 * (int)slots, d.H, 32) != cudaSuccess ||
             make_token_map(L->h16_maps, ptrs[13], (int)slots, d.I, kTcMaxTok) != cudaSuccess ||
             make_token_map(L->h16_maps + kTensorMapBytes, ptrs[13], (int)slots, d.I, 32) != cudaSuccess) {
             cudaGetLastError();
@@ -366,7 +367,9 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
                                      L->o, L->ctl, L->n_sm, L->smem_optin, L->trace, L->trace_cap, L->ring_stages,
                                      L->ring_blocks, s),
                  "persistent decode kernel");
-    } else if (dt == COLI_BF16 && L->use_tc && L->tc_shape_ok && L->tc_scale_ok) {
+    } else if ((L->tc_mode == 2 || (L->tc_mode == 1 && dt == COLI_BF16)) && L->tc_shape_ok && L->tc_scale_ok) {
+        // tensor cores; fp32 tokens as fp16 hi + lo operand rows (tiles of kTcMaxTok / 2 tokens)
+        const bool pairs = dt == COLI_F32;
         prof_mark(L, COLI_STAGE_ROUTER, s);
         CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
         prof_mark(L, COLI_STAGE_TOPK, s);
@@ -375,23 +378,25 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
         prof_mark(L, COLI_STAGE_GATEUP, s);
         __half* h16 = reinterpret_cast<__half*>(L->h);
-        CUDA_TRY(launch_prefill_prep(x, T, d.H, d.K, d.S, p.pos, reinterpret_cast<const float*>(L->meta), L->xs,
+        CUDA_TRY(launch_prefill_prep(x, dt, T, d.H, d.K, d.S, p.pos, reinterpret_cast<const float*>(L->meta), L->xs,
                                      L->tscale, s),
                  "prep");
-        CUDA_TRY(launch_prefill_plan(p, T, d.K, d.S, L->tscale, L->slot, L->tiles, L->n_tiles, s), "tile plan");
+        CUDA_TRY(launch_prefill_plan(p, T, d.K, d.S, pairs ? kTcMaxTok / 2 : kTcMaxTok, L->tscale, L->slot, L->tiles,
+                                     L->n_tiles, s),
+                 "tile plan");
         // with a trace buffer: block timeline of the gate/up launch, then of the down launch
         const int tcap = L->trace ? (L->trace_cap - 256) / 16 : 0;
-        CUDA_TRY(launch_prefill_gemm(0, L->weights, d, L->xs_maps, p, L->slot, L->tiles, L->n_tiles, h16, nullptr,
+        CUDA_TRY(launch_prefill_gemm(0, pairs, L->weights, d, L->xs_maps, p, L->slot, L->tiles, L->n_tiles, h16, nullptr,
                                      L->ctl + kCtlError, L->n_sm, tcap > 0 ? L->trace : nullptr, tcap, s),
                  "gate/up (tensor cores)");
         prof_mark(L, COLI_STAGE_DOWN, s);
         CUDA_TRY(cudaMemsetAsync(L->o, 0, (size_t)T * d.H * 4, s), "clear output");
-        CUDA_TRY(launch_prefill_gemm(1, L->weights, d, L->h16_maps, p, L->slot, L->tiles, L->n_tiles, nullptr, L->o,
-                                     L->ctl + kCtlError, L->n_sm, tcap > 0 ? L->trace + (size_t)tcap * 8 + 128 : nullptr,
-                                     tcap, s),
+        CUDA_TRY(launch_prefill_gemm(1, false, L->weights, d, L->h16_maps, p, L->slot, L->tiles, L->n_tiles, nullptr,
+                                     L->o, L->ctl + kCtlError, L->n_sm,
+                                     tcap > 0 ? L->trace + (size_t)tcap * 8 + 128 : nullptr, tcap, s),
                  "down (tensor cores)");
         prof_mark(L, COLI_STAGE_COMBINE, s);
-        CUDA_TRY(launch_prefill_out(L->o, residual, T, d.H, y, s), "output");
+        CUDA_TRY(launch_prefill_out(L->o, residual, T, d.H, y, dt, s), "output");
         prof_mark(L, COLI_STAGE_FUSED, s);
     } else {
         prof_mark(L, COLI_STAGE_ROUTER, s);
@@ -488,12 +493,13 @@ COLI_API coli_status coli_moe_set_fused(coli_moe_layer* L, int enable) {
     return COLI_OK;
 }
 
-COLI_API coli_status coli_moe_set_tensor_cores(coli_moe_layer* L, int enable) {
+COLI_API coli_status coli_moe_set_tensor_cores(coli_moe_layer* L, int mode) {
     if (!L) return fail(COLI_EINVAL, "layer is NULL");
-    if (enable && !L->tc_shape_ok)
+    if (mode < 0 || mode > 2) return fail(COLI_EINVAL, "mode must be 0, 1 or 2");
+    if (mode && !L->tc_shape_ok)
         return fail(COLI_EUNSUPPORTED, "tensor-core path needs sm_100, hidden % 256 == 0 and inter % 128 == 0");
-    if (enable && !L->tc_scale_ok) return fail(COLI_EUNSUPPORTED, "a weight scale exceeds 4096 in magnitude");
-    L->use_tc = enable != 0;
+    if (mode && !L->tc_scale_ok) return fail(COLI_EUNSUPPORTED, "a weight scale exceeds 4096 in magnitude");
+    L->tc_mode = mode;
     return COLI_OK;
 }
 

@@ -140,7 +140,10 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
     }
 }
 
-template <int kPhase>
+// kPairs (gate/up only): the token operand holds two fp16 rows per position,
+// hi and lo parts of an fp32 input; the MMA columns 2i and 2i+1 of a tile are
+// the two parts of its token i and the epilogue adds them.
+template <int kPhase, bool kPairs>
 __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __grid_constant__ TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -200,12 +203,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, it0 += KB) {
             const int4 tile = a.tiles[item / a.RT2];
             const int pair = item % a.RT2;
-            const int n = tile.z, start = tile.y, nm = (n + 15) & ~15;
+            const int n = tile.z, start = tile.y;
+            const int ncol = kPairs ? 2 * n : n, nm = (ncol + 15) & ~15;  // MMA columns
+            constexpr int kTokPerChunk = kPairs ? 8 : 16;                    // tokens per 16 columns
 #pragma unroll
             for (int h = 0; h < kSlotPerWarp / 32; ++h) {
-                const int lc = lane + 32 * h;
-                const int c = 16 * (2 * (lc >> 4) + kh) + (lc & 15);
-                if (c < n) sinfo[lc] = a.slot[start + c];
+                const int lc = lane + 32 * h;  // local index (j / 2) * kTokPerChunk + i for token i of chunk j
+                const int c = kTokPerChunk * (2 * (lc / kTokPerChunk) + kh) + (lc % kTokPerChunk);
+                if (c < n && lc < (kSlotPerWarp / 16) * kTokPerChunk) sinfo[lc] = a.slot[start + c];
             }
             for (int kb = hb; kb < KB; kb += 2) {
                 const uint32_t it = it0 + kb;
@@ -256,7 +261,28 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                 const int c16 = 16 * j, lc0 = (j >> 1) * 16;
                 uint32_t v[16];
                 tc_ld16_wait(tacc + c16, v);
-                if (kPhase == 0) {
+                if (kPhase == 0 && kPairs) {
+                    // columns 2i, 2i+1: hi and lo parts of token c16/2 + i. The gate lane (isb = 0)
+                    // forms h for tokens 0..3 of the chunk, the up lane (isb = 1) for 4..7.
+                    const int jh = (row >> 4) * 8 + (row & 7);
+                    float tv[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) tv[i] = __uint_as_float(v[2 * i]) + __uint_as_float(v[2 * i + 1]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float send = isb ? tv[i] : tv[4 + i];
+                        const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+                        const float g = isb ? recv : tv[i];
+                        const float u = isb ? tv[4 + i] : recv;
+                        const int ti = 4 * isb + i;          // token within the chunk
+                        const int nn = c16 / 2 + ti;
+                        if (nn < n) {
+                            const float4 si = sinfo[(j >> 1) * 8 + ti];
+                            const float hv = silu_fast(g * si.x) * (u * si.x);
+                            a.h16[(size_t)(start + nn) * a.I + jh] = __float2half_rn(hv * si.y);
+                        }
+                    }
+                } else if (kPhase == 0) {
                     // gate row (isb = 0) and up row (isb = 1) of the same h index sit 8 lanes apart:
                     // the gate lane forms h for even tokens, the up lane for odd ones.
                     const int jh = (row >> 4) * 8 + (row & 7);
@@ -304,7 +330,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
             const int4 tile = a.tiles[item / a.RT2];
             const int pair = item % a.RT2;
             const int n = tile.z, start = tile.y;
-            const bool small = n <= kSmallBox;
+            const int rows = kPairs ? 2 * n : n, row0 = kPairs ? 2 * start : start;
+            const bool small = rows <= kSmallBox;
             const void* map = small ? (const void*)&a.tmap_small : (const void*)&a.tmap_big;
             const uint32_t tx_bytes = 2 * kBlockBytes + (small ? kSmallBox : kTcMaxTok) * 128;
             const uint8_t* w0 = a.weights + (size_t)tile.x * a.expert_stride + a.mat_offset +
@@ -318,7 +345,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                 mbar_arrive_expect_tx(&full[s], tx_bytes);
                 bulk_g2s(wdst, w0 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s]);
                 bulk_g2s(wdst + kBlockBytes, w1 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s]);
-                tma_load_2d(smem_addr(sm + kOffB + s * kBTileBytes), map, kb * 64, start, &full[s]);
+                tma_load_2d(smem_addr(sm + kOffB + s * kBTileBytes), map, kb * 64, row0, &full[s]);
                 tc_stamp(a, it, 7);
             }
         }
@@ -343,7 +370,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
         bool ok = true, issued = false;
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const int4 tile = a.tiles[item / a.RT2];
-            const int nm = (tile.z + 15) & ~15;
+            const int nm = ((kPairs ? 2 * tile.z : tile.z) + 15) & ~15;
             const uint32_t idesc = tc_idesc_f16(nm, false);
             if (!tc_wait_warp(&accempty[t2], (icount & 1) ^ 1, abort_flag, a.err, 25)) { ok = false; break; }
             tc_fence_after();
@@ -395,24 +422,40 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
 // One warp per token: max |x_t|, the power-of-two scales, and the row
 // fp16(x_t * 2^e_t) written to every position of the token (its K routed
 // positions pos[t][k], then T*K + j*T + t for each shared expert j), so each
-// expert's tokens are consecutive rows of xs.
-__global__ void prefill_prep_kernel(const __nv_bfloat16* __restrict__ x, int T, int H, int K, int S,
+// expert's tokens are consecutive rows of xs. bf16 input: one row per
+// position (exact). fp32 input: two rows per position, 2p = hi = fp16(x 2^e)
+// and 2p+1 = lo = fp16(x 2^e - hi), about 22 significant bits together.
+template <typename XT>
+__global__ void prefill_prep_kernel(const XT* __restrict__ x, int T, int H, int K, int S,
                                     const int32_t* __restrict__ pos, const float* __restrict__ meta,
                                     __half* __restrict__ xs, float4* __restrict__ tscale) {
+    constexpr bool kF32 = sizeof(XT) == 4;
+    constexpr int kV = 8;  // elements per lane per step (16 bytes of bf16, 32 of fp32)
     const int lane = threadIdx.x & 31;
     const int nwarps = gridDim.x * (blockDim.x >> 5);
     const double bound = (double)meta[0] * (1.0 + 1e-3);  // max_j L1(gate_j) L1(up_j), with rounding margin
-    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
-        const uint4* row = reinterpret_cast<const uint4*>(x + (size_t)t * H);
-        float mx = 0.0f;
-        for (int i = lane; i < H / 8; i += 32) {
-            const uint4 v = row[i];
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    auto load8 = [&](const XT* p, float v[kV]) {
+        if constexpr (kF32) {
+            const float4 a0 = reinterpret_cast<const float4*>(p)[0], a1 = reinterpret_cast<const float4*>(p)[1];
+            v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w; v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
+        } else {
+            const uint4 u = *reinterpret_cast<const uint4*>(p);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                mx = fmaxf(mx, fabsf(__uint_as_float(w[k] << 16)));
-                mx = fmaxf(mx, fabsf(__uint_as_float(w[k] & 0xFFFF0000u)));
+                v[2 * k] = __uint_as_float(w[k] << 16);
+                v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
             }
+        }
+    };
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
+        const XT* row = x + (size_t)t * H;
+        float mx = 0.0f;
+        for (int i = lane * kV; i < H; i += 32 * kV) {
+            float v[kV];
+            load8(row + i, v);
+#pragma unroll
+            for (int k = 0; k < kV; ++k) mx = fmaxf(mx, fabsf(v[k]));
         }
 #pragma unroll
         for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -426,18 +469,30 @@ __global__ void prefill_prep_kernel(const __nv_bfloat16* __restrict__ x, int T, 
         const int np = K + S;
         for (int k = 0; k < K; ++k) dst[k] = pos[(size_t)t * K + k];
         for (int j = 0; j < S; ++j) dst[K + j] = T * K + j * T + t;
-        for (int i = lane; i < H / 8; i += 32) {
-            const uint4 v = row[i];
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            uint32_t o4[4];
+        for (int i = lane * kV; i < H; i += 32 * kV) {
+            float v[kV];
+            load8(row + i, v);
+            uint32_t hi4[4], lo4[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const __half lo = __float2half_rn(ldexpf(__uint_as_float(w[k] << 16), e));
-                const __half hi = __float2half_rn(ldexpf(__uint_as_float(w[k] & 0xFFFF0000u), e));
-                o4[k] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+                const float a0 = ldexpf(v[2 * k], e), a1 = ldexpf(v[2 * k + 1], e);
+                const __half h0 = __float2half_rn(a0), h1 = __float2half_rn(a1);
+                hi4[k] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+                if constexpr (kF32) {
+                    const __half l0 = __float2half_rn(a0 - __half2float(h0)), l1 = __float2half_rn(a1 - __half2float(h1));
+                    lo4[k] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+                }
             }
-            const uint4 ov = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-            for (int q = 0; q < np; ++q) reinterpret_cast<uint4*>(xs + (size_t)dst[q] * H)[i] = ov;
+            const uint4 hv = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+            for (int q = 0; q < np; ++q) {
+                if constexpr (kF32) {
+                    reinterpret_cast<uint4*>(xs + (size_t)(2 * dst[q]) * H + i)[0] = hv;
+                    reinterpret_cast<uint4*>(xs + (size_t)(2 * dst[q] + 1) * H + i)[0] =
+                        make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+                } else {
+                    reinterpret_cast<uint4*>(xs + (size_t)dst[q] * H + i)[0] = hv;
+                }
+            }
         }
         if (lane == 0) tscale[t] = make_float4(ldexpf(1.0f, -e), ldexpf(1.0f, f), ldexpf(1.0f, -f), 0.0f);
     }
@@ -445,7 +500,8 @@ __global__ void prefill_prep_kernel(const __nv_bfloat16* __restrict__ x, int T, 
 
 // Per-position epilogue factors and the tile list (one CTA). Tiles hold at
 // most kTcMaxTok tokens of one expert and are ordered by decreasing size.
-__global__ void __launch_bounds__(1024) prefill_plan_kernel(Plan p, int T, int K, int S, const float4* __restrict__ tscale,
+__global__ void __launch_bounds__(1024) prefill_plan_kernel(Plan p, int T, int K, int S, int max_tok,
+                                                            const float4* __restrict__ tscale,
                                                             float4* __restrict__ slot, int4* __restrict__ tiles,
                                                             int* __restrict__ n_tiles) {
     __shared__ int bcnt[kTcMaxTok / 16], bbase[kTcMaxTok / 16], bcur[kTcMaxTok / 16];
@@ -468,7 +524,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(Plan p, int T, int K
         for (int u = threadIdx.x; u < na; u += blockDim.x) {
             const int cnt = p.act_cnt[u];
             if (cnt <= 0) continue;
-            const int nt = (cnt + kTcMaxTok - 1) / kTcMaxTok;
+            const int nt = (cnt + max_tok - 1) / max_tok;
             const int sz = (cnt + nt - 1) / nt;
             for (int j = 0; j < nt; ++j) {
                 const int n = min(sz, cnt - j * sz);
@@ -495,19 +551,24 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(Plan p, int T, int K
     }
 }
 
+template <typename YT>
 __global__ void prefill_out_kernel(const float* __restrict__ y32, const float* __restrict__ residual, size_t n,
-                                   __nv_bfloat16* __restrict__ y) {
+                                   YT* __restrict__ y) {
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n / 4; i += (size_t)gridDim.x * blockDim.x) {
         float4 v = reinterpret_cast<const float4*>(y32)[i];
         if (residual) {
             const float4 r = reinterpret_cast<const float4*>(residual)[i];
             v.x += r.x; v.y += r.y; v.z += r.z; v.w += r.w;
         }
-        __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-        uint2 o;
-        o.x = *reinterpret_cast<uint32_t*>(&lo);
-        o.y = *reinterpret_cast<uint32_t*>(&hi);
-        reinterpret_cast<uint2*>(y)[i] = o;
+        if constexpr (sizeof(YT) == 4) {
+            reinterpret_cast<float4*>(y)[i] = v;
+        } else {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+            uint2 o;
+            o.x = *reinterpret_cast<uint32_t*>(&lo);
+            o.y = *reinterpret_cast<uint32_t*>(&hi);
+            reinterpret_cast<uint2*>(y)[i] = o;
+        }
     }
 }
 
@@ -609,21 +670,25 @@ cudaError_t launch_l1_bound(const uint8_t* q, const uint16_t* s, int H, int I, u
     return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_prep(const void* x, int T, int H, int K, int S, const int32_t* pos, const float* meta,
-                                __half* xs, float4* tscale, cudaStream_t st) {
+cudaError_t launch_prefill_prep(const void* x, coli_dtype dt, int T, int H, int K, int S, const int32_t* pos,
+                                const float* meta, __half* xs, float4* tscale, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int grid = (T + 7) / 8 < 1184 ? (T + 7) / 8 : 1184;
-    prefill_prep_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, H, K, S, pos, meta, xs, tscale);
+    if (dt == COLI_F32)
+        prefill_prep_kernel<float><<<grid, 256, 0, st>>>((const float*)x, T, H, K, S, pos, meta, xs, tscale);
+    else
+        prefill_prep_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, T, H, K, S, pos, meta, xs,
+                                                                 tscale);
     return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, const float4* tscale, float4* slot, int4* tiles,
-                                int* n_tiles, cudaStream_t st) {
-    prefill_plan_kernel<<<1, 1024, 0, st>>>(p, T, K, S, tscale, slot, tiles, n_tiles);
+cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, int max_tok, const float4* tscale, float4* slot,
+                                int4* tiles, int* n_tiles, cudaStream_t st) {
+    prefill_plan_kernel<<<1, 1024, 0, st>>>(p, T, K, S, max_tok, tscale, slot, tiles, n_tiles);
     return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_gemm(int phase, const uint8_t* weights, const Dims& d, const void* token_maps,
+cudaError_t launch_prefill_gemm(int phase, bool pairs, const uint8_t* weights, const Dims& d, const void* token_maps,
                                 const Plan& p, const float4* slot, const int4* tiles, const int* n_tiles, __half* h16,
                                 float* y32, int* err, int n_sm, long long* trace, int trace_cap, cudaStream_t st) {
     TcArgs a;
@@ -645,23 +710,30 @@ cudaError_t launch_prefill_gemm(int phase, const uint8_t* weights, const Dims& d
     a.H = d.H;
     a.err = err;
     cudaError_t e;
-    if (phase == 0) {
-        e = cudaFuncSetAttribute(moe_prefill_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTc);
-        if (e != cudaSuccess) return e;
-        moe_prefill_tc_kernel<0><<<n_sm, kThreadsTc, kSmemTc, st>>>(a);
-    } else {
-        e = cudaFuncSetAttribute(moe_prefill_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTc);
-        if (e != cudaSuccess) return e;
-        moe_prefill_tc_kernel<1><<<n_sm, kThreadsTc, kSmemTc, st>>>(a);
-    }
+    auto run = [&](auto kern) {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTc);
+        if (r != cudaSuccess) return r;
+        kern<<<n_sm, kThreadsTc, kSmemTc, st>>>(a);
+        return cudaSuccess;
+    };
+    if (phase == 0)
+        e = pairs ? run(moe_prefill_tc_kernel<0, true>) : run(moe_prefill_tc_kernel<0, false>);
+    else
+        e = run(moe_prefill_tc_kernel<1, false>);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-cudaError_t launch_prefill_out(const float* y32, const float* residual, int T, int H, void* y, cudaStream_t st) {
+cudaError_t launch_prefill_out(const float* y32, const float* residual, int T, int H, void* y, coli_dtype dt,
+                               cudaStream_t st) {
     const size_t n = (size_t)T * H;
     if (n == 0) return cudaSuccess;
     const size_t blocks = (n / 4 + 255) / 256;
-    prefill_out_kernel<<<(int)(blocks < 4736 ? blocks : 4736), 256, 0, st>>>(y32, residual, n, (__nv_bfloat16*)y);
+    const int grid = (int)(blocks < 4736 ? blocks : 4736);
+    if (dt == COLI_F32)
+        prefill_out_kernel<float><<<grid, 256, 0, st>>>(y32, residual, n, (float*)y);
+    else
+        prefill_out_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(y32, residual, n, (__nv_bfloat16*)y);
     return cudaGetLastError();
 }
 

@@ -327,6 +327,15 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         *p.n_unique = n_unique;
         *p.n_active = n_unique + S;
     }
+    __syncthreads();
+    if (threadIdx.x == 0) {  // chunks of kCoreTok tokens per active expert, prefix (work items of the CUDA-core kernels)
+        int run = 0;
+        for (int a = 0; a < n_unique + S; ++a) {
+            p.act_chunk[a] = run;
+            run += (p.act_cnt[a] + kCoreTok - 1) / kCoreTok;
+        }
+        p.act_chunk[n_unique + S] = run;
+    }
     // positions: each warp walks its chunk in token order
     for (int t = tb; t < te; ++t) {
         if (lane < K) {
@@ -353,7 +362,7 @@ cudaError_t launch_router_logits(const float* wr, const float* bias, const void*
         const int tiles = ((T + kRgT - 1) / kRgT) * ((E + kRgE - 1) / kRgE);
         const int nk = H / kRgK;
         int nsplit = 1;
-        for (int sp = 2; sp <= 16; ++sp)
+        for (int sp = 2; sp <= 64; ++sp)
             if (nk % sp == 0 && (size_t)sp * T * E <= part_cap && tiles * sp <= 2 * 148) nsplit = sp;
         dim3 g((T + kRgT - 1) / kRgT, (E + kRgE - 1) / kRgE, nsplit);
         double* dst = nsplit == 1 ? logits : part;

@@ -180,3 +180,29 @@ def test_full_prefill_2048_hot_expert_tokens(gpu, coli):
         y_ref, _, _ = _oracle_for_tokens(c, wr, bias, xb[t:t + 1])
         assert _l2_rel(y[t:t + 1], y_ref) <= BF16_TOL
     layer.close()
+
+
+@pytest.mark.parametrize("T", [5, 40, 200])
+def test_tiny_fp32_tensor_cores_and_cuda_cores(gpu, tiny_big, T):
+    """fp32 batches of more than 4 tokens run the CUDA-core kernels by default;
+    mode 2 runs them on the tensor cores with hi + lo operand rows (tiles of up
+    to 64 tokens). Both meet the fp32-path tolerance on one layer."""
+    c, L, layer = tiny_big
+    x = synth.x_f32(c["seed"], 600 + T, T, c["H"])
+    xd = torch.from_numpy(x).to(gpu)
+    y_tc = torch.full_like(xd, float("nan"))
+    y_cc = torch.full_like(xd, float("nan"))
+    layer.forward(xd, y_cc)
+    layer.set_tensor_cores(2)
+    try:
+        layer.forward(xd, y_tc)
+    finally:
+        layer.set_tensor_cores(1)
+    layer.sync()
+    y_ref, ids_ref, _ = oracle.moe_forward(cases.oracle_cfg(c), L["wr"], None, L["experts"], x)
+    _check_plan(layer.plan(T), ids_ref, c["E"])
+    scale = np.abs(y_ref).max()
+    for y in (y_tc, y_cc):
+        yv = y.cpu().numpy().astype(np.float64)
+        assert np.isfinite(yv).all()
+        assert np.abs(yv - y_ref).max() <= 1e-3 * scale
