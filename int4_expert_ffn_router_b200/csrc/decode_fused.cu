@@ -614,7 +614,7 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
             const uint8_t* stage = ring + (size_t)slot_s * stage_bytes;
             const int g0 = i * a.sb;
             const int nb = min(a.sb, G - g0);
-#pragma unroll 2
+#pragma unroll 4
             for (int bb = 0; bb < nb; ++bb) {
                 const int g = g0 + bb;
                 const uint8_t* bp = stage + bb * kBlockBytes;

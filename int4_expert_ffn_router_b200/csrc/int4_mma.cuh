@@ -116,14 +116,16 @@ __device__ __forceinline__ void group_mma_aw(uint4 w, uint32_t sv, uint4 xb0, ui
 //     row gi:   -1032 * X,   row gi+8:  -1152 * X     (X = the column's sum of
 // the group's 64 B values), so the MMAs return sum(q x) and 16 sum(q x).
 // c = {row gi hi, row gi lo, row gi+8 hi, row gi+8 lo} corrections of token t.
+// Steps 0, 2 and 1, 3 accumulate separately (two shorter dependency chains).
 __device__ __forceinline__ void group_mma_aw_off(uint4 w, uint32_t sv, uint4 xb0, uint4 xb1, float4 c, float& acc0,
                                                  float& acc1) {
-    float d[4] = {c.x, c.y, c.z, c.w};
+    float dd[2][4] = {{c.x, c.y, c.z, c.w}, {0.f, 0.f, 0.f, 0.f}};
     const uint32_t words[4] = {w.x, w.y, w.z, w.w};
     const uint32_t bx[8] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w};
     constexpr uint32_t MAGIC = 0x64006400u;
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
+        float* d = dd[s & 1];
         const uint32_t wv = words[s], ws = wv >> 8;
         const uint32_t r0 = lop3_and_or(wv, 0x000F000Fu, MAGIC);  // row gi,   k lo: 1024 + v
         const uint32_t r8 = lop3_and_or(wv, 0x00F000F0u, MAGIC);  // row gi+8, k lo: 1024 + 16 v
@@ -135,6 +137,7 @@ __device__ __forceinline__ void group_mma_aw_off(uint4 w, uint32_t sv, uint4 xb0
             : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
             : "r"(r0), "r"(r8), "r"(r1), "r"(r9), "r"(bx[2 * s]), "r"(bx[2 * s + 1]));
     }
+    float d[4] = {dd[0][0] + dd[1][0], dd[0][1] + dd[1][1], dd[0][2] + dd[1][2], dd[0][3] + dd[1][3]};
     const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sv));
     acc0 = fmaf(sc.x, d[0] + d[1], acc0);            // row gi: hi + lo columns of token t
     acc1 = fmaf(sc.y * 0.0625f, d[2] + d[3], acc1);  // row gi+8 (values carry a factor 16)
