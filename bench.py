@@ -71,6 +71,77 @@ DEFAULT_STEPS = {"decode_b1": 10000, "decode_b32": 2000, "prefill_2048": 100, "d
                  "stack30_b1": 300, "stack30_b8": 200, "stack30_b64": 100}
 
 
+def step_seed(step, rank):
+    """Seed of the activations of `step` on `rank`: every replica draws its own token stream."""
+    return X_SEED0 + step + 100000 * rank
+
+
+def max_over_ranks(value, dist, device):
+    """The largest of the ranks' values (every rank gets it); `dist` None: single process."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world_size, steps, tokens_per_step, total_ms):
+    """Whole-job throughput: the tokens every replica processed over the slowest rank's time."""
+    return world_size * steps * tokens_per_step / (total_ms * 1e-3)
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except OSError:
+        return {}
+
+
+def dominant_roofline(stages, n_launches, T, mean_unique, E, elt, tc, peaks):
+    """Roofline of the kernel with the largest device time.
+
+    stages: total device ms per stage over `n_launches` launches of each stage
+    kernel. Algorithmic work per launch:
+      persistent decode kernel: active experts + router bytes + x and y;
+      CUDA-core gate/up: active gate/up bytes + x + h (fp32);
+      CUDA-core down: active down bytes + h + o (fp32);
+      tensor-core gate/up: 2 * T (K + S) * H * 2I flops; down: 2 * T (K + S) * I * H.
+    """
+    dom = max(stages, key=lambda k: stages[k])
+    avg_s = stages[dom] / max(n_launches, 1) * 1e-3
+    pairs = T * (K + S)
+    router_bytes = E * H * 4
+    act = 2 * T * H * elt
+    if tc and dom in ("gateup", "down"):
+        flops = 2.0 * pairs * H * 2 * I if dom == "gateup" else 2.0 * pairs * I * H
+        ach = flops / avg_s / 1e12
+        peak = peaks.get("bf16_tflops", 1590.0)
+        roof = {"bound": "tensor", "kernel": f"moe_prefill_tc_kernel ({dom})", "achieved": round(ach, 1),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
+                "peak_source": "measured burst (MEASURED_PEAKS.json bf16_tflops; the f16 MMA rate equals bf16)"
+                if "bf16_tflops" in peaks else "fallback 1.59 PFLOP/s",
+                "flops_per_launch": flops, "avg_launch_us": round(avg_s * 1e6, 2)}
+        if "bf16_tflops_sustained" in peaks:
+            roof["frac_of_sustained"] = round(ach / peaks["bf16_tflops_sustained"], 4)
+        return dom, roof
+    alg = {"gateup": (mean_unique + S) * GU_BYTES + T * H * elt + pairs * I * 4,
+           "down": (mean_unique + S) * DOWN_BYTES + pairs * (I + H) * 4,
+           "router": router_bytes + T * H * elt,
+           "fused": (mean_unique + S) * EXPERT_BYTES + router_bytes + act}
+    if dom not in alg:
+        return dom, None
+    ach = alg[dom] / avg_s / 1e9
+    peak = peaks.get("hbm_gbs", 6650.0)
+    names = {"fused": "moe_decode_fused_kernel", "gateup": "gateup_core_kernel", "down": "down_core_kernel",
+             "router": "router kernels"}
+    return dom, {"bound": "hbm", "kernel": names[dom], "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                 "frac": round(ach / peak, 4), "traffic": None,
+                 "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in peaks else "fallback 6.65 TB/s",
+                 "bytes_per_launch": int(alg[dom]), "avg_launch_us": round(avg_s * 1e6, 2)}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -261,7 +332,7 @@ def run_ours(args, wl, ws, rank, local):
     xs = torch.empty((nsteps, T, H), dtype=xdt, device=dev)
     stream = torch.cuda.current_stream(dev)
     for i in range(nsteps):  # rank r draws its own token stream
-        synth.x_dev(X_SEED0 + i + 100000 * rank, 0, T, H, 1 if wl["bf16"] else 0, xs[i].data_ptr(), stream.cuda_stream)
+        synth.x_dev(step_seed(i, rank), 0, T, H, 1 if wl["bf16"] else 0, xs[i].data_ptr(), stream.cuda_stream)
     y = torch.empty((T, H), dtype=xdt, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
@@ -282,6 +353,7 @@ def run_ours(args, wl, ws, rank, local):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks = Clocks(local)
+    n0 = layer.launch_count()
     for i in range(args.warmup, nsteps):
         ev[i][0].record(stream)
         layer.forward(xs[i], y, stream=stream)
@@ -289,6 +361,7 @@ def run_ours(args, wl, ws, rank, local):
         flush.zero_()
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
+    launches = layer.launch_count() - n0
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -302,10 +375,7 @@ def run_ours(args, wl, ws, rank, local):
     stages, nprof = layer.profile()
     layer.set_profiling(False)
     total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     # end to end through the C ABI with host buffers: pinned H2D of the step's
     # x, forward, D2H of y, every step inside the events.
@@ -325,10 +395,8 @@ def run_ours(args, wl, ws, rank, local):
         flush.zero_()
     torch.cuda.synchronize(dev)
     e2e_ms = sum(ev2[j][0].elapsed_time(ev2[j][1]) for j in range(args.steps))
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
 
     if rank != 0:
@@ -337,41 +405,17 @@ def run_ours(args, wl, ws, rank, local):
             dist.destroy_process_group()
         return None
 
-    tokens = ws * args.steps * T
     u = uniq[args.warmup:]
     mean_unique = sum(u) / len(u)
     router_bytes = wl.get("E", E_FULL) * H * 4
     bytes_step = [(n + S) * EXPERT_BYTES + router_bytes for n in u]
     gbs = sum(bytes_step) / (sum(step_ms) * 1e-3) / 1e9
-    # dominant kernel by device time
-    dom = max(stages, key=lambda k: stages[k])
-    dom_avg_s = stages[dom] / max(nprof, 1) * 1e-3
-    elt = xs.element_size()
-    act_bytes = 2 * T * H * elt  # x in, y out
-    gu_bytes = sum((n + S) * GU_BYTES for n in u) / len(u) + T * H * elt + (T * K + T * S) * I * 4
-    down_bytes = sum((n + S) * DOWN_BYTES for n in u) / len(u) + (T * K + T * S) * (I + H) * 4
-    alg = {"gateup": gu_bytes, "down": down_bytes, "router": router_bytes + T * H * elt,
-           # the persistent kernel streams every active expert and the router once
-           "fused": sum(bytes_step) / len(bytes_step) + act_bytes}
-    peaks = {}
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peaks = json.load(f)
-    except OSError:
-        pass
+    peaks = load_peaks()
     peak_gbs = peaks.get("hbm_gbs", 6650.0)
-    roof = None
-    if dom in alg:
-        ach = alg[dom] / dom_avg_s / 1e9
-        roof = {"bound": "hbm", "kernel": "moe_decode_fused_kernel" if dom == "fused" else dom,
-                "achieved": round(ach, 1), "peak": peak_gbs, "unit": "GB/s",
-                "frac": round(ach / peak_gbs, 4), "traffic": None,
-                "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in peaks else "fallback",
-                "bytes_per_launch": int(alg[dom]), "avg_launch_us": round(dom_avg_s * 1e6, 2),
-                "frac_of_8tbs": round(ach / 8000.0, 4)}
-    fused = stages.get("fused", 0.0) > 0.5 * sum(stages.values())
+    tc = wl["bf16"] and T > 4  # bf16 batches of more than 4 tokens run on the tensor cores
+    dom, roof = dominant_roofline(stages, nprof, T, mean_unique, wl.get("E", E_FULL), xs.element_size(), tc, peaks)
     out = {
-        "metric": METRIC, "value": round(tokens / (total_ms * 1e-3), 2), "unit": "tokens/s", "n_gpus": ws,
+        "metric": METRIC, "value": round(job_tokens_per_s(ws, args.steps, T, total_ms), 2), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl["bf16"] else "f32",
@@ -387,8 +431,12 @@ def run_ours(args, wl, ws, rank, local):
         "bytes_per_step": int(sum(bytes_step) / len(bytes_step)),
         "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items()},
         "roofline": roof,
-        "gpu_launches": (1 if fused else 6) * args.steps,
-        "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+        "gpu_launches": launches,
+        "compute": ("int4 weights dequantised to f16 in tensor memory, tcgen05 f16 MMA, f32 accumulate; "
+                    "bf16 tokens scaled by powers of two to f16 (exact)") if tc else
+                   ("int4 weights as raw f16 codes in mma.sync, f32 accumulate, fp64 router" if T <= 4 else
+                    "int4 weights dequantised to f32 on CUDA cores, fp64 router"),
+        "e2e": {"value": round(job_tokens_per_s(ws, args.steps, T, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * xs.element_size(), "d2h_bytes_per_step": T * H * xs.element_size()},
         "clocks": clk,
     }
@@ -418,7 +466,7 @@ def run_stack(args, wl, ws, rank, local):
     xs = torch.empty((nsteps, T, H), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     for i in range(nsteps):
-        synth.x_dev(X_SEED0 + i + 100000 * rank, 0, T, H, 0, xs[i].data_ptr(), stream.cuda_stream)
+        synth.x_dev(step_seed(i, rank), 0, T, H, 0, xs[i].data_ptr(), stream.cuda_stream)
     xw = torch.empty((T, H), dtype=torch.float32, device=dev)
 
     # routing statistics from a few untimed steps: distinct experts per layer -> bytes
@@ -442,6 +490,7 @@ def run_stack(args, wl, ws, rank, local):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks = Clocks(local)
+    n0 = sum(L.launch_count() for L in layers)
     for i in range(args.warmup, nsteps):
         xw.copy_(xs[i])
         ev[i][0].record(stream)
@@ -449,6 +498,7 @@ def run_stack(args, wl, ws, rank, local):
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
+    launches = sum(L.launch_count() for L in layers) - n0
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -468,10 +518,7 @@ def run_stack(args, wl, ws, rank, local):
         for k, v in st.items():
             stages[k] = stages.get(k, 0.0) + v
         L.set_profiling(False)
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     # end to end through the C ABI with host buffers (pinned x in, result out)
     xh = xs[args.warmup:].cpu().pin_memory()
@@ -488,10 +535,8 @@ def run_stack(args, wl, ws, rank, local):
         ev2[j][1].record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = sum(ev2[j][0].elapsed_time(ev2[j][1]) for j in range(args.steps))
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     if dist:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
     for L in layers:
         L.close()
@@ -500,19 +545,13 @@ def run_stack(args, wl, ws, rank, local):
             dist.destroy_process_group()
         return None
 
-    tokens = ws * args.steps * T
     gbs = bytes_step / (total_ms / args.steps * 1e-3) / 1e9
-    peaks = {}
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peaks = json.load(f)
-    except OSError:
-        pass
+    peaks = load_peaks()
     peak_gbs = peaks.get("hbm_gbs", 6650.0)
-    fused = stages.get("fused", 0.0) > 0.5 * sum(stages.values())
-    per_layer_launches = 2 if fused else (8 if T >= 64 else 7)
+    # stage totals are summed over the layers: nprof forwards of each of NL layers
+    dom, roof = dominant_roofline(stages, nprof * NL, T, mean_unique, E_FULL, 4, False, peaks)
     out = {
-        "metric": METRIC, "value": round(tokens / (total_ms * 1e-3), 2), "unit": "tokens/s", "n_gpus": ws,
+        "metric": METRIC, "value": round(job_tokens_per_s(ws, args.steps, T, total_ms), 2), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded generator; random-init int4 weights of the full-size layer shape, per layer)",
@@ -525,11 +564,9 @@ def run_stack(args, wl, ws, rank, local):
         "hbm_frac_of_measured": round(gbs / peak_gbs, 4),
         "bytes_per_step": int(bytes_step), "unique_experts_per_layer": round(mean_unique, 2),
         "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items()},
-        "roofline": {"bound": "hbm", "kernel": "whole stack step", "achieved": round(gbs, 1), "peak": peak_gbs,
-                     "unit": "GB/s", "frac": round(gbs / peak_gbs, 4), "traffic": None,
-                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if "hbm_gbs" in peaks else "fallback"},
-        "gpu_launches": per_layer_launches * NL * args.steps,
-        "e2e": {"value": round(tokens / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+        "roofline": roof,
+        "gpu_launches": launches,
+        "e2e": {"value": round(job_tokens_per_s(ws, args.steps, T, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4},
         "clocks": clk,
     }

@@ -146,6 +146,15 @@ coli_status coli_moe_get_stats(coli_moe_layer* layer, int* n_unique, int64_t* by
                                int32_t* per_expert_counts);
 
 /*
+ * Number of kernels of this library that route, forward and stack calls on
+ * this layer have enqueued since it was created (load-time kernels and the
+ * driver memset that clears the tensor-core path's fp32 output are not
+ * counted). Host-side counter: no synchronisation. n must not be NULL
+ * (COLI_EINVAL).
+ */
+coli_status coli_moe_get_launch_count(const coli_moe_layer* layer, int64_t* n);
+
+/*
  * The batch-union plan of the last forward (synchronises; host outputs, any
  * of them NULL to skip):
  *   ids [T][K], weights [T][K]      routing
@@ -165,7 +174,9 @@ coli_status coli_moe_get_plan(coli_moe_layer* layer, int32_t* ids, float* weight
  * finished forward into running totals). coli_moe_get_profile waits for the
  * profiled forwards to finish and writes, per stage, the total device ms over
  * all forwards since profiling was enabled, and their number. Enabling again
- * resets the totals.
+ * resets the totals. On the tensor-core path the plan stage also covers the
+ * operand rows, the tile list and the clear of the fp32 output, so the
+ * gate/up and down stages each time one grouped-GEMM kernel alone.
  */
 enum { COLI_STAGE_ROUTER = 0, COLI_STAGE_TOPK, COLI_STAGE_PLAN, COLI_STAGE_GATEUP, COLI_STAGE_DOWN,
        COLI_STAGE_COMBINE, COLI_STAGE_FUSED, COLI_N_STAGES };

@@ -23,7 +23,7 @@ EXPORTS = (
     "coli_moe_route", "coli_moe_forward", "coli_moe_stack_forward", "coli_moe_get_stats", "coli_moe_get_plan",
     "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
     "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused", "coli_moe_set_tensor_cores",
-    "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc",
+    "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc", "coli_moe_get_launch_count",
 )
 NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 64, 1024
 N_STAGES = 7
@@ -57,6 +57,7 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_forward.argtypes = [vp, vp, vp, i32, i32, vp]
     L.coli_moe_stack_forward.argtypes = [vp, i32, vp, i32, f32, vp]
     L.coli_moe_get_stats.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(ctypes.c_int64), vp]
+    L.coli_moe_get_launch_count.argtypes = [vp, ctypes.POINTER(ctypes.c_int64)]
     L.coli_moe_get_plan.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.POINTER(i32), vp, vp]
     L.coli_moe_expert_bytes.argtypes = [i32, i32]
     L.coli_moe_expert_bytes.restype = ctypes.c_int64
@@ -171,6 +172,12 @@ class Layer:
         _check(lib.coli_moe_get_stats(self.handle, ctypes.byref(nu), ctypes.byref(b), _ptr(counts)),
                "coli_moe_get_stats")
         return nu.value, b.value
+
+    def launch_count(self) -> int:
+        """Kernels of the library this layer's route/forward/stack calls enqueued so far."""
+        n = ctypes.c_int64()
+        _check(lib.coli_moe_get_launch_count(self.handle, ctypes.byref(n)), "coli_moe_get_launch_count")
+        return n.value
 
     def sync(self) -> None:
         """Wait for the last forward; raises if the device reported a timeout."""

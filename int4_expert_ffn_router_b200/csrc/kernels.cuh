@@ -13,6 +13,8 @@ namespace coli {
 // (batches of kRouterGemmMinTok tokens and more use the blocked GEMM form).
 cudaError_t launch_router_logits(const float* wr, const float* bias, const void* x, coli_dtype dt, int T, int H, int E,
                                  double* logits, cudaStream_t st, double* part = nullptr, size_t part_cap = 0);
+// Kernels launch_router_logits enqueues for these arguments (0, 1 or 2).
+int router_kernel_count(int T, int H, int E, const double* part, size_t part_cap);
 cudaError_t launch_topk(const double* logits, int T, int E, int K, int32_t* ids, float* w, cudaStream_t st);
 size_t plan_smem_bytes(int E);
 cudaError_t launch_plan(const int32_t* ids, int T, int K, int E, int S, const Plan& p, cudaStream_t st);

@@ -70,6 +70,7 @@ struct coli_moe_layer {
     uint8_t* ws = nullptr;
     size_t ws_bytes = 0;
     double* logits = nullptr;
+    int64_t launches = 0;  // kernels of this library enqueued by route/forward/stack calls
     Plan plan{};
     float* h = nullptr;
     float* o = nullptr;
@@ -351,6 +352,7 @@ COLI_API coli_status coli_moe_route(coli_moe_layer* L, const void* x, coli_dtype
     const Dims& d = L->d;
     CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
     CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, ids, weights, s), "topk");
+    L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
     return COLI_OK;
 }
 
@@ -367,6 +369,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
                                      L->o, L->ctl, L->n_sm, L->smem_optin, L->trace, L->trace_cap, L->ring_stages,
                                      L->ring_blocks, s),
                  "persistent decode kernel");
+        L->launches += 1;
     } else if ((L->tc_mode == 2 || (L->tc_mode == 1 && dt == COLI_BF16)) && L->tc_shape_ok && L->tc_scale_ok) {
         // tensor cores; fp32 tokens as fp16 hi + lo operand rows (tiles of kTcMaxTok / 2 tokens)
         const bool pairs = dt == COLI_F32;
@@ -376,7 +379,8 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
-        prof_mark(L, COLI_STAGE_GATEUP, s);
+        // the plan stage also covers the operand rows, the tile list and the output clear,
+        // so the gate/up and down stages time the grouped GEMMs alone
         __half* h16 = reinterpret_cast<__half*>(L->h);
         CUDA_TRY(launch_prefill_prep(x, dt, T, d.H, d.K, d.S, p.pos, reinterpret_cast<const float*>(L->meta), L->xs,
                                      L->tscale, s),
@@ -384,13 +388,14 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         CUDA_TRY(launch_prefill_plan(p, T, d.K, d.S, pairs ? kTcMaxTok / 2 : kTcMaxTok, L->tscale, L->slot, L->tiles,
                                      L->n_tiles, s),
                  "tile plan");
+        CUDA_TRY(cudaMemsetAsync(L->o, 0, (size_t)T * d.H * 4, s), "clear output");
+        prof_mark(L, COLI_STAGE_GATEUP, s);
         // with a trace buffer: block timeline of the gate/up launch, then of the down launch
         const int tcap = L->trace ? (L->trace_cap - 256) / 16 : 0;
         CUDA_TRY(launch_prefill_gemm(0, pairs, L->weights, d, L->xs_maps, p, L->slot, L->tiles, L->n_tiles, h16, nullptr,
                                      L->ctl + kCtlError, L->n_sm, tcap > 0 ? L->trace : nullptr, tcap, s),
                  "gate/up (tensor cores)");
         prof_mark(L, COLI_STAGE_DOWN, s);
-        CUDA_TRY(cudaMemsetAsync(L->o, 0, (size_t)T * d.H * 4, s), "clear output");
         CUDA_TRY(launch_prefill_gemm(1, false, L->weights, d, L->h16_maps, p, L->slot, L->tiles, L->n_tiles, nullptr,
                                      L->o, L->ctl + kCtlError, L->n_sm,
                                      tcap > 0 ? L->trace + (size_t)tcap * 8 + 128 : nullptr, tcap, s),
@@ -398,6 +403,8 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_prefill_out(L->o, residual, T, d.H, y, dt, s), "output");
         prof_mark(L, COLI_STAGE_FUSED, s);
+        // router, top-k, plan, prep, tile plan, two grouped GEMMs, output (the clear is a driver memset)
+        L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 7;
     } else {
         prof_mark(L, COLI_STAGE_ROUTER, s);
         CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
@@ -412,6 +419,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_combine(L->o, p, T, d.H, d.K, d.S, residual, y, dt, s), "combine");
         prof_mark(L, COLI_STAGE_FUSED, s);
+        L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 5;
     }
     prof_mark(L, COLI_N_STAGES, s);
     if (L->profiling) {
@@ -456,6 +464,7 @@ COLI_API coli_status coli_moe_stack_forward(coli_moe_layer* const* layers, int n
     for (int l = 0; l < n_layers; ++l) {
         coli_moe_layer* L = layers[l];
         CUDA_TRY(launch_rmsnorm(x, T, L->d.H, eps, L->xn, s), "rmsnorm");
+        L->launches += 1;
         coli_status st = forward_impl(L, L->xn, x, COLI_F32, T, x, s);
         if (st != COLI_OK) return st;
     }
@@ -536,6 +545,13 @@ COLI_API coli_status coli_moe_get_stats(coli_moe_layer* L, int* n_unique, int64_
         *bytes_streamed = (int64_t)(nu + L->d.S) * coli_moe_expert_bytes(L->d.H, L->d.I) + (int64_t)L->d.E * L->d.H * 4;
     if (per_expert_counts)
         CUDA_TRY(cudaMemcpy(per_expert_counts, L->plan.cnt, (size_t)L->d.E * 4, cudaMemcpyDeviceToHost), "read counts");
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_get_launch_count(const coli_moe_layer* L, int64_t* n) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (!n) return fail(COLI_EINVAL, "n is NULL");
+    *n = L->launches;
     return COLI_OK;
 }
 

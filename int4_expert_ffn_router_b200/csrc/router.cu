@@ -354,16 +354,28 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
 // ---------------------------------------------------------------------------
 // Host launchers.
 // ---------------------------------------------------------------------------
+// Split of the input dimension for the blocked router GEMM (0: the GEMV
+// kernel serves this call): split until about two CTAs per SM are busy.
+static int router_nsplit(int T, int H, int E, const double* part, size_t part_cap) {
+    if (T < kRouterGemmMinTok || !part || part_cap < (size_t)T * E) return 0;
+    const int tiles = ((T + kRgT - 1) / kRgT) * ((E + kRgE - 1) / kRgE);
+    const int nk = H / kRgK;
+    int nsplit = 1;
+    for (int sp = 2; sp <= 64; ++sp)
+        if (nk % sp == 0 && (size_t)sp * T * E <= part_cap && tiles * sp <= 2 * 148) nsplit = sp;
+    return nsplit;
+}
+
+int router_kernel_count(int T, int H, int E, const double* part, size_t part_cap) {
+    if (T == 0) return 0;
+    return router_nsplit(T, H, E, part, part_cap) > 1 ? 2 : 1;
+}
+
 cudaError_t launch_router_logits(const float* wr, const float* bias, const void* x, coli_dtype dt, int T, int H, int E,
                                  double* logits, cudaStream_t st, double* part, size_t part_cap) {
     if (T == 0) return cudaSuccess;
-    if (T >= kRouterGemmMinTok && part && part_cap >= (size_t)T * E) {
-        // split the input dimension until about two CTAs per SM are busy
-        const int tiles = ((T + kRgT - 1) / kRgT) * ((E + kRgE - 1) / kRgE);
-        const int nk = H / kRgK;
-        int nsplit = 1;
-        for (int sp = 2; sp <= 64; ++sp)
-            if (nk % sp == 0 && (size_t)sp * T * E <= part_cap && tiles * sp <= 2 * 148) nsplit = sp;
+    const int nsplit = router_nsplit(T, H, E, part, part_cap);
+    if (nsplit > 0) {
         dim3 g((T + kRgT - 1) / kRgT, (E + kRgE - 1) / kRgE, nsplit);
         double* dst = nsplit == 1 ? logits : part;
         if (dt == COLI_F32)
