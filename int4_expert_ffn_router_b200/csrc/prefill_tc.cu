@@ -212,13 +212,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                 const int c = kTokPerChunk * (2 * (lc / kTokPerChunk) + kh) + (lc % kTokPerChunk);
                 if (c < n && lc < (kSlotPerWarp / 16) * kTokPerChunk) sinfo[lc] = a.slot[start + c];
             }
+            // phases of this warp's next block seen complete while it worked on the current one
+            bool seen_full = false, seen_aempty = false;
             for (int kb = hb; kb < KB; kb += 2) {
                 const uint32_t it = it0 + kb;
                 const uint32_t p2 = it >> 1;           // A stage use counter
                 const uint32_t s = it & (kSStages - 1), sa = p2 & (kAStages - 1);
-                if (!tc_wait_warp(&full[s], (it / kSStages) & 1, abort_flag, a.err, 21)) { ok = false; break; }
+                if (!seen_full && !tc_wait_warp(&full[s], (it / kSStages) & 1, abort_flag, a.err, 21)) { ok = false; break; }
                 if (warp == 0 && lane == 0) tc_stamp(a, it, 0);
-                if (!tc_wait_warp(&aempty[2 * sa + rt2], ((p2 / kAStages) & 1) ^ 1, abort_flag, a.err, 22)) { ok = false; break; }
+                if (!seen_aempty && !tc_wait_warp(&aempty[2 * sa + rt2], ((p2 / kAStages) & 1) ^ 1, abort_flag, a.err, 22)) { ok = false; break; }
                 if (warp == 0 && lane == 0) tc_stamp(a, it, 1);
                 tc_fence_after();
                 const uint8_t* blk = sm + kOffW + s * kWStageBytes + rt2 * kBlockBytes;
@@ -227,6 +229,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
 #pragma unroll
                 for (int ti = 0; ti < 4; ++ti) wv[ti] = *reinterpret_cast<const uint4*>(rowp + 128 * ti);
                 const uint32_t sp = *reinterpret_cast<const uint32_t*>(blk + kNibbleBytes + sub * 32 + gi * 4);
+                // test the next block's phases now (non-blocking): the answers are read after the
+                // dequantisation, so a barrier that is already complete costs no wait latency
+                bool nf = false, na = false;
+                if (kb + 2 < KB) {
+                    const uint32_t itn = it + 2, p2n = itn >> 1;
+                    nf = mbar_test_wait(&full[itn & (kSStages - 1)], (itn / kSStages) & 1);
+                    na = mbar_test_wait(&aempty[2 * (p2n & (kAStages - 1)) + rt2], ((p2n / kAStages) & 1) ^ 1);
+                }
                 const uint32_t s2 = __byte_perm(sp, 0, isb ? 0x3232 : 0x1010);
                 uint32_t r[32];
 #pragma unroll
@@ -249,6 +259,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                 __syncwarp();
                 mbar_arrive_elect(&aready[2 * sa + rt2]);
                 if (warp == 0 && lane == 0) tc_stamp(a, it, 2);
+                seen_full = __all_sync(0xffffffffu, nf);
+                seen_aempty = __all_sync(0xffffffffu, na);
             }
             if (!ok) break;
             // ---------------------------------------------------- epilogue
