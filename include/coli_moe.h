@@ -221,7 +221,9 @@ coli_status coli_moe_set_tensor_cores(coli_moe_layer* layer, int mode);
  * stage, ns the item was published by the CTA's producer, total ns warp 0
  * waited for weight stages, 0, 0}; kind 1 router rows, 2 gate/up tile,
  * 3 down tile; times from the GPU global timer. NULL disables tracing.
- * The tensor-core path writes, with c = (capacity - 256) / 16 when positive,
+ * In a library built with COLI_TC_TRACE=1 (a profiling build; the default
+ * build records nothing there), the tensor-core path writes, with
+ * c = (capacity - 256) / 16 when positive,
  * the timeline of CTA 0 of its gate/up launch at int64 0 and of its down
  * launch at int64 8c + 128: per 64-input block b < c, 8 SM clock stamps at
  * 8b (transform warp has the block, its A stage is free, its stores issued,

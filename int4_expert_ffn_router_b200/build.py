@@ -15,8 +15,13 @@ NVCC_FLAGS = [
 
 
 def build(verbose: bool = False, extra: list[str] | None = None) -> str:
+    """COLI_TC_TRACE=1 in the environment builds the profiling variant whose
+    tensor-core kernels record a block timeline into the trace buffer."""
     srcs = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
-    cmd = ["nvcc", *NVCC_FLAGS, *(extra or []), "-o", SO, *srcs]
+    flags = list(extra or [])
+    if os.environ.get("COLI_TC_TRACE") == "1":
+        flags.append("-DCOLI_TC_TRACE=1")
+    cmd = ["nvcc", *NVCC_FLAGS, *flags, "-o", SO, *srcs]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

@@ -77,7 +77,7 @@ constexpr int kOffSlot = kOffW + kSStages * kWStageBytes;          // per transf
 constexpr int kSlotPerWarp = kTcMaxTok / 2;
 constexpr int kOffBar = kOffSlot + kTransformWarps * kSlotPerWarp * 16;
 constexpr int kNumBars = 2 * kSStages + 4 * kAStages + 6;
-static_assert((kSStages & (kSStages - 1)) == 0 && (kAStages & (kAStages - 1)) == 0, "stage counts are powers of two");
+static_assert(kSStages % 2 == 0, "a pair of blocks never wraps the shared-memory ring");
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemTc = kOffMisc + 16 + 1024;                      // + alignment slack
 static_assert(kOffBar % 8 == 0, "alignment");
@@ -107,11 +107,20 @@ struct __align__(64) TcArgs {
 // stage is free, 2 its stores are issued, 3 MMA has the block, 4 MMA has the
 // A stage, 5 MMAs issued, 6 producer has the stage, 7 copies issued; then per
 // item i, trace[cap * 8 + 2 i] epilogue start, [.. + 1] epilogue end.
+// Recorded only in profiling builds (COLI_TC_TRACE=1): the stamps cost
+// issue slots in the loops they time.
+#ifndef COLI_TC_TRACE
+#define COLI_TC_TRACE 0
+#endif
 __device__ __forceinline__ void tc_stamp(const TcArgs& a, uint32_t it, int j) {
-    if (a.trace && blockIdx.x == 0 && it < (uint32_t)a.trace_cap) a.trace[(size_t)it * 8 + j] = clock64();
+    if constexpr (COLI_TC_TRACE != 0) {
+        if (a.trace && blockIdx.x == 0 && it < (uint32_t)a.trace_cap) a.trace[(size_t)it * 8 + j] = clock64();
+    }
 }
 __device__ __forceinline__ void tc_stamp_item(const TcArgs& a, uint32_t i, int j) {
-    if (a.trace && blockIdx.x == 0 && i < 64u) a.trace[(size_t)a.trace_cap * 8 + 2 * i + j] = clock64();
+    if constexpr (COLI_TC_TRACE != 0) {
+        if (a.trace && blockIdx.x == 0 && i < 64u) a.trace[(size_t)a.trace_cap * 8 + 2 * i + j] = clock64();
+    }
 }
 
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site);
@@ -217,7 +226,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
             for (int kb = hb; kb < KB; kb += 2) {
                 const uint32_t it = it0 + kb;
                 const uint32_t p2 = it >> 1;           // A stage use counter
-                const uint32_t s = it & (kSStages - 1), sa = p2 & (kAStages - 1);
+                const uint32_t s = it % kSStages, sa = p2 % kAStages;
                 if (!seen_full && !tc_wait_warp(&full[s], (it / kSStages) & 1, abort_flag, a.err, 21)) { ok = false; break; }
                 if (warp == 0 && lane == 0) tc_stamp(a, it, 0);
                 if (!seen_aempty && !tc_wait_warp(&aempty[2 * sa + rt2], ((p2 / kAStages) & 1) ^ 1, abort_flag, a.err, 22)) { ok = false; break; }
@@ -234,8 +243,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                 bool nf = false, na = false;
                 if (kb + 2 < KB) {
                     const uint32_t itn = it + 2, p2n = itn >> 1;
-                    nf = mbar_test_wait(&full[itn & (kSStages - 1)], (itn / kSStages) & 1);
-                    na = mbar_test_wait(&aempty[2 * (p2n & (kAStages - 1)) + rt2], ((p2n / kAStages) & 1) ^ 1);
+                    nf = mbar_test_wait(&full[itn % kSStages], (itn / kSStages) & 1);
+                    na = mbar_test_wait(&aempty[2 * (p2n % kAStages) + rt2], ((p2n / kAStages) & 1) ^ 1);
                 }
                 const uint32_t s2 = __byte_perm(sp, 0, isb ? 0x3232 : 0x1010);
                 uint32_t r[32];
@@ -350,7 +359,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                                 (size_t)(2 * pair) * KB * kBlockBytes;
             const uint8_t* w1 = w0 + (size_t)KB * kBlockBytes;
             for (int kb = 0; kb < KB; ++kb, ++it) {
-                const uint32_t s = it & (kSStages - 1);
+                const uint32_t s = it % kSStages;
                 if (!tc_wait(&sempty[s], ((it / kSStages) & 1) ^ 1, abort_flag, a.err, 24)) { ok = false; break; }
                 tc_stamp(a, it, 6);
                 uint8_t* wdst = sm + kOffW + s * kWStageBytes;
@@ -388,25 +397,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
             tc_fence_after();
             for (int kb = 0; kb < KB; kb += 2, it += 2) {
                 const uint32_t p2 = it >> 1;
-                const uint32_t s0 = it & (kSStages - 1), sa = p2 & (kAStages - 1);
+                const uint32_t s0 = it % kSStages, sa = p2 % kAStages;
                 // aready implies full: the transform warps waited for both blocks' stages before arriving
                 if (!tc_wait_warp(&aready[2 * sa + t2], (p2 / kAStages) & 1, abort_flag, a.err, 27)) { ok = false; break; }
                 tc_fence_after();
                 const uint64_t bd0 = bdesc0 + s0 * (kBTileBytes >> 4);
-                const uint64_t bd1 = bdesc0 + ((s0 + 1) & (kSStages - 1)) * (kBTileBytes >> 4);
+                const uint64_t bd1 = bdesc0 + ((s0 + 1) % kSStages) * (kBTileBytes >> 4);
                 const uint32_t acol = abase + 128 * sa;
-                tc_mma_ts_elect(dacc, acol, bd0, idesc, kb != 0);
-                tc_mma_ts_elect(dacc, acol + 8, bd0 + 2, idesc, 1);
-                tc_mma_ts_elect(dacc, acol + 16, bd0 + 4, idesc, 1);
-                tc_mma_ts_elect(dacc, acol + 24, bd0 + 6, idesc, 1);
-                tc_mma_ts_elect(dacc, acol + 32, bd1, idesc, 1);
-                tc_mma_ts_elect(dacc, acol + 40, bd1 + 2, idesc, 1);
-                tc_mma_ts_elect(dacc, acol + 48, bd1 + 4, idesc, 1);
-                tc_mma_ts_elect(dacc, acol + 56, bd1 + 6, idesc, 1);
+                tc_mma8_commit3(dacc, acol, bd0, bd1, idesc, kb != 0, smem_addr(&sempty[s0]),
+                                smem_addr(&sempty[(s0 + 1) % kSStages]), smem_addr(&aempty[2 * sa + t2]));
                 issued = true;
-                tc_commit_elect(&sempty[s0]);
-                tc_commit_elect(&sempty[(s0 + 1) & (kSStages - 1)]);
-                tc_commit_elect(&aempty[2 * sa + t2]);
                 if (t2 == 0 && lane == 0) {
                     tc_stamp(a, it, 5);
                     tc_stamp(a, it + 1, 5);

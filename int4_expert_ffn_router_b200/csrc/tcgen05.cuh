@@ -93,6 +93,39 @@ __device__ __forceinline__ void mbar_arrive_elect(uint64_t* bar) {
         : "memory");
 }
 
+// The eight MMAs of two 64-input blocks into one accumulator, then one
+// commit to each of three barriers: D[d] (+)= A[a + 8 j] * B[desc_j]^T for
+// j = 0..7, where desc_j is b0 + 2 j (j < 4) or b1 + 2 (j - 4) (the start
+// address advances 32 bytes per 16 inputs), the first MMA accumulating only
+// if `accumulate` != 0; bar0..bar2 (shared addresses) each receive one
+// arrival when the MMAs have completed. Warp-converged: a single elect, one
+// lane issues everything.
+__device__ __forceinline__ void tc_mma8_commit3(uint32_t d, uint32_t a, uint64_t b0, uint64_t b1, uint32_t idesc,
+                                                uint32_t accumulate, uint32_t bar0, uint32_t bar1, uint32_t bar2) {
+    asm volatile(
+        "{\n\t.reg .pred e, p, t;\n\t.reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t"
+        ".reg .b64 d1, d2, d3, d5, d6, d7;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\tsetp.eq.b32 t, %5, %5;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\tadd.u32 a4, %1, 32;\n\t"
+        "add.u32 a5, %1, 40;\n\tadd.u32 a6, %1, 48;\n\tadd.u32 a7, %1, 56;\n\t"
+        "add.s64 d1, %2, 2;\n\tadd.s64 d2, %2, 4;\n\tadd.s64 d3, %2, 6;\n\t"
+        "add.s64 d5, %3, 2;\n\tadd.s64 d6, %3, 4;\n\tadd.s64 d7, %3, 6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], d1, %4, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], d2, %4, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], d3, %4, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], %3, %4, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], d5, %4, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], d6, %4, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], d7, %4, t;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%8];\n\t}" ::"r"(d),
+        "r"(a), "l"(b0), "l"(b1), "r"(idesc), "r"(accumulate), "r"(bar0), "r"(bar1), "r"(bar2)
+        : "memory");
+}
+
 // Thread i of the warp writes lane (taddr.lane + i), columns taddr.col .. +15.
 __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t* r) {
     asm volatile(
