@@ -18,11 +18,14 @@ namespace coli {
 // blocks of 128 rows x one 64-input group:
 //     block(rt, g) at ((rt * C/64) + g) * kBlockBytes
 // so the 128-row tile `rt` is one contiguous run over its groups. A block is
-//     nibbles [8 sub-tiles of 16 rows][4 ti][8 gi][16 bytes]  (4096 B)
+//     nibbles [8 sub-tiles of 16 rows][4 ti][8 slots][16 bytes]  (4096 B)
 //     scales  [8 sub-tiles][8] x {fp16 of row i, fp16 of row i+8} (256 B)
-// Lane l = 4*gi + ti of a sub-tile (its 16 bytes at lane_slot(l) * 16 within
-// the sub-tile: ti-major, so the four lanes of one row lie 128 bytes apart
-// and the eight rows of one ti are 128 contiguous bytes) owns rows gi and
+// Lane l = 4*gi + ti of a sub-tile keeps its 16 bytes in slot
+// lane_slot(l) = 8 ti + (gi ^ 2 ti) of the sub-tile. Both ways the kernels
+// read a sub-tile then touch 8 distinct slots modulo 8 in every quarter-warp
+// (conflict-free 16-byte shared-memory loads): a warp reading lanes 0..31
+// (quarter-warp q holds gi = 2q, 2q+1 with ti = 0..3), and eight row-owning
+// lanes gi = 0..7 reading the slots of one ti. The lane owns rows gi and
 // gi+8 and, for each
 // 16-input step s = 0..3 of the group, the inputs 16s + {2ti, 2ti+1, 2ti+8,
 // 2ti+9}: 32 nibbles in four 32-bit words, word s holding
@@ -42,7 +45,21 @@ namespace coli {
 constexpr int kGroup = 64;
 constexpr int kTileRows = 128;
 // 16-byte slot of lane l = 4*gi + ti within a 512-byte sub-tile.
-__host__ __device__ constexpr int lane_slot(int l) { return (l & 3) * 8 + (l >> 2); }
+__host__ __device__ constexpr int lane_slot(int l) { return (l & 3) * 8 + ((l >> 2) ^ (2 * (l & 3))); }
+constexpr bool lane_slots_conflict_free() {
+    for (int q = 0; q < 4; ++q) {  // a warp reading lanes 0..31, one quarter-warp at a time
+        int seen = 0;
+        for (int l = 8 * q; l < 8 * q + 8; ++l) seen |= 1 << (lane_slot(l) & 7);
+        if (seen != 0xFF) return false;
+    }
+    for (int ti = 0; ti < 4; ++ti) {  // rows gi = 0..7 reading the slots of one ti
+        int seen = 0;
+        for (int gi = 0; gi < 8; ++gi) seen |= 1 << (lane_slot(4 * gi + ti) & 7);
+        if (seen != 0xFF) return false;
+    }
+    return true;
+}
+static_assert(lane_slots_conflict_free(), "every quarter-warp reads 8 distinct 16-byte slots modulo 8");
 constexpr int kSubRows = 16;
 constexpr int kNibbleBytes = 4096;
 constexpr int kScaleBytes = 256;

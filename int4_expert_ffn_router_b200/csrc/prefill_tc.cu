@@ -233,10 +233,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                 if (warp == 0 && lane == 0) tc_stamp(a, it, 1);
                 tc_fence_after();
                 const uint8_t* blk = sm + kOffW + s * kWStageBytes + rt2 * kBlockBytes;
-                const uint8_t* rowp = blk + sub * 512 + gi * 16;  // lane 4gi+ti at slot 8ti+gi
+                const uint8_t* subp = blk + sub * 512;  // lane 4gi+ti of the sub-tile at lane_slot(4gi+ti)
                 uint4 wv[4];
 #pragma unroll
-                for (int ti = 0; ti < 4; ++ti) wv[ti] = *reinterpret_cast<const uint4*>(rowp + 128 * ti);
+                for (int ti = 0; ti < 4; ++ti) wv[ti] = *reinterpret_cast<const uint4*>(subp + 16 * lane_slot(4 * gi + ti));
                 const uint32_t sp = *reinterpret_cast<const uint32_t*>(blk + kNibbleBytes + sub * 32 + gi * 4);
                 // test the next block's phases now (non-blocking): the answers are read after the
                 // dequantisation, so a barrier that is already complete costs no wait latency
