@@ -601,10 +601,17 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
     const uint32_t stage_bytes = (uint32_t)a.sb * kBlockBytes;
     const bool has_b = lane < L;
     const int nst = (G + a.sb - 1) / a.sb;
+    bool seen = false;  // this thread saw the stage complete while working on the previous one
     for (int i = 0; i < nst; ++i) {
         uint64_t tw = 0;
         if (a.trace && ctid == 0) tw = globaltimer_ns();
-        const bool ok = wait_bar(&S.full[slot_s], phase_s, abort_flag, a, 7);
+        const bool ok = seen || wait_bar(&S.full[slot_s], phase_s, abort_flag, a, 7);
+        // test the next stage now (non-blocking); the answer is used after this stage's groups
+        bool next_full = false;
+        if (i + 1 < nst) {
+            const uint32_t ns = slot_s + 1 == (uint32_t)a.nstages ? 0 : slot_s + 1;
+            next_full = mbar_test_wait(&S.full[ns], ns == 0 ? phase_s ^ 1 : phase_s);
+        }
         if (a.trace && ctid == 0) {
             const uint64_t dw = globaltimer_ns() - tw;
             if (i == 0) S.first_wait_ns = dw;
@@ -631,6 +638,7 @@ __device__ void weight_item(FusedArgs& a, FusedSmem& S, const Item& it, uint8_t*
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.empty[slot_s]);
         if (++slot_s == (uint32_t)a.nstages) { slot_s = 0; phase_s ^= 1; }
+        seen = next_full;
     }
     const bool live = t4 < nt && !*abort_flag;
     float hv = 0.0f;
@@ -733,13 +741,16 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
     __syncthreads();
     if (tid == 0) {
         __threadfence();
-        if (atomicAdd(&a.ctl[kCtlExit], 1) == (int)gridDim.x - 1) {
-            // last CTA out: clear the control block for the next launch (keep the error)
-            const int n = ctl_ints(a.d.E, a.d.S, a.d.H, a.d.K);
-            for (int i = 0; i < n; ++i)
-                if (i != kCtlError) a.ctl[i] = 0;
-            __threadfence();
-        }
+        S.last = atomicAdd(&a.ctl[kCtlExit], 1) == (int)gridDim.x - 1;
+    }
+    __syncthreads();
+    if (S.last) {
+        // last CTA out: clear the control block for the next launch (keep the error)
+        __threadfence();
+        const int n = ctl_ints(a.d.E, a.d.S, a.d.H, a.d.K);
+        for (int i = tid; i < n; i += blockDim.x)
+            if (i != kCtlError) a.ctl[i] = 0;
+        __threadfence();
     }
 }
 

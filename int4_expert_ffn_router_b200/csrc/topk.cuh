@@ -7,10 +7,6 @@ namespace coli {
 
 constexpr int kMaxPerLane = 32;  // E <= 1024
 
-__device__ __forceinline__ bool better(double a, int ia, double b, int ib) {
-    return a > b || (a == b && ia < ib);
-}
-
 // Order-preserving 64-bit key of a double (larger value -> larger key); -0 is
 // folded into +0 so that equal values compare equal. Integer compares keep
 // the selection exact and are much cheaper than fp64 ones.
@@ -19,14 +15,12 @@ __device__ __forceinline__ unsigned long long order_key(double v) {
     return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
 }
 
-__device__ __forceinline__ bool key_better(unsigned long long ka, int ia, unsigned long long kb, int ib) {
-    return ka > kb || (ka == kb && ia < ib);
-}
-
 // One warp selects the K largest of the E logits l[0..E) (descending, ties to
 // the lower id) and their softmax weights over the selection (fp64, fixed
 // summation order). Lane k < K returns slot k in (*id, *wt). Each lane keeps
-// the best of its own values; a round takes the warp's best and only the lane
+// the best of its own values; a round takes the warp's best (three warp
+// reductions: the key's high word, its low word among the lanes holding that
+// high word, the lowest id among the lanes holding the key) and only the lane
 // that supplied it refreshes its own best. `coherent`: read the logits
 // through L2 only (they were written by another CTA).
 // Inverse of order_key.
@@ -55,14 +49,13 @@ __device__ __forceinline__ void warp_topk(const double* __restrict__ l, int E, i
     unsigned long long my_key = 0ull, top_key = 0ull;
     int my_id = -1;
     for (int k = 0; k < K; ++k) {
-        unsigned long long bk = mk;
-        int bi = mi;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long ok = __shfl_xor_sync(0xffffffffu, bk, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (key_better(ok, oi, bk, bi)) { bk = ok; bi = oi; }
-        }
+        // the warp's best: largest key (high word, then low word), then lowest id
+        const unsigned khi = (unsigned)(mk >> 32), klo = (unsigned)mk;
+        const unsigned bhi = __reduce_max_sync(0xffffffffu, khi);
+        const unsigned blo = __reduce_max_sync(0xffffffffu, khi == bhi ? klo : 0u);
+        const bool holds = khi == bhi && klo == blo;
+        const int bi = (int)__reduce_min_sync(0xffffffffu, holds ? (unsigned)mi : 0x7fffffffu);
+        const unsigned long long bk = ((unsigned long long)bhi << 32) | blo;
         if ((bi & 31) == lane && bi != 0x7fffffff) {  // the supplier drops it and refreshes its best
             mk = 0ull;
             mi = 0x7fffffff;
