@@ -215,7 +215,10 @@ coli_status coli_moe_set_tensor_cores(coli_moe_layer* layer, int mode);
  * caller; int64 [0] counts records (it may exceed capacity: later records are
  * dropped); [1..5] global-timer stamps of the plan path: the last router
  * completion seen, its atomic done, plan published, top-k started, top-k
- * done, [6..8] plan steps (scan, entries stored, before the flag release).
+ * done, [6..8] plan steps (scan, entries stored, before the flag release),
+ * [9] the earliest CTA start (atomic minimum: the caller sets it to
+ * INT64_MAX for this stamp), [10] the last CTA's exit, [11] the latest end
+ * of an output block's combine.
  * Record r at int64 16 + 8r: {cta << 40 | kind << 32 |
  * expert << 16 | tile, begin ns, end ns, ns waited for the item's first weight
  * stage, ns the item was published by the CTA's producer, total ns warp 0

@@ -372,17 +372,56 @@ template <typename XT>
 __device__ void signal_combine(FusedArgs& a, int rt, int lane) {
     const Dims& d = a.d;
     const int T = a.T, K = d.K, TK = T * d.K;
-    for (int idx = lane; idx < T * kTileRows; idx += 32) {
-        const int t = idx / kTileRows, r = rt * kTileRows + (idx % kTileRows);
-        float acc = a.residual ? a.residual[(size_t)t * d.H + r] : 0.0f;
-        for (int j = 0; j < d.S; ++j) acc += __ldcg(a.o + (size_t)(TK + j * T + t) * d.H + r);
-        for (int k = 0; k < K; ++k) {
-            const float wk = __ldcg(a.p.w + t * K + k);
-            const int q = __ldcg(a.p.pos + t * K + k);
-            acc = fmaf(wk, __ldcg(a.o + (size_t)q * d.H + r), acc);
+    constexpr int kJ = kTileRows / 32;  // rows per lane: rt * 128 + 32 j + lane
+    static_assert(kTileRows % 32 == 0, "a lane covers every 32nd row of the block");
+    // every load of a token is issued before its sums (a few round trips per
+    // token instead of one per routed slot and row)
+    for (int t = 0; t < T; ++t) {
+        float acc[kJ];
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const int r = rt * kTileRows + j * 32 + lane;
+            acc[j] = a.residual ? a.residual[(size_t)t * d.H + r] : 0.0f;
         }
-        if constexpr (sizeof(XT) == 4) reinterpret_cast<float*>(a.y)[(size_t)t * d.H + r] = acc;
-        else reinterpret_cast<__nv_bfloat16*>(a.y)[(size_t)t * d.H + r] = __float2bfloat16_rn(acc);
+        for (int s = 0; s < d.S; ++s) {
+            const float* os = a.o + (size_t)(TK + s * T + t) * d.H + rt * kTileRows + lane;
+            float v[kJ];
+#pragma unroll
+            for (int j = 0; j < kJ; ++j) v[j] = __ldcg(os + 32 * j);
+#pragma unroll
+            for (int j = 0; j < kJ; ++j) acc[j] += v[j];
+        }
+        // routed slots 32 at a time: lane k holds the position and weight of slot k0 + k;
+        // the slots' rows are read together, then added in routing order
+        for (int k0 = 0; k0 < K; k0 += 32) {
+            const int nk = min(32, K - k0);
+            const int q_l = lane < nk ? __ldcg(a.p.pos + t * K + k0 + lane) : 0;
+            const float w_l = lane < nk ? __ldcg(a.p.w + t * K + k0 + lane) : 0.0f;
+            for (int c0 = 0; c0 < nk; c0 += 8) {
+                float v[8][kJ];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int q = __shfl_sync(0xffffffffu, q_l, (c0 + c) & 31);
+                    const float* orow = a.o + (size_t)q * d.H + rt * kTileRows + lane;
+#pragma unroll
+                    for (int j = 0; j < kJ; ++j) v[c][j] = c0 + c < nk ? __ldcg(orow + 32 * j) : 0.0f;
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const float w = __shfl_sync(0xffffffffu, w_l, (c0 + c) & 31);
+                    if (c0 + c < nk) {
+#pragma unroll
+                        for (int j = 0; j < kJ; ++j) acc[j] = fmaf(w, v[c][j], acc[j]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kJ; ++j) {
+            const size_t at = (size_t)t * d.H + rt * kTileRows + j * 32 + lane;
+            if constexpr (sizeof(XT) == 4) reinterpret_cast<float*>(a.y)[at] = acc[j];
+            else reinterpret_cast<__nv_bfloat16*>(a.y)[at] = __float2bfloat16_rn(acc[j]);
+        }
     }
 }
 
@@ -408,7 +447,10 @@ __device__ void fused_signaler(FusedArgs& a, FusedSmem& S, int lane) {
             }
         }
         last = __shfl_sync(0xffffffffu, last, 0);
-        if (last && !*abort_flag) signal_combine<XT>(a, r.rt, lane);
+        if (last && !*abort_flag) {
+            signal_combine<XT>(a, r.rt, lane);
+            if (a.trace && lane == 0) atomicMax(reinterpret_cast<unsigned long long*>(a.trace) + 11, globaltimer_ns());
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&S.dempty[slot]);
     }
@@ -685,6 +727,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
         S.abort_flag = 0;
         S.staged_n = -1;
         mbar_fence_init();
+        if (a.trace) atomicMin(reinterpret_cast<unsigned long long*>(a.trace) + 9, globaltimer_ns());
     }
     __syncthreads();
     if (warp == kProducerWarp) {
@@ -746,6 +789,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_fused_kernel(FusedArgs a) {
     __syncthreads();
     if (S.last) {
         // last CTA out: clear the control block for the next launch (keep the error)
+        if (a.trace && tid == 0) a.trace[10] = (long long)globaltimer_ns();
         __threadfence();
         const int n = ctl_ints(a.d.E, a.d.S, a.d.H, a.d.K);
         for (int i = tid; i < n; i += blockDim.x)
