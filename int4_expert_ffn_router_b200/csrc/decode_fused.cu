@@ -177,10 +177,14 @@ __device__ void fused_producer(FusedArgs& a, FusedSmem& S, uint8_t* ring) {
     volatile int* abort_flag = &S.abort_flag;
     const unsigned long long* entries = entries_of(a);
     uint32_t q = 0, gs = 0, slot_s = 0, phase_s = 0;
+    bool first_ticket = true;
     while (true) {
         Item it{IT_END, 0, 0, 0, 0, 0, 0, 0, 0};
         if (!*abort_flag) {
-            const int t = atomicAdd(&a.ctl[kCtlTicket], 1);
+            // the first ticket of CTA b is b (no contended atomic at start-up); later ones
+            // come from the shared counter, after the gridDim.x static ones
+            const int t = first_ticket ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(&a.ctl[kCtlTicket], 1);
+            first_ticket = false;
             const bool routed = (t >= t_ug && t < t_sd) || (t >= t_ud && t < t_end);
             if (t < t_sg) {
                 it.kind = IT_ROUTER;
