@@ -91,6 +91,33 @@ def job_tokens_per_s(world_size, steps, tokens_per_step, total_ms):
     return world_size * steps * tokens_per_step / (total_ms * 1e-3)
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# one ncu capture, keyed by (kernel, workload). A value stands only while the
+# kernel's sources hash to the recorded digest; otherwise `traffic` is null.
+NCU_TRAFFIC = {
+    ("moe_decode_fused_kernel", "decode_b1"): dict(
+        bytes=191_460_000,
+        sources=("decode_fused.cu", "int4_mma.cuh", "common.cuh", "topk.cuh", "kernels.cuh"),
+        sha256_16="ae00eab94779e77d",
+        note="decode_b1_e16 capture (185.56 MB per launch) + 5.90 MB for the 256-expert router "
+             "(profiles/moe_decode_fused_decode_b1.md)"),
+}
+
+
+def ncu_traffic(kernel, workload):
+    rec = NCU_TRAFFIC.get((kernel, workload))
+    if rec is None:
+        return None, None
+    import hashlib
+    h = hashlib.sha256()
+    for f in rec["sources"]:
+        with open(os.path.join(ROOT, "int4_expert_ffn_router_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != rec["sha256_16"]:
+        return None, "kernel sources changed since the ncu capture"
+    return rec["bytes"], rec["note"]
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -414,6 +441,8 @@ def run_ours(args, wl, ws, rank, local):
     peak_gbs = peaks.get("hbm_gbs", 6650.0)
     tc = wl["bf16"] and T > 4  # bf16 batches of more than 4 tokens run on the tensor cores
     dom, roof = dominant_roofline(stages, nprof, T, mean_unique, wl.get("E", E_FULL), xs.element_size(), tc, peaks)
+    if roof is not None:
+        roof["traffic"], roof["traffic_note"] = ncu_traffic(roof["kernel"], args.workload)
     out = {
         "metric": METRIC, "value": round(job_tokens_per_s(ws, args.steps, T, total_ms), 2), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
