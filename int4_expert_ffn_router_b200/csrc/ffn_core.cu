@@ -25,20 +25,14 @@ constexpr int kThreads = 256;  // 8 warps = 8 sub-tiles of one 128-row tile
 constexpr int kTB = kCoreTok;  // tokens per pass over the weights (one work item)
 constexpr int kNP = 8;         // groups in flight per warp
 
-// One 128-row tile of an int4 matrix times up to kTB staged input rows.
-// Returns, per token, the fp32 results of rows gi (acc0) and gi+8 (acc1) of
-// this warp's sub-tile, summed over the four lanes of the row (valid in all).
-__device__ __forceinline__ void tile_dot(const uint8_t* __restrict__ tile, int G, const float4* xs, int nt,
-                                         float acc0[kTB], float acc1[kTB]) {
+// Issue the loads of the first kNP groups of this warp's sub-tile of a
+// 128-row tile (called before the item's inputs are staged, so their latency
+// overlaps the staging).
+__device__ __forceinline__ void tile_prefetch(const uint8_t* __restrict__ tile, int G, uint4 wb[kNP], uint32_t sb[kNP]) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gi = lane >> 2, ti = lane & 3;
+    const int gi = lane >> 2;
     const uint8_t* wp = tile + warp * 512 + lane_slot(lane) * 16;
     const uint8_t* sp = tile + kNibbleBytes + warp * 32 + gi * 4;
-#pragma unroll
-    for (int tb = 0; tb < kTB; ++tb) { acc0[tb] = 0.0f; acc1[tb] = 0.0f; }
-
-    uint4 wb[kNP];
-    uint32_t sb[kNP];
 #pragma unroll
     for (int i = 0; i < kNP; ++i) {
         if (i < G) {
@@ -46,6 +40,20 @@ __device__ __forceinline__ void tile_dot(const uint8_t* __restrict__ tile, int G
             sb[i] = ldg_stream32(sp + (size_t)i * kBlockBytes);
         }
     }
+}
+
+// One 128-row tile of an int4 matrix times up to kTB staged input rows, the
+// first kNP groups already loaded by tile_prefetch. Returns, per token, the
+// fp32 results of rows gi (acc0) and gi+8 (acc1) of this warp's sub-tile,
+// summed over the four lanes of the row (valid in all).
+__device__ __forceinline__ void tile_dot(const uint8_t* __restrict__ tile, int G, const float4* xs, int nt,
+                                         float acc0[kTB], float acc1[kTB], uint4 wb[kNP], uint32_t sb[kNP]) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gi = lane >> 2, ti = lane & 3;
+    const uint8_t* wp = tile + warp * 512 + lane_slot(lane) * 16;
+    const uint8_t* sp = tile + kNibbleBytes + warp * 32 + gi * 4;
+#pragma unroll
+    for (int tb = 0; tb < kTB; ++tb) { acc0[tb] = 0.0f; acc1[tb] = 0.0f; }
     for (int g0 = 0; g0 < G; g0 += kNP) {
 #pragma unroll
         for (int i = 0; i < kNP; ++i) {
@@ -103,13 +111,16 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_core_kernel(const uint8_t*
         const int t0 = (c - p.act_chunk[a]) * kTB;
         {
             const int nt = min(kTB, cnt - t0);
+            uint4 wb[kNP];
+            uint32_t sb[kNP];
+            tile_prefetch(tile, G, wb, sb);
             __syncthreads();
             if (threadIdx.x < nt) rows[threadIdx.x] = p.tok[off + t0 + threadIdx.x];
             __syncthreads();
             stage_rows<XT>(xs, x, rows, nt, d.H, threadIdx.x, blockDim.x);
             __syncthreads();
             float g_acc[kTB], u_acc[kTB];
-            tile_dot(tile, G, xs, nt, g_acc, u_acc);
+            tile_dot(tile, G, xs, nt, g_acc, u_acc, wb, sb);
             if (ti == 0) {
 #pragma unroll
                 for (int tb = 0; tb < kTB; ++tb)
@@ -139,13 +150,16 @@ __global__ void __launch_bounds__(kThreads, 2) down_core_kernel(const uint8_t* _
         const int t0 = (c - p.act_chunk[a]) * kTB;
         {
             const int nt = min(kTB, cnt - t0);
+            uint4 wb[kNP];
+            uint32_t sb[kNP];
+            tile_prefetch(tile, G, wb, sb);
             __syncthreads();
             if (threadIdx.x < nt) rows[threadIdx.x] = off + t0 + threadIdx.x;  // h is indexed by position
             __syncthreads();
             stage_rows<float>(xs, h, rows, nt, d.I, threadIdx.x, blockDim.x);
             __syncthreads();
             float a0[kTB], a1[kTB];
-            tile_dot(tile, G, xs, nt, a0, a1);
+            tile_dot(tile, G, xs, nt, a0, a1, wb, sb);
             if (ti == 0) {
 #pragma unroll
                 for (int tb = 0; tb < kTB; ++tb) {
