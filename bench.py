@@ -98,7 +98,7 @@ NCU_TRAFFIC = {
     ("moe_decode_fused_kernel", "decode_b1"): dict(
         bytes=191_460_000,
         sources=("decode_fused.cu", "int4_mma.cuh", "common.cuh", "topk.cuh", "kernels.cuh"),
-        sha256_16="ae00eab94779e77d",
+        sha256_16="ccc55600172f2930",
         note="decode_b1_e16 capture (185.56 MB per launch) + 5.90 MB for the 256-expert router "
              "(profiles/moe_decode_fused_decode_b1.md)"),
 }

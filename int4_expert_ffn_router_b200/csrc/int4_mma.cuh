@@ -4,14 +4,12 @@
 // A decode step multiplies each streamed weight by one to four tokens: the
 // contraction is far too thin for shared-memory tensor-core tiles, but the
 // CUDA-core instruction budget per streamed weight is the limit at HBM speed.
-// Here the weights are the B operand of mma.m16n8k16 (8 weight rows x 16
-// inputs per instruction) and the tokens the A operand: row m < 8 of A is the
-// high fp16 part of token m, row 8 + m its low part (x = hi + lo to ~22 bits
-// after a per-token power-of-two scale), so one instruction serves up to 8
-// tokens at full precision and the dequantisation costs 9 instructions per 8
-// weights: the nibbles are OR-ed into the mantissa of fp16 1024 (one LOP3 per
-// two weights) and one HFMA2 removes the bias, the bit position and the +8
-// offset exactly.
+// Here the weights are the A operand of mma.m16n8k16 (16 weight rows x 16
+// inputs per instruction) in their raw offset-binary fp16 form (one LOP3 per
+// two weights, no per-weight arithmetic), the tokens the B operand as fp16
+// hi + lo columns (about 22 significant bits after a per-token power-of-two
+// scale), and the nibble offset is removed once per group through the
+// accumulator's starting value.
 #pragma once
 
 #include "common.cuh"
@@ -24,93 +22,10 @@ __device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) 
     return d;
 }
 
-// d += A (16x16 fp16, row) * B (16x8 fp16, col), fp32 accumulate.
-__device__ __forceinline__ void mma_16816(float d[4], const uint4& a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
-}
-
-// One 32-bit weight word (layout in common.cuh) -> the B fragments of the two
-// 8-row halves of the sub-tile for one 16-input step:
-//   b00/b01: rows gi   (k = 2ti,2ti+1 | 2ti+8,2ti+9)
-//   b10/b11: rows gi+8 (same k)
-__device__ __forceinline__ void dequant_word_f16(uint32_t w, uint32_t& b00, uint32_t& b01, uint32_t& b10,
-                                                 uint32_t& b11) {
-    constexpr uint32_t MAGIC = 0x64006400u;    // fp16 1024, 1024
-    constexpr uint32_t ONE = 0x3C003C00u;      // 1.0, 1.0
-    constexpr uint32_t M1032 = 0xE408E408u;    // -1032, -1032
-    constexpr uint32_t SIXTEENTH = 0x2C002C00u;  // 1/16
-    constexpr uint32_t M72 = 0xD480D480u;      // -72, -72
-    const uint32_t ws = w >> 8;
-    const uint32_t lo0 = lop3_and_or(w, 0x000F000Fu, MAGIC);   // 1024 + v   (row gi,   k lo)
-    const uint32_t hi0 = lop3_and_or(w, 0x00F000F0u, MAGIC);   // 1024 + 16v (row gi+8, k lo)
-    const uint32_t lo1 = lop3_and_or(ws, 0x000F000Fu, MAGIC);  // row gi,   k hi
-    const uint32_t hi1 = lop3_and_or(ws, 0x00F000F0u, MAGIC);  // row gi+8, k hi
-    b00 = hfma2_u(lo0, ONE, M1032);        // v - 8
-    b01 = hfma2_u(lo1, ONE, M1032);
-    b10 = hfma2_u(hi0, SIXTEENTH, M72);    // (1024 + 16v)/16 - 72 = v - 8
-    b11 = hfma2_u(hi1, SIXTEENTH, M72);
-}
-
-// One 64-input group of a 16-row sub-tile for up to 8 tokens.
-// w: this lane's 16 bytes of the group; sc: the lane's two fp16 scale pairs
-// {(row 2t, row 2t+8), (row 2t+1, row 2t+9)}; xa: the group's A fragments
-// (4 steps x ntok x 4 lanes-of-row x 16 B); tok = lane / 4.
-// acc[0..3]: token `tok`, sub-tile rows 2t, 2t+1, 8+2t, 9+2t.
-template <int NT>
-__device__ __forceinline__ void group_mma(uint4 w, uint2 sc, const uint4* __restrict__ xa, int tok, int t, int nt,
-                                          float acc[4]) {
-    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        uint4 a = make_uint4(0u, 0u, 0u, 0u);
-        if (tok < nt) a = xa[(s * NT + tok) * 4 + t];
-        uint32_t b00, b01, b10, b11;
-        dequant_word_f16(words[s], b00, b01, b10, b11);
-        mma_16816(d0, a, b00, b01);
-        mma_16816(d1, a, b10, b11);
-    }
-    const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));  // rows 2t, 2t+8
-    const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));  // rows 2t+1, 2t+9
-    acc[0] = fmaf(s01.x, d0[0] + d0[2], acc[0]);
-    acc[1] = fmaf(s23.x, d0[1] + d0[3], acc[1]);
-    acc[2] = fmaf(s01.y, d1[0] + d1[2], acc[2]);
-    acc[3] = fmaf(s23.y, d1[1] + d1[3], acc[3]);
-}
-
 // Weights as the A operand (16 rows x 16 inputs per mma), tokens as B: column
 // n = 2j + p of B is part p (0 hi, 1 lo) of token j, so one instruction covers
-// 256 weights for up to 4 tokens. The word's four dequantised pairs are
-// exactly A fragments a0 (row gi, k lo), a1 (row gi+8, k lo), a2 (row gi,
-// k hi), a3 (row gi+8, k hi).
-// w: this lane's 16 bytes of the group; sv: fp16 scales (row gi, row gi+8);
-// xb0/xb1: the lane's B fragments for steps 0,1 and 2,3 of the group.
-// acc0/acc1: token t = lane % 4, rows gi and gi+8 (valid for t < tokens).
-__device__ __forceinline__ void group_mma_aw(uint4 w, uint32_t sv, uint4 xb0, uint4 xb1, float& acc0, float& acc1) {
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-    const uint32_t bx[8] = {xb0.x, xb0.y, xb0.z, xb0.w, xb1.x, xb1.y, xb1.z, xb1.w};
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        uint32_t r0, r1, r8, r9;  // (row gi, k lo), (row gi, k hi), (row gi+8, k lo), (row gi+8, k hi)
-        dequant_word_f16(words[s], r0, r1, r8, r9);
-        asm volatile(
-            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-            : "r"(r0), "r"(r8), "r"(r1), "r"(r9), "r"(bx[2 * s]), "r"(bx[2 * s + 1]));
-    }
-    const float2 sc = __half22float2(*reinterpret_cast<const __half2*>(&sv));
-    acc0 = fmaf(sc.x, d[0] + d[1], acc0);  // row gi: hi + lo columns of token t
-    acc1 = fmaf(sc.y, d[2] + d[3], acc1);  // row gi+8
-}
-
-// As group_mma_aw, without removing the nibble offset per weight: the A
-// fragments are the raw fp16 values 1024 + v (row gi) and 1024 + 16 v (row
+// 256 weights for up to 4 tokens. The nibble offset is not removed per weight:
+// the A fragments are the raw fp16 values 1024 + v (row gi) and 1024 + 16 v (row
 // gi+8) of the offset-binary codes v = q + 8 (one logic op per pair), and the
 // accumulators start at the group's offset correction
 //     row gi:   -1032 * X,   row gi+8:  -1152 * X     (X = the column's sum of
@@ -189,62 +104,9 @@ __device__ __forceinline__ uint32_t split_pair(float a, float b, uint32_t& lo) {
     return (uint32_t)__half_as_ushort(ha) | ((uint32_t)__half_as_ushort(hb) << 16);
 }
 
-// Stage nt (<= NT) input rows of C values as A fragments, scaled per row by a
-// power of two so that the row's largest magnitude lies in [2^14, 2^15), and
-// split into fp16 hi + lo. xa[((g*4 + s)*NT + tok)*4 + t] = {hi(k,k+1),
-// lo(k,k+1), hi(k+8,k+9), lo(k+8,k+9)}, k = 64g + 16s + 2t. scale_out[tok] =
-// the factor that undoes the row scaling. Uses consumer threads tid < nthr
-// and named barrier `bar` (two barriers); red: nthr/32 * NT floats.
-template <typename XT, int NT>
-__device__ __forceinline__ void stage_afrag(uint4* __restrict__ xa, float* scale_out, const XT* __restrict__ in,
-                                            const int* rows, int nt, int C, bool coherent, int tid, int nthr,
-                                            int bar, float* red) {
-    const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
-    float m[NT];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-        m[j] = 0.0f;
-        if (j < nt) {
-            const XT* r = in + (size_t)rows[j] * C;
-            for (int c = tid; c < C; c += nthr) m[j] = fmaxf(m[j], fabsf(load_in<XT>(r + c, coherent)));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], o));
-        if (lane == 0) red[warp * NT + j] = m[j];
-    }
-    named_bar(bar, nthr);
-    if (tid < NT) {
-        float mx = 0.0f;
-        for (int w = 0; w < nw; ++w) mx = fmaxf(mx, red[w * NT + tid]);
-        int k = 0;  // zero, subnormal or non-finite maxima: no scaling
-        const uint32_t eb = (__float_as_uint(mx) >> 23) & 0xFF;
-        if (eb != 0 && eb != 0xFF) {
-            k = 14 - ((int)eb - 127);
-            k = k < -126 ? -126 : (k > 126 ? 126 : k);
-        }
-        red[nw * NT + tid] = exp2i(k);       // multiply inputs by this
-        scale_out[tid] = exp2i(-k);          // multiply results by this
-    }
-    named_bar(bar, nthr);
-    const int G = C / kGroup;
-    for (int idx = tid; idx < nt * G * 16; idx += nthr) {
-        const int tok = idx / (G * 16);
-        const int r = idx - tok * G * 16;
-        const int g = r >> 4, s = (r >> 2) & 3, t = r & 3;
-        const int k = g * 64 + s * 16 + t * 2;
-        const XT* src = in + (size_t)rows[tok] * C + k;
-        const float f = red[nw * NT + tok];
-        const float v0 = load_in<XT>(src, coherent) * f, v1 = load_in<XT>(src + 1, coherent) * f;
-        const float v8 = load_in<XT>(src + 8, coherent) * f, v9 = load_in<XT>(src + 9, coherent) * f;
-        uint4 o;
-        o.x = split_pair(v0, v1, o.y);
-        o.z = split_pair(v8, v9, o.w);
-        xa[((g * 4 + s) * NT + tok) * 4 + t] = o;
-    }
-}
-
-// Stage nt (<= NT) rows as B fragments for group_mma_aw, per-row power-of-two
-// scaling and fp16 hi + lo split as in stage_afrag. Entry
+// Stage nt (<= NT) rows as B fragments for group_mma_aw_off, scaled per row by a
+// power of two so that the row's largest magnitude lies in [2^14, 2^15) and
+// split into fp16 hi + lo (about 22 significant bits together). Entry
 //   xb[(g*2 + h)*8*NT + lane], lane < 8*NT: column n = lane/4 (token n/2, part
 //   n%2), t = lane%4, steps s = 2h, 2h+1: {b0(s), b1(s), b0(s+1), b1(s+1)},
 //   b0(s) = pair (k, k+1), b1(s) = pair (k+8, k+9), k = 64g + 16s + 2t.

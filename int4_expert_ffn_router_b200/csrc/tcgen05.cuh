@@ -54,32 +54,10 @@ __device__ __forceinline__ void tc_dealloc(uint32_t taddr, uint32_t ncols) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Arrives once on `bar` when every tcgen05.mma this thread issued so far has completed.
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
-
-// D[tmem d] (+)= A[tmem a] * B[smem desc]^T, M = 128, kind::f16.
-__device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-        "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // Warp-converged forms: the whole warp executes them, one elected lane
-// performs the operation (keeps the operands on the uniform datapath, which
-// is several times cheaper to issue from than a one-lane branch).
-__device__ __forceinline__ void tc_mma_ts_elect(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc,
-                                                uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-        "r"(a), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
+// performs the operation (several times cheaper to issue than from a
+// one-lane branch). tc_commit_elect arrives once on `bar` when every
+// tcgen05.mma the electing thread issued so far has completed.
 __device__ __forceinline__ void tc_commit_elect(uint64_t* bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
@@ -146,36 +124,6 @@ __device__ __forceinline__ void tc_ld16_wait(uint32_t taddr, uint32_t* r) {
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
           "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
-        : "memory");
-}
-
-// 16-byte global -> shared copy; completion tracked by the issuing thread's
-// cp.async groups or by cp_async_mbar_arrive.
-__device__ __forceinline__ void cp_async16(uint32_t dst_saddr, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_saddr), "l"(src) : "memory");
-}
-// Arrive on `bar` once this thread's earlier cp.async copies have landed
-// (the arrival is one of the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// TMA gather: rows r0..r3 of a 2D tensor map (box: one row of 128 bytes,
-// 128-byte swizzle) into 4 consecutive 128-byte rows of shared memory at
-// `dst`, completing 512 bytes of transaction on `bar`. x: innermost
-// coordinate (elements; x * element size must be a multiple of 16 bytes).
-// `tmap` must be a global, constant or __grid_constant__ parameter address.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int x, int r0, int r1, int r2, int r3,
-                                            uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_addr(bar))
         : "memory");
 }
 
