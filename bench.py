@@ -118,6 +118,15 @@ def ncu_traffic(kernel, workload):
     return rec["bytes"], rec["note"]
 
 
+def step_percentiles(step_ms):
+    """p10 / median / p90 of this rank's per-step device times (ms)."""
+    v = sorted(step_ms)
+    if not v:
+        return None
+    pick = lambda q: v[min(len(v) - 1, int(round(q * (len(v) - 1))))]
+    return {"p10": round(pick(0.1), 5), "p50": round(pick(0.5), 5), "p90": round(pick(0.9), 5)}
+
+
 def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -446,6 +455,7 @@ def run_ours(args, wl, ws, rank, local):
     out = {
         "metric": METRIC, "value": round(job_tokens_per_s(ws, args.steps, T, total_ms), 2), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+        "step_ms_rank0": step_percentiles(step_ms),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if wl["bf16"] else "f32",
         "stage_note": "stage_us from a separate profiled pass (stage events add host gaps)",
@@ -531,7 +541,8 @@ def run_stack(args, wl, ws, rank, local):
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    total_ms = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, nsteps))
+    step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, nsteps)]
+    total_ms = sum(step_ms)
     # per-stage device times from a separate pass (not in the timed region)
     for L in layers:
         L.set_profiling(True)
@@ -582,6 +593,7 @@ def run_stack(args, wl, ws, rank, local):
     out = {
         "metric": METRIC, "value": round(job_tokens_per_s(ws, args.steps, T, total_ms), 2), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+        "step_ms_rank0": step_percentiles(step_ms),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded generator; random-init int4 weights of the full-size layer shape, per layer)",
         "config": {"workload": args.workload, "desc": wl["desc"], "layers": NL, "hidden": H, "inter": I,
