@@ -333,3 +333,42 @@ def test_stack_step_is_residual_of_normalised_layer(tiny):
     y, ids2, _ = oracle.moe_forward(cfg, L["wr"], None, L["experts"], nf)
     np.testing.assert_array_equal(ids, ids2)
     np.testing.assert_array_equal(xs, (x0.astype(np.float64) + y).astype(np.float32))
+
+
+# ------------------------------------------------------------- page figures
+
+
+def _page_figures():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "page_figures.txt")
+    out = {}
+    with open(path, encoding="utf-8") as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                k, v = line.split()
+                out[k] = float(v)
+    return out
+
+
+def test_expert_size_and_counts_match_the_pages_figures():
+    """The full-size expert (hidden 6144, inter 2048, int4 gs64 with fp16
+    scales) against the sizes the Colibrì background section prints: about
+    19 MB per expert, 19,456 routed experts (75 layers x 256 + the MTP head)
+    taking about 370 GB, and 6,300 of them filling 120 GB of VRAM."""
+    fig = _page_figures()
+    H, I = 6144, 2048
+    per_expert = 3 * H * I // 2 + 3 * H * I // 64 * 2   # nibbles + fp16 scales
+    assert per_expert == 20_054_016
+    assert abs(per_expert / 1e6 - fig["expert_megabytes_int4"]) / fig["expert_megabytes_int4"] < 0.1
+    assert fig["moe_layers"] * fig["routed_experts_per_layer"] + fig["routed_experts_per_layer"] == fig["routed_experts_total"]
+    total_gb = fig["routed_experts_total"] * per_expert / 1e9
+    assert abs(total_gb - fig["routed_experts_total_gigabytes"]) / fig["routed_experts_total_gigabytes"] < 0.1
+    per_hot = fig["vram_hot_gigabytes"] * 1e9 / fig["vram_hot_experts"]
+    assert abs(per_hot - per_expert) / per_expert < 0.1
+    # 8 of the 256 experts per layer; the whole model's active share from these counts
+    assert fig["routed_per_token"] == 8 and fig["routed_experts_per_layer"] == 256
+    w = 3 * H * I
+    whole = (fig["moe_layers"] * fig["routed_per_token"] * w + fig["dense_params_billion"] * 1e9) / \
+            (fig["routed_experts_total"] * w + fig["dense_params_billion"] * 1e9)
+    assert abs(whole - fig["active_fraction"]) < 0.002
+    assert abs(fig["active_params_billion"] / fig["total_params_billion"] - fig["active_fraction"]) < 0.001
