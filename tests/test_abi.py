@@ -70,4 +70,7 @@ def test_null_arguments_are_rejected(lib):
     assert L.coli_moe_route(None, None, 0, 1, None, None, None) == lib.COLI_EINVAL
     assert L.coli_moe_get_stats(None, None, None, None) == lib.COLI_EINVAL
     assert L.coli_moe_stack_forward(None, 1, None, 1, 1e-6, None) == lib.COLI_EINVAL
+    n = ctypes.c_int64(-1)
+    assert L.coli_moe_get_launch_count(None, ctypes.byref(n)) == lib.COLI_EINVAL and n.value == -1
+    assert L.coli_moe_set_tensor_cores(None, 1) == lib.COLI_EINVAL
     L.coli_moe_layer_destroy(None)  # no-op
