@@ -99,8 +99,8 @@ NCU_TRAFFIC = {
         bytes=191_460_000,
         sources=("decode_fused.cu", "int4_mma.cuh", "common.cuh", "topk.cuh", "kernels.cuh"),
         sha256_16="ccc55600172f2930",
-        note="decode_b1_e16 capture (185.56 MB per launch) + 5.90 MB for the 256-expert router "
-             "(profiles/moe_decode_fused_decode_b1.md)"),
+        note="ncu capture of the 16-expert decode case (185.56 MB per launch) + 5.90 MB for the "
+             "256-expert router"),
 }
 
 

@@ -253,18 +253,21 @@ coli_status coli_moe_set_ring(coli_moe_layer* layer, int stages, int blocks_per_
  * router_w [n_experts][hidden] fp32 and router_bias [n_experts] fp32 (or
  * NULL) are DEVICE pointers the caller owns, as are x [n_tokens][hidden]
  * (fp32 or bf16 bits), ids [n_tokens][top_k] and weights [n_tokens][top_k];
- * the results equal coli_moe_route's for the same inputs.
- * Its only scratch, the fp64 logits, is a fixed 512 KiB array in device
+ * the results equal coli_moe_route's for the same inputs (the logits are
+ * summed in the same order).
+ * Its only scratch, the fp64 logits, is a fixed 504 KiB array in device
  * memory that every GPU loading this library holds until the process exits:
  * n_tokens <= COLI_NOALLOC_MAX_TOKENS and n_experts <= COLI_NOALLOC_MAX_EXPERTS,
  * larger requests return COLI_EINVAL. All calls on a device share that array,
  * so calls that overlap on the GPU (different streams without ordering) race
  * and give wrong results; order them on one stream. The first call on each
  * device looks the array's device address up (cudaGetSymbolAddress, with that
- * device current): make that first call before any stream capture.
+ * device current): make that first call before any stream capture. The
+ * address is looked up again when the device's context has changed (after a
+ * cudaDeviceReset); make the first call after a reset outside a capture too.
  * Asynchronous on `stream`; argument errors return before any work.
  */
-#define COLI_NOALLOC_MAX_TOKENS 64
+#define COLI_NOALLOC_MAX_TOKENS 63
 #define COLI_NOALLOC_MAX_EXPERTS 1024
 coli_status coli_moe_route_noalloc(const float* router_w, const float* router_bias, int n_experts, int hidden,
                                    int top_k, const void* x, coli_dtype dtype, int n_tokens, int32_t* ids,

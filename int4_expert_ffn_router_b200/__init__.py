@@ -25,7 +25,7 @@ EXPORTS = (
     "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused", "coli_moe_set_tensor_cores",
     "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc", "coli_moe_get_launch_count",
 )
-NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 64, 1024
+NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 63, 1024
 N_STAGES = 7
 
 

@@ -12,37 +12,41 @@ namespace coli {
 template <typename YT>
 __global__ void combine_kernel(const float* __restrict__ o, Plan p, int T, int H, int K, int S,
                                const float* __restrict__ residual, YT* __restrict__ y) {
-    const int t = blockIdx.y;
-    const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c4 * 4 >= H) return;
-    float4 acc = residual ? reinterpret_cast<const float4*>(residual + (size_t)t * H)[c4] : make_float4(0, 0, 0, 0);
-    for (int j = 0; j < S; ++j) {
-        const float4 v = reinterpret_cast<const float4*>(o + (size_t)(T * K + j * T + t) * H)[c4];
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    for (int k = 0; k < K; ++k) {
-        const float wk = p.w[t * K + k];
-        const float4 v = reinterpret_cast<const float4*>(o + (size_t)p.pos[t * K + k] * H)[c4];
-        acc.x = fmaf(wk, v.x, acc.x);
-        acc.y = fmaf(wk, v.y, acc.y);
-        acc.z = fmaf(wk, v.z, acc.z);
-        acc.w = fmaf(wk, v.w, acc.w);
-    }
-    if constexpr (sizeof(YT) == 4) {
-        reinterpret_cast<float4*>(y + (size_t)t * H)[c4] = acc;
-    } else {
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 u;
-        u.x = *reinterpret_cast<uint32_t*>(&lo);
-        u.y = *reinterpret_cast<uint32_t*>(&hi);
-        reinterpret_cast<uint2*>(y + (size_t)t * H)[c4] = u;
+    // one thread per (token, 4 columns); a grid-stride loop covers any T
+    const int H4 = H / 4;
+    const size_t n = (size_t)T * H4;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        const int t = (int)(i / H4), c4 = (int)(i % H4);
+        float4 acc = residual ? reinterpret_cast<const float4*>(residual + (size_t)t * H)[c4] : make_float4(0, 0, 0, 0);
+        for (int j = 0; j < S; ++j) {
+            const float4 v = reinterpret_cast<const float4*>(o + (size_t)(T * K + j * T + t) * H)[c4];
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        for (int k = 0; k < K; ++k) {
+            const float wk = p.w[t * K + k];
+            const float4 v = reinterpret_cast<const float4*>(o + (size_t)p.pos[t * K + k] * H)[c4];
+            acc.x = fmaf(wk, v.x, acc.x);
+            acc.y = fmaf(wk, v.y, acc.y);
+            acc.z = fmaf(wk, v.z, acc.z);
+            acc.w = fmaf(wk, v.w, acc.w);
+        }
+        if constexpr (sizeof(YT) == 4) {
+            reinterpret_cast<float4*>(y + (size_t)t * H)[c4] = acc;
+        } else {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 u;
+            u.x = *reinterpret_cast<uint32_t*>(&lo);
+            u.y = *reinterpret_cast<uint32_t*>(&hi);
+            reinterpret_cast<uint2*>(y + (size_t)t * H)[c4] = u;
+        }
     }
 }
 
 cudaError_t launch_combine(const float* o, const Plan& p, int T, int H, int K, int S, const float* residual, void* y,
                            coli_dtype ydt, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    dim3 grid((H / 4 + 127) / 128, T);
+    const size_t blocks = ((size_t)T * (H / 4) + 127) / 128;
+    const int grid = (int)(blocks < 148 * 32 ? blocks : 148 * 32);
     if (ydt == COLI_F32)
         combine_kernel<float><<<grid, 128, 0, st>>>(o, p, T, H, K, S, residual, (float*)y);
     else

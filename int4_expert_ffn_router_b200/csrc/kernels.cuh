@@ -9,6 +9,9 @@
 namespace coli {
 
 // router.cu
+// From this batch size on (with a partial-sum scratch) the router uses the
+// blocked GEMM form, which sums each logit in another order.
+constexpr int kRouterGemmMinTok = 64;
 // part: optional scratch of part_cap doubles for split-input partial sums
 // (batches of kRouterGemmMinTok tokens and more use the blocked GEMM form).
 cudaError_t launch_router_logits(const float* wr, const float* bias, const void* x, coli_dtype dt, int T, int H, int E,

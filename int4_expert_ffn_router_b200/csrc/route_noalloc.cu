@@ -9,6 +9,8 @@
 // allocated at create time; this entry point needs neither: its only scratch,
 // the fp64 logits, lives in a fixed array in device memory that every GPU
 // loading the library holds until the process exits.
+#include <cuda.h>
+
 #include <mutex>
 #include <string>
 
@@ -20,14 +22,51 @@
 namespace {
 
 // fp64 logits of up to COLI_NOALLOC_MAX_TOKENS x COLI_NOALLOC_MAX_EXPERTS
-// (512 KiB). Every call on a device shares it and it keeps the last call's
+// (504 KiB). Every call on a device shares it and it keeps the last call's
 // values; the router kernel writes every logit it later reads, so nothing in
-// it has to start at zero.
+// it has to start at zero. The token limit stays below the batch size from
+// which coli_moe_route switches to its split blocked form, so both entry
+// points sum every logit in the same order.
+static_assert(COLI_NOALLOC_MAX_TOKENS < coli::kRouterGemmMinTok,
+              "the no-alloc routing must sum logits in the same order as coli_moe_route");
 __device__ __align__(256) double g_noalloc_logits[COLI_NOALLOC_MAX_TOKENS * COLI_NOALLOC_MAX_EXPERTS];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
-double* g_scratch[kMaxDevices] = {};  // device address of g_noalloc_logits, per device
+// Device address of g_noalloc_logits per device, with the id of the context
+// it was looked up in: a device reset makes a new context (new id) in which
+// the module, and the array, may sit at another address.
+double* g_scratch[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current context, or 0 when it cannot be read
+// (then the address is looked up on every call).
+unsigned long long current_ctx_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static bool resolved = false;
+    if (!resolved) {
+        void* f0 = nullptr;
+        void* f1 = nullptr;
+        cudaDriverEntryPointQueryResult q0, q1;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f0, cudaEnableDefault, &q0) == cudaSuccess &&
+            q0 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f0);
+            get_id = reinterpret_cast<CtxGetIdFn>(f1);
+        }
+        resolved = true;
+    }
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 coli_status fail(coli_status s, const std::string& what) {
     coli::set_last_error(what);  // reported by coli_last_error()
@@ -57,14 +96,17 @@ COLI_API coli_status coli_moe_route_noalloc(const float* router_w, const float* 
     if (dev < 0 || dev >= kMaxDevices) return fail(COLI_EUNSUPPORTED, "device index above 63");
     double* scratch = nullptr;
     {
-        // First call on a device: look up the device address of the array
+        // First call on a device (or in a new context after a device reset):
+        // look up the device address of the array, with that device current
         // (in host code its name is only a host-side stand-in).
         std::lock_guard<std::mutex> lock(g_mutex);
-        if (!g_scratch[dev]) {
+        const unsigned long long ctx = g_scratch[dev] ? current_ctx_id() : 0;
+        if (!g_scratch[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
             void* p = nullptr;
             e = cudaGetSymbolAddress(&p, g_noalloc_logits);
             if (e != cudaSuccess) return fail(COLI_ECUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
             g_scratch[dev] = static_cast<double*>(p);
+            g_scratch_ctx[dev] = current_ctx_id();
         }
         scratch = g_scratch[dev];
     }

@@ -21,7 +21,6 @@ namespace coli {
 // four quarters are summed in a fixed order through shared memory.
 // ---------------------------------------------------------------------------
 constexpr int kRouterTok = 4;
-constexpr int kRouterGemmMinTok = 64;  // from this batch size on, the blocked GEMM form
 
 template <typename XT>
 __device__ __forceinline__ void load4(const XT* p, double v[4]);

@@ -31,11 +31,22 @@ def test_tensor_roofline_counts_algorithmic_flops():
     assert roof["frac_of_sustained"] == pytest.approx(roof["achieved"] / 1200.0, rel=1e-3)
 
 
+def _digest(files):
+    import hashlib
+    import os
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(bench.ROOT, "int4_expert_ffn_router_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def test_recorded_traffic_needs_unchanged_sources(monkeypatch):
-    b, note = bench.ncu_traffic("moe_decode_fused_kernel", "decode_b1")
-    assert b is not None and b > 186_000_000  # recorded for the current sources
+    key = ("moe_decode_fused_kernel", "decode_b1")
     assert bench.ncu_traffic("moe_decode_fused_kernel", "decode_b32") == (None, None)
-    rec = dict(bench.NCU_TRAFFIC[("moe_decode_fused_kernel", "decode_b1")], sha256_16="0" * 16)
-    monkeypatch.setitem(bench.NCU_TRAFFIC, ("moe_decode_fused_kernel", "decode_b1"), rec)
-    b, note = bench.ncu_traffic("moe_decode_fused_kernel", "decode_b1")
+    rec = dict(bytes=190_000_000, sources=("decode_fused.cu", "common.cuh"), note="test record")
+    monkeypatch.setitem(bench.NCU_TRAFFIC, key, dict(rec, sha256_16=_digest(rec["sources"])))
+    assert bench.ncu_traffic(*key) == (190_000_000, "test record")  # sources as captured
+    monkeypatch.setitem(bench.NCU_TRAFFIC, key, dict(rec, sha256_16="0" * 16))
+    b, note = bench.ncu_traffic(*key)
     assert b is None and "changed" in note

@@ -2,7 +2,7 @@
 
 Routing (ids, order, weights' selection), the batch-union plan (counts,
 offsets, unique set, permutation) are compared bit for bit; outputs within
-the benchmark spec's tolerances:
+these tolerances:
   fp32 path: max|y - y_ref| <= 1e-3 * max|y_ref|
   bf16 path: ||y - y_ref||_2 <= 5e-3 * ||y_ref||_2
 """

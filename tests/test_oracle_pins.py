@@ -335,6 +335,83 @@ def test_stack_step_is_residual_of_normalised_layer(tiny):
     np.testing.assert_array_equal(xs, (x0.astype(np.float64) + y).astype(np.float32))
 
 
+def _zero_layer(c):
+    """Zero router, all-zero routed and shared experts (codes 0, scales 0)."""
+    nq, ns = synth.expert_sizes(c["H"], c["I"])
+    zero = (np.zeros(nq, np.uint8), np.zeros(ns, np.uint16))
+    return np.zeros((c["E"], c["H"]), np.float32), [zero] * (c["E"] + c["S"])
+
+
+def test_stack_step_with_a_zero_layer_returns_x_bit_for_bit():
+    """Zero router (all logits tie at 0) and all-zero experts: the MoE term is
+    exactly 0, so the step must hand back x itself. Replacing x by the layer
+    output, or scaling the residual, fails here."""
+    c = cases.TINY
+    wr, experts = _zero_layer(c)
+    x = (synth.x_f32(9, 0, 3, c["H"]) * 13.0).astype(np.float32)
+    xs = x.copy()
+    ids = oracle.stack_step(cases.oracle_cfg(c), wr, None, experts, xs)
+    assert np.array_equal(xs.view(np.uint32), x.view(np.uint32))
+    assert ids.tolist() == [[0, 1]] * 3  # equal logits go to the lower ids
+
+
+def test_stack_step_increment_does_not_depend_on_the_scale_of_x(tiny):
+    """With eps = 0, RMSNorm(2^k x) == RMSNorm(x) exactly (every operation is
+    scaled by a power of two), so the increment x_out - x of a step must be the
+    same for x and 2^k x up to the final fp32 rounding of each sum. A norm
+    applied to the layer output instead of its input, or a missing norm, makes
+    the increment grow with the scale (SwiGLU is not homogeneous)."""
+    c, L, x = tiny
+    cfg = cases.oracle_cfg(c)
+    x0 = x.astype(np.float32)
+    inc = {}
+    out = {}
+    for k in (0, 5):
+        xs = (x0 * np.float32(2.0 ** k)).astype(np.float32)
+        xin = xs.astype(np.float64)
+        oracle.stack_step(cfg, L["wr"], None, L["experts"], xs, eps=0.0)
+        out[k] = xs
+        inc[k] = xs.astype(np.float64) - xin
+    half_ulp = lambda a: np.spacing(np.abs(a).astype(np.float32)).astype(np.float64) / 2
+    bound = half_ulp(out[0]) + half_ulp(out[5])
+    assert np.all(np.abs(inc[5] - inc[0]) <= bound)
+    assert np.abs(inc[0]).max() > 1e-3  # the layer term is not trivially zero
+
+
+def test_stack_step_closed_form_with_one_basis_expert():
+    """Zero router and routed experts; the shared expert has gate/up codes only
+    in column j and down = identity on the first I rows. Then, with
+    n = x / sqrt(mean(x^2) + eps) rounded to fp32,
+        out[r] = fp32(x[r] + silu(n_j G_rj sg) * (n_j U_rj su))   for r < I,
+        out[r] = x[r]                                             for r >= I.
+    eps is large enough that putting it outside the square root, or using the
+    sum instead of the mean, changes n_j by far more than the tolerance."""
+    c = dict(cases.TINY, S=1)
+    H, I, E = c["H"], c["I"], c["E"]
+    j, eps = 37, 0.25
+    gate_q = np.array([(r % 15) - 7 for r in range(I)])
+    up_q = np.array([7 - (r % 13) for r in range(I)])
+    wr, experts = _zero_layer(c)
+    experts = list(experts)
+    experts[E] = _basis_expert(H, I, j, gate_q, up_q, 0.5, 0.25)
+    rng = np.random.default_rng(11)
+    x = (rng.integers(-8, 9, size=(2, H)) * 0.125).astype(np.float32)  # sum of squares exact in fp64
+    xs = x.copy()
+    oracle.stack_step(cases.oracle_cfg(c), wr, None, experts, xs, eps=eps)
+    for t in range(2):
+        xt = x[t].astype(np.float64)
+        ms = float(np.sum(xt * xt)) / H
+        nj = float(np.float32(xt[j] / math.sqrt(ms + eps)))
+        ref = xt.copy()
+        for r in range(I):
+            g = nj * gate_q[r] * 0.5
+            u = nj * up_q[r] * 0.25
+            ref[r] = xt[r] + g / (1.0 + math.exp(-g)) * u
+        ref32 = ref.astype(np.float32).astype(np.float64)
+        np.testing.assert_allclose(xs[t].astype(np.float64), ref32, rtol=2.5e-7, atol=1e-30)
+        assert np.array_equal(xs[t, I:], x[t, I:])
+
+
 # ------------------------------------------------------------- page figures
 
 
