@@ -273,6 +273,15 @@ coli_status coli_moe_route_noalloc(const float* router_w, const float* router_bi
                                    int top_k, const void* x, coli_dtype dtype, int n_tokens, int32_t* ids,
                                    float* weights, coli_stream stream);
 
+/*
+ * Testing aid for the out-of-memory paths: from now on, the nth device
+ * allocation this library makes for a layer (create, set_experts) fails as
+ * if the device had no memory left; 0 disables. The failing call returns
+ * COLI_ENOMEM, frees what it had allocated, and create leaves *out NULL.
+ * Process-wide; nth < 0 returns COLI_EINVAL.
+ */
+coli_status coli_moe_debug_fail_alloc(int nth);
+
 /* Bytes of one expert in the int4 gs64 container (nibbles + fp16 scales). */
 int64_t coli_moe_expert_bytes(int hidden, int inter);
 

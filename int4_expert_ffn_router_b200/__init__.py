@@ -24,6 +24,7 @@ EXPORTS = (
     "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
     "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused", "coli_moe_set_tensor_cores",
     "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc", "coli_moe_get_launch_count",
+    "coli_moe_debug_fail_alloc",
 )
 NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 63, 1024
 N_STAGES = 7
@@ -71,6 +72,7 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_route_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, i32, i32, vp, vp, vp]
     L.coli_moe_set_fused.argtypes = [vp, i32]
     L.coli_moe_set_tensor_cores.argtypes = [vp, i32]
+    L.coli_moe_debug_fail_alloc.argtypes = [i32]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
     L.coli_last_error.argtypes = []
@@ -229,7 +231,7 @@ class Layer:
 def route_noalloc(router_w, router_bias, n_experts: int, hidden: int, top_k: int, x, ids, weights,
                   n_tokens: int | None = None, stream=None) -> None:
     """Routing without a layer and without any device allocation (fixed
-    512 KiB scratch in the library; at most 64 tokens and 1024 experts)."""
+    504 KiB scratch in the library; at most 63 tokens and 1024 experts)."""
     T = x.shape[0] if n_tokens is None else n_tokens
     _check(lib.coli_moe_route_noalloc(_ptr(router_w), _ptr(router_bias), n_experts, hidden, top_k, _ptr(x),
                                       _dtype_of(x), T, _ptr(ids), _ptr(weights), _stream(stream)),
@@ -242,6 +244,11 @@ def stack_forward(layers, x, n_tokens: int | None = None, eps: float = 1e-6, str
     arr = (ctypes.c_void_p * len(layers))(*[l.handle.value for l in layers])
     _check(lib.coli_moe_stack_forward(ctypes.cast(arr, ctypes.c_void_p), len(layers), _ptr(x), T, eps,
                                       _stream(stream)), "coli_moe_stack_forward")
+
+
+def debug_fail_alloc(nth: int) -> None:
+    """Make the nth device allocation of the library from now on fail (0: off)."""
+    _check(lib.coli_moe_debug_fail_alloc(nth), "coli_moe_debug_fail_alloc")
 
 
 def make_config(hidden, inter, n_experts, top_k, n_shared, max_tokens) -> Config:

@@ -1,6 +1,7 @@
 // layer.cu -- the C ABI (include/coli_moe.h): layer object, weight upload and
 // repack, workspace, and the forward sequence on one stream.
 #include <algorithm>
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -33,6 +34,30 @@ coli_status cuda_fail(cudaError_t e, const char* where) {
     } while (0)
 
 size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// Testing aid (coli_moe_debug_fail_alloc): when positive, the allocation
+// that brings the count to zero fails as if the device were out of memory.
+std::atomic<int> g_fail_alloc{0};
+
+// Every device allocation of a layer goes through here.
+cudaError_t dev_alloc(void** p, size_t bytes) {
+    int k = g_fail_alloc.load();
+    while (k > 0 && !g_fail_alloc.compare_exchange_weak(k, k - 1)) {
+    }
+    if (k == 1) {
+        *p = nullptr;
+        return cudaErrorMemoryAllocation;
+    }
+    return cudaMalloc(p, bytes);
+}
+
+template <typename T>
+cudaError_t dev_alloc(T** p, size_t bytes) {
+    void* v = nullptr;
+    cudaError_t e = dev_alloc(&v, bytes);
+    *p = static_cast<T*>(v);
+    return e;
+}
 
 // Switches to `dev` for the lifetime of the guard.
 struct DeviceGuard {
@@ -155,6 +180,12 @@ static void free_layer(coli_moe_layer* L) {
     delete L;
 }
 
+COLI_API coli_status coli_moe_debug_fail_alloc(int nth) {
+    if (nth < 0) return fail(COLI_EINVAL, "nth must be >= 0");
+    g_fail_alloc.store(nth);
+    return COLI_OK;
+}
+
 COLI_API int64_t coli_moe_expert_bytes(int hidden, int inter) {
     return 3LL * hidden * inter / 2 + 3LL * hidden * inter / 64 * 2;
 }
@@ -176,7 +207,11 @@ COLI_API coli_status coli_moe_layer_set_experts(coli_moe_layer* L, int first, in
         const uint8_t* eq = q + (size_t)i * nq;
         const uint16_t* es = scales + (size_t)i * ns;
         if (!dev_q || !dev_s) {
-            if (!L->staging) CUDA_TRY(cudaMalloc(&L->staging, align256(nq) + ns * 2), "cudaMalloc(staging)");
+            if (!L->staging) {
+                cudaError_t e = dev_alloc(&L->staging, align256(nq) + ns * 2);
+                if (e == cudaErrorMemoryAllocation) return fail(COLI_ENOMEM, "cudaMalloc(staging): out of memory");
+                if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(staging)");
+            }
             CUDA_TRY(cudaMemcpy(L->staging, eq, nq, cudaMemcpyDefault), "copy expert nibbles");
             CUDA_TRY(cudaMemcpy(L->staging + align256(nq), es, ns * 2, cudaMemcpyDefault), "copy expert scales");
             eq = L->staging;
@@ -240,9 +275,9 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
         return s;
     };
     cudaError_t e;
-    if ((e = cudaMalloc(&L->weights, (size_t)(d.E + d.S) * d.expert_stride)) != cudaSuccess) return bail(e, "cudaMalloc(weights)");
-    if ((e = cudaMalloc(&L->router_w, (size_t)d.E * d.H * 4)) != cudaSuccess) return bail(e, "cudaMalloc(router)");
-    if ((e = cudaMalloc(&L->router_b, (size_t)d.E * 4)) != cudaSuccess) return bail(e, "cudaMalloc(bias)");
+    if ((e = dev_alloc(&L->weights, (size_t)(d.E + d.S) * d.expert_stride)) != cudaSuccess) return bail(e, "cudaMalloc(weights)");
+    if ((e = dev_alloc(&L->router_w, (size_t)d.E * d.H * 4)) != cudaSuccess) return bail(e, "cudaMalloc(router)");
+    if ((e = dev_alloc(&L->router_b, (size_t)d.E * 4)) != cudaSuccess) return bail(e, "cudaMalloc(bias)");
 
     // workspace
     const size_t TE = (size_t)Tm * d.E;
@@ -255,7 +290,7 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     constexpr int kRegions = sizeof(sz) / sizeof(sz[0]);
     size_t total = 0;
     for (size_t s : sz) total += align256(s);
-    if ((e = cudaMalloc(&L->ws, total)) != cudaSuccess) return bail(e, "cudaMalloc(workspace)");
+    if ((e = dev_alloc(&L->ws, total)) != cudaSuccess) return bail(e, "cudaMalloc(workspace)");
     L->ws_bytes = total;
     uint8_t* cur = L->ws;
     void* ptrs[kRegions];

@@ -74,3 +74,8 @@ def test_null_arguments_are_rejected(lib):
     assert L.coli_moe_get_launch_count(None, ctypes.byref(n)) == lib.COLI_EINVAL and n.value == -1
     assert L.coli_moe_set_tensor_cores(None, 1) == lib.COLI_EINVAL
     L.coli_moe_layer_destroy(None)  # no-op
+
+
+def test_debug_fail_alloc_validates_its_argument(lib):
+    assert lib.lib.coli_moe_debug_fail_alloc(-1) == lib.COLI_EINVAL
+    assert lib.lib.coli_moe_debug_fail_alloc(0) == lib.COLI_OK

@@ -1,0 +1,67 @@
+"""Failure handling on the GPU, without making the GPU fault or hang.
+
+Out of memory is made on the host: coli_moe_debug_fail_alloc makes the nth
+device allocation of layer creation fail as if the device were full. Each
+failing create must return COLI_ENOMEM, leave nothing allocated (the
+device's free memory is the same before and after) and leave the library
+usable.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import cases
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def _host_args(coli, c, max_tokens=8):
+    L = cases.host_layer(c, seed=c["seed"])
+    q = np.concatenate([e[0] for e in L["experts"]])
+    s = np.concatenate([e[1] for e in L["experts"]])
+    nq, ns = synth.expert_sizes(c["H"], c["I"])
+    E = c["E"]
+    cfg = coli.make_config(c["H"], c["I"], E, c["K"], c["S"], max_tokens)
+    return L, (cfg, L["wr"], None, q[:E * nq], s[:E * ns], q[E * nq:], s[E * ns:])
+
+
+def test_create_out_of_memory_at_each_allocation(gpu):
+    import int4_expert_ffn_router_b200 as coli
+
+    c = cases.TINY
+    L, args = _host_args(coli, c)
+    coli.Layer(*args, device=0).close()  # module loading and the context are not counted below
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    failed = 0
+    try:
+        for nth in range(1, 9):
+            coli.debug_fail_alloc(nth)
+            try:
+                layer = coli.Layer(*args, device=0)
+            except coli.ColiError as e:
+                assert e.status == coli.COLI_ENOMEM, str(e)
+                failed += 1
+                assert torch.cuda.mem_get_info()[0] == free0, f"allocation {nth}: device memory leaked"
+                continue
+            layer.close()  # fewer than nth allocations: the create succeeded
+            break
+    finally:
+        coli.debug_fail_alloc(0)
+    # weights, router, bias, workspace and the staging buffer of host sources
+    assert failed == 5
+    assert torch.cuda.mem_get_info()[0] == free0
+    # the library still works: a forward through a fresh layer matches the oracle
+    layer = coli.Layer(*args, device=0)
+    x = synth.x_f32(c["seed"], 3, 2, c["H"])
+    xd = torch.from_numpy(x).to(gpu)
+    yd = torch.empty_like(xd)
+    layer.forward(xd, yd)
+    layer.sync()
+    y_ref, _, _ = oracle.moe_forward(cases.oracle_cfg(c), L["wr"], None, L["experts"], x)
+    y = yd.cpu().numpy().astype(np.float64)
+    assert np.abs(y - y_ref).max() <= 1e-3 * np.abs(y_ref).max()
+    layer.close()
