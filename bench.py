@@ -281,48 +281,93 @@ def oracle_sample(wl, budget_s):
 
 # -------------------------------------------------------------------- GPU side
 class Clocks:
-    """nvidia-smi sampler for the timed region."""
+    """SM clocks over the timed region, two ways: nvidia-smi sampled every
+    20 ms (clock and throttle reasons), and per-SM clock-counter / global-timer
+    stamps taken by a one-block-per-SM kernel just before and just after the
+    timed loop, which give each SM's mean clock rate over the region however
+    short it is."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, index):
+    def __init__(self, index, coli=None, torch=None, stream=None):
         self.index = index
+        self.coli, self.torch, self.stream = coli, torch, stream
         self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.file, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+        self.stamps = None
+        if coli is not None:
+            n = torch.cuda.get_device_properties(index).multi_processor_count
+            self.n_sm = n
+            self.stamps = torch.zeros((2, n, 3), dtype=torch.int64, device=torch.device("cuda", index))
+            coli.clock_stamp(self.stamps[0], n, stream=stream)
+
+    def end_region(self):
+        """Second stamp, enqueued right after the timed loop."""
+        if self.stamps is not None:
+            self.coli.clock_stamp(self.stamps[1], self.n_sm, stream=self.stream)
+
+    @staticmethod
+    def query_once(index):
+        """One nvidia-smi reading (max clock and throttle reasons right now)."""
+        try:
+            out = subprocess.run(["nvidia-smi", "-i", str(index), f"--query-gpu={Clocks.FIELDS}",
+                                  "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=20)
+            return [out.stdout.strip().split(",")]
+        except Exception:
+            return []
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(5)
-        except Exception:
-            self.proc.kill()
-        self.file.flush()
-        self.file.seek(0)
-        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        rows = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(5)
+            except Exception:
+                self.proc.kill()
+            self.file.flush()
+            self.file.seek(0)
+            rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
         os.unlink(self.file.name)
+        sampled = len(rows)
+        if not rows:
+            rows = self.query_once(self.index)
         sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
             try:
-                sm.append(float(r[1]))
+                if sampled:
+                    sm.append(float(r[1]))
                 mx = max(mx, float(r[2]))
-                for n, v in zip(names, r[5:9]):
+                for n, v in zip(self.REASONS, r[5:9]):
                     if v.strip().lower() == "active":
                         reasons.add(n)
             except (ValueError, IndexError):
                 continue
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        out = {"sm_max_mhz": mx or None, "reasons": sorted(reasons), "samples": sampled}
+        if sm:
+            out["sm_mhz"] = statistics.median(sm)
+            out["sm_mhz_source"] = "nvidia-smi, sampled every 20 ms during the timed region"
+        if self.stamps is not None:
+            st = self.stamps.cpu().numpy()
+            mhz = self.coli.sm_clock_mhz(st[0], st[1])
+            if mhz:
+                out["sm_mhz_stamps"] = round(statistics.median(mhz), 1)
+                out["sm_mhz_stamps_min"] = round(min(mhz), 1)
+                out["stamped_sms"] = len(mhz)
+                if "sm_mhz" not in out:
+                    out["sm_mhz"] = out["sm_mhz_stamps"]
+                    out["sm_mhz_source"] = ("median over SMs of clock cycles / global-timer ns between "
+                                            "stamps taken right before and after the timed loop")
+        if not sampled:
+            out["reasons_note"] = "region shorter than one sample: reasons read once right after it"
+        return out
 
 
 def build_layer(torch, coli, synth, wl, device, max_tokens, layer_idx=0):
@@ -346,6 +391,90 @@ def build_layer(torch, coli, synth, wl, device, max_tokens, layer_idx=0):
     del q, s, wr
     torch.cuda.empty_cache()
     return layer
+
+
+E2E_METHOD = ("pipelined through the public API: pinned host x of step j copied to a device buffer on an upload "
+              "stream, the forward on the compute stream, y copied back to pinned host memory on a download "
+              "stream; two buffers per side, so step j+1's upload and step j-1's download overlap step j's "
+              "forward; one event pair around all steps; L2 not flushed (each step reads its weights from HBM)")
+
+
+def e2e_pipelined(torch, dev, stream, xdev_steps, forward, shape, dtype, steps, dist, inplace=False):
+    """Device ms for `steps` end-to-end steps: H2D of the step's input from
+    pinned host memory, forward(x, y), D2H of y into pinned host memory
+    (inplace: forward(x, None) updates x, which is downloaded)."""
+    xh = xdev_steps[:steps].cpu().pin_memory()
+    yh = [torch.empty(shape, dtype=dtype).pin_memory() for _ in range(2)]
+    xin = [torch.empty(shape, dtype=dtype, device=dev) for _ in range(2)]
+    yout = [torch.empty(shape, dtype=dtype, device=dev) for _ in range(2)]
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    h2d = [ev() for _ in range(steps)]
+    fwd = [ev() for _ in range(steps)]
+    d2h = [ev() for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    up.wait_event(t0)
+    for j in range(steps):
+        b = j % 2
+        if j >= 2:
+            # xin[b] is free once forward j-2 has read it (and, in place, once it is downloaded)
+            up.wait_event(d2h[j - 2] if inplace else fwd[j - 2])
+        with torch.cuda.stream(up):
+            xin[b].copy_(xh[j], non_blocking=True)
+        h2d[j].record(up)
+        stream.wait_event(h2d[j])
+        if j >= 2:
+            stream.wait_event(d2h[j - 2])  # yout[b] is free once its download is done
+        forward(xin[b], None if inplace else yout[b])
+        fwd[j].record(stream)
+        down.wait_event(fwd[j])
+        with torch.cuda.stream(down):
+            yh[b].copy_(xin[b] if inplace else yout[b], non_blocking=True)
+        d2h[j].record(down)
+    stream.wait_event(d2h[steps - 1])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1)
+    return max_over_ranks(ms, dist, dev)
+
+
+def output_error(torch, coli, synth, wl, layer, x_step, y, stream, n_tok=2):
+    """Error of one step's outputs against the fp64 oracle, on its first
+    n_tok tokens (only the experts they select are generated): max relative
+    error for fp32, relative L2 for bf16."""
+    import numpy as np
+    import oracle
+    layer.forward(x_step, y, stream=stream)
+    torch.cuda.synchronize()
+    T = x_step.shape[0]
+    n = min(n_tok, T)
+    E = wl.get("E", E_FULL)
+    if wl["bf16"]:
+        xh = x_step[:n].view(torch.int16).cpu().numpy().view(np.uint16)
+        yg = (y[:n].view(torch.int16).cpu().numpy().view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+    else:
+        xh = x_step[:n].cpu().numpy()
+        yg = y[:n].cpu().numpy()
+    bias = synth.zipf_bias(0, 0, E)[0] if wl["zipf"] else None
+    wr = synth.router(0, 0, E, H)
+    ids, _ = oracle.topk(oracle.router_logits(wr, bias, xh), K)
+    experts = [None] * (E + S)
+    for e in set(ids.ravel().tolist()) | set(range(E, E + S)):
+        experts[e] = synth.expert(0, 0, e, H, I)
+    cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S)
+    y_ref, _, _ = oracle.moe_forward(cfg, wr, bias, experts, xh)
+    yg = yg.astype(np.float64)
+    if wl["bf16"]:
+        val = float(np.linalg.norm(yg - y_ref) / np.linalg.norm(y_ref))
+        kind = "relative L2 error (bf16 path)"
+    else:
+        val = float(np.abs(yg - y_ref).max() / np.abs(y_ref).max())
+        kind = "max |y - y_oracle| / max |y_oracle| (fp32 path)"
+    return {"value": val, "kind": kind, "sample": f"tokens 0..{n - 1} of the first timed step vs the fp64 oracle"}
 
 
 def run_ours(args, wl, ws, rank, local):
@@ -388,13 +517,14 @@ def run_ours(args, wl, ws, rank, local):
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks = Clocks(local)
+    clocks = Clocks(local, coli, torch, stream)
     n0 = layer.launch_count()
     for i in range(args.warmup, nsteps):
         ev[i][0].record(stream)
         layer.forward(xs[i], y, stream=stream)
         ev[i][1].record(stream)
         flush.zero_()
+    clocks.end_region()
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
     launches = layer.launch_count() - n0
@@ -413,27 +543,10 @@ def run_ours(args, wl, ws, rank, local):
     total_ms = sum(step_ms)
     total_ms = max_over_ranks(total_ms, dist, dev)
 
-    # end to end through the C ABI with host buffers: pinned H2D of the step's
-    # x, forward, D2H of y, every step inside the events.
-    xh = xs[args.warmup:].cpu().pin_memory()
-    yh = torch.empty((T, H), dtype=xdt).pin_memory()
-    xin = torch.empty((T, H), dtype=xdt, device=dev)
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    for j in range(args.steps):
-        ev2[j][0].record(stream)
-        xin.copy_(xh[j], non_blocking=True)
-        layer.forward(xin, y, stream=stream)
-        yh.copy_(y, non_blocking=True)
-        ev2[j][1].record(stream)
-        flush.zero_()
-    torch.cuda.synchronize(dev)
-    e2e_ms = sum(ev2[j][0].elapsed_time(ev2[j][1]) for j in range(args.steps))
-    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
-    if dist:
-        dist.barrier()
+    # end to end through the C ABI with host buffers (pinned x in, y out)
+    e2e_ms = e2e_pipelined(torch, dev, stream, xs[args.warmup:], lambda xin, yout: layer.forward(xin, yout, stream=stream),
+                           (T, H), xdt, args.steps, dist)
+    err = output_error(torch, coli, synth, wl, layer, xs[args.warmup], y, stream) if rank == 0 else None
 
     if rank != 0:
         layer.close()
@@ -468,21 +581,51 @@ def run_ours(args, wl, ws, rank, local):
         "hbm_frac_of_measured": round(gbs / peak_gbs, 4),
         "unique_experts_per_step": round(mean_unique, 2),
         "bytes_per_step": int(sum(bytes_step) / len(bytes_step)),
-        "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items()},
+        "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items() if v > 0},
         "roofline": roof,
         "gpu_launches": launches,
+        "gpu_launches_note": "forward kernels in the timed loop; two clock-stamp kernels bracket the loop",
+        "max_rel_err": err,
         "compute": ("int4 weights dequantised to f16 in tensor memory, tcgen05 f16 MMA, f32 accumulate; "
                     "bf16 tokens scaled by powers of two to f16 (exact)") if tc else
                    ("int4 weights as raw f16 codes in mma.sync, f32 accumulate, fp64 router" if T <= 4 else
                     "int4 weights dequantised to f32 on CUDA cores, fp64 router"),
         "e2e": {"value": round(job_tokens_per_s(ws, args.steps, T, e2e_ms), 2), "unit": "tokens/s",
-                "h2d_bytes_per_step": T * H * xs.element_size(), "d2h_bytes_per_step": T * H * xs.element_size()},
+                "h2d_bytes_per_step": T * H * xs.element_size(), "d2h_bytes_per_step": T * H * xs.element_size(),
+                "method": E2E_METHOD},
         "clocks": clk,
     }
     layer.close()
     if dist:
         dist.destroy_process_group()
     return out
+
+
+def stack_output_error(torch, coli, synth, wl, layers, x_step, stream, n_layers=2):
+    """Error of token 0 of a step through the first n_layers layers of the
+    stack against the fp64 oracle (max relative error)."""
+    import numpy as np
+    import oracle
+    E = wl.get("E", E_FULL)
+    xw = x_step[:1].clone()
+    coli.stack_forward(layers[:n_layers], xw, stream=stream)
+    torch.cuda.synchronize()
+    xr = x_step[:1].cpu().numpy().copy()
+    cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S)
+    for l in range(n_layers):
+        wr = synth.router(0, l, E, H)
+        bias = synth.zipf_bias(0, l, E)[0]
+        xn = oracle.rmsnorm(xr).astype(np.float32)
+        ids, _ = oracle.topk(oracle.router_logits(wr, bias, xn), K)
+        experts = [None] * (E + S)
+        for e in set(ids.ravel().tolist()) | set(range(E, E + S)):
+            experts[e] = synth.expert(0, l, e, H, I)
+        oracle.stack_step(cfg, wr, bias, experts, xr)
+    yg = xw.cpu().numpy().astype(np.float64)
+    ref = xr.astype(np.float64)
+    val = float(np.abs(yg - ref).max() / np.abs(ref).max())
+    return {"value": val, "kind": "max |x - x_oracle| / max |x_oracle| (fp32 residual stream)",
+            "sample": f"token 0 of the first timed step through the first {n_layers} layers vs the fp64 oracle"}
 
 
 def run_stack(args, wl, ws, rank, local):
@@ -528,13 +671,14 @@ def run_stack(args, wl, ws, rank, local):
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks = Clocks(local)
+    clocks = Clocks(local, coli, torch, stream)
     n0 = sum(L.launch_count() for L in layers)
     for i in range(args.warmup, nsteps):
         xw.copy_(xs[i])
         ev[i][0].record(stream)
         coli.stack_forward(layers, xw, stream=stream)
         ev[i][1].record(stream)
+    clocks.end_region()
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
     launches = sum(L.launch_count() for L in layers) - n0
@@ -561,23 +705,10 @@ def run_stack(args, wl, ws, rank, local):
     total_ms = max_over_ranks(total_ms, dist, dev)
 
     # end to end through the C ABI with host buffers (pinned x in, result out)
-    xh = xs[args.warmup:].cpu().pin_memory()
-    yh = torch.empty((T, H), dtype=torch.float32).pin_memory()
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    for j in range(args.steps):
-        ev2[j][0].record(stream)
-        xw.copy_(xh[j], non_blocking=True)
-        coli.stack_forward(layers, xw, stream=stream)
-        yh.copy_(xw, non_blocking=True)
-        ev2[j][1].record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = sum(ev2[j][0].elapsed_time(ev2[j][1]) for j in range(args.steps))
-    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
-    if dist:
-        dist.barrier()
+    e2e_ms = e2e_pipelined(torch, dev, stream, xs[args.warmup:],
+                           lambda xin, _: coli.stack_forward(layers, xin, stream=stream), (T, H), torch.float32,
+                           args.steps, dist, inplace=True)
+    err = stack_output_error(torch, coli, synth, wl, layers, xs[args.warmup], stream) if rank == 0 else None
     for L in layers:
         L.close()
     if rank != 0:
@@ -604,11 +735,13 @@ def run_stack(args, wl, ws, rank, local):
         "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / 8000.0, 4),
         "hbm_frac_of_measured": round(gbs / peak_gbs, 4),
         "bytes_per_step": int(bytes_step), "unique_experts_per_layer": round(mean_unique, 2),
-        "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items()},
+        "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items() if v > 0},
         "roofline": roof,
         "gpu_launches": launches,
+        "gpu_launches_note": "forward kernels in the timed loop; two clock-stamp kernels bracket the loop",
+        "max_rel_err": err,
         "e2e": {"value": round(job_tokens_per_s(ws, args.steps, T, e2e_ms), 2), "unit": "tokens/s",
-                "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4},
+                "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4, "method": E2E_METHOD},
         "clocks": clk,
     }
     if dist:

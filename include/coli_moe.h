@@ -282,6 +282,16 @@ coli_status coli_moe_route_noalloc(const float* router_w, const float* router_bi
  */
 coli_status coli_moe_debug_fail_alloc(int nth);
 
+/*
+ * Measurement aid: enqueues one kernel of n_blocks blocks (one per SM is the
+ * intent; launch as many as the device has SMs) in which block b writes
+ * {SM id, SM clock counter, global timer in ns} as int64 at buffer[3 b ..].
+ * Two stamps around a timed region give each SM's mean clock rate there:
+ * (clock difference) / (timer difference) for blocks on the same SM.
+ * buffer: DEVICE memory of 3 * n_blocks int64; 1 <= n_blocks <= 65535.
+ */
+coli_status coli_clock_stamp(long long* buffer, int n_blocks, coli_stream stream);
+
 /* Bytes of one expert in the int4 gs64 container (nibbles + fp16 scales). */
 int64_t coli_moe_expert_bytes(int hidden, int inter);
 

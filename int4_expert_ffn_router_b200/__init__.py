@@ -24,7 +24,7 @@ EXPORTS = (
     "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
     "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused", "coli_moe_set_tensor_cores",
     "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc", "coli_moe_get_launch_count",
-    "coli_moe_debug_fail_alloc",
+    "coli_moe_debug_fail_alloc", "coli_clock_stamp",
 )
 NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 63, 1024
 N_STAGES = 7
@@ -73,6 +73,7 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_set_fused.argtypes = [vp, i32]
     L.coli_moe_set_tensor_cores.argtypes = [vp, i32]
     L.coli_moe_debug_fail_alloc.argtypes = [i32]
+    L.coli_clock_stamp.argtypes = [vp, i32, vp]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
     L.coli_last_error.argtypes = []
@@ -249,6 +250,25 @@ def stack_forward(layers, x, n_tokens: int | None = None, eps: float = 1e-6, str
 def debug_fail_alloc(nth: int) -> None:
     """Make the nth device allocation of the library from now on fail (0: off)."""
     _check(lib.coli_moe_debug_fail_alloc(nth), "coli_moe_debug_fail_alloc")
+
+
+def clock_stamp(buffer, n_blocks: int, stream=None) -> None:
+    """Per-SM {SM id, clock counter, global timer ns} into a device int64 buffer [n_blocks][3]."""
+    _check(lib.coli_clock_stamp(_ptr(buffer), n_blocks, _stream(stream)), "coli_clock_stamp")
+
+
+def sm_clock_mhz(stamp0, stamp1):
+    """Mean clock rate (MHz) of each SM between two stamps (host int64 arrays [n][3]),
+    over the SMs present in both; a list of floats."""
+    first = {int(r[0]): (int(r[1]), int(r[2])) for r in stamp0}
+    out = {}
+    for r in stamp1:
+        sm = int(r[0])
+        if sm in first and sm not in out:
+            dc, dt = int(r[1]) - first[sm][0], int(r[2]) - first[sm][1]
+            if dt > 0 and dc > 0:
+                out[sm] = dc / dt * 1e3
+    return list(out.values())
 
 
 def make_config(hidden, inter, n_experts, top_k, n_shared, max_tokens) -> Config:

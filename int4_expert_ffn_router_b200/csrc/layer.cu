@@ -132,15 +132,22 @@ struct coli_moe_layer {
     int64_t prof_folded = 0;           // forwards folded into the totals
     double prof_total[COLI_N_STAGES] = {};
     cudaEvent_t ev[kRing][COLI_N_STAGES + 1] = {};
+    unsigned prof_mask[kRing] = {};    // stages marked in each ring slot
 };
 
-// Adds the durations of ring slot `r` to the totals (waits for its last event).
+// Adds the durations of ring slot `r` to the totals (waits for its last
+// event). A stage runs from its mark to the next recorded mark; stages a
+// path does not run are not marked and add nothing.
 static cudaError_t prof_fold(coli_moe_layer* L, int r) {
     cudaError_t e = cudaEventSynchronize(L->ev[r][COLI_N_STAGES]);
     if (e != cudaSuccess) return e;
+    const unsigned mask = L->prof_mask[r] | (1u << COLI_N_STAGES);
     for (int i = 0; i < COLI_N_STAGES; ++i) {
+        if (!(mask & (1u << i))) continue;
+        int j = i + 1;
+        while (!(mask & (1u << j))) ++j;
         float ms = 0.0f;
-        e = cudaEventElapsedTime(&ms, L->ev[r][i], L->ev[r][i + 1]);
+        e = cudaEventElapsedTime(&ms, L->ev[r][i], L->ev[r][j]);
         if (e != cudaSuccess) return e;
         L->prof_total[i] += ms;
     }
@@ -151,7 +158,9 @@ static cudaError_t prof_fold(coli_moe_layer* L, int r) {
 // Records the boundary before stage `i` of the current forward
 // (i == COLI_N_STAGES: after the last stage).
 static void prof_mark(coli_moe_layer* L, int i, cudaStream_t s) {
-    if (L->profiling) cudaEventRecord(L->ev[L->prof_next][i], s);
+    if (!L->profiling) return;
+    cudaEventRecord(L->ev[L->prof_next][i], s);
+    if (i < COLI_N_STAGES) L->prof_mask[L->prof_next] |= 1u << i;
 }
 
 static coli_status check_cfg(const coli_moe_config* c) {
@@ -398,8 +407,9 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
     const Plan& p = L->plan;
     if (L->profiling && L->prof_issued - L->prof_folded >= coli_moe_layer::kRing)
         CUDA_TRY(prof_fold(L, L->prof_next), "profile");  // recycle the oldest slot
+    if (L->profiling) L->prof_mask[L->prof_next] = 0;
     if (L->fused && T <= kFusedMaxTok) {
-        for (int i = 0; i <= COLI_STAGE_FUSED; ++i) prof_mark(L, i, s);
+        prof_mark(L, COLI_STAGE_FUSED, s);
         CUDA_TRY(launch_decode_fused(L->weights, d, L->router_w, L->router_b, x, dt, T, y, residual, p, L->logits, L->h,
                                      L->o, L->ctl, L->n_sm, L->smem_optin, L->trace, L->trace_cap, L->ring_stages,
                                      L->ring_blocks, s),
@@ -437,7 +447,6 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
                  "down (tensor cores)");
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_prefill_out(L->o, residual, T, d.H, y, dt, s), "output");
-        prof_mark(L, COLI_STAGE_FUSED, s);
         // router, top-k, plan, prep, tile plan, two grouped GEMMs, output (the clear is a driver memset)
         L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 7;
     } else {
@@ -453,7 +462,6 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         CUDA_TRY(launch_down_core(L->weights, d, L->h, T, p, L->o, L->max_active, L->n_sm, s), "down");
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_combine(L->o, p, T, d.H, d.K, d.S, residual, y, dt, s), "combine");
-        prof_mark(L, COLI_STAGE_FUSED, s);
         L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 5;
     }
     prof_mark(L, COLI_N_STAGES, s);
