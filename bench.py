@@ -65,6 +65,7 @@ WORKLOADS = {
                         desc="30-layer stack of the full-size layer, decode batch 64, Zipf(1.1) per layer"),
 }
 X_SEED0 = 1000  # step s draws its activations with seed X_SEED0 + s
+FUSED_MODE = {"i8": 1, "separate": 0}
 
 
 DEFAULT_STEPS = {"decode_b1": 10000, "decode_b32": 2000, "prefill_2048": 100, "decode_b1_e16": 1000, "prefill_e64": 100,
@@ -94,14 +95,7 @@ def job_tokens_per_s(world_size, steps, tokens_per_step, total_ms):
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
 # one ncu capture, keyed by (kernel, workload). A value stands only while the
 # kernel's sources hash to the recorded digest; otherwise `traffic` is null.
-NCU_TRAFFIC = {
-    ("moe_decode_fused_kernel", "decode_b1"): dict(
-        bytes=191_460_000,
-        sources=("decode_fused.cu", "int4_mma.cuh", "common.cuh", "topk.cuh", "kernels.cuh"),
-        sha256_16="ccc55600172f2930",
-        note="ncu capture of the 16-expert decode case (185.56 MB per launch) + 5.90 MB for the "
-             "256-expert router"),
-}
+NCU_TRAFFIC = {}
 
 
 def ncu_traffic(kernel, workload):
@@ -170,7 +164,7 @@ def dominant_roofline(stages, n_launches, T, mean_unique, E, elt, tc, peaks):
         return dom, None
     ach = alg[dom] / avg_s / 1e9
     peak = peaks.get("hbm_gbs", 6650.0)
-    names = {"fused": "moe_decode_fused_kernel", "gateup": "gateup_core_kernel", "down": "down_core_kernel",
+    names = {"fused": "moe_decode_i8_kernel", "gateup": "gateup_core_kernel", "down": "down_core_kernel",
              "router": "router kernels"}
     return dom, {"bound": "hbm", "kernel": names[dom], "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                  "frac": round(ach / peak, 4), "traffic": None,
@@ -187,6 +181,9 @@ def parse():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b1")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-kernel", choices=["i8", "separate"], default="i8",
+                    help="batches of up to 64 tokens: the persistent integer-MMA kernel (default) or the separate "
+                         "kernels")
     a = ap.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.workload]
@@ -399,6 +396,29 @@ E2E_METHOD = ("pipelined through the public API: pinned host x of step j copied 
               "forward; one event pair around all steps; L2 not flushed (each step reads its weights from HBM)")
 
 
+def small_batch_limit(kernel):
+    return {"i8": 64, "separate": 0}[kernel]
+
+
+def path_dtype(kernel, T, bf16, tc):
+    """Arithmetic of the path a batch of T tokens takes."""
+    if T <= small_batch_limit(kernel):
+        return "s8xu8->s32 + f32"
+    if tc:
+        return "f16->f32"
+    return "f32"
+
+
+def compute_desc(kernel, T, tc):
+    if T <= small_batch_limit(kernel):
+        return ("one persistent kernel; int4 codes x 8-bit token parts (15-bit block floating point per 64 "
+                "inputs) on mma.sync s32, exact per group, f32 scales and accumulation; fp64 router")
+    if tc:
+        return ("int4 weights dequantised to f16 in tensor memory, tcgen05 f16 MMA, f32 accumulate; "
+                "bf16 tokens scaled by powers of two to f16 (exact)")
+    return "int4 weights dequantised to f32 on CUDA cores, fp64 router"
+
+
 def e2e_pipelined(torch, dev, stream, xdev_steps, forward, shape, dtype, steps, dist, inplace=False):
     """Device ms for `steps` end-to-end steps: H2D of the step's input from
     pinned host memory, forward(x, y), D2H of y into pinned host memory
@@ -492,6 +512,7 @@ def run_ours(args, wl, ws, rank, local):
 
     T = wl["T"]
     layer = build_layer(torch, coli, synth, wl, local, max_tokens=T)
+    layer.set_fused(FUSED_MODE[args.decode_kernel])
     nsteps = args.warmup + args.steps
     xdt = torch.bfloat16 if wl["bf16"] else torch.float32
     xs = torch.empty((nsteps, T, H), dtype=xdt, device=dev)
@@ -561,7 +582,7 @@ def run_ours(args, wl, ws, rank, local):
     gbs = sum(bytes_step) / (sum(step_ms) * 1e-3) / 1e9
     peaks = load_peaks()
     peak_gbs = peaks.get("hbm_gbs", 6650.0)
-    tc = wl["bf16"] and T > 4  # bf16 batches of more than 4 tokens run on the tensor cores
+    tc = wl["bf16"] and T > small_batch_limit(args.decode_kernel)  # larger bf16 batches: tcgen05 grouped GEMMs
     dom, roof = dominant_roofline(stages, nprof, T, mean_unique, wl.get("E", E_FULL), xs.element_size(), tc, peaks)
     if roof is not None:
         roof["traffic"], roof["traffic_note"] = ncu_traffic(roof["kernel"], args.workload)
@@ -570,7 +591,7 @@ def run_ours(args, wl, ws, rank, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
         "step_ms_rank0": step_percentiles(step_ms),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if wl["bf16"] else "f32",
+        "dtype": path_dtype(args.decode_kernel, T, wl["bf16"], tc),
         "stage_note": "stage_us from a separate profiled pass (stage events add host gaps)",
         "data": "synthetic (seeded generator; random-init int4 weights of the full-size layer shape)",
         "config": {"workload": args.workload, "desc": wl["desc"], "hidden": H, "inter": I, "experts": wl.get("E", E_FULL),
@@ -586,10 +607,7 @@ def run_ours(args, wl, ws, rank, local):
         "gpu_launches": launches,
         "gpu_launches_note": "forward kernels in the timed loop; two clock-stamp kernels bracket the loop",
         "max_rel_err": err,
-        "compute": ("int4 weights dequantised to f16 in tensor memory, tcgen05 f16 MMA, f32 accumulate; "
-                    "bf16 tokens scaled by powers of two to f16 (exact)") if tc else
-                   ("int4 weights as raw f16 codes in mma.sync, f32 accumulate, fp64 router" if T <= 4 else
-                    "int4 weights dequantised to f32 on CUDA cores, fp64 router"),
+        "compute": compute_desc(args.decode_kernel, T, tc),
         "e2e": {"value": round(job_tokens_per_s(ws, args.steps, T, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * xs.element_size(), "d2h_bytes_per_step": T * H * xs.element_size(),
                 "method": E2E_METHOD},
@@ -644,6 +662,8 @@ def run_stack(args, wl, ws, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
     T, NL = wl["T"], wl["layers"]
     layers = [build_layer(torch, coli, synth, wl, local, max_tokens=T, layer_idx=l) for l in range(NL)]
+    for L in layers:
+        L.set_fused(FUSED_MODE[args.decode_kernel])
     nsteps = args.warmup + args.steps
     xs = torch.empty((nsteps, T, H), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -725,7 +745,7 @@ def run_stack(args, wl, ws, rank, local):
         "metric": METRIC, "value": round(job_tokens_per_s(ws, args.steps, T, total_ms), 2), "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
         "step_ms_rank0": step_percentiles(step_ms),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": path_dtype(args.decode_kernel, T, False, False),
         "data": "synthetic (seeded generator; random-init int4 weights of the full-size layer shape, per layer)",
         "config": {"workload": args.workload, "desc": wl["desc"], "layers": NL, "hidden": H, "inter": I,
                    "experts": E_FULL, "top_k": K, "shared": S, "tokens_per_step": T,

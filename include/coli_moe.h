@@ -112,17 +112,26 @@ coli_status coli_moe_route(coli_moe_layer* layer, const void* x, coli_dtype dtyp
 
 /*
  * The layer: y [n_tokens][H] = MoE(x), y of the same dtype as x. x and y must
- * not overlap. Paths: n_tokens <= 4 runs the persistent decode kernel (see
- * coli_moe_set_fused). Above that, bf16 runs the tcgen05 tensor-core grouped
- * GEMMs (fp16 operands: tokens scaled by powers of two and converted
- * exactly, weights rounded once to fp16, fp32 accumulation; the combine adds
- * with fp32 atomics, so the summation order, and the last bits of y, may vary
- * between runs) and fp32 the CUDA-core kernels (fp32 arithmetic); see
- * coli_moe_set_tensor_cores. The tensor-core path needs an sm_100 device,
- * hidden % 256 == 0, inter % 128 == 0 and weight scales of magnitude <= 4096;
- * otherwise bf16 also runs the CUDA-core kernels. Sparse-expert forward as the
- * Colibrì pages describe it (top-8 of 256 routed experts plus the always-on
- * shared expert, each distinct expert's int4 weights read once per batch).
+ * not overlap. Paths (see coli_moe_set_fused and coli_moe_set_tensor_cores):
+ *  - up to 64 tokens (and at most 512 routed slots, n_tokens * top_k): one
+ *    persistent kernel runs the whole layer on integer tensor-core MMAs. Each
+ *    64-input group of a token (or of a SwiGLU output row) is encoded as a
+ *    15-bit signed integer times a power of two chosen from the group's
+ *    largest magnitude (relative step 2^-15 of that magnitude), split into two
+ *    signed 8-bit parts; the int4 weights enter as their codes, each group's
+ *    sum is exact in 32-bit integers, and the group scales, the SwiGLU and the
+ *    combine are fp32. The output is deterministic.
+ *  - larger bf16 batches: the tcgen05 tensor-core grouped GEMMs (fp16
+ *    operands: tokens scaled by powers of two and converted exactly, weights
+ *    rounded once to fp16, fp32 accumulation; the combine adds with fp32
+ *    atomics, so the summation order, and the last bits of y, may vary
+ *    between runs). The tensor-core path needs an sm_100 device,
+ *    hidden % 256 == 0, inter % 128 == 0 and weight scales of magnitude
+ *    <= 4096; otherwise bf16 also runs the CUDA-core kernels.
+ *  - larger fp32 batches: the CUDA-core kernels (fp32 arithmetic).
+ * Sparse-expert forward as the Colibrì pages describe it (top-8 of 256 routed
+ * experts plus the always-on shared expert, each distinct expert's int4
+ * weights read once per batch).
  */
 coli_status coli_moe_forward(coli_moe_layer* layer, const void* x, void* y, coli_dtype dtype, int n_tokens,
                              coli_stream stream);
@@ -192,9 +201,11 @@ const char* coli_moe_stage_name(int stage);
 coli_status coli_moe_sync(coli_moe_layer* layer);
 
 /*
- * Selects the path for n_tokens <= 4: 1 (default) runs the whole layer in one
- * persistent kernel (router, top-k, plan, experts, combine), 0 runs the
- * separate kernels. Results agree within rounding; routing is identical.
+ * Selects the path for small batches: 1 (default) runs the whole layer for up
+ * to 64 tokens in one persistent kernel on integer MMAs (router, top-k, plan,
+ * experts, combine); 0 runs the separate kernels. Routing is identical;
+ * outputs agree within rounding. Returns COLI_EUNSUPPORTED when the shapes do
+ * not fit the kernel's shared memory, COLI_EINVAL for another value.
  */
 coli_status coli_moe_set_fused(coli_moe_layer* layer, int enable);
 
@@ -213,17 +224,17 @@ coli_status coli_moe_set_tensor_cores(coli_moe_layer* layer, int mode);
  * Item timeline of the persistent decode kernel, for profiling. `buffer` is a
  * caller-owned DEVICE buffer of 8 * (16 + 8 * capacity) bytes, zeroed by the
  * caller; int64 [0] counts records (it may exceed capacity: later records are
- * dropped); [1..5] global-timer stamps of the plan path: the last router
- * completion seen, its atomic done, plan published, top-k started, top-k
- * done, [6..8] plan steps (scan, entries stored, before the flag release),
- * [9] the earliest CTA start (atomic minimum: the caller sets it to
- * INT64_MAX for this stamp), [10] the last CTA's exit, [11] the latest end
- * of an output block's combine.
- * Record r at int64 16 + 8r: {cta << 40 | kind << 32 |
- * expert << 16 | tile, begin ns, end ns, ns waited for the item's first weight
- * stage, ns the item was published by the CTA's producer, total ns warp 0
- * waited for weight stages, 0, 0}; kind 1 router rows, 2 gate/up tile,
- * 3 down tile; times from the GPU global timer. NULL disables tracing.
+ * dropped); [1..8] global-timer stamps of the plan path: [1] the last router
+ * item seen done, [2] after its counter update, [3] plan published, [4] top-k
+ * started, [5] top-k done, [6] counts and scans done, [7] positions written,
+ * [8] before the release of the plan flag; [9] the earliest CTA start (atomic
+ * minimum: the caller sets it to INT64_MAX), [10] the last CTA's exit, [11]
+ * the latest end of an output block's combine.
+ * Record r at int64 16 + 8r: {cta << 40 | kind << 32 | expert << 16 | tile,
+ * begin ns, end ns, ns waited for the item's first weight stage, tokens of the
+ * item, total ns consumer 0 waited for weight stages, chunk id, 0}; kind 1
+ * router rows, 2 gate/up tile, 3 down tile, 4 token quantisation; times from
+ * the GPU global timer. NULL disables tracing.
  * In a library built with COLI_TC_TRACE=1 (a profiling build; the default
  * build records nothing there), the tensor-core path writes, with
  * c = (capacity - 256) / 16 when positive,
@@ -272,6 +283,16 @@ coli_status coli_moe_set_ring(coli_moe_layer* layer, int stages, int blocks_per_
 coli_status coli_moe_route_noalloc(const float* router_w, const float* router_bias, int n_experts, int hidden,
                                    int top_k, const void* x, coli_dtype dtype, int n_tokens, int32_t* ids,
                                    float* weights, coli_stream stream);
+
+/*
+ * Testing aid for the bounded waits of the integer-MMA persistent kernel:
+ * every wait of its launches on this layer gives up after wait_ns
+ * nanoseconds (0: the default, 1 s), and with enable != 0 one gate/up item of
+ * each launch waits on a flag that nothing sets, so the launch gives up: its
+ * CTAs drain their copies and exit, and coli_moe_sync then returns COLI_ECUDA
+ * and resets the layer, which stays usable. No GPU fault or hang is involved.
+ */
+coli_status coli_moe_debug_wait_test(coli_moe_layer* layer, int enable, int64_t wait_ns);
 
 /*
  * Testing aid for the out-of-memory paths: from now on, the nth device

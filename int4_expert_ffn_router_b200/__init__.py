@@ -24,7 +24,7 @@ EXPORTS = (
     "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
     "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused", "coli_moe_set_tensor_cores",
     "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc", "coli_moe_get_launch_count",
-    "coli_moe_debug_fail_alloc", "coli_clock_stamp",
+    "coli_moe_debug_fail_alloc", "coli_clock_stamp", "coli_moe_debug_wait_test",
 )
 NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 63, 1024
 N_STAGES = 7
@@ -74,6 +74,7 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_set_tensor_cores.argtypes = [vp, i32]
     L.coli_moe_debug_fail_alloc.argtypes = [i32]
     L.coli_clock_stamp.argtypes = [vp, i32, vp]
+    L.coli_moe_debug_wait_test.argtypes = [vp, i32, ctypes.c_int64]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
     L.coli_last_error.argtypes = []
@@ -186,8 +187,14 @@ class Layer:
         """Wait for the last forward; raises if the device reported a timeout."""
         _check(lib.coli_moe_sync(self.handle), "coli_moe_sync")
 
-    def set_fused(self, on: bool) -> None:
+    def set_fused(self, on) -> None:
+        """True: the persistent kernel for batches of up to 64 tokens (default); False: separate kernels."""
         _check(lib.coli_moe_set_fused(self.handle, 1 if on else 0), "coli_moe_set_fused")
+
+    def debug_wait_test(self, enable: bool, wait_ns: int = 0) -> None:
+        """Testing aid: bound the persistent kernel's waits to wait_ns and, when
+        enabled, make each launch give up on a flag that nothing sets."""
+        _check(lib.coli_moe_debug_wait_test(self.handle, 1 if enable else 0, wait_ns), "coli_moe_debug_wait_test")
 
     def set_tensor_cores(self, mode) -> None:
         """0 / False: CUDA-core kernels; 1 / True: tensor cores for bf16 (default);

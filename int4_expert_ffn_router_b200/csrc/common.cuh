@@ -65,30 +65,14 @@ constexpr int kNibbleBytes = 4096;
 constexpr int kScaleBytes = 256;
 constexpr int kBlockBytes = kNibbleBytes + kScaleBytes;  // 4352
 
-// Persistent decode kernel: tokens per launch, ring stages, control block.
-constexpr int kFusedMaxTok = 4;
 // CUDA-core expert kernels: tokens per pass over a weight tile (one work item).
 constexpr int kCoreTok = 4;
 // Tensor-core path: tokens of one expert per GEMM tile (the MMA N).
 constexpr int kTcMaxTok = 128;
 constexpr int kMaxStages = 24;
-// Control block (ints in the workspace, zero between launches):
-//   [kCtlTicket] work ticket, [kCtlRouter] finished router items,
-//   [kCtlPlan] 0, or 1 + number of distinct routed experts once the plan is
-//   published, [kCtlExit] CTAs done, [kCtlError] timeout code,
-//   [kCtlGuDone + e] finished gate/up tiles of expert e (E + S entries),
-//   [kCtlGuDone + E + S + rt] finished down tiles of output block rt (H/128),
-//   then kFusedMaxTok * (K + S) float bit patterns: max |h| of each position,
-//   then 2 * kFusedMaxTok * K ints: one 64-bit plan entry per distinct routed
-//   expert u (bit 63 valid; expert, first position, tokens, token ids).
-enum { kCtlTicket = 0, kCtlRouter = 1, kCtlPlan = 2, kCtlExit = 3, kCtlError = 4, kCtlGuDone = 8 };
-__host__ __device__ inline int ctl_hmax_at(int E, int S, int H) { return kCtlGuDone + E + S + H / 128; }
-__host__ __device__ inline int ctl_entries_at(int E, int S, int H, int K) {
-    return (ctl_hmax_at(E, S, H) + kFusedMaxTok * (K + S) + 1) & ~1;  // 8-byte aligned
-}
-__host__ __device__ inline int ctl_ints(int E, int S, int H, int K) {
-    return ctl_entries_at(E, S, H, K) + 2 * kFusedMaxTok * K;
-}
+// Word of the layer's control block where a persistent kernel that gave up
+// on a bounded wait records its site code (0: none).
+constexpr int kCtlError = 4;
 
 inline int64_t matrix_bytes(int rows, int cols) {
     return (int64_t)(rows / kTileRows) * (cols / kGroup) * kBlockBytes;
@@ -116,8 +100,6 @@ struct Plan {
     int32_t* act_cnt;    // [E+S] tokens of active expert a
     int32_t* n_active;   // [1] n_unique + S
     int32_t* act_chunk;  // [E+S+1] prefix of ceil(act_cnt / kCoreTok) over the active experts
-    int4* table;         // [E] per distinct expert u (ascending): {expert, first position, tokens,
-                         //     tokens packed 8 bits each when <= 4} (persistent decode kernel)
 };
 
 // ---------------------------------------------------------------------------

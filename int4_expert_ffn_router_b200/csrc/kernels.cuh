@@ -36,16 +36,44 @@ cudaError_t launch_gateup_core(const uint8_t* weights, const Dims& d, const void
 cudaError_t launch_down_core(const uint8_t* weights, const Dims& d, const float* h, int T, const Plan& p, float* o,
                              int max_active, int n_sm, cudaStream_t st);
 
-// decode_fused.cu: the whole layer for 1..kFusedMaxTok tokens in one
-// persistent launch (n_sm CTAs). ctl: control block of ctl_ints() ints,
-// zero at launch (the kernel leaves it zero, except a timeout code).
-cudaError_t launch_decode_fused(const uint8_t* weights, const Dims& d, const float* wr, const float* bias,
-                                const void* x, coli_dtype dt, int T, void* y, const float* residual, const Plan& p,
-                                double* logits, float* h, float* o, int* ctl, int n_sm, size_t smem_limit,
-                                long long* trace, int trace_cap, int max_stages, int max_sb, cudaStream_t st);
-int fused_stages_for(const Dims& d, int NT, size_t smem_limit);
-constexpr int kDefaultStages = 3;  // ring stages in flight per SM (see fused_geometry)
+// Persistent decode kernel ring defaults: bulk copies in flight per SM and
+// 4352-byte blocks per copy (coli_moe_set_ring).
+constexpr int kDefaultStages = 3;
 constexpr int kDefaultStageBlocks = 8;
+
+// decode_i8.cu: the whole layer for 1..kI8MaxTok tokens (at most kI8MaxSlots
+// routed slots) in one persistent launch of n_sm CTAs, on integer MMAs.
+constexpr int kI8MaxTok = 64;
+constexpr int kI8MaxSlots = 512;
+struct I8Launch {
+    const uint8_t* weights;
+    Dims d;
+    const float* wr;
+    const float* bias;
+    const void* x;
+    coli_dtype dt;
+    int T;
+    void* y;
+    const float* residual;
+    Plan p;
+    double* logits;
+    uint8_t* xq;   // [T][H/64][128] token parts (written by the kernel)
+    uint8_t* xm;   // [T][H/64][16]
+    uint8_t* hq;   // [slots][I/64][128] SwiGLU output parts
+    uint8_t* hm;   // [slots][I/64][16]
+    float* o;      // [slots][H]
+    int* ctl;      // control block of i8_ctl_ints_for(d, T) ints, zero at launch (left zero but a timeout code)
+    int n_sm;
+    size_t smem_limit;
+    long long* trace;
+    int trace_cap;
+    int max_stages, max_sb;
+    int64_t wait_ns;  // bound of every wait (<= 0: 1 s)
+    int wait_test;    // testing aid: one gate/up item waits on a flag that nothing sets
+};
+cudaError_t launch_decode_i8(const I8Launch& l, cudaStream_t st);
+bool decode_i8_supported(const Dims& d, int T, size_t smem_limit);
+int i8_ctl_ints_for(const Dims& d, int T);
 
 // prefill_tc.cu: the expert FFNs of a bf16 token batch on the tensor cores.
 // meta: [0] max over gate/up row pairs of L1(gate row) * L1(up row) (float

@@ -100,8 +100,17 @@ struct coli_moe_layer {
     float* h = nullptr;
     float* o = nullptr;
     float* xn = nullptr;
-    int* ctl = nullptr;             // control block of the persistent decode kernel
-    // tensor-core path (bf16 batches of more than kFusedMaxTok tokens)
+    int* ctl = nullptr;             // control block of the persistent decode kernels
+    int ctl_n = 0;                  // its ints
+    // integer-MMA persistent kernel (decode_i8.cu): token parts and SwiGLU output parts
+    uint8_t* xq = nullptr;
+    uint8_t* xm = nullptr;
+    uint8_t* hq = nullptr;
+    uint8_t* hm = nullptr;
+    int i8_max_tok = 0;             // largest batch its workspace holds
+    int64_t wait_ns = 0;            // bound of its waits (0: 1 s)
+    int wait_test = 0;              // testing aid (coli_moe_debug_wait_test)
+    // tensor-core path (bf16 batches too large for the persistent kernel)
     __half* xs = nullptr;           // [2 slots][H] scaled fp16 rows of x in position order (hi, lo for fp32 x)
     float4* tscale = nullptr;       // [max_tokens] per-token power-of-two scales
     float4* slot = nullptr;         // [slots] per-position epilogue factors
@@ -116,7 +125,7 @@ struct coli_moe_layer {
     alignas(64) unsigned char xs_maps[2 * kTensorMapBytes] = {};  // TMA maps of the token operands
     alignas(64) unsigned char h16_maps[2 * kTensorMapBytes] = {};  // (boxes of kTcMaxTok and 32 rows)
     size_t smem_optin = 0;
-    bool fused = true;              // use the persistent kernel for n_tokens <= kFusedMaxTok
+    int fused = 1;                  // coli_moe_set_fused: 1 persistent kernel for small batches, 0 separate kernels
     long long* trace = nullptr;     // caller-owned device buffer for the item timeline
     int trace_cap = 0;
     int ring_stages = kDefaultStages;        // persistent kernel: bulk copies in flight per SM
@@ -292,10 +301,17 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     const size_t TE = (size_t)Tm * d.E;
     const size_t rpart_cap = std::max<size_t>(TE, std::min<size_t>(64 * TE, (size_t)1 << 23));  // <= 64 MB unless TE is larger
     const size_t TK = (size_t)Tm * d.K, slots = TK + (size_t)d.S * Tm, EA = (size_t)d.E + d.S;
+    // the integer-MMA kernel's batches: up to kI8MaxTok tokens and kI8MaxSlots routed slots
+    const int Tf = (int)std::min<int64_t>(std::min<int64_t>(Tm, kI8MaxTok), kI8MaxSlots / d.K);
+    L->i8_max_tok = Tf;
+    const size_t slots_f = (size_t)Tf * d.K + (size_t)d.S * Tf;
+    L->ctl_n = std::max(kCtlError + 1, Tf > 0 ? i8_ctl_ints_for(d, Tf) : 0);
     size_t sz[] = {Tm * (size_t)d.E * 8, TK * 4, TK * 4, (size_t)d.E * 4, (size_t)(d.E + 1) * 4, (size_t)d.E * 4, 4,
                    TK * 4, slots * 4, EA * 4, EA * 4, EA * 4, 4, slots * d.I * 4, slots * d.H * 4, (size_t)Tm * d.H * 4,
-                   (size_t)ctl_ints(d.E, d.S, d.H, d.K) * 4, (size_t)d.E * 16, 2 * slots * d.H * 2, (size_t)Tm * 16,
-                   slots * 16, (size_t)prefill_tc_max_tiles(d, Tm) * 16, 4, 16, rpart_cap * 8, (EA + 1) * 4};
+                   (size_t)L->ctl_n * 4, 0, 2 * slots * d.H * 2, (size_t)Tm * 16,
+                   slots * 16, (size_t)prefill_tc_max_tiles(d, Tm) * 16, 4, 16, rpart_cap * 8, (EA + 1) * 4,
+                   (size_t)Tf * (d.H / 64) * 128, (size_t)Tf * (d.H / 64) * 16, slots_f * (d.I / 64) * 128,
+                   slots_f * (d.I / 64) * 16};
     constexpr int kRegions = sizeof(sz) / sizeof(sz[0]);
     size_t total = 0;
     for (size_t s : sz) total += align256(s);
@@ -305,7 +321,6 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     void* ptrs[kRegions];
     for (int i = 0; i < kRegions; ++i) { ptrs[i] = cur; cur += align256(sz[i]); }
     L->ctl = (int*)ptrs[16];
-    L->plan.table = (int4*)ptrs[17];
     L->xs = (__half*)ptrs[18];
     L->tscale = (float4*)ptrs[19];
     L->slot = (float4*)ptrs[20];
@@ -314,12 +329,16 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     L->meta = (unsigned*)ptrs[23];
     L->rpart = (double*)ptrs[24];
     L->plan.act_chunk = (int32_t*)ptrs[25];
+    L->xq = (uint8_t*)ptrs[26];
+    L->xm = (uint8_t*)ptrs[27];
+    L->hq = (uint8_t*)ptrs[28];
+    L->hm = (uint8_t*)ptrs[29];
     L->rpart_cap = rpart_cap;
     {
         int optin = 0;
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
         L->smem_optin = (size_t)optin;
-        L->fused = fused_stages_for(d, kFusedMaxTok, L->smem_optin) >= 2;
+        L->fused = (Tf > 0 && decode_i8_supported(d, 1, L->smem_optin)) ? 1 : 0;
         int cc_major = 0;
         cudaDeviceGetAttribute(&cc_major, cudaDevAttrComputeCapabilityMajor, device);
         L->tc_shape_ok = cc_major == 10 && d.H % 256 == 0 && d.I % 128 == 0 && L->smem_optin >= prefill_tc_smem_bytes();
@@ -408,12 +427,15 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
     if (L->profiling && L->prof_issued - L->prof_folded >= coli_moe_layer::kRing)
         CUDA_TRY(prof_fold(L, L->prof_next), "profile");  // recycle the oldest slot
     if (L->profiling) L->prof_mask[L->prof_next] = 0;
-    if (L->fused && T <= kFusedMaxTok) {
+    if (L->fused == 1 && T <= L->i8_max_tok && decode_i8_supported(d, T, L->smem_optin)) {
         prof_mark(L, COLI_STAGE_FUSED, s);
-        CUDA_TRY(launch_decode_fused(L->weights, d, L->router_w, L->router_b, x, dt, T, y, residual, p, L->logits, L->h,
-                                     L->o, L->ctl, L->n_sm, L->smem_optin, L->trace, L->trace_cap, L->ring_stages,
-                                     L->ring_blocks, s),
-                 "persistent decode kernel");
+        I8Launch l{};
+        l.weights = L->weights; l.d = d; l.wr = L->router_w; l.bias = L->router_b; l.x = x; l.dt = dt; l.T = T;
+        l.y = y; l.residual = residual; l.p = p; l.logits = L->logits; l.xq = L->xq; l.xm = L->xm; l.hq = L->hq;
+        l.hm = L->hm; l.o = L->o; l.ctl = L->ctl; l.n_sm = L->n_sm; l.smem_limit = L->smem_optin; l.trace = L->trace;
+        l.trace_cap = L->trace_cap; l.max_stages = L->ring_stages; l.max_sb = L->ring_blocks;
+        l.wait_ns = L->wait_ns; l.wait_test = L->wait_test;
+        CUDA_TRY(launch_decode_i8(l, s), "persistent decode kernel (integer MMA)");
         L->launches += 1;
     } else if ((L->tc_mode == 2 || (L->tc_mode == 1 && dt == COLI_BF16)) && L->tc_shape_ok && L->tc_scale_ok) {
         // tensor cores; fp32 tokens as fp16 hi + lo operand rows (tiles of kTcMaxTok / 2 tokens)
@@ -521,7 +543,7 @@ static coli_status sync_and_check(coli_moe_layer* L) {
     int err = 0;
     CUDA_TRY(cudaMemcpy(&err, L->ctl + kCtlError, 4, cudaMemcpyDeviceToHost), "read status");
     if (err != 0) {
-        CUDA_TRY(cudaMemset(L->ctl, 0, (size_t)ctl_ints(L->d.E, L->d.S, L->d.H, L->d.K) * 4), "reset control block");
+        CUDA_TRY(cudaMemset(L->ctl, 0, (size_t)L->ctl_n * 4), "reset control block");
         char msg[96];
         snprintf(msg, sizeof msg, "a bounded wait in a persistent kernel timed out (site %d)", err);
         g_last_error = msg;
@@ -539,9 +561,18 @@ COLI_API coli_status coli_moe_sync(coli_moe_layer* L) {
 
 COLI_API coli_status coli_moe_set_fused(coli_moe_layer* L, int enable) {
     if (!L) return fail(COLI_EINVAL, "layer is NULL");
-    if (enable && fused_stages_for(L->d, kFusedMaxTok, L->smem_optin) < 2)
+    if (enable < 0 || enable > 1) return fail(COLI_EINVAL, "enable must be 0 or 1");
+    if (enable && !(L->i8_max_tok > 0 && decode_i8_supported(L->d, 1, L->smem_optin)))
         return fail(COLI_EUNSUPPORTED, "shapes too large for the persistent kernel's shared memory");
-    L->fused = enable != 0;
+    L->fused = enable;
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_debug_wait_test(coli_moe_layer* L, int enable, int64_t wait_ns) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (wait_ns < 0) return fail(COLI_EINVAL, "wait_ns must be >= 0");
+    L->wait_test = enable != 0;
+    L->wait_ns = wait_ns;
     return COLI_OK;
 }
 

@@ -36,7 +36,6 @@
 #include <cstring>
 
 #include "common.cuh"
-#include "int4_mma.cuh"
 #include "kernels.cuh"
 #include "tcgen05.cuh"
 

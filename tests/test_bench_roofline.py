@@ -42,9 +42,9 @@ def _digest(files):
 
 
 def test_recorded_traffic_needs_unchanged_sources(monkeypatch):
-    key = ("moe_decode_fused_kernel", "decode_b1")
-    assert bench.ncu_traffic("moe_decode_fused_kernel", "decode_b32") == (None, None)
-    rec = dict(bytes=190_000_000, sources=("decode_fused.cu", "common.cuh"), note="test record")
+    key = ("moe_decode_i8_kernel", "decode_b1")
+    assert bench.ncu_traffic("moe_decode_i8_kernel", "decode_b32") == (None, None)
+    rec = dict(bytes=190_000_000, sources=("decode_i8.cu", "common.cuh"), note="test record")
     monkeypatch.setitem(bench.NCU_TRAFFIC, key, dict(rec, sha256_16=_digest(rec["sources"])))
     assert bench.ncu_traffic(*key) == (190_000_000, "test record")  # sources as captured
     monkeypatch.setitem(bench.NCU_TRAFFIC, key, dict(rec, sha256_16="0" * 16))

@@ -65,3 +65,40 @@ def test_create_out_of_memory_at_each_allocation(gpu):
     y = yd.cpu().numpy().astype(np.float64)
     assert np.abs(y - y_ref).max() <= 1e-3 * np.abs(y_ref).max()
     layer.close()
+
+
+def test_bounded_wait_expiry_returns_an_error_and_the_layer_recovers(gpu):
+    """A testing aid makes one gate/up item of the persistent kernel wait on a
+    flag that nothing sets, with every wait bounded to 2 ms. The launch gives
+    up by itself (its CTAs drain their copies and exit): coli_moe_sync reports
+    COLI_ECUDA promptly, and the next forward on the same layer matches the
+    oracle. Nothing faults or hangs."""
+    import time
+
+    import int4_expert_ffn_router_b200 as coli
+
+    c = cases.TINY
+    L, args = _host_args(coli, c)
+    layer = coli.Layer(*args, device=0)
+    x = synth.x_f32(c["seed"], 4, 3, c["H"])
+    xd = torch.from_numpy(x).to(gpu)
+    yd = torch.empty_like(xd)
+    layer.forward(xd, yd)  # warm: module loaded, control block in use once
+    layer.sync()
+    layer.debug_wait_test(True, 2_000_000)
+    t0 = time.time()
+    layer.forward(xd, yd)
+    with pytest.raises(coli.ColiError) as e:
+        layer.sync()
+    elapsed = time.time() - t0
+    assert e.value.status == coli.COLI_ECUDA and "timed out" in str(e.value)
+    assert elapsed < 2.0, f"the launch took {elapsed:.2f} s to give up"
+    layer.debug_wait_test(False, 0)
+    for _ in range(2):
+        yd.fill_(float("nan"))
+        layer.forward(xd, yd)
+        layer.sync()
+        y_ref, _, _ = oracle.moe_forward(cases.oracle_cfg(c), L["wr"], None, L["experts"], x)
+        y = yd.cpu().numpy().astype(np.float64)
+        assert np.abs(y - y_ref).max() <= 1e-3 * np.abs(y_ref).max()
+    layer.close()

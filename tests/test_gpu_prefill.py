@@ -1,5 +1,7 @@
-"""GPU parity of the tensor-core path (bf16 batches of more than 4 tokens)
-against the fp64 oracle, through the C ABI.
+"""GPU parity of the tensor-core path (the tcgen05 grouped GEMMs of bf16
+batches) against the fp64 oracle, through the C ABI. The tiny layer here has
+the persistent small-batch kernel switched off, so every batch size, down to
+5 tokens, runs the batch kernels.
 
 Routing and the batch-union plan bit for bit; outputs within the bf16-path
 tolerance ||y - y_ref||_2 <= 5e-3 ||y_ref||_2. Cases span ragged token tiles
@@ -45,6 +47,7 @@ def tiny_big(coli):
     L = cases.host_layer(c, seed=c["seed"])
     layer = _host_layer_to_device(coli, c, L, max_tokens=1024)
     layer.set_tensor_cores(True)  # the shapes qualify: raises otherwise
+    layer.set_fused(False)        # small batches too take the batch kernels
     yield c, L, layer
     layer.close()
 
@@ -184,9 +187,9 @@ def test_full_prefill_2048_hot_expert_tokens(gpu, coli):
 
 @pytest.mark.parametrize("T", [5, 40, 200])
 def test_tiny_fp32_tensor_cores_and_cuda_cores(gpu, tiny_big, T):
-    """fp32 batches of more than 4 tokens run the CUDA-core kernels by default;
-    mode 2 runs them on the tensor cores with hi + lo operand rows (tiles of up
-    to 64 tokens). Both meet the fp32-path tolerance on one layer."""
+    """fp32 batches on the batch kernels run on the CUDA cores by default; mode
+    2 runs them on the tensor cores with hi + lo operand rows (tiles of up to
+    64 tokens). Both meet the fp32-path tolerance on one layer."""
     c, L, layer = tiny_big
     x = synth.x_f32(c["seed"], 600 + T, T, c["H"])
     xd = torch.from_numpy(x).to(gpu)
