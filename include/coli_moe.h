@@ -232,7 +232,8 @@ coli_status coli_moe_set_tensor_cores(coli_moe_layer* layer, int mode);
  * the latest end of an output block's combine.
  * Record r at int64 16 + 8r: {cta << 40 | kind << 32 | expert << 16 | tile,
  * begin ns, end ns, ns waited for the item's first weight stage, tokens of the
- * item, total ns consumer 0 waited for weight stages, chunk id, 0}; kind 1
+ * item, total ns consumer 0 waited for weight stages, weight loop start ns,
+ * weight loop end ns (0 for items without weights)}; kind 1
  * router rows, 2 gate/up tile, 3 down tile, 4 token quantisation; times from
  * the GPU global timer. NULL disables tracing.
  * In a library built with COLI_TC_TRACE=1 (a profiling build; the default

@@ -34,7 +34,8 @@
 namespace coli {
 namespace {
 
-constexpr int kCW = 8;                       // consumer warps (one 16-row sub-tile each)
+constexpr int kSub = 8;                      // 16-row sub-tiles of a 128-row weight tile
+constexpr int kCW = 16;                      // consumer warps: two per sub-tile, on alternate blocks
 constexpr int kCT = kCW * 32;                // consumer threads
 constexpr int kProducerWarp = kCW;
 constexpr int kSignalWarp = kCW + 1;
@@ -42,8 +43,12 @@ constexpr int kFT = (kCW + 2) * 32;          // all threads
 constexpr int kMaxSB = 8;                    // 4352-byte blocks per ring stage (at most)
 constexpr int kQ = 2;                        // item queue slots (lookahead of one item)
 constexpr int kSQ = 4;                       // completion records in flight to the signaler
-constexpr int kRouterExperts = 2;            // experts per router item (4 warps each)
+constexpr int kRouterExperts = kCW / 8;      // experts per router item (8 warps each, one pass over H/8)
 constexpr int kChunkTok = 4;                 // tokens per 8-column MMA chunk (hi and lo parts)
+constexpr int kMetaRow = 16;                 // bytes of one group's data {2^-e, -8 sum(hi), -8 sum(lo), 0}
+// In shared memory each token slot's group data is followed by one unused
+// 16-byte entry, so the four tokens of an MMA chunk fall in different banks.
+__host__ __device__ constexpr size_t meta_slot_bytes(int G) { return (size_t)(G + 1) * kMetaRow; }
 
 enum { IT_END = 0, IT_PREP = 1, IT_ROUTER = 2, IT_GU = 3, IT_DOWN = 4 };
 
@@ -109,9 +114,11 @@ struct I8Smem {
     int staged_n, staged_key;
     int staged_tok[8];
     int wsum[kCW], wflag[kCW];
-    float hmaxw[kCW][8];    // gate/up epilogue: per warp, max |h| of each token of the item
-    int hsum[kCW][8][2];    // per warp, sums of the hi and lo parts of each token
+    float hmaxw[kSub][8];   // gate/up epilogue: per sub-tile, max |h| of each token of the item
+    int hsum[kSub][8][2];   // per sub-tile, sums of the hi and lo parts of each token
+    alignas(16) float accx[kSub][32][4];  // partial sums of the second warp of each sub-tile (read as float4)
     unsigned long long first_wait_ns, total_wait_ns;
+    unsigned long long t_loop0, t_loop1;  // trace: the item's weight loop started / ended
 };
 
 // ------------------------------------------------------------- small helpers
@@ -193,6 +200,28 @@ __device__ __forceinline__ int limb_offset(int k) {
     return t * 16 + 4 * s + b;
 }
 
+// 2^k as a float, k in [-126, 127] (exponent bits written directly).
+__device__ __forceinline__ float pow2f(int k) { return __uint_as_float((uint32_t)(127 + k) << 23); }
+
+// Exponent e of the block-floating-point encoding of a group whose largest
+// magnitude is m: m 2^e in [2^14, 32639], so that rint(v 2^e) = 256 hi + lo
+// with hi, lo in [-128, 127]. 0 for m = 0 (and for non-finite m).
+__device__ __forceinline__ int group_exponent(float m) {
+    const uint32_t b = __float_as_uint(m);
+    const int be = (int)((b >> 23) & 0xFF);
+    if (m <= 0.0f || be == 0xFF) return 0;
+    int e;
+    if (be == 0) {  // subnormal: m < 2^-126, the largest shift keeps every product finite
+        e = 126;
+    } else {
+        e = 14 - (be - 127);  // m 2^e in [2^14, 2^15)
+        e = e > 126 ? 126 : (e < -126 ? -126 : e);
+        // m 2^e = 2^14 (1 + f): above 32639 when the 23-bit fraction exceeds 0x7EFE00
+        if (e == 14 - (be - 127) && (b & 0x7FFFFFu) > 0x7EFE00u) e -= 1;
+    }
+    return e;
+}
+
 // Block-floating-point encoding of one 64-input group of one token (or
 // position), one warp, lane l holding inputs 2l and 2l+1 (v0, v1): scale 2^e
 // with max |v| 2^e in [2^14, 32639], integer x = rint(v 2^e) split as
@@ -202,15 +231,8 @@ __device__ __forceinline__ void encode_group(float v0, float v1, uint8_t* dst, u
     float m = fmaxf(fabsf(v0), fabsf(v1));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    int e = 0;
-    if (m > 0.0f && m <= 3.0e38f) {
-        int ex;
-        frexpf(m, &ex);                 // m = f 2^ex, f in [0.5, 1)
-        e = 15 - ex;                    // m 2^e in [2^14, 2^15)
-        e = e > 126 ? 126 : (e < -126 ? -126 : e);
-        if (ldexpf(m, e) > 32639.0f) e -= 1;
-    }
-    const float f = ldexpf(1.0f, e);
+    const int e = group_exponent(m);
+    const float f = pow2f(e);
     int hi[2], lo[2];
     const float v[2] = {v0, v1};
 #pragma unroll
@@ -228,7 +250,7 @@ __device__ __forceinline__ void encode_group(float v0, float v1, uint8_t* dst, u
         sh += __shfl_xor_sync(0xffffffffu, sh, o);
         sl += __shfl_xor_sync(0xffffffffu, sl, o);
     }
-    if (lane == 0) *reinterpret_cast<int4*>(meta) = make_int4(__float_as_int(ldexpf(1.0f, -e)), -8 * sh, -8 * sl, 0);
+    if (lane == 0) *reinterpret_cast<int4*>(meta) = make_int4(__float_as_int(pow2f(-e)), -8 * sh, -8 * sl, 0);
 }
 
 // u8 x s8 -> s32 MMA, 16 x 8 x 32, accumulating in place.
@@ -296,16 +318,18 @@ __device__ void i8_producer(I8Args& a, I8Smem& S, uint8_t* ring) {
                 int dd = t - f.t_dyn;
                 if (nc < 0) {
                     it.kind = IT_END;  // aborted
-                } else if (dd < nc * f.RTgu) {
-                    const unsigned long long v = __ldcg(entries + dd / f.RTgu);
-                    it = Item{IT_GU, (int)(v & 0xFFFF), dd % f.RTgu, f.SC + dd / f.RTgu, (int)((v >> 16) & 0xFFFFF),
+                } else if (dd < nc * f.RTgu || (dd >= nc * f.RTgu + f.SC * f.RTd &&
+                                                dd < nc * (f.RTgu + f.RTd) + f.SC * f.RTd)) {
+                    const bool gu = dd < nc * f.RTgu;
+                    const int RT = gu ? f.RTgu : f.RTd;
+                    const int r = gu ? dd : dd - nc * f.RTgu - f.SC * f.RTd;
+                    const int c = r / RT;
+                    const unsigned long long v = __ldcg(entries + c);
+                    it = Item{gu ? IT_GU : IT_DOWN, (int)(v & 0xFFFF), r % RT, f.SC + c, (int)((v >> 16) & 0xFFFFF),
                               (int)((v >> 36) & 0xF), -1, 0};
-                } else if ((dd -= nc * f.RTgu) < f.SC * f.RTd) {
+                } else if (dd >= nc * f.RTgu && dd < nc * f.RTgu + f.SC * f.RTd) {
+                    dd -= nc * f.RTgu;
                     it = shared_chunk(a, IT_DOWN, dd / f.RTd, dd % f.RTd);
-                } else if ((dd -= f.SC * f.RTd) < nc * f.RTd) {
-                    const unsigned long long v = __ldcg(entries + dd / f.RTd);
-                    it = Item{IT_DOWN, (int)(v & 0xFFFF), dd % f.RTd, f.SC + dd / f.RTd, (int)((v >> 16) & 0xFFFFF),
-                              (int)((v >> 36) & 0xF), -1, 0};
                 }
             }
             if (it.kind == IT_DOWN) it.ready = ld_acquire(&a.ctl[i8_ctl_gu(f.nch) + it.chunk]) >= f.RTgu;
@@ -454,15 +478,26 @@ template <typename XT>
 __device__ void prep_item(I8Args& a, int t, int ctid) {
     const int cw = ctid >> 5, lane = ctid & 31, G = a.d.H / kGroup;
     const XT* xr = reinterpret_cast<const XT*>(a.x) + (size_t)t * a.d.H;
-    for (int g = cw; g < G; g += kCW) {
-        const float2 v = load2<XT>(xr + g * kGroup + 2 * lane);
-        encode_group(v.x, v.y, a.xq + ((size_t)t * G + g) * 128, a.xm + ((size_t)t * G + g) * 16, lane);
+    constexpr int kBatch = 12;  // groups per warp whose loads are issued together (H = 6144: all of them)
+    for (int g0 = cw; g0 < G; g0 += kCW * kBatch) {
+        float2 v[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const int g = g0 + j * kCW;
+            v[j] = g < G ? load2<XT>(xr + g * kGroup + 2 * lane) : make_float2(0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const int g = g0 + j * kCW;
+            if (g < G) encode_group(v[j].x, v[j].y, a.xq + ((size_t)t * G + g) * 128, a.xm + ((size_t)t * G + g) * kMetaRow,
+                                    lane);
+        }
     }
 }
 
-// Router rows e0, e0+1 for every token: warps 4r..4r+3 take expert e0 + r,
-// each a quarter of H, with the weights held in registers across the tokens;
-// the four partial sums of a token are added in a fixed order (fp64).
+// Router rows e0, e0+1 for every token: warps 8r..8r+7 take expert e0 + r,
+// each an eighth of H, with the weights held in registers across the tokens;
+// the eight partial sums of a token are added in a fixed order (fp64).
 template <typename XT>
 __device__ void router_item(I8Args& a, I8Smem& S, double* rpart, int e0, int ctid) {
     const Dims& d = a.d;
@@ -472,39 +507,62 @@ __device__ void router_item(I8Args& a, I8Smem& S, double* rpart, int e0, int cti
     const int e = e0 + r;
     const int chunk = d.H / kParts;
     const XT* x = reinterpret_cast<const XT*>(a.x);
-    constexpr int kV = 12;  // float4 per lane per pass: one pass for H = 6144
+    constexpr int kV = 6;  // float4 per lane per pass: one pass for H = 6144
     for (int base = 0; base < chunk; base += kV * 128) {
-        float4 wv[kV];
+        float4 wv[kV], xv0[kV];
         const float* wrow = a.wr + (size_t)(e < d.E ? e : 0) * d.H + part * chunk;
+        auto load_x = [&](const XT* xr, int i) -> float4 {
+            if (i >= chunk) return make_float4(0.f, 0.f, 0.f, 0.f);
+            if constexpr (sizeof(XT) == 4) {
+                return __ldg(reinterpret_cast<const float4*>(xr + i));
+            } else {
+                const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr + i));
+                return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                                   __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+            }
+        };
+        // the weights and the first token's inputs in one batch of loads (one round trip)
 #pragma unroll
         for (int j = 0; j < kV; ++j) {
             const int i = base + lane * 4 + j * 128;
             wv[j] = (e < d.E && i < chunk) ? __ldg(reinterpret_cast<const float4*>(wrow + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            xv0[j] = load_x(x + part * chunk, i);
         }
-        for (int t = 0; t < T; ++t) {
-            const XT* xr = x + (size_t)t * d.H + part * chunk;
-            double sacc = 0.0;
-#pragma unroll
-            for (int j = 0; j < kV; ++j) {
-                const int i = base + lane * 4 + j * 128;
-                float4 xv = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (i < chunk) {
-                    if constexpr (sizeof(XT) == 4) {
-                        xv = __ldg(reinterpret_cast<const float4*>(xr + i));
-                    } else {
-                        const uint2 u = __ldg(reinterpret_cast<const uint2*>(xr + i));
-                        xv = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
-                                         __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
-                    }
-                }
-                sacc = fma((double)wv[j].x, (double)xv.x, sacc);
-                sacc = fma((double)wv[j].y, (double)xv.y, sacc);
-                sacc = fma((double)wv[j].z, (double)xv.z, sacc);
-                sacc = fma((double)wv[j].w, (double)xv.w, sacc);
-            }
+        auto store = [&](int t, double sacc) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) sacc += __shfl_xor_sync(0xffffffffu, sacc, o);
             if (lane == 0) rpart[(size_t)cw * T + t] = (base == 0 ? 0.0 : rpart[(size_t)cw * T + t]) + sacc;
+        };
+        {
+            double sacc = 0.0;
+#pragma unroll
+            for (int j = 0; j < kV; ++j) {
+                sacc = fma((double)wv[j].x, (double)xv0[j].x, sacc);
+                sacc = fma((double)wv[j].y, (double)xv0[j].y, sacc);
+                sacc = fma((double)wv[j].z, (double)xv0[j].z, sacc);
+                sacc = fma((double)wv[j].w, (double)xv0[j].w, sacc);
+            }
+            store(0, sacc);
+        }
+#pragma unroll 1
+        for (int t = 1; t < T; ++t) {
+            const XT* xr = x + (size_t)t * d.H + part * chunk;
+            double sacc = 0.0;
+#pragma unroll
+            for (int h2 = 0; h2 < kV; h2 += kV / 2) {  // x in two halves keeps registers bounded
+                float4 xv[kV / 2];
+#pragma unroll
+                for (int jj = 0; jj < kV / 2; ++jj) xv[jj] = load_x(xr, base + lane * 4 + (h2 + jj) * 128);
+#pragma unroll
+                for (int jj = 0; jj < kV / 2; ++jj) {
+                    const float4 wj = wv[h2 + jj];
+                    sacc = fma((double)wj.x, (double)xv[jj].x, sacc);
+                    sacc = fma((double)wj.y, (double)xv[jj].y, sacc);
+                    sacc = fma((double)wj.z, (double)xv[jj].z, sacc);
+                    sacc = fma((double)wj.w, (double)xv[jj].w, sacc);
+                }
+            }
+            store(t, sacc);
         }
     }
     named_bar(1, kCT);
@@ -555,7 +613,7 @@ __device__ void consumer_plan(I8Args& a, I8Smem& S, uint8_t* scratch, int ctid) 
     for (int t = cw; t < T; t += kCW) {
         int id;
         float wt;
-        if (E <= 256) warp_topk<true, 8>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
+        if (E <= 256) warp_topk8<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
         else warp_topk<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
         if (lane < K) {
             sids[t * K + lane] = id;
@@ -614,8 +672,7 @@ __device__ void consumer_plan(I8Args& a, I8Smem& S, uint8_t* scratch, int ctid) 
         *a.p.n_active = ucarry + d.S;
     }
     if (a.trace && ctid == 0) a.trace[7] = (long long)globaltimer_ns();
-    __threadfence();
-    named_bar(1, kCT);
+    named_bar(1, kCT);  // orders every consumer's plan writes before thread 0's release
     if (ctid == 0) {
         if (a.trace) a.trace[8] = (long long)globaltimer_ns();
         st_release(&a.ctl[kCI_Plan], ccarry + 1);
@@ -628,7 +685,7 @@ __device__ void consumer_plan(I8Args& a, I8Smem& S, uint8_t* scratch, int ctid) 
 // and per chunk the B fragment and the group meta of its token.
 template <int NCH>
 __device__ __forceinline__ void block_mma(const uint8_t* bp, const uint8_t* blimb, const uint8_t* bmeta, int g, int G,
-                                          int sub, int lane, float (&acc)[2][2]) {
+                                          int sub, int lane, int nt, float (&acc)[2][2]) {
     const int gi = lane >> 2, t4 = lane & 3;
     const uint4 w = *reinterpret_cast<const uint4*>(bp + sub * 512 + lane_slot(lane) * 16);
     const uint32_t sv = *reinterpret_cast<const uint32_t*>(bp + kNibbleBytes + sub * 32 + gi * 4);
@@ -640,17 +697,32 @@ __device__ __forceinline__ void block_mma(const uint8_t* bp, const uint8_t* blim
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
         // B column gi: token 4c + gi/2 of the item, part gi%2 (hi, lo)
-        const uint4 bf = *reinterpret_cast<const uint4*>(blimb + ((size_t)(c * kChunkTok + (gi >> 1)) * G + g) * 128 +
-                                                         (gi & 1) * 64 + t4 * 16);
-        const int4 mt = *reinterpret_cast<const int4*>(bmeta + ((size_t)(c * kChunkTok + t4) * G + g) * 16);
-        // accumulators start at the nibble offset's correction: -8 sum(part) (x16 for rows gi+8)
+        // columns of absent tokens are not read (zero): fewer shared-memory wavefronts
+        uint4 bf = make_uint4(0u, 0u, 0u, 0u);
+        int4 mt = make_int4(0, 0, 0, 0);
+        if (c * kChunkTok + (gi >> 1) < nt)
+            bf = *reinterpret_cast<const uint4*>(blimb + ((size_t)(c * kChunkTok + (gi >> 1)) * G + g) * 128 +
+                                                 (gi & 1) * 64 + t4 * 16);
+        if (c * kChunkTok + t4 < nt)
+            mt = *reinterpret_cast<const int4*>(bmeta + (size_t)(c * kChunkTok + t4) * meta_slot_bytes(G) +
+                                                (size_t)g * kMetaRow);
+        // one accumulator starts at the nibble offset's correction, -8 sum(part) (x16 for
+        // rows gi+8); the two 32-input halves accumulate separately (no dependency)
         int cc[4] = {mt.y, mt.z, mt.y * 16, mt.z * 16};
+        int cd[4] = {0, 0};
         mma_u8s8(cc, a0, a1, a2, a3, bf.x, bf.y);
-        mma_u8s8(cc, a4, a5, a6, a7, bf.z, bf.w);
+        mma_u8s8(cd, a4, a5, a6, a7, bf.z, bf.w);
         const float sx = __int_as_float(mt.x);
-        acc[c][0] = fmaf(s0 * sx, (float)(cc[0] * 256 + cc[1]), acc[c][0]);  // row gi,   token 4c + t4
-        acc[c][1] = fmaf(s1 * sx, (float)(cc[2] * 256 + cc[3]), acc[c][1]);  // row gi+8, token 4c + t4
+        const int p0 = (cc[0] + cd[0]) * 256 + (cc[1] + cd[1]), p1 = (cc[2] + cd[2]) * 256 + (cc[3] + cd[3]);
+        acc[c][0] = fmaf(s0 * sx, (float)p0, acc[c][0]);  // row gi,   token 4c + t4
+        acc[c][1] = fmaf(s1 * sx, (float)p1, acc[c][1]);  // row gi+8, token 4c + t4
     }
+}
+
+// Token i of a gate/up item: shared chunks hold consecutive tokens; routed
+// chunks read theirs from the published plan.
+__device__ __forceinline__ int item_token(const I8Args& a, const Item& it, int i) {
+    return it.tok0 >= 0 ? it.tok0 + i : __ldcg(a.p.tok + it.pos + i);
 }
 
 template <typename XT>
@@ -669,8 +741,7 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
     if (gu) {
         same = S.staged_kind == IT_GU && S.staged_n == nt;
         for (int i = 0; same && i < nt; ++i) {
-            const int tok = it.tok0 >= 0 ? it.tok0 + i : __ldcg(a.p.tok + it.pos + i);
-            same = S.staged_tok[i] == tok;
+            same = S.staged_tok[i] == item_token(a, it, i);
         }
     } else {
         same = S.staged_kind == IT_DOWN && S.staged_key == it.chunk;
@@ -686,19 +757,21 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
                 wait_geq(&a.ctl[kCI_Counters - 1], 1, abort_flag, a, 99);
             if (!*abort_flag) {
                 fence_proxy_async_global();
-                const uint32_t lbytes = (uint32_t)G * 128, mbytes = (uint32_t)G * 16;
+                const uint32_t lbytes = (uint32_t)G * 128, mbytes = (uint32_t)G * kMetaRow;
                 mbar_arrive_expect_tx(&S.bfull, (uint32_t)nt * (lbytes + mbytes));
                 S.bpending = 1;
                 if (gu) {
                     for (int i = 0; i < nt; ++i) {
-                        const int tok = it.tok0 >= 0 ? it.tok0 + i : __ldcg(a.p.tok + it.pos + i);
+                        const int tok = item_token(a, it, i);
                         S.staged_tok[i] = tok;
                         bulk_g2s(blimb + (size_t)i * lbytes, a.xq + (size_t)tok * lbytes, lbytes, &S.bfull);
-                        bulk_g2s(bmeta + (size_t)i * mbytes, a.xm + (size_t)tok * mbytes, mbytes, &S.bfull);
+                        bulk_g2s(bmeta + (size_t)i * meta_slot_bytes(G), a.xm + (size_t)tok * mbytes, mbytes, &S.bfull);
                     }
                 } else {
                     bulk_g2s(blimb, a.hq + (size_t)it.pos * lbytes, nt * lbytes, &S.bfull);
-                    bulk_g2s(bmeta, a.hm + (size_t)it.pos * mbytes, nt * mbytes, &S.bfull);
+                    for (int i = 0; i < nt; ++i)
+                        bulk_g2s(bmeta + (size_t)i * meta_slot_bytes(G), a.hm + (size_t)(it.pos + i) * mbytes, mbytes,
+                                 &S.bfull);
                 }
                 S.staged_kind = it.kind;
                 S.staged_n = nt;
@@ -718,8 +791,9 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
     }
 
     // ---- stream the weight tile through the ring
+    if (a.trace && ctid == 0) S.t_loop0 = globaltimer_ns();
     float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-    const int sub = cw;
+    const int sub = cw % kSub, half = cw / kSub;  // warps sub and sub + 8 share a sub-tile
     const uint32_t stage_bytes = (uint32_t)a.sb * kBlockBytes;
     const int nst = (G + a.sb - 1) / a.sb;
     const int nch = (nt + kChunkTok - 1) / kChunkTok;
@@ -744,11 +818,13 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
             const int g0 = i * a.sb;
             const int nb = min(a.sb, G - g0);
             if (nch == 1) {
-#pragma unroll 2
-                for (int bb = 0; bb < nb; ++bb) block_mma<1>(stage + bb * kBlockBytes, blimb, bmeta, g0 + bb, G, sub, lane, acc);
+#pragma unroll 4
+                for (int bb = half; bb < nb; bb += 2)
+                    block_mma<1>(stage + bb * kBlockBytes, blimb, bmeta, g0 + bb, G, sub, lane, nt, acc);
             } else {
 #pragma unroll 2
-                for (int bb = 0; bb < nb; ++bb) block_mma<2>(stage + bb * kBlockBytes, blimb, bmeta, g0 + bb, G, sub, lane, acc);
+                for (int bb = half; bb < nb; bb += 2)
+                    block_mma<2>(stage + bb * kBlockBytes, blimb, bmeta, g0 + bb, G, sub, lane, nt, acc);
             }
         }
         __syncwarp();
@@ -756,17 +832,24 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
         if (++slot_s == (uint32_t)a.nstages) { slot_s = 0; phase_s ^= 1; }
         seen = next_full;
     }
+    if (half == 1) *reinterpret_cast<float4*>(S.accx[sub][lane]) = make_float4(acc[0][0], acc[0][1], acc[1][0], acc[1][1]);
+    if (a.trace && ctid == 0) S.t_loop1 = globaltimer_ns();
     if (ctid == 0) S.aborted = *abort_flag;
     named_bar(1, kCT);
     const bool aborted = S.aborted != 0;  // uniform: read after the barrier
     if (aborted) return;
+    const bool lead = half == 0;  // the first warp of each sub-tile finishes the item
+    if (lead) {  // fixed order: blocks of the first warp, then those of the second
+        const float4 o = *reinterpret_cast<const float4*>(S.accx[sub][lane]);
+        acc[0][0] += o.x; acc[0][1] += o.y; acc[1][0] += o.z; acc[1][1] += o.w;
+    }
 
     // ---- epilogue: lane (gi, t4) holds rows gi, gi+8 of sub-tile `sub` for tokens t4 and 4 + t4
     if (!gu) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             const int i = c * kChunkTok + t4;
-            if (c < nch && i < nt) {
+            if (lead && c < nch && i < nt) {
                 const int r0 = it.rt * kTileRows + sub * kSubRows + gi;
                 float* orow = a.o + (size_t)(it.pos + i) * d.H;
                 orow[r0] = acc[c][0];
@@ -781,12 +864,12 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
     float hv[2] = {0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-        if (c < nch && c * kChunkTok + t4 < nt) hv[c] = silu_f(acc[c][0]) * acc[c][1];
+        if (lead && c < nch && c * kChunkTok + t4 < nt) hv[c] = silu_f(acc[c][0]) * acc[c][1];
         float m = fabsf(hv[c]);
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-        if (gi == 0) S.hmaxw[cw][c * kChunkTok + t4] = m;
+        if (lead && gi == 0) S.hmaxw[sub][c * kChunkTok + t4] = m;
     }
     named_bar(1, kCT);
     const int k = sub * 8 + gi;
@@ -796,34 +879,27 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
         const int i = c * kChunkTok + t4;
-        if (c < nch && i < nt) {
+        if (lead && c < nch && i < nt) {
             float m = 0.0f;
-            for (int w = 0; w < kCW; ++w) m = fmaxf(m, S.hmaxw[w][i]);
-            int e = 0;
-            if (m > 0.0f && m <= 3.0e38f) {
-                int ex;
-                frexpf(m, &ex);
-                e = 15 - ex;
-                e = e > 126 ? 126 : (e < -126 ? -126 : e);
-                if (ldexpf(m, e) > 32639.0f) e -= 1;
-            }
-            const int xi = __float2int_rn(hv[c] * ldexpf(1.0f, e));
+            for (int w = 0; w < kSub; ++w) m = fmaxf(m, S.hmaxw[w][i]);
+            const int e = group_exponent(m);
+            const int xi = __float2int_rn(hv[c] * pow2f(e));
             const int hi = (xi + 128) >> 8, lo = xi - 256 * hi;
             uint8_t* dst = a.hq + ((size_t)(it.pos + i) * f.Gd + g) * 128;
             dst[limb_offset(k)] = (uint8_t)(int8_t)hi;
             dst[64 + limb_offset(k)] = (uint8_t)(int8_t)lo;
             hs[c][0] = hi;
             hs[c][1] = lo;
-            sxv[c] = ldexpf(1.0f, -e);
+            sxv[c] = pow2f(-e);
         }
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             hs[c][0] += __shfl_xor_sync(0xffffffffu, hs[c][0], o);
             hs[c][1] += __shfl_xor_sync(0xffffffffu, hs[c][1], o);
         }
-        if (gi == 0) {
-            S.hsum[cw][c * kChunkTok + t4][0] = hs[c][0];
-            S.hsum[cw][c * kChunkTok + t4][1] = hs[c][1];
+        if (lead && gi == 0) {
+            S.hsum[sub][c * kChunkTok + t4][0] = hs[c][0];
+            S.hsum[sub][c * kChunkTok + t4][1] = hs[c][1];
         }
     }
     named_bar(1, kCT);
@@ -833,7 +909,7 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
             const int i = c * kChunkTok + t4;
             if (c < nch && i < nt) {
                 int sh = 0, sl = 0;
-                for (int w = 0; w < kCW; ++w) { sh += S.hsum[w][i][0]; sl += S.hsum[w][i][1]; }
+                for (int w = 0; w < kSub; ++w) { sh += S.hsum[w][i][0]; sl += S.hsum[w][i][1]; }
                 *reinterpret_cast<int4*>(a.hm + ((size_t)(it.pos + i) * f.Gd + g) * 16) =
                     make_int4(__float_as_int(sxv[c]), -8 * sh, -8 * sl, 0);
             }
@@ -845,7 +921,7 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
 // router items and of the plan).
 __host__ __device__ inline size_t b_area_bytes(const Dims& d, int T, int ntc) {
     const int G = (d.H > d.I ? d.H : d.I) / kGroup;
-    const size_t operands = (size_t)ntc * G * (128 + 16);
+    const size_t operands = (size_t)ntc * ((size_t)G * 128 + meta_slot_bytes(G));
     const size_t plan = (size_t)T * d.K * 8 + (size_t)2 * d.E * 4;
     const size_t router = (size_t)kCW * T * 8;
     size_t m = operands > plan ? operands : plan;
@@ -899,7 +975,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
             named_bar(1, kCT);
             const Item it = S.cur[q & 1];
             const uint64_t t_begin = (a.trace && ctid == 0) ? globaltimer_ns() : 0;
-            if (ctid == 0) S.first_wait_ns = S.total_wait_ns = 0;
+            if (ctid == 0) S.first_wait_ns = S.total_wait_ns = S.t_loop0 = S.t_loop1 = 0;
             if (it.kind == IT_PREP) {
                 prep_item<XT>(a, it.ex, ctid);
             } else if (it.kind == IT_ROUTER) {
@@ -910,7 +986,8 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
                 if (ctid == 0) {
                     const int n_router = (a.d.E + kRouterExperts - 1) / kRouterExperts;
                     const uint64_t t0 = a.trace ? globaltimer_ns() : 0;
-                    __threadfence();
+                    // the barrier orders the other consumers' logits before this
+                    // release, which carries them to the plan builders (cumulative)
                     S.last = atom_add_acq_rel(&a.ctl[kCI_Router], 1) == n_router - 1;
                     if (S.last && a.trace) { a.trace[1] = (long long)t0; a.trace[2] = (long long)globaltimer_ns(); }
                 }
@@ -926,7 +1003,8 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
                 if (k >= kSQ) wait_bar(&S.dempty[ds], ((k / kSQ) - 1) & 1, &S.abort_flag, a, 11);
                 S.done[ds] = it;
             }
-            __threadfence();
+            // every consumer's writes precede its arrival (release, CTA scope); the
+            // signaler's release atomic that follows carries them to other CTAs
             named_bar(1, kCT);
             mbar_arrive(&S.dfull[ds]);
             if (a.trace && ctid == 0 && it.kind != IT_END) {
@@ -941,8 +1019,8 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
                     rec[3] = (long long)S.first_wait_ns;
                     rec[4] = it.cnt;
                     rec[5] = (long long)S.total_wait_ns;
-                    rec[6] = it.chunk;
-                    rec[7] = 0;
+                    rec[6] = (long long)S.t_loop0;
+                    rec[7] = (long long)S.t_loop1;
                 }
             }
             if (ctid == 0 && it.kind != IT_END) mbar_arrive(&S.qempty[slot]);

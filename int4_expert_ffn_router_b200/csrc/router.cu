@@ -229,7 +229,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ lo
     if (t >= T) return;
     int id;
     float wt;
-    warp_topk<false>(logits + (size_t)t * E, E, K, lane, &id, &wt);
+    if (E <= 256) warp_topk8<false>(logits + (size_t)t * E, E, K, lane, &id, &wt);
+    else warp_topk<false>(logits + (size_t)t * E, E, K, lane, &id, &wt);
     if (lane < K) {
         ids[(size_t)t * K + lane] = id;
         w[(size_t)t * K + lane] = wt;
