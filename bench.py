@@ -12,7 +12,8 @@ batch. Inputs are resident in HBM before the timed region; L2 is flushed
 between steps by a 256 MiB memset recorded outside the per-step events.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload decode_b1|decode_b32|prefill_2048|stack30_b1|stack30_b8|stack30_b64]
+                    [--workload decode_b1|decode_b32|prefill_2048|stack30_b1|stack30_b8|stack30_b64|
+                                decode_b1_cached|stack4_b1_cached]
 
 Prints one JSON line (rank 0). N > 1 runs N independent replicas (one per
 rank, launched by torch.distributed.run), weak scaling, max time over ranks.
@@ -63,13 +64,26 @@ WORKLOADS = {
                        desc="30-layer stack of the full-size layer, decode batch 8, Zipf(1.1) per layer"),
     "stack30_b64": dict(T=64, zipf=True, bf16=False, layers=30,
                         desc="30-layer stack of the full-size layer, decode batch 64, Zipf(1.1) per layer"),
+    # expert cache over page-locked host memory: 64 of the 256 routed experts of a layer in HBM,
+    # all 256 in host memory; Zipf(1.1) routing; after an untimed learning pass the 48 experts
+    # routed to most often are pinned (the learned hot set), least-recently-used eviction in the
+    # other 16 slots; every miss is one host-to-HBM copy of the expert's 20 MB
+    "decode_b1_cached": dict(T=1, zipf=True, bf16=False, resident=64, pin=48,
+                             desc="one full-size layer as an expert cache (64 of 256 routed experts in HBM, 48 "
+                                  "pinned by learned usage, LRU), decode batch 1, Zipf(1.1) router bias, fp32"),
+    "stack4_b1_cached": dict(T=1, zipf=True, bf16=False, layers=4, resident=64, pin=48,
+                             desc="4-layer stack of expert-cache layers (64 of 256 in HBM each, 48 pinned, LRU), "
+                                  "each next layer's router run one layer ahead to prefetch, decode batch 1, "
+                                  "Zipf(1.1) per layer"),
 }
 X_SEED0 = 1000  # step s draws its activations with seed X_SEED0 + s
+LEARN_SEED0 = 500_000  # the cache workloads' learning pass draws its own tokens
 FUSED_MODE = {"i8": 1, "separate": 0}
 
 
 DEFAULT_STEPS = {"decode_b1": 10000, "decode_b32": 2000, "prefill_2048": 100, "decode_b1_e16": 1000, "prefill_e64": 100,
-                 "stack30_b1": 300, "stack30_b8": 200, "stack30_b64": 100}
+                 "stack30_b1": 300, "stack30_b8": 200, "stack30_b64": 100, "decode_b1_cached": 2000,
+                 "stack4_b1_cached": 500}
 
 
 def step_seed(step, rank):
@@ -367,9 +381,9 @@ class Clocks:
         return out
 
 
-def build_layer(torch, coli, synth, wl, device, max_tokens, layer_idx=0):
+def build_layer(torch, coli, synth, wl, device, max_tokens, layer_idx=0, resident=None):
     """Layer `layer_idx` of the workload: router, Zipf bias and experts drawn
-    with the generator's layer index."""
+    with the generator's layer index (resident: slots of an expert cache)."""
     E = wl.get("E", E_FULL)
     nq, ns = synth.expert_sizes(H, I)
     dev = torch.device("cuda", device)
@@ -384,7 +398,8 @@ def build_layer(torch, coli, synth, wl, device, max_tokens, layer_idx=0):
         bias = torch.from_numpy(synth.zipf_bias(0, layer_idx, E)[0]).to(dev)
     torch.cuda.synchronize(dev)
     cfg = coli.make_config(H, I, E, K, S, max_tokens)
-    layer = coli.Layer(cfg, wr, bias, q[:E * nq], s[:E * ns], q[E * nq:], s[E * ns:], device=device)
+    layer = coli.Layer(cfg, wr, bias, q[:E * nq], s[:E * ns], q[E * nq:], s[E * ns:], device=device,
+                       resident=resident)
     del q, s, wr
     torch.cuda.empty_cache()
     return layer
@@ -769,6 +784,191 @@ def run_stack(args, wl, ws, rank, local):
     return out
 
 
+def host_link_gbs(torch, dev, nbytes=1 << 30, reps=3):
+    """Best of `reps` plain copies of `nbytes` from page-locked host memory to
+    HBM (CUDA events): the host link's measured rate for the cache workloads."""
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    best = 0.0
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src, non_blocking=True)
+        b.record()
+        b.synchronize()
+        best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del src, dst
+    torch.cuda.empty_cache()
+    return best
+
+
+def run_cached(args, wl, ws, rank, local):
+    """Expert-cache workloads: layers with `resident` of their 256 routed
+    experts in HBM over a page-locked host copy of all of them. An untimed
+    learning pass (its own tokens) counts routing per expert; the `pin` most
+    used are pinned; the counters are then reset, and the timed steps measure
+    hits, misses and host-to-HBM bytes. One layer: coli_moe_forward; several:
+    coli_moe_stack_forward, whose next-layer lookahead prefetches."""
+    import numpy as np
+    import torch
+    import synth
+    import int4_expert_ffn_router_b200 as coli
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+    T, NL, R = wl["T"], wl.get("layers", 1), wl["resident"]
+    stack = NL > 1
+    link = host_link_gbs(torch, dev)
+    layers = [build_layer(torch, coli, synth, wl, local, max_tokens=T, layer_idx=l, resident=R) for l in range(NL)]
+    for L in layers:
+        L.set_fused(FUSED_MODE[args.decode_kernel])
+    nsteps = args.warmup + args.steps
+    stream = torch.cuda.current_stream(dev)
+    xs = torch.empty((nsteps, T, H), dtype=torch.float32, device=dev)
+    for i in range(nsteps):
+        synth.x_dev(step_seed(i, rank), 0, T, H, 0, xs[i].data_ptr(), stream.cuda_stream)
+    xw = torch.empty((T, H), dtype=torch.float32, device=dev)
+    y = torch.empty((T, H), dtype=torch.float32, device=dev)
+
+    def step(x):
+        if stack:
+            xw.copy_(x)
+            coli.stack_forward(layers, xw, stream=stream)
+        else:
+            layers[0].forward(x, y, stream=stream)
+
+    # learning pass: routing counts per expert, then the hot set is pinned
+    n_learn = 400
+    xl = torch.empty((T, H), dtype=torch.float32, device=dev)
+    for i in range(n_learn):
+        synth.x_dev(LEARN_SEED0 + i + 10_000 * rank, 0, T, H, 0, xl.data_ptr(), stream.cuda_stream)
+        step(xl)
+    torch.cuda.synchronize(dev)
+    for L in layers:
+        L.pin_hot(wl["pin"])
+    for i in range(args.warmup):
+        step(xs[i])
+    torch.cuda.synchronize(dev)
+    for L in layers:
+        L.cache_stats(reset=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
+    clocks = Clocks(local, coli, torch, stream)
+    n0 = sum(L.launch_count() for L in layers)
+    for i in range(args.warmup, nsteps):
+        ev[i][0].record(stream)
+        step(xs[i])
+        ev[i][1].record(stream)
+    clocks.end_region()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    launches = sum(L.launch_count() for L in layers) - n0
+    st = [L.cache_stats(reset=True) for L in layers]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    step_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.warmup, nsteps)]
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
+    # per-stage device times from a separate pass (not in the timed region)
+    for L in layers:
+        L.set_profiling(True)
+    for i in range(args.warmup, min(nsteps, args.warmup + 100)):
+        step(xs[i])
+    torch.cuda.synchronize(dev)
+    stages, nprof = {}, 0
+    for L in layers:
+        sp, nprof = L.profile()
+        for k, v in sp.items():
+            stages[k] = stages.get(k, 0.0) + v
+        L.set_profiling(False)
+    for L in layers:
+        L.cache_stats(reset=True)
+    # end to end through the C ABI with host buffers
+    if stack:
+        e2e_ms = e2e_pipelined(torch, dev, stream, xs[args.warmup:],
+                               lambda xin, _: coli.stack_forward(layers, xin, stream=stream), (T, H), torch.float32,
+                               args.steps, dist, inplace=True)
+    else:
+        e2e_ms = e2e_pipelined(torch, dev, stream, xs[args.warmup:],
+                               lambda xin, yout: layers[0].forward(xin, yout, stream=stream), (T, H), torch.float32,
+                               args.steps, dist)
+    if stack:
+        err = stack_output_error(torch, coli, synth, wl, layers, xs[args.warmup], stream) if rank == 0 else None
+    else:
+        err = output_error(torch, coli, synth, wl, layers[0], xs[args.warmup], y, stream) if rank == 0 else None
+    for L in layers:
+        L.close()
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return None
+
+    hits = sum(x["hits"] for x in st)
+    misses = sum(x["misses"] for x in st)
+    h2d = sum(x["bytes_h2d"] for x in st)
+    secs = sum(step_ms) * 1e-3
+    pred = sum(x["predicted"] for x in st)
+    pred_of = sum(x["predicted_of"] for x in st)
+    pref = sum(x["prefetched"] for x in st)
+    pref_used = sum(x["prefetch_used"] for x in st)
+    needed_per_step = (hits + misses) / args.steps
+    hbm_bytes = needed_per_step * EXPERT_BYTES + NL * (S * EXPERT_BYTES + E_FULL * H * 4)
+    peaks = load_peaks()
+    kernel_stages = {k: v for k, v in stages.items() if k != "cache"}
+    dom, roof = dominant_roofline(kernel_stages, nprof * NL, T, needed_per_step / NL, E_FULL, 4, False, peaks)
+    cache_ms = stages.get("cache", 0.0) / max(nprof, 1)
+    out = {
+        "metric": METRIC, "value": round(job_tokens_per_s(ws, args.steps, T, total_ms), 2), "unit": "tokens/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
+        "step_ms_rank0": step_percentiles(step_ms),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": path_dtype(args.decode_kernel, T, False, False),
+        "data": "synthetic (seeded generator; random-init int4 weights of the full-size layer shape)",
+        "config": {"workload": args.workload, "desc": wl["desc"], "layers": NL, "hidden": H, "inter": I,
+                   "experts": E_FULL, "top_k": K, "shared": S, "tokens_per_step": T, "resident_slots": R,
+                   "pinned": wl["pin"], "learning_steps": n_learn,
+                   "l2": "not flushed: every step copies experts from host memory or streams them from HBM",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "cache": {
+            "hit_rate": round(hits / max(hits + misses, 1), 4),
+            "misses_per_step": round(misses / args.steps, 3),
+            "needed_per_step": round(needed_per_step, 3),
+            "h2d_bytes_per_step": int(h2d / args.steps),
+            "h2d_gbs": round(h2d / secs / 1e9, 2),
+            "host_link_gbs_measured": round(link, 2),
+            "host_link_frac": round(h2d / secs / 1e9 / link, 4),
+            "host_pool_bytes_per_layer": E_FULL * EXPERT_BYTES,
+            "hbm_expert_bytes_per_layer": (R + S) * EXPERT_BYTES,
+            "cache_stage_us": round(cache_ms * 1e3 / NL, 2),
+            "lookahead_accuracy": round(pred / pred_of, 4) if pred_of else None,
+            "prefetched_per_step": round(pref / args.steps, 3),
+            "prefetch_used_frac": round(pref_used / pref, 4) if pref else None,
+            "note": ("hit = a needed expert already in HBM; h2d = page-locked host to HBM copies (misses and "
+                     "prefetches); lookahead accuracy = needed experts of layers 1.. that the previous layer's "
+                     "lookahead routing named"),
+        },
+        "hbm_bytes_per_step": int(hbm_bytes),
+        "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items() if v > 0},
+        "roofline": roof,
+        "gpu_launches": launches,
+        "gpu_launches_note": "forward kernels in the timed loop; two clock-stamp kernels bracket the loop",
+        "max_rel_err": err,
+        "e2e": {"value": round(job_tokens_per_s(ws, args.steps, T, e2e_ms), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4, "method": E2E_METHOD},
+        "clocks": clk,
+    }
+    if dist:
+        dist.destroy_process_group()
+    return out
+
+
 def main():
     args = parse()
     wl = WORKLOADS[args.workload]
@@ -804,7 +1004,12 @@ def main():
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(wl, args.cpu_seconds)
-    out = run_stack(args, wl, ws, rank, local) if wl.get("layers") else run_ours(args, wl, ws, rank, local)
+    if wl.get("resident"):
+        out = run_cached(args, wl, ws, rank, local)
+    elif wl.get("layers"):
+        out = run_stack(args, wl, ws, rank, local)
+    else:
+        out = run_ours(args, wl, ws, rank, local)
     if out is not None:
         out["cpu_baseline"] = cpu
         print(json.dumps(out))

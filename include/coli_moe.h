@@ -99,6 +99,88 @@ coli_status coli_moe_layer_set_experts(coli_moe_layer* layer, int first, int cou
 
 void coli_moe_layer_destroy(coli_moe_layer* layer);
 
+/*
+ * Expert cache: a layer whose routed experts do not all stay in HBM.
+ * The Colibri pages keep the hot experts in fast memory and fetch the others
+ * on demand ("Colibri: 2400 lines of pure C ..." (kechuai.cn), section 二: a
+ * per-layer cache with least-recently-used eviction, a hot set learned from
+ * routing counts that stays pinned, and the next layer's router run one
+ * layer ahead to prefetch; project page (gh.puless.com/p/colibri.html),
+ * placement tiers). Here HBM is the cache and page-locked host memory the
+ * store behind it.
+ *
+ * Arguments as coli_moe_layer_create, plus resident_slots R with
+ * min(n_experts, max_tokens * top_k) <= R <= n_experts; expert_q and
+ * expert_scales must not be NULL. HBM holds R routed experts and the shared
+ * experts; every routed expert is also kept, in the device layout, in
+ * page-locked host memory (n_experts * stride bytes, stride about
+ * coli_moe_expert_bytes rounded up to 256). Experts 0..R-1 start resident.
+ *
+ * coli_moe_forward on a cached layer routes the batch, reads the ids back
+ * (the call waits for them, so it cannot be captured in a CUDA graph), makes
+ * every routed expert the batch needs resident, then runs the resident
+ * layer's kernels through the slot table with that routing. A missing expert
+ * takes a free slot, else the slot whose expert was used least recently among
+ * those neither pinned nor needed by the batch; it arrives by one
+ * cudaMemcpyAsync of its gate/up and down matrices (adjacent) on the
+ * forward's stream. The output equals a resident layer's for the same
+ * routing, bit for bit. coli_moe_stack_forward over cached layers also runs
+ * each next layer's router on the current layer's input and prefetches the
+ * experts it picks on that layer's own copy stream while the current layer's
+ * kernels run (see coli_moe_cache_set_lookahead).
+ * coli_moe_layer_set_experts on a cached layer updates the host copy (and the
+ * HBM copy when resident).
+ */
+coli_status coli_moe_layer_create_cached(const coli_moe_config* cfg, const float* router_w, const float* router_bias,
+                                         const uint8_t* expert_q, const uint16_t* expert_scales,
+                                         const uint8_t* shared_q, const uint16_t* shared_scales,
+                                         int resident_slots, int device, coli_moe_layer** out);
+
+typedef struct {
+    int64_t hits;           /* experts a batch needed that were resident                */
+    int64_t misses;         /* experts a batch needed that were copied in before it     */
+    int64_t bytes_h2d;      /* expert bytes copied from host memory (misses + prefetch)  */
+    int64_t prefetched;     /* experts copied ahead of need (lookahead, prefetch, pin)   */
+    int64_t prefetch_used;  /* of those, the ones a batch needed before their eviction   */
+    int64_t predicted;      /* needed experts that the lookahead prediction named        */
+    int64_t predicted_of;   /* needed experts of the forwards that had a prediction      */
+    int32_t resident_slots; /* R                                                         */
+    int32_t n_pinned;       /* experts pinned by coli_moe_cache_pin                      */
+} coli_cache_stats;
+
+/*
+ * Counters of a cached layer since creation or the last reset (reset != 0
+ * clears them after reading; the usage counts are kept). usage: NULL or
+ * [n_experts] int64, the number of batches that routed to each expert since
+ * creation: the learned hot set (save it across sessions and pass its top
+ * entries to coli_moe_cache_pin). Waits for the layer's copies in flight.
+ * COLI_EINVAL on a layer that is not cached.
+ */
+coli_status coli_moe_cache_stats(coli_moe_layer* layer, coli_cache_stats* stats, int64_t* usage, int reset);
+
+/*
+ * Pins the n experts ids[0..n) (host int32; n == 0 unpins all): they become
+ * resident now and are never evicted. At most
+ * R - min(n_experts, max_tokens * top_k) experts may be pinned, so that any
+ * batch still fits. Synchronous.
+ */
+coli_status coli_moe_cache_pin(coli_moe_layer* layer, const int32_t* ids, int n);
+
+/*
+ * Copies the distinct experts among ids[0..n) (host int32) into HBM ahead of
+ * need, on the layer's copy stream, evicting by the same rule as a forward
+ * (as many as fit). Returns at once; the next forward waits for the copies.
+ */
+coli_status coli_moe_cache_prefetch(coli_moe_layer* layer, const int32_t* ids, int n);
+
+/* The cache slot of each routed expert (host int32 [n_experts]; -1: not in
+ * HBM), as placed by the calls made so far (copies may still be in flight). */
+coli_status coli_moe_cache_slots(const coli_moe_layer* layer, int32_t* slots);
+
+/* Whether this cached layer accepts the previous stack layer's lookahead
+ * prediction (1, the default) or not (0). */
+coli_status coli_moe_cache_set_lookahead(coli_moe_layer* layer, int enable);
+
 /* Copy of the layer's configuration. */
 coli_status coli_moe_layer_config(const coli_moe_layer* layer, coli_moe_config* cfg);
 
@@ -185,10 +267,13 @@ coli_status coli_moe_get_plan(coli_moe_layer* layer, int32_t* ids, float* weight
  * all forwards since profiling was enabled, and their number. Enabling again
  * resets the totals. On the tensor-core path the plan stage also covers the
  * operand rows, the tile list and the clear of the fp32 output, so the
- * gate/up and down stages each time one grouped-GEMM kernel alone.
+ * gate/up and down stages each time one grouped-GEMM kernel alone. The cache
+ * stage (cached layers) runs from the routed ids' read-back to the kernels:
+ * the next layer's lookahead routing, the copies of missing experts and the
+ * slot table upload, plus the host's wait for the ids.
  */
 enum { COLI_STAGE_ROUTER = 0, COLI_STAGE_TOPK, COLI_STAGE_PLAN, COLI_STAGE_GATEUP, COLI_STAGE_DOWN,
-       COLI_STAGE_COMBINE, COLI_STAGE_FUSED, COLI_N_STAGES };
+       COLI_STAGE_COMBINE, COLI_STAGE_FUSED, COLI_STAGE_CACHE, COLI_N_STAGES };
 coli_status coli_moe_set_profiling(coli_moe_layer* layer, int enable);
 coli_status coli_moe_get_profile(coli_moe_layer* layer, double* stage_ms_total, int64_t* n_forwards);
 const char* coli_moe_stage_name(int stage);
@@ -296,9 +381,9 @@ coli_status coli_moe_route_noalloc(const float* router_w, const float* router_bi
 coli_status coli_moe_debug_wait_test(coli_moe_layer* layer, int enable, int64_t wait_ns);
 
 /*
- * Testing aid for the out-of-memory paths: from now on, the nth device
- * allocation this library makes for a layer (create, set_experts) fails as
- * if the device had no memory left; 0 disables. The failing call returns
+ * Testing aid for the out-of-memory paths: from now on, the nth device or
+ * page-locked host allocation this library makes for a layer (create,
+ * set_experts) fails as if that memory were exhausted; 0 disables. The failing call returns
  * COLI_ENOMEM, frees what it had allocated, and create leaves *out NULL.
  * Process-wide; nth < 0 returns COLI_EINVAL.
  */

@@ -24,16 +24,24 @@ EXPORTS = (
     "coli_moe_expert_bytes", "coli_status_string", "coli_last_error", "coli_moe_set_profiling",
     "coli_moe_get_profile", "coli_moe_stage_name", "coli_moe_sync", "coli_moe_set_fused", "coli_moe_set_tensor_cores",
     "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc", "coli_moe_get_launch_count",
-    "coli_moe_debug_fail_alloc", "coli_clock_stamp", "coli_moe_debug_wait_test",
+    "coli_moe_debug_fail_alloc", "coli_clock_stamp", "coli_moe_debug_wait_test", "coli_moe_layer_create_cached",
+    "coli_moe_cache_stats", "coli_moe_cache_pin", "coli_moe_cache_prefetch", "coli_moe_cache_set_lookahead",
+    "coli_moe_cache_slots",
 )
 NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 63, 1024
-N_STAGES = 7
+N_STAGES = 8
 
 
 class Config(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("n_experts", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("n_shared", ctypes.c_int), ("group_size", ctypes.c_int),
                 ("max_tokens", ctypes.c_int)]
+
+
+class CacheStats(ctypes.Structure):
+    _fields_ = [("hits", ctypes.c_int64), ("misses", ctypes.c_int64), ("bytes_h2d", ctypes.c_int64),
+                ("prefetched", ctypes.c_int64), ("prefetch_used", ctypes.c_int64), ("predicted", ctypes.c_int64),
+                ("predicted_of", ctypes.c_int64), ("resident_slots", ctypes.c_int32), ("n_pinned", ctypes.c_int32)]
 
 
 class ColiError(RuntimeError):
@@ -75,6 +83,12 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_debug_fail_alloc.argtypes = [i32]
     L.coli_clock_stamp.argtypes = [vp, i32, vp]
     L.coli_moe_debug_wait_test.argtypes = [vp, i32, ctypes.c_int64]
+    L.coli_moe_layer_create_cached.argtypes = [pcfg, vp, vp, vp, vp, vp, vp, i32, i32, ctypes.POINTER(vp)]
+    L.coli_moe_cache_stats.argtypes = [vp, ctypes.POINTER(CacheStats), vp, i32]
+    L.coli_moe_cache_pin.argtypes = [vp, vp, i32]
+    L.coli_moe_cache_prefetch.argtypes = [vp, vp, i32]
+    L.coli_moe_cache_set_lookahead.argtypes = [vp, i32]
+    L.coli_moe_cache_slots.argtypes = [vp, vp]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
     L.coli_last_error.argtypes = []
@@ -127,17 +141,24 @@ def expert_bytes(hidden: int, inter: int) -> int:
 
 
 class Layer:
-    """One MoE layer resident on a CUDA device."""
+    """One MoE layer on a CUDA device: every expert resident in HBM, or, with
+    ``resident`` = R, an expert cache of R routed experts in HBM over a
+    page-locked host copy of all of them."""
 
     def __init__(self, cfg: Config, router_w, router_bias=None, expert_q=None, expert_scales=None,
-                 shared_q=None, shared_scales=None, device: int = 0):
+                 shared_q=None, shared_scales=None, device: int = 0, resident: int | None = None):
         h = ctypes.c_void_p()
-        _check(lib.coli_moe_layer_create(ctypes.byref(cfg), _ptr(router_w), _ptr(router_bias), _ptr(expert_q),
-                                         _ptr(expert_scales), _ptr(shared_q), _ptr(shared_scales), device,
-                                         ctypes.byref(h)), "coli_moe_layer_create")
+        args = (ctypes.byref(cfg), _ptr(router_w), _ptr(router_bias), _ptr(expert_q), _ptr(expert_scales),
+                _ptr(shared_q), _ptr(shared_scales))
+        if resident is None:
+            _check(lib.coli_moe_layer_create(*args, device, ctypes.byref(h)), "coli_moe_layer_create")
+        else:
+            _check(lib.coli_moe_layer_create_cached(*args, resident, device, ctypes.byref(h)),
+                   "coli_moe_layer_create_cached")
         self._h = h
         self.cfg = cfg
         self.device = device
+        self.resident = resident
 
     @property
     def handle(self) -> ctypes.c_void_p:
@@ -219,6 +240,51 @@ class Layer:
         _check(lib.coli_moe_get_profile(self.handle, ctypes.cast(buf, ctypes.c_void_p), ctypes.byref(n)),
                "coli_moe_get_profile")
         return {lib.coli_moe_stage_name(i).decode(): float(buf[i]) for i in range(N_STAGES)}, n.value
+
+    def cache_stats(self, reset: bool = False, usage: bool = False):
+        """Counters of a cached layer (dict); with usage=True also the per-expert
+        routing counts (numpy int64 [E]) under "usage"."""
+        import numpy as np
+        st = CacheStats()
+        use = np.zeros(self.cfg.n_experts, np.int64) if usage else None
+        _check(lib.coli_moe_cache_stats(self.handle, ctypes.byref(st), _ptr(use), 1 if reset else 0),
+               "coli_moe_cache_stats")
+        out = {name: getattr(st, name) for name, _ in CacheStats._fields_}
+        if usage:
+            out["usage"] = use
+        return out
+
+    def pin(self, ids) -> None:
+        """Pin these experts (resident, never evicted); an empty list unpins all."""
+        import numpy as np
+        a = np.ascontiguousarray(ids, dtype=np.int32)
+        _check(lib.coli_moe_cache_pin(self.handle, _ptr(a) if a.size else None, int(a.size)), "coli_moe_cache_pin")
+
+    def pin_hot(self, n: int, usage=None):
+        """Pin the n experts routed to most often (from `usage`, e.g. counts saved
+        by an earlier session, else this layer's own); returns their ids."""
+        import numpy as np
+        u = self.cache_stats(usage=True)["usage"] if usage is None else np.asarray(usage)
+        ids = np.argsort(-u, kind="stable")[:n].astype(np.int32)
+        self.pin(ids)
+        return ids
+
+    def prefetch(self, ids) -> None:
+        """Copy these experts into HBM ahead of need (asynchronous, copy stream)."""
+        import numpy as np
+        a = np.ascontiguousarray(ids, dtype=np.int32)
+        _check(lib.coli_moe_cache_prefetch(self.handle, _ptr(a) if a.size else None, int(a.size)),
+               "coli_moe_cache_prefetch")
+
+    def cache_slots(self):
+        """Slot of each routed expert in HBM (numpy int32 [E]; -1: not resident)."""
+        import numpy as np
+        out = np.zeros(self.cfg.n_experts, np.int32)
+        _check(lib.coli_moe_cache_slots(self.handle, _ptr(out)), "coli_moe_cache_slots")
+        return out
+
+    def set_lookahead(self, on: bool) -> None:
+        _check(lib.coli_moe_cache_set_lookahead(self.handle, 1 if on else 0), "coli_moe_cache_set_lookahead")
 
     def plan(self, T: int):
         """Host copies of the last forward's routing and batch-union plan."""

@@ -71,8 +71,8 @@ constexpr int kCoreTok = 4;
 constexpr int kTcMaxTok = 128;
 constexpr int kMaxStages = 24;
 // Word of the layer's control block where a persistent kernel that gave up
-// on a bounded wait records its site code (0: none).
-constexpr int kCtlError = 4;
+// on a bounded wait records its site code (0: none); alone in its 128-byte line.
+constexpr int kCtlError = 128;
 
 inline int64_t matrix_bytes(int rows, int cols) {
     return (int64_t)(rows / kTileRows) * (cols / kGroup) * kBlockBytes;
@@ -83,7 +83,13 @@ struct Dims {
     int64_t gu_bytes;      // gate/up matrix [2I][H]
     int64_t d_bytes;       // down matrix [H][I]
     int64_t expert_stride; // gu_bytes + d_bytes (multiple of 256)
+    const int32_t* slot_of;  // device [E + S]: weight slot of each expert (expert cache), or NULL: slot = id
 };
+
+// Byte offset of expert e's weights in the layer's weight pool.
+__device__ __forceinline__ size_t expert_offset(const Dims& d, int e) {
+    return (size_t)(d.slot_of ? __ldg(d.slot_of + e) : e) * (size_t)d.expert_stride;
+}
 
 // Per-call workspace views (device pointers into the layer's workspace).
 struct Plan {

@@ -53,7 +53,13 @@ __host__ __device__ constexpr size_t meta_slot_bytes(int G) { return (size_t)(G 
 enum { IT_END = 0, IT_PREP = 1, IT_ROUTER = 2, IT_GU = 3, IT_DOWN = 4 };
 
 // Control block (ints, zero between launches).
-enum { kCI_Ticket = 0, kCI_Router = 1, kCI_Plan = 2, kCI_Exit = 3, kCI_Error = kCtlError, kCI_Prep = 5, kCI_Counters = 8 };
+// Each word that many CTAs poll or update gets its own 128-byte line, so
+// pollers of one do not slow the atomics on another.
+enum {
+    kCI_Ticket = 0, kCI_Router = 32, kCI_Plan = 64, kCI_Exit = 96, kCI_Error = kCtlError, kCI_Prep = 160,
+    kCI_Never = 192,  // never set: the testing aid of coli_moe_debug_wait_test waits on it
+    kCI_Counters = 224
+};
 
 struct Item {
     int kind;
@@ -77,6 +83,8 @@ struct I8Args {
     int T;
     Plan p;
     double* logits;
+    const int32_t* given_ids;  // [T][K] routing computed before the launch (expert cache), or NULL
+    const float* given_w;      // [T][K] its weights
     uint8_t* xq;   // [T][H/64][128]  token limbs
     uint8_t* xm;   // [T][H/64][16]   token group meta
     uint8_t* hq;   // [slots][I/64][128]
@@ -168,19 +176,22 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
     }
 }
 
-// Bounded wait until *p >= target (acquire).
+// Bounded wait until *p >= target (acquire), polling with exponential backoff
+// (64 ns to 1 us) so that many waiting CTAs do not flood the word's L2 slice.
 __device__ __forceinline__ bool wait_geq(const int* p, int target, volatile int* abort_flag, I8Args& a, int code) {
     if (ld_acquire(p) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
+    uint32_t sleep_ns = 64;
     for (uint32_t n = 1;; ++n) {
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 1024) sleep_ns *= 2;
         if (ld_acquire(p) >= target) return true;
         if (*abort_flag) return false;
-        if ((n & 15) == 0 && others_gave_up(a, abort_flag)) return false;
+        if ((n & 7) == 0 && others_gave_up(a, abort_flag)) return false;
         if (globaltimer_ns() - t0 > (uint64_t)a.wait_ns) {
             set_error(a, abort_flag, code);
             return false;
         }
-        __nanosleep(64);
     }
 }
 
@@ -270,7 +281,7 @@ __device__ __forceinline__ Phases phases_of(const I8Args& a) {
     Phases f;
     const Dims& d = a.d;
     f.P = a.T;
-    f.R = (d.E + kRouterExperts - 1) / kRouterExperts;
+    f.R = a.given_ids ? 0 : (d.E + kRouterExperts - 1) / kRouterExperts;
     f.SC = d.S * a.cps;
     f.RTgu = 2 * d.I / kTileRows;
     f.RTd = d.H / kTileRows;
@@ -348,7 +359,7 @@ __device__ void i8_producer(I8Args& a, I8Smem& S, uint8_t* ring) {
         if (it.kind == IT_GU || it.kind == IT_DOWN) {
             const bool gu = it.kind == IT_GU;
             const int G = gu ? f.Ggu : f.Gd;
-            const uint8_t* tile = a.weights + (size_t)it.ex * d.expert_stride + (gu ? 0 : d.gu_bytes) +
+            const uint8_t* tile = a.weights + expert_offset(d, it.ex) + (gu ? 0 : d.gu_bytes) +
                                   (size_t)it.rt * G * kBlockBytes;
             const uint32_t stage_bytes = (uint32_t)a.sb * kBlockBytes;
             for (int b0 = 0; b0 < G; b0 += a.sb) {
@@ -610,14 +621,21 @@ __device__ void consumer_plan(I8Args& a, I8Smem& S, uint8_t* scratch, int ctid) 
     int* scnt = reinterpret_cast<int*>(sw + TK);           // [E]
     int* soff = scnt + E;                                  // [E]
     if (a.trace && ctid == 0) a.trace[4] = (long long)globaltimer_ns();
-    for (int t = cw; t < T; t += kCW) {
-        int id;
-        float wt;
-        if (E <= 256) warp_topk8<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
-        else warp_topk<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
-        if (lane < K) {
-            sids[t * K + lane] = id;
-            sw[t * K + lane] = wt;
+    if (a.given_ids) {  // routing computed before the launch
+        for (int sl = ctid; sl < TK; sl += kCT) {
+            sids[sl] = __ldcg(a.given_ids + sl);
+            sw[sl] = __ldcg(a.given_w + sl);
+        }
+    } else {
+        for (int t = cw; t < T; t += kCW) {
+            int id;
+            float wt;
+            if (E <= 256) warp_topk8<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
+            else warp_topk<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
+            if (lane < K) {
+                sids[t * K + lane] = id;
+                sw[t * K + lane] = wt;
+            }
         }
     }
     for (int e = ctid; e < E; e += kCT) scnt[e] = 0;
@@ -754,7 +772,7 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
             else ok = it.ready || wait_geq(&a.ctl[i8_ctl_gu(f.nch) + it.chunk], f.RTgu, abort_flag, a, 6);
             // testing aid: the launch's first gate/up tile waits on a flag that nothing sets
             if (ok && a.wait_test && gu && it.chunk == 0 && it.rt == 0)
-                wait_geq(&a.ctl[kCI_Counters - 1], 1, abort_flag, a, 99);
+                wait_geq(&a.ctl[kCI_Never], 1, abort_flag, a, 99);
             if (!*abort_flag) {
                 fence_proxy_async_global();
                 const uint32_t lbytes = (uint32_t)G * 128, mbytes = (uint32_t)G * kMetaRow;
@@ -978,6 +996,15 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
             if (ctid == 0) S.first_wait_ns = S.total_wait_ns = S.t_loop0 = S.t_loop1 = 0;
             if (it.kind == IT_PREP) {
                 prep_item<XT>(a, it.ex, ctid);
+                if (a.given_ids) {  // no router items: the CTA that finishes the last quantisation builds the plan
+                    named_bar(1, kCT);
+                    if (ctid == 0) {
+                        S.last = atom_add_acq_rel(&a.ctl[kCI_Router], 1) == a.T - 1;
+                        if (S.last) S.staged_kind = -1;  // the B area becomes scratch
+                    }
+                    named_bar(1, kCT);
+                    if (S.last) consumer_plan(a, S, barea, ctid);
+                }
             } else if (it.kind == IT_ROUTER) {
                 if (ctid == 0) S.staged_kind = -1;  // the B area becomes scratch
                 router_item<XT>(a, S, reinterpret_cast<double*>(barea), it.ex, ctid);
@@ -1104,7 +1131,7 @@ cudaError_t launch_decode_i8(const I8Launch& l, cudaStream_t st) {
     if (l.T < 1 || l.T > kI8MaxTok || l.T * l.d.K > kI8MaxSlots) return cudaErrorInvalidValue;
     I8Args a;
     a.weights = l.weights; a.d = l.d; a.wr = l.wr; a.bias = l.bias; a.x = l.x; a.y = l.y; a.residual = l.residual;
-    a.T = l.T; a.p = l.p; a.logits = l.logits; a.xq = l.xq; a.xm = l.xm; a.hq = l.hq; a.hm = l.hm; a.o = l.o;
+    a.T = l.T; a.p = l.p; a.logits = l.logits; a.given_ids = l.given_ids; a.given_w = l.given_w; a.xq = l.xq; a.xm = l.xm; a.hq = l.hq; a.hm = l.hm; a.o = l.o;
     a.ctl = l.ctl; a.trace = l.trace; a.trace_cap = l.trace_cap;
     a.wait_ns = l.wait_ns > 0 ? l.wait_ns : 1000000000ll;
     a.wait_test = l.wait_test;

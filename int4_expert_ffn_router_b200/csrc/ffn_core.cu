@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 2) gateup_core_kernel(const uint8_t*
         const int c = item / RT, rt = item - c * RT;
         const int a = chunk_owner(p.act_chunk, n_active, c);
         const int ex = p.act_expert[a], off = p.act_off[a], cnt = p.act_cnt[a];
-        const uint8_t* tile = weights + (size_t)ex * d.expert_stride + (size_t)rt * G * kBlockBytes;
+        const uint8_t* tile = weights + expert_offset(d, ex) + (size_t)rt * G * kBlockBytes;
         const int j = (rt * 8 + warp) * 8 + gi;  // gate row of this lane's row gi
         const int t0 = (c - p.act_chunk[a]) * kTB;
         {
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 2) down_core_kernel(const uint8_t* _
         const int c = item / RT, rt = item - c * RT;
         const int a = chunk_owner(p.act_chunk, n_active, c);
         const int ex = p.act_expert[a], off = p.act_off[a], cnt = p.act_cnt[a];
-        const uint8_t* tile = weights + (size_t)ex * d.expert_stride + d.gu_bytes + (size_t)rt * G * kBlockBytes;
+        const uint8_t* tile = weights + expert_offset(d, ex) + d.gu_bytes + (size_t)rt * G * kBlockBytes;
         const int r0 = rt * kTileRows + warp * kSubRows + gi;
         const int t0 = (c - p.act_chunk[a]) * kTB;
         {

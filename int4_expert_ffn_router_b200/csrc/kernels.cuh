@@ -57,6 +57,8 @@ struct I8Launch {
     const float* residual;
     Plan p;
     double* logits;
+    const int32_t* given_ids;  // [T][K] ids routed before the launch (then no router items run), or NULL
+    const float* given_w;      // [T][K] their weights
     uint8_t* xq;   // [T][H/64][128] token parts (written by the kernel)
     uint8_t* xm;   // [T][H/64][16]
     uint8_t* hq;   // [slots][I/64][128] SwiGLU output parts

@@ -7,8 +7,10 @@
 #include <cstring>
 #include <new>
 #include <string>
+#include <vector>
 
 #include "common.cuh"
+#include "expert_cache.h"
 #include "kernels.cuh"
 
 #define COLI_API extern "C" __attribute__((visibility("default")))
@@ -40,16 +42,29 @@ size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 // that brings the count to zero fails as if the device were out of memory.
 std::atomic<int> g_fail_alloc{0};
 
-// Every device allocation of a layer goes through here.
-cudaError_t dev_alloc(void** p, size_t bytes) {
+bool planned_failure() {
     int k = g_fail_alloc.load();
     while (k > 0 && !g_fail_alloc.compare_exchange_weak(k, k - 1)) {
     }
-    if (k == 1) {
-        *p = nullptr;
-        return cudaErrorMemoryAllocation;
-    }
+    return k == 1;
+}
+
+// Every device allocation of a layer goes through here.
+cudaError_t dev_alloc(void** p, size_t bytes) {
+    *p = nullptr;
+    if (planned_failure()) return cudaErrorMemoryAllocation;
     return cudaMalloc(p, bytes);
+}
+
+// And every page-locked host allocation (the expert cache's backing store).
+template <typename T>
+cudaError_t host_alloc(T** p, size_t bytes) {
+    *p = nullptr;
+    if (planned_failure()) return cudaErrorMemoryAllocation;
+    void* v = nullptr;
+    cudaError_t e = cudaHostAlloc(&v, bytes, cudaHostAllocDefault);
+    *p = static_cast<T*>(v);
+    return e;
 }
 
 template <typename T>
@@ -142,20 +157,39 @@ struct coli_moe_layer {
     int64_t prof_folded = 0;           // forwards folded into the totals
     double prof_total[COLI_N_STAGES] = {};
     cudaEvent_t ev[kRing][COLI_N_STAGES + 1] = {};
-    unsigned prof_mask[kRing] = {};    // stages marked in each ring slot
+    int prof_seq[kRing][COLI_N_STAGES] = {};  // stages marked in each ring slot, in the order marked
+    int prof_n[kRing] = {};
+    // expert cache (coli_moe_layer_create_cached): `cache.slots` routed experts in HBM
+    // (slots 0..R-1, the shared experts after them), all E in page-locked host memory
+    bool cached = false;
+    ExpertCache cache;
+    uint8_t* host_pool = nullptr;     // [E][expert_stride] device-layout bytes of every routed expert
+    uint8_t* repack_buf = nullptr;    // device: one expert, repacked before it goes to the host pool
+    int32_t* slot_dev = nullptr;      // [E + S] weight slot of each expert, read by the kernels
+    int32_t* slot_pin = nullptr;      // page-locked staging of that table
+    int32_t* ids_pin = nullptr;       // page-locked [max_tokens][K]: the batch's routed ids
+    int32_t* ahead_pin = nullptr;     // page-locked [max_tokens][K]: ids predicted by the previous layer
+    bool table_dirty = false;         // the host table changed since it was last uploaded
+    bool ahead_valid = false;         // ahead_pin holds a prediction for the next forward
+    int ahead_T = 0;
+    bool lookahead = true;            // accept predictions from the previous layer of a stack
+    cudaStream_t copy_stream = nullptr;   // prefetch copies
+    cudaEvent_t ev_table = nullptr;       // last upload of the table finished
+    cudaEvent_t ev_prefetch = nullptr;    // prefetch copies finished
+    cudaEvent_t ev_done = nullptr;        // the last forward's kernels finished reading the slots
+    std::vector<char> prefetched;     // [E] resident because of a prefetch, not yet needed
+    int64_t bytes_h2d = 0, n_prefetched = 0, prefetch_used = 0, predicted = 0, predicted_of = 0;
 };
 
 // Adds the durations of ring slot `r` to the totals (waits for its last
-// event). A stage runs from its mark to the next recorded mark; stages a
-// path does not run are not marked and add nothing.
+// event). A stage runs from its mark to the next mark recorded after it (or
+// the end mark); stages a path does not run are not marked and add nothing.
 static cudaError_t prof_fold(coli_moe_layer* L, int r) {
     cudaError_t e = cudaEventSynchronize(L->ev[r][COLI_N_STAGES]);
     if (e != cudaSuccess) return e;
-    const unsigned mask = L->prof_mask[r] | (1u << COLI_N_STAGES);
-    for (int i = 0; i < COLI_N_STAGES; ++i) {
-        if (!(mask & (1u << i))) continue;
-        int j = i + 1;
-        while (!(mask & (1u << j))) ++j;
+    const int n = L->prof_n[r];
+    for (int k = 0; k < n; ++k) {
+        const int i = L->prof_seq[r][k], j = k + 1 < n ? L->prof_seq[r][k + 1] : COLI_N_STAGES;
         float ms = 0.0f;
         e = cudaEventElapsedTime(&ms, L->ev[r][i], L->ev[r][j]);
         if (e != cudaSuccess) return e;
@@ -166,11 +200,12 @@ static cudaError_t prof_fold(coli_moe_layer* L, int r) {
 }
 
 // Records the boundary before stage `i` of the current forward
-// (i == COLI_N_STAGES: after the last stage).
+// (i == COLI_N_STAGES: after the last stage). Each stage is marked at most
+// once per forward.
 static void prof_mark(coli_moe_layer* L, int i, cudaStream_t s) {
     if (!L->profiling) return;
     cudaEventRecord(L->ev[L->prof_next][i], s);
-    if (i < COLI_N_STAGES) L->prof_mask[L->prof_next] |= 1u << i;
+    if (i < COLI_N_STAGES) L->prof_seq[L->prof_next][L->prof_n[L->prof_next]++] = i;
 }
 
 static coli_status check_cfg(const coli_moe_config* c) {
@@ -193,6 +228,15 @@ static void free_layer(coli_moe_layer* L) {
     if (L->router_b) cudaFree(L->router_b);
     if (L->ws) cudaFree(L->ws);
     if (L->staging) cudaFree(L->staging);
+    if (L->repack_buf) cudaFree(L->repack_buf);
+    if (L->slot_dev) cudaFree(L->slot_dev);
+    if (L->host_pool) cudaFreeHost(L->host_pool);
+    if (L->slot_pin) cudaFreeHost(L->slot_pin);
+    if (L->ids_pin) cudaFreeHost(L->ids_pin);
+    if (L->ahead_pin) cudaFreeHost(L->ahead_pin);
+    if (L->copy_stream) cudaStreamDestroy(L->copy_stream);
+    for (cudaEvent_t e : {L->ev_table, L->ev_prefetch, L->ev_done})
+        if (e) cudaEventDestroy(e);
     for (auto& set : L->ev)
         for (auto& e : set)
             if (e) cudaEventDestroy(e);
@@ -203,6 +247,30 @@ COLI_API coli_status coli_moe_debug_fail_alloc(int nth) {
     if (nth < 0) return fail(COLI_EINVAL, "nth must be >= 0");
     g_fail_alloc.store(nth);
     return COLI_OK;
+}
+
+// Weight slot of expert e (routed 0..E-1, shared E..E+S-1): its id, or in a
+// cached layer its cache slot (-1: not resident) and R + j for shared expert j.
+static int weight_slot(const coli_moe_layer* L, int e) {
+    if (!L->cached) return e;
+    return e < L->d.E ? L->cache.slot(e) : L->cache.slots + (e - L->d.E);
+}
+
+// Uploads a cached layer's slot table on stream s if it changed since the
+// last upload. Experts that are not resident map to slot 0, an in-bounds
+// placeholder: every expert a batch routes to is made resident first. The
+// page-locked staging copy is rewritten only after its previous upload ended.
+static cudaError_t upload_table(coli_moe_layer* L, cudaStream_t s) {
+    if (!L->table_dirty) return cudaSuccess;
+    cudaError_t e = cudaEventSynchronize(L->ev_table);
+    if (e != cudaSuccess) return e;
+    const int E = L->d.E, S = L->d.S;
+    for (int i = 0; i < E; ++i) L->slot_pin[i] = std::max(L->cache.slot(i), 0);
+    for (int j = 0; j < S; ++j) L->slot_pin[E + j] = L->cache.slots + j;
+    e = cudaMemcpyAsync(L->slot_dev, L->slot_pin, (size_t)(E + S) * 4, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    L->table_dirty = false;
+    return cudaEventRecord(L->ev_table, s);
 }
 
 COLI_API int64_t coli_moe_expert_bytes(int hidden, int inter) {
@@ -222,6 +290,7 @@ COLI_API coli_status coli_moe_layer_set_experts(coli_moe_layer* L, int first, in
     const size_t mq = (size_t)I * H / 2, ms = (size_t)I * H / 64;
     // device sources are read in place when 16-byte aligned; anything else goes through the staging buffer
     const bool dev_q = is_device_ptr(q) && ((uintptr_t)q & 15u) == 0, dev_s = is_device_ptr(scales);
+    if (L->cached) CUDA_TRY(cudaDeviceSynchronize(), "wait for expert copies");  // nothing reads the pool meanwhile
     for (int i = 0; i < count; ++i) {
         const uint8_t* eq = q + (size_t)i * nq;
         const uint16_t* es = scales + (size_t)i * ns;
@@ -236,11 +305,22 @@ COLI_API coli_status coli_moe_layer_set_experts(coli_moe_layer* L, int first, in
             eq = L->staging;
             es = reinterpret_cast<const uint16_t*>(L->staging + align256(nq));
         }
-        uint8_t* dst = L->weights + (size_t)(first + i) * L->d.expert_stride;
+        // a cached layer's routed expert is repacked once, then kept in the host pool
+        const int e = first + i;
+        const bool pooled = L->cached && e < L->d.E;
+        uint8_t* dst = pooled ? L->repack_buf : L->weights + (size_t)weight_slot(L, e) * L->d.expert_stride;
         CUDA_TRY(launch_repack(eq, es, eq + mq, es + ms, 2 * I, H, true, dst, 0), "repack gate/up");
         CUDA_TRY(launch_repack(eq + 2 * mq, es + 2 * ms, nullptr, nullptr, H, I, false, dst + L->d.gu_bytes, 0),
                  "repack down");
         CUDA_TRY(launch_l1_bound(eq, es, H, I, L->meta, 0), "weight bounds");
+        if (pooled) {
+            const size_t stride = (size_t)L->d.expert_stride;
+            CUDA_TRY(cudaMemcpy(L->host_pool + (size_t)e * stride, dst, stride, cudaMemcpyDeviceToHost), "expert to host pool");
+            const int sl = L->cache.slot(e);
+            if (sl >= 0)
+                CUDA_TRY(cudaMemcpy(L->weights + (size_t)sl * stride, dst, stride, cudaMemcpyDeviceToDevice),
+                         "expert to its slot");
+        }
         if (!dev_q || !dev_s) CUDA_TRY(cudaDeviceSynchronize(), "repack");  // staging is reused
     }
     CUDA_TRY(cudaDeviceSynchronize(), "repack");
@@ -253,10 +333,10 @@ COLI_API coli_status coli_moe_layer_set_experts(coli_moe_layer* L, int first, in
     return COLI_OK;
 }
 
-COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const float* router_w, const float* router_bias,
-                                           const uint8_t* expert_q, const uint16_t* expert_scales,
-                                           const uint8_t* shared_q, const uint16_t* shared_scales, int device,
-                                           coli_moe_layer** out) {
+// resident < 0: every expert in HBM; otherwise an expert cache of `resident` routed slots.
+static coli_status create_impl(const coli_moe_config* cfg, const float* router_w, const float* router_bias,
+                               const uint8_t* expert_q, const uint16_t* expert_scales, const uint8_t* shared_q,
+                               const uint16_t* shared_scales, int resident, int device, coli_moe_layer** out) {
     if (!out) return fail(COLI_EINVAL, "out is NULL");
     *out = nullptr;
     coli_status st = check_cfg(cfg);
@@ -265,6 +345,12 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     if ((expert_q == nullptr) != (expert_scales == nullptr)) return fail(COLI_EINVAL, "expert_q/expert_scales: both or neither");
     if ((shared_q == nullptr) != (shared_scales == nullptr)) return fail(COLI_EINVAL, "shared_q/shared_scales: both or neither");
     if (cfg->n_shared == 0 && shared_q) return fail(COLI_EINVAL, "shared weights given with n_shared == 0");
+    if (resident >= 0) {
+        const int64_t need = std::min<int64_t>((int64_t)cfg->max_tokens * cfg->top_k, cfg->n_experts);
+        if (resident < need || resident > cfg->n_experts)
+            return fail(COLI_EINVAL, "resident_slots must be in [min(n_experts, max_tokens * top_k), n_experts]");
+        if (!expert_q) return fail(COLI_EINVAL, "a cached layer needs expert_q and expert_scales");
+    }
     int ndev = 0;
     if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
         cudaGetLastError();
@@ -294,7 +380,8 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
         return s;
     };
     cudaError_t e;
-    if ((e = dev_alloc(&L->weights, (size_t)(d.E + d.S) * d.expert_stride)) != cudaSuccess) return bail(e, "cudaMalloc(weights)");
+    const size_t n_slots = (size_t)(resident >= 0 ? resident : d.E) + d.S;
+    if ((e = dev_alloc(&L->weights, n_slots * d.expert_stride)) != cudaSuccess) return bail(e, "cudaMalloc(weights)");
     if ((e = dev_alloc(&L->router_w, (size_t)d.E * d.H * 4)) != cudaSuccess) return bail(e, "cudaMalloc(router)");
     if ((e = dev_alloc(&L->router_b, (size_t)d.E * 4)) != cudaSuccess) return bail(e, "cudaMalloc(bias)");
 
@@ -362,7 +449,26 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     p.n_active = (int32_t*)ptrs[12];
     L->h = (float*)ptrs[13]; L->o = (float*)ptrs[14]; L->xn = (float*)ptrs[15];
     if ((e = cudaMemset(L->ws, 0, total)) != cudaSuccess) return bail(e, "cudaMemset(workspace)");
-    if ((e = cudaMemset(L->weights, 0, (size_t)(d.E + d.S) * d.expert_stride)) != cudaSuccess) return bail(e, "cudaMemset(weights)");
+    if ((e = cudaMemset(L->weights, 0, n_slots * d.expert_stride)) != cudaSuccess) return bail(e, "cudaMemset(weights)");
+    if (resident >= 0) {
+        // the backing store of every routed expert, page-locked, and the slot table
+        L->cached = true;
+        L->cache.init(d.E, resident);
+        L->prefetched.assign(d.E, 0);
+        const size_t TKm = (size_t)Tm * d.K;
+        if ((e = dev_alloc(&L->repack_buf, (size_t)d.expert_stride)) != cudaSuccess) return bail(e, "cudaMalloc(repack)");
+        if ((e = dev_alloc(&L->slot_dev, EA * 4)) != cudaSuccess) return bail(e, "cudaMalloc(slot table)");
+        if ((e = host_alloc(&L->host_pool, (size_t)d.E * d.expert_stride)) != cudaSuccess) return bail(e, "cudaHostAlloc(expert pool)");
+        if ((e = host_alloc(&L->slot_pin, EA * 4)) != cudaSuccess) return bail(e, "cudaHostAlloc(slot table)");
+        if ((e = host_alloc(&L->ids_pin, TKm * 4)) != cudaSuccess) return bail(e, "cudaHostAlloc(ids)");
+        if ((e = host_alloc(&L->ahead_pin, TKm * 4)) != cudaSuccess) return bail(e, "cudaHostAlloc(lookahead ids)");
+        if ((e = cudaStreamCreateWithFlags(&L->copy_stream, cudaStreamNonBlocking)) != cudaSuccess) return bail(e, "copy stream");
+        for (cudaEvent_t* ev : {&L->ev_table, &L->ev_prefetch, &L->ev_done})
+            if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return bail(e, "cudaEventCreate");
+        L->table_dirty = true;
+        if ((e = upload_table(L, nullptr)) != cudaSuccess) return bail(e, "upload slot table");
+        d.slot_of = L->slot_dev;
+    }
 
     if ((e = cudaMemcpy(L->router_w, router_w, (size_t)d.E * d.H * 4, cudaMemcpyDefault)) != cudaSuccess) return bail(e, "copy router");
     if (router_bias) {
@@ -381,6 +487,26 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
     if ((e = cudaDeviceSynchronize()) != cudaSuccess) return bail(e, "create");
     *out = L;
     return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const float* router_w, const float* router_bias,
+                                           const uint8_t* expert_q, const uint16_t* expert_scales,
+                                           const uint8_t* shared_q, const uint16_t* shared_scales, int device,
+                                           coli_moe_layer** out) {
+    return create_impl(cfg, router_w, router_bias, expert_q, expert_scales, shared_q, shared_scales, -1, device, out);
+}
+
+COLI_API coli_status coli_moe_layer_create_cached(const coli_moe_config* cfg, const float* router_w,
+                                                  const float* router_bias, const uint8_t* expert_q,
+                                                  const uint16_t* expert_scales, const uint8_t* shared_q,
+                                                  const uint16_t* shared_scales, int resident_slots, int device,
+                                                  coli_moe_layer** out) {
+    if (resident_slots < 0) {
+        if (out) *out = nullptr;
+        return fail(COLI_EINVAL, "resident_slots must be >= 0");
+    }
+    return create_impl(cfg, router_w, router_bias, expert_q, expert_scales, shared_q, shared_scales, resident_slots,
+                       device, out);
 }
 
 COLI_API void coli_moe_layer_destroy(coli_moe_layer* L) {
@@ -420,14 +546,26 @@ COLI_API coli_status coli_moe_route(coli_moe_layer* L, const void* x, coli_dtype
     return COLI_OK;
 }
 
+// Starts the profile record of a forward (recycles the oldest ring slot).
+static coli_status prof_begin(coli_moe_layer* L) {
+    if (!L->profiling) return COLI_OK;
+    if (L->prof_issued - L->prof_folded >= coli_moe_layer::kRing) CUDA_TRY(prof_fold(L, L->prof_next), "profile");
+    L->prof_n[L->prof_next] = 0;
+    return COLI_OK;
+}
+
 // x: layer input; residual: added to the output (stack) or NULL; y: output.
+// routed: the plan's ids and weights already hold this batch's routing (and
+// the caller began the profile record), so the router and top-k do not run.
 static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_dtype dt, int T, const float* residual,
-                                cudaStream_t s) {
+                                cudaStream_t s, bool routed = false) {
     const Dims& d = L->d;
     const Plan& p = L->plan;
-    if (L->profiling && L->prof_issued - L->prof_folded >= coli_moe_layer::kRing)
-        CUDA_TRY(prof_fold(L, L->prof_next), "profile");  // recycle the oldest slot
-    if (L->profiling) L->prof_mask[L->prof_next] = 0;
+    if (!routed) {
+        coli_status st = prof_begin(L);
+        if (st != COLI_OK) return st;
+    }
+    const int router_launches = routed ? 0 : router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
     if (L->fused == 1 && T <= L->i8_max_tok && decode_i8_supported(d, T, L->smem_optin)) {
         prof_mark(L, COLI_STAGE_FUSED, s);
         I8Launch l{};
@@ -436,15 +574,18 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         l.hm = L->hm; l.o = L->o; l.ctl = L->ctl; l.n_sm = L->n_sm; l.smem_limit = L->smem_optin; l.trace = L->trace;
         l.trace_cap = L->trace_cap; l.max_stages = L->ring_stages; l.max_sb = L->ring_blocks;
         l.wait_ns = L->wait_ns; l.wait_test = L->wait_test;
+        if (routed) { l.given_ids = p.ids; l.given_w = p.w; }
         CUDA_TRY(launch_decode_i8(l, s), "persistent decode kernel (integer MMA)");
         L->launches += 1;
     } else if ((L->tc_mode == 2 || (L->tc_mode == 1 && dt == COLI_BF16)) && L->tc_shape_ok && L->tc_scale_ok) {
         // tensor cores; fp32 tokens as fp16 hi + lo operand rows (tiles of kTcMaxTok / 2 tokens)
         const bool pairs = dt == COLI_F32;
-        prof_mark(L, COLI_STAGE_ROUTER, s);
-        CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
-        prof_mark(L, COLI_STAGE_TOPK, s);
-        CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+        if (!routed) {
+            prof_mark(L, COLI_STAGE_ROUTER, s);
+            CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
+            prof_mark(L, COLI_STAGE_TOPK, s);
+            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+        }
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
         // the plan stage also covers the operand rows, the tile list and the output clear,
@@ -471,12 +612,14 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_prefill_out(L->o, residual, T, d.H, y, dt, s), "output");
         // router, top-k, plan, prep, tile plan, two grouped GEMMs, output (the clear is a driver memset)
-        L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 7;
+        L->launches += router_launches + 6;
     } else {
-        prof_mark(L, COLI_STAGE_ROUTER, s);
-        CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
-        prof_mark(L, COLI_STAGE_TOPK, s);
-        CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+        if (!routed) {
+            prof_mark(L, COLI_STAGE_ROUTER, s);
+            CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
+            prof_mark(L, COLI_STAGE_TOPK, s);
+            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+        }
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
         prof_mark(L, COLI_STAGE_GATEUP, s);
@@ -485,7 +628,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         CUDA_TRY(launch_down_core(L->weights, d, L->h, T, p, L->o, L->max_active, L->n_sm, s), "down");
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_combine(L->o, p, T, d.H, d.K, d.S, residual, y, dt, s), "combine");
-        L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 5;
+        L->launches += router_launches + 4;
     }
     prof_mark(L, COLI_N_STAGES, s);
     if (L->profiling) {
@@ -494,6 +637,135 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
     }
     L->last_T = T;
     L->last_stream = s;
+    return COLI_OK;
+}
+
+// ---------------------------------------------------------------- expert cache
+
+// Issues one host-to-HBM copy per (expert, slot) pair on stream s: an
+// expert's gate/up and down matrices are adjacent, so each is one copy.
+static cudaError_t copy_experts(coli_moe_layer* L, const std::vector<std::pair<int, int>>& copies, cudaStream_t s) {
+    const size_t stride = (size_t)L->d.expert_stride, bytes = (size_t)(L->d.gu_bytes + L->d.d_bytes);
+    for (const auto& c : copies) {
+        cudaError_t e = cudaMemcpyAsync(L->weights + (size_t)c.second * stride, L->host_pool + (size_t)c.first * stride,
+                                        bytes, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return e;
+        L->bytes_h2d += (int64_t)bytes;
+    }
+    if (!copies.empty()) L->table_dirty = true;
+    return cudaSuccess;
+}
+
+// Distinct ids among ids[0..n), in first-appearance order; false if one is
+// outside [0, E).
+static bool distinct_ids(const int32_t* ids, int n, int E, std::vector<int32_t>* out) {
+    std::vector<char> seen(E, 0);
+    out->clear();
+    for (int i = 0; i < n; ++i) {
+        const int e = ids[i];
+        if (e < 0 || e >= E) return false;
+        if (!seen[e]) {
+            seen[e] = 1;
+            out->push_back(e);
+        }
+    }
+    return true;
+}
+
+// Best-effort prefetch of the distinct experts among ids[0..n) on the copy
+// stream, after the layer's last forward has finished reading its slots.
+static coli_status cache_prefetch(coli_moe_layer* L, const int32_t* ids, int n) {
+    std::vector<int32_t> ex;
+    if (!distinct_ids(ids, n, L->d.E, &ex)) return fail(COLI_EINVAL, "expert id out of range");
+    std::vector<std::pair<int, int>> copies;
+    L->cache.prefetch(ex.data(), (int)ex.size(), &copies);
+    for (int e = 0; e < L->d.E; ++e)
+        if (L->prefetched[e] && L->cache.slot(e) < 0) L->prefetched[e] = 0;  // evicted before use
+    if (copies.empty()) return COLI_OK;
+    CUDA_TRY(cudaStreamWaitEvent(L->copy_stream, L->ev_done, 0), "prefetch: wait for the last forward");
+    CUDA_TRY(copy_experts(L, copies, L->copy_stream), "prefetch copy");
+    CUDA_TRY(cudaEventRecord(L->ev_prefetch, L->copy_stream), "record prefetch");
+    for (const auto& c : copies) L->prefetched[c.first] = 1;
+    L->n_prefetched += (int64_t)copies.size();
+    return COLI_OK;
+}
+
+// Makes every routed expert of the batch whose ids are in ids_pin resident:
+// misses are copied on stream s after any pending prefetch, then the table.
+static coli_status cache_admit(coli_moe_layer* L, int T, cudaStream_t s) {
+    const int E = L->d.E, TK = T * L->d.K;
+    std::vector<int32_t> ex;
+    if (!distinct_ids(L->ids_pin, TK, E, &ex)) return fail(COLI_ECUDA, "routed expert id out of range");
+    if (L->ahead_valid) {  // how many of the needed experts the previous layer predicted
+        std::vector<char> pred(E, 0);
+        for (int i = 0; i < L->ahead_T * L->d.K; ++i) {
+            const int e = L->ahead_pin[i];
+            if (e >= 0 && e < E) pred[e] = 1;
+        }
+        for (int e : ex) L->predicted += pred[e];
+        L->predicted_of += (int64_t)ex.size();
+        L->ahead_valid = false;
+    }
+    for (int e : ex)
+        if (L->prefetched[e] && L->cache.slot(e) >= 0) {
+            L->prefetch_used += 1;
+            L->prefetched[e] = 0;
+        }
+    std::vector<std::pair<int, int>> copies;
+    if (!L->cache.admit(ex.data(), (int)ex.size(), &copies))
+        return fail(COLI_EUNSUPPORTED, "too many pinned experts for this batch");
+    for (int e = 0; e < E; ++e)
+        if (L->prefetched[e] && L->cache.slot(e) < 0) L->prefetched[e] = 0;
+    CUDA_TRY(cudaStreamWaitEvent(s, L->ev_prefetch, 0), "wait for prefetch copies");
+    CUDA_TRY(copy_experts(L, copies, s), "copy missing experts");
+    CUDA_TRY(upload_table(L, s), "upload slot table");
+    return COLI_OK;
+}
+
+// Forward of a cached layer: route, read the ids back (waits for them), make
+// the batch's experts resident, then the resident layer's kernels with the
+// given routing. `next`: the following layer of a stack or NULL; when it is a
+// cached layer accepting predictions, its router also runs on this layer's
+// input, and the experts it picks are prefetched into it while this layer's
+// kernels run.
+static coli_status cached_forward(coli_moe_layer* L, const void* x, void* y, coli_dtype dt, int T,
+                                  const float* residual, cudaStream_t s, coli_moe_layer* next) {
+    const Dims& d = L->d;
+    const Plan& p = L->plan;
+    coli_status st = prof_begin(L);
+    if (st != COLI_OK) return st;
+    prof_mark(L, COLI_STAGE_ROUTER, s);
+    CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap),
+             "router");
+    prof_mark(L, COLI_STAGE_TOPK, s);
+    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+    L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
+    prof_mark(L, COLI_STAGE_CACHE, s);
+    const bool ahead = next && next != L && next->cached && next->lookahead && T <= next->cfg.max_tokens &&
+                       next->d.H == d.H && next->device == L->device;
+    if (ahead) {
+        const Dims& dn = next->d;
+        CUDA_TRY(launch_router_logits(next->router_w, next->router_b, x, dt, T, dn.H, dn.E, next->logits, s,
+                                      next->rpart, next->rpart_cap),
+                 "lookahead router");
+        CUDA_TRY(launch_topk(next->logits, T, dn.E, dn.K, next->plan.ids, next->plan.w, s), "lookahead topk");
+        next->launches += router_kernel_count(T, dn.H, dn.E, next->rpart, next->rpart_cap) + 1;
+        CUDA_TRY(cudaMemcpyAsync(next->ahead_pin, next->plan.ids, (size_t)T * dn.K * 4, cudaMemcpyDeviceToHost, s),
+                 "read predicted ids");
+    }
+    CUDA_TRY(cudaMemcpyAsync(L->ids_pin, p.ids, (size_t)T * d.K * 4, cudaMemcpyDeviceToHost, s), "read routed ids");
+    CUDA_TRY(cudaStreamSynchronize(s), "wait for routed ids");
+    st = cache_admit(L, T, s);
+    if (st != COLI_OK) return st;
+    st = forward_impl(L, x, y, dt, T, residual, s, true);
+    if (st != COLI_OK) return st;
+    CUDA_TRY(cudaEventRecord(L->ev_done, s), "record forward");
+    if (ahead) {
+        next->ahead_valid = true;
+        next->ahead_T = T;
+        st = cache_prefetch(next, next->ahead_pin, T * next->d.K);
+        if (st != COLI_OK) return st;
+    }
     return COLI_OK;
 }
 
@@ -510,6 +782,7 @@ COLI_API coli_status coli_moe_forward(coli_moe_layer* L, const void* x, void* y,
     }
     if (T == 0) return COLI_OK;
     DeviceGuard guard(L->device);
+    if (L->cached) return cached_forward(L, x, y, dt, T, nullptr, (cudaStream_t)stream, nullptr);
     return forward_impl(L, x, y, dt, T, nullptr, (cudaStream_t)stream);
 }
 
@@ -531,7 +804,8 @@ COLI_API coli_status coli_moe_stack_forward(coli_moe_layer* const* layers, int n
         coli_moe_layer* L = layers[l];
         CUDA_TRY(launch_rmsnorm(x, T, L->d.H, eps, L->xn, s), "rmsnorm");
         L->launches += 1;
-        coli_status st = forward_impl(L, L->xn, x, COLI_F32, T, x, s);
+        coli_status st = L->cached ? cached_forward(L, L->xn, x, COLI_F32, T, x, s, l + 1 < n_layers ? layers[l + 1] : nullptr)
+                                   : forward_impl(L, L->xn, x, COLI_F32, T, x, s);
         if (st != COLI_OK) return st;
     }
     return COLI_OK;
@@ -684,8 +958,75 @@ COLI_API coli_status coli_moe_get_profile(coli_moe_layer* L, double* stage_ms_to
 }
 
 COLI_API const char* coli_moe_stage_name(int stage) {
-    static const char* names[COLI_N_STAGES] = {"router", "topk", "plan", "gateup", "down", "combine", "fused"};
+    static const char* names[COLI_N_STAGES] = {"router", "topk", "plan", "gateup", "down", "combine", "fused", "cache"};
     return (stage >= 0 && stage < COLI_N_STAGES) ? names[stage] : "";
+}
+
+COLI_API coli_status coli_moe_cache_stats(coli_moe_layer* L, coli_cache_stats* stats, int64_t* usage, int reset) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (!L->cached) return fail(COLI_EINVAL, "not a cached layer");
+    DeviceGuard guard(L->device);
+    CUDA_TRY(cudaStreamSynchronize(L->copy_stream), "wait for prefetch copies");
+    if (stats) {
+        stats->hits = L->cache.hits;
+        stats->misses = L->cache.misses;
+        stats->bytes_h2d = L->bytes_h2d;
+        stats->prefetched = L->n_prefetched;
+        stats->prefetch_used = L->prefetch_used;
+        stats->predicted = L->predicted;
+        stats->predicted_of = L->predicted_of;
+        stats->resident_slots = L->cache.slots;
+        int np = 0;
+        for (int e = 0; e < L->d.E; ++e) np += L->cache.is_pinned(e);
+        stats->n_pinned = np;
+    }
+    if (usage)
+        for (int e = 0; e < L->d.E; ++e) usage[e] = L->cache.uses[e];
+    if (reset) {
+        L->cache.hits = L->cache.misses = 0;
+        L->bytes_h2d = L->n_prefetched = L->prefetch_used = L->predicted = L->predicted_of = 0;
+    }
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_cache_pin(coli_moe_layer* L, const int32_t* ids, int n) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (!L->cached) return fail(COLI_EINVAL, "not a cached layer");
+    if (n < 0 || (n > 0 && !ids)) return fail(COLI_EINVAL, "bad id list");
+    const int reserve = (int)std::min<int64_t>((int64_t)L->cfg.max_tokens * L->d.K, L->d.E);
+    if (!L->cache.pin(ids, n, reserve))
+        return fail(COLI_EINVAL, "ids out of range, or more than resident_slots - min(n_experts, max_tokens * top_k)");
+    DeviceGuard guard(L->device);
+    coli_status st = cache_prefetch(L, ids, n);  // pinned experts are never the victims, so all of them fit
+    if (st != COLI_OK) return st;
+    CUDA_TRY(cudaStreamSynchronize(L->copy_stream), "pin copies");
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_cache_prefetch(coli_moe_layer* L, const int32_t* ids, int n) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (!L->cached) return fail(COLI_EINVAL, "not a cached layer");
+    if (n < 0 || (n > 0 && !ids)) return fail(COLI_EINVAL, "bad id list");
+    for (int i = 0; i < n; ++i)
+        if (ids[i] < 0 || ids[i] >= L->d.E) return fail(COLI_EINVAL, "expert id out of range");
+    DeviceGuard guard(L->device);
+    return cache_prefetch(L, ids, n);
+}
+
+COLI_API coli_status coli_moe_cache_slots(const coli_moe_layer* L, int32_t* slots) {
+    if (!L || !slots) return fail(COLI_EINVAL, "NULL argument");
+    if (!L->cached) return fail(COLI_EINVAL, "not a cached layer");
+    for (int e = 0; e < L->d.E; ++e) slots[e] = L->cache.slot(e);
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_cache_set_lookahead(coli_moe_layer* L, int enable) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (!L->cached) return fail(COLI_EINVAL, "not a cached layer");
+    if (enable < 0 || enable > 1) return fail(COLI_EINVAL, "enable must be 0 or 1");
+    L->lookahead = enable != 0;
+    if (!L->lookahead) L->ahead_valid = false;
+    return COLI_OK;
 }
 
 COLI_API const char* coli_status_string(coli_status s) {

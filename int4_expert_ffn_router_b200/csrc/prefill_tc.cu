@@ -87,6 +87,7 @@ struct __align__(64) TcArgs {
     CUtensorMap tmap_small; // the same with box 64 x kSmallBox rows (tiles of up to kSmallBox tokens)
     const uint8_t* weights;
     int64_t expert_stride;
+    const int32_t* slot_of;   // expert -> weight slot (expert cache) or NULL
     int64_t mat_offset;     // 0 (gate/up) or the down matrix offset within an expert
     int KB;                 // 64-input blocks per row (H/64 or I/64)
     int RT2;                // pairs of 128-row tiles
@@ -354,7 +355,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
             const bool small = rows <= kSmallBox;
             const void* map = small ? (const void*)&a.tmap_small : (const void*)&a.tmap_big;
             const uint32_t tx_bytes = 2 * kBlockBytes + (small ? kSmallBox : kTcMaxTok) * 128;
-            const uint8_t* w0 = a.weights + (size_t)tile.x * a.expert_stride + a.mat_offset +
+            const size_t eslot = a.slot_of ? (size_t)__ldg(a.slot_of + tile.x) : (size_t)tile.x;
+            const uint8_t* w0 = a.weights + eslot * a.expert_stride + a.mat_offset +
                                 (size_t)(2 * pair) * KB * kBlockBytes;
             const uint8_t* w1 = w0 + (size_t)KB * kBlockBytes;
             for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -709,6 +711,7 @@ cudaError_t launch_prefill_gemm(int phase, bool pairs, const uint8_t* weights, c
     a.trace_cap = trace_cap;
     a.weights = weights;
     a.expert_stride = d.expert_stride;
+    a.slot_of = d.slot_of;
     a.mat_offset = phase == 0 ? 0 : d.gu_bytes;
     a.KB = phase == 0 ? d.H / kGroup : d.I / kGroup;
     a.RT2 = phase == 0 ? (2 * d.I / kTileRows) / 2 : (d.H / kTileRows) / 2;

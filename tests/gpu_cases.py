@@ -9,8 +9,9 @@ import synth
 import int4_expert_ffn_router_b200 as coli
 
 
-def device_layer(c, seed=0, layer=0, bias=None, max_tokens=64, device=0):
-    """Create a layer whose canonical weights are generated on the device.
+def device_layer(c, seed=0, layer=0, bias=None, max_tokens=64, device=0, resident=None):
+    """Create a layer whose canonical weights are generated on the device
+    (``resident``: routed-expert slots of an expert cache, None: all in HBM).
 
     Peak device memory: the canonical buffers (E+S experts) plus the layer."""
     H, I, E, S = c["H"], c["I"], c["E"], c["S"]
@@ -26,7 +27,7 @@ def device_layer(c, seed=0, layer=0, bias=None, max_tokens=64, device=0):
     torch.cuda.synchronize(dev)
     cfg = coli.make_config(H, I, E, c["K"], S, max_tokens)
     L = coli.Layer(cfg, wr, b, q[:E * nq], s[:E * ns], q[E * nq:] if S else None, s[E * ns:] if S else None,
-                   device=device)
+                   device=device, resident=resident)
     del q, s
     torch.cuda.empty_cache()
     return L

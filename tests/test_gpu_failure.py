@@ -1,7 +1,8 @@
 """Failure handling on the GPU, without making the GPU fault or hang.
 
 Out of memory is made on the host: coli_moe_debug_fail_alloc makes the nth
-device allocation of layer creation fail as if the device were full. Each
+device (or page-locked host) allocation of layer creation fail as if the
+memory were full. Each
 failing create must return COLI_ENOMEM, leave nothing allocated (the
 device's free memory is the same before and after) and leave the library
 usable.
@@ -28,20 +29,23 @@ def _host_args(coli, c, max_tokens=8):
     return L, (cfg, L["wr"], None, q[:E * nq], s[:E * ns], q[E * nq:], s[E * ns:])
 
 
-def test_create_out_of_memory_at_each_allocation(gpu):
+@pytest.mark.parametrize("resident", [None, 6])
+def test_create_out_of_memory_at_each_allocation(gpu, resident):
+    """resident=6: an expert cache of 6 slots, whose create also allocates
+    page-locked host memory (those allocations fail the same way)."""
     import int4_expert_ffn_router_b200 as coli
 
     c = cases.TINY
-    L, args = _host_args(coli, c)
-    coli.Layer(*args, device=0).close()  # module loading and the context are not counted below
+    L, args = _host_args(coli, c, max_tokens=2)
+    coli.Layer(*args, device=0, resident=resident).close()  # module loading and the context are not counted below
     torch.cuda.synchronize()
     free0 = torch.cuda.mem_get_info()[0]
     failed = 0
     try:
-        for nth in range(1, 9):
+        for nth in range(1, 16):
             coli.debug_fail_alloc(nth)
             try:
-                layer = coli.Layer(*args, device=0)
+                layer = coli.Layer(*args, device=0, resident=resident)
             except coli.ColiError as e:
                 assert e.status == coli.COLI_ENOMEM, str(e)
                 failed += 1
@@ -51,11 +55,13 @@ def test_create_out_of_memory_at_each_allocation(gpu):
             break
     finally:
         coli.debug_fail_alloc(0)
-    # weights, router, bias, workspace and the staging buffer of host sources
-    assert failed == 5
+    # weights, router, bias, workspace and the staging buffer of host sources;
+    # a cache adds the repack buffer, the slot table, and four page-locked
+    # buffers: expert pool, table staging, routed ids, predicted ids
+    assert failed == (5 if resident is None else 11)
     assert torch.cuda.mem_get_info()[0] == free0
     # the library still works: a forward through a fresh layer matches the oracle
-    layer = coli.Layer(*args, device=0)
+    layer = coli.Layer(*args, device=0, resident=resident)
     x = synth.x_f32(c["seed"], 3, 2, c["H"])
     xd = torch.from_numpy(x).to(gpu)
     yd = torch.empty_like(xd)
