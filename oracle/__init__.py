@@ -19,7 +19,7 @@ F32, BF16 = 0, 1
 
 class Cfg(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("inter", ctypes.c_int), ("n_experts", ctypes.c_int),
-                ("top_k", ctypes.c_int), ("n_shared", ctypes.c_int)]
+                ("top_k", ctypes.c_int), ("n_shared", ctypes.c_int), ("expert_top_p", ctypes.c_double)]
 
 
 def build(verbose: bool = False) -> None:
@@ -51,6 +51,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_topk.argtypes = [vp, i32, i32, i32, vp, vp]
         L.oracle_topk.restype = i32
         L.oracle_weights_full_softmax.argtypes = [vp, i32, i32, i32, vp, vp]
+        L.oracle_expert_topp.argtypes = [i32, i32, f64, vp, vp]
+        L.oracle_expert_topp.restype = i32
         L.oracle_union.argtypes = [vp, i32, i32, i32, vp, vp, vp, vp, vp, vp]
         L.oracle_union.restype = i32
         L.oracle_expert_ffn.argtypes = [vp, vp, i32, i32, vp, vp, vp]
@@ -112,14 +114,25 @@ def router_logits(wr, bias, x):
     return out
 
 
-def topk(logits, K):
+def topk(logits, K, top_p=None):
+    """ids [T][K], weights [T][K]; with top_p in (0, 1) the adaptive expert
+    top-p reduction follows (dropped slots: id -1, weight 0)."""
     logits = np.ascontiguousarray(logits, np.float64)
     T, E = logits.shape
     ids = np.empty((T, K), np.int32)
     w = np.empty((T, K), np.float64)
     if lib().oracle_topk(_p(logits), T, E, K, _p(ids), _p(w)):
         raise ValueError("oracle_topk: bad arguments or NaN logit")
+    if top_p is not None and 0.0 < top_p < 1.0:
+        lib().oracle_expert_topp(T, K, top_p, _p(ids), _p(w))
     return ids, w
+
+
+def expert_topp(ids, w, p):
+    """In-place adaptive expert top-p on a top-K result; returns slots kept."""
+    assert ids.dtype == np.int32 and w.dtype == np.float64 and ids.flags["C_CONTIGUOUS"] and w.flags["C_CONTIGUOUS"]
+    T, K = ids.shape
+    return lib().oracle_expert_topp(T, K, p, _p(ids), _p(w))
 
 
 def weights_full_softmax(logits, ids):

@@ -118,6 +118,39 @@ ORACLE_API int oracle_topk(const double* logits, int T, int E, int K, int32_t* i
     return bad ? -1 : 0;
 }
 
+/* Adaptive expert top-p ("colibri: 1300 lines of C ..." (jsqmd.com), usage
+ * section: topp=0.7, adaptive expert top-p, fewer expert reads per token):
+ * per token, the experts of the top-K in selection order are kept until
+ * their weights (the router probabilities renormalised over the K) sum to at
+ * least p; the kept weights are renormalised to sum to 1. */
+ORACLE_API int oracle_expert_topp(int T, int K, double p, int32_t* ids, double* w)
+{
+    int kept_total = 0;
+    for (int t = 0; t < T; ++t) {
+        int32_t* it = ids + (size_t)t * K;
+        double* wt = w + (size_t)t * K;
+        int keep = K;
+        double cum = 0.0;
+        for (int k = 0; k < K; ++k) {
+            cum += wt[k];
+            if (p < 1.0 && cum >= p) {
+                keep = k + 1;
+                break;
+            }
+        }
+        for (int k = 0; k < K; ++k) {
+            if (k < keep) {
+                wt[k] = wt[k] / cum;
+            } else {
+                wt[k] = 0.0;
+                it[k] = -1;
+            }
+        }
+        kept_total += keep;
+    }
+    return kept_total;
+}
+
 ORACLE_API void oracle_weights_full_softmax(const double* logits, int T, int E, int K, const int32_t* ids, double* w)
 {
     for (int t = 0; t < T; ++t) {
@@ -230,8 +263,9 @@ static int forward_impl(const oracle_cfg* cfg, const float* wr, const float* bia
     if (!logits || !ids || !w || !xt || !o) { rc = -1; goto done; }
     oracle_router_logits(wr, bias, x, xdtype, T, H, E, logits);
     if (oracle_topk(logits, T, E, K, ids, w)) { rc = -1; goto done; }
+    if (cfg->expert_top_p > 0.0 && cfg->expert_top_p < 1.0) oracle_expert_topp(T, K, cfg->expert_top_p, ids, w);
     for (int i = 0; i < T * K; ++i)
-        if (!eq[ids[i]] || !es[ids[i]]) { rc = -2; goto done; }
+        if (ids[i] >= 0 && (!eq[ids[i]] || !es[ids[i]])) { rc = -2; goto done; }
     for (int t = 0; t < T; ++t) {
         double* yt = y + (size_t)t * H;
         for (int h = 0; h < H; ++h) { xt[h] = load_x(x, xdtype, (size_t)t * H + h); yt[h] = 0.0; }
@@ -242,6 +276,7 @@ static int forward_impl(const oracle_cfg* cfg, const float* wr, const float* bia
         if (!dense) {
             for (int k = 0; k < K; ++k) {
                 int e = ids[(size_t)t * K + k];
+                if (e < 0) continue; /* dropped by expert top-p */
                 oracle_expert_ffn(eq[e], es[e], H, I, xt, o, NULL);
                 for (int h = 0; h < H; ++h) yt[h] += w[(size_t)t * K + k] * o[h];
             }

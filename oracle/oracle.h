@@ -42,6 +42,7 @@ typedef struct {
     int n_experts;  /* E, routed */
     int top_k;      /* K */
     int n_shared;   /* shared experts, weight 1 each */
+    double expert_top_p; /* adaptive expert top-p (oracle_expert_topp); 0 or >= 1: off */
 } oracle_cfg;
 
 enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
@@ -60,6 +61,12 @@ void oracle_router_logits(const float* wr, const float* bias, const void* x, int
 /* K largest logits per token, descending, ties to the lower id; weights are the
  * softmax over the selected logits. Returns 0, or -1 on bad sizes. */
 int oracle_topk(const double* logits, int T, int E, int K, int32_t* ids, double* w);
+/* Adaptive expert top-p on a top-K result (ids and weights [T][K] in
+ * selection order, weights summing to 1 per token): keep the shortest prefix
+ * whose weights sum (in order, fp64) to at least p, renormalise the kept
+ * weights by that sum, and mark the dropped slots id -1, weight 0. At least
+ * one expert is kept; p >= 1 keeps all K. Returns the number of slots kept. */
+int oracle_expert_topp(int T, int K, double p, int32_t* ids, double* w);
 /* Second form of the weights: softmax over all E logits, renormalised over the
  * selected ids (self-check of oracle_topk's weights). */
 void oracle_weights_full_softmax(const double* logits, int T, int E, int K, const int32_t* ids, double* w);
@@ -78,7 +85,8 @@ void oracle_expert_ffn(const uint8_t* q, const uint16_t* s, int H, int I, const 
                        double* out, double* h_out);
 
 /* The layer: y[t] = sum_j shared_j(x_t) + sum_k w[t][k] * E_ids[t][k](x_t),
- * the routed sum taken in routing order. eq/es hold E + n_shared expert pointers
+ * the routed sum taken in routing order; with cfg->expert_top_p in (0, 1) the
+ * routing is reduced by oracle_expert_topp first (dropped slots: id -1). eq/es hold E + n_shared expert pointers
  * (routed 0..E-1, then shared); a routed entry may be NULL if never selected.
  * ids/w may be NULL. Returns 0, -1 on bad arguments, -2 if a selected expert is NULL. */
 int oracle_moe_forward(const oracle_cfg* cfg, const float* wr, const float* bias,

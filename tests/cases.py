@@ -18,9 +18,10 @@ TINY = dict(H=512, I=256, E=16, K=2, S=1, T=4, seed=0)
 FULL = dict(H=6144, I=2048, E=256, K=8, S=1)
 
 
-def oracle_cfg(c):
+def oracle_cfg(c, top_p=0.0):
     import oracle
-    return oracle.Cfg(hidden=c["H"], inter=c["I"], n_experts=c["E"], top_k=c["K"], n_shared=c["S"])
+    return oracle.Cfg(hidden=c["H"], inter=c["I"], n_experts=c["E"], top_k=c["K"], n_shared=c["S"],
+                      expert_top_p=top_p)
 
 
 def host_layer(c, seed=0, layer=0, which=None, bias=None):

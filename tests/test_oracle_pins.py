@@ -130,6 +130,74 @@ def test_topk_weights_closed_form_and_full_softmax_form():
     np.testing.assert_allclose(oracle.weights_full_softmax(lg, ids), w, rtol=0, atol=1e-15)
 
 
+@pytest.mark.parametrize("p,ids_ref,w_ref", [
+    (0.65, [3, 2, -1, -1], [4 / 7, 3 / 7, 0, 0]),   # 0.4 < 0.65 <= 0.7
+    (0.75, [3, 2, 1, -1], [4 / 9, 3 / 9, 2 / 9, 0]),  # 0.7 < 0.75 <= 0.9
+    (0.3, [3, -1, -1, -1], [1, 0, 0, 0]),            # the first expert alone reaches p
+    (0.95, [3, 2, 1, 0], [0.4, 0.3, 0.2, 0.1]),      # all four needed
+    (1.0, [3, 2, 1, 0], [0.4, 0.3, 0.2, 0.1]),       # p = 1: plain top-K
+])
+def test_expert_top_p_closed_forms(p, ids_ref, w_ref):
+    """Adaptive expert top-p on logits ln 1..ln 4 (K = 4, weights 0.4, 0.3,
+    0.2, 0.1): keep the shortest prefix whose weights reach p, renormalise."""
+    logits = np.log(np.array([[1.0, 2.0, 3.0, 4.0]]))
+    ids, w = oracle.topk(logits, 4, top_p=p)
+    assert ids[0].tolist() == ids_ref
+    np.testing.assert_allclose(w[0], w_ref, rtol=0, atol=1e-15)
+
+
+def test_expert_top_p_invariants_on_random_routers():
+    """Kept counts grow with p, kept weights sum to 1, the kept ids are the
+    plain top-K's prefix, and the mass the kept experts carried before the
+    renormalisation reaches p while the prefix one shorter does not."""
+    rng = np.random.default_rng(11)
+    lg = rng.standard_normal((200, 64)) * 2
+    ids0, w0 = oracle.topk(lg, 8)
+    prev = None
+    for p in (0.2, 0.5, 0.7, 0.9, 0.99):
+        ids, w = oracle.topk(lg, 8, top_p=p)
+        keep = (ids >= 0).sum(axis=1)
+        assert keep.min() >= 1
+        if prev is not None:
+            assert (keep >= prev).all()
+        prev = keep
+        for t in range(200):
+            n = keep[t]
+            assert ids[t, :n].tolist() == ids0[t, :n].tolist() and (ids[t, n:] == -1).all()
+            np.testing.assert_allclose(w[t, :n].sum(), 1.0, rtol=0, atol=1e-14)
+            assert (w[t, n:] == 0).all()
+            assert w0[t, :n].sum() >= p - 1e-15
+            assert n == 1 or w0[t, :n - 1].sum() < p + 1e-15
+            np.testing.assert_allclose(w[t, :n], w0[t, :n] / w0[t, :n].sum(), rtol=1e-15, atol=0)
+
+
+def test_expert_top_p_layer_reductions(tiny):
+    """A layer with top-K and p below every token's top weight is the top-1
+    layer (one expert at weight 1); p = 1 is the plain layer; in between the
+    output equals the layer rebuilt from single-expert calls over the kept
+    experts with the renormalised weights."""
+    c, L, x = tiny
+    cK = dict(c, K=4)
+    y1, ids1, _ = oracle.moe_forward(cases.oracle_cfg(dict(c, K=1)), L["wr"], None, L["experts"], x)
+    yp, idsp, wp = oracle.moe_forward(cases.oracle_cfg(cK, top_p=1e-9), L["wr"], None, L["experts"], x)
+    assert (idsp[:, 1:] == -1).all() and (idsp[:, 0] == ids1[:, 0]).all() and (wp[:, 0] == 1.0).all()
+    np.testing.assert_array_equal(yp, y1)
+    yK, idsK, _ = oracle.moe_forward(cases.oracle_cfg(cK), L["wr"], None, L["experts"], x)
+    y_one, ids_one, _ = oracle.moe_forward(cases.oracle_cfg(cK, top_p=1.0), L["wr"], None, L["experts"], x)
+    np.testing.assert_array_equal(yK, y_one)
+    y7, ids7, w7 = oracle.moe_forward(cases.oracle_cfg(cK, top_p=0.7), L["wr"], None, L["experts"], x)
+    logits = oracle.router_logits(L["wr"], None, x)
+    ids_k, w_k = oracle.topk(logits, 4)
+    assert (ids7 >= 0).sum() < ids7.size            # something was dropped
+    for t in range(c["T"]):
+        xt = x[t].astype(np.float64)
+        n = int((ids7[t] >= 0).sum())
+        ref = oracle.expert_ffn(*L["experts"][c["E"]], c["H"], c["I"], xt)
+        for k in range(n):
+            ref = ref + (w_k[t, k] / w_k[t, :n].sum()) * oracle.expert_ffn(*L["experts"][ids_k[t, k]], c["H"], c["I"], xt)
+        np.testing.assert_allclose(y7[t], ref, rtol=0, atol=1e-13 * np.abs(ref).max())
+
+
 def test_topk_rejects_nan():
     with pytest.raises(ValueError):
         oracle.topk(np.array([[0.0, np.nan, 1.0]]), 2)
