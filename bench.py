@@ -77,6 +77,12 @@ WORKLOADS = {
                                   "Zipf(1.1) per layer"),
 }
 X_SEED0 = 1000  # step s draws its activations with seed X_SEED0 + s
+TOPP = 1.0      # --expert-top-p: adaptive expert top-p of every layer (1: plain top-K)
+
+
+def topp_arg():
+    """The oracle's top_p argument for TOPP (None: plain top-K)."""
+    return TOPP if TOPP < 1.0 else None
 LEARN_SEED0 = 500_000  # the cache workloads' learning pass draws its own tokens
 FUSED_MODE = {"i8": 1, "separate": 0}
 
@@ -195,6 +201,8 @@ def parse():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b1")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--expert-top-p", type=float, default=1.0,
+                    help="adaptive expert top-p of every layer, in (0, 1] (opt-in routing variant; 1: plain top-8)")
     ap.add_argument("--decode-kernel", choices=["i8", "separate"], default="i8",
                     help="batches of up to 64 tokens: the persistent integer-MMA kernel (default) or the separate "
                          "kernels")
@@ -223,7 +231,7 @@ class OracleLeg:
         self.E = E = wl.get("E", E_FULL)
         self.bias = synth.zipf_bias(0, 0, E)[0] if wl["zipf"] else None
         self.wr = synth.router(0, 0, E, H)
-        self.cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S)
+        self.cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S, expert_top_p=topp_arg() or 0.0)
         self.cache = {}
         self.Ts = wl["T"] if wl["T"] <= 2 else 2   # tokens of a step the sample covers
         self.layers = wl.get("layers", 0)
@@ -241,10 +249,10 @@ class OracleLeg:
             return self._stack_step(i)
         x = syn.x_bf16(X_SEED0 + i, 0, wl["T"], H) if wl["bf16"] else syn.x_f32(X_SEED0 + i, 0, wl["T"], H)
         x = np.ascontiguousarray(x[:self.Ts])
-        ids, _ = self.oracle.topk(self.oracle.router_logits(self.wr, self.bias, x), K)
+        ids, _ = self.oracle.topk(self.oracle.router_logits(self.wr, self.bias, x), K, top_p=topp_arg())
         E = self.E
         experts = [None] * (E + S)
-        for e in set(ids.ravel().tolist()) | set(range(E, E + S)):
+        for e in {e for e in ids.ravel().tolist() if e >= 0} | set(range(E, E + S)):
             if e not in self.cache:
                 self.cache[e] = syn.expert(0, 0, e, H, I)
             experts[e] = self.cache[e]
@@ -259,9 +267,9 @@ class OracleLeg:
         spent = 0.0
         for l in range(self.Ls):
             xn = orc.rmsnorm(x).astype(np.float32)  # the layer input the oracle step forms
-            ids, _ = orc.topk(orc.router_logits(self.wrs[l], self.biases[l], xn), K)
+            ids, _ = orc.topk(orc.router_logits(self.wrs[l], self.biases[l], xn), K, top_p=topp_arg())
             experts = [None] * (E + S)
-            for e in set(ids.ravel().tolist()) | set(range(E, E + S)):
+            for e in {e for e in ids.ravel().tolist() if e >= 0} | set(range(E, E + S)):
                 if (l, e) not in self.cache:
                     self.cache[(l, e)] = syn.expert(0, l, e, H, I)
                 experts[e] = self.cache[(l, e)]
@@ -496,11 +504,11 @@ def output_error(torch, coli, synth, wl, layer, x_step, y, stream, n_tok=2):
         yg = y[:n].cpu().numpy()
     bias = synth.zipf_bias(0, 0, E)[0] if wl["zipf"] else None
     wr = synth.router(0, 0, E, H)
-    ids, _ = oracle.topk(oracle.router_logits(wr, bias, xh), K)
+    ids, _ = oracle.topk(oracle.router_logits(wr, bias, xh), K, top_p=topp_arg())
     experts = [None] * (E + S)
-    for e in set(ids.ravel().tolist()) | set(range(E, E + S)):
+    for e in {e for e in ids.ravel().tolist() if e >= 0} | set(range(E, E + S)):
         experts[e] = synth.expert(0, 0, e, H, I)
-    cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S)
+    cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S, expert_top_p=topp_arg() or 0.0)
     y_ref, _, _ = oracle.moe_forward(cfg, wr, bias, experts, xh)
     yg = yg.astype(np.float64)
     if wl["bf16"]:
@@ -528,6 +536,7 @@ def run_ours(args, wl, ws, rank, local):
     T = wl["T"]
     layer = build_layer(torch, coli, synth, wl, local, max_tokens=T)
     layer.set_fused(FUSED_MODE[args.decode_kernel])
+    layer.set_expert_top_p(TOPP)
     nsteps = args.warmup + args.steps
     xdt = torch.bfloat16 if wl["bf16"] else torch.float32
     xs = torch.empty((nsteps, T, H), dtype=xdt, device=dev)
@@ -612,7 +621,8 @@ def run_ours(args, wl, ws, rank, local):
         "config": {"workload": args.workload, "desc": wl["desc"], "hidden": H, "inter": I, "experts": wl.get("E", E_FULL),
                    "top_k": K, "shared": S, "tokens_per_step": T, "weights": "int4 gs64 + fp16 scales",
                    "l2": "flushed between steps (256 MiB memset outside the step events)",
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "expert_top_p": TOPP},
         "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / 8000.0, 4),
         "hbm_frac_of_measured": round(gbs / peak_gbs, 4),
         "unique_experts_per_step": round(mean_unique, 2),
@@ -644,14 +654,14 @@ def stack_output_error(torch, coli, synth, wl, layers, x_step, stream, n_layers=
     coli.stack_forward(layers[:n_layers], xw, stream=stream)
     torch.cuda.synchronize()
     xr = x_step[:1].cpu().numpy().copy()
-    cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S)
+    cfg = oracle.Cfg(hidden=H, inter=I, n_experts=E, top_k=K, n_shared=S, expert_top_p=topp_arg() or 0.0)
     for l in range(n_layers):
         wr = synth.router(0, l, E, H)
         bias = synth.zipf_bias(0, l, E)[0]
         xn = oracle.rmsnorm(xr).astype(np.float32)
-        ids, _ = oracle.topk(oracle.router_logits(wr, bias, xn), K)
+        ids, _ = oracle.topk(oracle.router_logits(wr, bias, xn), K, top_p=topp_arg())
         experts = [None] * (E + S)
-        for e in set(ids.ravel().tolist()) | set(range(E, E + S)):
+        for e in {e for e in ids.ravel().tolist() if e >= 0} | set(range(E, E + S)):
             experts[e] = synth.expert(0, l, e, H, I)
         oracle.stack_step(cfg, wr, bias, experts, xr)
     yg = xw.cpu().numpy().astype(np.float64)
@@ -679,6 +689,7 @@ def run_stack(args, wl, ws, rank, local):
     layers = [build_layer(torch, coli, synth, wl, local, max_tokens=T, layer_idx=l) for l in range(NL)]
     for L in layers:
         L.set_fused(FUSED_MODE[args.decode_kernel])
+        L.set_expert_top_p(TOPP)
     nsteps = args.warmup + args.steps
     xs = torch.empty((nsteps, T, H), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -766,7 +777,8 @@ def run_stack(args, wl, ws, rank, local):
                    "experts": E_FULL, "top_k": K, "shared": S, "tokens_per_step": T,
                    "weights": "int4 gs64 + fp16 scales, 154.8 GB resident",
                    "l2": f"not flushed: each step streams {bytes_step / 1e9:.2f} GB of weights (L2 is 126 MB)",
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "expert_top_p": TOPP},
         "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / 8000.0, 4),
         "hbm_frac_of_measured": round(gbs / peak_gbs, 4),
         "bytes_per_step": int(bytes_step), "unique_experts_per_layer": round(mean_unique, 2),
@@ -827,6 +839,7 @@ def run_cached(args, wl, ws, rank, local):
     layers = [build_layer(torch, coli, synth, wl, local, max_tokens=T, layer_idx=l, resident=R) for l in range(NL)]
     for L in layers:
         L.set_fused(FUSED_MODE[args.decode_kernel])
+        L.set_expert_top_p(TOPP)
     nsteps = args.warmup + args.steps
     stream = torch.cuda.current_stream(dev)
     xs = torch.empty((nsteps, T, H), dtype=torch.float32, device=dev)
@@ -935,7 +948,8 @@ def run_cached(args, wl, ws, rank, local):
                    "experts": E_FULL, "top_k": K, "shared": S, "tokens_per_step": T, "resident_slots": R,
                    "pinned": wl["pin"], "learning_steps": n_learn,
                    "l2": "not flushed: every step copies experts from host memory or streams them from HBM",
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "expert_top_p": TOPP},
         "cache": {
             "hit_rate": round(hits / max(hits + misses, 1), 4),
             "misses_per_step": round(misses / args.steps, 3),
@@ -970,7 +984,11 @@ def run_cached(args, wl, ws, rank, local):
 
 
 def main():
+    global TOPP
     args = parse()
+    if not 0.0 < args.expert_top_p <= 1.0:
+        raise SystemExit("--expert-top-p must be in (0, 1]")
+    TOPP = args.expert_top_p
     wl = WORKLOADS[args.workload]
     ws, rank, local = dist_env()
     if args.impl == "reference":
@@ -994,7 +1012,8 @@ def main():
                           "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
                           "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
                           "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                          "data": "synthetic", "config": {"workload": args.workload, "desc": wl["desc"]},
+                          "data": "synthetic", "config": {"workload": args.workload, "desc": wl["desc"],
+                                                                "expert_top_p": TOPP},
                           "cpu_baseline": cb,
                           "e2e": {"value": round(val, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                                   "d2h_bytes_per_step": 0}}))

@@ -306,6 +306,21 @@ coli_status coli_moe_set_fused(coli_moe_layer* layer, int enable);
 coli_status coli_moe_set_tensor_cores(coli_moe_layer* layer, int mode);
 
 /*
+ * Adaptive expert top-p, opt-in ("colibri: 1300 lines of C ..." (jsqmd.com),
+ * usage section: topp=0.7, adaptive expert top-p, 30-40% fewer expert reads).
+ * It changes the routing: with 0 < p < 1, after the top-K of a token (slots
+ * in descending logit order, weights w_k renormalised over the K) the slots
+ * are kept while the running sum of w in slot order (fp64) has not reached p,
+ * the slot that reaches it included; the kept weights are divided by that
+ * sum. A dropped slot reports slot 0's id with weight 0 (route, plan and
+ * forward alike): the batch-union reads no expert for it and the combine
+ * adds exactly 0. p = 1 (the default) is the plain top-K. Applies to
+ * coli_moe_route, coli_moe_forward and the stack on this layer (not to
+ * coli_moe_route_noalloc). p outside (0, 1] returns COLI_EINVAL.
+ */
+coli_status coli_moe_set_expert_top_p(coli_moe_layer* layer, double p);
+
+/*
  * Item timeline of the persistent decode kernel, for profiling. `buffer` is a
  * caller-owned DEVICE buffer of 8 * (16 + 8 * capacity) bytes, zeroed by the
  * caller; int64 [0] counts records (it may exceed capacity: later records are

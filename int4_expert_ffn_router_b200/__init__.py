@@ -26,7 +26,7 @@ EXPORTS = (
     "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc", "coli_moe_get_launch_count",
     "coli_moe_debug_fail_alloc", "coli_clock_stamp", "coli_moe_debug_wait_test", "coli_moe_layer_create_cached",
     "coli_moe_cache_stats", "coli_moe_cache_pin", "coli_moe_cache_prefetch", "coli_moe_cache_set_lookahead",
-    "coli_moe_cache_slots",
+    "coli_moe_cache_slots", "coli_moe_set_expert_top_p",
 )
 NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 63, 1024
 N_STAGES = 8
@@ -89,6 +89,7 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_cache_prefetch.argtypes = [vp, vp, i32]
     L.coli_moe_cache_set_lookahead.argtypes = [vp, i32]
     L.coli_moe_cache_slots.argtypes = [vp, vp]
+    L.coli_moe_set_expert_top_p.argtypes = [vp, ctypes.c_double]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
     L.coli_last_error.argtypes = []
@@ -211,6 +212,11 @@ class Layer:
     def set_fused(self, on) -> None:
         """True: the persistent kernel for batches of up to 64 tokens (default); False: separate kernels."""
         _check(lib.coli_moe_set_fused(self.handle, 1 if on else 0), "coli_moe_set_fused")
+
+    def set_expert_top_p(self, p: float) -> None:
+        """Adaptive expert top-p (opt-in; changes routing): keep the shortest
+        prefix of each token's top-K whose weights reach p. 1.0: plain top-K."""
+        _check(lib.coli_moe_set_expert_top_p(self.handle, float(p)), "coli_moe_set_expert_top_p")
 
     def debug_wait_test(self, enable: bool, wait_ns: int = 0) -> None:
         """Testing aid: bound the persistent kernel's waits to wait_ns and, when

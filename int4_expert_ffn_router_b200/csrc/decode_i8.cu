@@ -85,6 +85,7 @@ struct I8Args {
     double* logits;
     const int32_t* given_ids;  // [T][K] routing computed before the launch (expert cache), or NULL
     const float* given_w;      // [T][K] its weights
+    double topp;               // adaptive expert top-p of the in-kernel routing (>= 1: plain top-K)
     uint8_t* xq;   // [T][H/64][128]  token limbs
     uint8_t* xm;   // [T][H/64][16]   token group meta
     uint8_t* hq;   // [slots][I/64][128]
@@ -176,15 +177,15 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
     }
 }
 
-// Bounded wait until *p >= target (acquire), polling with exponential backoff
-// (64 ns to 1 us) so that many waiting CTAs do not flood the word's L2 slice.
+// Bounded wait until *p >= target (acquire), polling every ~64 ns: the
+// waits on the plan and on the prepared tokens are on the critical path, so
+// the poll interval stays short (a longer backoff measurably lengthened the
+// batch-1 step).
 __device__ __forceinline__ bool wait_geq(const int* p, int target, volatile int* abort_flag, I8Args& a, int code) {
     if (ld_acquire(p) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t sleep_ns = 64;
     for (uint32_t n = 1;; ++n) {
-        __nanosleep(sleep_ns);
-        if (sleep_ns < 1024) sleep_ns *= 2;
+        __nanosleep(64);
         if (ld_acquire(p) >= target) return true;
         if (*abort_flag) return false;
         if ((n & 7) == 0 && others_gave_up(a, abort_flag)) return false;
@@ -630,8 +631,8 @@ __device__ void consumer_plan(I8Args& a, I8Smem& S, uint8_t* scratch, int ctid) 
         for (int t = cw; t < T; t += kCW) {
             int id;
             float wt;
-            if (E <= 256) warp_topk8<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
-            else warp_topk<true>(a.logits + (size_t)t * E, E, K, lane, &id, &wt);
+            if (E <= 256) warp_topk8<true>(a.logits + (size_t)t * E, E, K, a.topp, lane, &id, &wt);
+            else warp_topk<true>(a.logits + (size_t)t * E, E, K, a.topp, lane, &id, &wt);
             if (lane < K) {
                 sids[t * K + lane] = id;
                 sw[t * K + lane] = wt;
@@ -994,32 +995,30 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
             const Item it = S.cur[q & 1];
             const uint64_t t_begin = (a.trace && ctid == 0) ? globaltimer_ns() : 0;
             if (ctid == 0) S.first_wait_ns = S.total_wait_ns = S.t_loop0 = S.t_loop1 = 0;
-            if (it.kind == IT_PREP) {
-                prep_item<XT>(a, it.ex, ctid);
-                if (a.given_ids) {  // no router items: the CTA that finishes the last quantisation builds the plan
+            if (it.kind == IT_PREP || it.kind == IT_ROUTER) {
+                // the CTA that finishes the last router item (with the routing
+                // given: the last quantisation item) builds the plan
+                if (it.kind == IT_PREP) {
+                    prep_item<XT>(a, it.ex, ctid);
+                } else {
+                    if (ctid == 0) S.staged_kind = -1;  // the B area becomes scratch
+                    router_item<XT>(a, S, reinterpret_cast<double*>(barea), it.ex, ctid);
+                }
+                const bool counted = it.kind == IT_ROUTER || a.given_ids;
+                if (counted) {
                     named_bar(1, kCT);
                     if (ctid == 0) {
-                        S.last = atom_add_acq_rel(&a.ctl[kCI_Router], 1) == a.T - 1;
-                        if (S.last) S.staged_kind = -1;  // the B area becomes scratch
+                        const int n_items = it.kind == IT_ROUTER ? (a.d.E + kRouterExperts - 1) / kRouterExperts : a.T;
+                        const uint64_t t0 = a.trace ? globaltimer_ns() : 0;
+                        // the barrier orders the other consumers' logits before this
+                        // release, which carries them to the plan builders (cumulative)
+                        S.last = atom_add_acq_rel(&a.ctl[kCI_Router], 1) == n_items - 1;
+                        if (S.last) S.staged_kind = -1;  // the B area becomes the plan's scratch
+                        if (S.last && a.trace) { a.trace[1] = (long long)t0; a.trace[2] = (long long)globaltimer_ns(); }
                     }
                     named_bar(1, kCT);
-                    if (S.last) consumer_plan(a, S, barea, ctid);
+                    if (S.last) consumer_plan(a, S, barea, ctid);  // uniform: S.last is read after the barrier
                 }
-            } else if (it.kind == IT_ROUTER) {
-                if (ctid == 0) S.staged_kind = -1;  // the B area becomes scratch
-                router_item<XT>(a, S, reinterpret_cast<double*>(barea), it.ex, ctid);
-                // the CTA that finishes the last router item builds the plan
-                named_bar(1, kCT);
-                if (ctid == 0) {
-                    const int n_router = (a.d.E + kRouterExperts - 1) / kRouterExperts;
-                    const uint64_t t0 = a.trace ? globaltimer_ns() : 0;
-                    // the barrier orders the other consumers' logits before this
-                    // release, which carries them to the plan builders (cumulative)
-                    S.last = atom_add_acq_rel(&a.ctl[kCI_Router], 1) == n_router - 1;
-                    if (S.last && a.trace) { a.trace[1] = (long long)t0; a.trace[2] = (long long)globaltimer_ns(); }
-                }
-                named_bar(1, kCT);
-                if (S.last) consumer_plan(a, S, barea, ctid);  // uniform: S.last is read after the barrier
             } else if (it.kind == IT_GU || it.kind == IT_DOWN) {
                 weight_item<XT>(a, S, it, ring, blimb, bmeta, slot_s, phase_s, ctid);
             }
@@ -1131,7 +1130,7 @@ cudaError_t launch_decode_i8(const I8Launch& l, cudaStream_t st) {
     if (l.T < 1 || l.T > kI8MaxTok || l.T * l.d.K > kI8MaxSlots) return cudaErrorInvalidValue;
     I8Args a;
     a.weights = l.weights; a.d = l.d; a.wr = l.wr; a.bias = l.bias; a.x = l.x; a.y = l.y; a.residual = l.residual;
-    a.T = l.T; a.p = l.p; a.logits = l.logits; a.given_ids = l.given_ids; a.given_w = l.given_w; a.xq = l.xq; a.xm = l.xm; a.hq = l.hq; a.hm = l.hm; a.o = l.o;
+    a.T = l.T; a.p = l.p; a.logits = l.logits; a.given_ids = l.given_ids; a.given_w = l.given_w; a.topp = l.topp; a.xq = l.xq; a.xm = l.xm; a.hq = l.hq; a.hm = l.hm; a.o = l.o;
     a.ctl = l.ctl; a.trace = l.trace; a.trace_cap = l.trace_cap;
     a.wait_ns = l.wait_ns > 0 ? l.wait_ns : 1000000000ll;
     a.wait_test = l.wait_test;

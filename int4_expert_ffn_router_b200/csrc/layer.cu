@@ -142,6 +142,7 @@ struct coli_moe_layer {
     alignas(64) unsigned char h16_maps[2 * kTensorMapBytes] = {};  // (boxes of kTcMaxTok and 32 rows)
     size_t smem_optin = 0;
     int fused = 1;                  // coli_moe_set_fused: 1 persistent kernel for small batches, 0 separate kernels
+    double topp = 1.0;              // coli_moe_set_expert_top_p (1: plain top-K)
     long long* trace = nullptr;     // caller-owned device buffer for the item timeline
     int trace_cap = 0;
     int ring_stages = kDefaultStages;        // persistent kernel: bulk copies in flight per SM
@@ -541,7 +542,7 @@ COLI_API coli_status coli_moe_route(coli_moe_layer* L, const void* x, coli_dtype
     cudaStream_t s = (cudaStream_t)stream;
     const Dims& d = L->d;
     CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
-    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, ids, weights, s), "topk");
+    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, ids, weights, s, L->topp), "topk");
     L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
     return COLI_OK;
 }
@@ -574,6 +575,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         l.hm = L->hm; l.o = L->o; l.ctl = L->ctl; l.n_sm = L->n_sm; l.smem_limit = L->smem_optin; l.trace = L->trace;
         l.trace_cap = L->trace_cap; l.max_stages = L->ring_stages; l.max_sb = L->ring_blocks;
         l.wait_ns = L->wait_ns; l.wait_test = L->wait_test;
+        l.topp = L->topp;
         if (routed) { l.given_ids = p.ids; l.given_w = p.w; }
         CUDA_TRY(launch_decode_i8(l, s), "persistent decode kernel (integer MMA)");
         L->launches += 1;
@@ -584,7 +586,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
             prof_mark(L, COLI_STAGE_ROUTER, s);
             CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
             prof_mark(L, COLI_STAGE_TOPK, s);
-            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp), "topk");
         }
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
@@ -618,7 +620,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
             prof_mark(L, COLI_STAGE_ROUTER, s);
             CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
             prof_mark(L, COLI_STAGE_TOPK, s);
-            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp), "topk");
         }
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
@@ -738,7 +740,7 @@ static coli_status cached_forward(coli_moe_layer* L, const void* x, void* y, col
     CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap),
              "router");
     prof_mark(L, COLI_STAGE_TOPK, s);
-    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s), "topk");
+    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp), "topk");
     L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
     prof_mark(L, COLI_STAGE_CACHE, s);
     const bool ahead = next && next != L && next->cached && next->lookahead && T <= next->cfg.max_tokens &&
@@ -748,7 +750,8 @@ static coli_status cached_forward(coli_moe_layer* L, const void* x, void* y, col
         CUDA_TRY(launch_router_logits(next->router_w, next->router_b, x, dt, T, dn.H, dn.E, next->logits, s,
                                       next->rpart, next->rpart_cap),
                  "lookahead router");
-        CUDA_TRY(launch_topk(next->logits, T, dn.E, dn.K, next->plan.ids, next->plan.w, s), "lookahead topk");
+        CUDA_TRY(launch_topk(next->logits, T, dn.E, dn.K, next->plan.ids, next->plan.w, s, next->topp),
+                 "lookahead topk");
         next->launches += router_kernel_count(T, dn.H, dn.E, next->rpart, next->rpart_cap) + 1;
         CUDA_TRY(cudaMemcpyAsync(next->ahead_pin, next->plan.ids, (size_t)T * dn.K * 4, cudaMemcpyDeviceToHost, s),
                  "read predicted ids");
@@ -840,6 +843,13 @@ COLI_API coli_status coli_moe_set_fused(coli_moe_layer* L, int enable) {
     if (enable && !(L->i8_max_tok > 0 && decode_i8_supported(L->d, 1, L->smem_optin)))
         return fail(COLI_EUNSUPPORTED, "shapes too large for the persistent kernel's shared memory");
     L->fused = enable;
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_set_expert_top_p(coli_moe_layer* L, double p) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (!(p > 0.0 && p <= 1.0)) return fail(COLI_EINVAL, "p must be in (0, 1]");
+    L->topp = p;
     return COLI_OK;
 }
 

@@ -223,14 +223,14 @@ __global__ void router_reduce_kernel(const double* __restrict__ part, const floa
 // Top-k: one warp per token (warp_topk in topk.cuh).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ logits, int T, int E, int K,
-                                                   int32_t* __restrict__ ids, float* __restrict__ w) {
+                                                   double topp, int32_t* __restrict__ ids, float* __restrict__ w) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + warp;
     if (t >= T) return;
     int id;
     float wt;
-    if (E <= 256) warp_topk8<false>(logits + (size_t)t * E, E, K, lane, &id, &wt);
-    else warp_topk<false>(logits + (size_t)t * E, E, K, lane, &id, &wt);
+    if (E <= 256) warp_topk8<false>(logits + (size_t)t * E, E, K, topp, lane, &id, &wt);
+    else warp_topk<false>(logits + (size_t)t * E, E, K, topp, lane, &id, &wt);
     if (lane < K) {
         ids[(size_t)t * K + lane] = id;
         w[(size_t)t * K + lane] = wt;
@@ -397,9 +397,10 @@ cudaError_t launch_router_logits(const float* wr, const float* bias, const void*
     return cudaGetLastError();
 }
 
-cudaError_t launch_topk(const double* logits, int T, int E, int K, int32_t* ids, float* w, cudaStream_t st) {
+cudaError_t launch_topk(const double* logits, int T, int E, int K, int32_t* ids, float* w, cudaStream_t st,
+                        double topp) {
     if (T == 0) return cudaSuccess;
-    topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, K, ids, w);
+    topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, K, topp, ids, w);
     return cudaGetLastError();
 }
 

@@ -29,8 +29,44 @@ __device__ __forceinline__ double key_value(unsigned long long k) {
     return __longlong_as_double((long long)u);
 }
 
+// Weights of the selection (lane k < K holds slot k: its key, its id) and
+// the adaptive expert top-p ("colibri: 1300 lines of C ..." (jsqmd.com),
+// usage section: topp, adaptive expert top-p). w_k = exp(l_k - l_0) / z over
+// the K selected logits (fp64). With 0 < topp < 1 the slots are kept while
+// the running sum of w in slot order (fp64, sequential) has not yet reached
+// topp, the first slot that reaches it included; the kept weights are
+// divided by that sum, and each dropped slot repeats slot 0's id with weight
+// 0, so the batch-union gains nothing from it and the combine adds exactly 0.
+__device__ __forceinline__ void topk_weights(unsigned long long my_key, unsigned long long top_key, int my_id, int K,
+                                             double topp, int lane, int* id_out, float* wt_out) {
+    const double ex = (lane < K) ? exp(key_value(my_key) - key_value(top_key)) : 0.0;
+    double z = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    const double w = ex / z;
+    if (!(topp > 0.0 && topp < 1.0)) {
+        *id_out = my_id;
+        *wt_out = (float)w;
+        return;
+    }
+    int keep = K;
+    double cum = 0.0, cum_keep = 0.0;
+    for (int j = 0; j < K; ++j) {
+        cum += __shfl_sync(0xffffffffu, w, j);
+        if (keep == K && cum >= topp) {
+            keep = j + 1;
+            cum_keep = cum;
+        }
+    }
+    if (keep == K) cum_keep = cum;
+    const int first = __shfl_sync(0xffffffffu, my_id, 0);
+    *id_out = lane < keep ? my_id : first;
+    *wt_out = lane < keep ? (float)(w / cum_keep) : 0.0f;
+}
+
 template <bool coherent, int PER = kMaxPerLane>
-__device__ __forceinline__ void warp_topk(const double* __restrict__ l, int E, int K, int lane, int* id, float* wt) {
+__device__ __forceinline__ void warp_topk(const double* __restrict__ l, int E, int K, double topp, int lane, int* id,
+                                          float* wt) {
     const int per = (E + 31) / 32;  // <= PER
     unsigned long long key[PER];     // 0: absent or taken (below every logit's key)
 #pragma unroll
@@ -68,12 +104,7 @@ __device__ __forceinline__ void warp_topk(const double* __restrict__ l, int E, i
         if (k == 0) top_key = bk;
         if (lane == k) { my_key = bk; my_id = bi; }
     }
-    const double ex = (lane < K) ? exp(key_value(my_key) - key_value(top_key)) : 0.0;
-    double z = ex;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    *id = my_id;
-    *wt = (float)(ex / z);
+    topk_weights(my_key, top_key, my_id, K, topp, lane, id, wt);
 }
 
 // The same selection for E <= 256 (at most 8 logits per lane), faster: each
@@ -90,8 +121,8 @@ __device__ __forceinline__ void cx8(unsigned long long (&k)[8], int (&id)[8], in
 }
 
 template <bool coherent>
-__device__ __forceinline__ void warp_topk8(const double* __restrict__ l, int E, int K, int lane, int* id_out,
-                                           float* wt_out) {
+__device__ __forceinline__ void warp_topk8(const double* __restrict__ l, int E, int K, double topp, int lane,
+                                           int* id_out, float* wt_out) {
     unsigned long long k[8];
     int id[8];
 #pragma unroll
@@ -129,12 +160,7 @@ __device__ __forceinline__ void warp_topk8(const double* __restrict__ l, int E, 
         if (r == 0) top_key = bk;
         if (lane == r) { my_key = bk; my_id = bi; }
     }
-    const double ex = (lane < K) ? exp(key_value(my_key) - key_value(top_key)) : 0.0;
-    double z = ex;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    *id_out = my_id;
-    *wt_out = (float)(ex / z);
+    topk_weights(my_key, top_key, my_id, K, topp, lane, id_out, wt_out);
 }
 
 }  // namespace coli
