@@ -107,6 +107,14 @@ def max_over_ranks(value, dist, device):
     return float(t.item())
 
 
+def ep_combine(y, dist):
+    """Exchange step of the expert-parallel layer: every rank's partial output
+    is replaced by the sum over the ranks (all-reduce; NCCL on GPUs)."""
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(y, op=dist.ReduceOp.SUM)
+    return y
+
+
 def job_tokens_per_s(world_size, steps, tokens_per_step, total_ms):
     """Whole-job throughput: the tokens every replica processed over the slowest rank's time."""
     return world_size * steps * tokens_per_step / (total_ms * 1e-3)
@@ -201,6 +209,9 @@ def parse():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="decode_b1")
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--parallel", choices=["replicas", "ep"], default="replicas",
+                    help="N > 1: independent replicas (default, weak scaling) or one layer with its experts "
+                         "sharded over the ranks (expert parallelism, strong scaling)")
     ap.add_argument("--expert-top-p", type=float, default=1.0,
                     help="adaptive expert top-p of every layer, in (0, 1] (opt-in routing variant; 1: plain top-8)")
     ap.add_argument("--decode-kernel", choices=["i8", "separate"], default="i8",
@@ -389,9 +400,10 @@ class Clocks:
         return out
 
 
-def build_layer(torch, coli, synth, wl, device, max_tokens, layer_idx=0, resident=None):
+def build_layer(torch, coli, synth, wl, device, max_tokens, layer_idx=0, resident=None, ep=None):
     """Layer `layer_idx` of the workload: router, Zipf bias and experts drawn
-    with the generator's layer index (resident: slots of an expert cache)."""
+    with the generator's layer index (resident: slots of an expert cache;
+    ep: (rank, world) of an expert-parallel layer)."""
     E = wl.get("E", E_FULL)
     nq, ns = synth.expert_sizes(H, I)
     dev = torch.device("cuda", device)
@@ -407,7 +419,7 @@ def build_layer(torch, coli, synth, wl, device, max_tokens, layer_idx=0, residen
     torch.cuda.synchronize(dev)
     cfg = coli.make_config(H, I, E, K, S, max_tokens)
     layer = coli.Layer(cfg, wr, bias, q[:E * nq], s[:E * ns], q[E * nq:], s[E * ns:], device=device,
-                       resident=resident)
+                       resident=resident, ep=ep)
     del q, s, wr
     torch.cuda.empty_cache()
     return layer
@@ -491,7 +503,8 @@ def output_error(torch, coli, synth, wl, layer, x_step, y, stream, n_tok=2):
     error for fp32, relative L2 for bf16."""
     import numpy as np
     import oracle
-    layer.forward(x_step, y, stream=stream)
+    if layer is not None:  # (None: y already holds the step's output)
+        layer.forward(x_step, y, stream=stream)
     torch.cuda.synchronize()
     T = x_step.shape[0]
     n = min(n_tok, T)
@@ -534,17 +547,26 @@ def run_ours(args, wl, ws, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     T = wl["T"]
-    layer = build_layer(torch, coli, synth, wl, local, max_tokens=T)
+    # expert parallelism: every rank holds 1/ws of the experts and sees the same tokens;
+    # replicas: every rank holds the whole layer and draws its own tokens
+    ep = args.parallel == "ep" and ws > 1
+    layer = build_layer(torch, coli, synth, wl, local, max_tokens=T, ep=(rank, ws) if ep else None)
     layer.set_fused(FUSED_MODE[args.decode_kernel])
     layer.set_expert_top_p(TOPP)
     nsteps = args.warmup + args.steps
     xdt = torch.bfloat16 if wl["bf16"] else torch.float32
     xs = torch.empty((nsteps, T, H), dtype=xdt, device=dev)
     stream = torch.cuda.current_stream(dev)
-    for i in range(nsteps):  # rank r draws its own token stream
-        synth.x_dev(step_seed(i, rank), 0, T, H, 1 if wl["bf16"] else 0, xs[i].data_ptr(), stream.cuda_stream)
+    for i in range(nsteps):
+        synth.x_dev(step_seed(i, 0 if ep else rank), 0, T, H, 1 if wl["bf16"] else 0, xs[i].data_ptr(),
+                    stream.cuda_stream)
     y = torch.empty((T, H), dtype=xdt, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def fwd(x, yout):
+        layer.forward(x, yout, stream=stream)
+        if ep:
+            ep_combine(yout, dist)  # the exchange step: all-reduce of the partial outputs (NCCL)
 
     # routing statistics of every step (untimed pre-pass): unique experts -> bytes
     uniq = []
@@ -552,11 +574,16 @@ def run_ours(args, wl, ws, rank, local):
         layer.forward(xs[i], y, stream=stream)
         uniq.append(layer.stats()[0])
     torch.cuda.synchronize(dev)
+    uniq_local = list(uniq)
+    if ep:  # distinct experts of the whole layer = the sum of the ranks' (disjoint) sets
+        u = torch.tensor(uniq, dtype=torch.float64, device=dev)
+        dist.all_reduce(u)
+        uniq = u.cpu().tolist()
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
     # warm-up
     for i in range(args.warmup):
-        layer.forward(xs[i], y, stream=stream)
+        fwd(xs[i], y)
         flush.zero_()
     torch.cuda.synchronize(dev)
     if dist:
@@ -566,7 +593,7 @@ def run_ours(args, wl, ws, rank, local):
     n0 = layer.launch_count()
     for i in range(args.warmup, nsteps):
         ev[i][0].record(stream)
-        layer.forward(xs[i], y, stream=stream)
+        fwd(xs[i], y)
         ev[i][1].record(stream)
         flush.zero_()
     clocks.end_region()
@@ -580,7 +607,7 @@ def run_ours(args, wl, ws, rank, local):
     # per-stage device times from a separate pass (the stage events are not in the timed region)
     layer.set_profiling(True)
     for i in range(args.warmup, min(nsteps, args.warmup + 200)):
-        layer.forward(xs[i], y, stream=stream)
+        fwd(xs[i], y)
         flush.zero_()
     torch.cuda.synchronize(dev)
     stages, nprof = layer.profile()
@@ -589,9 +616,11 @@ def run_ours(args, wl, ws, rank, local):
     total_ms = max_over_ranks(total_ms, dist, dev)
 
     # end to end through the C ABI with host buffers (pinned x in, y out)
-    e2e_ms = e2e_pipelined(torch, dev, stream, xs[args.warmup:], lambda xin, yout: layer.forward(xin, yout, stream=stream),
-                           (T, H), xdt, args.steps, dist)
-    err = output_error(torch, coli, synth, wl, layer, xs[args.warmup], y, stream) if rank == 0 else None
+    e2e_ms = e2e_pipelined(torch, dev, stream, xs[args.warmup:], fwd, (T, H), xdt, args.steps, dist)
+    if ep:
+        fwd(xs[args.warmup], y)  # every rank takes part in the exchange; rank 0 checks the sum
+        torch.cuda.synchronize(dev)
+    err = output_error(torch, coli, synth, wl, None if ep else layer, xs[args.warmup], y, stream) if rank == 0 else None
 
     if rank != 0:
         layer.close()
@@ -607,21 +636,25 @@ def run_ours(args, wl, ws, rank, local):
     peaks = load_peaks()
     peak_gbs = peaks.get("hbm_gbs", 6650.0)
     tc = wl["bf16"] and T > small_batch_limit(args.decode_kernel)  # larger bf16 batches: tcgen05 grouped GEMMs
-    dom, roof = dominant_roofline(stages, nprof, T, mean_unique, wl.get("E", E_FULL), xs.element_size(), tc, peaks)
+    # the roofline of this rank's kernel: its own distinct experts (expert parallelism) or all of them
+    mean_local = sum(uniq_local[args.warmup:]) / len(uniq_local[args.warmup:])
+    dom, roof = dominant_roofline(stages, nprof, T, mean_local, wl.get("E", E_FULL), xs.element_size(), tc, peaks)
     if roof is not None:
         roof["traffic"], roof["traffic_note"] = ncu_traffic(roof["kernel"], args.workload)
     out = {
-        "metric": METRIC, "value": round(job_tokens_per_s(ws, args.steps, T, total_ms), 2), "unit": "tokens/s", "n_gpus": ws,
+        "metric": METRIC, "value": round(job_tokens_per_s(1 if ep else ws, args.steps, T, total_ms), 2), "unit": "tokens/s",
+        "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 5),
         "step_ms_rank0": step_percentiles(step_ms),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if ep else "weak", "vs_baseline": None,
         "dtype": path_dtype(args.decode_kernel, T, wl["bf16"], tc),
         "stage_note": "stage_us from a separate profiled pass (stage events add host gaps)",
         "data": "synthetic (seeded generator; random-init int4 weights of the full-size layer shape)",
         "config": {"workload": args.workload, "desc": wl["desc"], "hidden": H, "inter": I, "experts": wl.get("E", E_FULL),
                    "top_k": K, "shared": S, "tokens_per_step": T, "weights": "int4 gs64 + fp16 scales",
                    "l2": "flushed between steps (256 MiB memset outside the step events)",
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                   "parallelism": (f"expert parallel x{ws} (NCCL all-reduce of partial outputs)" if ep else
+                                   f"replicas x{ws}" if ws > 1 else "single GPU"),
                    "expert_top_p": TOPP},
         "hbm_gbs": round(gbs, 1), "hbm_frac_of_8tbs": round(gbs / 8000.0, 4),
         "hbm_frac_of_measured": round(gbs / peak_gbs, 4),
@@ -633,7 +666,7 @@ def run_ours(args, wl, ws, rank, local):
         "gpu_launches_note": "forward kernels in the timed loop; two clock-stamp kernels bracket the loop",
         "max_rel_err": err,
         "compute": compute_desc(args.decode_kernel, T, tc),
-        "e2e": {"value": round(job_tokens_per_s(ws, args.steps, T, e2e_ms), 2), "unit": "tokens/s",
+        "e2e": {"value": round(job_tokens_per_s(1 if ep else ws, args.steps, T, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * xs.element_size(), "d2h_bytes_per_step": T * H * xs.element_size(),
                 "method": E2E_METHOD},
         "clocks": clk,

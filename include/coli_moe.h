@@ -136,6 +136,34 @@ coli_status coli_moe_layer_create_cached(const coli_moe_config* cfg, const float
                                          const uint8_t* shared_q, const uint16_t* shared_scales,
                                          int resident_slots, int device, coli_moe_layer** out);
 
+/*
+ * Expert parallelism (an MoE layer sharded by expert over `world` GPUs, one
+ * process per GPU): rank r holds the routed experts
+ * [E*r/world, E*(r+1)/world) (coli_moe_ep_range) and, on rank 0 only, the
+ * shared experts. Arguments as coli_moe_layer_create (expert_q and
+ * expert_scales hold all E experts in the canonical layout; only this rank's
+ * are read; shared_q is read on rank 0 only), plus rank and world
+ * (1 <= world <= n_experts).
+ *
+ * The router is replicated: every rank computes the full top-K of every token.
+ * A forward then writes this rank's PARTIAL output,
+ *   y_r[t] = [r == 0] * sum_j shared_j(x_t) + sum over the token's slots k
+ *            whose expert this rank holds of w[t][k] * E_ids[t][k](x_t),
+ * with the same kernels as a whole layer (the plan lists only this rank's
+ * experts; the other slots are empty: coli_moe_get_plan reports them as id
+ * -1 and position -1). The caller sums y_r over the ranks (an all-reduce, for
+ * example NCCL over NVLink); the sum is the layer's output up to the order of
+ * the fp32 additions. A bf16 layer's partial outputs are bf16.
+ * coli_moe_route on such a layer returns the full routing.
+ */
+coli_status coli_moe_layer_create_ep(const coli_moe_config* cfg, const float* router_w, const float* router_bias,
+                                     const uint8_t* expert_q, const uint16_t* expert_scales,
+                                     const uint8_t* shared_q, const uint16_t* shared_scales,
+                                     int rank, int world, int device, coli_moe_layer** out);
+
+/* The routed experts [*first, *end) that rank `rank` of `world` holds. */
+coli_status coli_moe_ep_range(int n_experts, int rank, int world, int* first, int* end);
+
 typedef struct {
     int64_t hits;           /* experts a batch needed that were resident                */
     int64_t misses;         /* experts a batch needed that were copied in before it     */

@@ -26,7 +26,7 @@ EXPORTS = (
     "coli_moe_set_trace", "coli_moe_set_ring", "coli_moe_route_noalloc", "coli_moe_get_launch_count",
     "coli_moe_debug_fail_alloc", "coli_clock_stamp", "coli_moe_debug_wait_test", "coli_moe_layer_create_cached",
     "coli_moe_cache_stats", "coli_moe_cache_pin", "coli_moe_cache_prefetch", "coli_moe_cache_set_lookahead",
-    "coli_moe_cache_slots", "coli_moe_set_expert_top_p",
+    "coli_moe_cache_slots", "coli_moe_set_expert_top_p", "coli_moe_layer_create_ep", "coli_moe_ep_range",
 )
 NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 63, 1024
 N_STAGES = 8
@@ -90,6 +90,8 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_cache_set_lookahead.argtypes = [vp, i32]
     L.coli_moe_cache_slots.argtypes = [vp, vp]
     L.coli_moe_set_expert_top_p.argtypes = [vp, ctypes.c_double]
+    L.coli_moe_layer_create_ep.argtypes = [pcfg, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.POINTER(vp)]
+    L.coli_moe_ep_range.argtypes = [i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
     L.coli_last_error.argtypes = []
@@ -142,16 +144,22 @@ def expert_bytes(hidden: int, inter: int) -> int:
 
 
 class Layer:
-    """One MoE layer on a CUDA device: every expert resident in HBM, or, with
+    """One MoE layer on a CUDA device: every expert resident in HBM; with
     ``resident`` = R, an expert cache of R routed experts in HBM over a
-    page-locked host copy of all of them."""
+    page-locked host copy of all of them; with ``ep`` = (rank, world), rank's
+    share of an expert-parallel layer (forward writes its partial output)."""
 
     def __init__(self, cfg: Config, router_w, router_bias=None, expert_q=None, expert_scales=None,
-                 shared_q=None, shared_scales=None, device: int = 0, resident: int | None = None):
+                 shared_q=None, shared_scales=None, device: int = 0, resident: int | None = None, ep=None):
         h = ctypes.c_void_p()
         args = (ctypes.byref(cfg), _ptr(router_w), _ptr(router_bias), _ptr(expert_q), _ptr(expert_scales),
                 _ptr(shared_q), _ptr(shared_scales))
-        if resident is None:
+        if ep is not None:
+            if resident is not None:
+                raise ValueError("an expert-parallel layer has no expert cache")
+            _check(lib.coli_moe_layer_create_ep(*args, int(ep[0]), int(ep[1]), device, ctypes.byref(h)),
+                   "coli_moe_layer_create_ep")
+        elif resident is None:
             _check(lib.coli_moe_layer_create(*args, device, ctypes.byref(h)), "coli_moe_layer_create")
         else:
             _check(lib.coli_moe_layer_create_cached(*args, resident, device, ctypes.byref(h)),
@@ -306,6 +314,13 @@ class Layer:
         out["unique"] = out["unique"][:nu.value]
         out["tok"] = out["tok"][:T * K]
         return out
+
+
+def ep_range(n_experts: int, rank: int, world: int) -> tuple[int, int]:
+    """The routed experts [first, end) rank `rank` of `world` holds."""
+    a, b = ctypes.c_int(), ctypes.c_int()
+    _check(lib.coli_moe_ep_range(n_experts, rank, world, ctypes.byref(a), ctypes.byref(b)), "coli_moe_ep_range")
+    return a.value, b.value
 
 
 def route_noalloc(router_w, router_bias, n_experts: int, hidden: int, top_k: int, x, ids, weights,

@@ -23,8 +23,10 @@ __global__ void combine_kernel(const float* __restrict__ o, Plan p, int T, int H
             acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
         }
         for (int k = 0; k < K; ++k) {
+            const int q = p.pos[t * K + k];
+            if (q < 0) continue;  // an empty slot (expert of another rank)
             const float wk = p.w[t * K + k];
-            const float4 v = reinterpret_cast<const float4*>(o + (size_t)p.pos[t * K + k] * H)[c4];
+            const float4 v = reinterpret_cast<const float4*>(o + (size_t)q * H)[c4];
             acc.x = fmaf(wk, v.x, acc.x);
             acc.y = fmaf(wk, v.y, acc.y);
             acc.z = fmaf(wk, v.z, acc.z);

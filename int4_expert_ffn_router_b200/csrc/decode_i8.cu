@@ -86,6 +86,7 @@ struct I8Args {
     const int32_t* given_ids;  // [T][K] routing computed before the launch (expert cache), or NULL
     const float* given_w;      // [T][K] its weights
     double topp;               // adaptive expert top-p of the in-kernel routing (>= 1: plain top-K)
+    int ep_lo, ep_hi;          // routed experts of this rank; the others become empty slots (id -1)
     uint8_t* xq;   // [T][H/64][128]  token limbs
     uint8_t* xm;   // [T][H/64][16]   token group meta
     uint8_t* hq;   // [slots][I/64][128]
@@ -120,6 +121,7 @@ struct I8Smem {
     int bpending;           // a B staging was issued and not yet seen complete
     int aborted;            // snapshot of abort_flag taken by consumer 0 before a barrier
     int staged_kind;        // IT_GU / IT_DOWN / -1: what the B area holds
+    int plan_chunks;        // routed chunks of the plan this CTA built
     int staged_n, staged_key;
     int staged_tok[8];
     int wsum[kCW], wflag[kCW];
@@ -418,9 +420,10 @@ __device__ void signal_combine(I8Args& a, int rt, int lane) {
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const int qq = __shfl_sync(0xffffffffu, q_l, (c0 + c) & 31);
-                    const float* orow = a.o + (size_t)qq * d.H + rt * kTileRows + lane;
+                    const float* orow = a.o + (size_t)max(qq, 0) * d.H + rt * kTileRows + lane;
+                    // an empty slot (qq < 0: expert of another rank) reads nothing and adds 0
 #pragma unroll
-                    for (int j = 0; j < kJ; ++j) v[c][j] = c0 + c < nk ? __ldcg(orow + 32 * j) : 0.0f;
+                    for (int j = 0; j < kJ; ++j) v[c][j] = (c0 + c < nk && qq >= 0) ? __ldcg(orow + 32 * j) : 0.0f;
                 }
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
@@ -634,7 +637,7 @@ __device__ void consumer_plan(I8Args& a, I8Smem& S, uint8_t* scratch, int ctid) 
             if (E <= 256) warp_topk8<true>(a.logits + (size_t)t * E, E, K, a.topp, lane, &id, &wt);
             else warp_topk<true>(a.logits + (size_t)t * E, E, K, a.topp, lane, &id, &wt);
             if (lane < K) {
-                sids[t * K + lane] = id;
+                sids[t * K + lane] = (id >= a.ep_lo && id < a.ep_hi) ? id : -1;
                 sw[t * K + lane] = wt;
             }
         }
@@ -642,7 +645,8 @@ __device__ void consumer_plan(I8Args& a, I8Smem& S, uint8_t* scratch, int ctid) 
     for (int e = ctid; e < E; e += kCT) scnt[e] = 0;
     named_bar(1, kCT);
     if (a.trace && ctid == 0) a.trace[5] = (long long)globaltimer_ns();
-    for (int sl = ctid; sl < TK; sl += kCT) atomicAdd(&scnt[sids[sl]], 1);
+    for (int sl = ctid; sl < TK; sl += kCT)
+        if (sids[sl] >= 0) atomicAdd(&scnt[sids[sl]], 1);  // < 0: an empty slot
     named_bar(1, kCT);
     // per expert: first position, distinct-expert rank, first chunk
     unsigned long long* entries = entries_of(a, d.S * a.cps + a.ncmax);
@@ -676,13 +680,17 @@ __device__ void consumer_plan(I8Args& a, I8Smem& S, uint8_t* scratch, int ctid) 
     // slot (t, k): position = first position of its expert + earlier tokens of that expert
     for (int sl = ctid; sl < TK; sl += kCT) {
         const int e = sids[sl], t = sl / K;
+        a.p.ids[sl] = e;
+        a.p.w[sl] = sw[sl];
+        if (e < 0) {
+            a.p.pos[sl] = -1;
+            continue;
+        }
         int rank = 0;
         for (int s2 = 0; s2 < t * K; ++s2) rank += sids[s2] == e;
         const int q = soff[e] + rank;
         a.p.pos[sl] = q;
         a.p.tok[q] = t;
-        a.p.ids[sl] = e;
-        a.p.w[sl] = sw[sl];
     }
     for (int i = ctid; i < d.S * T; i += kCT) a.p.tok[TK + i] = i % T;
     if (ctid == 0) {
@@ -691,6 +699,7 @@ __device__ void consumer_plan(I8Args& a, I8Smem& S, uint8_t* scratch, int ctid) 
         *a.p.n_active = ucarry + d.S;
     }
     if (a.trace && ctid == 0) a.trace[7] = (long long)globaltimer_ns();
+    if (ctid == 0) S.plan_chunks = ccarry;
     named_bar(1, kCT);  // orders every consumer's plan writes before thread 0's release
     if (ctid == 0) {
         if (a.trace) a.trace[8] = (long long)globaltimer_ns();
@@ -1017,7 +1026,19 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
                         if (S.last && a.trace) { a.trace[1] = (long long)t0; a.trace[2] = (long long)globaltimer_ns(); }
                     }
                     named_bar(1, kCT);
-                    if (S.last) consumer_plan(a, S, barea, ctid);  // uniform: S.last is read after the barrier
+                    if (S.last) {  // uniform: S.last is read after the barrier
+                        consumer_plan(a, S, barea, ctid);
+                        // no routed chunk and no shared expert (a rank of an expert-parallel layer
+                        // that holds none of the batch's experts): no down item will combine the
+                        // output, so it is the residual (or 0) here
+                        if (S.plan_chunks == 0 && a.d.S == 0) {
+                            for (size_t i = ctid; i < (size_t)a.T * a.d.H; i += kCT) {
+                                const float v = a.residual ? a.residual[i] : 0.0f;
+                                if constexpr (sizeof(XT) == 4) reinterpret_cast<float*>(a.y)[i] = v;
+                                else reinterpret_cast<__nv_bfloat16*>(a.y)[i] = __float2bfloat16_rn(v);
+                            }
+                        }
+                    }
                 }
             } else if (it.kind == IT_GU || it.kind == IT_DOWN) {
                 weight_item<XT>(a, S, it, ring, blimb, bmeta, slot_s, phase_s, ctid);
@@ -1130,7 +1151,7 @@ cudaError_t launch_decode_i8(const I8Launch& l, cudaStream_t st) {
     if (l.T < 1 || l.T > kI8MaxTok || l.T * l.d.K > kI8MaxSlots) return cudaErrorInvalidValue;
     I8Args a;
     a.weights = l.weights; a.d = l.d; a.wr = l.wr; a.bias = l.bias; a.x = l.x; a.y = l.y; a.residual = l.residual;
-    a.T = l.T; a.p = l.p; a.logits = l.logits; a.given_ids = l.given_ids; a.given_w = l.given_w; a.topp = l.topp; a.xq = l.xq; a.xm = l.xm; a.hq = l.hq; a.hm = l.hm; a.o = l.o;
+    a.T = l.T; a.p = l.p; a.logits = l.logits; a.given_ids = l.given_ids; a.given_w = l.given_w; a.topp = l.topp; a.ep_lo = l.ep_lo; a.ep_hi = l.ep_hi > 0 ? l.ep_hi : l.d.E; a.xq = l.xq; a.xm = l.xm; a.hq = l.hq; a.hm = l.hm; a.o = l.o;
     a.ctl = l.ctl; a.trace = l.trace; a.trace_cap = l.trace_cap;
     a.wait_ns = l.wait_ns > 0 ? l.wait_ns : 1000000000ll;
     a.wait_test = l.wait_test;

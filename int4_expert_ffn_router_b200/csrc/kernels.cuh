@@ -19,8 +19,9 @@ cudaError_t launch_router_logits(const float* wr, const float* bias, const void*
 // Kernels launch_router_logits enqueues for these arguments (0, 1 or 2).
 int router_kernel_count(int T, int H, int E, const double* part, size_t part_cap);
 // topp in (0, 1): adaptive expert top-p after the top-K (topk.cuh, topk_weights); else plain top-K.
+// Selected experts outside [e_lo, e_hi) (e_hi < 0: E) are written as empty slots (id -1).
 cudaError_t launch_topk(const double* logits, int T, int E, int K, int32_t* ids, float* w, cudaStream_t st,
-                        double topp = 1.0);
+                        double topp = 1.0, int e_lo = 0, int e_hi = -1);
 size_t plan_smem_bytes(int E);
 cudaError_t launch_plan(const int32_t* ids, int T, int K, int E, int S, const Plan& p, cudaStream_t st);
 
@@ -62,6 +63,7 @@ struct I8Launch {
     const int32_t* given_ids;  // [T][K] ids routed before the launch (then no router items run), or NULL
     const float* given_w;      // [T][K] their weights
     double topp;               // adaptive expert top-p of the in-kernel routing (>= 1 or 0: plain top-K)
+    int ep_lo, ep_hi;          // routed experts of this rank (expert parallelism): others become empty slots
     uint8_t* xq;   // [T][H/64][128] token parts (written by the kernel)
     uint8_t* xm;   // [T][H/64][16]
     uint8_t* hq;   // [slots][I/64][128] SwiGLU output parts

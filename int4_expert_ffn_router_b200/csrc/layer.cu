@@ -179,6 +179,10 @@ struct coli_moe_layer {
     cudaEvent_t ev_prefetch = nullptr;    // prefetch copies finished
     cudaEvent_t ev_done = nullptr;        // the last forward's kernels finished reading the slots
     std::vector<char> prefetched;     // [E] resident because of a prefetch, not yet needed
+    // expert parallelism (coli_moe_layer_create_ep): this rank's routed experts [ep_lo, ep_hi)
+    // in slots 0.., its shared experts (rank 0: all, else none) after them
+    bool ep = false;
+    int ep_lo = 0, ep_hi = 0;
     int64_t bytes_h2d = 0, n_prefetched = 0, prefetch_used = 0, predicted = 0, predicted_of = 0;
 };
 
@@ -253,6 +257,10 @@ COLI_API coli_status coli_moe_debug_fail_alloc(int nth) {
 // Weight slot of expert e (routed 0..E-1, shared E..E+S-1): its id, or in a
 // cached layer its cache slot (-1: not resident) and R + j for shared expert j.
 static int weight_slot(const coli_moe_layer* L, int e) {
+    if (L->ep) {  // -1: held by another rank
+        if (e < L->d.E) return (e >= L->ep_lo && e < L->ep_hi) ? e - L->ep_lo : -1;
+        return e - L->d.E < L->d.S ? (L->ep_hi - L->ep_lo) + (e - L->d.E) : -1;
+    }
     if (!L->cached) return e;
     return e < L->d.E ? L->cache.slot(e) : L->cache.slots + (e - L->d.E);
 }
@@ -308,6 +316,7 @@ COLI_API coli_status coli_moe_layer_set_experts(coli_moe_layer* L, int first, in
         }
         // a cached layer's routed expert is repacked once, then kept in the host pool
         const int e = first + i;
+        if (L->ep && weight_slot(L, e) < 0) continue;  // another rank's expert
         const bool pooled = L->cached && e < L->d.E;
         uint8_t* dst = pooled ? L->repack_buf : L->weights + (size_t)weight_slot(L, e) * L->d.expert_stride;
         CUDA_TRY(launch_repack(eq, es, eq + mq, es + ms, 2 * I, H, true, dst, 0), "repack gate/up");
@@ -335,9 +344,11 @@ COLI_API coli_status coli_moe_layer_set_experts(coli_moe_layer* L, int first, in
 }
 
 // resident < 0: every expert in HBM; otherwise an expert cache of `resident` routed slots.
+// ep_world > 0: expert parallelism, this layer holding rank ep_rank's share (no cache).
 static coli_status create_impl(const coli_moe_config* cfg, const float* router_w, const float* router_bias,
                                const uint8_t* expert_q, const uint16_t* expert_scales, const uint8_t* shared_q,
-                               const uint16_t* shared_scales, int resident, int device, coli_moe_layer** out) {
+                               const uint16_t* shared_scales, int resident, int device, coli_moe_layer** out,
+                               int ep_rank = 0, int ep_world = 0) {
     if (!out) return fail(COLI_EINVAL, "out is NULL");
     *out = nullptr;
     coli_status st = check_cfg(cfg);
@@ -366,6 +377,13 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
     L->device = device;
     Dims& d = L->d;
     d.H = cfg->hidden; d.I = cfg->inter; d.E = cfg->n_experts; d.K = cfg->top_k; d.S = cfg->n_shared;
+    L->ep_hi = d.E;
+    if (ep_world > 0) {  // rank r holds [E r / world, E (r + 1) / world) and, on rank 0, the shared experts
+        L->ep = true;
+        L->ep_lo = (int)((int64_t)d.E * ep_rank / ep_world);
+        L->ep_hi = (int)((int64_t)d.E * (ep_rank + 1) / ep_world);
+        if (ep_rank != 0) d.S = 0;
+    }
     d.max_tokens = cfg->max_tokens;
     d.gu_bytes = matrix_bytes(2 * d.I, d.H);
     d.d_bytes = matrix_bytes(d.H, d.I);
@@ -381,7 +399,7 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
         return s;
     };
     cudaError_t e;
-    const size_t n_slots = (size_t)(resident >= 0 ? resident : d.E) + d.S;
+    const size_t n_slots = (size_t)(resident >= 0 ? resident : L->ep_hi - L->ep_lo) + d.S;
     if ((e = dev_alloc(&L->weights, n_slots * d.expert_stride)) != cudaSuccess) return bail(e, "cudaMalloc(weights)");
     if ((e = dev_alloc(&L->router_w, (size_t)d.E * d.H * 4)) != cudaSuccess) return bail(e, "cudaMalloc(router)");
     if ((e = dev_alloc(&L->router_b, (size_t)d.E * 4)) != cudaSuccess) return bail(e, "cudaMalloc(bias)");
@@ -470,6 +488,14 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
         if ((e = upload_table(L, nullptr)) != cudaSuccess) return bail(e, "upload slot table");
         d.slot_of = L->slot_dev;
     }
+    if (L->ep) {  // slot table of this rank's experts (others: slot 0, never read)
+        std::vector<int32_t> table(EA, 0);
+        for (int x = 0; x < (int)EA; ++x) table[x] = std::max(weight_slot(L, x), 0);
+        if ((e = dev_alloc(&L->slot_dev, EA * 4)) != cudaSuccess) return bail(e, "cudaMalloc(slot table)");
+        if ((e = cudaMemcpy(L->slot_dev, table.data(), EA * 4, cudaMemcpyHostToDevice)) != cudaSuccess)
+            return bail(e, "upload slot table");
+        d.slot_of = L->slot_dev;
+    }
 
     if ((e = cudaMemcpy(L->router_w, router_w, (size_t)d.E * d.H * 4, cudaMemcpyDefault)) != cudaSuccess) return bail(e, "copy router");
     if (router_bias) {
@@ -481,7 +507,7 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
         st = coli_moe_layer_set_experts(L, 0, d.E, expert_q, expert_scales);
         if (st != COLI_OK) { free_layer(L); return st; }
     }
-    if (shared_q) {
+    if (shared_q && d.S > 0) {
         st = coli_moe_layer_set_experts(L, d.E, d.S, shared_q, shared_scales);
         if (st != COLI_OK) { free_layer(L); return st; }
     }
@@ -495,6 +521,26 @@ COLI_API coli_status coli_moe_layer_create(const coli_moe_config* cfg, const flo
                                            const uint8_t* shared_q, const uint16_t* shared_scales, int device,
                                            coli_moe_layer** out) {
     return create_impl(cfg, router_w, router_bias, expert_q, expert_scales, shared_q, shared_scales, -1, device, out);
+}
+
+COLI_API coli_status coli_moe_ep_range(int n_experts, int rank, int world, int* first, int* end) {
+    if (n_experts < 1 || world < 1 || rank < 0 || rank >= world || !first || !end)
+        return fail(COLI_EINVAL, "need n_experts >= 1, 0 <= rank < world, non-NULL outputs");
+    *first = (int)((int64_t)n_experts * rank / world);
+    *end = (int)((int64_t)n_experts * (rank + 1) / world);
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_layer_create_ep(const coli_moe_config* cfg, const float* router_w,
+                                              const float* router_bias, const uint8_t* expert_q,
+                                              const uint16_t* expert_scales, const uint8_t* shared_q,
+                                              const uint16_t* shared_scales, int rank, int world, int device,
+                                              coli_moe_layer** out) {
+    if (out) *out = nullptr;
+    if (!cfg || world < 1 || rank < 0 || rank >= world || world > cfg->n_experts)
+        return fail(COLI_EINVAL, "need 1 <= world <= n_experts and 0 <= rank < world");
+    return create_impl(cfg, router_w, router_bias, expert_q, expert_scales, shared_q, shared_scales, -1, device, out,
+                       rank, world);
 }
 
 COLI_API coli_status coli_moe_layer_create_cached(const coli_moe_config* cfg, const float* router_w,
@@ -576,6 +622,8 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         l.trace_cap = L->trace_cap; l.max_stages = L->ring_stages; l.max_sb = L->ring_blocks;
         l.wait_ns = L->wait_ns; l.wait_test = L->wait_test;
         l.topp = L->topp;
+        l.ep_lo = L->ep_lo;
+        l.ep_hi = L->ep_hi;
         if (routed) { l.given_ids = p.ids; l.given_w = p.w; }
         CUDA_TRY(launch_decode_i8(l, s), "persistent decode kernel (integer MMA)");
         L->launches += 1;
@@ -586,7 +634,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
             prof_mark(L, COLI_STAGE_ROUTER, s);
             CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
             prof_mark(L, COLI_STAGE_TOPK, s);
-            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp), "topk");
+            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp, L->ep_lo, L->ep_hi), "topk");
         }
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
@@ -620,7 +668,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
             prof_mark(L, COLI_STAGE_ROUTER, s);
             CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
             prof_mark(L, COLI_STAGE_TOPK, s);
-            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp), "topk");
+            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp, L->ep_lo, L->ep_hi), "topk");
         }
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
@@ -740,7 +788,7 @@ static coli_status cached_forward(coli_moe_layer* L, const void* x, void* y, col
     CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap),
              "router");
     prof_mark(L, COLI_STAGE_TOPK, s);
-    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp), "topk");
+    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp, L->ep_lo, L->ep_hi), "topk");
     L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
     prof_mark(L, COLI_STAGE_CACHE, s);
     const bool ahead = next && next != L && next->cached && next->lookahead && T <= next->cfg.max_tokens &&

@@ -498,6 +498,7 @@ __global__ void prefill_prep_kernel(const XT* __restrict__ x, int T, int H, int 
             }
             const uint4 hv = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
             for (int q = 0; q < np; ++q) {
+                if (dst[q] < 0) continue;  // an empty slot (expert of another rank)
                 if constexpr (kF32) {
                     reinterpret_cast<uint4*>(xs + (size_t)(2 * dst[q]) * H + i)[0] = hv;
                     reinterpret_cast<uint4*>(xs + (size_t)(2 * dst[q] + 1) * H + i)[0] =
@@ -523,7 +524,7 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(Plan p, int T, int K
     for (int i = threadIdx.x; i < TK; i += blockDim.x) {
         const int t = i / K;
         const float4 ts = tscale[t];
-        slot[p.pos[i]] = make_float4(ts.x, ts.y, p.w[i] * ts.z, __int_as_float(t));
+        if (p.pos[i] >= 0) slot[p.pos[i]] = make_float4(ts.x, ts.y, p.w[i] * ts.z, __int_as_float(t));
     }
     for (int i = threadIdx.x; i < S * T; i += blockDim.x) {
         const int t = i % T;

@@ -223,7 +223,8 @@ __global__ void router_reduce_kernel(const double* __restrict__ part, const floa
 // Top-k: one warp per token (warp_topk in topk.cuh).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ logits, int T, int E, int K,
-                                                   double topp, int32_t* __restrict__ ids, float* __restrict__ w) {
+                                                   double topp, int e_lo, int e_hi, int32_t* __restrict__ ids,
+                                                   float* __restrict__ w) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + warp;
     if (t >= T) return;
@@ -232,7 +233,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const double* __restrict__ lo
     if (E <= 256) warp_topk8<false>(logits + (size_t)t * E, E, K, topp, lane, &id, &wt);
     else warp_topk<false>(logits + (size_t)t * E, E, K, topp, lane, &id, &wt);
     if (lane < K) {
-        ids[(size_t)t * K + lane] = id;
+        // experts outside [e_lo, e_hi) belong to another rank: an empty slot here
+        ids[(size_t)t * K + lane] = (id >= e_lo && id < e_hi) ? id : -1;
         w[(size_t)t * K + lane] = wt;
     }
 }
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     for (int t = tb; t < te; ++t) {
         if (lane < K) {
             int e = ids[(size_t)t * K + lane];
-            wcnt[warp * E + e] += 1;
+            if (e >= 0) wcnt[warp * E + e] += 1;  // e < 0: an empty slot
         }
         __syncwarp();
     }
@@ -340,10 +342,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     for (int t = tb; t < te; ++t) {
         if (lane < K) {
             int e = ids[(size_t)t * K + lane];
-            int q = off[e] + wcnt[warp * E + e];
-            wcnt[warp * E + e] += 1;
-            p.pos[(size_t)t * K + lane] = q;
-            p.tok[q] = t;
+            if (e >= 0) {
+                int q = off[e] + wcnt[warp * E + e];
+                wcnt[warp * E + e] += 1;
+                p.pos[(size_t)t * K + lane] = q;
+                p.tok[q] = t;
+            } else {
+                p.pos[(size_t)t * K + lane] = -1;
+            }
         }
         __syncwarp();
     }
@@ -398,9 +404,10 @@ cudaError_t launch_router_logits(const float* wr, const float* bias, const void*
 }
 
 cudaError_t launch_topk(const double* logits, int T, int E, int K, int32_t* ids, float* w, cudaStream_t st,
-                        double topp) {
+                        double topp, int e_lo, int e_hi) {
     if (T == 0) return cudaSuccess;
-    topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, K, topp, ids, w);
+    if (e_hi < 0) e_hi = E;
+    topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, K, topp, e_lo, e_hi, ids, w);
     return cudaGetLastError();
 }
 
