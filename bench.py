@@ -71,6 +71,16 @@ WORKLOADS = {
     "decode_b1_cached": dict(T=1, zipf=True, bf16=False, resident=64, pin=48,
                              desc="one full-size layer as an expert cache (64 of 256 routed experts in HBM, 48 "
                                   "pinned by learned usage, LRU), decode batch 1, Zipf(1.1) router bias, fp32"),
+    # speculative verify: one sequence's current token and 3 draft positions as one batch, so
+    # the batch-union reads each distinct expert once for all four; positions of one sequence
+    # share part of their hidden state (x_j = 0.6 x_0 + 0.8 z_j); accepted tokens per forward
+    # taken as 2.5 (the pages report 2.2-2.8 with an int8 draft head)
+    "verify_b4": dict(T=4, zipf=True, bf16=False, verify=dict(rho=0.6, tau=2.5),
+                      desc="one full-size layer, speculative verify batch of 1 + 3 draft positions of one "
+                           "sequence (correlated tokens), Zipf(1.1) router bias, fp32"),
+    "verify_b4_cached": dict(T=4, zipf=True, bf16=False, resident=64, pin=32, verify=dict(rho=0.6, tau=2.5),
+                             desc="speculative verify batch (1 + 3 draft positions) on an expert-cache layer "
+                                  "(64 of 256 in HBM, 32 pinned, LRU), Zipf(1.1), fp32"),
     "stack4_b1_cached": dict(T=1, zipf=True, bf16=False, layers=4, resident=64, pin=48,
                              desc="4-layer stack of expert-cache layers (64 of 256 in HBM each, 48 pinned, LRU), "
                                   "each next layer's router run one layer ahead to prefetch, decode batch 1, "
@@ -89,7 +99,7 @@ FUSED_MODE = {"i8": 1, "separate": 0}
 
 DEFAULT_STEPS = {"decode_b1": 10000, "decode_b32": 2000, "prefill_2048": 100, "decode_b1_e16": 1000, "prefill_e64": 100,
                  "stack30_b1": 300, "stack30_b8": 200, "stack30_b64": 100, "decode_b1_cached": 2000,
-                 "stack4_b1_cached": 500}
+                 "stack4_b1_cached": 500, "verify_b4": 5000, "verify_b4_cached": 1000}
 
 
 def step_seed(step, rank):
@@ -105,6 +115,32 @@ def max_over_ranks(value, dist, device):
     t = torch.tensor([float(value)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def fill_tokens(torch, synth, wl, xs, seed_of, stream):
+    """Step i's tokens into xs[i] (device): N(0,1) rows drawn with seed
+    seed_of(i); for a verify workload rows 1.. become positions of the same
+    sequence as row 0, x_j = rho x_0 + sqrt(1 - rho^2) z_j."""
+    T = xs.shape[1]
+    for i in range(xs.shape[0]):
+        synth.x_dev(seed_of(i), 0, T, H, 1 if wl["bf16"] else 0, xs[i].data_ptr(), stream.cuda_stream)
+    v = wl.get("verify")
+    if v:
+        rho = v["rho"]
+        xs[:, 1:] = rho * xs[:, :1] + (1.0 - rho * rho) ** 0.5 * xs[:, 1:]
+
+
+def verify_report(wl, mean_loads, forwards_per_s):
+    """Expert loads and accepted tokens of a verify workload (loads = distinct
+    routed experts of the batch + the shared experts)."""
+    v = wl["verify"]
+    return {"positions": wl["T"], "rho": v["rho"], "tokens_per_forward_assumed": v["tau"],
+            "expert_loads_per_forward": round(mean_loads, 2),
+            "expert_loads_per_token": round(mean_loads / v["tau"], 2),
+            "expert_loads_per_token_plain_decode": K + S,
+            "accepted_tokens_per_s": round(forwards_per_s * v["tau"], 1),
+            "note": ("accepted tokens per forward is a property of the draft head, not of this layer; "
+                     "the value assumed is the middle of the pages' 2.2-2.8")}
 
 
 def ep_combine(y, dist):
@@ -259,6 +295,9 @@ class OracleLeg:
         if self.layers:
             return self._stack_step(i)
         x = syn.x_bf16(X_SEED0 + i, 0, wl["T"], H) if wl["bf16"] else syn.x_f32(X_SEED0 + i, 0, wl["T"], H)
+        if wl.get("verify"):  # positions of one sequence, as fill_tokens forms them
+            rho = wl["verify"]["rho"]
+            x[1:] = (np.float32(rho) * x[:1] + np.float32((1.0 - rho * rho) ** 0.5) * x[1:]).astype(np.float32)
         x = np.ascontiguousarray(x[:self.Ts])
         ids, _ = self.oracle.topk(self.oracle.router_logits(self.wr, self.bias, x), K, top_p=topp_arg())
         E = self.E
@@ -557,9 +596,7 @@ def run_ours(args, wl, ws, rank, local):
     xdt = torch.bfloat16 if wl["bf16"] else torch.float32
     xs = torch.empty((nsteps, T, H), dtype=xdt, device=dev)
     stream = torch.cuda.current_stream(dev)
-    for i in range(nsteps):
-        synth.x_dev(step_seed(i, 0 if ep else rank), 0, T, H, 1 if wl["bf16"] else 0, xs[i].data_ptr(),
-                    stream.cuda_stream)
+    fill_tokens(torch, synth, wl, xs, lambda i: step_seed(i, 0 if ep else rank), stream)
     y = torch.empty((T, H), dtype=xdt, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
@@ -665,6 +702,7 @@ def run_ours(args, wl, ws, rank, local):
         "gpu_launches": launches,
         "gpu_launches_note": "forward kernels in the timed loop; two clock-stamp kernels bracket the loop",
         "max_rel_err": err,
+        "verify": verify_report(wl, mean_unique + S, args.steps / (sum(step_ms) * 1e-3)) if wl.get("verify") else None,
         "compute": compute_desc(args.decode_kernel, T, tc),
         "e2e": {"value": round(job_tokens_per_s(1 if ep else ws, args.steps, T, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * H * xs.element_size(), "d2h_bytes_per_step": T * H * xs.element_size(),
@@ -876,8 +914,7 @@ def run_cached(args, wl, ws, rank, local):
     nsteps = args.warmup + args.steps
     stream = torch.cuda.current_stream(dev)
     xs = torch.empty((nsteps, T, H), dtype=torch.float32, device=dev)
-    for i in range(nsteps):
-        synth.x_dev(step_seed(i, rank), 0, T, H, 0, xs[i].data_ptr(), stream.cuda_stream)
+    fill_tokens(torch, synth, wl, xs, lambda i: step_seed(i, rank), stream)
     xw = torch.empty((T, H), dtype=torch.float32, device=dev)
     y = torch.empty((T, H), dtype=torch.float32, device=dev)
 
@@ -889,11 +926,14 @@ def run_cached(args, wl, ws, rank, local):
             layers[0].forward(x, y, stream=stream)
 
     # learning pass: routing counts per expert, then the hot set is pinned
-    n_learn = 400
-    xl = torch.empty((T, H), dtype=torch.float32, device=dev)
+    n_learn, n_cold = 400, 100
+    xl = torch.empty((n_learn, T, H), dtype=torch.float32, device=dev)
+    fill_tokens(torch, synth, wl, xl, lambda i: LEARN_SEED0 + i + 10_000 * rank, stream)
     for i in range(n_learn):
-        synth.x_dev(LEARN_SEED0 + i + 10_000 * rank, 0, T, H, 0, xl.data_ptr(), stream.cuda_stream)
-        step(xl)
+        step(xl[i])
+        if i == n_cold - 1:  # the first forwards from the initial placement: a cold cache
+            torch.cuda.synchronize(dev)
+            cold = [L.cache_stats() for L in layers]
     torch.cuda.synchronize(dev)
     for L in layers:
         L.pin_hot(wl["pin"])
@@ -956,6 +996,8 @@ def run_cached(args, wl, ws, rank, local):
             dist.destroy_process_group()
         return None
 
+    cold_hits = sum(x["hits"] for x in cold)
+    cold_misses = sum(x["misses"] for x in cold)
     hits = sum(x["hits"] for x in st)
     misses = sum(x["misses"] for x in st)
     h2d = sum(x["bytes_h2d"] for x in st)
@@ -984,6 +1026,9 @@ def run_cached(args, wl, ws, rank, local):
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
                    "expert_top_p": TOPP},
         "cache": {
+            "cold_hit_rate": round(cold_hits / max(cold_hits + cold_misses, 1), 4),
+            "cold_misses_per_step": round(cold_misses / n_cold, 3),
+            "cold_note": f"the first {n_cold} forwards of the learning pass, from experts 0..R-1 resident, no pins",
             "hit_rate": round(hits / max(hits + misses, 1), 4),
             "misses_per_step": round(misses / args.steps, 3),
             "needed_per_step": round(needed_per_step, 3),
@@ -1002,6 +1047,7 @@ def run_cached(args, wl, ws, rank, local):
                      "lookahead routing named"),
         },
         "hbm_bytes_per_step": int(hbm_bytes),
+        "verify": verify_report(wl, needed_per_step + NL * S, args.steps / secs) if wl.get("verify") else None,
         "stage_us": {k: round(v / max(nprof, 1) * 1e3, 2) for k, v in stages.items() if v > 0},
         "roofline": roof,
         "gpu_launches": launches,
