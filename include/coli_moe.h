@@ -378,9 +378,11 @@ coli_status coli_moe_set_trace(coli_moe_layer* layer, void* buffer, int capacity
 
 /*
  * Weight-streaming geometry of the persistent decode kernel: each SM keeps up
- * to `stages` bulk copies of `blocks_per_stage` x 4352 bytes in flight
- * (defaults 3 and 8; fewer if shared memory is short). stages in [2, 24],
- * blocks_per_stage even in [2, 8]. A tuning knob: results do not change.
+ * to `stages` bulk copies of at most `blocks_per_stage` x 4352 bytes in flight
+ * (defaults 3 and 16; what fits in shared memory beside the token operands:
+ * two copies of 16 blocks up to 32 tokens, three of 8 blocks above).
+ * stages in [2, 24], blocks_per_stage even in [2, 16]. A tuning knob: results
+ * do not change.
  */
 coli_status coli_moe_set_ring(coli_moe_layer* layer, int stages, int blocks_per_stage);
 

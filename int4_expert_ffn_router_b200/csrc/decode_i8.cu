@@ -35,7 +35,11 @@ namespace coli {
 namespace {
 
 constexpr int kSub = 8;                      // 16-row sub-tiles of a 128-row weight tile
-constexpr int kCW = 16;                      // consumer warps: two per sub-tile, on alternate blocks
+// One consumer warp per sub-tile: ten warps per CTA leave 158 registers per
+// thread, where two warps per sub-tile (on alternate blocks) left 96 and spilled
+// in the weight loop (measured 2.5% slower at batch 1, 5% at batch 8).
+constexpr int kWS = 1;                       // consumer warps per sub-tile
+constexpr int kCW = kSub * kWS;              // consumer warps
 constexpr int kCT = kCW * 32;                // consumer threads
 constexpr int kProducerWarp = kCW;
 constexpr int kSignalWarp = kCW + 1;
@@ -43,7 +47,8 @@ constexpr int kFT = (kCW + 2) * 32;          // all threads
 constexpr int kMaxSB = 8;                    // 4352-byte blocks per ring stage (at most)
 constexpr int kQ = 2;                        // item queue slots (lookahead of one item)
 constexpr int kSQ = 4;                       // completion records in flight to the signaler
-constexpr int kRouterExperts = kCW / 8;      // experts per router item (8 warps each, one pass over H/8)
+constexpr int kRouterExperts = 2;            // experts per router item (kCW / 2 warps each)
+static_assert(kWS == 1 || kWS == 2, "one or two consumer warps per sub-tile");
 constexpr int kChunkTok = 4;                 // tokens per 8-column MMA chunk (hi and lo parts)
 constexpr int kMetaRow = 16;                 // bytes of one group's data {2^-e, -8 sum(hi), -8 sum(lo), 0}
 // In shared memory each token slot's group data is followed by one unused
@@ -821,7 +826,7 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
     // ---- stream the weight tile through the ring
     if (a.trace && ctid == 0) S.t_loop0 = globaltimer_ns();
     float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-    const int sub = cw % kSub, half = cw / kSub;  // warps sub and sub + 8 share a sub-tile
+    const int sub = cw % kSub, half = cw / kSub;  // warps sub and sub + 8 (two per sub-tile) share a sub-tile
     const uint32_t stage_bytes = (uint32_t)a.sb * kBlockBytes;
     const int nst = (G + a.sb - 1) / a.sb;
     const int nch = (nt + kChunkTok - 1) / kChunkTok;
@@ -847,11 +852,11 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
             const int nb = min(a.sb, G - g0);
             if (nch == 1) {
 #pragma unroll 4
-                for (int bb = half; bb < nb; bb += 2)
+                for (int bb = half; bb < nb; bb += kWS)
                     block_mma<1>(stage + bb * kBlockBytes, blimb, bmeta, g0 + bb, G, sub, lane, nt, acc);
             } else {
 #pragma unroll 2
-                for (int bb = half; bb < nb; bb += 2)
+                for (int bb = half; bb < nb; bb += kWS)
                     block_mma<2>(stage + bb * kBlockBytes, blimb, bmeta, g0 + bb, G, sub, lane, nt, acc);
             }
         }
@@ -867,7 +872,7 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
     const bool aborted = S.aborted != 0;  // uniform: read after the barrier
     if (aborted) return;
     const bool lead = half == 0;  // the first warp of each sub-tile finishes the item
-    if (lead) {  // fixed order: blocks of the first warp, then those of the second
+    if (kWS == 2 && lead) {  // fixed order: blocks of the first warp, then those of the second
         const float4 o = *reinterpret_cast<const float4*>(S.accx[sub][lane]);
         acc[0][0] += o.x; acc[0][1] += o.y; acc[1][0] += o.z; acc[1][1] += o.w;
     }
@@ -1117,10 +1122,14 @@ int i8_ctl_ints_for(const Dims& d, int T) {
     return i8_ctl_ints(d.S * ((T + 3) / 4) + ncmax, d.H, ncmax);
 }
 
-// Ring geometry and item size for T tokens: 8 tokens per item when the B area
-// for them leaves room for at least three 34,816-byte copies in flight, else 4.
+// Ring geometry and item size for T tokens. Four-token items leave room for
+// the largest copies (two stages of up to 16 blocks, 69,632 bytes each: fewer
+// stage hand-offs per block); eight-token items stream a hot expert's weights
+// half as often but fit only smaller copies (three stages of 8 blocks). On a
+// B200 the first is faster up to 32 tokens, the second at 64 (Zipf routing).
 bool i8_geometry(const Dims& d, int T, size_t smem_limit, int max_stages, int max_sb, int* ntc, int* nstages, int* sb) {
-    for (int nt = (T > 4 ? 8 : 4); nt >= 4; nt -= 4) {
+    const int order[2] = {T > 32 ? 8 : 4, T > 32 ? 4 : (T > 4 ? 8 : 4)};
+    for (int nt : order) {
         for (int b = max_sb; b >= 2; b -= 2) {
             int ns = max_stages < kMaxStages ? max_stages : kMaxStages;
             while (ns > 0 && i8_smem_bytes(d, T, nt, ns, b) > smem_limit) --ns;

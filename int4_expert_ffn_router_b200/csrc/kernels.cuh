@@ -42,7 +42,7 @@ cudaError_t launch_down_core(const uint8_t* weights, const Dims& d, const float*
 // Persistent decode kernel ring defaults: bulk copies in flight per SM and
 // 4352-byte blocks per copy (coli_moe_set_ring).
 constexpr int kDefaultStages = 3;
-constexpr int kDefaultStageBlocks = 8;
+constexpr int kDefaultStageBlocks = 16;
 
 // decode_i8.cu: the whole layer for 1..kI8MaxTok tokens (at most kI8MaxSlots
 // routed slots) in one persistent launch of n_sm CTAs, on integer MMAs.

@@ -921,8 +921,8 @@ COLI_API coli_status coli_moe_set_tensor_cores(coli_moe_layer* L, int mode) {
 
 COLI_API coli_status coli_moe_set_ring(coli_moe_layer* L, int stages, int blocks_per_stage) {
     if (!L) return fail(COLI_EINVAL, "layer is NULL");
-    if (stages < 2 || stages > 24 || blocks_per_stage < 2 || blocks_per_stage > 8 || (blocks_per_stage & 1))
-        return fail(COLI_EINVAL, "stages in [2, 24], blocks_per_stage even in [2, 8]");
+    if (stages < 2 || stages > 24 || blocks_per_stage < 2 || blocks_per_stage > 16 || (blocks_per_stage & 1))
+        return fail(COLI_EINVAL, "stages in [2, 24], blocks_per_stage even in [2, 16]");
     L->ring_stages = stages;
     L->ring_blocks = blocks_per_stage;
     return COLI_OK;
