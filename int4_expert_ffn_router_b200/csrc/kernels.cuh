@@ -16,6 +16,16 @@ constexpr int kRouterGemmMinTok = 64;
 // (batches of kRouterGemmMinTok tokens and more use the blocked GEMM form).
 cudaError_t launch_router_logits(const float* wr, const float* bias, const void* x, coli_dtype dt, int T, int H, int E,
                                  double* logits, cudaStream_t st, double* part = nullptr, size_t part_cap = 0);
+// The router of token batches in fp32 with a certified selection (router_certified.cu):
+// logits in fp32 with a rigorous bound, the top-K set taken from them when the bound
+// separates it, the K selected logits recomputed in fp64 for the order and weights,
+// and every logit of the other tokens in fp64. Five kernels (and a driver memset).
+bool router_certified_supported(int H, int E);
+cudaError_t launch_router_norms(const float* wr, int H, int E, double* wn, cudaStream_t st);
+cudaError_t launch_router_certified(const float* wr, const double* wn, const float* bias, const void* x, coli_dtype dt,
+                                    int T, int H, int E, int K, double topp, int e_lo, int e_hi, float* l32,
+                                    double* xnorm, int* fail, double* logits, int32_t* ids, float* w, cudaStream_t st);
+constexpr int kRouterCertifiedSplit = 4;  // input-dimension ranges of the fp32 router (l32 holds one per range)
 // Kernels launch_router_logits enqueues for these arguments (0, 1 or 2).
 int router_kernel_count(int T, int H, int E, const double* part, size_t part_cap);
 // topp in (0, 1): adaptive expert top-p after the top-K (topk.cuh, topk_weights); else plain top-K.

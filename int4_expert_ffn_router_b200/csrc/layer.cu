@@ -134,6 +134,12 @@ struct coli_moe_layer {
     int* n_tiles = nullptr;
     unsigned* meta = nullptr;       // [0] max L1(gate row) * L1(up row), [1] max |scale| (float bits)
     double* rpart = nullptr;        // router partial sums (split input dimension)
+    // certified fp32 router of token batches (router_certified.cu)
+    bool cert_ok = false;           // shapes allow it and the workspace holds its buffers
+    float* l32 = nullptr;           // [max_tokens][E] fp32 logits
+    double* wnorm = nullptr;        // [E] ||Wr_e||_2, rounded up
+    int* cert_fail = nullptr;       // [1 + max_tokens]: count, then the tokens sent to the fp64 fallback
+    double* xnorm = nullptr;        // [max_tokens] ||x_t||_2
     size_t rpart_cap = 0;           // doubles
     bool tc_shape_ok = false;       // shapes and shared memory allow the tensor-core kernels
     bool tc_scale_ok = true;        // every weight scale keeps q * scale finite in fp16
@@ -406,7 +412,10 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
 
     // workspace
     const size_t TE = (size_t)Tm * d.E;
-    const size_t rpart_cap = std::max<size_t>(TE, std::min<size_t>(64 * TE, (size_t)1 << 23));  // <= 64 MB unless TE is larger
+    // batches of kRouterGemmMinTok tokens and more take the certified fp32 router when the
+    // shapes allow it; the split fp64 GEMM and its partial sums serve the others
+    const bool cert = Tm >= kRouterGemmMinTok && router_certified_supported(d.H, d.E);
+    const size_t rpart_cap = cert ? 0 : std::max<size_t>(TE, std::min<size_t>(64 * TE, (size_t)1 << 23));  // <= 64 MB unless TE is larger
     const size_t TK = (size_t)Tm * d.K, slots = TK + (size_t)d.S * Tm, EA = (size_t)d.E + d.S;
     // the integer-MMA kernel's batches: up to kI8MaxTok tokens and kI8MaxSlots routed slots
     const int Tf = (int)std::min<int64_t>(std::min<int64_t>(Tm, kI8MaxTok), kI8MaxSlots / d.K);
@@ -418,7 +427,10 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
                    (size_t)L->ctl_n * 4, 0, 2 * slots * d.H * 2, (size_t)Tm * 16,
                    slots * 16, (size_t)prefill_tc_max_tiles(d, Tm) * 16, 4, 16, rpart_cap * 8, (EA + 1) * 4,
                    (size_t)Tf * (d.H / 64) * 128, (size_t)Tf * (d.H / 64) * 16, slots_f * (d.I / 64) * 128,
-                   slots_f * (d.I / 64) * 16};
+                   slots_f * (d.I / 64) * 16,
+                   // certified router: fp32 logits, router row norms, fallback list
+                   cert ? (size_t)kRouterCertifiedSplit * Tm * d.E * 4 : 0, (size_t)d.E * 8, (size_t)(Tm + 1) * 4,
+                   cert ? (size_t)Tm * 8 : 0};
     constexpr int kRegions = sizeof(sz) / sizeof(sz[0]);
     size_t total = 0;
     for (size_t s : sz) total += align256(s);
@@ -440,6 +452,11 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
     L->xm = (uint8_t*)ptrs[27];
     L->hq = (uint8_t*)ptrs[28];
     L->hm = (uint8_t*)ptrs[29];
+    L->l32 = (float*)ptrs[30];
+    L->wnorm = (double*)ptrs[31];
+    L->cert_fail = (int*)ptrs[32];
+    L->xnorm = (double*)ptrs[33];
+    L->cert_ok = cert;
     L->rpart_cap = rpart_cap;
     {
         int optin = 0;
@@ -503,6 +520,7 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
     } else if ((e = cudaMemset(L->router_b, 0, (size_t)d.E * 4)) != cudaSuccess) {
         return bail(e, "clear bias");
     }
+    if ((e = launch_router_norms(L->router_w, d.H, d.E, L->wnorm, nullptr)) != cudaSuccess) return bail(e, "router norms");
     if (expert_q) {
         st = coli_moe_layer_set_experts(L, 0, d.E, expert_q, expert_scales);
         if (st != COLI_OK) { free_layer(L); return st; }
@@ -578,6 +596,26 @@ static coli_status check_call(const coli_moe_layer* L, const void* x, coli_dtype
     return COLI_OK;
 }
 
+// Router and top-K of a batch into ids/weights: batches of kRouterGemmMinTok
+// tokens and more take the certified fp32 router (fp64 only where the bound
+// does not settle the selection), smaller ones the fp64 GEMV and top-K.
+// Returns the number of kernels enqueued, or -1 on a launch error.
+static int route_batch(coli_moe_layer* L, const void* x, coli_dtype dt, int T, int32_t* ids, float* w, int e_lo,
+                       int e_hi, cudaStream_t s) {
+    const Dims& d = L->d;
+    if (L->cert_ok && T >= kRouterGemmMinTok) {
+        if (launch_router_certified(L->router_w, L->wnorm, L->router_b, x, dt, T, d.H, d.E, d.K, L->topp, e_lo, e_hi,
+                                    L->l32, L->xnorm, L->cert_fail, L->logits, ids, w, s) != cudaSuccess)
+            return -1;
+        return 5;
+    }
+    if (launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap) !=
+            cudaSuccess ||
+        launch_topk(L->logits, T, d.E, d.K, ids, w, s, L->topp, e_lo, e_hi) != cudaSuccess)
+        return -1;
+    return router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
+}
+
 COLI_API coli_status coli_moe_route(coli_moe_layer* L, const void* x, coli_dtype dt, int T, int32_t* ids,
                                     float* weights, coli_stream stream) {
     coli_status st = check_call(L, x, dt, T);
@@ -586,10 +624,9 @@ COLI_API coli_status coli_moe_route(coli_moe_layer* L, const void* x, coli_dtype
     if (T == 0) return COLI_OK;
     DeviceGuard guard(L->device);
     cudaStream_t s = (cudaStream_t)stream;
-    const Dims& d = L->d;
-    CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
-    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, ids, weights, s, L->topp), "topk");
-    L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
+    const int n = route_batch(L, x, dt, T, ids, weights, 0, L->d.E, s);
+    if (n < 0) return cuda_fail(cudaGetLastError(), "router");
+    L->launches += n;
     return COLI_OK;
 }
 
@@ -612,7 +649,6 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         coli_status st = prof_begin(L);
         if (st != COLI_OK) return st;
     }
-    const int router_launches = routed ? 0 : router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
     if (L->fused == 1 && T <= L->i8_max_tok && decode_i8_supported(d, T, L->smem_optin)) {
         prof_mark(L, COLI_STAGE_FUSED, s);
         I8Launch l{};
@@ -632,9 +668,9 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         const bool pairs = dt == COLI_F32;
         if (!routed) {
             prof_mark(L, COLI_STAGE_ROUTER, s);
-            CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
-            prof_mark(L, COLI_STAGE_TOPK, s);
-            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp, L->ep_lo, L->ep_hi), "topk");
+            const int n = route_batch(L, x, dt, T, p.ids, p.w, L->ep_lo, L->ep_hi, s);
+            if (n < 0) return cuda_fail(cudaGetLastError(), "router");
+            L->launches += n;
         }
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
@@ -661,14 +697,14 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
                  "down (tensor cores)");
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_prefill_out(L->o, residual, T, d.H, y, dt, s), "output");
-        // router, top-k, plan, prep, tile plan, two grouped GEMMs, output (the clear is a driver memset)
-        L->launches += router_launches + 6;
+        // plan, prep, tile plan, two grouped GEMMs, output (the clear is a driver memset; the router counted above)
+        L->launches += 6;
     } else {
         if (!routed) {
             prof_mark(L, COLI_STAGE_ROUTER, s);
-            CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap), "router");
-            prof_mark(L, COLI_STAGE_TOPK, s);
-            CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp, L->ep_lo, L->ep_hi), "topk");
+            const int n = route_batch(L, x, dt, T, p.ids, p.w, L->ep_lo, L->ep_hi, s);
+            if (n < 0) return cuda_fail(cudaGetLastError(), "router");
+            L->launches += n;
         }
         prof_mark(L, COLI_STAGE_PLAN, s);
         CUDA_TRY(launch_plan(p.ids, T, d.K, d.E, d.S, p, s), "plan");
@@ -678,7 +714,7 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         CUDA_TRY(launch_down_core(L->weights, d, L->h, T, p, L->o, L->max_active, L->n_sm, s), "down");
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_combine(L->o, p, T, d.H, d.K, d.S, residual, y, dt, s), "combine");
-        L->launches += router_launches + 4;
+        L->launches += 4;
     }
     prof_mark(L, COLI_N_STAGES, s);
     if (L->profiling) {
@@ -785,22 +821,17 @@ static coli_status cached_forward(coli_moe_layer* L, const void* x, void* y, col
     coli_status st = prof_begin(L);
     if (st != COLI_OK) return st;
     prof_mark(L, COLI_STAGE_ROUTER, s);
-    CUDA_TRY(launch_router_logits(L->router_w, L->router_b, x, dt, T, d.H, d.E, L->logits, s, L->rpart, L->rpart_cap),
-             "router");
-    prof_mark(L, COLI_STAGE_TOPK, s);
-    CUDA_TRY(launch_topk(L->logits, T, d.E, d.K, p.ids, p.w, s, L->topp, L->ep_lo, L->ep_hi), "topk");
-    L->launches += router_kernel_count(T, d.H, d.E, L->rpart, L->rpart_cap) + 1;
+    const int nr = route_batch(L, x, dt, T, p.ids, p.w, L->ep_lo, L->ep_hi, s);
+    if (nr < 0) return cuda_fail(cudaGetLastError(), "router");
+    L->launches += nr;
     prof_mark(L, COLI_STAGE_CACHE, s);
     const bool ahead = next && next != L && next->cached && next->lookahead && T <= next->cfg.max_tokens &&
                        next->d.H == d.H && next->device == L->device;
     if (ahead) {
         const Dims& dn = next->d;
-        CUDA_TRY(launch_router_logits(next->router_w, next->router_b, x, dt, T, dn.H, dn.E, next->logits, s,
-                                      next->rpart, next->rpart_cap),
-                 "lookahead router");
-        CUDA_TRY(launch_topk(next->logits, T, dn.E, dn.K, next->plan.ids, next->plan.w, s, next->topp),
-                 "lookahead topk");
-        next->launches += router_kernel_count(T, dn.H, dn.E, next->rpart, next->rpart_cap) + 1;
+        const int nn = route_batch(next, x, dt, T, next->plan.ids, next->plan.w, 0, dn.E, s);
+        if (nn < 0) return cuda_fail(cudaGetLastError(), "lookahead router");
+        next->launches += nn;
         CUDA_TRY(cudaMemcpyAsync(next->ahead_pin, next->plan.ids, (size_t)T * dn.K * 4, cudaMemcpyDeviceToHost, s),
                  "read predicted ids");
     }
