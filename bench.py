@@ -716,6 +716,10 @@ def run_ours(args, wl, ws, rank, local):
                 "method": E2E_METHOD},
         "clocks": clk,
     }
+    if T >= 64:  # batches of 64 tokens and more: the certified integer-MMA router, if the layer uses it
+        cert, n_fb = layer.router_fallbacks()
+        out["router"] = {"certified": cert, "fallback_tokens_last_batch": n_fb, "tokens_per_batch": T,
+                         "note": "tokens whose logits and top-K the certified router left to the fp64 fallback"}
     layer.close()
     if dist:
         dist.destroy_process_group()

@@ -287,6 +287,26 @@ coli_status coli_moe_get_plan(coli_moe_layer* layer, int32_t* ids, float* weight
                               int32_t* offsets, int32_t* unique, int32_t* n_unique, int32_t* pos, int32_t* tok);
 
 /*
+ * The certified router of token batches (batches of 64 tokens and more, on a
+ * device and with shapes that allow it: H a multiple of 16 in [128, 65536],
+ * E <= 256): router rows and tokens as four signed 8-bit digit planes under
+ * power-of-two row scales, every logit from one exact int8 tensor-core GEMM
+ * with a rigorous bound of its representation error, and the top-K, its
+ * order and its weights taken from those logits when the bounds prove them
+ * ("Colibri: 2400 lines of pure C ..." (kechuai.cn), section 一, defines the
+ * router and its top-K). A token whose selection the bounds do not settle (a
+ * near tie at or above the K-th place, a weight bound above 5e-7, with
+ * expert top-p a running sum within the bound of p, or a non-finite input)
+ * gets all of its logits and its top-K in fp64 instead.
+ * *certified: 1 when this layer routes such batches with it, else 0.
+ * *n: tokens of the last batch it routed that took the fp64 fallback (0 when
+ * it is not in use). Synchronises with the device: call after the routing
+ * finished (coli_moe_sync, or a synchronisation of the stream it ran on).
+ * Either output may be NULL.
+ */
+coli_status coli_moe_router_fallbacks(coli_moe_layer* layer, int32_t* certified, int32_t* n);
+
+/*
  * Per-stage device timing of forward calls, for profiling. While enabled,
  * every forward records CUDA events between its kernels on its own stream
  * (no host synchronisation; a ring of event sets is recycled, folding each

@@ -27,6 +27,7 @@ EXPORTS = (
     "coli_moe_debug_fail_alloc", "coli_clock_stamp", "coli_moe_debug_wait_test", "coli_moe_layer_create_cached",
     "coli_moe_cache_stats", "coli_moe_cache_pin", "coli_moe_cache_prefetch", "coli_moe_cache_set_lookahead",
     "coli_moe_cache_slots", "coli_moe_set_expert_top_p", "coli_moe_layer_create_ep", "coli_moe_ep_range",
+    "coli_moe_router_fallbacks",
 )
 NOALLOC_MAX_TOKENS, NOALLOC_MAX_EXPERTS = 63, 1024
 N_STAGES = 8
@@ -92,6 +93,7 @@ def _load() -> ctypes.CDLL:
     L.coli_moe_set_expert_top_p.argtypes = [vp, ctypes.c_double]
     L.coli_moe_layer_create_ep.argtypes = [pcfg, vp, vp, vp, vp, vp, vp, i32, i32, i32, ctypes.POINTER(vp)]
     L.coli_moe_ep_range.argtypes = [i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    L.coli_moe_router_fallbacks.argtypes = [vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
     L.coli_status_string.argtypes = [i32]
     L.coli_status_string.restype = ctypes.c_char_p
     L.coli_last_error.argtypes = []
@@ -194,6 +196,14 @@ class Layer:
         T = x.shape[0] if n_tokens is None else n_tokens
         _check(lib.coli_moe_route(self.handle, _ptr(x), _dtype_of(x), T, _ptr(ids), _ptr(weights), _stream(stream)),
                "coli_moe_route")
+
+    def router_fallbacks(self) -> tuple[bool, int]:
+        """(the certified router routes this layer's batches of 64 tokens and more,
+        tokens of its last batch that took the fp64 fallback); synchronises."""
+        c, n = ctypes.c_int32(), ctypes.c_int32()
+        _check(lib.coli_moe_router_fallbacks(self.handle, ctypes.byref(c), ctypes.byref(n)),
+               "coli_moe_router_fallbacks")
+        return bool(c.value), int(n.value)
 
     def forward(self, x, y, n_tokens: int | None = None, stream=None) -> None:
         T = x.shape[0] if n_tokens is None else n_tokens

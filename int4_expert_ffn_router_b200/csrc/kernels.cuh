@@ -16,16 +16,31 @@ constexpr int kRouterGemmMinTok = 64;
 // (batches of kRouterGemmMinTok tokens and more use the blocked GEMM form).
 cudaError_t launch_router_logits(const float* wr, const float* bias, const void* x, coli_dtype dt, int T, int H, int E,
                                  double* logits, cudaStream_t st, double* part = nullptr, size_t part_cap = 0);
-// The router of token batches in fp32 with a certified selection (router_certified.cu):
-// logits in fp32 with a rigorous bound, the top-K set taken from them when the bound
-// separates it, the K selected logits recomputed in fp64 for the order and weights,
-// and every logit of the other tokens in fp64. Five kernels (and a driver memset).
+// The router of token batches on the integer tensor cores with a certified
+// selection (router_certified.cu): Wr and x as four signed 8-bit digit planes
+// under power-of-two row scales, every logit from one exact int8 GEMM with a
+// rigorous bound of its representation error, the top-K, its order and its
+// weights taken from those logits where the bounds prove them, and the fp64
+// logits and top-K for the other tokens. Five kernels.
+struct RouterCert {
+    uint8_t* maps = nullptr;       // host: two CUtensorMap (router planes, batch planes), 64-byte aligned
+    uint8_t* wd8 = nullptr;        // [4][E][H] router digit planes
+    int* wscale = nullptr;         // [E] row scale exponents r_e
+    double* wb = nullptr;          // [E][3] ||Wr_e - wh_e||, ||wh_e||, rounding-bound factor
+    uint8_t* xd8 = nullptr;        // [4][Tm][H] batch digit planes
+    int* xscale = nullptr;         // [Tm] token scale exponents s_t
+    double* xb = nullptr;          // [Tm][3] ||x_t||, ||x_t - xh_t||, ||xh_t||
+    int* fail = nullptr;           // [1 + Tm]: count, then the tokens sent to the fp64 fallback
+    int Tm = 0, H = 0, E = 0;
+};
 bool router_certified_supported(int H, int E);
-cudaError_t launch_router_norms(const float* wr, int H, int E, double* wn, cudaStream_t st);
-cudaError_t launch_router_certified(const float* wr, const double* wn, const float* bias, const void* x, coli_dtype dt,
-                                    int T, int H, int E, int K, double topp, int e_lo, int e_hi, float* l32,
-                                    double* xnorm, int* fail, double* logits, int32_t* ids, float* w, cudaStream_t st);
-constexpr int kRouterCertifiedSplit = 4;  // input-dimension ranges of the fp32 router (l32 holds one per range)
+size_t router_certified_smem_bytes();
+// Digit planes and bound factors of the router rows, the tensor maps (once).
+cudaError_t router_certified_prepare(RouterCert& rc, const float* wr, cudaStream_t st);
+// err: timeout site of the GEMM's bounded waits (control block).
+cudaError_t launch_router_certified(const RouterCert& rc, const float* wr, const float* bias, const void* x,
+                                    coli_dtype dt, int T, int K, double topp, int e_lo, int e_hi, double* logits,
+                                    int32_t* ids, float* w, int* err, cudaStream_t st);
 // Kernels launch_router_logits enqueues for these arguments (0, 1 or 2).
 int router_kernel_count(int T, int H, int E, const double* part, size_t part_cap);
 // topp in (0, 1): adaptive expert top-p after the top-K (topk.cuh, topk_weights); else plain top-K.

@@ -134,12 +134,10 @@ struct coli_moe_layer {
     int* n_tiles = nullptr;
     unsigned* meta = nullptr;       // [0] max L1(gate row) * L1(up row), [1] max |scale| (float bits)
     double* rpart = nullptr;        // router partial sums (split input dimension)
-    // certified fp32 router of token batches (router_certified.cu)
-    bool cert_ok = false;           // shapes allow it and the workspace holds its buffers
-    float* l32 = nullptr;           // [max_tokens][E] fp32 logits
-    double* wnorm = nullptr;        // [E] ||Wr_e||_2, rounded up
-    int* cert_fail = nullptr;       // [1 + max_tokens]: count, then the tokens sent to the fp64 fallback
-    double* xnorm = nullptr;        // [max_tokens] ||x_t||_2
+    // certified integer-MMA router of token batches (router_certified.cu)
+    bool cert_ok = false;           // shapes and device allow it and the workspace holds its buffers
+    RouterCert rc;
+    alignas(64) unsigned char rc_maps[2 * kTensorMapBytes] = {};  // TMA maps of its digit planes
     size_t rpart_cap = 0;           // doubles
     bool tc_shape_ok = false;       // shapes and shared memory allow the tensor-core kernels
     bool tc_scale_ok = true;        // every weight scale keeps q * scale finite in fp16
@@ -395,6 +393,9 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
     d.d_bytes = matrix_bytes(d.H, d.I);
     d.expert_stride = (int64_t)align256((size_t)(d.gu_bytes + d.d_bytes));
     cudaDeviceGetAttribute(&L->n_sm, cudaDevAttrMultiProcessorCount, device);
+    int cc_major = 0, optin = 0;
+    cudaDeviceGetAttribute(&cc_major, cudaDevAttrComputeCapabilityMajor, device);
+    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
     const int Tm = d.max_tokens;
     L->max_active = (int)std::min<int64_t>((int64_t)Tm * d.K, d.E) + d.S;
 
@@ -412,9 +413,10 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
 
     // workspace
     const size_t TE = (size_t)Tm * d.E;
-    // batches of kRouterGemmMinTok tokens and more take the certified fp32 router when the
-    // shapes allow it; the split fp64 GEMM and its partial sums serve the others
-    const bool cert = Tm >= kRouterGemmMinTok && router_certified_supported(d.H, d.E);
+    // batches of kRouterGemmMinTok tokens and more take the certified integer-MMA router when
+    // the shapes and the device allow it; the split fp64 GEMM and its partial sums serve the others
+    const bool cert = Tm >= kRouterGemmMinTok && router_certified_supported(d.H, d.E) && cc_major == 10 &&
+                      (size_t)optin >= router_certified_smem_bytes();
     const size_t rpart_cap = cert ? 0 : std::max<size_t>(TE, std::min<size_t>(64 * TE, (size_t)1 << 23));  // <= 64 MB unless TE is larger
     const size_t TK = (size_t)Tm * d.K, slots = TK + (size_t)d.S * Tm, EA = (size_t)d.E + d.S;
     // the integer-MMA kernel's batches: up to kI8MaxTok tokens and kI8MaxSlots routed slots
@@ -428,9 +430,11 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
                    slots * 16, (size_t)prefill_tc_max_tiles(d, Tm) * 16, 4, 16, rpart_cap * 8, (EA + 1) * 4,
                    (size_t)Tf * (d.H / 64) * 128, (size_t)Tf * (d.H / 64) * 16, slots_f * (d.I / 64) * 128,
                    slots_f * (d.I / 64) * 16,
-                   // certified router: fp32 logits, router row norms, fallback list
-                   cert ? (size_t)kRouterCertifiedSplit * Tm * d.E * 4 : 0, (size_t)d.E * 8, (size_t)(Tm + 1) * 4,
-                   cert ? (size_t)Tm * 8 : 0};
+                   // certified router: batch digit planes, token scales, fallback list, token norms,
+                   // router digit planes, expert scales, expert bound factors
+                   cert ? (size_t)4 * Tm * d.H : 0, cert ? (size_t)Tm * 4 : 0, cert ? (size_t)(Tm + 1) * 4 : 0,
+                   cert ? (size_t)Tm * 24 : 0, cert ? (size_t)4 * d.E * d.H : 0, cert ? (size_t)d.E * 4 : 0,
+                   cert ? (size_t)d.E * 24 : 0};
     constexpr int kRegions = sizeof(sz) / sizeof(sz[0]);
     size_t total = 0;
     for (size_t s : sz) total += align256(s);
@@ -452,19 +456,22 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
     L->xm = (uint8_t*)ptrs[27];
     L->hq = (uint8_t*)ptrs[28];
     L->hm = (uint8_t*)ptrs[29];
-    L->l32 = (float*)ptrs[30];
-    L->wnorm = (double*)ptrs[31];
-    L->cert_fail = (int*)ptrs[32];
-    L->xnorm = (double*)ptrs[33];
+    L->rc.maps = L->rc_maps;
+    L->rc.xd8 = (uint8_t*)ptrs[30];
+    L->rc.xscale = (int*)ptrs[31];
+    L->rc.fail = (int*)ptrs[32];
+    L->rc.xb = (double*)ptrs[33];
+    L->rc.wd8 = (uint8_t*)ptrs[34];
+    L->rc.wscale = (int*)ptrs[35];
+    L->rc.wb = (double*)ptrs[36];
+    L->rc.Tm = Tm;
+    L->rc.H = d.H;
+    L->rc.E = d.E;
     L->cert_ok = cert;
     L->rpart_cap = rpart_cap;
     {
-        int optin = 0;
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
         L->smem_optin = (size_t)optin;
         L->fused = (Tf > 0 && decode_i8_supported(d, 1, L->smem_optin)) ? 1 : 0;
-        int cc_major = 0;
-        cudaDeviceGetAttribute(&cc_major, cudaDevAttrComputeCapabilityMajor, device);
         L->tc_shape_ok = cc_major == 10 && d.H % 256 == 0 && d.I % 128 == 0 && L->smem_optin >= prefill_tc_smem_bytes();
     }
     if (L->tc_shape_ok) {
@@ -520,7 +527,8 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
     } else if ((e = cudaMemset(L->router_b, 0, (size_t)d.E * 4)) != cudaSuccess) {
         return bail(e, "clear bias");
     }
-    if ((e = launch_router_norms(L->router_w, d.H, d.E, L->wnorm, nullptr)) != cudaSuccess) return bail(e, "router norms");
+    if (L->cert_ok && (e = router_certified_prepare(L->rc, L->router_w, nullptr)) != cudaSuccess)
+        return bail(e, "router digit planes");
     if (expert_q) {
         st = coli_moe_layer_set_experts(L, 0, d.E, expert_q, expert_scales);
         if (st != COLI_OK) { free_layer(L); return st; }
@@ -597,15 +605,15 @@ static coli_status check_call(const coli_moe_layer* L, const void* x, coli_dtype
 }
 
 // Router and top-K of a batch into ids/weights: batches of kRouterGemmMinTok
-// tokens and more take the certified fp32 router (fp64 only where the bound
-// does not settle the selection), smaller ones the fp64 GEMV and top-K.
+// tokens and more take the certified integer-MMA router (fp64 only where the
+// bounds do not settle the selection), smaller ones the fp64 GEMV and top-K.
 // Returns the number of kernels enqueued, or -1 on a launch error.
 static int route_batch(coli_moe_layer* L, const void* x, coli_dtype dt, int T, int32_t* ids, float* w, int e_lo,
                        int e_hi, cudaStream_t s) {
     const Dims& d = L->d;
     if (L->cert_ok && T >= kRouterGemmMinTok) {
-        if (launch_router_certified(L->router_w, L->wnorm, L->router_b, x, dt, T, d.H, d.E, d.K, L->topp, e_lo, e_hi,
-                                    L->l32, L->xnorm, L->cert_fail, L->logits, ids, w, s) != cudaSuccess)
+        if (launch_router_certified(L->rc, L->router_w, L->router_b, x, dt, T, d.K, L->topp, e_lo, e_hi, L->logits, ids,
+                                    w, L->ctl + kCtlError, s) != cudaSuccess)
             return -1;
         return 5;
     }
@@ -990,6 +998,17 @@ COLI_API coli_status coli_moe_get_launch_count(const coli_moe_layer* L, int64_t*
     if (!L) return fail(COLI_EINVAL, "layer is NULL");
     if (!n) return fail(COLI_EINVAL, "n is NULL");
     *n = L->launches;
+    return COLI_OK;
+}
+
+COLI_API coli_status coli_moe_router_fallbacks(coli_moe_layer* L, int32_t* certified, int32_t* n) {
+    if (!L) return fail(COLI_EINVAL, "layer is NULL");
+    if (certified) *certified = L->cert_ok ? 1 : 0;
+    if (!n) return COLI_OK;
+    *n = 0;
+    if (!L->cert_ok) return COLI_OK;
+    DeviceGuard guard(L->device);
+    CUDA_TRY(cudaMemcpy(n, L->rc.fail, 4, cudaMemcpyDeviceToHost), "read fallback count");
     return COLI_OK;
 }
 

@@ -1,46 +1,82 @@
-// router_certified.cu -- the router of token batches in fp32 with a certified
-// selection, recomputing in fp64 only what the selection cannot settle.
+// router_certified.cu -- the router of token batches on the integer tensor
+// cores, with a certified selection and fp64 only where the certificate fails.
 //
-// The router and its top-K are those of router.cu (fp64 logits, K largest,
-// equal logits to the lower id, softmax over the K): "Colibri: 2400 lines of
-// pure C ..." (kechuai.cn), section 一. The fp64 GEMM of a 2048-token batch
-// is bound by the FP64 rate; this form computes the logits in fp32 with a
-// known summation order and a rigorous error bound per logit, and the set of
-// the K largest logits is taken from the fp32 values only when the bound
-// proves it is the set of the exact logits:
-//   |v_e - l_e| <= eps_e = c * ||Wr_e||_2 * ||x_t||_2   (c from the order)
-//   min over the selected (v - eps) > max over the others (v + eps)
-// => every selected exact logit exceeds every other one, so the selection of
-// the exact (and of any fp64) logits is the same set. The order within the
-// set and the weights then come from the K selected logits recomputed in
-// fp64. A token whose bound does not separate the set (a near tie at the
-// K-th place) gets all of its logits in fp64 and the fp64 top-K.
+// The router and its top-K are those of router.cu (logits Wr x + b, the K
+// largest, equal logits to the lower id, softmax over the K): "Colibri: 2400
+// lines of pure C ..." (kechuai.cn), section 一. An fp64 GEMM of a 2048-token
+// batch is bound by the FP64 rate; this form computes every logit exactly up
+// to a tiny, rigorously bounded representation error:
+//
+//   x_t ~ xh_t = 2^s_t * qx_t,  qx_t integers, |qx| < 2^30 (per-token scale)
+//   Wr_e ~ wh_e = 2^r_e * qw_e,  qw_e integers, |qw| < 2^30 (per-expert scale)
+//   each q as four signed base-256 digits d_0 .. d_3 (d_0 most significant):
+//     q = d_0 2^24 + d_1 2^16 + d_2 2^8 + d_3,  every d in [-128, 127]
+//
+// One int8 tensor-core GEMM (tcgen05.mma kind::i8, exact int32 accumulation)
+// forms all 16 digit products P_pq = sum_h dw_p[h] dx_q[h] of a (token,
+// expert) pair; sum_pq 2^(8(6-p-q)) P_pq = qw . qx exactly, and
+//   v = 2^(s+r) (qw . qx) + b   (fp64, three additions and the bias rounded)
+// differs from the exact logit by at most
+//   eps = ||Wr_e - wh_e|| ||x_t|| + ||wh_e|| ||x_t - xh_t||
+//         + 7u max|Wr_e| sqrt(H) ||xh_t|| + 2u |v|,   u = 2^-53
+// (norms in fp64, rounded up). The scales keep the largest element of a row
+// in [2^29, 2^30), so fp32 and bf16 values at most 2^6 below a row's largest
+// are represented exactly; eps is about 1e-9 of ||Wr_e|| ||x_t||. A token is
+// certified when its K selected intervals [v - eps, v + eps] lie strictly
+// above every other expert's and strictly ordered among themselves, and the
+// weights' error bound (at most 2.01 max eps relative) stays below 5e-7
+// (with top-p, no running sum within that bound of p). Then the ids and their
+// order are those of the exact logits, and of any fp64 evaluation that does
+// not itself hit such a tie; the weights come from v. Any other token gets all
+// of its logits in fp64 and the fp64 top-K, as router.cu computes them.
+#include <cuda.h>
+
+#include <cfloat>
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tcgen05.cuh"
 #include "topk.cuh"
 
 namespace coli {
 namespace {
 
-// fp32 GEMM: CTA tile 64 tokens x 128 experts x one of kCfSplit ranges of
-// the input dimension, 256 threads; thread (ty, tx) owns tokens 8ty..8ty+7
-// and experts 4tx..4tx+3. Each output sums kCfBlk inputs at a time by
-// sequential FMAs from 0 into `part`, then adds `part` to `tot`; the
-// kCfSplit range sums are added in fp64 by the certify kernel. The error of a
-// logit is at most
-//   (gamma_kCfBlk + gamma_(blocks per range - 1) (1 + gamma_kCfBlk)) * sum |w x|
-// (plus the fp64 additions, far below).
-constexpr int kCfT = 64, kCfE = 128, kCfK = 16, kCfBlk = 128, kCfSplit = 4, kCfThreads = 256;
+// GEMM tile: 32 experts x 4 digit planes = 128 rows of A (the MMA's M) and
+// 64 tokens x 4 digit planes = 256 rows of B (its N); 128 inputs (bytes) of
+// the input dimension per pipeline stage, four K = 32 MMAs each.
+constexpr int kRxE = 32, kRxT = 64, kRxK = 128;
+constexpr int kRxM = 4 * kRxE, kRxN = 4 * kRxT;
+constexpr int kRxStages = 2;
+constexpr int kRxABytes = kRxM * kRxK;                 // 16 KB
+constexpr int kRxBBytes = kRxN * kRxK;                 // 32 KB
+constexpr int kRxStageBytes = kRxABytes + kRxBBytes;   // 48 KB
+constexpr int kRxStageOut = 4 * kRxT * kRxE * 8;       // epilogue: the four digit-plane terms, fp64
+static_assert(kRxStageOut <= kRxStages * kRxStageBytes, "the epilogue reuses the pipeline buffers");
+constexpr int kRxOffBar = kRxStages * kRxStageBytes;
+constexpr int kRxSmem = kRxOffBar + 64 + 1024;         // barriers, tensor-memory slot, flag, alignment slack
+constexpr int kRxThreads = 192;                        // producer, MMA, four epilogue warps
+constexpr uint32_t kRxTmemCols = 256;
+constexpr uint64_t kRxWaitNs = 1000000000ull;          // every wait gives up after 1 s
+
+// Error-bound constants (u = 2^-53): the three fp64 additions of the digit
+// terms, at most 3.01u of sum |term| <= 2.02 max|Wr_e| sqrt(H) ||xh_t||, with
+// margin; the bias addition; the norms' own rounding (fp64 sums of at most
+// 2^16 squares).
+constexpr double kRxAddBound = 7.0 * 1.1102230246251565e-16;
+constexpr double kRxBiasBound = 2.3e-16;
+constexpr double kRxNormUp = 1.0 + 1e-10;
+constexpr double kRxWeightTol = 5e-7;
 
 template <typename XT>
-__device__ __forceinline__ void cf_load8(const XT* p, float v[8]);
+__device__ __forceinline__ void rx_load8(const XT* p, float v[8]);
 template <>
-__device__ __forceinline__ void cf_load8<float>(const float* p, float v[8]) {
+__device__ __forceinline__ void rx_load8<float>(const float* p, float v[8]) {
     const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 template <>
-__device__ __forceinline__ void cf_load8<__nv_bfloat16>(const __nv_bfloat16* p, float v[8]) {
+__device__ __forceinline__ void rx_load8<__nv_bfloat16>(const __nv_bfloat16* p, float v[8]) {
     const uint4 u = *reinterpret_cast<const uint4*>(p);
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -50,169 +86,379 @@ __device__ __forceinline__ void cf_load8<__nv_bfloat16>(const __nv_bfloat16* p, 
     }
 }
 
-template <typename XT>
-__global__ void __launch_bounds__(kCfThreads, 2) router_f32_kernel(const float* __restrict__ wr, const XT* __restrict__ x,
-                                                            int T, int H, int E, float* __restrict__ l32) {
-    __shared__ __align__(16) float xs[2][kCfK][kCfT];  // 8 KB, k-major
-    __shared__ __align__(16) float ws[2][kCfK][kCfE];  // 16 KB, k-major
-    const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
-    const int t0 = blockIdx.x * kCfT, e0 = blockIdx.y * kCfE;
-    const int hspan = H / kCfSplit, h0 = blockIdx.z * hspan;
-    // loaders: x row tid / 4, inputs 4 (tid & 3) .. +3; Wr row tid / 2, inputs 8 (tid & 1) .. +7
-    const int xr = tid >> 2, xk = (tid & 3) * 4, wrow = tid >> 1, wk = (tid & 1) * 8;
-    const bool xok = t0 + xr < T, wok = e0 + wrow < E;
-    const XT* xp = x + (size_t)(xok ? t0 + xr : 0) * H + h0 + xk;
-    const float* wp = wr + (size_t)(wok ? e0 + wrow : 0) * H + h0 + wk;
-    float xv[4], wv[8];
-    auto fetch = [&](int k0) {
-        if (xok) {
-            if constexpr (sizeof(XT) == 4) {
-                const float4 f = *reinterpret_cast<const float4*>(xp + k0);
-                xv[0] = f.x; xv[1] = f.y; xv[2] = f.z; xv[3] = f.w;
-            } else {
-                const uint2 u = *reinterpret_cast<const uint2*>(xp + k0);
-                xv[0] = __uint_as_float(u.x << 16); xv[1] = __uint_as_float(u.x & 0xFFFF0000u);
-                xv[2] = __uint_as_float(u.y << 16); xv[3] = __uint_as_float(u.y & 0xFFFF0000u);
-            }
-        } else {
-            xv[0] = xv[1] = xv[2] = xv[3] = 0.0f;
-        }
-        if (wok) {
-            cf_load8<float>(wp + k0, wv);
-        } else {
+// The four signed base-256 digits of q (|q| < 2^30) as the bytes of one word,
+// byte k the digit of weight 2^8k: adding 128 at each of the three low digit
+// positions makes every low digit d + 128 an ordinary byte (0..255) and leaves
+// the top digit in the arithmetic top byte; xor 0x80 takes 128 off again.
+__device__ __forceinline__ uint32_t rx_digits(int q) { return (uint32_t)(q + 0x808080) ^ 0x808080u; }
+
+// Byte transpose of four digit words (elements 0..3) into four plane words:
+// plane word k holds byte k of each element, element i in byte i.
+__device__ __forceinline__ void rx_planes4(const uint32_t w[4], uint32_t out[4]) {
+    const uint32_t lo01 = __byte_perm(w[0], w[1], 0x5140), lo23 = __byte_perm(w[2], w[3], 0x5140);
+    const uint32_t hi01 = __byte_perm(w[0], w[1], 0x7362), hi23 = __byte_perm(w[2], w[3], 0x7362);
+    out[0] = __byte_perm(lo01, lo23, 0x5410);
+    out[1] = __byte_perm(lo01, lo23, 0x7632);
+    out[2] = __byte_perm(hi01, hi23, 0x5410);
+    out[3] = __byte_perm(hi01, hi23, 0x7632);
+}
+
+// Block-wide fp64 sums over 256 threads; `red` holds 8 x 4 doubles.
+__device__ __forceinline__ void rx_block_sum3(double& a, double& b, double& c, double* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) wv[i] = 0.0f;
-        }
-    };
-    auto stash = [&](int b) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) xs[b][xk + i][xr] = xv[i];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ws[b][wk + i][wrow] = wv[i];
-    };
-    float part[8][4], tot[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) part[i][j] = tot[i][j] = 0.0f;
-    const int nk = hspan / kCfK;
-    fetch(0);
-    stash(0);
+    for (int o = 16; o > 0; o >>= 1) {
+        a += __shfl_xor_sync(0xffffffffu, a, o);
+        b += __shfl_xor_sync(0xffffffffu, b, o);
+        c += __shfl_xor_sync(0xffffffffu, c, o);
+    }
     __syncthreads();
-    for (int c = 0; c < nk; ++c) {
-        const int b = c & 1;
-        if (c + 1 < nk) fetch((c + 1) * kCfK);
+    if (lane == 0) { red[4 * warp] = a; red[4 * warp + 1] = b; red[4 * warp + 2] = c; }
+    __syncthreads();
+    a = b = c = 0.0;
+    for (int w = 0; w < 8; ++w) { a += red[4 * w]; b += red[4 * w + 1]; c += red[4 * w + 2]; }
+}
+
+// One CTA (256 threads) per row of n values (n % 8 == 0): the power-of-two
+// scale 2^s that puts the row's largest magnitude in [2^29, 2^30), the four
+// digit planes of the row scaled by 2^-s and rounded to integers (plane p at
+// out + p * plane), and the norms ||v||, ||v - vh||, ||vh|| rounded up. A row
+// holding a non-finite value gets a NaN norm (its logits then fail every
+// certificate) and zero digits.
+template <typename XT>
+__device__ __forceinline__ void rx_split_row(const XT* __restrict__ row, int n, uint8_t* __restrict__ out,
+                                             size_t plane, int* scale, double* nv, double* nd, double* nq,
+                                             float* vmax) {
+    __shared__ unsigned smax;
+    __shared__ int sbad;
+    __shared__ double red[32];
+    if (threadIdx.x == 0) { smax = 0u; sbad = 0; }
+    __syncthreads();
+    float m = 0.0f;
+    bool bad = false;
+    for (int h = 8 * threadIdx.x; h < n; h += 8 * blockDim.x) {
+        float v[8];
+        rx_load8<XT>(row + h, v);
 #pragma unroll
-        for (int k = 0; k < kCfK; ++k) {
-            const float4 xa = *reinterpret_cast<const float4*>(&xs[b][k][8 * ty]);
-            const float4 xb = *reinterpret_cast<const float4*>(&xs[b][k][8 * ty + 4]);
-            const float4 wa = *reinterpret_cast<const float4*>(&ws[b][k][4 * tx]);
-            const float xq[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-            const float wq[4] = {wa.x, wa.y, wa.z, wa.w};
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) part[i][j] = fmaf(wq[j], xq[i], part[i][j]);
+        for (int i = 0; i < 8; ++i) {
+            const float a = fabsf(v[i]);
+            bad |= !(a <= FLT_MAX);
+            m = fmaxf(m, a);
         }
-        if (((c + 1) * kCfK) % kCfBlk == 0 || c + 1 == nk) {  // end of a summation block
+    }
+    atomicMax(&smax, __float_as_uint(m));
+    if (bad) sbad = 1;
+    __syncthreads();
+    const float amax = __uint_as_float(smax);
+    const bool any_bad = sbad != 0;
+    int ex = 0;
+    if (amax > 0.0f && !any_bad) frexpf(amax, &ex);  // amax = f 2^ex, f in [0.5, 1)
+    const int s = (amax > 0.0f && !any_bad) ? ex - 30 : 0;
+    // y = v 2^-s exactly (fp64; s in [-180, 130]), q = rint(y), y - q exact:
+    // ||v - vh||^2 = 2^2s sum (y - q)^2, ||vh||^2 = 2^2s sum q^2
+    const double down = __longlong_as_double((long long)(1023 - s) << 52);
+    double sv = 0.0, sd = 0.0, sq = 0.0;
+    for (int h = 8 * threadIdx.x; h < n; h += 8 * blockDim.x) {
+        float v[8];
+        rx_load8<XT>(row + h, v);
+        uint32_t wd[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 8; ++i) {
+            const double xv = (double)v[i];
+            const double y = any_bad ? 0.0 : xv * down;
+            const double yr = rint(y);
+            const double res = y - yr;
+            sv = fma(xv, xv, sv);
+            sd = fma(res, res, sd);
+            sq = fma(yr, yr, sq);
+            wd[i] = rx_digits((int)yr);
+        }
+        uint32_t pa[4], pb[4];  // plane words of elements 0..3 and 4..7; byte 3 is digit d_0 (plane 0)
+        rx_planes4(wd, pa);
+        rx_planes4(wd + 4, pb);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    tot[i][j] += part[i][j];
-                    part[i][j] = 0.0f;
+        for (int p = 0; p < 4; ++p)
+            *reinterpret_cast<uint2*>(out + (size_t)p * plane + h) = make_uint2(pa[3 - p], pb[3 - p]);
+    }
+    const double up2 = __longlong_as_double((long long)(1023 + 2 * s) << 52);
+    sd *= up2;
+    sq *= up2;
+    rx_block_sum3(sv, sd, sq, red);
+    if (threadIdx.x == 0) {
+        *scale = s;
+        *nv = any_bad ? __longlong_as_double(0x7ff8000000000000ll) : sqrt(sv) * kRxNormUp;
+        *nd = sqrt(sd) * kRxNormUp;
+        *nq = sqrt(sq) * kRxNormUp;
+        if (vmax) *vmax = amax;
+    }
+}
+
+// Digit planes of the router rows (once, when the weights are loaded):
+// wd8 [4][E][H], scale r_e, and the per-expert bound factors
+// wb[e] = {||Wr_e - wh_e||, ||wh_e||, 7u max|Wr_e| sqrt(H)}.
+__global__ void __launch_bounds__(256) router_split_w_kernel(const float* __restrict__ wr, int E, int H,
+                                                             uint8_t* __restrict__ wd8, int* __restrict__ wscale,
+                                                             double* __restrict__ wb) {
+    const int e = blockIdx.x;
+    __shared__ float wmax;
+    double nv;
+    rx_split_row<float>(wr + (size_t)e * H, H, wd8 + (size_t)e * H, (size_t)E * H, wscale + e, &nv, wb + 3 * e,
+                        wb + 3 * e + 1, &wmax);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // wb[3e] was ||Wr_e - wh_e||; a non-finite row makes every bound NaN
+        if (nv != nv) wb[3 * e] = nv;
+        wb[3 * e + 2] = kRxAddBound * (double)wmax * sqrt((double)H) * kRxNormUp;
+    }
+}
+
+// Digit planes of a token batch: xd8 [4][Tm][H] (plane stride Tm * H), scale
+// s_t, and xb[t] = {||x_t||, ||x_t - xh_t||, ||xh_t||}. CTA 0 also clears the
+// fallback count of this call.
+template <typename XT>
+__global__ void __launch_bounds__(256) router_split_x_kernel(const XT* __restrict__ x, int T, int H, int Tm,
+                                                             uint8_t* __restrict__ xd8, int* __restrict__ xscale,
+                                                             double* __restrict__ xb, int* __restrict__ fail) {
+    const int t = blockIdx.x;
+    if (t == 0 && threadIdx.x == 0) *fail = 0;
+    rx_split_row<XT>(x + (size_t)t * H, H, xd8 + (size_t)t * H, (size_t)Tm * H, xscale + t, xb + 3 * t,
+                     xb + 3 * t + 1, xb + 3 * t + 2, nullptr);
+}
+
+// TMA tile load of box (x, y, z) of a 3D tensor map (no multicast).
+__device__ __forceinline__ void rx_tma_3d(uint32_t dst, const void* tmap, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Four MMAs (K = 32 each, one 128-byte stage row) of int8 digits into the
+// int32 accumulator, then one commit to `bar`. Warp-converged: one elected
+// lane issues.
+__device__ __forceinline__ void rx_mma4_commit(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate,
+                                               uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred e, p, t;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+        "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], a1, b1, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], a2, b2, %3, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::i8 [%0], a3, b3, %3, t;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(bar)
+        : "memory");
+}
+
+// Instruction descriptor of kind::i8: D s32 (bits 4-5 = 2), A and B signed
+// 8-bit (bits 7-9, 10-12 = 1), both K-major, N / 8 at bit 17, M / 16 at bit 24.
+__host__ __device__ constexpr uint32_t rx_idesc_s8(int m, int n) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ bool rx_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site) {
+    if (mbar_try_wait_sleep(bar, parity, 200000)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, 200000)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kRxWaitNs) {
+            *abort_flag = 1;
+            atomicCAS(err, 0, site);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ bool rx_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
+                                             int site) {
+    const bool ok = rx_wait(bar, parity, abort_flag, err, site);
+    return __all_sync(0xffffffffu, ok);
+}
+
+struct __align__(64) RxArgs {
+    CUtensorMap wmap;  // digit planes of the router rows: dims (H, E, 4), box (128, 32, 1)
+    CUtensorMap xmap;  // digit planes of the batch: dims (H, Tm, 4), box (128, 64, 1)
+    const int* wscale;
+    const int* xscale;
+    const float* bias;
+    double* logits;    // [T][E]
+    int T, H, E;
+    int* err;
+};
+
+// CTA (bx, by): experts 32 bx .. +31, tokens 64 by .. +63. Warp 0 (one lane)
+// loads each stage's 4 + 4 digit boxes with TMA; warp 1 allocates the
+// accumulator (128 lanes x 256 int32 columns: lane 32 p + e, column 64 q + t)
+// and issues the MMAs; warps 2..5 (lane quarter p = warp % 4) read it back:
+// term_p(t, e) = 2^(8(3-p)) sum_q 2^(8(3-q)) P_pq, exact in fp64 (below
+// 2^53), staged in shared memory, then v = ((term_0 + term_1) + term_2) +
+// term_3 scaled by 2^(s_t + r_e), plus the bias.
+__global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_constant__ RxArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kRxOffBar);  // [kRxStages]
+    uint64_t* empty = full + kRxStages;                              // [kRxStages]
+    uint64_t* accfull = empty + kRxStages;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e0 = blockIdx.x * kRxE, t0 = blockIdx.y * kRxT;
+    const int nkb = (a.H + kRxK - 1) / kRxK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kRxStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accfull, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        tc_alloc(tmem_slot, kRxTmemCols);
+        tc_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int kb = 0;
+            for (; kb < nkb; ++kb) {
+                const int s = kb % kRxStages;
+                if (!rx_wait(&empty[s], ((kb / kRxStages) & 1) ^ 1, abort_flag, a.err, 41)) break;
+                uint8_t* st = sm + s * kRxStageBytes;
+                mbar_arrive_expect_tx(&full[s], kRxStageBytes);
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    rx_tma_3d(smem_addr(st + p * (kRxE * kRxK)), &a.wmap, kb * kRxK, e0, p, &full[s]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    rx_tma_3d(smem_addr(st + kRxABytes + q * (kRxT * kRxK)), &a.xmap, kb * kRxK, t0, q, &full[s]);
+            }
+            // copies still in flight (after an abort) land before the CTA exits
+            const int first = kb > kRxStages ? kb - kRxStages : 0;
+            const uint64_t tw = globaltimer_ns();
+            for (int k = first; k < kb; ++k)
+                while (!mbar_try_wait(&full[k % kRxStages], (k / kRxStages) & 1) && globaltimer_ns() - tw < kRxWaitNs) {
                 }
         }
-        if (c + 1 < nk) {
-            stash(b ^ 1);
-            __syncthreads();
+        __syncwarp();
+    } else if (warp == 1) {
+        const uint32_t idesc = rx_idesc_s8(kRxM, kRxN);
+        const uint64_t adesc0 = tc_sdesc_sw128(smem_addr(sm));
+        bool issued = false;
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % kRxStages;
+            if (!rx_wait_warp(&full[s], (kb / kRxStages) & 1, abort_flag, a.err, 42)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t ad = adesc0 + (uint64_t)((s * kRxStageBytes) >> 4);
+            const uint64_t bd = ad + (uint64_t)(kRxABytes >> 4);
+            rx_mma4_commit(tmem, ad, bd, idesc, kb != 0, smem_addr(&empty[s]));
+            issued = true;
+        }
+        if (issued) {
+            // accfull completes when every MMA issued above has completed (also after an abort,
+            // so the tensor memory is never released under a running MMA)
+            tc_commit_elect(accfull);
+            const uint64_t tw = globaltimer_ns();
+            while (!mbar_try_wait(accfull, 0) && globaltimer_ns() - tw < kRxWaitNs) {
+            }
+        }
+        __syncwarp();
+    } else {
+        const int p = warp & 3;
+        double* stage = reinterpret_cast<double*>(sm);  // [4][kRxT][kRxE]
+        ok = rx_wait_warp(accfull, 0, abort_flag, a.err, 43) && !*abort_flag;
+        if (ok) {
+            tc_fence_after();
+            const uint32_t tl = tmem + ((uint32_t)(32 * p) << 16);
+            const double wp = p == 0 ? 16777216.0 : p == 1 ? 65536.0 : p == 2 ? 256.0 : 1.0;
+#pragma unroll 1
+            for (int c = 0; c < kRxT / 16; ++c) {
+                uint32_t v0[16], v1[16], v2[16], v3[16];
+                tc_ld16_wait(tl + 0 * kRxT + 16 * c, v0);
+                tc_ld16_wait(tl + 1 * kRxT + 16 * c, v1);
+                tc_ld16_wait(tl + 2 * kRxT + 16 * c, v2);
+                tc_ld16_wait(tl + 3 * kRxT + 16 * c, v3);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const long long sp = ((long long)(int)v0[i] << 24) + ((long long)(int)v1[i] << 16) +
+                                         ((long long)(int)v2[i] << 8) + (long long)(int)v3[i];
+                    stage[((size_t)p * kRxT + 16 * c + i) * kRxE + lane] = (double)sp * wp;
+                }
+            }
+        }
+        // the four epilogue warps (128 threads) meet; the pipeline buffers now hold the terms
+        named_bar(1, 128);
+        const bool all_ok = ok && !*abort_flag;
+        if (all_ok) {
+            const int e = e0 + lane;
+            const bool ein = e < a.E;
+            const int r = ein ? __ldg(a.wscale + e) : 0;
+            const double b = ein ? (double)__ldg(a.bias + e) : 0.0;
+            for (int tt = warp - 2; tt < kRxT; tt += 4) {
+                const int t = t0 + tt;
+                if (t >= a.T || !ein) continue;
+                const double v = ((stage[(0 * kRxT + tt) * kRxE + lane] + stage[(1 * kRxT + tt) * kRxE + lane]) +
+                                  stage[(2 * kRxT + tt) * kRxE + lane]) +
+                                 stage[(3 * kRxT + tt) * kRxE + lane];
+                a.logits[(size_t)t * a.E + e] = ldexp(v, __ldg(a.xscale + t) + r) + b;
+            }
         }
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int t = t0 + 8 * ty + i;
-        if (t >= T) continue;
-        const int e = e0 + 4 * tx;
-        float* dst = l32 + ((size_t)blockIdx.z * T + t) * E + e;
-        if (e + 3 < E) *reinterpret_cast<float4*>(dst) = make_float4(tot[i][0], tot[i][1], tot[i][2], tot[i][3]);
-        else
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (e + j < E) dst[j] = tot[i][j];
-    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tc_dealloc(tmem, kRxTmemCols);
 }
 
-// ||Wr_e||_2, rounded up (fp64 sum of squares, square root, one ulp up).
-__global__ void router_norm_kernel(const float* __restrict__ wr, int H, int E, double* __restrict__ wn) {
-    const int e = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (e >= E) return;
-    double s = 0.0;
-    for (int h = lane; h < H; h += 32) s = fma((double)wr[(size_t)e * H + h], (double)wr[(size_t)e * H + h], s);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) wn[e] = sqrt(s) * (1.0 + 1e-14);
-}
-
-// One warp per token: the K largest of the fp32 logits (plus bias, in fp64),
-// the certificate, then either the K logits in fp64 with their order and
-// weights, or the token on the list of tokens for the fp64 fallback.
-// ||x_t||_2 in fp64, rounded up, one warp per token.
-template <typename XT>
-__global__ void __launch_bounds__(256) token_norm_kernel(const XT* __restrict__ x, int T, int H, double* __restrict__ xn) {
-    const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (t >= T) return;
-    double ss = 0.0;
-    for (int h = 8 * lane; h < H; h += 256) {
-        float v[8];
-        cf_load8<XT>(x + (size_t)t * H + h, v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ss = fma((double)v[i], (double)v[i], ss);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) xn[t] = sqrt(ss) * (1.0 + 1e-14);
-}
-
-template <typename XT>
-__global__ void __launch_bounds__(256) router_certify_kernel(const float* __restrict__ l32, const double* __restrict__ wn,
-                                                             const double* __restrict__ xnorm,
-                                                             const float* __restrict__ wr, const float* __restrict__ bias,
-                                                             const XT* __restrict__ x, int T, int H, int E, int K,
-                                                             double c_bound, double topp, int e_lo, int e_hi,
+// One warp per token: the bound of each logit, the K largest (descending,
+// equal values to the lower id), the certificate, then either the ids and
+// weights (adaptive top-p included) or the token on the fallback list.
+__global__ void __launch_bounds__(256) router_certify_kernel(const double* __restrict__ logits,
+                                                             const double* __restrict__ wb,
+                                                             const double* __restrict__ xb, int T, int E, int K,
+                                                             double topp, int e_lo, int e_hi,
                                                              int32_t* __restrict__ ids, float* __restrict__ w,
                                                              int* __restrict__ fail) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + warp;
     if (t >= T) return;
-    const XT* xrow = x + (size_t)t * H;
-    const double xn = xnorm[t];
-    // this lane's experts lane + 32 i (i < 8): value and bound
-    unsigned long long k8[8];
-    int id8[8];
+    const double xn = xb[3 * t], xd = xb[3 * t + 1], xq = xb[3 * t + 2];
+    auto bound = [&](int e, double v) {
+        return (wb[3 * e] * xn + wb[3 * e + 1] * xd + wb[3 * e + 2] * xq) * (1.0 + 1e-9) + kRxBiasBound * fabs(v) +
+               1e-300;
+    };
+    // this lane's experts lane + 32 i (i < 8): key and interval
+    unsigned long long ks[8];
+    int is[8];
     double lo8[8], hi8[8];
+    bool present[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int e = lane + 32 * i;
-        k8[i] = 0ull;
-        id8[i] = 0x7fffffff;
+        present[i] = e < E;
+        ks[i] = 0ull;
+        is[i] = 0x7fffffff;
         lo8[i] = hi8[i] = 0.0;
-        if (e < E) {
-            double v = (double)bias[e];
-#pragma unroll
-            for (int z = 0; z < kCfSplit; ++z) v += (double)l32[((size_t)z * T + t) * E + e];
-            const double eps = c_bound * wn[e] * xn * (1.0 + 1e-12) + fabs(v) * 4.5e-16 + 1e-300;
-            k8[i] = order_key(v);
-            id8[i] = e;
+        if (present[i]) {
+            const double v = logits[(size_t)t * E + e];
+            const double eps = bound(e, v);
+            ks[i] = order_key(v);
+            is[i] = e;
             lo8[i] = v - eps;
             hi8[i] = v + eps;
         }
     }
-    // the K largest values (descending, equal values to the lower id): each lane sorts its
-    // 8 entries, then K rounds take the warp's best head
-    unsigned long long ks[8];
-    int is[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) { ks[i] = k8[i]; is[i] = id8[i]; }
+    // the K largest: each lane sorts its 8 entries, then K rounds take the warp's best head
     cx8(ks, is, 0, 1); cx8(ks, is, 2, 3); cx8(ks, is, 4, 5); cx8(ks, is, 6, 7);
     cx8(ks, is, 0, 2); cx8(ks, is, 1, 3); cx8(ks, is, 4, 6); cx8(ks, is, 5, 7);
     cx8(ks, is, 1, 2); cx8(ks, is, 5, 6);
@@ -220,7 +466,8 @@ __global__ void __launch_bounds__(256) router_certify_kernel(const float* __rest
     cx8(ks, is, 2, 4); cx8(ks, is, 3, 5);
     cx8(ks, is, 1, 2); cx8(ks, is, 3, 4); cx8(ks, is, 5, 6);
     int my_id = -1;
-    unsigned selmask = 0u;  // which of this lane's entries were selected (expert lane + 32 i: bit i)
+    unsigned long long my_key = 0ull, top_key = 0ull;
+    unsigned selmask = 0u;  // this lane's selected entries (expert lane + 32 i: bit i)
     for (int r = 0; r < K; ++r) {
         const unsigned khi = (unsigned)(ks[0] >> 32), klo = (unsigned)ks[0];
         const unsigned bhi = __reduce_max_sync(0xffffffffu, khi);
@@ -234,77 +481,53 @@ __global__ void __launch_bounds__(256) router_certify_kernel(const float* __rest
             ks[7] = 0ull;
             is[7] = 0x7fffffff;
         }
-        if (lane == r) my_id = bi;
+        const unsigned long long bk = ((unsigned long long)bhi << 32) | blo;
+        if (r == 0) top_key = bk;
+        if (lane == r) { my_id = bi; my_key = bk; }
     }
-    // certificate: every selected lower bound above every other upper bound
+    // certificate 1: every selected interval above every other one
     double sel_lo = 1e300, oth_hi = -1e300;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        if (id8[i] == 0x7fffffff) continue;
+        if (!present[i]) continue;
         if ((selmask >> i) & 1u) sel_lo = fmin(sel_lo, lo8[i]);
         else oth_hi = fmax(oth_hi, hi8[i]);
     }
+    // certificate 2: the selected intervals strictly ordered; the largest bound among them
+    const bool mine = lane < K && my_id >= 0 && my_id < E;
+    const double my_v = mine ? key_value(my_key) : 0.0;
+    const double my_eps = mine ? bound(my_id, my_v) : 0.0;
+    const double next_hi = __shfl_down_sync(0xffffffffu, my_v + my_eps, 1);
+    bool ok = lane >= K - 1 || (mine && my_v - my_eps > next_hi);
+    double m = my_eps;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         sel_lo = fmin(sel_lo, __shfl_xor_sync(0xffffffffu, sel_lo, o));
         oth_hi = fmax(oth_hi, __shfl_xor_sync(0xffffffffu, oth_hi, o));
+        m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
     }
-    if (!(sel_lo > oth_hi)) {  // not separated: every logit of this token in fp64 (fallback kernels)
+    // certificate 3: the weights' error bound (relative 2.01 m), and with top-p no running
+    // sum of the weights within that bound of p
+    ok = __all_sync(0xffffffffu, ok) && sel_lo > oth_hi && 2.01 * m <= kRxWeightTol;
+    if (ok && topp > 0.0 && topp < 1.0) {
+        const double ex = lane < K ? exp(my_v - key_value(top_key)) : 0.0;
+        double z = ex;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        const double wk = ex / z;
+        double cum = 0.0;
+        for (int j = 0; j < K; ++j) {
+            cum += __shfl_sync(0xffffffffu, wk, j);
+            ok = ok && fabs(cum - topp) > 2.01 * m + 1e-12;
+        }
+    }
+    if (!ok) {
         if (lane == 0) fail[1 + atomicAdd(fail, 1)] = t;
         return;
     }
-    // the selected logits in fp64, eight at a time by the whole warp: lane l sums inputs
-    // 4l + 128 i (i = 0, 1, ...) of each, then a fixed xor tree
-    double my_l = 0.0;
-    for (int k0 = 0; k0 < K; k0 += 8) {
-        int ek[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) ek[j] = __shfl_sync(0xffffffffu, my_id, (k0 + j) & 31);
-        double sj[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        for (int h = 4 * lane; h < H; h += 128) {
-            float xv[4];
-            if constexpr (sizeof(XT) == 4) {
-                const float4 f = *reinterpret_cast<const float4*>(xrow + h);
-                xv[0] = f.x; xv[1] = f.y; xv[2] = f.z; xv[3] = f.w;
-            } else {
-                const uint2 u = *reinterpret_cast<const uint2*>(xrow + h);
-                xv[0] = __uint_as_float(u.x << 16); xv[1] = __uint_as_float(u.x & 0xFFFF0000u);
-                xv[2] = __uint_as_float(u.y << 16); xv[3] = __uint_as_float(u.y & 0xFFFF0000u);
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                if (k0 + j >= K) continue;
-                const float4 w4 = *reinterpret_cast<const float4*>(wr + (size_t)ek[j] * H + h);
-                sj[j] = fma((double)w4.x, (double)xv[0], sj[j]);
-                sj[j] = fma((double)w4.y, (double)xv[1], sj[j]);
-                sj[j] = fma((double)w4.z, (double)xv[2], sj[j]);
-                sj[j] = fma((double)w4.w, (double)xv[3], sj[j]);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sj[j] += __shfl_xor_sync(0xffffffffu, sj[j], o);
-            if (lane == k0 + j && k0 + j < K) my_l = sj[j] + (double)bias[ek[j]];
-        }
-    }
-    // order among the selected: rank by (fp64 logit descending, id ascending)
-    const unsigned long long my_key = lane < K ? order_key(my_l) : 0ull;
-    int rank = 0;
-    for (int k = 0; k < K; ++k) {
-        const unsigned long long ok = __shfl_sync(0xffffffffu, my_key, k);
-        const int oi = __shfl_sync(0xffffffffu, my_id, k);
-        rank += ok > my_key || (ok == my_key && oi < my_id);
-    }
-    // lane r takes the entry of rank r
-    int src = 0;
-    for (int k = 0; k < K; ++k) src = __shfl_sync(0xffffffffu, rank, k) == lane ? k : src;
-    const unsigned long long skey = __shfl_sync(0xffffffffu, my_key, src);
-    const int sid = __shfl_sync(0xffffffffu, my_id, src);
-    const unsigned long long top = __shfl_sync(0xffffffffu, skey, 0);
     int id;
     float wt;
-    topk_weights(lane < K ? skey : 0ull, top, lane < K ? sid : -1, K, topp, lane, &id, &wt);
+    topk_weights(lane < K ? my_key : 0ull, top_key, lane < K ? my_id : -1, K, topp, lane, &id, &wt);
     if (lane < K) {
         ids[(size_t)t * K + lane] = (id >= e_lo && id < e_hi) ? id : -1;
         w[(size_t)t * K + lane] = wt;
@@ -361,8 +584,7 @@ __global__ void __launch_bounds__(256) router_fallback_topk_kernel(const double*
         const int t = fail[1 + f];
         int id;
         float wt;
-        if (E <= 256) warp_topk8<true>(logits + (size_t)t * E, E, K, topp, lane, &id, &wt);
-        else warp_topk<true>(logits + (size_t)t * E, E, K, topp, lane, &id, &wt);
+        warp_topk8<true>(logits + (size_t)t * E, E, K, topp, lane, &id, &wt);
         if (lane < K) {
             ids[(size_t)t * K + lane] = (id >= e_lo && id < e_hi) ? id : -1;
             w[(size_t)t * K + lane] = wt;
@@ -370,50 +592,87 @@ __global__ void __launch_bounds__(256) router_fallback_topk_kernel(const double*
     }
 }
 
-double gamma_n(int n) {
-    const double u = 1.0 / 16777216.0;  // 2^-24
-    return n * u / (1.0 - n * u);
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// 3D int8 map over four digit planes of rows x H bytes (plane stride rows *
+// H): box 128 bytes x box_rows rows x 1 plane, 128-byte swizzle, zero fill
+// outside the tensor.
+cudaError_t rx_encode(void* map, const uint8_t* base, int rows, int H, int box_rows) {
+    static EncodeFn encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+        encode = reinterpret_cast<EncodeFn>(fn);
+    }
+    if (((uintptr_t)base & 15u) || H % 16 || rows < 1) return cudaErrorInvalidValue;
+    const cuuint64_t dims[3] = {(cuuint64_t)H, (cuuint64_t)rows, 4};
+    const cuuint64_t strides[2] = {(cuuint64_t)H, (cuuint64_t)rows * H};
+    const cuuint32_t box[3] = {(cuuint32_t)kRxK, (cuuint32_t)box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = encode(reinterpret_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                              const_cast<uint8_t*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-bool router_certified_supported(int H, int E) { return H % (kCfSplit * kCfBlk) == 0 && E <= 256; }
+bool router_certified_supported(int H, int E) { return H % 16 == 0 && H >= kRxK && H <= 65536 && E >= 1 && E <= 256; }
 
-cudaError_t launch_router_norms(const float* wr, int H, int E, double* wn, cudaStream_t st) {
-    router_norm_kernel<<<(E + 7) / 8, 256, 0, st>>>(wr, H, E, wn);
-    return cudaGetLastError();
+size_t router_certified_smem_bytes() { return kRxSmem; }
+
+cudaError_t router_certified_prepare(RouterCert& rc, const float* wr, cudaStream_t st) {
+    if (!router_certified_supported(rc.H, rc.E) || rc.Tm < 1) return cudaErrorInvalidValue;
+    router_split_w_kernel<<<rc.E, 256, 0, st>>>(wr, rc.E, rc.H, rc.wd8, rc.wscale, rc.wb);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if ((e = rx_encode(rc.maps, rc.wd8, rc.E, rc.H, kRxE)) != cudaSuccess) return e;
+    if ((e = rx_encode(rc.maps + sizeof(CUtensorMap), rc.xd8, rc.Tm, rc.H, kRxT)) != cudaSuccess) return e;
+    return cudaFuncSetAttribute(router_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRxSmem);
 }
 
-cudaError_t launch_router_certified(const float* wr, const double* wn, const float* bias, const void* x, coli_dtype dt,
-                                    int T, int H, int E, int K, double topp, int e_lo, int e_hi, float* l32,
-                                    double* xnorm, int* fail, double* logits, int32_t* ids, float* w, cudaStream_t st) {
+cudaError_t launch_router_certified(const RouterCert& rc, const float* wr, const float* bias, const void* x,
+                                    coli_dtype dt, int T, int K, double topp, int e_lo, int e_hi, double* logits,
+                                    int32_t* ids, float* w, int* err, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    if (e_hi < 0) e_hi = E;
-    const int nb = H / kCfSplit / kCfBlk;  // summation blocks per range
-    // fp32 sums, plus the fp64 additions of the ranges and the bias
-    const double c = gamma_n(kCfBlk) + gamma_n(nb - 1) * (1.0 + gamma_n(kCfBlk)) + 1e-15;
-    cudaError_t e = cudaMemsetAsync(fail, 0, sizeof(int), st);
-    if (e != cudaSuccess) return e;
-    dim3 g((T + kCfT - 1) / kCfT, (E + kCfE - 1) / kCfE, kCfSplit);
-    if (dt == COLI_F32) router_f32_kernel<float><<<g, kCfThreads, 0, st>>>(wr, (const float*)x, T, H, E, l32);
-    else router_f32_kernel<__nv_bfloat16><<<g, kCfThreads, 0, st>>>(wr, (const __nv_bfloat16*)x, T, H, E, l32);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (dt == COLI_F32) token_norm_kernel<float><<<(T + 7) / 8, 256, 0, st>>>((const float*)x, T, H, xnorm);
-    else token_norm_kernel<__nv_bfloat16><<<(T + 7) / 8, 256, 0, st>>>((const __nv_bfloat16*)x, T, H, xnorm);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (T > rc.Tm || K < 1 || K > 32) return cudaErrorInvalidValue;
+    if (e_hi < 0) e_hi = rc.E;
+    const int H = rc.H, E = rc.E;
     if (dt == COLI_F32)
-        router_certify_kernel<float><<<(T + 7) / 8, 256, 0, st>>>(l32, wn, xnorm, wr, bias, (const float*)x, T, H, E, K,
-                                                                  c, topp, e_lo, e_hi, ids, w, fail);
+        router_split_x_kernel<float><<<T, 256, 0, st>>>((const float*)x, T, H, rc.Tm, rc.xd8, rc.xscale, rc.xb, rc.fail);
     else
-        router_certify_kernel<__nv_bfloat16><<<(T + 7) / 8, 256, 0, st>>>(l32, wn, xnorm, wr, bias,
-                                                                          (const __nv_bfloat16*)x, T, H, E, K, c, topp,
-                                                                          e_lo, e_hi, ids, w, fail);
+        router_split_x_kernel<__nv_bfloat16><<<T, 256, 0, st>>>((const __nv_bfloat16*)x, T, H, rc.Tm, rc.xd8,
+                                                                rc.xscale, rc.xb, rc.fail);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    RxArgs a;
+    memcpy(&a.wmap, rc.maps, sizeof(CUtensorMap));
+    memcpy(&a.xmap, rc.maps + sizeof(CUtensorMap), sizeof(CUtensorMap));
+    a.wscale = rc.wscale;
+    a.xscale = rc.xscale;
+    a.bias = bias;
+    a.logits = logits;
+    a.T = T;
+    a.H = H;
+    a.E = E;
+    a.err = err;
+    const dim3 g((E + kRxE - 1) / kRxE, (T + kRxT - 1) / kRxT);
+    router_i8_kernel<<<g, kRxThreads, kRxSmem, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    dim3 gf((E + 1) / 2, 64);
-    if (dt == COLI_F32) router_fallback_kernel<float><<<gf, 256, 0, st>>>(wr, bias, (const float*)x, H, E, fail, logits);
-    else router_fallback_kernel<__nv_bfloat16><<<gf, 256, 0, st>>>(wr, bias, (const __nv_bfloat16*)x, H, E, fail, logits);
+    router_certify_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, rc.wb, rc.xb, T, E, K, topp, e_lo, e_hi, ids, w,
+                                                       rc.fail);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    router_fallback_topk_kernel<<<16, 256, 0, st>>>(logits, E, K, topp, e_lo, e_hi, fail, ids, w);
+    const dim3 gf((E + 1) / 2, 4);
+    if (dt == COLI_F32) router_fallback_kernel<float><<<gf, 256, 0, st>>>(wr, bias, (const float*)x, H, E, rc.fail, logits);
+    else router_fallback_kernel<__nv_bfloat16><<<gf, 256, 0, st>>>(wr, bias, (const __nv_bfloat16*)x, H, E, rc.fail, logits);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    router_fallback_topk_kernel<<<16, 256, 0, st>>>(logits, E, K, topp, e_lo, e_hi, rc.fail, ids, w);
     return cudaGetLastError();
 }
 

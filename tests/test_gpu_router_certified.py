@@ -1,13 +1,14 @@
-"""GPU parity of the router of token batches (64 tokens and more): logits in
-fp32 with a rigorous error bound per logit, the top-K set taken from them when
-the bound separates it from the other experts, the K selected logits then
-recomputed in fp64 for their order and weights, and every logit of the other
-tokens (near ties at the K-th place) recomputed in fp64.
+"""GPU parity of the router of token batches (64 tokens and more): router rows
+and tokens as four signed 8-bit digit planes under power-of-two row scales,
+every logit from one exact int8 tensor-core GEMM with a rigorous bound of its
+representation error, the top-K set, its order and its weights taken from
+those logits where the bounds prove them, and every logit of the other tokens
+(near ties) recomputed in fp64.
 
 The ids and their order must equal the fp64 oracle's bit for bit, also for
-tokens whose selection the bound cannot settle: router rows that are exact or
-near copies of each other (relative difference 2^-20, far below the fp32
-bound) put such ties at the boundary.
+tokens whose selection the bounds cannot settle: router rows that are exact
+copies of each other put exact ties at the boundary (fallback), and rows that
+differ by a relative 2^-20 put near ties there that the bounds must resolve.
 """
 import numpy as np
 import pytest
@@ -60,15 +61,18 @@ def test_certified_router_matches_the_oracle(gpu, coli, T, bf16):
     ids_ref, w_ref = oracle.topk(oracle.router_logits(L["wr"], bias, x), c["K"])
     np.testing.assert_array_equal(ids, ids_ref)
     np.testing.assert_allclose(w, w_ref, rtol=0, atol=1e-6)
+    # random logits: the bounds (about 1e-9 of ||Wr_e|| ||x_t||) settle every token
+    assert layer.router_fallbacks() == (True, 0)
     layer.close()
 
 
 @pytest.mark.parametrize("T", [64, 300])
 def test_near_ties_at_the_boundary_fall_back_to_fp64(gpu, coli, T):
     """Rows 1 and 2 are exact copies of row 0, rows 4 and 5 near copies of row
-    3 (relative 2^-20): whenever such a pair straddles the K-th place the
-    fp32 bound cannot separate it, and the fp64 fallback decides (equal
-    logits to the lower id)."""
+    3 (relative 2^-20): an exact pair within or at the edge of the top-K has
+    equal logits, which no bound separates, so the fp64 fallback decides
+    (equal logits to the lower id); the near copies differ by far more than
+    the bounds and are settled by them."""
     c = dict(cases.TINY, E=32, K=4)
     L = cases.host_layer(c, seed=32)
     wr = L["wr"].copy()
@@ -89,10 +93,43 @@ def test_near_ties_at_the_boundary_fall_back_to_fp64(gpu, coli, T):
     rows = [set(r) for r in ids_ref.tolist()]
     assert any((0 in r) != (1 in r) or (1 in r) != (2 in r) for r in rows)
     assert any((3 in r) != (4 in r) or (3 in r) != (5 in r) for r in rows)
+    # some tokens went to the fp64 fallback, and only tokens with a copied row among their
+    # K + 1 largest logits (random rows leave no other near tie)
+    certified, n_fb = layer.router_fallbacks()
+    lg = oracle.router_logits(wr, None, x)
+    order = np.argsort(-lg, axis=1, kind="stable")
+    near = sum(1 for t in range(T) if {0, 1, 2, 3, 4, 5} & set(order[t, :c["K"] + 1].tolist()))
+    assert certified and 0 < n_fb <= near
     # and the forward takes the same routing
     yd = torch.empty((T, c["H"]), device=gpu)
     layer.set_fused(False)
     layer.forward(torch.from_numpy(x).to(gpu), yd)
     layer.sync()
     np.testing.assert_array_equal(layer.plan(T)["ids"], ids_ref)
+    layer.close()
+
+
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_extreme_and_zero_rows(gpu, coli, with_bias):
+    """Row scales at the ends of the fp32 range (1e30, 1e-30, all-subnormal
+    rows) exercise the per-token power-of-two scale; an all-zero row has
+    logits equal to the bias, or, without bias, all equal, which no bound
+    separates (fp64 fallback: the K lowest ids, equal weights)."""
+    c = dict(cases.TINY, E=64, K=8)
+    bias = synth.zipf_bias(33, 0, c["E"])[0] if with_bias else None
+    L = cases.host_layer(c, seed=33, bias=bias)
+    T = 96
+    layer = _layer(coli, c, L["wr"], L, T)
+    x = synth.x_f32(33, T, T, c["H"]).copy()
+    x[3] = 0.0
+    x[10] *= np.float32(1e30)
+    x[20] *= np.float32(1e-30)
+    x[30] = (x[30].astype(np.float64) * 2.0 ** -140).astype(np.float32)  # subnormal fp32 row
+    ids, w = _route(coli, layer, x, gpu, c["K"])
+    ids_ref, w_ref = oracle.topk(oracle.router_logits(L["wr"], bias, x), c["K"])
+    np.testing.assert_array_equal(ids, ids_ref)
+    np.testing.assert_allclose(w, w_ref, rtol=0, atol=1e-6)
+    if not with_bias:
+        np.testing.assert_array_equal(ids[3], np.arange(c["K"]))
+        assert layer.router_fallbacks()[1] >= 1
     layer.close()
