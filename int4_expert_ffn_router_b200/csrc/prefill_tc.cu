@@ -33,6 +33,7 @@
 // rounded once to fp16 (relative error <= 2^-11); all sums are fp32.
 #include <cuda.h>
 
+#include <algorithm>
 #include <cstring>
 
 #include "common.cuh"
@@ -478,10 +479,13 @@ __global__ void prefill_prep_kernel(const XT* __restrict__ x, int T, int H, int 
             const double hb = bound * (double)mx * (double)mx;
             if (hb > 0.0) f = min(120, max(-120, ilogb(16384.0 / hb)));
         }
-        int dst[32 + 64];  // positions of this token (K <= 32 routed + S <= 64 shared)
+        // positions of this token (K <= 32 routed, then S <= 64 shared): position q is held
+        // by lane q % 32 in dst_r[q / 32] and broadcast with a shuffle
         const int np = K + S;
-        for (int k = 0; k < K; ++k) dst[k] = pos[(size_t)t * K + k];
-        for (int j = 0; j < S; ++j) dst[K + j] = T * K + j * T + t;
+        auto position = [&](int q) { return q < K ? pos[(size_t)t * K + q] : T * K + (q - K) * T + t; };
+        int dst_r[3];
+#pragma unroll
+        for (int r = 0; r < 3; ++r) dst_r[r] = 32 * r + lane < np ? position(32 * r + lane) : -1;
         for (int i = lane * kV; i < H; i += 32 * kV) {
             float v[kV];
             load8(row + i, v);
@@ -498,13 +502,14 @@ __global__ void prefill_prep_kernel(const XT* __restrict__ x, int T, int H, int 
             }
             const uint4 hv = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
             for (int q = 0; q < np; ++q) {
-                if (dst[q] < 0) continue;  // an empty slot (expert of another rank)
+                const int d = __shfl_sync(0xffffffffu, q < 32 ? dst_r[0] : q < 64 ? dst_r[1] : dst_r[2], q & 31);
+                if (d < 0) continue;  // an empty slot (expert of another rank)
                 if constexpr (kF32) {
-                    reinterpret_cast<uint4*>(xs + (size_t)(2 * dst[q]) * H + i)[0] = hv;
-                    reinterpret_cast<uint4*>(xs + (size_t)(2 * dst[q] + 1) * H + i)[0] =
+                    reinterpret_cast<uint4*>(xs + (size_t)(2 * d) * H + i)[0] = hv;
+                    reinterpret_cast<uint4*>(xs + (size_t)(2 * d + 1) * H + i)[0] =
                         make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
                 } else {
-                    reinterpret_cast<uint4*>(xs + (size_t)dst[q] * H + i)[0] = hv;
+                    reinterpret_cast<uint4*>(xs + (size_t)d * H + i)[0] = hv;
                 }
             }
         }
@@ -512,8 +517,9 @@ __global__ void prefill_prep_kernel(const XT* __restrict__ x, int T, int H, int 
     }
 }
 
-// Per-position epilogue factors and the tile list (one CTA). Tiles hold at
-// most kTcMaxTok tokens of one expert and are ordered by decreasing size.
+// Per-position epilogue factors (every CTA, grid-stride) and the tile list
+// (CTA 0). Tiles hold at most kTcMaxTok tokens of one expert and are ordered
+// by decreasing size.
 __global__ void __launch_bounds__(1024) prefill_plan_kernel(Plan p, int T, int K, int S, int max_tok,
                                                             const float4* __restrict__ tscale,
                                                             float4* __restrict__ slot, int4* __restrict__ tiles,
@@ -521,16 +527,18 @@ __global__ void __launch_bounds__(1024) prefill_plan_kernel(Plan p, int T, int K
     __shared__ int bcnt[kTcMaxTok / 16], bbase[kTcMaxTok / 16], bcur[kTcMaxTok / 16];
     constexpr int NB = kTcMaxTok / 16;
     const int TK = T * K;
-    for (int i = threadIdx.x; i < TK; i += blockDim.x) {
+    const int stride = gridDim.x * blockDim.x, i0 = blockIdx.x * blockDim.x + threadIdx.x;
+    for (int i = i0; i < TK; i += stride) {
         const int t = i / K;
         const float4 ts = tscale[t];
         if (p.pos[i] >= 0) slot[p.pos[i]] = make_float4(ts.x, ts.y, p.w[i] * ts.z, __int_as_float(t));
     }
-    for (int i = threadIdx.x; i < S * T; i += blockDim.x) {
+    for (int i = i0; i < S * T; i += stride) {
         const int t = i % T;
         const float4 ts = tscale[t];
         slot[TK + i] = make_float4(ts.x, ts.y, ts.z, __int_as_float(t));
     }
+    if (blockIdx.x != 0) return;
     if (threadIdx.x < NB) bcnt[threadIdx.x] = bcur[threadIdx.x] = 0;
     __syncthreads();
     const int na = *p.n_active;
@@ -698,7 +706,9 @@ cudaError_t launch_prefill_prep(const void* x, coli_dtype dt, int T, int H, int 
 
 cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, int max_tok, const float4* tscale, float4* slot,
                                 int4* tiles, int* n_tiles, cudaStream_t st) {
-    prefill_plan_kernel<<<1, 1024, 0, st>>>(p, T, K, S, max_tok, tscale, slot, tiles, n_tiles);
+    const int positions = T * K + S * T;
+    const int grid = std::max(1, std::min(148, (positions + 1023) / 1024));
+    prefill_plan_kernel<<<grid, 1024, 0, st>>>(p, T, K, S, max_tok, tscale, slot, tiles, n_tiles);
     return cudaGetLastError();
 }
 

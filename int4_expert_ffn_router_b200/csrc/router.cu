@@ -261,15 +261,23 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     const int chunk = (T + kPlanWarps - 1) / kPlanWarps;
     const int tb = warp * chunk, te = min(T, tb + chunk);
 
+    // A warp walks its chunk 32 / K tokens at a time: lane l holds slot l % K of
+    // token l / K, so lane order is (token, slot) order, and one coalesced load
+    // (issued an iteration ahead) brings the ids of every token of the step.
+    const int tpi = 32 / K, li = lane / K, lk = lane % K;
+    auto slot_id = [&](int t0) { return (li < tpi && t0 + li < te) ? __ldg(ids + (size_t)(t0 + li) * K + lk) : -2; };
     for (int i = threadIdx.x; i < kPlanWarps * E; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
-    // per-warp counts over its token chunk (distinct ids within a token: lane k owns slot k)
-    for (int t = tb; t < te; ++t) {
-        if (lane < K) {
-            int e = ids[(size_t)t * K + lane];
-            if (e >= 0) wcnt[warp * E + e] += 1;  // e < 0: an empty slot
+    // per-warp counts over its token chunk; lanes holding the same expert add as one (e < 0: an
+    // empty slot, or no slot)
+    {
+        int e_next = slot_id(tb);
+        for (int t0 = tb; t0 < te; t0 += tpi) {
+            const int e = e_next;
+            e_next = slot_id(t0 + tpi);
+            const unsigned m = __match_any_sync(0xffffffffu, e);
+            if (e >= 0 && lane == __ffs(m) - 1) wcnt[warp * E + e] += __popc(m);
         }
-        __syncwarp();
     }
     __syncthreads();
     // per expert: exclusive scan over warps -> warp cursor base, total count
@@ -338,20 +346,26 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         }
         p.act_chunk[n_unique + S] = run;
     }
-    // positions: each warp walks its chunk in token order
-    for (int t = tb; t < te; ++t) {
-        if (lane < K) {
-            int e = ids[(size_t)t * K + lane];
+    // positions: each warp walks its chunk in (token, slot) order; lanes holding the same
+    // expert take consecutive positions in lane order, then the lowest of them advances the cursor
+    {
+        int e_next = slot_id(tb);
+        for (int t0 = tb; t0 < te; t0 += tpi) {
+            const int e = e_next;
+            e_next = slot_id(t0 + tpi);
+            const int t = t0 + li;
+            const unsigned m = __match_any_sync(0xffffffffu, e);
             if (e >= 0) {
-                int q = off[e] + wcnt[warp * E + e];
-                wcnt[warp * E + e] += 1;
-                p.pos[(size_t)t * K + lane] = q;
+                const int q = off[e] + wcnt[warp * E + e] + __popc(m & ((1u << lane) - 1u));
+                p.pos[(size_t)t * K + lk] = q;
                 p.tok[q] = t;
-            } else {
-                p.pos[(size_t)t * K + lane] = -1;
+            } else if (e == -1) {
+                p.pos[(size_t)t * K + lk] = -1;  // an empty slot
             }
+            __syncwarp();
+            if (e >= 0 && lane == __ffs(m) - 1) wcnt[warp * E + e] += __popc(m);
+            __syncwarp();
         }
-        __syncwarp();
     }
     // shared experts: all tokens in order
     for (int i = threadIdx.x; i < S * T; i += blockDim.x) p.tok[T * K + i] = i % T;
