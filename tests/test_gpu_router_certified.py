@@ -133,3 +133,28 @@ def test_extreme_and_zero_rows(gpu, coli, with_bias):
         np.testing.assert_array_equal(ids[3], np.arange(c["K"]))
         assert layer.router_fallbacks()[1] >= 1
     layer.close()
+
+
+@pytest.mark.parametrize("bf16", [True, False])
+def test_full_size_router_every_token(gpu, coli, bf16):
+    """The full-size router (256 experts, hidden 6144) on 2048 tokens with
+    Zipf bias: ids and order of every token bit-exact against the fp64
+    oracle, weights within 1e-6, and no token left to the fp64 fallback. The
+    layer is rank 0 of a 32-way expert-parallel split (8 routed experts in
+    HBM, no expert weights loaded): routing through `coli_moe_route` always
+    covers all experts."""
+    c = cases.FULL
+    T, E, K = 2048, c["E"], c["K"]
+    wr = synth.router(40, 0, E, c["H"])
+    bias, _ = synth.zipf_bias(40, 0, E)
+    cfg = coli.make_config(c["H"], c["I"], E, K, c["S"], T)
+    layer = coli.Layer(cfg, wr, bias, device=0, ep=(0, 32))
+    x = synth.x_bf16(40, 0, T, c["H"]) if bf16 else synth.x_f32(40, 0, T, c["H"])
+    ids, w = _route(coli, layer, x, gpu, K)
+    ids_ref, w_ref = oracle.topk(oracle.router_logits(wr, bias, x), K)
+    np.testing.assert_array_equal(ids, ids_ref)
+    np.testing.assert_allclose(w, w_ref, rtol=0, atol=1e-6)
+    assert layer.router_fallbacks() == (True, 0)
+    print(f"full-size router, {T} {'bf16' if bf16 else 'fp32'} tokens: ids bit-exact, max |w - w_ref| "
+          f"{np.abs(w - w_ref).max():.2e}")
+    layer.close()
