@@ -214,8 +214,13 @@ coli_status coli_moe_layer_config(const coli_moe_layer* layer, coli_moe_config* 
 
 /*
  * Router only: ids[t][k] (int32) and weights[t][k] (fp32, summing to 1 per
- * token) for x [n_tokens][H] (fp32 or bf16 bits). Logits are accumulated in
- * fp64 from the exact products of fp32 inputs. 0 <= n_tokens <= max_tokens.
+ * token) for x [n_tokens][H] (fp32 or bf16 bits). 0 <= n_tokens <= max_tokens.
+ * Below 64 tokens the logits are accumulated in fp64 from the exact products
+ * of fp32 inputs. From 64 tokens, where the layer allows it, the certified
+ * router (coli_moe_router_fallbacks) computes them exactly up to a rigorous
+ * per-logit bound and falls back to fp64 for every token the bound does not
+ * settle. Either way the ids and their order are those of the exact logits,
+ * ties going to the lower id.
  */
 coli_status coli_moe_route(coli_moe_layer* layer, const void* x, coli_dtype dtype, int n_tokens,
                            int32_t* ids, float* weights, coli_stream stream);
