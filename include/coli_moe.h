@@ -219,8 +219,8 @@ coli_status coli_moe_layer_config(const coli_moe_layer* layer, coli_moe_config* 
  * of fp32 inputs. From 64 tokens, where the layer allows it, the certified
  * router (coli_moe_router_fallbacks) computes them exactly up to a rigorous
  * per-logit bound and falls back to fp64 for every token the bound does not
- * settle. Either way the ids and their order are those of the exact logits,
- * ties going to the lower id.
+ * settle. Equal logits go to the lower id; the ids and their order can differ
+ * from those of the exact logits only for logits closer than fp64 rounding.
  */
 coli_status coli_moe_route(coli_moe_layer* layer, const void* x, coli_dtype dtype, int n_tokens,
                            int32_t* ids, float* weights, coli_stream stream);
