@@ -441,12 +441,15 @@ coli_status coli_moe_route_noalloc(const float* router_w, const float* router_bi
                                    float* weights, coli_stream stream);
 
 /*
- * Testing aid for the bounded waits of the integer-MMA persistent kernel:
- * every wait of its launches on this layer gives up after wait_ns
- * nanoseconds (0: the default, 1 s), and with enable != 0 one gate/up item of
- * each launch waits on a flag that nothing sets, so the launch gives up: its
- * CTAs drain their copies and exit, and coli_moe_sync then returns COLI_ECUDA
- * and resets the layer, which stays usable. No GPU fault or hang is involved.
+ * Testing aid for the bounded waits of the kernels that wait on barriers or
+ * flags (the integer-MMA persistent kernel, the certified router's GEMM and the
+ * tensor-core grouped GEMMs): every wait of their launches on this layer gives
+ * up after wait_ns nanoseconds (0: the default, 1 s), and with enable != 0 one
+ * gate/up item of each persistent launch waits on a flag that nothing sets, and
+ * one MMA warp of each GEMM launch on a barrier that nothing completes, so the
+ * launches give up: their CTAs drain their copies and exit, and coli_moe_sync
+ * then returns COLI_ECUDA (naming the site of the first wait that gave up) and
+ * resets the layer, which stays usable. No GPU fault or hang is involved.
  */
 coli_status coli_moe_debug_wait_test(coli_moe_layer* layer, int enable, int64_t wait_ns);
 

@@ -37,10 +37,13 @@ bool router_certified_supported(int H, int E);
 size_t router_certified_smem_bytes();
 // Digit planes and bound factors of the router rows, the tensor maps (once).
 cudaError_t router_certified_prepare(RouterCert& rc, const float* wr, cudaStream_t st);
-// err: timeout site of the GEMM's bounded waits (control block).
+// err: timeout site of the GEMM's bounded waits (control block); wait_ns: their
+// bound (0: 1 s); wait_test: testing aid, the GEMM's MMA warp first waits on a
+// barrier that nothing completes, so the launch gives up and reports a timeout.
 cudaError_t launch_router_certified(const RouterCert& rc, const float* wr, const float* bias, const void* x,
                                     coli_dtype dt, int T, int K, double topp, int e_lo, int e_hi, double* logits,
-                                    int32_t* ids, float* w, int* err, cudaStream_t st);
+                                    int32_t* ids, float* w, int* err, int64_t wait_ns, int wait_test,
+                                    cudaStream_t st);
 // Kernels launch_router_logits enqueues for these arguments (0, 1 or 2).
 int router_kernel_count(int T, int H, int E, const double* part, size_t part_cap);
 // topp in (0, 1): adaptive expert top-p after the top-K (topk.cuh, topk_weights); else plain top-K.
@@ -124,9 +127,12 @@ cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, int max_tok,
 // token_maps: host copies of two 2D tensor maps (make_token_map; boxes of
 // kTcMaxTok and 32 rows) over xs (phase 0) or h16 (phase 1).
 // pairs (phase 0): the operand holds hi and lo rows per position (fp32 input).
+// wait_ns: bound of the kernel's waits (0: 1 s); wait_test: testing aid, one MMA warp first
+// waits on a barrier that nothing completes, so the launch gives up and reports a timeout.
 cudaError_t launch_prefill_gemm(int phase, bool pairs, const uint8_t* weights, const Dims& d, const void* token_maps,
                                 const Plan& p, const float4* slot, const int4* tiles, const int* n_tiles, __half* h16,
-                                float* y32, int* err, int n_sm, long long* trace, int trace_cap, cudaStream_t st);
+                                float* y32, int* err, int n_sm, long long* trace, int trace_cap, int64_t wait_ns,
+                                int wait_test, cudaStream_t st);
 // Encodes a 2D fp16 tensor map (128 bytes, written to `map`) over
 // [rows][cols] at `base`: box 64 x box_rows, 128-byte swizzle.
 cudaError_t make_token_map(void* map, const void* base, int rows, int cols, int box_rows);

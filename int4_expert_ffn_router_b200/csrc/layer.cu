@@ -613,7 +613,7 @@ static int route_batch(coli_moe_layer* L, const void* x, coli_dtype dt, int T, i
     const Dims& d = L->d;
     if (L->cert_ok && T >= kRouterGemmMinTok) {
         if (launch_router_certified(L->rc, L->router_w, L->router_b, x, dt, T, d.K, L->topp, e_lo, e_hi, L->logits, ids,
-                                    w, L->ctl + kCtlError, s) != cudaSuccess)
+                                    w, L->ctl + kCtlError, L->wait_ns, L->wait_test, s) != cudaSuccess)
             return -1;
         return 5;
     }
@@ -696,12 +696,13 @@ static coli_status forward_impl(coli_moe_layer* L, const void* x, void* y, coli_
         // with a trace buffer: block timeline of the gate/up launch, then of the down launch
         const int tcap = L->trace ? (L->trace_cap - 256) / 16 : 0;
         CUDA_TRY(launch_prefill_gemm(0, pairs, L->weights, d, L->xs_maps, p, L->slot, L->tiles, L->n_tiles, h16, nullptr,
-                                     L->ctl + kCtlError, L->n_sm, tcap > 0 ? L->trace : nullptr, tcap, s),
+                                     L->ctl + kCtlError, L->n_sm, tcap > 0 ? L->trace : nullptr, tcap, L->wait_ns,
+                                     L->wait_test, s),
                  "gate/up (tensor cores)");
         prof_mark(L, COLI_STAGE_DOWN, s);
         CUDA_TRY(launch_prefill_gemm(1, false, L->weights, d, L->h16_maps, p, L->slot, L->tiles, L->n_tiles, nullptr,
                                      L->o, L->ctl + kCtlError, L->n_sm,
-                                     tcap > 0 ? L->trace + (size_t)tcap * 8 + 128 : nullptr, tcap, s),
+                                     tcap > 0 ? L->trace + (size_t)tcap * 8 + 128 : nullptr, tcap, L->wait_ns, L->wait_test, s),
                  "down (tensor cores)");
         prof_mark(L, COLI_STAGE_COMBINE, s);
         CUDA_TRY(launch_prefill_out(L->o, residual, T, d.H, y, dt, s), "output");
@@ -901,8 +902,8 @@ COLI_API coli_status coli_moe_stack_forward(coli_moe_layer* const* layers, int n
     return COLI_OK;
 }
 
-// Waits for the layer's last forward and reports a device-side timeout of the
-// persistent kernel (then clears the control block so the layer stays usable).
+// Waits for the layer's last forward and reports a device-side timeout of one
+// of its kernels (then clears the control block so the layer stays usable).
 static coli_status sync_and_check(coli_moe_layer* L) {
     CUDA_TRY(cudaStreamSynchronize(L->last_stream), "sync");
     int err = 0;
@@ -910,7 +911,7 @@ static coli_status sync_and_check(coli_moe_layer* L) {
     if (err != 0) {
         CUDA_TRY(cudaMemset(L->ctl, 0, (size_t)L->ctl_n * 4), "reset control block");
         char msg[96];
-        snprintf(msg, sizeof msg, "a bounded wait in a persistent kernel timed out (site %d)", err);
+        snprintf(msg, sizeof msg, "a bounded wait in a kernel of this layer timed out (site %d)", err);
         g_last_error = msg;
         return COLI_ECUDA;
     }

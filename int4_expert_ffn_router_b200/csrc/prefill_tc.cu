@@ -68,7 +68,7 @@ constexpr int kABase = 0;
 constexpr int kAccBase = kAStages * 128;           // 256
 constexpr int kAccCols = kTcMaxTok;                // accumulator of one row tile
 static_assert(kAccBase + 2 * kAccCols <= (int)kTmemCols, "tensor memory budget");
-constexpr uint64_t kTcWaitNs = 1000000000ull;      // every wait gives up after 1 s
+constexpr uint64_t kTcWaitNs = 1000000000ull;      // every wait gives up after 1 s (default)
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int kOffB = 0;
@@ -99,6 +99,8 @@ struct __align__(64) TcArgs {
     float* y32;             // down output [T][H] (accumulated)
     int I, H;
     int* err;               // timeout site (control block)
+    uint64_t wait_ns;       // bound of every wait
+    int wait_test;          // testing aid: MMA warp 0 first waits on a barrier that nothing completes
     long long* trace;       // CTA 0 timeline (clock64 stamps) or NULL
     int trace_cap;          // 64-input blocks recorded
 };
@@ -124,25 +126,27 @@ __device__ __forceinline__ void tc_stamp_item(const TcArgs& a, uint32_t i, int j
     }
 }
 
-__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site);
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site,
+                                        uint64_t limit);
 
 // Every lane polls (a one-lane poll plus broadcast costs more); the warp goes
 // on only if all lanes saw the phase complete, so warp-collective tcgen05
 // instructions stay converged.
 __device__ __forceinline__ bool tc_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
-                                             int site) {
-    const bool ok = tc_wait(bar, parity, abort_flag, err, site);
+                                             int site, uint64_t limit) {
+    const bool ok = tc_wait(bar, parity, abort_flag, err, site, limit);
     return __all_sync(0xffffffffu, ok);
 }
 
-__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site) {
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site,
+                                        uint64_t limit) {
     // sleep in the barrier for up to 0.2 ms at a time; the bound stays 1 s
     if (mbar_try_wait_sleep(bar, parity, 200000)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 200000)) return true;
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > kTcWaitNs) {
+        if (globaltimer_ns() - t0 > limit) {
             *abort_flag = 1;
             atomicCAS(err, 0, site);
             return false;
@@ -228,9 +232,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                 const uint32_t it = it0 + kb;
                 const uint32_t p2 = it >> 1;           // A stage use counter
                 const uint32_t s = it % kSStages, sa = p2 % kAStages;
-                if (!seen_full && !tc_wait_warp(&full[s], (it / kSStages) & 1, abort_flag, a.err, 21)) { ok = false; break; }
+                if (!seen_full && !tc_wait_warp(&full[s], (it / kSStages) & 1, abort_flag, a.err, 21, a.wait_ns)) { ok = false; break; }
                 if (warp == 0 && lane == 0) tc_stamp(a, it, 0);
-                if (!seen_aempty && !tc_wait_warp(&aempty[2 * sa + rt2], ((p2 / kAStages) & 1) ^ 1, abort_flag, a.err, 22)) { ok = false; break; }
+                if (!seen_aempty && !tc_wait_warp(&aempty[2 * sa + rt2], ((p2 / kAStages) & 1) ^ 1, abort_flag, a.err, 22, a.wait_ns)) { ok = false; break; }
                 if (warp == 0 && lane == 0) tc_stamp(a, it, 1);
                 tc_fence_after();
                 const uint8_t* blk = sm + kOffW + s * kWStageBytes + rt2 * kBlockBytes;
@@ -274,7 +278,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
             }
             if (!ok) break;
             // ---------------------------------------------------- epilogue
-            if (!tc_wait_warp(&accfull[rt2], icount & 1, abort_flag, a.err, 23)) { ok = false; break; }
+            if (!tc_wait_warp(&accfull[rt2], icount & 1, abort_flag, a.err, 23, a.wait_ns)) { ok = false; break; }
             if (warp == 0 && lane == 0) tc_stamp_item(a, icount, 0);
             tc_fence_after();
             const uint32_t tacc = tmem + lane_base + kAccBase + rt2 * kAccCols;
@@ -362,7 +366,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
             const uint8_t* w1 = w0 + (size_t)KB * kBlockBytes;
             for (int kb = 0; kb < KB; ++kb, ++it) {
                 const uint32_t s = it % kSStages;
-                if (!tc_wait(&sempty[s], ((it / kSStages) & 1) ^ 1, abort_flag, a.err, 24)) { ok = false; break; }
+                if (!tc_wait(&sempty[s], ((it / kSStages) & 1) ^ 1, abort_flag, a.err, 24, a.wait_ns)) { ok = false; break; }
                 tc_stamp(a, it, 6);
                 uint8_t* wdst = sm + kOffW + s * kWStageBytes;
                 mbar_arrive_expect_tx(&full[s], tx_bytes);
@@ -376,7 +380,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
         const uint32_t first = it > (uint32_t)kSStages ? it - kSStages : 0;
         const uint64_t t0 = globaltimer_ns();
         for (uint32_t k = first; k < it; ++k) {
-            while (!mbar_try_wait(&full[k % kSStages], (k / kSStages) & 1) && globaltimer_ns() - t0 < kTcWaitNs) {
+            while (!mbar_try_wait(&full[k % kSStages], (k / kSStages) & 1) && globaltimer_ns() - t0 < a.wait_ns) {
             }
         }
       }
@@ -391,17 +395,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
         const uint64_t bdesc0 = tc_sdesc_sw128(smem_addr(sm + kOffB));
         uint32_t it = 0, icount = 0;
         bool ok = true, issued = false;
+        // testing aid: drained[0] completes only after this warp's own final commit, so the launch gives up
+        if (a.wait_test && t2 == 0) ok = tc_wait_warp(&drained[0], 0, abort_flag, a.err, 29, a.wait_ns);
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const int4 tile = a.tiles[item / a.RT2];
             const int nm = ((kPairs ? 2 * tile.z : tile.z) + 15) & ~15;
             const uint32_t idesc = tc_idesc_f16(nm, false);
-            if (!tc_wait_warp(&accempty[t2], (icount & 1) ^ 1, abort_flag, a.err, 25)) { ok = false; break; }
+            if (!tc_wait_warp(&accempty[t2], (icount & 1) ^ 1, abort_flag, a.err, 25, a.wait_ns)) { ok = false; break; }
             tc_fence_after();
             for (int kb = 0; kb < KB; kb += 2, it += 2) {
                 const uint32_t p2 = it >> 1;
                 const uint32_t s0 = it % kSStages, sa = p2 % kAStages;
                 // aready implies full: the transform warps waited for both blocks' stages before arriving
-                if (!tc_wait_warp(&aready[2 * sa + t2], (p2 / kAStages) & 1, abort_flag, a.err, 27)) { ok = false; break; }
+                if (!tc_wait_warp(&aready[2 * sa + t2], (p2 / kAStages) & 1, abort_flag, a.err, 27, a.wait_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint64_t bd0 = bdesc0 + s0 * (kBTileBytes >> 4);
                 const uint64_t bd1 = bdesc0 + ((s0 + 1) % kSStages) * (kBTileBytes >> 4);
@@ -422,7 +428,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
             // every MMA must complete before the tensor memory is released
             tc_commit_elect(&drained[t2]);
             const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&drained[t2], 0) && globaltimer_ns() - t0 < kTcWaitNs) {
+            while (!mbar_try_wait(&drained[t2], 0) && globaltimer_ns() - t0 < a.wait_ns) {
             }
         }
         __syncwarp();
@@ -714,7 +720,8 @@ cudaError_t launch_prefill_plan(const Plan& p, int T, int K, int S, int max_tok,
 
 cudaError_t launch_prefill_gemm(int phase, bool pairs, const uint8_t* weights, const Dims& d, const void* token_maps,
                                 const Plan& p, const float4* slot, const int4* tiles, const int* n_tiles, __half* h16,
-                                float* y32, int* err, int n_sm, long long* trace, int trace_cap, cudaStream_t st) {
+                                float* y32, int* err, int n_sm, long long* trace, int trace_cap, int64_t wait_ns,
+                                int wait_test, cudaStream_t st) {
     TcArgs a;
     memcpy(&a.tmap_big, token_maps, sizeof(CUtensorMap));
     memcpy(&a.tmap_small, static_cast<const uint8_t*>(token_maps) + sizeof(CUtensorMap), sizeof(CUtensorMap));
@@ -734,6 +741,8 @@ cudaError_t launch_prefill_gemm(int phase, bool pairs, const uint8_t* weights, c
     a.I = d.I;
     a.H = d.H;
     a.err = err;
+    a.wait_ns = wait_ns > 0 ? (uint64_t)wait_ns : kTcWaitNs;
+    a.wait_test = wait_test;
     cudaError_t e;
     auto run = [&](auto kern) {
         cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemTc);

@@ -57,7 +57,7 @@ constexpr int kRxOffBar = kRxStages * kRxStageBytes;
 constexpr int kRxSmem = kRxOffBar + 64 + 1024;         // barriers, tensor-memory slot, flag, alignment slack
 constexpr int kRxThreads = 192;                        // producer, MMA, four epilogue warps
 constexpr uint32_t kRxTmemCols = 256;
-constexpr uint64_t kRxWaitNs = 1000000000ull;          // every wait gives up after 1 s
+constexpr uint64_t kRxWaitNs = 1000000000ull;          // every wait gives up after 1 s (default)
 
 // Error-bound constants (u = 2^-53): the three fp64 additions of the digit
 // terms, at most 3.01u of sum |term| <= 2.02 max|Wr_e| sqrt(H) ||xh_t||, with
@@ -260,13 +260,14 @@ __host__ __device__ constexpr uint32_t rx_idesc_s8(int m, int n) {
     return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
-__device__ __forceinline__ bool rx_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site) {
+__device__ __forceinline__ bool rx_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err, int site,
+                                        uint64_t limit) {
     if (mbar_try_wait_sleep(bar, parity, 200000)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (mbar_try_wait_sleep(bar, parity, 200000)) return true;
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > kRxWaitNs) {
+        if (globaltimer_ns() - t0 > limit) {
             *abort_flag = 1;
             atomicCAS(err, 0, site);
             return false;
@@ -274,8 +275,8 @@ __device__ __forceinline__ bool rx_wait(uint64_t* bar, uint32_t parity, volatile
     }
 }
 __device__ __forceinline__ bool rx_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* err,
-                                             int site) {
-    const bool ok = rx_wait(bar, parity, abort_flag, err, site);
+                                             int site, uint64_t limit) {
+    const bool ok = rx_wait(bar, parity, abort_flag, err, site, limit);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -288,6 +289,8 @@ struct __align__(64) RxArgs {
     double* logits;    // [T][E]
     int T, H, E;
     int* err;
+    uint64_t wait_ns;  // bound of every wait
+    int wait_test;     // testing aid: the MMA warp first waits on a barrier that nothing completes
 };
 
 // CTA (bx, by): experts 32 bx .. +31, tokens 64 by .. +63. Warp 0 (one lane)
@@ -333,7 +336,7 @@ __global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_c
             int kb = 0;
             for (; kb < nkb; ++kb) {
                 const int s = kb % kRxStages;
-                if (!rx_wait(&empty[s], ((kb / kRxStages) & 1) ^ 1, abort_flag, a.err, 41)) break;
+                if (!rx_wait(&empty[s], ((kb / kRxStages) & 1) ^ 1, abort_flag, a.err, 41, a.wait_ns)) break;
                 uint8_t* st = sm + s * kRxStageBytes;
                 mbar_arrive_expect_tx(&full[s], kRxStageBytes);
 #pragma unroll
@@ -347,7 +350,7 @@ __global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_c
             const int first = kb > kRxStages ? kb - kRxStages : 0;
             const uint64_t tw = globaltimer_ns();
             for (int k = first; k < kb; ++k)
-                while (!mbar_try_wait(&full[k % kRxStages], (k / kRxStages) & 1) && globaltimer_ns() - tw < kRxWaitNs) {
+                while (!mbar_try_wait(&full[k % kRxStages], (k / kRxStages) & 1) && globaltimer_ns() - tw < a.wait_ns) {
                 }
         }
         __syncwarp();
@@ -355,9 +358,11 @@ __global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_c
         const uint32_t idesc = rx_idesc_s8(kRxM, kRxN);
         const uint64_t adesc0 = tc_sdesc_sw128(smem_addr(sm));
         bool issued = false;
-        for (int kb = 0; kb < nkb; ++kb) {
+        // testing aid: accfull completes only after this warp's own commit, so the launch gives up
+        if (a.wait_test) ok = rx_wait_warp(accfull, 0, abort_flag, a.err, 44, a.wait_ns);
+        for (int kb = 0; ok && kb < nkb; ++kb) {
             const int s = kb % kRxStages;
-            if (!rx_wait_warp(&full[s], (kb / kRxStages) & 1, abort_flag, a.err, 42)) { ok = false; break; }
+            if (!rx_wait_warp(&full[s], (kb / kRxStages) & 1, abort_flag, a.err, 42, a.wait_ns)) { ok = false; break; }
             tc_fence_after();
             const uint64_t ad = adesc0 + (uint64_t)((s * kRxStageBytes) >> 4);
             const uint64_t bd = ad + (uint64_t)(kRxABytes >> 4);
@@ -369,14 +374,14 @@ __global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_c
             // so the tensor memory is never released under a running MMA)
             tc_commit_elect(accfull);
             const uint64_t tw = globaltimer_ns();
-            while (!mbar_try_wait(accfull, 0) && globaltimer_ns() - tw < kRxWaitNs) {
+            while (!mbar_try_wait(accfull, 0) && globaltimer_ns() - tw < a.wait_ns) {
             }
         }
         __syncwarp();
     } else {
         const int p = warp & 3;
         double* stage = reinterpret_cast<double*>(sm);  // [4][kRxT][kRxE]
-        ok = rx_wait_warp(accfull, 0, abort_flag, a.err, 43) && !*abort_flag;
+        ok = rx_wait_warp(accfull, 0, abort_flag, a.err, 43, a.wait_ns) && !*abort_flag;
         if (ok) {
             tc_fence_after();
             const uint32_t tl = tmem + ((uint32_t)(32 * p) << 16);
@@ -639,7 +644,8 @@ cudaError_t router_certified_prepare(RouterCert& rc, const float* wr, cudaStream
 
 cudaError_t launch_router_certified(const RouterCert& rc, const float* wr, const float* bias, const void* x,
                                     coli_dtype dt, int T, int K, double topp, int e_lo, int e_hi, double* logits,
-                                    int32_t* ids, float* w, int* err, cudaStream_t st) {
+                                    int32_t* ids, float* w, int* err, int64_t wait_ns, int wait_test,
+                                    cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     if (T > rc.Tm || K < 1 || K > 32) return cudaErrorInvalidValue;
     if (e_hi < 0) e_hi = rc.E;
@@ -662,6 +668,8 @@ cudaError_t launch_router_certified(const RouterCert& rc, const float* wr, const
     a.H = H;
     a.E = E;
     a.err = err;
+    a.wait_ns = wait_ns > 0 ? (uint64_t)wait_ns : kRxWaitNs;
+    a.wait_test = wait_test;
     const dim3 g((E + kRxE - 1) / kRxE, (T + kRxT - 1) / kRxT);
     router_i8_kernel<<<g, kRxThreads, kRxSmem, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -108,3 +108,52 @@ def test_bounded_wait_expiry_returns_an_error_and_the_layer_recovers(gpu):
         y = yd.cpu().numpy().astype(np.float64)
         assert np.abs(y - y_ref).max() <= 1e-3 * np.abs(y_ref).max()
     layer.close()
+
+
+@pytest.mark.parametrize("E,sites", [(16, r"4[1-4]"), (300, r"2[1-9]")])
+def test_bounded_wait_expiry_in_the_batch_kernels(gpu, E, sites):
+    """The same testing aid on a 96-token bf16 batch: the certified router's
+    int8 GEMM and both tensor-core grouped GEMMs each make one MMA warp wait
+    on a barrier that nothing completes, every wait bounded to 2 ms. Each
+    launch gives up by itself (its copies drain, no MMA is left running when
+    tensor memory is released): coli_moe_sync reports COLI_ECUDA promptly,
+    naming a site of the first launch that gave up, and the next forwards on
+    the same layer match the oracle. With 16 experts that is the router GEMM
+    (sites 41-44); with 300 experts (more than the certified router takes) the
+    router is the fp64 one, and the grouped GEMMs report (sites 21-29)."""
+    import time
+
+    import int4_expert_ffn_router_b200 as coli
+
+    c = dict(cases.TINY, E=E)
+    T = 96
+    L, args = _host_args(coli, c, max_tokens=T)
+    layer = coli.Layer(*args, device=0)
+    assert layer.router_fallbacks()[0] == (E <= 256)  # the certified router serves this batch
+    xb = synth.x_bf16(c["seed"], 5, T, c["H"])
+    xd = torch.from_numpy(xb.view(np.int16)).to(gpu).view(torch.bfloat16)
+    yd = torch.empty_like(xd)
+    layer.forward(xd, yd)
+    layer.sync()
+    layer.debug_wait_test(True, 2_000_000)
+    t0 = time.time()
+    layer.forward(xd, yd)
+    with pytest.raises(coli.ColiError) as e:
+        layer.sync()
+    elapsed = time.time() - t0
+    # the first wait to give up belongs to the first launch with the aid: its MMA warp's, or
+    # the wait of another warp for the same barrier
+    import re
+    assert e.value.status == coli.COLI_ECUDA and re.search(r"timed out \(site " + sites + r"\)", str(e.value))
+    assert elapsed < 2.0, f"the launches took {elapsed:.2f} s to give up"
+    layer.debug_wait_test(False, 0)
+    y_ref, _, _ = oracle.moe_forward(cases.oracle_cfg(c), L["wr"], None, L["experts"], xb)
+    for _ in range(2):
+        yd.fill_(float("nan"))
+        layer.forward(xd, yd)
+        layer.sync()
+        y = yd.float().cpu().numpy().astype(np.float64)
+        assert np.linalg.norm(y - y_ref) <= 5e-3 * np.linalg.norm(y_ref)
+        ids_ref, _ = oracle.topk(oracle.router_logits(L["wr"], None, xb), c["K"])
+        np.testing.assert_array_equal(layer.plan(T)["ids"], ids_ref)
+    layer.close()
