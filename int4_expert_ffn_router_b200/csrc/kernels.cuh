@@ -23,7 +23,7 @@ cudaError_t launch_router_logits(const float* wr, const float* bias, const void*
 // weights taken from those logits where the bounds prove them, and the fp64
 // logits and top-K for the other tokens. Five kernels.
 struct RouterCert {
-    uint8_t* maps = nullptr;       // host: two CUtensorMap (router planes, batch planes), 64-byte aligned
+    uint8_t* maps = nullptr;       // host: 6 CUtensorMap (router planes; batch planes for 5 tile heights), 64-byte aligned
     uint8_t* wd8 = nullptr;        // [4][E][H] router digit planes
     int* wscale = nullptr;         // [E] row scale exponents r_e
     double* wb = nullptr;          // [E][3] ||Wr_e - wh_e||, ||wh_e||, rounding-bound factor
@@ -31,7 +31,7 @@ struct RouterCert {
     int* xscale = nullptr;         // [Tm] token scale exponents s_t
     double* xb = nullptr;          // [Tm][3] ||x_t||, ||x_t - xh_t||, ||xh_t||
     int* fail = nullptr;           // [1 + Tm]: count, then the tokens sent to the fp64 fallback
-    int Tm = 0, H = 0, E = 0;
+    int Tm = 0, H = 0, E = 0, n_sm = 148;
 };
 bool router_certified_supported(int H, int E);
 size_t router_certified_smem_bytes();

@@ -137,7 +137,7 @@ struct coli_moe_layer {
     // certified integer-MMA router of token batches (router_certified.cu)
     bool cert_ok = false;           // shapes and device allow it and the workspace holds its buffers
     RouterCert rc;
-    alignas(64) unsigned char rc_maps[2 * kTensorMapBytes] = {};  // TMA maps of its digit planes
+    alignas(64) unsigned char rc_maps[6 * kTensorMapBytes] = {};  // TMA maps of its digit planes
     size_t rpart_cap = 0;           // doubles
     bool tc_shape_ok = false;       // shapes and shared memory allow the tensor-core kernels
     bool tc_scale_ok = true;        // every weight scale keeps q * scale finite in fp16
@@ -467,6 +467,7 @@ static coli_status create_impl(const coli_moe_config* cfg, const float* router_w
     L->rc.Tm = Tm;
     L->rc.H = d.H;
     L->rc.E = d.E;
+    L->rc.n_sm = L->n_sm;
     L->cert_ok = cert;
     L->rpart_cap = rpart_cap;
     {

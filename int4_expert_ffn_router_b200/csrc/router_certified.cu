@@ -43,9 +43,11 @@ namespace coli {
 namespace {
 
 // GEMM tile: 32 experts x 4 digit planes = 128 rows of A (the MMA's M) and
-// 64 tokens x 4 digit planes = 256 rows of B (its N); 128 inputs (bytes) of
+// tb tokens x 4 digit planes = 4 tb rows of B (its N; tb <= 64, a multiple of
+// 8, chosen per call so that the SMs' loads are even); 128 inputs (bytes) of
 // the input dimension per pipeline stage, four K = 32 MMAs each.
 constexpr int kRxE = 32, kRxT = 64, kRxK = 128;
+constexpr int kRxTiles[5] = {64, 56, 48, 40, 32};  // token rows per tile the launcher chooses from
 constexpr int kRxM = 4 * kRxE, kRxN = 4 * kRxT;
 constexpr int kRxStages = 2;
 constexpr int kRxABytes = kRxM * kRxK;                 // 16 KB
@@ -282,20 +284,21 @@ __device__ __forceinline__ bool rx_wait_warp(uint64_t* bar, uint32_t parity, vol
 
 struct __align__(64) RxArgs {
     CUtensorMap wmap;  // digit planes of the router rows: dims (H, E, 4), box (128, 32, 1)
-    CUtensorMap xmap;  // digit planes of the batch: dims (H, Tm, 4), box (128, 64, 1)
+    CUtensorMap xmap;  // digit planes of the batch: dims (H, Tm, 4), box (128, tb, 1)
     const int* wscale;
     const int* xscale;
     const float* bias;
     double* logits;    // [T][E]
     int T, H, E;
+    int tb;            // token rows per tile
     int* err;
     uint64_t wait_ns;  // bound of every wait
     int wait_test;     // testing aid: the MMA warp first waits on a barrier that nothing completes
 };
 
-// CTA (bx, by): experts 32 bx .. +31, tokens 64 by .. +63. Warp 0 (one lane)
+// CTA (bx, by): experts 32 bx .. +31, tokens tb by .. +tb-1. Warp 0 (one lane)
 // loads each stage's 4 + 4 digit boxes with TMA; warp 1 allocates the
-// accumulator (128 lanes x 256 int32 columns: lane 32 p + e, column 64 q + t)
+// accumulator (128 lanes x 4 tb int32 columns: lane 32 p + e, column tb q + t)
 // and issues the MMAs; warps 2..5 (lane quarter p = warp % 4) read it back:
 // term_p(t, e) = 2^(8(3-p)) sum_q 2^(8(3-q)) P_pq, exact in fp64 (below
 // 2^53), staged in shared memory, then v = ((term_0 + term_1) + term_2) +
@@ -309,7 +312,9 @@ __global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_c
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e0 = blockIdx.x * kRxE, t0 = blockIdx.y * kRxT;
+    const int tb = a.tb;
+    const int e0 = blockIdx.x * kRxE, t0 = blockIdx.y * tb;
+    const uint32_t stage_tx = kRxABytes + 4 * tb * kRxK;  // bytes one stage's boxes bring
     const int nkb = (a.H + kRxK - 1) / kRxK;
 
     if (threadIdx.x == 0) {
@@ -338,13 +343,13 @@ __global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_c
                 const int s = kb % kRxStages;
                 if (!rx_wait(&empty[s], ((kb / kRxStages) & 1) ^ 1, abort_flag, a.err, 41, a.wait_ns)) break;
                 uint8_t* st = sm + s * kRxStageBytes;
-                mbar_arrive_expect_tx(&full[s], kRxStageBytes);
+                mbar_arrive_expect_tx(&full[s], stage_tx);
 #pragma unroll
                 for (int p = 0; p < 4; ++p)
                     rx_tma_3d(smem_addr(st + p * (kRxE * kRxK)), &a.wmap, kb * kRxK, e0, p, &full[s]);
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    rx_tma_3d(smem_addr(st + kRxABytes + q * (kRxT * kRxK)), &a.xmap, kb * kRxK, t0, q, &full[s]);
+                    rx_tma_3d(smem_addr(st + kRxABytes + q * (tb * kRxK)), &a.xmap, kb * kRxK, t0, q, &full[s]);
             }
             // copies still in flight (after an abort) land before the CTA exits
             const int first = kb > kRxStages ? kb - kRxStages : 0;
@@ -355,7 +360,7 @@ __global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_c
         }
         __syncwarp();
     } else if (warp == 1) {
-        const uint32_t idesc = rx_idesc_s8(kRxM, kRxN);
+        const uint32_t idesc = rx_idesc_s8(kRxM, 4 * tb);
         const uint64_t adesc0 = tc_sdesc_sw128(smem_addr(sm));
         bool issued = false;
         // testing aid: accfull completes only after this warp's own commit, so the launch gives up
@@ -387,14 +392,17 @@ __global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_c
             const uint32_t tl = tmem + ((uint32_t)(32 * p) << 16);
             const double wp = p == 0 ? 16777216.0 : p == 1 ? 65536.0 : p == 2 ? 256.0 : 1.0;
 #pragma unroll 1
-            for (int c = 0; c < kRxT / 16; ++c) {
+            // chunks of 16 columns per plane; a last chunk that runs past the plane's tb
+            // columns reads columns that are skipped (all inside the 256 allocated)
+            for (int c = 0; 16 * c < tb; ++c) {
                 uint32_t v0[16], v1[16], v2[16], v3[16];
-                tc_ld16_wait(tl + 0 * kRxT + 16 * c, v0);
-                tc_ld16_wait(tl + 1 * kRxT + 16 * c, v1);
-                tc_ld16_wait(tl + 2 * kRxT + 16 * c, v2);
-                tc_ld16_wait(tl + 3 * kRxT + 16 * c, v3);
+                tc_ld16_wait(tl + 0 * tb + 16 * c, v0);
+                tc_ld16_wait(tl + 1 * tb + 16 * c, v1);
+                tc_ld16_wait(tl + 2 * tb + 16 * c, v2);
+                tc_ld16_wait(tl + 3 * tb + 16 * c, v3);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
+                    if (16 * c + i >= tb) break;
                     const long long sp = ((long long)(int)v0[i] << 24) + ((long long)(int)v1[i] << 16) +
                                          ((long long)(int)v2[i] << 8) + (long long)(int)v3[i];
                     stage[((size_t)p * kRxT + 16 * c + i) * kRxE + lane] = (double)sp * wp;
@@ -409,7 +417,7 @@ __global__ void __launch_bounds__(kRxThreads, 1) router_i8_kernel(const __grid_c
             const bool ein = e < a.E;
             const int r = ein ? __ldg(a.wscale + e) : 0;
             const double b = ein ? (double)__ldg(a.bias + e) : 0.0;
-            for (int tt = warp - 2; tt < kRxT; tt += 4) {
+            for (int tt = warp - 2; tt < tb; tt += 4) {
                 const int t = t0 + tt;
                 if (t >= a.T || !ein) continue;
                 const double v = ((stage[(0 * kRxT + tt) * kRxE + lane] + stage[(1 * kRxT + tt) * kRxE + lane]) +
@@ -638,7 +646,9 @@ cudaError_t router_certified_prepare(RouterCert& rc, const float* wr, cudaStream
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if ((e = rx_encode(rc.maps, rc.wd8, rc.E, rc.H, kRxE)) != cudaSuccess) return e;
-    if ((e = rx_encode(rc.maps + sizeof(CUtensorMap), rc.xd8, rc.Tm, rc.H, kRxT)) != cudaSuccess) return e;
+    for (int i = 0; i < 5; ++i)
+        if ((e = rx_encode(rc.maps + (1 + i) * sizeof(CUtensorMap), rc.xd8, rc.Tm, rc.H, kRxTiles[i])) != cudaSuccess)
+            return e;
     return cudaFuncSetAttribute(router_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRxSmem);
 }
 
@@ -659,7 +669,16 @@ cudaError_t launch_router_certified(const RouterCert& rc, const float* wr, const
     if (e != cudaSuccess) return e;
     RxArgs a;
     memcpy(&a.wmap, rc.maps, sizeof(CUtensorMap));
-    memcpy(&a.xmap, rc.maps + sizeof(CUtensorMap), sizeof(CUtensorMap));
+    // the tile height whose busiest SM has the least work: tiles per SM (2 resident) x rows per tile
+    int pick = 0;
+    long best = -1;
+    for (int i = 0; i < 5; ++i) {
+        const long tiles = (long)((E + kRxE - 1) / kRxE) * ((T + kRxTiles[i] - 1) / kRxTiles[i]);
+        const long load = ((tiles + rc.n_sm - 1) / rc.n_sm) * kRxTiles[i];
+        if (best < 0 || load < best) { best = load; pick = i; }
+    }
+    a.tb = kRxTiles[pick];
+    memcpy(&a.xmap, rc.maps + (1 + pick) * sizeof(CUtensorMap), sizeof(CUtensorMap));
     a.wscale = rc.wscale;
     a.xscale = rc.xscale;
     a.bias = bias;
@@ -670,7 +689,7 @@ cudaError_t launch_router_certified(const RouterCert& rc, const float* wr, const
     a.err = err;
     a.wait_ns = wait_ns > 0 ? (uint64_t)wait_ns : kRxWaitNs;
     a.wait_test = wait_test;
-    const dim3 g((E + kRxE - 1) / kRxE, (T + kRxT - 1) / kRxT);
+    const dim3 g((E + kRxE - 1) / kRxE, (T + a.tb - 1) / a.tb);
     router_i8_kernel<<<g, kRxThreads, kRxSmem, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     router_certify_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, rc.wb, rc.xb, T, E, K, topp, e_lo, e_hi, ids, w,
