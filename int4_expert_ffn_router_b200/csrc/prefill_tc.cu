@@ -352,6 +352,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
         // the tensor, where TMA fills zeros; their columns are never read).
         uint32_t it = 0;
         bool ok = true;
+        const uint64_t wpolicy = l2_policy_evict_first();
         for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
             const int4 tile = a.tiles[item / a.RT2];
             const int pair = item % a.RT2;
@@ -370,8 +371,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) moe_prefill_tc_kernel(const __g
                 tc_stamp(a, it, 6);
                 uint8_t* wdst = sm + kOffW + s * kWStageBytes;
                 mbar_arrive_expect_tx(&full[s], tx_bytes);
-                bulk_g2s(wdst, w0 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s]);
-                bulk_g2s(wdst + kBlockBytes, w1 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s]);
+                // weights leave L2 first, so the tile's token rows (read again by every pair of row
+                // tiles) stay there
+                bulk_g2s_policy(wdst, w0 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s], wpolicy);
+                bulk_g2s_policy(wdst + kBlockBytes, w1 + (size_t)kb * kBlockBytes, kBlockBytes, &full[s], wpolicy);
                 tma_load_2d(smem_addr(sm + kOffB + s * kBTileBytes), map, kb * 64, row0, &full[s]);
                 tc_stamp(a, it, 7);
             }
