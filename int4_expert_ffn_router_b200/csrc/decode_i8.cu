@@ -317,6 +317,7 @@ __device__ void i8_producer(I8Args& a, I8Smem& S, uint8_t* ring) {
     const unsigned long long* entries = entries_of(a, f.nch);
     uint32_t q = 0, gs = 0, slot_s = 0, phase_s = 0;
     bool first_ticket = true;
+    const uint64_t wpolicy = l2_policy_evict_first();
     int nc = -1;  // routed chunks, once the plan is published
     while (true) {
         Item it{IT_END, 0, 0, 0, 0, 0, -1, 0};
@@ -375,8 +376,10 @@ __device__ void i8_producer(I8Args& a, I8Smem& S, uint8_t* ring) {
                 // slot_s = gs % nstages, phase_s = (gs / nstages) & 1
                 if (gs >= (uint32_t)a.nstages && !wait_bar(&S.empty[slot_s], phase_s ^ 1, abort_flag, a, 4)) break;
                 mbar_arrive_expect_tx(&S.full[slot_s], nb * kBlockBytes);
-                bulk_g2s(ring + (size_t)slot_s * stage_bytes, tile + (size_t)b0 * kBlockBytes, nb * kBlockBytes,
-                         &S.full[slot_s]);
+                // weights are read once: they leave L2 first, ahead of the token limbs, h rows and
+                // expert outputs that other CTAs read again
+                bulk_g2s_policy(ring + (size_t)slot_s * stage_bytes, tile + (size_t)b0 * kBlockBytes, nb * kBlockBytes,
+                                &S.full[slot_s], wpolicy);
                 ++gs;
                 if (++slot_s == (uint32_t)a.nstages) { slot_s = 0; phase_s ^= 1; }
             }
