@@ -51,8 +51,8 @@ constexpr int kRxTiles[5] = {64, 56, 48, 40, 32};  // token rows per tile the la
 constexpr int kRxM = 4 * kRxE, kRxN = 4 * kRxT;
 constexpr int kRxStages = 2;
 constexpr int kRxABytes = kRxM * kRxK;                 // 16 KB
-constexpr int kRxBBytes = kRxN * kRxK;                 // 32 KB
-constexpr int kRxStageBytes = kRxABytes + kRxBBytes;   // 48 KB
+constexpr int kRxBBytes = kRxN * kRxK;                 // 32 KB for the largest tile (64 tokens)
+constexpr int kRxStageBytes = kRxABytes + kRxBBytes;   // 48 KB: the stride of a stage
 constexpr int kRxStageOut = 4 * kRxT * kRxE * 8;       // epilogue: the four digit-plane terms, fp64
 static_assert(kRxStageOut <= kRxStages * kRxStageBytes, "the epilogue reuses the pipeline buffers");
 constexpr int kRxOffBar = kRxStages * kRxStageBytes;
