@@ -161,15 +161,15 @@ def job_tokens_per_s(world_size, steps, tokens_per_step, total_ms):
 # kernel's sources hash to the recorded digest; otherwise `traffic` is null.
 NCU_TRAFFIC = {
     ("moe_decode_i8_kernel", "decode_b1"): dict(
-        bytes=190_530_000,
+        bytes=190_110_000,
         sources=('decode_i8.cu', 'common.cuh', 'topk.cuh', 'kernels.cuh'),
-        sha256_16="b4f29e362aec56b8",
-        note="ncu capture of the 16-expert decode case (184.63 MB read + written per launch) + 5.90 MB for "
+        sha256_16="f065e23c972e8b9a",
+        note="ncu capture of the 16-expert decode case (184.21 MB read + written per launch) + 5.90 MB for "
              "the 256-expert router"),
     ("moe_prefill_tc_kernel (gateup)", "prefill_2048"): dict(
         bytes=4_531_153_152,
         sources=('prefill_tc.cu', 'tcgen05.cuh', 'common.cuh', 'kernels.cuh'),
-        sha256_16="50a98688dc04f6cb",
+        sha256_16="4bbb8b0b50917590",
         note="ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one pass) of the first gate/up launch of "
              "this workload: 4,464 MB read + 67 MB written, against 3,738 MB algorithmic (1.21x: a hot expert's "
              "weights are read again per token tile, the token rows again per pair of row tiles)"),

@@ -73,6 +73,9 @@ constexpr int kMaxStages = 24;
 // Word of the layer's control block where a persistent kernel that gave up
 // on a bounded wait records its site code (0: none); alone in its 128-byte line.
 constexpr int kCtlError = 128;
+// Code in that word of a decode work item whose positions exceed its operand
+// buffer (a broken launch invariant; the item is not staged and the launch stops).
+constexpr int kCtlErrBufferOverflow = 13;
 
 inline int64_t matrix_bytes(int rows, int cols) {
     return (int64_t)(rows / kTileRows) * (cols / kGroup) * kBlockBytes;

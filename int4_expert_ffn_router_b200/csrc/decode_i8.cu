@@ -8,7 +8,9 @@
 // keep every per-weight instruction count far below what HBM speed allows
 // (about 41 weights per SM clock at 6.5 TB/s). One CTA per SM, three roles:
 //  * a producer thread takes work tickets and streams each item's 128-row
-//    weight tile into a shared-memory ring with bulk asynchronous copies;
+//    weight tile into a shared-memory ring with bulk asynchronous copies; at
+//    one or two tokens it also copies the next item's token operands into a
+//    second buffer while the current item streams;
 //  * eight consumer warps (one 16-row sub-tile each) multiply on the tensor
 //    cores from registers with integer MMAs (mma.m16n8k32, u8 x s8 -> s32):
 //    the weights enter as their offset-binary codes (one logic op per four
@@ -75,6 +77,7 @@ struct Item {
     int cnt;     // tokens of the chunk (<= 8)
     int tok0;    // shared chunk: its first token; routed: -1 (tokens from the plan)
     int ready;   // down: gate/up of the chunk already complete when published
+    int staged;  // two B buffers: the producer issued the B operands' copies into this slot's buffer
 };
 
 struct I8Args {
@@ -103,6 +106,8 @@ struct I8Args {
     int ncmax;     // bound on routed chunks
     int nstages;   // ring stages
     int sb;        // 4352-byte blocks per stage
+    int nbuf;      // B buffers: 2 (one per item-queue slot) when two items' operands fit, else 1
+    int nbt;       // positions one B buffer holds (ntc with one buffer)
     int64_t wait_ns;   // bound of every wait
     int wait_test;     // nonzero: the first gate/up tile waits on a flag nothing sets (testing aid)
     long long* trace;  // item timeline (NULL: off)
@@ -117,6 +122,9 @@ __host__ __device__ inline int i8_ctl_ints(int nchunks, int H, int ncmax) { retu
 
 struct I8Smem {
     uint64_t full[kMaxStages], empty[kMaxStages], qfull[kQ], qempty[kQ], dfull[kSQ], dempty[kSQ], bfull;
+    uint64_t bslot_full[kQ];   // two B buffers: one phase per item of the queue slot
+    int bslot_pending[kQ];     // copies into the buffer issued and not yet seen complete
+    uint32_t bslot_parity[kQ]; // parity of that phase
     Item items[kQ];
     Item cur[2];
     Item done[kSQ];
@@ -309,6 +317,58 @@ __device__ __forceinline__ Item shared_chunk(const I8Args& a, int kind, int sc, 
     return Item{kind, a.d.E + j, rt, sc, a.T * a.d.K + j * a.T + tok0, cnt, tok0, 0};
 }
 
+// Token i of a gate/up item: shared chunks hold consecutive tokens; routed
+// chunks read theirs from the published plan (with one token, token 0).
+__device__ __forceinline__ int item_token(const I8Args& a, const Item& it, int i) {
+    return it.tok0 >= 0 ? it.tok0 + i : a.T == 1 ? 0 : __ldcg(a.p.tok + it.pos + i);
+}
+
+// B buffers in the B area, each the operands of a.nbt positions (limbs, then
+// group data): one buffer of ntc positions, or two (one per item-queue slot)
+// of the largest chunk a launch can form.
+__device__ __forceinline__ uint8_t* buf_limbs(const I8Args& a, uint8_t* barea, int k) {
+    const int G = (a.d.H > a.d.I ? a.d.H : a.d.I) / kGroup;
+    return barea + (size_t)k * a.nbt * ((size_t)G * 128 + meta_slot_bytes(G));
+}
+__device__ __forceinline__ uint8_t* buf_meta(const I8Args& a, uint8_t* barea, int k) {
+    const int G = (a.d.H > a.d.I ? a.d.H : a.d.I) / kGroup;
+    return buf_limbs(a, barea, k) + (size_t)a.nbt * G * 128;
+}
+
+// Two B buffers: the copies of weight item it's B operands (token limbs and
+// group data for gate/up, h rows for down) into the buffer of queue slot k,
+// completing the slot's phase of the given parity. The caller (the producer,
+// or consumer 0 when the inputs were not ready at publication) has acquired
+// the completion of whatever wrote them.
+__device__ void stage_slot(I8Args& a, I8Smem& S, const Item& it, int k, uint32_t parity, uint8_t* barea) {
+    const Phases f = phases_of(a);
+    const bool gu = it.kind == IT_GU;
+    const int G = gu ? f.Ggu : f.Gd, nt = it.cnt;
+    if (nt > a.nbt) {  // cannot happen when the host sized the buffers; never write past one
+        set_error(a, &S.abort_flag, kCtlErrBufferOverflow);
+        return;
+    }
+    uint8_t* lb = buf_limbs(a, barea, k);
+    uint8_t* mb = buf_meta(a, barea, k);
+    uint64_t* bar = &S.bslot_full[k];
+    fence_proxy_async_global();
+    const uint32_t lbytes = (uint32_t)G * 128, mbytes = (uint32_t)G * kMetaRow;
+    S.bslot_parity[k] = parity;
+    S.bslot_pending[k] = 1;
+    mbar_arrive_expect_tx(bar, (uint32_t)nt * (lbytes + mbytes));
+    if (gu) {
+        for (int i = 0; i < nt; ++i) {
+            const int tok = item_token(a, it, i);
+            bulk_g2s(lb + (size_t)i * lbytes, a.xq + (size_t)tok * lbytes, lbytes, bar);
+            bulk_g2s(mb + (size_t)i * meta_slot_bytes(G), a.xm + (size_t)tok * mbytes, mbytes, bar);
+        }
+    } else {
+        bulk_g2s(lb, a.hq + (size_t)it.pos * lbytes, nt * lbytes, bar);
+        for (int i = 0; i < nt; ++i)
+            bulk_g2s(mb + (size_t)i * meta_slot_bytes(G), a.hm + (size_t)(it.pos + i) * mbytes, mbytes, bar);
+    }
+}
+
 // ------------------------------------------------------------------ producer
 __device__ void i8_producer(I8Args& a, I8Smem& S, uint8_t* ring) {
     const Dims& d = a.d;
@@ -317,6 +377,8 @@ __device__ void i8_producer(I8Args& a, I8Smem& S, uint8_t* ring) {
     const unsigned long long* entries = entries_of(a, f.nch);
     uint32_t q = 0, gs = 0, slot_s = 0, phase_s = 0;
     bool first_ticket = true;
+    bool prep_seen = false;  // every token's quantisation is complete (acquired)
+    uint8_t* barea = ring + (size_t)a.nstages * a.sb * kBlockBytes;
     const uint64_t wpolicy = l2_policy_evict_first();
     int nc = -1;  // routed chunks, once the plan is published
     while (true) {
@@ -356,6 +418,31 @@ __device__ void i8_producer(I8Args& a, I8Smem& S, uint8_t* ring) {
         }
         const uint32_t slot = q % kQ;
         if (q >= kQ && !wait_bar(&S.qempty[slot], ((q / kQ) - 1) & 1, abort_flag, a, 3)) it.kind = IT_END;
+        if (a.nbuf == 2) {
+            // the slot's buffer is free (the consumers are done with the slot's previous item):
+            // stage a weight item's B operands now when their inputs are complete, so that the
+            // consumers find them landed; otherwise consumer 0 stages them. Every other item
+            // completes the slot's phase with a plain arrival (one phase per item), except
+            // after an abort, when the slot's last phase may still wait for copies in flight
+            // and nothing but the exit drain waits on it.
+            const bool w = it.kind == IT_GU || it.kind == IT_DOWN;
+            bool ready = false;
+            if (w && !*abort_flag) {
+                if (it.kind == IT_GU) {
+                    if (!prep_seen) prep_seen = ld_acquire(&a.ctl[kCI_Prep]) >= f.P;
+                    // the testing aid's item keeps the consumers' staging path, where it waits
+                    ready = prep_seen && !(a.wait_test && it.chunk == 0 && it.rt == 0);
+                } else {
+                    ready = it.ready != 0;
+                }
+            }
+            if (ready) {
+                stage_slot(a, S, it, (int)slot, (q / kQ) & 1, barea);
+                it.staged = 1;
+            } else if (!w && !*abort_flag) {
+                mbar_arrive(&S.bslot_full[slot]);
+            }
+        }
         S.items[slot] = it;
         mbar_arrive(&S.qfull[slot]);
         ++q;
@@ -755,14 +842,8 @@ __device__ __forceinline__ void block_mma(const uint8_t* bp, const uint8_t* blim
     }
 }
 
-// Token i of a gate/up item: shared chunks hold consecutive tokens; routed
-// chunks read theirs from the published plan.
-__device__ __forceinline__ int item_token(const I8Args& a, const Item& it, int i) {
-    return it.tok0 >= 0 ? it.tok0 + i : __ldcg(a.p.tok + it.pos + i);
-}
-
 template <typename XT>
-__device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring, uint8_t* blimb, uint8_t* bmeta,
+__device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint32_t q, uint8_t* ring, uint8_t* barea,
                             uint32_t& slot_s, uint32_t& phase_s, int ctid) {
     const Dims& d = a.d;
     const Phases f = phases_of(a);
@@ -772,58 +853,85 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
     const int nt = it.cnt;
     volatile int* abort_flag = &S.abort_flag;
 
-    // ---- the item's tokens as B operands (staged once, reused by items with the same tokens)
-    bool same;
-    if (gu) {
-        same = S.staged_kind == IT_GU && S.staged_n == nt;
-        for (int i = 0; same && i < nt; ++i) {
-            same = S.staged_tok[i] == item_token(a, it, i);
+    uint8_t* blimb = buf_limbs(a, barea, 0);
+    uint8_t* bmeta = buf_meta(a, barea, 0);
+    bool have;  // the B operands are in place (false only after an abort)
+    if (a.nbuf == 2) {
+        // ---- two B buffers: the operands are in the buffer of the item's queue slot, staged
+        // by the producer when it published the item, else by consumer 0 now
+        const int k = (int)(q % kQ);
+        const uint32_t par = (q / kQ) & 1;
+        blimb = buf_limbs(a, barea, k);
+        bmeta = buf_meta(a, barea, k);
+        if (!it.staged) {  // uniform: every consumer read the same item
+            if (ctid == 0) {
+                bool ok;
+                if (gu) ok = wait_geq(&a.ctl[kCI_Prep], f.P, abort_flag, a, 5);
+                else ok = it.ready || wait_geq(&a.ctl[i8_ctl_gu(f.nch) + it.chunk], f.RTgu, abort_flag, a, 6);
+                // testing aid: the launch's first gate/up tile waits on a flag that nothing sets
+                if (ok && a.wait_test && gu && it.chunk == 0 && it.rt == 0)
+                    wait_geq(&a.ctl[kCI_Never], 1, abort_flag, a, 99);
+                if (!*abort_flag) stage_slot(a, S, it, k, par, barea);
+            }
+            named_bar(1, kCT);
         }
+        have = wait_bar(&S.bslot_full[k], par, abort_flag, a, 8);
+        if (ctid == 0 && have) S.bslot_pending[k] = 0;
     } else {
-        same = S.staged_kind == IT_DOWN && S.staged_key == it.chunk;
-    }
-    named_bar(1, kCT);  // every consumer has read the staging record before it changes
-    if (!same) {  // uniform: every consumer read the same shared values
-        if (ctid == 0) {
-            bool ok;
-            if (gu) ok = wait_geq(&a.ctl[kCI_Prep], f.P, abort_flag, a, 5);
-            else ok = it.ready || wait_geq(&a.ctl[i8_ctl_gu(f.nch) + it.chunk], f.RTgu, abort_flag, a, 6);
-            // testing aid: the launch's first gate/up tile waits on a flag that nothing sets
-            if (ok && a.wait_test && gu && it.chunk == 0 && it.rt == 0)
-                wait_geq(&a.ctl[kCI_Never], 1, abort_flag, a, 99);
-            if (!*abort_flag) {
-                fence_proxy_async_global();
-                const uint32_t lbytes = (uint32_t)G * 128, mbytes = (uint32_t)G * kMetaRow;
-                mbar_arrive_expect_tx(&S.bfull, (uint32_t)nt * (lbytes + mbytes));
-                S.bpending = 1;
-                if (gu) {
-                    for (int i = 0; i < nt; ++i) {
-                        const int tok = item_token(a, it, i);
-                        S.staged_tok[i] = tok;
-                        bulk_g2s(blimb + (size_t)i * lbytes, a.xq + (size_t)tok * lbytes, lbytes, &S.bfull);
-                        bulk_g2s(bmeta + (size_t)i * meta_slot_bytes(G), a.xm + (size_t)tok * mbytes, mbytes, &S.bfull);
+        // ---- the item's tokens as B operands (staged once, reused by items with the same tokens)
+        bool same;
+        if (gu) {
+            same = S.staged_kind == IT_GU && S.staged_n == nt;
+            for (int i = 0; same && i < nt; ++i) {
+                same = S.staged_tok[i] == item_token(a, it, i);
+            }
+        } else {
+            same = S.staged_kind == IT_DOWN && S.staged_key == it.chunk;
+        }
+        named_bar(1, kCT);  // every consumer has read the staging record before it changes
+        if (!same) {  // uniform: every consumer read the same shared values
+            if (ctid == 0) {
+                bool ok;
+                if (gu) ok = wait_geq(&a.ctl[kCI_Prep], f.P, abort_flag, a, 5);
+                else ok = it.ready || wait_geq(&a.ctl[i8_ctl_gu(f.nch) + it.chunk], f.RTgu, abort_flag, a, 6);
+                // testing aid: the launch's first gate/up tile waits on a flag that nothing sets
+                if (ok && a.wait_test && gu && it.chunk == 0 && it.rt == 0)
+                    wait_geq(&a.ctl[kCI_Never], 1, abort_flag, a, 99);
+                if (!*abort_flag) {
+                    fence_proxy_async_global();
+                    const uint32_t lbytes = (uint32_t)G * 128, mbytes = (uint32_t)G * kMetaRow;
+                    mbar_arrive_expect_tx(&S.bfull, (uint32_t)nt * (lbytes + mbytes));
+                    S.bpending = 1;
+                    if (gu) {
+                        for (int i = 0; i < nt; ++i) {
+                            const int tok = item_token(a, it, i);
+                            S.staged_tok[i] = tok;
+                            bulk_g2s(blimb + (size_t)i * lbytes, a.xq + (size_t)tok * lbytes, lbytes, &S.bfull);
+                            bulk_g2s(bmeta + (size_t)i * meta_slot_bytes(G), a.xm + (size_t)tok * mbytes, mbytes, &S.bfull);
+                        }
+                    } else {
+                        bulk_g2s(blimb, a.hq + (size_t)it.pos * lbytes, nt * lbytes, &S.bfull);
+                        for (int i = 0; i < nt; ++i)
+                            bulk_g2s(bmeta + (size_t)i * meta_slot_bytes(G), a.hm + (size_t)(it.pos + i) * mbytes, mbytes,
+                                     &S.bfull);
                     }
+                    S.staged_kind = it.kind;
+                    S.staged_n = nt;
+                    S.staged_key = it.chunk;
                 } else {
-                    bulk_g2s(blimb, a.hq + (size_t)it.pos * lbytes, nt * lbytes, &S.bfull);
-                    for (int i = 0; i < nt; ++i)
-                        bulk_g2s(bmeta + (size_t)i * meta_slot_bytes(G), a.hm + (size_t)(it.pos + i) * mbytes, mbytes,
-                                 &S.bfull);
+                    S.staged_kind = -1;
                 }
-                S.staged_kind = it.kind;
-                S.staged_n = nt;
-                S.staged_key = it.chunk;
-            } else {
-                S.staged_kind = -1;
+            }
+            named_bar(1, kCT);
+            bool landed = true;
+            if (S.staged_kind == it.kind) landed = wait_bar(&S.bfull, S.bphase & 1, abort_flag, a, 8);
+            named_bar(1, kCT);
+            if (ctid == 0 && S.staged_kind == it.kind && landed) {
+                ++S.bphase;
+                S.bpending = 0;
             }
         }
-        named_bar(1, kCT);
-        bool landed = true;
-        if (S.staged_kind == it.kind) landed = wait_bar(&S.bfull, S.bphase & 1, abort_flag, a, 8);
-        named_bar(1, kCT);
-        if (ctid == 0 && S.staged_kind == it.kind && landed) {
-            ++S.bphase;
-            S.bpending = 0;
-        }
+        have = S.staged_kind == it.kind;
     }
 
     // ---- stream the weight tile through the ring
@@ -849,7 +957,7 @@ __device__ void weight_item(I8Args& a, I8Smem& S, const Item& it, uint8_t* ring,
             if (i == 0) S.first_wait_ns = dw;
             S.total_wait_ns += dw;
         }
-        if (ok && S.staged_kind == it.kind) {
+        if (ok && have) {
             const uint8_t* stage = ring + (size_t)slot_s * stage_bytes;
             const int g0 = i * a.sb;
             const int nb = min(a.sb, G - g0);
@@ -972,15 +1080,16 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
     I8Smem& S = *reinterpret_cast<I8Smem*>(smem);
     uint8_t* ring = smem + head_bytes();
     uint8_t* barea = ring + (size_t)a.nstages * a.sb * kBlockBytes;
-    const int Gmax = (a.d.H > a.d.I ? a.d.H : a.d.I) / kGroup;
-    uint8_t* blimb = barea;
-    uint8_t* bmeta = barea + (size_t)a.ntc * Gmax * 128;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int i = 0; i < a.nstages; ++i) { mbar_init(&S.full[i], 1); mbar_init(&S.empty[i], kCW); }
         for (int i = 0; i < kQ; ++i) { mbar_init(&S.qfull[i], 1); mbar_init(&S.qempty[i], 1); }
         for (int i = 0; i < kSQ; ++i) { mbar_init(&S.dfull[i], kCT); mbar_init(&S.dempty[i], 1); }
         mbar_init(&S.bfull, 1);
+        for (int i = 0; i < kQ; ++i) {
+            mbar_init(&S.bslot_full[i], 1);
+            S.bslot_pending[i] = 0;
+        }
         S.abort_flag = 0;
         S.bphase = 0;
         S.bpending = 0;
@@ -1049,7 +1158,7 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
                     }
                 }
             } else if (it.kind == IT_GU || it.kind == IT_DOWN) {
-                weight_item<XT>(a, S, it, ring, blimb, bmeta, slot_s, phase_s, ctid);
+                weight_item<XT>(a, S, it, q, ring, barea, slot_s, phase_s, ctid);
             }
             // hand the completion to the signaler: the record first, then every
             // consumer thread arrives after its own global writes
@@ -1089,6 +1198,12 @@ __global__ void __launch_bounds__(kFT, 1) moe_decode_i8_kernel(I8Args a) {
         if (S.bpending) {
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&S.bfull, S.bphase & 1) && globaltimer_ns() - t0 < (uint64_t)a.wait_ns) {
+            }
+        }
+        for (int i = 0; i < kQ; ++i) {
+            if (!S.bslot_pending[i]) continue;
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&S.bslot_full[i], S.bslot_parity[i]) && globaltimer_ns() - t0 < (uint64_t)a.wait_ns) {
             }
         }
         __threadfence();
@@ -1170,6 +1285,15 @@ cudaError_t launch_decode_i8(const I8Launch& l, cudaStream_t st) {
     if (!i8_geometry(l.d, l.T, l.smem_limit, l.max_stages, l.max_sb, &a.ntc, &a.nstages, &a.sb))
         return cudaErrorInvalidConfiguration;
     a.cps = (l.T + a.ntc - 1) / a.ntc;
+    // two B buffers (the next item's operands staged by the producer while the current
+    // item streams) when two of the largest chunks fit in the area sized for ntc positions.
+    // A chunk holds distinct tokens, so at most T positions, except under expert top-p,
+    // where a token's dropped slots repeat its first expert (weight 0): up to T K.
+    const bool topp_on = l.topp > 0.0 && l.topp < 1.0;  // the top-k's own test
+    const int span = topp_on ? l.T * l.d.K : l.T;
+    const int maxchunk = span < a.ntc ? span : a.ntc;
+    a.nbuf = 2 * maxchunk <= a.ntc ? 2 : 1;
+    a.nbt = a.nbuf == 2 ? maxchunk : a.ntc;
     a.ncmax = i8_ncmax(l.d, l.T, a.ntc);
     if (l.dt == COLI_F32) return launch_i8_t<float>(a, l.n_sm, l.smem_limit, st);
     return launch_i8_t<__nv_bfloat16>(a, l.n_sm, l.smem_limit, st);

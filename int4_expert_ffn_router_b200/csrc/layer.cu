@@ -912,7 +912,10 @@ static coli_status sync_and_check(coli_moe_layer* L) {
     if (err != 0) {
         CUDA_TRY(cudaMemset(L->ctl, 0, (size_t)L->ctl_n * 4), "reset control block");
         char msg[96];
-        snprintf(msg, sizeof msg, "a bounded wait in a kernel of this layer timed out (site %d)", err);
+        if (err == kCtlErrBufferOverflow)
+            snprintf(msg, sizeof msg, "a decode work item exceeded its operand buffer (site %d)", err);
+        else
+            snprintf(msg, sizeof msg, "a bounded wait in a kernel of this layer timed out (site %d)", err);
         g_last_error = msg;
         return COLI_ECUDA;
     }
