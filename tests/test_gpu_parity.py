@@ -273,11 +273,13 @@ def test_full_decode_batch1(gpu, full, step, fused):
     assert _max_rel(yd.cpu().numpy().astype(np.float64), y_ref) <= FP32_TOL
 
 
-def test_full_decode_batch4_zipf_fused_matches_oracle(gpu, full):
-    """Four tokens through the persistent kernel, Zipf-skewed bias absent:
-    routing/union bit-exact, all four outputs against the oracle."""
+@pytest.mark.parametrize("T", [2, 4])
+def test_full_decode_small_batch_fused_matches_oracle(gpu, full, T):
+    """T tokens through the persistent kernel (no router bias): routing and
+    union bit-exact, every output against the oracle. At 2 tokens the
+    kernel's producer stages each item's token operands into a buffer per
+    item-queue slot; at 4 the consumers stage them into one buffer."""
     c, layer, wr = full
-    T = 4
     x = synth.x_f32(4000, 0, T, c["H"])
     xd = torch.from_numpy(x).to(gpu)
     yd = torch.empty_like(xd)
