@@ -73,12 +73,14 @@ def test_create_out_of_memory_at_each_allocation(gpu, resident):
     layer.close()
 
 
-def test_bounded_wait_expiry_returns_an_error_and_the_layer_recovers(gpu):
+@pytest.mark.parametrize("T", [3, 1])
+def test_bounded_wait_expiry_returns_an_error_and_the_layer_recovers(gpu, T):
     """A testing aid makes one gate/up item of the persistent kernel wait on a
     flag that nothing sets, with every wait bounded to 2 ms. The launch gives
     up by itself (its CTAs drain their copies and exit): coli_moe_sync reports
     COLI_ECUDA promptly, and the next forward on the same layer matches the
-    oracle. Nothing faults or hangs."""
+    oracle. Nothing faults or hangs. At 1 token the kernel's producer stages
+    the other items' operands into per-slot buffers, which the drain covers."""
     import time
 
     import int4_expert_ffn_router_b200 as coli
@@ -86,7 +88,7 @@ def test_bounded_wait_expiry_returns_an_error_and_the_layer_recovers(gpu):
     c = cases.TINY
     L, args = _host_args(coli, c)
     layer = coli.Layer(*args, device=0)
-    x = synth.x_f32(c["seed"], 4, 3, c["H"])
+    x = synth.x_f32(c["seed"], 4, T, c["H"])
     xd = torch.from_numpy(x).to(gpu)
     yd = torch.empty_like(xd)
     layer.forward(xd, yd)  # warm: module loaded, control block in use once
